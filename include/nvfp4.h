@@ -1,0 +1,219 @@
+/*
+ * nvfp4.h -- C ABI of the NVFP4 W4A4 routed-expert hot path for B200 (sm_100a).
+ *
+ * What the operations compute comes from these pages (cited by title and
+ * section):
+ *  [P1] "Qwen3.8-Flash-Next-NVFP4 ..." (lpnh.cn/news/2736522), section on the
+ *       W4A4 two-level scaling: every 16 elements along the last dimension
+ *       share one FP8 E4M3 block scale, each tensor has one FP32 global
+ *       scale, 4.5 effective bits; weights are quantized statically,
+ *       activations dynamically with the same per-16 rule; only the routed
+ *       experts' gate_up_proj / down_proj are quantized.
+ *  [P2] "DeepSeek-V4.1-Flash-NVFP4 ..." (kwkr.cn/news/613851), sections on the
+ *       format (E2M1 values {0,0.5,1,1.5,2,3,4,6}, two per byte, group 16;
+ *       MXFP4 32-element UE8M0 blocks remapped losslessly block by block) and
+ *       on why NVFP4 (Blackwell tensor cores take 4-bit operands natively).
+ *  [P3] "Qwen3.8-2.4T-A95B-NVFP4 ..." (hnwysp.cn/news/107543): NVFP4 KV cache.
+ *
+ * Conventions shared by every entry point
+ *  - All tensor pointers are DEVICE pointers owned by the caller.  The
+ *    library allocates nothing; scratch space is a caller-supplied
+ *    `workspace` of at least nvfp4_workspace_size() bytes (device memory).
+ *  - Every call is asynchronous on `stream` and never synchronises the host
+ *    or copies device data to the host.
+ *  - Return value: argument/shape/launch errors found on the host.
+ *    Data-dependent errors are written by the kernels to the optional device
+ *    word `dev_status` (int32): the first error wins (compare-and-swap from
+ *    NVFP4_OK), and nothing traps.  The caller zeroes it before use.
+ *  - Pointers to packed tensors must be 16-byte aligned.
+ *  - Number formats: E2M1 codes packed two per byte, element 2j in bits
+ *    [3:0] and element 2j+1 in bits [7:4]; block scales are E4M3 bytes; the
+ *    global scale s_g is the fp32 dequantisation multiplier, so an element
+ *    decodes to (e2m1(code) * e4m3(S)) * s_g.
+ *  - Scale-factor layouts (nvfp4_sf_layout):
+ *      ROWMAJOR:  sf[r * (K/16) + j] for row r, block j.
+ *      MMA_TILED: the tensor-core operand layout.  Rows are grouped in
+ *        128-row blocks and scales in groups of 4 (64 elements); each
+ *        (row-block, 4-group) pair is a 512-byte atom, atoms ordered
+ *        row-block-major, and inside an atom the scale of row r, block j is
+ *        at (r%32)*16 + ((r%128)/32)*4 + (j%4).  Requires K % 64 == 0; the
+ *        tensor holds roundup(rows,128) rows.
+ *  - Grouped (MoE) row placement: with `group_offsets` (int32 [G+1], raw
+ *    prefix sums of the rows of each expert group, on the device), packed
+ *    rows of group g start at the 128-aligned slot
+ *    slot[g] = sum_{h<g} roundup(rows_h, 128); rows of a slot past the
+ *    group's rows are written as zero codes and zero scales.  Size packed
+ *    buffers with nvfp4_padded_rows_bound().
+ */
+#ifndef NVFP4_H_
+#define NVFP4_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    NVFP4_OK = 0,
+    NVFP4_ERR_INVALID_ARG = 1,       /* null / misaligned pointer, bad enum */
+    NVFP4_ERR_UNSUPPORTED_SHAPE = 2, /* shape outside the documented limits */
+    NVFP4_ERR_CUDA = 3,              /* a launch or runtime call failed */
+    /* data-dependent errors, written to *dev_status by the kernels */
+    NVFP4_ERR_NONFINITE = 16,        /* an input element (or amax) is NaN or inf */
+    NVFP4_ERR_NOT_REPRESENTABLE = 17,/* MXFP4 exponent byte 0xFF or spread > 17 */
+    NVFP4_ERR_TIMEOUT = 18           /* a bounded wait inside a kernel gave up */
+} nvfp4_status;
+
+typedef enum { NVFP4_SF_ROWMAJOR = 0, NVFP4_SF_MMA_TILED = 1 } nvfp4_sf_layout;
+typedef enum { NVFP4_GS_FROM_AMAX = 0, NVFP4_GS_GIVEN = 1 } nvfp4_gs_mode;
+typedef enum { NVFP4_OUT_F32 = 0, NVFP4_OUT_BF16 = 1 } nvfp4_out_dtype;
+typedef enum { NVFP4_EPI_NONE = 0 } nvfp4_epilogue;
+
+/* Human-readable name of a status code (static string). */
+const char *nvfp4_status_string(int status);
+
+/* Bytes of device workspace needed by any call below for up to `num_groups`
+ * groups / experts / tensors (num_groups >= 1). */
+size_t nvfp4_workspace_size(int num_groups);
+
+/* Upper bound on packed rows when `rows` gathered rows are split into
+ * `num_groups` 128-aligned slots (= rows + 127*num_groups, rounded to 128). */
+int64_t nvfp4_padded_rows_bound(int64_t rows, int num_groups);
+
+/*
+ * nvfp4_quantize -- dynamic (or static) NVFP4 quantisation of bf16 rows.
+ * [P1 two-level scaling: per-16 E4M3 block scale + FP32 global; activations
+ *  quantized on the fly; P2 format: E2M1 codes packed two per byte.]
+ *
+ *   x           bf16 [*, ld_x]; ld_x >= K, in elements, ld_x % 8 == 0.
+ *   rows, K     rows of the (gathered) result and row length; K % 16 == 0,
+ *               K % 64 == 0 for MMA_TILED; rows >= 0 (0 is a no-op).
+ *   row_index   nullable int32 [rows]: result row r is x[row_index[r]].
+ *   group_offsets, num_groups
+ *               nullable int32 [num_groups+1] device prefix sums over result
+ *               rows (offsets[0] == 0, offsets[G] == rows).  Each group has
+ *               its own global scale and its own 128-aligned slot in q/sf.
+ *               NULL: one group, rows written contiguously (padded to 128 rows
+ *               only for MMA_TILED).
+ *   gs_mode, global_scale
+ *               fp32 [max(1,num_groups)] device.  FROM_AMAX: written with
+ *               s_g = amax/2688 (2688 = 6*448: the block holding the amax gets
+ *               scale 448), or 1 for an all-zero group.  GIVEN: read (a
+ *               calibrated input scale or a static KV scale), must be > 0.
+ *   q           uint8 [packed rows, K/2]; sf uint8 scales in `sf_layout`.
+ *   workspace   >= nvfp4_workspace_size(num_groups) bytes.
+ *   dev_status  nullable int32: NVFP4_ERR_NONFINITE when an input element of a
+ *               group is NaN/inf (that group's outputs are unspecified).
+ * Arithmetic (each step one IEEE fp32 round-to-nearest-even operation):
+ *   block amax a_b; S = e4m3_rne_satfinite(a_b / (6*s_g));
+ *   r = 1/(S*s_g) (0 when S*s_g == 0); code_i = e2m1_rne_satfinite(x_i * r).
+ */
+nvfp4_status nvfp4_quantize(const void *x, int64_t rows, int64_t K, int64_t ld_x,
+                            const int32_t *row_index, const int32_t *group_offsets,
+                            int num_groups, nvfp4_gs_mode gs_mode, float *global_scale,
+                            uint8_t *q, uint8_t *sf, nvfp4_sf_layout sf_layout,
+                            void *workspace, int32_t *dev_status, cudaStream_t stream);
+
+/*
+ * nvfp4_dequantize -- y = (e2m1(code) * e4m3(S)) * s_g, rounded once to the
+ * output type.  [P1: quantized tensors are dequantized with their scales.]
+ *   q, sf, sf_layout  packed input (grouped slots when group_offsets != NULL).
+ *   global_scale      fp32 [max(1,num_groups)].
+ *   y                 [rows, K] fp32 or bf16, rows in unpadded order.
+ */
+nvfp4_status nvfp4_dequantize(const uint8_t *q, const uint8_t *sf, nvfp4_sf_layout sf_layout,
+                              const float *global_scale, const int32_t *group_offsets,
+                              int num_groups, int64_t rows, int64_t K, void *y,
+                              nvfp4_out_dtype out_dtype, cudaStream_t stream);
+
+/*
+ * mxfp4_to_nvfp4 -- lossless block-by-block MXFP4 -> NVFP4 weight remap.
+ * [P2: MXFP4 uses 32-element blocks with UE8M0 (power-of-two) scales, NVFP4
+ *  16-element blocks with a finer scale, and the weights "can be remapped
+ *  block by block without loss"; the conversion script does the E2M1->E4M3
+ *  remap.]
+ *   n_tensors tensors of [rows, K] laid back to back (K % 32 == 0).
+ *   q_mx uint8 [n*rows, K/2]; ue8m0 uint8 [n*rows, K/32].
+ *   q_nv uint8 [n*rows, K/2] (codes copied unchanged; may equal q_mx);
+ *   sf_nv scales in sf_layout (MMA_TILED needs rows % 128 == 0, K % 64 == 0);
+ *   global_scale fp32 [n]: s_g = 2^g with g = e_max - 8 over the blocks that
+ *   are not all +-0 (g = 0 if none); every 32-block of exponent e gets the
+ *   E4M3 scale 2^clamp(e-g, -9, 8) on both halves.
+ *   workspace >= nvfp4_workspace_size(n_tensors).
+ *   dev_status: NVFP4_ERR_NOT_REPRESENTABLE when a byte is 0xFF or a tensor's
+ *   exponent spread exceeds 17 (E4M3 holds exactly 2^-9 .. 2^8).
+ */
+nvfp4_status mxfp4_to_nvfp4(const uint8_t *q_mx, const uint8_t *ue8m0, int64_t n_tensors,
+                            int64_t rows, int64_t K, uint8_t *q_nv, uint8_t *sf_nv,
+                            nvfp4_sf_layout sf_layout, float *global_scale, void *workspace,
+                            int32_t *dev_status, cudaStream_t stream);
+
+/*
+ * nvfp4_grouped_gemm -- Y_e = (a_gs[e] * b_gs[e]) * A_e B_e^T for every expert e,
+ * block-scaled FP4 x FP4 on the tcgen05 tensor cores, fp32 accumulation.
+ * [P2 "why NVFP4": Blackwell tensor cores multiply 4-bit operands natively;
+ *  P1: routed experts' gate_up_proj / down_proj in W4A4.]
+ *   a_q, a_sf   packed activations in 128-aligned expert slots (the output of
+ *               nvfp4_quantize with group_offsets), MMA_TILED scales.
+ *   a_gs        fp32 [E] activation global scales.
+ *   b_q, b_sf   packed weights [E, N, K/2], MMA_TILED scales over E*N rows.
+ *   b_gs        fp32 [E] weight global scales.
+ *   expert_offsets  nullable int32 [E+1] device prefix sums of routed rows
+ *               (offsets[E] == M_total).  NULL means one dense GEMM (E = 1).
+ *   M_total, N, K   Y is [M_total, N]; N % 128 == 0, K % 256 == 0.
+ *   y, out_dtype    fp32 or bf16 [M_total, N], rows in routed (unpadded) order.
+ *   epi             NVFP4_EPI_NONE.
+ *   workspace   >= nvfp4_workspace_size(E); dev_status: NVFP4_ERR_TIMEOUT if a
+ *               pipeline wait gave up (the output is then incomplete).
+ */
+nvfp4_status nvfp4_grouped_gemm(const uint8_t *a_q, const uint8_t *a_sf, const float *a_gs,
+                                const uint8_t *b_q, const uint8_t *b_sf, const float *b_gs,
+                                const int32_t *expert_offsets, int num_experts,
+                                int64_t M_total, int64_t N, int64_t K, void *y,
+                                nvfp4_out_dtype out_dtype, nvfp4_epilogue epi,
+                                void *workspace, int32_t *dev_status, cudaStream_t stream);
+
+/*
+ * nvfp4_swiglu_quantize -- the step between the two expert projections:
+ * h = bf16(silu(g) * u) with g = y[:, :I] (gate rows of the fused gate_up
+ * weight come first) and u = y[:, I:], then h is NVFP4-quantized per expert
+ * group exactly as nvfp4_quantize(FROM_AMAX) would quantize it.
+ *   y        fp32 or bf16 [rows, 2I] (the gate_up GEMM output, routed order).
+ *   h        nullable bf16 [rows, I]: also store h.
+ *   group_offsets / num_groups / global_scale / q / sf / sf_layout: as in
+ *   nvfp4_quantize (global scales are always computed from the amax of h).
+ *   silu(g) = g / (1 + exp(-g)) in fp32 with the device expf.
+ */
+nvfp4_status nvfp4_swiglu_quantize(const void *y, nvfp4_out_dtype y_dtype, int64_t rows,
+                                   int64_t I, const int32_t *group_offsets, int num_groups,
+                                   float *global_scale, uint8_t *q, uint8_t *sf,
+                                   nvfp4_sf_layout sf_layout, void *h, void *workspace,
+                                   int32_t *dev_status, cudaStream_t stream);
+
+/*
+ * nvfp4_kv_quantize -- NVFP4 KV-cache write for one attention layer: K and V
+ * (bf16 [tokens, heads, head_dim] each) quantized in groups of 16 along
+ * head_dim, one global scale per tensor.  [P3: --kv-cache-dtype nvfp4.]
+ * Same arithmetic as nvfp4_quantize with rows = tokens*heads and
+ * K = head_dim; k_gs / v_gs are fp32 [1] each, written (FROM_AMAX) or read
+ * (GIVEN, the serving case).  Scales are ROWMAJOR.
+ *   workspace >= nvfp4_workspace_size(2).
+ */
+nvfp4_status nvfp4_kv_quantize(const void *k, const void *v, int64_t tokens, int64_t heads,
+                               int64_t head_dim, nvfp4_gs_mode gs_mode, float *k_gs, float *v_gs,
+                               uint8_t *k_q, uint8_t *k_sf, uint8_t *v_q, uint8_t *v_sf,
+                               void *workspace, int32_t *dev_status, cudaStream_t stream);
+
+/* nvfp4_kv_dequantize -- the attention-side read: both tensors back to bf16. */
+nvfp4_status nvfp4_kv_dequantize(const uint8_t *k_q, const uint8_t *k_sf, const float *k_gs,
+                                 const uint8_t *v_q, const uint8_t *v_sf, const float *v_gs,
+                                 int64_t tokens, int64_t heads, int64_t head_dim,
+                                 void *k_out, void *v_out, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* NVFP4_H_ */

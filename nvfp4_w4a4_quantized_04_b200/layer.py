@@ -1,0 +1,160 @@
+"""Host-side orchestration of the NVFP4 routed-expert path on the C ABI.
+
+Torch provides device memory and the stream; each step is one call into
+``libnvfp4.so``.  ``MoEExperts.forward`` is the MoE layer's expert part:
+gather + per-group dynamic quantize -> grouped gate_up GEMM -> SwiGLU +
+per-group requantize -> grouped down GEMM (the routed-expert projections of
+the "Qwen3.8-Flash-Next-NVFP4" page, quantized W4A4).
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+from . import (EPI_NONE, GS_FROM_AMAX, GS_GIVEN, OUT_BF16, OUT_F32, SF_MMA_TILED, SF_ROWMAJOR,
+               mxfp4_to_nvfp4, nvfp4_dequantize, nvfp4_grouped_gemm, nvfp4_padded_rows_bound,
+               nvfp4_quantize, nvfp4_swiglu_quantize, nvfp4_workspace_size)
+
+
+@dataclass
+class Packed:
+    """An NVFP4 tensor in device memory.
+
+    q: uint8 [rows_alloc, K/2]; sf: uint8 scales (``layout``); gs: fp32 [G]
+    global scales.  With ``offsets`` (int32 [G+1] on the device) rows sit in
+    128-aligned per-group slots.
+    """
+    q: torch.Tensor
+    sf: torch.Tensor
+    gs: torch.Tensor
+    rows: int
+    K: int
+    layout: int
+    offsets: Optional[torch.Tensor] = None
+    num_groups: int = 1
+
+
+def workspace(num_groups: int, device="cuda") -> torch.Tensor:
+    n = nvfp4_workspace_size(max(1, num_groups))
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def alloc_rows(rows: int, num_groups: int, grouped: bool, layout: int) -> int:
+    if grouped:
+        return nvfp4_padded_rows_bound(rows, num_groups)
+    return (rows + 127) // 128 * 128 if layout == SF_MMA_TILED else rows
+
+
+def sf_bytes(rows_alloc: int, K: int) -> int:
+    return rows_alloc * (K // 16)
+
+
+def empty_packed(rows: int, K: int, num_groups: int = 1, offsets=None, layout=SF_MMA_TILED,
+                 device="cuda") -> Packed:
+    ra = alloc_rows(rows, num_groups, offsets is not None, layout)
+    q = torch.empty((max(ra, 1), K // 2), dtype=torch.uint8, device=device)
+    sf = torch.empty(max(sf_bytes(ra, K), 1), dtype=torch.uint8, device=device)
+    gs = torch.empty(max(1, num_groups), dtype=torch.float32, device=device)
+    return Packed(q, sf, gs, rows, K, layout, offsets, num_groups if offsets is not None else 1)
+
+
+def quantize(x: torch.Tensor, row_index=None, offsets=None, num_groups: int = 1, layout=SF_MMA_TILED,
+             global_scale=None, out: Optional[Packed] = None, ws=None, dev_status=None, rows=None) -> Packed:
+    """NVFP4-quantize bf16 rows (dynamic global scale unless ``global_scale`` is given)."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2
+    K = x.shape[1]
+    R = rows if rows is not None else (row_index.shape[0] if row_index is not None else x.shape[0])
+    G = num_groups if offsets is not None else 1
+    p = out if out is not None else empty_packed(R, K, G, offsets, layout, x.device)
+    p.offsets, p.num_groups, p.rows = offsets, G, R
+    mode = GS_FROM_AMAX
+    if global_scale is not None:
+        p.gs.copy_(global_scale)
+        mode = GS_GIVEN
+    ws = ws if ws is not None else workspace(G, x.device)
+    nvfp4_quantize(x, R, K, x.stride(0), row_index, offsets, G, mode, p.gs, p.q, p.sf, layout, ws, dev_status)
+    return p
+
+
+def dequantize(p: Packed, out_dtype=OUT_F32) -> torch.Tensor:
+    dt = torch.float32 if out_dtype == OUT_F32 else torch.bfloat16
+    y = torch.empty((p.rows, p.K), dtype=dt, device=p.q.device)
+    nvfp4_dequantize(p.q, p.sf, p.layout, p.gs, p.offsets, p.num_groups, p.rows, p.K, y, out_dtype)
+    return y
+
+
+def remap_mxfp4(q_mx: torch.Tensor, e8: torch.Tensor, n_tensors: int, rows: int, K: int, layout=SF_MMA_TILED,
+                ws=None, dev_status=None, inplace: bool = False) -> Packed:
+    """Lossless MXFP4 -> NVFP4 remap of n_tensors [rows, K] tensors."""
+    q_nv = q_mx if inplace else torch.empty_like(q_mx)
+    sf = torch.empty(n_tensors * rows * (K // 16), dtype=torch.uint8, device=q_mx.device)
+    gs = torch.empty(n_tensors, dtype=torch.float32, device=q_mx.device)
+    ws = ws if ws is not None else workspace(n_tensors, q_mx.device)
+    mxfp4_to_nvfp4(q_mx, e8, n_tensors, rows, K, q_nv, sf, layout, gs, ws, dev_status)
+    return Packed(q_nv, sf, gs, n_tensors * rows, K, layout, None, n_tensors)
+
+
+def grouped_gemm(a: Packed, w: Packed, N: int, out_dtype=OUT_BF16, y=None, dev_status=None) -> torch.Tensor:
+    """Y [a.rows, N] = per expert (a_gs[e] * w_gs[e]) * A_e W_e^T."""
+    assert a.layout == SF_MMA_TILED and w.layout == SF_MMA_TILED
+    E = a.num_groups if a.offsets is not None else 1
+    dt = torch.float32 if out_dtype == OUT_F32 else torch.bfloat16
+    if y is None:
+        y = torch.empty((a.rows, N), dtype=dt, device=a.q.device)
+    nvfp4_grouped_gemm(a.q, a.sf, a.gs, w.q, w.sf, w.gs, a.offsets, E, a.rows, N, a.K, y, out_dtype, EPI_NONE,
+                       None, dev_status)
+    return y
+
+
+def swiglu_quantize(y: torch.Tensor, offsets, num_groups: int, layout=SF_MMA_TILED, out: Optional[Packed] = None,
+                    h=None, ws=None, dev_status=None):
+    rows, I2 = y.shape
+    I = I2 // 2
+    G = num_groups if offsets is not None else 1
+    p = out if out is not None else empty_packed(rows, I, G, offsets, layout, y.device)
+    p.offsets, p.num_groups, p.rows = offsets, G, rows
+    h = h if h is not None else torch.empty((rows, I), dtype=torch.bfloat16, device=y.device)
+    ws = ws if ws is not None else workspace(G, y.device)
+    ydt = OUT_F32 if y.dtype == torch.float32 else OUT_BF16
+    nvfp4_swiglu_quantize(y, ydt, rows, I, offsets, G, p.gs, p.q, p.sf, layout, h, ws, dev_status)
+    return p, h
+
+
+class MoEExperts:
+    """Routed experts of one MoE layer in NVFP4 W4A4.
+
+    w_gate_up: packed [E*2I, H] (rows 0..I-1 of each expert = gate, I..2I-1 = up),
+    one global scale per expert; w_down: packed [E*H, I].
+    forward(x bf16 [T, H], row_index int32 [R], offsets int32 [E+1]) -> Y bf16 [R, H]
+    in routed order (the weighted combine is outside this layer).
+    """
+
+    def __init__(self, w_gate_up: Packed, w_down: Packed, E: int, H: int, I: int, max_rows: int,
+                 out_dtype=OUT_BF16, mid_dtype=OUT_BF16, device="cuda"):
+        self.w_gate_up, self.w_down = w_gate_up, w_down
+        self.E, self.H, self.I = E, H, I
+        self.out_dtype, self.mid_dtype = out_dtype, mid_dtype
+        self.ws = workspace(E, device)
+        self.a1 = empty_packed(max_rows, H, E, torch.empty(0), SF_MMA_TILED, device)
+        self.a2 = empty_packed(max_rows, I, E, torch.empty(0), SF_MMA_TILED, device)
+        mdt = torch.bfloat16 if mid_dtype == OUT_BF16 else torch.float32
+        odt = torch.bfloat16 if out_dtype == OUT_BF16 else torch.float32
+        self.y1 = torch.empty((max_rows, 2 * I), dtype=mdt, device=device)
+        self.h = torch.empty((max_rows, I), dtype=torch.bfloat16, device=device)
+        self.y2 = torch.empty((max_rows, H), dtype=odt, device=device)
+        self.max_rows = max_rows
+
+    def forward(self, x: torch.Tensor, row_index: torch.Tensor, offsets: torch.Tensor, dev_status=None):
+        R = row_index.shape[0]
+        assert R <= self.max_rows
+        E, H, I = self.E, self.H, self.I
+        a1 = quantize(x, row_index, offsets, E, SF_MMA_TILED, out=self.a1, ws=self.ws, dev_status=dev_status, rows=R)
+        y1 = self.y1[:R]
+        grouped_gemm(a1, self.w_gate_up, 2 * I, self.mid_dtype, y=y1, dev_status=dev_status)
+        a2, _ = swiglu_quantize(y1, offsets, E, SF_MMA_TILED, out=self.a2, h=self.h[:R], ws=self.ws,
+                                dev_status=dev_status)
+        y2 = self.y2[:R]
+        grouped_gemm(a2, self.w_down, H, self.out_dtype, y=y2, dev_status=dev_status)
+        return y2

@@ -113,17 +113,52 @@ def outlier_positions(seed: int, numel: int, frac: float = 0.001) -> np.ndarray:
     return np.sort(order[:n_out]).astype(np.int64)
 
 
+_HG = None
+
+
+def _hostgen():
+    """The C twin of ``normal_z`` + bf16 rounding (hostgen.c), built on first use."""
+    global _HG
+    if _HG is None:
+        import ctypes
+        import os
+        import subprocess
+        here = os.path.dirname(os.path.abspath(__file__))
+        src, so = os.path.join(here, "hostgen.c"), os.path.join(here, "libhostgen.so")
+        if not os.path.exists(so) or os.path.getmtime(so) < os.path.getmtime(src):
+            tmp = so + f".tmp{os.getpid()}"
+            subprocess.check_call(["gcc", "-O2", "-fPIC", "-shared", "-fopenmp", "-ffp-contract=off", src,
+                                   "-o", tmp])
+            os.replace(tmp, so)
+        L = ctypes.CDLL(so)
+        L.hg_normal_bf16.restype = None
+        L.hg_normal_bf16.argtypes = [ctypes.c_uint64, ctypes.c_uint64, ctypes.c_int64, ctypes.c_int64,
+                                     ctypes.c_double, ctypes.c_int, ctypes.c_void_p]
+        _HG = L
+    return _HG
+
+
+def gaussian_bf16_bits_fast(seed: int, stream: int, start: int, n: int, sigma: float) -> np.ndarray:
+    out = np.empty(n, dtype=np.uint16)
+    _hostgen().hg_normal_bf16(seed, stream, start, n, float(sigma), int(sigma != 1.0),
+                              out.ctypes.data_as(__import__("ctypes").c_void_p))
+    return out
+
+
 def gaussian_bf16(seed: int, stream: int, shape, sigma: float = 1.0,
                   outlier_frac: float = 0.0, outlier_mult: float = 50.0,
-                  start: int = 0) -> np.ndarray:
+                  start: int = 0, reference: bool = False) -> np.ndarray:
     """bf16 bits (uint16) of N(0, sigma^2) deviates, optional outliers.
 
     ``start`` offsets the flat element index, so a slice of a large tensor
     can be regenerated alone.  Outliers are defined over the tensor starting
-    at index 0 and are not supported together with ``start``.
+    at index 0 and are not supported together with ``start``.  Large tensors
+    go through the C twin (same bits); ``reference=True`` forces numpy.
     """
     shape = tuple(int(s) for s in shape)
     n = int(np.prod(shape)) if shape else 1
+    if outlier_frac == 0.0 and not reference and n >= (1 << 16):
+        return gaussian_bf16_bits_fast(seed, stream, start, n, sigma).reshape(shape)
     z = normal_z(seed, stream, start, n)
     f = (z * float(sigma)).astype(np.float32) if sigma != 1.0 else z.astype(np.float32)
     if outlier_frac > 0.0:

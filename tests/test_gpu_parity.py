@@ -1,0 +1,510 @@
+"""CUDA path vs the oracle on small seeded inputs (bit-exact for codes/scales,
+the stated tolerance for GEMM outputs).  Calls go through the C ABI."""
+import numpy as np
+import pytest
+
+import oracle
+import synthetic
+from tests._util import bf16_dev, slot_rows, tile, to_dev, to_np, untile
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _setup():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from nvfp4_w4a4_quantized_04_b200 import build
+    build.build()
+    import synthetic.cuda as sc
+    sc.build()
+
+
+def nvmod():
+    import nvfp4_w4a4_quantized_04_b200 as nv
+    return nv
+
+
+def layer():
+    from nvfp4_w4a4_quantized_04_b200 import layer as L
+    return L
+
+
+def status_word():
+    return torch.zeros(1, dtype=torch.int32, device="cuda")
+
+
+def gemm_tol(y, y_ref, s_ref):
+    """|y - y_ref| <= 1e-5 * sum|a*b| + 1e-6 elementwise."""
+    err = np.abs(y.astype(np.float64) - y_ref)
+    bound = 1e-5 * s_ref + 1e-6
+    return err <= bound, err, bound
+
+
+# --------------------------------------------------------------------------- quantize
+@pytest.mark.parametrize("layout", [0, 1])
+def test_quantize_dense_config1_bitexact(layout):
+    L = layer()
+    x = synthetic.gaussian_bf16(0, synthetic.STREAMS["x"], (128, 512), outlier_frac=0.001)
+    q_ref, sf_ref, gs_ref, st = oracle.quantize(x)
+    assert st == 0
+    p = L.quantize(bf16_dev(x), layout=layout)
+    torch.cuda.synchronize()
+    assert to_np(p.gs)[0] == gs_ref[0]
+    assert np.array_equal(to_np(p.q)[:128], q_ref)
+    sf = to_np(p.sf)
+    sf = untile(sf, 128, 32) if layout == 1 else sf.reshape(128, 32)
+    assert np.array_equal(sf, sf_ref)
+
+
+@pytest.mark.parametrize("layout", [0, 1])
+def test_quantize_grouped_gather_bitexact(layout):
+    L = layer()
+    T, H, E, k = 256, 512, 12, 2
+    x = synthetic.gaussian_bf16(1, synthetic.STREAMS["x"], (T, H))
+    r = synthetic.route_topk_softmax(1, T, E, k)
+    counts = np.diff(r["offsets"])
+    assert counts.max() > 128            # a group spanning two slot tiles
+    q_ref, sf_ref, gs_ref, st = oracle.quantize(x, r["row_index"], r["offsets"])
+    assert st == 0
+    off = to_dev(r["offsets"])
+    p = L.quantize(bf16_dev(x), to_dev(r["row_index"]), off, E, layout=layout)
+    torch.cuda.synchronize()
+    assert np.array_equal(to_np(p.gs), gs_ref)
+    rows, starts = slot_rows(r["offsets"])
+    used = int(starts[-1])
+    q = to_np(p.q)
+    assert np.array_equal(q[rows], q_ref)
+    pad = np.setdiff1d(np.arange(used), rows)
+    assert (q[pad] == 0).all()
+    sf = to_np(p.sf)
+    sfm = untile(sf, p.q.shape[0], H // 16) if layout == 1 else sf.reshape(-1, H // 16)
+    assert np.array_equal(sfm[rows], sf_ref)
+    assert (sfm[pad] == 0).all()
+
+
+def test_quantize_groups_with_empty_experts():
+    L = layer()
+    H = 256
+    offsets = np.array([0, 0, 3, 3, 3, 200, 200, 201], dtype=np.int32)
+    x = synthetic.gaussian_bf16(2, synthetic.STREAMS["x"], (201, H))
+    q_ref, sf_ref, gs_ref, st = oracle.quantize(x, None, offsets)
+    p = L.quantize(bf16_dev(x), None, to_dev(offsets), 7, layout=1)
+    torch.cuda.synchronize()
+    assert np.array_equal(to_np(p.gs), gs_ref)        # empty groups: s_g = 1
+    rows, _ = slot_rows(offsets)
+    assert np.array_equal(to_np(p.q)[rows], q_ref)
+    assert np.array_equal(untile(to_np(p.sf), p.q.shape[0] // 128 * 128, H // 16)[rows], sf_ref)
+
+
+@pytest.mark.parametrize("shape", [(1, 16), (5, 48), (3, 208), (0, 64), (1000, 16)])
+def test_quantize_ragged_shapes(shape):
+    L = layer()
+    x = synthetic.gaussian_bf16(7, synthetic.STREAMS["x"], shape, outlier_frac=0.01)
+    R, K = shape
+    if R == 0:
+        xd = torch.empty((0, K), dtype=torch.bfloat16, device="cuda")
+        p = L.quantize(xd, layout=0)
+        torch.cuda.synchronize()
+        assert to_np(p.gs)[0] == 1.0
+        return
+    q_ref, sf_ref, gs_ref, st = oracle.quantize(x)
+    p = L.quantize(bf16_dev(x), layout=0)
+    torch.cuda.synchronize()
+    assert to_np(p.gs)[0] == gs_ref[0]
+    assert np.array_equal(to_np(p.q)[:R], q_ref)
+    assert np.array_equal(to_np(p.sf)[:R * K // 16].reshape(R, K // 16), sf_ref)
+
+
+def _special_tensor():
+    """Zeros, -0, tiny and huge magnitudes, exact E2M1 midpoints after scaling."""
+    f = np.zeros((8, 64), dtype=np.float32)
+    f[0, :16] = 6.0 * np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5, 6, -0.25, -0.75, -1.25, -1.75, -2.5, -3.5, -5, -6]) / 6
+    f[1, :] = -0.0
+    f[2, :16] = np.float32(1e-30)
+    f[2, 16:32] = -np.float32(3e-38)
+    f[3, :] = np.linspace(-3, 3, 64)
+    f[4, 5] = 1e30
+    f[5, :16] = [1, 1e-5, 2e-6, 0, -0.0, 1e-7, 3e-8, 1, 0.5, 0.25, 0.125, 0.0625, 0.03125, 1e-3, 1e-4, 1e-9]
+    return synthetic.f32_to_bf16_bits(f)
+
+
+def test_quantize_special_values():
+    L = layer()
+    x = _special_tensor()
+    for layout in (0, 1):
+        q_ref, sf_ref, gs_ref, st = oracle.quantize(x)
+        p = L.quantize(bf16_dev(x), layout=layout)
+        torch.cuda.synchronize()
+        assert to_np(p.gs)[0] == gs_ref[0]
+        assert np.array_equal(to_np(p.q)[:8], q_ref)
+    # a tensor whose amax is tiny (subnormal global scale)
+    tiny = np.zeros((2, 32), dtype=np.float32)
+    tiny[0, 3] = 3e-38
+    tiny[1, 9] = -1.2e-39
+    tiny[1, 10] = -0.0
+    xb = synthetic.f32_to_bf16_bits(tiny)
+    q_ref, sf_ref, gs_ref, st = oracle.quantize(xb)
+    p = L.quantize(bf16_dev(xb), layout=0)
+    torch.cuda.synchronize()
+    assert to_np(p.gs)[0] == gs_ref[0]
+    assert np.array_equal(to_np(p.q)[:2], q_ref)
+    assert np.array_equal(to_np(p.sf)[:4].reshape(2, 2), sf_ref)
+
+
+def test_quantize_all_zero_tensor():
+    L = layer()
+    x = np.zeros((4, 128), dtype=np.uint16)
+    x[2, 7] = 0x8000
+    q_ref, sf_ref, gs_ref, st = oracle.quantize(x)
+    p = L.quantize(bf16_dev(x), layout=0)
+    torch.cuda.synchronize()
+    assert to_np(p.gs)[0] == 1.0 == gs_ref[0]
+    assert np.array_equal(to_np(p.q)[:4], q_ref)
+    assert (to_np(p.sf)[:32] == 0).all()
+
+
+def test_quantize_given_scale_and_nonfinite_status():
+    L = layer()
+    x = synthetic.gaussian_bf16(3, synthetic.STREAMS["x"], (64, 256))
+    gs = np.array([0.0123], dtype=np.float32)
+    q_ref, sf_ref, _, st = oracle.quantize(x, global_scale=gs)
+    p = L.quantize(bf16_dev(x), layout=0, global_scale=to_dev(gs))
+    torch.cuda.synchronize()
+    assert np.array_equal(to_np(p.q)[:64], q_ref)
+    assert np.array_equal(to_np(p.sf)[:64 * 16].reshape(64, 16), sf_ref)
+    for bad in (0x7FC0, 0x7F80, 0xFF80):
+        xb = x.copy()
+        xb[10, 100] = bad
+        for given in (None, to_dev(gs)):
+            s = status_word()
+            L.quantize(bf16_dev(xb), layout=0, global_scale=given, dev_status=s)
+            torch.cuda.synchronize()
+            assert int(s.item()) == oracle.ERR_NONFINITE == 16
+
+
+# --------------------------------------------------------------------------- dequantize
+@pytest.mark.parametrize("layout", [0, 1])
+def test_dequantize_bitexact(layout):
+    L = layer()
+    rng = np.random.default_rng(0)
+    R, K = 256, 256
+    q = rng.integers(0, 256, (R, K // 2), dtype=np.uint8)
+    sf = rng.integers(0, 0x7F, (R, K // 16), dtype=np.uint8)
+    gs = np.array([0.0371], dtype=np.float32)
+    ref32 = oracle.dequantize(q, sf, np.full(R, gs[0], np.float32))
+    ref16 = oracle.dequantize(q, sf, np.full(R, gs[0], np.float32), out="bf16")
+    sfd = tile(sf) if layout == 1 else sf.reshape(-1)
+    p = L.Packed(to_dev(q), to_dev(sfd), to_dev(gs), R, K, layout)
+    y32 = L.dequantize(p, 0)
+    y16 = L.dequantize(p, 1)
+    torch.cuda.synchronize()
+    assert np.array_equal(to_np(y32).view(np.uint32), ref32.view(np.uint32))
+    assert np.array_equal(to_np(y16), ref16)
+
+
+def test_dequantize_grouped_slots():
+    L = layer()
+    T, H, E = 128, 256, 5
+    x = synthetic.gaussian_bf16(4, synthetic.STREAMS["x"], (T, H))
+    r = synthetic.route_topk_softmax(4, T, E, 2)
+    q_ref, sf_ref, gs_ref, _ = oracle.quantize(x, r["row_index"], r["offsets"])
+    ref = oracle.dequantize(q_ref, sf_ref, oracle.rows_global_scale(gs_ref, r["offsets"], len(r["row_index"])))
+    p = L.quantize(bf16_dev(x), to_dev(r["row_index"]), to_dev(r["offsets"]), E, layout=1)
+    y = L.dequantize(p, 0)
+    torch.cuda.synchronize()
+    assert np.array_equal(to_np(y).view(np.uint32), ref.view(np.uint32))
+
+
+# --------------------------------------------------------------------------- remap
+def _mx(seed, n, rows, K, lo=-10):
+    q = synthetic.mxfp4_codes(seed, synthetic.STREAMS["mx_codes"], n * rows * K // 2).reshape(n * rows, K // 2)
+    e = synthetic.mxfp4_exponents(seed, synthetic.STREAMS["mx_exp"], n * rows * K // 32, lo=lo).reshape(n * rows, K // 32)
+    return q, e
+
+
+@pytest.mark.parametrize("layout", [0, 1])
+def test_remap_bitexact(layout):
+    L = layer()
+    n, rows, K = 3, 128, 512
+    q, e = _mx(0, n, rows, K)
+    q[5, :16] = 0x88                            # one all -0 block (exempt)
+    e[5, 0] = 3
+    q_ref, sf_ref, gs_ref, st = oracle.remap_mxfp4(q, e, n, rows, K)
+    assert st == 0
+    s = status_word()
+    p = L.remap_mxfp4(to_dev(q), to_dev(e), n, rows, K, layout=layout, dev_status=s)
+    torch.cuda.synchronize()
+    assert int(s.item()) == 0
+    assert np.array_equal(to_np(p.gs), gs_ref)
+    assert np.array_equal(to_np(p.q), q_ref)
+    sf = to_np(p.sf)
+    sf = untile(sf, n * rows, K // 16) if layout == 1 else sf.reshape(n * rows, K // 16)
+    assert np.array_equal(sf, sf_ref)
+    # lossless: the GPU's NVFP4 dequantizes to the MXFP4 values exactly
+    for t in range(n):
+        sl = slice(t * rows, (t + 1) * rows)
+        dq = oracle.dequantize_f64(to_np(p.q)[sl], sf[sl], np.full(rows, to_np(p.gs)[t], np.float32))
+        assert np.array_equal(dq, oracle.dequantize_mxfp4_f64(q[sl], e[sl]))
+
+
+def test_remap_errors_and_inplace():
+    L = layer()
+    rows, K = 128, 64
+    q = np.full((rows, K // 2), 0x22, dtype=np.uint8)
+    e = np.full((rows, K // 32), 127, dtype=np.uint8)
+    e[0, 0] = 127 + 8
+    e[3, 1] = 127 - 9
+    q_ref, sf_ref, gs_ref, st = oracle.remap_mxfp4(q, e, 1, rows, K)
+    qd = to_dev(q)
+    s = status_word()
+    p = L.remap_mxfp4(qd, to_dev(e), 1, rows, K, layout=0, dev_status=s, inplace=True)
+    torch.cuda.synchronize()
+    assert int(s.item()) == 0 and p.q.data_ptr() == qd.data_ptr()
+    assert np.array_equal(to_np(p.sf).reshape(rows, K // 16), sf_ref)
+    assert to_np(p.gs)[0] == gs_ref[0]
+    for bad in (127 - 10, 0xFF):
+        e2 = e.copy()
+        e2[3, 1] = bad
+        s = status_word()
+        L.remap_mxfp4(to_dev(q), to_dev(e2), 1, rows, K, layout=0, dev_status=s)
+        torch.cuda.synchronize()
+        assert int(s.item()) == oracle.ERR_NOT_REPRESENTABLE
+    # tiny exponents: subnormal global scale 2^g with g < -126
+    e3 = np.full((rows, K // 32), 2, dtype=np.uint8)
+    q3, sf3, gs3, st3 = oracle.remap_mxfp4(q, e3, 1, rows, K)
+    p3 = L.remap_mxfp4(to_dev(q), to_dev(e3), 1, rows, K, layout=0)
+    torch.cuda.synchronize()
+    assert to_np(p3.gs)[0] == gs3[0] and np.array_equal(to_np(p3.sf).reshape(rows, K // 16), sf3)
+
+
+# --------------------------------------------------------------------------- GEMM
+def _packed_weights(w_bits, E, N, K):
+    """Oracle-quantized weights [E*N, K], one global per expert, MMA-tiled scales."""
+    offs = np.arange(0, (E + 1) * N, N, dtype=np.int32)
+    q, sf, gs, st = oracle.quantize(w_bits, None, offs)
+    assert st == 0
+    return q, sf, gs
+
+
+def _packed_acts(x_bits, row_index, offsets, E):
+    q, sf, gs, st = oracle.quantize(x_bits, row_index, offsets)
+    assert st == 0
+    R, K2 = q.shape
+    rows, starts = slot_rows(offsets)
+    alloc = max(int(starts[-1]), 128)
+    alloc = (alloc + 127) // 128 * 128
+    qs = np.zeros((alloc, K2), np.uint8)
+    ss = np.zeros((alloc, K2 // 8), np.uint8)
+    qs[rows] = q
+    ss[rows] = sf
+    return q, sf, gs, qs, ss
+
+
+def _run_gemm(qs, ss, gs_a, qw, sfw, gs_w, offsets, E, R, N, K, out_dtype):
+    L = layer()
+    nv = nvmod()
+    bound = nv.nvfp4_padded_rows_bound(R, E)
+    qa = np.zeros((bound, K // 2), np.uint8)
+    qa[:qs.shape[0]] = qs
+    sa = np.zeros((((bound + 127) // 128) * 128, K // 16), np.uint8)
+    sa[:ss.shape[0]] = ss
+    a = L.Packed(to_dev(qa), to_dev(tile(sa)), to_dev(gs_a), R, K, 1,
+                 to_dev(offsets) if offsets is not None else None, E)
+    w = L.Packed(to_dev(qw), to_dev(tile(sfw)), to_dev(gs_w), qw.shape[0], K, 1)
+    s = status_word()
+    y = L.grouped_gemm(a, w, N, out_dtype, dev_status=s)
+    torch.cuda.synchronize()
+    assert int(s.item()) == 0
+    return to_np(y)
+
+
+def test_gemm_closed_form_integer_case():
+    """All scales 1.0 and s_g = 1: every product is a multiple of 1/4 and the
+    fp32 sum is exact, so the tensor-core result must equal the oracle exactly."""
+    rng = np.random.default_rng(0)
+    M, N, K = 128, 256, 512
+    qa = rng.integers(0, 256, (M, K // 2), dtype=np.uint8)
+    qw = rng.integers(0, 256, (N, K // 2), dtype=np.uint8)
+    sa = np.full((M, K // 16), 0x38, np.uint8)
+    sw = np.full((N, K // 16), 0x38, np.uint8)
+    one = np.ones(1, np.float32)
+    y = _run_gemm(qa, sa, one, qw, sw, one, None, 1, M, N, K, 0)
+    a = oracle.dequantize_f64(qa, sa, np.ones(M, np.float32))
+    b = oracle.dequantize_f64(qw, sw, np.ones(N, np.float32))
+    y_ref, _ = oracle.gemm_f64(a, b)
+    assert np.array_equal(y.astype(np.float64), y_ref)
+
+
+@pytest.mark.parametrize("out_dtype", [0, 1])
+def test_gemm_dense_config1(out_dtype):
+    M, N, K = 128, 256, 512
+    x = synthetic.gaussian_bf16(0, synthetic.STREAMS["x"], (M, K), outlier_frac=0.001)
+    w = synthetic.gaussian_bf16(0, synthetic.STREAMS["w"], (N, K), sigma=0.02)
+    qx, sx, gx, st = oracle.quantize(x)
+    qw, sw, gw = _packed_weights(w, 1, N, K)
+    y = _run_gemm(qx, sx, gx, qw, sw, gw, None, 1, M, N, K, out_dtype)
+    a = oracle.dequantize_f64(qx, sx, np.full(M, gx[0], np.float32))
+    b = oracle.dequantize_f64(qw, sw, np.full(N, gw[0], np.float32))
+    y_ref, s_ref = oracle.gemm_f64(a, b)
+    if out_dtype == 0:
+        ok, err, bound = gemm_tol(y, y_ref, s_ref)
+        assert ok.all(), (err.max(), (err / bound).max())
+    else:
+        y32 = _run_gemm(qx, sx, gx, qw, sw, gw, None, 1, M, N, K, 0)
+        assert np.array_equal(y, synthetic.f32_to_bf16_bits(y32))
+
+
+def test_gemm_grouped_ragged():
+    E, N, K = 6, 256, 512
+    counts = [0, 5, 130, 300, 16, 257]
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    R = int(offsets[-1])
+    x = synthetic.gaussian_bf16(5, synthetic.STREAMS["x"], (R, K), outlier_frac=0.001)
+    w = synthetic.gaussian_bf16(5, synthetic.STREAMS["w"], (E * N, K), sigma=0.02)
+    q, sf, gs, qs, ss = _packed_acts(x, None, offsets, E)
+    qw, sw, gw = _packed_weights(w, E, N, K)
+    y = _run_gemm(qs, ss, gs, qw, sw, gw, offsets, E, R, N, K, 0)
+    a = oracle.dequantize_f64(q, sf, oracle.rows_global_scale(gs, offsets, R))
+    bw = oracle.dequantize_f64(qw, sw, np.repeat(gw, N))
+    y_ref, s_ref = oracle.grouped_gemm_f64(a, bw.reshape(E, N, K), offsets)
+    ok, err, bound = gemm_tol(y, y_ref, s_ref)
+    assert ok.all(), (err.max(), (err / bound).max(), np.argwhere(~ok)[:5])
+
+
+def test_gemm_long_k_tolerance():
+    """K = 17408 (the dense MLP's down projection) on a thin slice."""
+    M, N, K = 64, 128, 17408
+    x = synthetic.gaussian_bf16(9, synthetic.STREAMS["x"], (M, K), outlier_frac=0.001)
+    w = synthetic.gaussian_bf16(9, synthetic.STREAMS["w"], (N, K), sigma=0.02)
+    qx, sx, gx, _ = oracle.quantize(x)
+    qw, sw, gw = _packed_weights(w, 1, N, K)
+    y = _run_gemm(qx, sx, gx, qw, sw, gw, None, 1, M, N, K, 0)
+    a = oracle.dequantize_f64(qx, sx, np.full(M, gx[0], np.float32))
+    b = oracle.dequantize_f64(qw, sw, np.full(N, gw[0], np.float32))
+    y_ref, s_ref = oracle.gemm_f64(a, b)
+    ok, err, bound = gemm_tol(y, y_ref, s_ref)
+    assert ok.all(), (err.max(), (err / bound).max())
+
+
+# --------------------------------------------------------------------------- SwiGLU + requantize
+@pytest.mark.parametrize("ydt", [0, 1])
+def test_swiglu_requantize(ydt):
+    L = layer()
+    E, I = 5, 256
+    counts = [3, 0, 140, 17, 40]
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    R = int(offsets[-1])
+    yb = synthetic.gaussian_bf16(11, synthetic.STREAMS["x"], (R, 2 * I))
+    yf = synthetic.bf16_bits_to_f32(yb) * np.float32(3.0)
+    yd = to_dev(yf) if ydt == 0 else bf16_dev(synthetic.f32_to_bf16_bits(yf))
+    yin = yf if ydt == 0 else synthetic.bf16_bits_to_f32(synthetic.f32_to_bf16_bits(yf))
+    p, h = L.swiglu_quantize(yd, to_dev(offsets), E, layout=1)
+    torch.cuda.synchronize()
+    h_gpu = to_np(h)
+    h_ref = oracle.swiglu(yin)
+    # h: within one bf16 ulp of the fp64 reference (device expf vs host exp)
+    d = np.abs(h_gpu.astype(np.int32) - h_ref.astype(np.int32))
+    assert (d <= 1).all() and (d == 0).mean() > 0.99
+    # requantize of the GPU's h is bit-exact with the oracle's quantizer
+    q_ref, sf_ref, gs_ref, st = oracle.quantize(h_gpu, None, offsets)
+    assert np.array_equal(to_np(p.gs), gs_ref)
+    rows, _ = slot_rows(offsets)
+    assert np.array_equal(to_np(p.q)[rows], q_ref)
+    assert np.array_equal(untile(to_np(p.sf), p.q.shape[0] // 128 * 128, I // 16)[rows], sf_ref)
+
+
+# --------------------------------------------------------------------------- KV cache
+@pytest.mark.parametrize("mode", [0, 1])
+def test_kv_quantize_dequantize(mode):
+    nv = nvmod()
+    L = layer()
+    T, Hh, D = 64, 4, 256
+    k = synthetic.gaussian_bf16(0, synthetic.STREAMS["kv_k"], (T * Hh, D))
+    v = synthetic.gaussian_bf16(0, synthetic.STREAMS["kv_v"], (T * Hh, D))
+    if mode == 1:
+        kg, vg = np.array([0.002], np.float32), np.array([0.0017], np.float32)
+        rk = oracle.quantize(k, global_scale=kg)
+        rv = oracle.quantize(v, global_scale=vg)
+    else:
+        rk, rv = oracle.quantize(k), oracle.quantize(v)
+    kd, vd = bf16_dev(k), bf16_dev(v)
+    kq = torch.empty((T * Hh, D // 2), dtype=torch.uint8, device="cuda")
+    vq = torch.empty_like(kq)
+    ks = torch.empty(T * Hh * D // 16, dtype=torch.uint8, device="cuda")
+    vs = torch.empty_like(ks)
+    kgs = to_dev(rk[2]) if mode == 1 else torch.empty(1, device="cuda")
+    vgs = to_dev(rv[2]) if mode == 1 else torch.empty(1, device="cuda")
+    s = status_word()
+    nv.nvfp4_kv_quantize(kd, vd, T, Hh, D, mode, kgs, vgs, kq, ks, vq, vs, L.workspace(2), s)
+    ko = torch.empty((T * Hh, D), dtype=torch.bfloat16, device="cuda")
+    vo = torch.empty_like(ko)
+    nv.nvfp4_kv_dequantize(kq, ks, kgs, vq, vs, vgs, T, Hh, D, ko, vo)
+    torch.cuda.synchronize()
+    assert int(s.item()) == 0
+    for (qr, sr, gr, _), qg, sg, gg, og in ((rk, kq, ks, kgs, ko), (rv, vq, vs, vgs, vo)):
+        assert to_np(gg)[0] == gr[0]
+        assert np.array_equal(to_np(qg), qr)
+        assert np.array_equal(to_np(sg).reshape(-1, D // 16), sr)
+        ref = oracle.dequantize(qr, sr, np.full(T * Hh, gr[0], np.float32), out="bf16")
+        assert np.array_equal(to_np(og), ref)
+
+
+# --------------------------------------------------------------------------- MoE layer
+def test_moe_layer_small_stagewise():
+    """gather-quantize -> gate_up -> SwiGLU+requant -> down, each stage against the oracle."""
+    L = layer()
+    T, H, I, E, k = 96, 256, 256, 8, 3
+    x = synthetic.gaussian_bf16(2, synthetic.STREAMS["x"], (T, H))
+    r = synthetic.route_topk_softmax(2, T, E, k)
+    off = r["offsets"]
+    R = len(r["row_index"])
+    wgu = synthetic.gaussian_bf16(2, synthetic.STREAMS["w_gate_up"], (E * 2 * I, H), sigma=0.02)
+    wd = synthetic.gaussian_bf16(2, synthetic.STREAMS["w_down"], (E * H, I), sigma=0.02)
+    qg, sg, gg = _packed_weights(wgu, E, 2 * I, H)
+    qd, sd, gd = _packed_weights(wd, E, H, I)
+    Wgu = L.Packed(to_dev(qg), to_dev(tile(sg)), to_dev(gg), E * 2 * I, H, 1)
+    Wd = L.Packed(to_dev(qd), to_dev(tile(sd)), to_dev(gd), E * H, I, 1)
+    moe = L.MoEExperts(Wgu, Wd, E, H, I, max_rows=R, out_dtype=0, mid_dtype=0)
+    s = status_word()
+    y2 = moe.forward(bf16_dev(x), to_dev(r["row_index"]), to_dev(off), dev_status=s)
+    torch.cuda.synchronize()
+    assert int(s.item()) == 0
+    # stage 1: gather-quantize
+    q1, sf1, gs1, _ = oracle.quantize(x, r["row_index"], off)
+    rows, _ = slot_rows(off)
+    assert np.array_equal(to_np(moe.a1.q)[rows], q1)
+    # stage 2: gate_up GEMM (fp32) against the fp64 oracle on the same operands
+    a1 = oracle.dequantize_f64(q1, sf1, oracle.rows_global_scale(gs1, off, R))
+    bgu = oracle.dequantize_f64(qg, sg, np.repeat(gg, 2 * I)).reshape(E, 2 * I, H)
+    y1_ref, s1_ref = oracle.grouped_gemm_f64(a1, bgu, off)
+    y1 = to_np(moe.y1[:R])
+    ok, err, bound = gemm_tol(y1, y1_ref, s1_ref)
+    assert ok.all(), (err / bound).max()
+    # stage 3: SwiGLU of the GPU's y1, requantized
+    h = to_np(moe.h[:R])
+    d = np.abs(h.astype(np.int32) - oracle.swiglu(y1).astype(np.int32))
+    assert (d <= 1).all()
+    q2, sf2, gs2, _ = oracle.quantize(h, None, off)
+    assert np.array_equal(to_np(moe.a2.q)[rows], q2)
+    # stage 4: down GEMM on the GPU's quantized h
+    a2 = oracle.dequantize_f64(q2, sf2, oracle.rows_global_scale(gs2, off, R))
+    bd = oracle.dequantize_f64(qd, sd, np.repeat(gd, H)).reshape(E, H, I)
+    y2_ref, s2_ref = oracle.grouped_gemm_f64(a2, bd, off)
+    ok, err, bound = gemm_tol(to_np(y2), y2_ref, s2_ref)
+    assert ok.all(), (err / bound).max()
+
+
+def test_device_generator_matches_host():
+    import synthetic.cuda as sc
+    g = sc.gaussian_bf16(3, 5, (1000, 64), sigma=0.02, start=12345)
+    h = synthetic.gaussian_bf16(3, 5, (1000, 64), sigma=0.02, start=12345)
+    assert np.array_equal(to_np(g), h)
+    g = sc.gaussian_bf16(3, 5, (777,))
+    assert np.array_equal(to_np(g), synthetic.gaussian_bf16(3, 5, (777,)))
+    c = sc.mxfp4_codes(1, 9, 4096, start_byte=64)
+    assert np.array_equal(to_np(c), synthetic.mxfp4_codes(1, 9, 4096, start_byte=64))
+    e = sc.mxfp4_exponents(1, 10, 999, lo=-10, start=7)
+    assert np.array_equal(to_np(e), synthetic.mxfp4_exponents(1, 10, 999, lo=-10, start=7))
