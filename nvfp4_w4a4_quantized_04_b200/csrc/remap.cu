@@ -76,7 +76,7 @@ __global__ void __launch_bounds__(256) remap_scale_kernel(
     const int g = hi ? (int)hi - 1 - 127 - 8 : 0;
     const int64_t within = i - t * per_tensor;
     if (within == 0) {
-      gs[t] = __uint_as_float((uint32_t)(127 + g) << 23);   // 2^g, g in [-135, 120]
+      gs[t] = ldexpf(1.0f, g);   // 2^g exactly, g in [-135, 119] (subnormal below -126)
       if (hi) {
         const int emin = 256 - (int)lo - 127;
         if (emin - g < -9) report(dev_status, NVFP4_ERR_NOT_REPRESENTABLE);

@@ -62,7 +62,7 @@ def test_quantize_dense_config1_bitexact(layout):
 @pytest.mark.parametrize("layout", [0, 1])
 def test_quantize_grouped_gather_bitexact(layout):
     L = layer()
-    T, H, E, k = 256, 512, 12, 2
+    T, H, E, k = 1024, 512, 12, 2
     x = synthetic.gaussian_bf16(1, synthetic.STREAMS["x"], (T, H))
     r = synthetic.route_topk_softmax(1, T, E, k)
     counts = np.diff(r["offsets"])
