@@ -1,15 +1,22 @@
-"""Benchmark: NVFP4 W4A4 routed-expert MoE layer on B200.
+"""Benchmark: NVFP4 W4A4 routed-expert path on B200.
 
-One step = one pass of the hot path over one batch: gather + per-expert
-dynamic NVFP4 quantize of the routed activations -> block-scaled FP4 grouped
-gate_up GEMM -> SwiGLU + per-expert requantize -> grouped down GEMM, for the
-MoE layer with 512 experts, top-10 routing, 8192 tokens, hidden 4096, expert
-intermediate 1024 (weights resident in HBM as NVFP4).
+Headline step = one pass of the hot path over one batch of the MoE layer
+with 512 experts, top-10 routing, 8192 tokens, hidden 4096, expert
+intermediate 1024: gather + per-expert dynamic NVFP4 quantize of the routed
+activations -> block-scaled FP4 grouped gate_up GEMM -> SwiGLU + per-expert
+requantize -> grouped down GEMM (weights resident in HBM as NVFP4).
+
+The other rows of the path are measured in the same run as "components":
+the dense MLP (4096 tokens, 5120 -> 2x17408 -> 5120), the decode MoE (384
+experts, 64 tokens, Zipf routing, MXFP4 weights remapped to NVFP4), the
+NVFP4 KV cache (4 heads x 256 x 262144 tokens, K and V), the activation
+quantize sweep [T, 5120] and the MXFP4 -> NVFP4 remap of 2^28 elements.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-Under torchrun each rank runs its own replica (independent batch, its own
-experts): weak scaling, no collective in the data path; timing is the max
-over ranks.  Rank 0 prints one JSON line.
+       [--experts E --tokens T] [--components all|none|<name,...>] [--no-cpu-baseline]
+Under torchrun each rank runs its own replica (its own batch and experts):
+weak scaling, no collective in the data path; timing is the max over ranks.
+Rank 0 prints one JSON line.
 """
 from __future__ import annotations
 
@@ -28,23 +35,21 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "NVFP4 W4A4 expert GEMM TFLOPS & % FP4 peak; quantize GB/s & % HBM"
-WORKLOAD = "moe_routed_experts_e512_top10_t8192_h4096_i1024"
-CFG = dict(E=512, topk=10, T=8192, H=4096, I=1024, seed=0)
-
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-FP4_OVER_BF16 = 9.0 / 2.25      # nominal dense ratio (4x)
+FP4_OVER_BF16 = 9.0 / 2.25      # nominal dense FP4 / BF16 tensor ratio
+L2_BYTES = 126 << 20
 
 
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
-        d = json.load(open(p))
-        return d, "measured"
+        return json.load(open(p)), "measured"
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def moe_flops(R, H, I):
-    return 2.0 * R * (2 * I * H + H * I)
+PEAKS, PEAKS_KIND = load_peaks()
+HBM_PEAK = PEAKS.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+FP4_PEAK = PEAKS.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]) * FP4_OVER_BF16
 
 
 # --------------------------------------------------------------------------- clocks
@@ -54,9 +59,7 @@ class ClockSampler:
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, gpu_index: int):
-        self.idx = gpu_index
-        self.proc = None
-        self.path = None
+        self.idx, self.proc, self.path = gpu_index, None, None
 
     def start(self):
         try:
@@ -77,44 +80,88 @@ class ClockSampler:
             self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
-        rows = []
-        for line in open(self.path):
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) >= 9:
-                rows.append(parts)
+        rows = [[p.strip() for p in line.split(",")] for line in open(self.path)]
+        rows = [r for r in rows if len(r) >= 9]
         os.unlink(self.path)
         if not rows:
             return out
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+
+        def num(v):
+            try:
+                return float(v)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        mx = [num(r[2]) for r in rows if num(r[2]) is not None]
+        pw = [num(r[3]) for r in rows if num(r[3]) is not None]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
         out.update(sm_mhz=statistics.median(sm) if sm else None, sm_max_mhz=max(mx) if mx else None,
-                   reasons=reasons, samples=len(rows))
+                   reasons=reasons, samples=len(rows), power_w_max=max(pw) if pw else None)
         return out
 
 
-# --------------------------------------------------------------------------- setup
-def setup_moe(device, seed):
+# --------------------------------------------------------------------------- timing helpers
+def timed(fn, iters, warmup, flush=None):
+    """Median device time (ms) of fn() over iters, CUDA events on the current
+    stream; L2 flushed between iterations (outside the events) when given."""
+    import torch
+    s = torch.cuda.current_stream()
+    for _ in range(max(3, warmup)):
+        fn()
+    ts = []
+    for i in range(iters):
+        if flush is not None:
+            flush.fill_(i & 0xFF)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(s)
+        fn()
+        b.record(s)
+        b.synchronize()
+        ts.append(a.elapsed_time(b))
+    return statistics.median(ts)
+
+
+def gbs(nbytes, ms):
+    return nbytes / (ms * 1e-3) / 1e9
+
+
+def moe_flops(R, H, I):
+    return 2.0 * R * (2 * I * H + H * I)
+
+
+def gemm_bytes(R, e_touched, N, K, out_bytes=2):
+    """Algorithmic bytes of one grouped GEMM launch: the touched experts'
+    packed weights (0.5625 B/element) and the packed activations, each read
+    once, and the output written once."""
+    return e_touched * N * K * 0.5625 + R * K * 0.5625 + R * N * out_bytes
+
+
+def pack_weights(w_bf16, E, rows_per, ws):
+    """Static NVFP4 quantization of [E*rows_per, K] weights, one global per expert."""
+    import torch
+    from nvfp4_w4a4_quantized_04_b200 import layer as L
+    offs = torch.arange(0, (E + 1) * rows_per, rows_per, dtype=torch.int32, device=w_bf16.device)
+    p = L.quantize(w_bf16, None, offs, E, layout=1, ws=ws)
+    p.offsets, p.num_groups, p.rows = None, 1, E * rows_per
+    return p
+
+
+# --------------------------------------------------------------------------- headline: MoE layer
+def setup_moe(device, seed, E, T, H, I, topk):
     import torch
 
     import synthetic
     import synthetic.cuda as sc
     from nvfp4_w4a4_quantized_04_b200 import layer as L
 
-    E, k, T, H, I = CFG["E"], CFG["topk"], CFG["T"], CFG["H"], CFG["I"]
-    r = synthetic.route_topk_softmax(seed, T, E, k)
+    r = synthetic.route_topk_softmax(seed, T, E, topk)
     R = len(r["row_index"])
     ws = L.workspace(E, device)
-    # weights: N(0, 0.02^2) bf16 generated on the device, quantized statically
-    # (one global scale per expert and projection) by the same library.
     packs = []
     for name, rows_per, K in (("w_gate_up", 2 * I, H), ("w_down", H, I)):
         w = sc.gaussian_bf16(seed, synthetic.STREAMS[name], (E * rows_per, K), sigma=0.02)
-        offs = torch.arange(0, (E + 1) * rows_per, rows_per, dtype=torch.int32, device=device)
-        p = L.quantize(w, None, offs, E, layout=1, ws=ws)
-        p.offsets, p.num_groups, p.rows = None, 1, E * rows_per
-        packs.append(p)
+        packs.append(pack_weights(w, E, rows_per, ws))
         del w
     torch.cuda.synchronize()
     x = sc.gaussian_bf16(seed, synthetic.STREAMS["x"], (T, H))
@@ -124,79 +171,65 @@ def setup_moe(device, seed):
     return moe, x, ri, off, r, R
 
 
-def gemm_bytes(R, E_touched, N, K, out_bytes=2):
-    """Algorithmic bytes of one grouped GEMM: touched expert weights + packed
-    activations, each read once, plus the output written once."""
-    w = E_touched * N * K * 0.5625
-    a = R * K * 0.5625
-    return w + a + R * N * out_bytes
-
-
-def run_ours(args, rank, world, device):
+def run_headline(args, rank, world, device):
     import torch
     import torch.distributed as dist
+    from nvfp4_w4a4_quantized_04_b200 import layer as L
 
-    peaks, peaks_kind = load_peaks()
-    moe, x, ri, off, r, R = setup_moe(device, CFG["seed"] + rank)
-    E, H, I = CFG["E"], CFG["H"], CFG["I"]
+    E, T, H, I, k = args.experts, args.tokens, 4096, 1024, 10
+    moe, x, ri, off, r, R = setup_moe(device, rank, E, T, H, I, k)
     flops = moe_flops(R, H, I)
     e_touched = int((np.diff(r["offsets"]) > 0).sum())
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream()
 
-    def step():
-        return moe.forward(x, ri, off)
+    def stages(evs=None):
+        rec = (lambda i: evs[i].record(stream)) if evs else (lambda i: None)
+        rec(0)
+        a1 = L.quantize(x, ri, off, E, layout=1, out=moe.a1, ws=moe.ws, rows=R)
+        rec(1)
+        L.grouped_gemm(a1, moe.w_gate_up, 2 * I, moe.mid_dtype, y=moe.y1[:R])
+        rec(2)
+        a2, _ = L.swiglu_quantize(moe.y1[:R], off, E, layout=1, out=moe.a2, h=moe.h[:R], ws=moe.ws)
+        rec(3)
+        L.grouped_gemm(a2, moe.w_down, H, moe.out_dtype, y=moe.y2[:R])
+        rec(4)
 
     for _ in range(max(3, args.warmup)):
-        step()
+        stages()
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
 
-    # timed region: per-step events, L2 flushed between steps (outside the events)
     clocks = ClockSampler(torch.cuda.current_device())
     clocks.start()
-    time.sleep(0.3)
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-           torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    torch.cuda.synchronize()
-    from nvfp4_w4a4_quantized_04_b200 import layer as L
+    time.sleep(0.25)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     for i in range(args.steps):
-        flush.fill_(i & 0xFF)
-        s0, g0, g1, s1 = ev[i]
-        s0.record(stream)
-        a1 = L.quantize(x, ri, off, E, layout=1, out=moe.a1, ws=moe.ws, rows=R)
-        g0.record(stream)
-        L.grouped_gemm(a1, moe.w_gate_up, 2 * I, moe.mid_dtype, y=moe.y1[:R])
-        g1.record(stream)
-        a2, _ = L.swiglu_quantize(moe.y1[:R], off, E, layout=1, out=moe.a2, h=moe.h[:R], ws=moe.ws)
-        L.grouped_gemm(a2, moe.w_down, H, moe.out_dtype, y=moe.y2[:R])
-        s1.record(stream)
+        flush.fill_(i & 0xFF)               # L2 flush between steps, outside the events
+        stages(evs[i])
     torch.cuda.synchronize()
+    time.sleep(0.15)
     clk = clocks.stop()
-    step_ms = [e[0].elapsed_time(e[3]) for e in ev]
-    gemm_ms = [e[1].elapsed_time(e[2]) for e in ev]
-    total_ms = sum(step_ms)
+    per = np.array([[e[j].elapsed_time(e[j + 1]) for j in range(4)] for e in evs])
+    step_ms = per.sum(axis=1)
+    total_ms = float(step_ms.sum())
     t = torch.tensor([total_ms], dtype=torch.float64, device=device)
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     total_ms = float(t.item())
-    ms_per_step = total_ms / args.steps
     value = world * flops * args.steps / (total_ms * 1e-3) / 1e12
 
-    # e2e through the public API with host buffers: H2D inputs, D2H result
-    x_host = x.cpu().pin_memory()
-    ri_host = ri.cpu().pin_memory()
-    off_host = off.cpu().pin_memory()
+    # e2e through the public API with host buffers: pinned H2D of the step's
+    # inputs, the layer, D2H of its result, all inside the timed region
+    x_host, ri_host, off_host = x.cpu().pin_memory(), ri.cpu().pin_memory(), off.cpu().pin_memory()
     y_host = torch.empty((R, H), dtype=torch.bfloat16).pin_memory()
-    x_d = torch.empty_like(x)
-    ri_d = torch.empty_like(ri)
-    off_d = torch.empty_like(off)
-    e2e_steps = max(2, min(args.steps, 5))
+    x_d, ri_d, off_d = torch.empty_like(x), torch.empty_like(ri), torch.empty_like(off)
+    n_e2e = max(2, min(args.steps, 5))
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(e2e_steps):
+    for _ in range(n_e2e):
         x_d.copy_(x_host, non_blocking=True)
         ri_d.copy_(ri_host, non_blocking=True)
         off_d.copy_(off_host, non_blocking=True)
@@ -204,7 +237,7 @@ def run_ours(args, rank, world, device):
         y_host.copy_(y, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    e2e_ms = e0.elapsed_time(e1) / n_e2e
     t = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -212,58 +245,241 @@ def run_ours(args, rank, world, device):
     h2d = x.numel() * 2 + ri.numel() * 4 + off.numel() * 4
     d2h = R * H * 2
 
-    # roofline of the dominant kernel (gate_up grouped GEMM), HBM-bound at this shape
-    gemm_avg_s = statistics.mean(gemm_ms) * 1e-3
-    gbytes = gemm_bytes(R, e_touched, 2 * I, H, out_bytes=2)
-    g_flops = 2.0 * R * 2 * I * H
-    fp4_peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]) * FP4_OVER_BF16
-    hbm_peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
-    roof = {"bound": "hbm", "kernel": "nvfp4::gemm::grouped_gemm_kernel (gate_up)",
-            "achieved": round(gbytes / gemm_avg_s / 1e9, 1), "peak": hbm_peak, "unit": "GB/s",
-            "frac": round(gbytes / gemm_avg_s / 1e9 / hbm_peak, 4), "traffic": None,
-            "peak_source": f"{peaks_kind} hbm_gbs",
-            "tensor_tflops": round(g_flops / gemm_avg_s / 1e12, 1),
-            "pct_fp4_peak": round(100 * g_flops / gemm_avg_s / 1e12 / fp4_peak, 2),
-            "fp4_peak_tflops": round(fp4_peak, 1),
-            "algorithmic_bytes_per_launch": int(gbytes), "gemm_ms": round(1e3 * gemm_avg_s, 4)}
-
-    out = {
+    med = np.median(per, axis=0)
+    g1_ms, g2_ms = float(np.mean(per[:, 1])), float(np.mean(per[:, 3]))
+    g1_bytes = gemm_bytes(R, e_touched, 2 * I, H)
+    g1_flops = 2.0 * R * 2 * I * H
+    g2_bytes = gemm_bytes(R, e_touched, H, I)
+    g2_flops = 2.0 * R * H * I
+    roof = {"bound": "hbm", "kernel": "nvfp4::gemm::grouped_gemm_kernel (gate_up launch)",
+            "achieved": round(gbs(g1_bytes, g1_ms), 1), "peak": HBM_PEAK, "unit": "GB/s",
+            "frac": round(gbs(g1_bytes, g1_ms) / HBM_PEAK, 4), "traffic": None,
+            "peak_source": f"{PEAKS_KIND} hbm_gbs (burst copy)",
+            "algorithmic_bytes_per_launch": int(g1_bytes), "avg_launch_ms": round(g1_ms, 4),
+            "tensor_tflops": round(g1_flops / (g1_ms * 1e-3) / 1e12, 1),
+            "pct_fp4_peak": round(100 * g1_flops / (g1_ms * 1e-3) / 1e12 / FP4_PEAK, 2),
+            "fp4_peak_tflops": round(FP4_PEAK, 1),
+            "fp4_peak_source": f"{PEAKS_KIND} bf16_tflops x 4 (nominal fp4/bf16 ratio)"}
+    breakdown = {
+        "gather_quantize_ms": round(float(med[0]), 4),
+        "gate_up_gemm_ms": round(float(med[1]), 4),
+        "swiglu_requantize_ms": round(float(med[2]), 4),
+        "down_gemm_ms": round(float(med[3]), 4),
+        "gate_up_gbs": round(gbs(g1_bytes, g1_ms), 1), "gate_up_tflops": round(g1_flops / (g1_ms * 1e-3) / 1e12, 1),
+        "down_gbs": round(gbs(g2_bytes, g2_ms), 1), "down_tflops": round(g2_flops / (g2_ms * 1e-3) / 1e12, 1),
+        "layer_roofline_ms": round(1e3 * max((g1_bytes + g2_bytes) / (HBM_PEAK * 1e9),
+                                             flops / (FP4_PEAK * 1e12)), 4),
+    }
+    workload = f"moe_routed_experts_e{E}_top{k}_t{T}_h{H}_i{I}"
+    return {
         "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
-        "warmup": max(3, args.warmup), "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e2m1, e4m3 block scales) -> fp32 accum, bf16 io",
-        "data": "synthetic (seeded SplitMix64 / Irwin-Hall N(0,1) activations, N(0,0.02^2) weights, softmax top-10 routing)",
-        "config": {"workload": WORKLOAD, "experts": E, "topk": CFG["topk"], "tokens": CFG["T"], "hidden": H,
-                   "intermediate": I, "routed_rows": R, "experts_touched": e_touched,
-                   "flops_per_step": flops, "l2": "flushed between steps (256 MB write)",
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "warmup": max(3, args.warmup), "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4 e2m1 x e2m1 (e4m3 block scales), fp32 accumulate, bf16 io",
+        "data": "synthetic: seeded SplitMix64 / Irwin-Hall N(0,1) activations, N(0,0.02^2) weights, softmax top-10 routing",
+        "config": {"workload": workload, "experts": E, "topk": k, "tokens": T, "hidden": H, "intermediate": I,
+                   "routed_rows": R, "experts_touched": e_touched, "flops_per_step": flops,
+                   "l2": "flushed between steps (256 MB write, outside the timed events)",
+                   "parallelism": f"{world} independent replicas" if world > 1 else "single GPU"},
         "roofline": roof,
+        "breakdown": breakdown,
         "e2e": {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": round(e2e_ms, 3)},
         "gpu_launches": 8 * args.steps,
         "clocks": clk,
     }
+
+
+# --------------------------------------------------------------------------- components
+def comp_dense_mlp(device, iters, warmup, flush):
+    """Dense MLP of the 64-layer hybrid model, one layer: 4096 tokens, hidden
+    5120, intermediate 17408, X with 0.1% outliers x50."""
+    import torch
+
+    import synthetic
+    import synthetic.cuda as sc
+    from nvfp4_w4a4_quantized_04_b200 import layer as L
+    M, H, I = 4096, 5120, 17408
+    ws = L.workspace(1, device)
+    wgu = pack_weights(sc.gaussian_bf16(0, synthetic.STREAMS["w_gate_up"], (2 * I, H), sigma=0.02), 1, 2 * I, ws)
+    wd = pack_weights(sc.gaussian_bf16(0, synthetic.STREAMS["w_down"], (H, I), sigma=0.02), 1, H, ws)
+    xb = synthetic.gaussian_bf16(0, synthetic.STREAMS["x"], (M, H), outlier_frac=0.001)
+    x = torch.from_numpy(xb.view(np.int16)).to(device).view(torch.bfloat16)
+    a1 = L.empty_packed(M, H, 1, None, 1, device)
+    a2 = L.empty_packed(M, I, 1, None, 1, device)
+    y1 = torch.empty((M, 2 * I), dtype=torch.bfloat16, device=device)
+    h = torch.empty((M, I), dtype=torch.bfloat16, device=device)
+    y2 = torch.empty((M, H), dtype=torch.bfloat16, device=device)
+    t = {}
+
+    def q():
+        L.quantize(x, layout=1, out=a1, ws=ws)
+
+    def g1():
+        L.grouped_gemm(a1, wgu, 2 * I, 1, y=y1)
+
+    def sq():
+        L.swiglu_quantize(y1, None, 1, layout=1, out=a2, h=h, ws=ws)
+
+    def g2():
+        L.grouped_gemm(a2, wd, H, 1, y=y2)
+
+    def layer():
+        q(); g1(); sq(); g2()
+    for name, fn in (("quantize", q), ("gate_up", g1), ("swiglu_requantize", sq), ("down", g2), ("layer", layer)):
+        t[name] = timed(fn, iters, warmup, flush)
+    f1, f2 = 2.0 * M * 2 * I * H, 2.0 * M * H * I
+    tf = (f1 + f2) / (t["layer"] * 1e-3) / 1e12
+    return {"workload": "dense_mlp_t4096_h5120_i17408", "layer_ms": round(t["layer"], 4),
+            "layer_tflops": round(tf, 1), "pct_fp4_peak": round(100 * tf / FP4_PEAK, 2),
+            "gate_up_ms": round(t["gate_up"], 4), "gate_up_tflops": round(f1 / (t["gate_up"] * 1e-3) / 1e12, 1),
+            "gate_up_pct_fp4_peak": round(100 * f1 / (t["gate_up"] * 1e-3) / 1e12 / FP4_PEAK, 2),
+            "down_ms": round(t["down"], 4), "down_tflops": round(f2 / (t["down"] * 1e-3) / 1e12, 1),
+            "quantize_ms": round(t["quantize"], 4), "swiglu_requantize_ms": round(t["swiglu_requantize"], 4),
+            "roofline": {"bound": "tensor", "peak_tflops": round(FP4_PEAK, 1),
+                         "frac": round(tf / FP4_PEAK, 4)}}
+
+
+def comp_decode_moe(device, iters, warmup, flush):
+    """Decode MoE: 384 experts, 64 tokens, top-10 Zipf(1.1) routing (seed 7),
+    hidden 7168, intermediate 2048, weights generated as MXFP4 and remapped."""
+    import torch
+
+    import synthetic
+    import synthetic.cuda as sc
+    from nvfp4_w4a4_quantized_04_b200 import layer as L
+    E, T, H, I, k = 384, 64, 7168, 2048, 10
+    r = synthetic.route_zipf_gumbel(7, T, E, k)
+    R = len(r["row_index"])
+    ws = L.workspace(2 * E, device)
+    packs, remap_ms, remap_bytes = [], 0.0, 0.0
+    for name, rows_per, K in (("gate_up", 2 * I, H), ("down", H, I)):
+        n = E * rows_per * K
+        q = sc.mxfp4_codes(7, synthetic.STREAMS["mx_codes_" + name], n // 2).view(E * rows_per, K // 2)
+        e8 = sc.mxfp4_exponents(7, synthetic.STREAMS["mx_exp_" + name], n // 32, lo=-10)
+        qn = torch.empty_like(q)
+        sf = torch.empty(n // 16, dtype=torch.uint8, device=device)
+        gs = torch.empty(E, dtype=torch.float32, device=device)
+        st = torch.zeros(1, dtype=torch.int32, device=device)
+        from nvfp4_w4a4_quantized_04_b200 import mxfp4_to_nvfp4
+
+        def remap():
+            mxfp4_to_nvfp4(q, e8, E, rows_per, K, qn, sf, 1, gs, ws, st)
+        remap_ms += timed(remap, max(2, iters // 2), 1, flush)
+        remap_bytes += n * (0.5 + 1 / 32) + n * (0.5 + 1 / 16)
+        assert int(st.item()) == 0
+        packs.append(L.Packed(qn, sf, gs, E * rows_per, K, 1))
+        del q, e8
+    xb = sc.gaussian_bf16(7, synthetic.STREAMS["x"], (T, H))
+    moe = L.MoEExperts(packs[0], packs[1], E, H, I, max_rows=R, out_dtype=1, mid_dtype=1, device=device)
+    ri = torch.from_numpy(r["row_index"]).to(device)
+    off = torch.from_numpy(r["offsets"]).to(device)
+    ms = timed(lambda: moe.forward(xb, ri, off), iters, warmup, flush)
+    touched = int((np.diff(r["offsets"]) > 0).sum())
+    wbytes = touched * (2 * I * H + H * I) * 0.5625
+    return {"workload": "decode_moe_e384_top10_zipf1.1_t64_h7168_i2048", "experts_touched": touched,
+            "routed_rows": R, "layer_ms": round(ms, 4),
+            "touched_weight_gbs": round(gbs(wbytes, ms), 1),
+            "roofline": {"bound": "hbm", "frac": round(gbs(wbytes, ms) / HBM_PEAK, 4), "peak": HBM_PEAK},
+            "remap_ms": round(remap_ms, 4), "remap_gbs": round(gbs(remap_bytes, remap_ms), 1)}
+
+
+def comp_kv(device, iters, warmup, flush):
+    """NVFP4 KV cache for one full-attention layer: K, V [262144 tokens, 4, 256]."""
+    import torch
+
+    import synthetic
+    import synthetic.cuda as sc
+    from nvfp4_w4a4_quantized_04_b200 import layer as L, nvfp4_kv_dequantize, nvfp4_kv_quantize
+    T, Hh, D = 262144, 4, 256
+    n = T * Hh * D
+    k = sc.gaussian_bf16(0, synthetic.STREAMS["kv_k"], (T * Hh, D))
+    v = sc.gaussian_bf16(0, synthetic.STREAMS["kv_v"], (T * Hh, D))
+    kq, vq = (torch.empty((T * Hh, D // 2), dtype=torch.uint8, device=device) for _ in range(2))
+    ks, vs = (torch.empty(n // 16, dtype=torch.uint8, device=device) for _ in range(2))
+    kg, vg = (torch.empty(1, dtype=torch.float32, device=device) for _ in range(2))
+    ko, vo = torch.empty_like(k), torch.empty_like(v)
+    ws = L.workspace(2, device)
+    nvfp4_kv_quantize(k, v, T, Hh, D, 0, kg, vg, kq, ks, vq, vs, ws)
+    t_amax = timed(lambda: nvfp4_kv_quantize(k, v, T, Hh, D, 0, kg, vg, kq, ks, vq, vs, ws), iters, warmup, flush)
+    t_given = timed(lambda: nvfp4_kv_quantize(k, v, T, Hh, D, 1, kg, vg, kq, ks, vq, vs, ws), iters, warmup, flush)
+    t_dq = timed(lambda: nvfp4_kv_dequantize(kq, ks, kg, vq, vs, vg, T, Hh, D, ko, vo), iters, warmup, flush)
+    b_given = 2 * n * (2 + 0.5625)
+    b_amax = 2 * n * (2 + 2 + 0.5625)
+    b_dq = 2 * n * (0.5625 + 2)
+    return {"workload": "kv_cache_t262144_h4_d256_k_and_v",
+            "quantize_given_scale_ms": round(t_given, 4), "quantize_given_scale_gbs": round(gbs(b_given, t_given), 1),
+            "quantize_given_scale_frac_hbm": round(gbs(b_given, t_given) / HBM_PEAK, 4),
+            "quantize_amax_ms": round(t_amax, 4), "quantize_amax_gbs": round(gbs(b_amax, t_amax), 1),
+            "quantize_amax_frac_hbm": round(gbs(b_amax, t_amax) / HBM_PEAK, 4),
+            "dequantize_ms": round(t_dq, 4), "dequantize_gbs": round(gbs(b_dq, t_dq), 1),
+            "dequantize_frac_hbm": round(gbs(b_dq, t_dq) / HBM_PEAK, 4)}
+
+
+def comp_act_sweep(device, iters, warmup, flush):
+    """Standalone dynamic activation quantize on [T, 5120] bf16."""
+    import torch
+
+    import synthetic
+    import synthetic.cuda as sc
+    from nvfp4_w4a4_quantized_04_b200 import layer as L
+    out = {}
+    H = 5120
+    ws = L.workspace(1, device)
+    for T in (1, 64, 1024, 16384, 131072):
+        x = sc.gaussian_bf16(0, synthetic.STREAMS["x_sweep"], (T, H))
+        p = L.empty_packed(T, H, 1, None, 1, device)
+        ms = timed(lambda: L.quantize(x, layout=1, out=p, ws=ws), iters, warmup, flush)
+        per_el = 2.5625 if T * H * 2 <= L2_BYTES // 2 else 4.5625
+        b = T * H * per_el
+        out[f"T{T}"] = {"us": round(ms * 1e3, 2), "gbs": round(gbs(b, ms), 1),
+                        "frac_hbm": round(gbs(b, ms) / HBM_PEAK, 4), "bytes_per_element": per_el}
+        del x, p
     return out
+
+
+def comp_remap(device, iters, warmup, flush):
+    """MXFP4 -> NVFP4 remap of 2^28 elements as 1024 tensors of [512, 512]."""
+    import torch
+
+    import synthetic
+    import synthetic.cuda as sc
+    from nvfp4_w4a4_quantized_04_b200 import layer as L, mxfp4_to_nvfp4
+    nt, rows, K = 1024, 512, 512
+    n = nt * rows * K
+    q = sc.mxfp4_codes(0, synthetic.STREAMS["mx_codes"], n // 2).view(nt * rows, K // 2)
+    e8 = sc.mxfp4_exponents(0, synthetic.STREAMS["mx_exp"], n // 32)
+    qn = torch.empty_like(q)
+    sf = torch.empty(n // 16, dtype=torch.uint8, device=device)
+    gs = torch.empty(nt, dtype=torch.float32, device=device)
+    ws = L.workspace(nt, device)
+    ms = timed(lambda: mxfp4_to_nvfp4(q, e8, nt, rows, K, qn, sf, 1, gs, ws), iters, warmup, flush)
+    b = n * (0.5 + 1 / 32) + n * (0.5 + 1 / 16)
+    return {"workload": "remap_2^28_as_1024x512x512", "ms": round(ms, 4), "gbs": round(gbs(b, ms), 1),
+            "frac_hbm": round(gbs(b, ms) / HBM_PEAK, 4)}
+
+
+COMPONENTS = {"dense_mlp": comp_dense_mlp, "decode_moe": comp_decode_moe, "kv_cache": comp_kv,
+              "act_quant_sweep": comp_act_sweep, "remap": comp_remap}
 
 
 # --------------------------------------------------------------------------- CPU oracle baseline
 _SAMPLE_INPUTS = {}
 
 
-def oracle_sample(seconds: float, seed: int = 0):
-    """Time the oracle on a bounded sample of the same workload: whole experts
-    (their routed rows) through gather-quantize, fp64 gate_up, SwiGLU,
-    requantize and fp64 down, until ``seconds`` of CPU work.  Returns
-    (TFLOP/s, experts done, rows done, threads)."""
+def oracle_sample(seconds: float, seed: int = 0, E=512, T=8192, H=4096, I=1024, k=10):
+    """Time the oracle on a bounded sample of the headline workload: whole
+    experts (their routed rows) through gather-quantize, fp64 gate_up,
+    SwiGLU, requantize and fp64 down, until ``seconds`` of CPU work.
+    Returns (TFLOP/s, experts done, rows done, seconds of work)."""
     import oracle
     import synthetic
 
-    E, k, T, H, I = CFG["E"], CFG["topk"], CFG["T"], CFG["H"], CFG["I"]
-    if seed not in _SAMPLE_INPUTS:
-        _SAMPLE_INPUTS[seed] = (synthetic.route_topk_softmax(seed, T, E, k),
-                                synthetic.gaussian_bf16(seed, synthetic.STREAMS["x"], (T, H)))
-    r, x = _SAMPLE_INPUTS[seed]
-    done_flops, experts, rows = 0.0, 0, 0
-    t_work = 0.0
+    key = (seed, E, T, H)
+    if key not in _SAMPLE_INPUTS:
+        _SAMPLE_INPUTS[key] = (synthetic.route_topk_softmax(seed, T, E, k),
+                               synthetic.gaussian_bf16(seed, synthetic.STREAMS["x"], (T, H)))
+    r, x = _SAMPLE_INPUTS[key]
+    done_flops, experts, rows, t_work = 0.0, 0, 0, 0.0
     for e in range(E):
         r0, r1 = int(r["offsets"][e]), int(r["offsets"][e + 1])
         m = r1 - r0
@@ -298,30 +514,28 @@ def cpu_threads():
         return os.cpu_count() or 1
 
 
-def run_reference(args, rank, world):
-    """The oracle as the reference arm (host cores), each step a bounded sample."""
+def run_reference(args, world):
+    """The oracle as the reference arm (host cores); each step a bounded sample."""
     import oracle
     oracle.build()
-    secs = []
-    vals = []
-    for _ in range(max(1, args.warmup if args.warmup < 2 else 1)):
-        oracle_sample(0.5)
+    oracle_sample(0.5, E=args.experts, T=args.tokens)
+    vals, secs, ne, nr = [], [], 0, 0
     for _ in range(args.steps):
-        v, ne, nr, t = oracle_sample(2.0)
+        v, ne, nr, t = oracle_sample(2.0, E=args.experts, T=args.tokens)
         vals.append(v)
         secs.append(t)
     value = statistics.mean(vals)
-    out = {
+    workload = f"moe_routed_experts_e{args.experts}_top10_t{args.tokens}_h4096_i1024"
+    return {
         "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * statistics.mean(secs), 1),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)",
-        "data": "synthetic", "config": {"workload": WORKLOAD},
+        "data": "synthetic", "config": {"workload": workload},
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
                          "sample": f"whole experts of the same MoE layer until ~2 s of CPU work per step "
                                    f"(last step: {ne} experts, {nr} routed rows)"},
         "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
-    return out
 
 
 def main():
@@ -330,6 +544,9 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--experts", type=int, default=512)
+    ap.add_argument("--tokens", type=int, default=8192)
+    ap.add_argument("--components", default="auto")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
 
@@ -339,7 +556,7 @@ def main():
 
     if args.impl == "reference":
         if rank == 0:
-            print(json.dumps(run_reference(args, rank, world)), flush=True)
+            print(json.dumps(run_reference(args, world)), flush=True)
         return
 
     import torch
@@ -348,21 +565,34 @@ def main():
     if world > 1:
         import datetime
         import torch.distributed as dist
-        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
     from nvfp4_w4a4_quantized_04_b200 import build as nvbuild
     nvbuild.build()
     import synthetic.cuda as sc
     sc.build()
 
-    out = run_ours(args, rank, world, device)
+    out = run_headline(args, rank, world, device)
+    torch.cuda.empty_cache()
+
+    comps = args.components
+    if comps == "auto":
+        comps = "all" if world == 1 else "none"
+    names = list(COMPONENTS) if comps == "all" else ([] if comps == "none" else comps.split(","))
+    if names:
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+        out["components"] = {}
+        for n in names:
+            out["components"][n] = COMPONENTS[n](device, 7, 3, flush)
+            torch.cuda.empty_cache()
+
     if rank == 0 and not args.no_cpu_baseline:
         import oracle
         oracle.build()
-        v, ne, nr, t = oracle_sample(12.0)
+        v, ne, nr, t = oracle_sample(12.0, E=args.experts, T=args.tokens)
         out["cpu_baseline"] = {"value": round(v, 6), "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
                                "sample": f"{ne} whole experts ({nr} routed rows) of the same layer, "
-                                         f"{t:.1f} s of CPU work"}
+                                         f"{t:.1f} s of CPU work (gather-quantize, fp64 gate_up, SwiGLU, "
+                                         f"requantize, fp64 down)"}
     if world > 1:
         import torch.distributed as dist
         dist.barrier()

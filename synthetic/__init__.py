@@ -83,6 +83,16 @@ def normal_z(seed: int, stream: int, start: int, count: int) -> np.ndarray:
     return (s - 393210).astype(np.float64) / 65536.0
 
 
+def _normal_z_at(seed: int, stream: int, idx: np.ndarray) -> np.ndarray:
+    """``normal_z`` at arbitrary element indices."""
+    key = stream_key(seed, stream)
+    w_idx = (3 * idx.astype(np.uint64)[:, None] + np.arange(3, dtype=np.uint64)[None, :] + np.uint64(1))
+    with np.errstate(over="ignore"):
+        w = _mix(key + w_idx * G)
+    s = np.ascontiguousarray(w).view(np.uint16).reshape(len(idx), 12).sum(axis=1, dtype=np.int64)
+    return (s - 393210).astype(np.float64) / 65536.0
+
+
 def uniform(seed: int, stream: int, start: int, count: int) -> np.ndarray:
     w = words(seed, stream, start, count)
     return ((w >> np.uint64(11)).astype(np.float64) + 0.5) * (2.0 ** -53)
@@ -109,7 +119,9 @@ def outlier_positions(seed: int, numel: int, frac: float = 0.001) -> np.ndarray:
     if n_out == 0:
         return np.zeros(0, dtype=np.int64)
     w = words(seed, STREAMS["outlier_pos"], 0, numel)
-    order = np.argsort(w, kind="stable")
+    thr = np.partition(w, n_out - 1)[n_out - 1]        # the n_out-th smallest word
+    cand = np.nonzero(w <= thr)[0]                      # ascending index
+    order = cand[np.argsort(w[cand], kind="stable")]    # by word, then lower index
     return np.sort(order[:n_out]).astype(np.int64)
 
 
@@ -157,8 +169,16 @@ def gaussian_bf16(seed: int, stream: int, shape, sigma: float = 1.0,
     """
     shape = tuple(int(s) for s in shape)
     n = int(np.prod(shape)) if shape else 1
-    if outlier_frac == 0.0 and not reference and n >= (1 << 16):
-        return gaussian_bf16_bits_fast(seed, stream, start, n, sigma).reshape(shape)
+    if not reference and n >= (1 << 16):
+        bits = gaussian_bf16_bits_fast(seed, stream, start, n, sigma)
+        if outlier_frac > 0.0:
+            assert start == 0
+            pos = outlier_positions(seed, n, outlier_frac)
+            zp = np.concatenate([normal_z(seed, stream, int(p), 1) for p in pos]) if len(pos) < 64 else \
+                _normal_z_at(seed, stream, pos)
+            fp = (zp * float(sigma)).astype(np.float32) if sigma != 1.0 else zp.astype(np.float32)
+            bits[pos] = f32_to_bf16_bits((fp * np.float32(outlier_mult)).astype(np.float32))
+        return bits.reshape(shape)
     z = normal_z(seed, stream, start, n)
     f = (z * float(sigma)).astype(np.float32) if sigma != 1.0 else z.astype(np.float32)
     if outlier_frac > 0.0:

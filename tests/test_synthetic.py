@@ -13,6 +13,15 @@ def test_fast_host_generator_matches_numpy_definition():
             assert np.array_equal(a, b)
 
 
+def test_fast_path_with_outliers_matches_numpy_definition():
+    a = synthetic.gaussian_bf16(0, 1, (512, 512), outlier_frac=0.001)
+    b = synthetic.gaussian_bf16(0, 1, (512, 512), outlier_frac=0.001, reference=True)
+    assert np.array_equal(a, b)
+    a = synthetic.gaussian_bf16(2, 4, (256, 1024), sigma=0.02, outlier_frac=0.001)
+    b = synthetic.gaussian_bf16(2, 4, (256, 1024), sigma=0.02, outlier_frac=0.001, reference=True)
+    assert np.array_equal(a, b)
+
+
 def test_normal_moments_and_slices():
     z = synthetic.normal_z(0, 1, 0, 1 << 20)
     assert abs(z.mean()) < 5e-3 and abs(z.var() - 1.0) < 5e-3
