@@ -11,17 +11,24 @@
 //  * tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X: E2M1
 //    operands straight from shared memory, E4M3 scales per 16 elements from
 //    tensor memory, FP32 accumulator in tensor memory.
-//  * Swap-AB: the MMA's M side (128) walks weight rows, the N side (16..256,
+//  * Swap-AB: the MMA's M side (128) walks weight rows, the N side (16..192,
 //    step 16) walks the tokens of one expert, so a group of m tokens costs
-//    roundup(m,16) MMA columns instead of a 128-row tile.
+//    roundup(m,16) MMA columns instead of a 128-row tile.  Experts with more
+//    than 192 tokens are cut into equal chunks on 64-row boundaries.
 //  * Operands are staged by TMA (128-byte swizzle, K-major, 256 elements of K
-//    per stage); the per-16 scales arrive by bulk copy in the tensor-core atom
-//    layout (512-byte atoms of 128 rows x 4 scales) and are moved to tensor
-//    memory with tcgen05.cp (32x128b, replicated to the four lane quadrants).
-//  * Persistent grid (one CTA per SM), warp-specialised: warp 0 issues TMA,
-//    warp 1 issues MMAs, warps 2..5 drain the accumulator (tcgen05.ld) and
-//    store Y.  A 4-stage mbarrier ring links TMA and MMA; two barriers hand
-//    the accumulator between MMA and epilogue.
+//    per stage): the weight tile by one 128-row box, the token tile by at most
+//    two boxes (128/64/32 rows); the per-16 scales arrive by bulk copy in the
+//    tensor-core atom layout (512-byte atoms of 128 rows x 4 scales).
+//  * Scale factors reach tensor memory through four helper warps (ld.shared +
+//    tcgen05.st, one lane quadrant each, double-buffered), not tcgen05.cp
+//    from the MMA thread: on B200 each scale copy costs the MMA issuer about
+//    as much as an MMA, and the MoE tiles need 8-12 of them per K stage.
+//  * Persistent grid (one CTA per SM), warp-specialised: warp 0 loads weights
+//    and scales, warp 10 loads tokens, warp 1 issues MMAs, warps 6..9 write
+//    scales to tensor memory, warps 2..5 drain the accumulator (tcgen05.ld)
+//    and store Y.  A 4-stage mbarrier ring links loads and MMA; the two
+//    accumulators (2 x 192 columns) are double-buffered so the epilogue of one
+//    tile overlaps the main loop of the next.
 //  * Every mbarrier wait is bounded: past the budget the kernel records
 //    NVFP4_ERR_TIMEOUT, every role leaves its loop, outstanding copies and
 //    MMAs are drained (again bounded) and tensor memory is freed.
@@ -38,30 +45,40 @@ namespace nvfp4 {
 namespace gemm {
 
 constexpr int BM = 128;                 // weight rows per tile (MMA M)
-constexpr int BN = 256;                 // max tokens per tile (MMA N)
+constexpr int BN = 192;                 // max tokens per tile (MMA N)
 constexpr int BK = 256;                 // K elements per stage = 128 bytes of codes
 constexpr int STAGES = 4;
 constexpr int W_STAGE = BM * 128;       // 16 KB
-constexpr int X_STAGE = BN * 128;       // 32 KB
+constexpr int X_STAGE = BN * 128;       // 24 KB
 constexpr int SFW_STAGE = 2048;         // 128 rows x 16 scales (4 atoms)
-constexpr int SFX_STAGE = 4096;         // 256 rows x 16 scales (2 x 4 atoms)
+constexpr int SFX_STAGE = 4096;         // up to 2 row blocks x 4 atoms
 constexpr int OFF_W = 0;
 constexpr int OFF_X = OFF_W + STAGES * W_STAGE;
 constexpr int OFF_SFW = OFF_X + STAGES * X_STAGE;
 constexpr int OFF_SFX = OFF_SFW + STAGES * SFW_STAGE;
 constexpr int OFF_BAR = OFF_SFX + STAGES * SFX_STAGE;        // 8-byte mbarriers
-constexpr int NUM_BARS = 2 * STAGES + 3;                      // full, empty, acc_full, acc_empty, drain
+// full[S], empty[S], sf_full[2], acc_full[2], acc_empty[2], drain
+constexpr int NUM_BARS = 2 * STAGES + 2 + 2 + 2 + 1;
 constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;              // tmem base, abort flag
 constexpr int OFF_GROUPS = OFF_MISC + 16;                     // off / slot / tile arrays
-constexpr int kMaxExperts = 768;
-constexpr int SMEM_BYTES = OFF_GROUPS + 3 * (kMaxExperts + 1) * 4 + 64 + 1024;  // +1024 for alignment
-constexpr int NUM_THREADS = 192;
+constexpr int kMaxExperts = 1024;
+constexpr int NUM_WARPS = 11;
+constexpr int NUM_THREADS = NUM_WARPS * 32;
+constexpr int SMEM_BYTES = OFF_GROUPS + 3 * (kMaxExperts + 1) * 4 + 2 * NUM_WARPS * 4 + 1024;  // + scan scratch, +1024 for alignment
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t TMEM_SFW = 256;      // column of the weight scales (4 kk x 4 columns)
-constexpr uint32_t TMEM_SFX = 288;      // column of the token scales (4 kk x 8 columns)
+constexpr uint32_t TMEM_ACC_STRIDE = BN;       // accumulator b at column b*192
+constexpr uint32_t TMEM_SF = 2 * BN;           // scale buffers at 384 and 448
+constexpr uint32_t TMEM_SF_STRIDE = 64;        // per buffer: W scales 16 cols, token scales 32 cols
 constexpr long long kWaitBudgetCycles = 4000000000LL;   // ~2 s at 2 GHz
 
+// warp roles (warps 2..5: epilogue, lane quadrants 2,3,0,1)
+constexpr int W_PRODUCER = 0;     // weights + scales
+constexpr int W_MMA = 1;
+constexpr int W_SF0 = 6;          // 6..9: scale factors smem -> tensor memory (quadrants 2,3,0,1)
+constexpr int W_XLOAD = 10;       // token tiles
+
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+static_assert(TMEM_SF + 2 * TMEM_SF_STRIDE <= TMEM_COLS, "tensor memory budget");
 
 // ------------------------------------------------------------------ PTX wrappers
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
@@ -152,16 +169,6 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t addr) {
          ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
 
-// Scale atom for tcgen05.cp: 32 rows x 16 bytes, no swizzle, 8-row core
-// matrices 128 bytes apart.
-__device__ __forceinline__ uint64_t desc_sf(uint32_t addr) {
-  return (uint64_t)((addr & 0x3FFFFu) >> 4) | ((uint64_t)(128 >> 4) << 32) | ((uint64_t)1 << 46);
-}
-
-__device__ __forceinline__ void tc_cp_sf(uint32_t taddr, uint64_t desc) {
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" :: "r"(taddr), "l"(desc) : "memory");
-}
-
 __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                        uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
   asm volatile(
@@ -176,7 +183,7 @@ __device__ __forceinline__ void tc_commit(uint32_t bar) {
                :: "r"(bar) : "memory");
 }
 
-__device__ __forceinline__ void tc_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+__device__ __forceinline__ void tc_ld32_nowait(uint32_t taddr, uint32_t *r) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
       "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
@@ -185,7 +192,6 @@ __device__ __forceinline__ void tc_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
         "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
 // Instruction descriptor, kind::mxf4nvf4: E2M1 x E2M1, K-major both,
@@ -194,38 +200,61 @@ __device__ __forceinline__ uint32_t idesc_mxf4nvf4(uint32_t n) {
   return (1u << 7) | (1u << 10) | ((n >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
 }
 
+__device__ __forceinline__ void tc_st_x4(uint32_t taddr, uint4 v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};"
+               :: "r"(taddr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
+}
+
+__device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
 // ------------------------------------------------------------------ tile map
+// Tiles are (expert, 128-row weight block, token chunk), weight-block-major
+// inside an expert so that the chunks of one weight block run on adjacent
+// CTAs.  An expert with m tokens is cut into ceil(m/192) chunks of equal size
+// rounded up to 64, so every chunk starts on a 64-row boundary of the expert's
+// 128-aligned slot: its scale atoms start at row (start & ~127) and the MMA
+// reads them from tensor-memory column offset (start & 127)/32 (0 or 2).
 struct Tile {
   int e;          // expert
   int w_row0;     // first weight row (over E*N rows)
   int n_col0;     // first output column
   int x_row0;     // first activation row (slot space)
   int y_row0;     // first output row
-  int n_valid;    // tokens in this tile (1..256)
+  int n_valid;    // tokens in this tile (1..192)
 };
 
+__device__ __forceinline__ int chunks_of(int m) { return (m + BN - 1) / BN; }
+
 __device__ __forceinline__ Tile decode_tile(int t, const int32_t *s_off, const int32_t *s_slot,
-                                            const int32_t *s_tile, int E, int n_mtiles, int N) {
+                                            const int32_t *s_tile, int E, int N) {
   Tile T;
   const int e = upper_group(s_tile, E, t);
   const int m_e = s_off[e + 1] - s_off[e];
-  const int nch = (m_e + BN - 1) / BN;
+  const int nch = chunks_of(m_e);
+  const int csz = ((m_e + nch - 1) / nch + 63) & ~63;
   const int local = t - s_tile[e];
   const int mt = local / nch, ch = local - mt * nch;
+  const int start = ch * csz;
   T.e = e;
   T.n_col0 = mt * BM;
   T.w_row0 = e * N + mt * BM;
-  T.x_row0 = s_slot[e] + ch * BN;
-  T.y_row0 = s_off[e] + ch * BN;
-  T.n_valid = min(BN, m_e - ch * BN);
-  (void)n_mtiles;
+  T.x_row0 = s_slot[e] + start;
+  T.y_row0 = s_off[e] + start;
+  T.n_valid = min(csz, m_e - start);
   return T;
 }
 
 // ------------------------------------------------------------------ kernel
 template <bool kBf16Out>
 __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(
-    const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
+    const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x128,
+    const __grid_constant__ CUtensorMap tmap_x64, const __grid_constant__ CUtensorMap tmap_x32,
     const uint8_t *__restrict__ w_sf, const uint8_t *__restrict__ x_sf,
     const float *__restrict__ w_gs, const float *__restrict__ x_gs,
     const int32_t *__restrict__ expert_offsets, int E, int M_total, int N, int K,
@@ -233,11 +262,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   const uint32_t sbase = smem_u32(smem);
-  const uint32_t bar_full = sbase + OFF_BAR;
-  const uint32_t bar_empty = bar_full + 8 * STAGES;
-  const uint32_t bar_acc_full = bar_empty + 8 * STAGES;
-  const uint32_t bar_acc_empty = bar_acc_full + 8;
-  const uint32_t bar_drain = bar_acc_empty + 8;
+  const uint32_t bar_full = sbase + OFF_BAR;              // [STAGES], count 2 (two producer threads)
+  const uint32_t bar_empty = bar_full + 8 * STAGES;       // [STAGES], count 1 (MMA commit)
+  const uint32_t bar_sf_full = bar_empty + 8 * STAGES;    // [2], count 128 (scale warps)
+  const uint32_t bar_acc_full = bar_sf_full + 16;         // [2], count 1 (MMA commit)
+  const uint32_t bar_acc_empty = bar_acc_full + 16;       // [2], count 128 (epilogue threads)
+  const uint32_t bar_drain = bar_acc_empty + 16;
   volatile uint32_t *tmem_holder = reinterpret_cast<volatile uint32_t *>(smem + OFF_MISC);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
   int32_t *s_off = reinterpret_cast<int32_t *>(smem + OFF_GROUPS);
@@ -259,71 +289,106 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(
   if (threadIdx.x == 0) {
     *abort_flag = 0;
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_full + 8 * s, 2);
       mbar_init(bar_empty + 8 * s, 1);
     }
-    mbar_init(bar_acc_full, 1);
-    mbar_init(bar_acc_empty, 128);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar_sf_full + 8 * b, 128);
+      mbar_init(bar_acc_full + 8 * b, 1);
+      mbar_init(bar_acc_empty + 8 * b, 128);
+    }
     mbar_init(bar_drain, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 1) {
+  if (warp == W_MMA) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
                  :: "r"(smem_u32((const void *)tmem_holder)), "r"(TMEM_COLS) : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
   __syncthreads();
-  // slot starts (128-aligned groups) and tile starts, one thread (E <= 768)
-  if (threadIdx.x == 0) {
-    int32_t slot = 0, tiles = 0;
-    for (int e = 0; e < E; ++e) {
+  {
+    // slot starts (128-aligned groups) and tile starts: block-wide exclusive scans
+    const int per = (E + NUM_THREADS - 1) / NUM_THREADS;
+    const int e0 = min(E, (int)threadIdx.x * per), e1 = min(E, e0 + per);
+    int32_t ls = 0, lt = 0;
+    for (int e = e0; e < e1; ++e) {
       const int32_t m = s_off[e + 1] - s_off[e];
-      s_slot[e] = slot;
-      s_tile[e] = tiles;
-      slot += (m + kSlotAlign - 1) / kSlotAlign * kSlotAlign;
-      tiles += n_mtiles * ((m + BN - 1) / BN);
+      ls += (m + kSlotAlign - 1) / kSlotAlign * kSlotAlign;
+      lt += n_mtiles * chunks_of(m);
     }
-    s_slot[E] = slot;
-    s_tile[E] = tiles;
+    int32_t is = ls, it = lt;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int32_t a = __shfl_up_sync(0xffffffffu, is, d), b = __shfl_up_sync(0xffffffffu, it, d);
+      if (lane >= d) { is += a; it += b; }
+    }
+    if (lane == 31) { s_scratch[warp] = is; s_scratch[NUM_WARPS + warp] = it; }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      int32_t as = 0, at = 0;
+      for (int w = 0; w < NUM_WARPS; ++w) {
+        const int32_t vs = s_scratch[w], vt = s_scratch[NUM_WARPS + w];
+        s_scratch[w] = as; s_scratch[NUM_WARPS + w] = at;
+        as += vs; at += vt;
+      }
+    }
+    __syncthreads();
+    int32_t rs = s_scratch[warp] + is - ls, rt = s_scratch[NUM_WARPS + warp] + it - lt;
+    for (int e = e0; e < e1; ++e) {
+      const int32_t m = s_off[e + 1] - s_off[e];
+      s_slot[e] = rs;
+      s_tile[e] = rt;
+      rs += (m + kSlotAlign - 1) / kSlotAlign * kSlotAlign;
+      rt += n_mtiles * chunks_of(m);
+    }
+    if (e1 == E && e0 < e1) { s_slot[E] = rs; s_tile[E] = rt; }
   }
-  (void)s_scratch;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
   const int total_tiles = s_tile[E];
+  const int64_t sf_row_stride = (int64_t)(K / 64) * 512;   // bytes per 128-row block of scales
 
-  if (warp == 0) {
-    // ================================================================ TMA producer
+  if (warp == W_PRODUCER || warp == W_XLOAD) {
+    // ================================================================ TMA producers
+    // warp 0 lane 0: weight tile, weight scales, token scales; warp 10 lane 0:
+    // token tile.  Each arms the stage's full barrier with its own bytes.
     if (lane == 0) {
-      const uint64_t pol_w = policy_evict_first();
-      const uint64_t pol_x = policy_evict_last();
-      const int64_t sf_row_stride = (int64_t)(K / 64) * 512;   // bytes per 128-row block of scales
+      const bool is_w = warp == W_PRODUCER;
+      const uint64_t pol = is_w ? policy_evict_first() : policy_evict_last();
       int stage = 0;
       uint32_t phase = 0;
       bool armed[STAGES] = {};
       uint32_t armed_parity[STAGES] = {};
       bool ok = true;
       for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
-        const Tile T = decode_tile(t, s_off, s_slot, s_tile, E, n_mtiles, N);
+        const Tile T = decode_tile(t, s_off, s_slot, s_tile, E, N);
         const int rows_ld = (T.n_valid + 31) & ~31;
-        const int nrb = (T.n_valid + 127) >> 7;
-        const uint32_t bytes = W_STAGE + rows_ld * 128 + SFW_STAGE + nrb * 2048;
+        const int xr0 = T.x_row0 & ~127;                               // first scale row block
+        const int nrb = ((T.x_row0 & 127) + T.n_valid + 127) >> 7;     // 1 or 2
+        const uint32_t bytes = is_w ? (uint32_t)(W_STAGE + SFW_STAGE + nrb * 2048) : (uint32_t)(rows_ld * 128);
         const uint8_t *sfw_tile = w_sf + (int64_t)(T.w_row0 >> 7) * sf_row_stride;
-        const uint8_t *sfx_tile = x_sf + (int64_t)(T.x_row0 >> 7) * sf_row_stride;
+        const uint8_t *sfx_tile = x_sf + (int64_t)(xr0 >> 7) * sf_row_stride;
         for (int ks = 0; ks < ksteps; ++ks) {
           if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1, abort_flag, dev_status)) { ok = false; break; }
           const uint32_t fb = bar_full + 8 * stage;
           mbar_arrive_expect_tx(fb, bytes);
           armed[stage] = true;
           armed_parity[stage] = phase;
-          tma_load_2d(sbase + OFF_W + stage * W_STAGE, &tmap_w, ks * 128, T.w_row0, fb, pol_w);
-          for (int i = 0; i < rows_ld / 32; ++i)
-            tma_load_2d(sbase + OFF_X + stage * X_STAGE + i * 4096, &tmap_x, ks * 128, T.x_row0 + 32 * i, fb, pol_x);
-          bulk_load(sbase + OFF_SFW + stage * SFW_STAGE, sfw_tile + ks * 2048, 2048, fb);
-          for (int rb = 0; rb < nrb; ++rb)
-            bulk_load(sbase + OFF_SFX + stage * SFX_STAGE + rb * 2048, sfx_tile + rb * sf_row_stride + ks * 2048,
-                      2048, fb);
+          if (is_w) {
+            tma_load_2d(sbase + OFF_W + stage * W_STAGE, &tmap_w, ks * 128, T.w_row0, fb, pol);
+            bulk_load(sbase + OFF_SFW + stage * SFW_STAGE, sfw_tile + ks * 2048, 2048, fb);
+            for (int rb = 0; rb < nrb; ++rb)
+              bulk_load(sbase + OFF_SFX + stage * SFX_STAGE + rb * 2048, sfx_tile + rb * sf_row_stride + ks * 2048,
+                        2048, fb);
+          } else {
+            uint32_t dst = sbase + OFF_X + stage * X_STAGE;
+            int row = T.x_row0, left = rows_ld;
+            if (left >= 128) { tma_load_2d(dst, &tmap_x128, ks * 128, row, fb, pol); dst += 16384; row += 128; left -= 128; }
+            if (left >= 64) { tma_load_2d(dst, &tmap_x64, ks * 128, row, fb, pol); dst += 8192; row += 64; left -= 64; }
+            if (left >= 32) { tma_load_2d(dst, &tmap_x32, ks * 128, row, fb, pol); }
+          }
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
       }
@@ -334,38 +399,76 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(
         while (!mbar_try_wait(bar_full + 8 * s, armed_parity[s]) && clock64() - t0 < kWaitBudgetCycles) {}
       }
     }
-  } else if (warp == 1) {
-    // ================================================================ MMA issuer
+  } else if (warp >= W_SF0 && warp < W_SF0 + 4) {
+    // ================================================================ scale factors -> TMEM
+    // Each warp writes its lane quadrant: lane l of every quadrant gets the 16
+    // bytes of atom row l (the scales of rows l, l+32, l+64, l+96), i.e. the
+    // replicated 32x128b layout the block-scaled MMA reads.
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     int stage = 0;
-    uint32_t phase = 0, acc_phase = 0;
+    uint32_t phase = 0;
+    uint32_t kiter = 0;                 // global k-step counter (selects the scale buffer)
     bool ok = true;
-    const uint32_t t_acc = tmem_base;
-    const uint32_t t_sfw = tmem_base + TMEM_SFW;
-    const uint32_t t_sfx = tmem_base + TMEM_SFX;
     for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
-      const Tile T = decode_tile(t, s_off, s_slot, s_tile, E, n_mtiles, N);
-      const uint32_t n_mma = (T.n_valid + 15) & ~15;
-      const int nrb = (T.n_valid + 127) >> 7;
-      const uint32_t idesc = idesc_mxf4nvf4(n_mma);
-      if (!mbar_wait_warp(bar_acc_empty, acc_phase ^ 1, abort_flag, dev_status)) { ok = false; break; }
-      tc_fence_after();
-      for (int ks = 0; ks < ksteps; ++ks) {
+      const Tile T = decode_tile(t, s_off, s_slot, s_tile, E, N);
+      const int nrb = ((T.x_row0 & 127) + T.n_valid + 127) >> 7;
+      for (int ks = 0; ks < ksteps; ++ks, ++kiter) {
+        const uint32_t sb = kiter & 1;
+        // buffer sb was last read by the MMAs of k-step kiter-2: wait for them
+        if (kiter >= 2) {
+          const uint32_t prev = kiter - 2;
+          if (!mbar_wait_warp(bar_empty + 8 * (prev % STAGES), (prev / STAGES) & 1, abort_flag, dev_status)) {
+            ok = false; break;
+          }
+        }
         if (!mbar_wait_warp(bar_full + 8 * stage, phase, abort_flag, dev_status)) { ok = false; break; }
         tc_fence_after();
+        const uint32_t tcol = tmem_base + lane_base + TMEM_SF + sb * TMEM_SF_STRIDE;
+        const uint32_t sfw_addr = sbase + OFF_SFW + stage * SFW_STAGE + lane * 16;
+        const uint32_t sfx_addr = sbase + OFF_SFX + stage * SFX_STAGE + lane * 16;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) tc_st_x4(tcol + kk * 4, lds128(sfw_addr + kk * 512));
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) tc_st_x4(tcol + 16 + kk * 8, lds128(sfx_addr + kk * 512));
+        if (nrb > 1) {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) tc_st_x4(tcol + 16 + kk * 8 + 4, lds128(sfx_addr + 2048 + kk * 512));
+        }
+        tc_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar_sf_full + 8 * sb);
+        if (++stage == STAGES) { stage = 0; phase ^= 1; }
+      }
+    }
+  } else if (warp == W_MMA) {
+    // ================================================================ MMA issuer
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t kiter = 0, titer = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++titer) {
+      const Tile T = decode_tile(t, s_off, s_slot, s_tile, E, N);
+      const uint32_t n_mma = (T.n_valid + 15) & ~15;
+      const uint32_t idesc = idesc_mxf4nvf4(n_mma);
+      const uint32_t xoff = (uint32_t)(T.x_row0 & 127) >> 5;      // 0 or 2 columns
+      const uint32_t ab = titer & 1;
+      const uint32_t t_acc = tmem_base + ab * TMEM_ACC_STRIDE;
+      if (!mbar_wait_warp(bar_acc_empty + 8 * ab, ((titer >> 1) & 1) ^ 1, abort_flag, dev_status)) { ok = false; break; }
+      tc_fence_after();
+      for (int ks = 0; ks < ksteps; ++ks, ++kiter) {
+        const uint32_t sb = kiter & 1;
+        if (!mbar_wait_warp(bar_full + 8 * stage, phase, abort_flag, dev_status)) { ok = false; break; }
+        if (!mbar_wait_warp(bar_sf_full + 8 * sb, (kiter >> 1) & 1, abort_flag, dev_status)) { ok = false; break; }
+        tc_fence_after();
         if (lane == 0) {
-          const uint32_t w_addr = sbase + OFF_W + stage * W_STAGE;
-          const uint32_t x_addr = sbase + OFF_X + stage * X_STAGE;
-          const uint32_t sfw_addr = sbase + OFF_SFW + stage * SFW_STAGE;
-          const uint32_t sfx_addr = sbase + OFF_SFX + stage * SFX_STAGE;
+          const uint32_t t_sf = tmem_base + TMEM_SF + sb * TMEM_SF_STRIDE;
+          const uint64_t dw = desc_sw128(sbase + OFF_W + stage * W_STAGE);
+          const uint64_t dx = desc_sw128(sbase + OFF_X + stage * X_STAGE);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            tc_cp_sf(t_sfw + kk * 4, desc_sf(sfw_addr + kk * 512));
-            for (int rb = 0; rb < nrb; ++rb) tc_cp_sf(t_sfx + kk * 8 + rb * 4, desc_sf(sfx_addr + rb * 2048 + kk * 512));
-          }
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            tc_mma(t_acc, desc_sw128(w_addr + kk * 32), desc_sw128(x_addr + kk * 32), idesc, t_sfw + kk * 4,
-                   t_sfx + kk * 8, (ks > 0 || kk > 0) ? 1u : 0u);
+            // +32 bytes of K per MMA: +2 in the descriptor's 16-byte address field
+            tc_mma(t_acc, dw + 2 * kk, dx + 2 * kk, idesc, t_sf + kk * 4, t_sf + 16 + kk * 8 + xoff,
+                   (ks > 0 || kk > 0) ? 1u : 0u);
           }
           tc_commit(bar_empty + 8 * stage);
         }
@@ -373,11 +476,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(
         if (++stage == STAGES) { stage = 0; phase ^= 1; }
       }
       if (!ok) break;
-      if (lane == 0) tc_commit(bar_acc_full);
+      if (lane == 0) tc_commit(bar_acc_full + 8 * ab);
       __syncwarp();
-      acc_phase ^= 1;
     }
-    // Drain: all MMAs / copies this thread issued complete before TMEM is freed.
+    // Drain: all MMAs this thread issued complete before TMEM is freed.
     if (lane == 0) {
       tc_commit(bar_drain);
       const long long t0 = clock64();
@@ -388,39 +490,45 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(
     // ================================================================ epilogue
     const int quad = warp & 3;                    // TMEM lane quadrant of this warp
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
-    uint32_t acc_phase = 0;
-    for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
-      const Tile T = decode_tile(t, s_off, s_slot, s_tile, E, n_mtiles, N);
-      if (!mbar_wait_warp(bar_acc_full, acc_phase, abort_flag, dev_status)) break;
+    uint32_t titer = 0;
+    for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++titer) {
+      const Tile T = decode_tile(t, s_off, s_slot, s_tile, E, N);
+      const uint32_t ab = titer & 1;
+      if (!mbar_wait_warp(bar_acc_full + 8 * ab, (titer >> 1) & 1, abort_flag, dev_status)) break;
       tc_fence_after();
       const float alpha = __fmul_rn(x_gs[T.e], w_gs[T.e]);
       const int n_col = T.n_col0 + quad * 32 + lane;
-      for (int c0 = 0; c0 < T.n_valid; c0 += 32) {
-        uint32_t r[32];
-        tc_ld32(tmem_base + lane_base + (uint32_t)c0, r);
-        const int lim = min(32, T.n_valid - c0);
+      const uint32_t tacc = tmem_base + lane_base + ab * TMEM_ACC_STRIDE;
+      for (int c0 = 0; c0 < T.n_valid; c0 += 64) {
+        uint32_t r[64];
+        tc_ld32_nowait(tacc + (uint32_t)c0, r);
+        if (c0 + 32 < T.n_valid) tc_ld32_nowait(tacc + (uint32_t)c0 + 32, r + 32);
+        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+        if (c0 + 64 >= T.n_valid) {
+          // the whole accumulator has been read: hand it back to the MMA warp
+          tc_fence_before();
+          mbar_arrive(bar_acc_empty + 8 * ab);
+        }
+        const int lim = min(64, T.n_valid - c0);
         if (kBf16Out) {
           __nv_bfloat16 *yp = reinterpret_cast<__nv_bfloat16 *>(y) + (int64_t)(T.y_row0 + c0) * N + n_col;
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
+          for (int i = 0; i < 64; ++i)
             if (i < lim) yp[(int64_t)i * N] = __float2bfloat16_rn(__fmul_rn(__uint_as_float(r[i]), alpha));
         } else {
           float *yp = reinterpret_cast<float *>(y) + (int64_t)(T.y_row0 + c0) * N + n_col;
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
+          for (int i = 0; i < 64; ++i)
             if (i < lim) yp[(int64_t)i * N] = __fmul_rn(__uint_as_float(r[i]), alpha);
         }
       }
-      tc_fence_before();
-      mbar_arrive(bar_acc_empty);
-      acc_phase ^= 1;
     }
   }
 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) {
+  if (warp == W_MMA) {
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem_base), "r"(TMEM_COLS) : "memory");
   }
 }
@@ -484,9 +592,11 @@ extern "C" nvfp4_status nvfp4_grouped_gemm(const uint8_t *a_q, const uint8_t *a_
     return NVFP4_ERR_INVALID_ARG;
   if (!get_encoder()) return NVFP4_ERR_CUDA;
   const int64_t x_rows = nvfp4_padded_rows_bound(M_total, E);
-  CUtensorMap tw, tx;
+  CUtensorMap tw, tx128, tx64, tx32;
   if (!make_map(&tw, b_q, (uint64_t)E * N, (uint64_t)K / 2, 128)) return NVFP4_ERR_CUDA;
-  if (!make_map(&tx, a_q, (uint64_t)x_rows, (uint64_t)K / 2, 32)) return NVFP4_ERR_CUDA;
+  if (!make_map(&tx128, a_q, (uint64_t)x_rows, (uint64_t)K / 2, 128)) return NVFP4_ERR_CUDA;
+  if (!make_map(&tx64, a_q, (uint64_t)x_rows, (uint64_t)K / 2, 64)) return NVFP4_ERR_CUDA;
+  if (!make_map(&tx32, a_q, (uint64_t)x_rows, (uint64_t)K / 2, 32)) return NVFP4_ERR_CUDA;
   if (g_sms == 0) {
     int dev = 0;
     cudaGetDevice(&dev);
@@ -500,7 +610,8 @@ extern "C" nvfp4_status nvfp4_grouped_gemm(const uint8_t *a_q, const uint8_t *a_
       return NVFP4_ERR_CUDA;
     g_attr_set[bf] = true;
   }
-  kern<<<g_sms, gemm::NUM_THREADS, gemm::SMEM_BYTES, stream>>>(tw, tx, b_sf, a_sf, b_gs, a_gs, expert_offsets, E,
-                                                               (int)M_total, (int)N, (int)K, y, dev_status);
+  kern<<<g_sms, gemm::NUM_THREADS, gemm::SMEM_BYTES, stream>>>(tw, tx128, tx64, tx32, b_sf, a_sf, b_gs, a_gs,
+                                                               expert_offsets, E, (int)M_total, (int)N, (int)K, y,
+                                                               dev_status);
   return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }

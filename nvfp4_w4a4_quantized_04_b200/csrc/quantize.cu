@@ -138,11 +138,52 @@ __global__ void finalize_scales_kernel(const uint32_t *__restrict__ amax_bits, i
 
 // ---------------------------------------------------------------- pass 2: encode
 // One thread pair per 16-element block (8 elements = one 16-byte load per
-// thread); a warp covers 16 consecutive blocks.  The index space is the
+// thread); a warp covers 16 consecutive blocks per chunk and owns a
+// contiguous range of chunks, so its output-row -> expert-group lookup only
+// ever moves forward and is kept across iterations.  The index space is the
 // padded output rows, so slot padding is zero-filled by the same pass.
+struct EncodeItem {
+  uint4 v;
+  uint32_t p, j;
+  int g;
+  bool in_range, real;
+};
+
+template <bool kTiled>
+__device__ __forceinline__ void encode_finish(const EncodeItem &it, int half, uint32_t nblk, uint32_t K,
+                                              const float *__restrict__ gs, uint8_t *__restrict__ q,
+                                              uint8_t *__restrict__ sf, bool &bad) {
+  uint32_t m = halves_max(absmax8_bits(it.v, 0));
+  m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
+  if (it.real && m >= 0x7F80u) bad = true;
+  const float s_g = it.real ? gs[it.g] : 1.0f;
+  const float a_b = __uint_as_float(m << 16);
+  uint32_t S = 0;
+  if (it.real) S = f32_to_e4m3_satfinite(__fdiv_rn(a_b, __fmul_rn(6.0f, s_g)));
+  const float e = __fmul_rn(e4m3_to_f32(S), s_g);
+  const float r = (e == 0.0f) ? 0.0f : __frcp_rn(e);
+  float f[8];
+  const uint32_t w[4] = {it.v.x, it.v.y, it.v.z, it.v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float lo = __fmul_rn(bf16_bits_to_f32(w[i] & 0xFFFFu), r);
+    const float hi = __fmul_rn(bf16_bits_to_f32(w[i] >> 16), r);
+    f[2 * i] = isnan(lo) ? 0.0f : lo;
+    f[2 * i + 1] = isnan(hi) ? 0.0f : hi;
+  }
+  const uint32_t codes = f32x8_to_e2m1x8(f);
+  if (it.in_range) {
+    *reinterpret_cast<uint32_t *>(q + (uint64_t)it.p * (K >> 1) + it.j * 8 + half * 4) = codes;
+    if (half == 0) {
+      if (kTiled) sf[sf_tiled_offset(it.p, it.j, nblk)] = (uint8_t)S;
+      else sf[(uint64_t)it.p * nblk + it.j] = (uint8_t)S;
+    }
+  }
+}
+
 template <bool kTiled>
 __global__ void __launch_bounds__(256) quantize_kernel(
-    const uint16_t *__restrict__ x, int64_t ld_x, int64_t K, int64_t rows,
+    const uint16_t *__restrict__ x, int64_t ld_x, int64_t K64, int64_t rows,
     const int32_t *__restrict__ row_index, const int32_t *__restrict__ group_offsets, int G,
     int64_t P, const float *__restrict__ gs, uint8_t *__restrict__ q, uint8_t *__restrict__ sf,
     int32_t *dev_status) {
@@ -150,61 +191,64 @@ __global__ void __launch_bounds__(256) quantize_kernel(
   int32_t *off = smem, *slot = smem + (G + 1), *scratch = smem + 2 * (G + 1);
   if (group_offsets) load_groups(group_offsets, G, off, slot, scratch);
   const int lane = threadIdx.x & 31, half = lane & 1;
-  const int64_t nblk = K >> 4;
-  const int64_t total = P * nblk;
-  const int64_t nchunks = (total + 15) >> 4;
-  const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-  const int64_t p_end = group_offsets ? (int64_t)slot[G] : P;
+  const uint32_t K = (uint32_t)K64, nblk = K >> 4;
+  const uint32_t p_end = group_offsets ? (uint32_t)slot[G] : (uint32_t)P;
+  const uint64_t total = (uint64_t)p_end * nblk;             // blocks to write
+  const uint64_t nchunks = (total + 15) >> 4;
+  const uint64_t warp = ((uint64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const uint64_t nwarps = ((uint64_t)gridDim.x * blockDim.x) >> 5;
+  const uint64_t per = (nchunks + nwarps - 1) / nwarps;
+  const uint64_t c0 = warp * per, c1 = min(nchunks, c0 + per);
+  if (c0 >= c1) return;
+  int g = 0;
+  if (group_offsets) {
+    const uint64_t b0 = c0 * 16 + (lane >> 1);
+    g = upper_group(slot, G, (int64_t)(min(b0, total - 1) / nblk));
+  }
   bool bad = false;
-  for (int64_t c = warp; c < nchunks; c += nwarps) {
-    const int64_t blk = c * 16 + (lane >> 1);
-    const bool in_range = blk < total;
-    const int64_t p = in_range ? blk / nblk : 0;
-    const int64_t j = in_range ? blk - p * nblk : 0;
-    bool real = false;
+  const bool small = total < 0xFFFFFFF0ull;
+  auto prepare = [&](uint64_t c, EncodeItem &it) {
+    const uint64_t b = c * 16 + (lane >> 1);
+    it.in_range = b < total;
+    if (small) {                       // 32-bit index math when it fits
+      const uint32_t b32 = it.in_range ? (uint32_t)b : 0u;
+      it.p = b32 / nblk;
+      it.j = b32 - it.p * nblk;
+    } else {
+      it.p = it.in_range ? (uint32_t)(b / nblk) : 0u;
+      it.j = it.in_range ? (uint32_t)(b - (uint64_t)it.p * nblk) : 0u;
+    }
+    it.real = false;
+    it.g = 0;
     int64_t src = 0;
-    int g = 0;
-    if (in_range && p < p_end) {
+    if (it.in_range) {
       if (group_offsets) {
-        g = upper_group(slot, G, p);
-        const int64_t local = p - slot[g];
-        real = local < (int64_t)(off[g + 1] - off[g]);
-        if (real) src = off[g] + local;
+        while (g + 1 < G && (uint32_t)slot[g + 1] <= it.p) ++g;
+        it.g = g;
+        const uint32_t local = it.p - (uint32_t)slot[g];
+        it.real = local < (uint32_t)(off[g + 1] - off[g]);
+        src = (int64_t)off[g] + local;
       } else {
-        real = p < rows;
-        src = p;
+        it.real = it.p < (uint64_t)rows;
+        src = it.p;
       }
-      if (real && row_index) src = row_index[src];
+      if (it.real && row_index) src = row_index[src];
     }
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (real) v = ldg_nc_v4(x + src * ld_x + j * 16 + half * 8);
-    uint32_t m = halves_max(absmax8_bits(v, 0));
-    m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
-    if (real && m >= 0x7F80u) bad = true;
-    const float s_g = real ? gs[g] : 1.0f;
-    const float a_b = __uint_as_float(m << 16);
-    uint32_t S = 0;
-    if (real) S = f32_to_e4m3_satfinite(__fdiv_rn(a_b, __fmul_rn(6.0f, s_g)));
-    const float e = __fmul_rn(e4m3_to_f32(S), s_g);
-    const float r = (e == 0.0f) ? 0.0f : __frcp_rn(e);
-    float f[8];
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      float lo = __fmul_rn(bf16_bits_to_f32(w[i] & 0xFFFFu), r);
-      float hi = __fmul_rn(bf16_bits_to_f32(w[i] >> 16), r);
-      f[2 * i] = isnan(lo) ? 0.0f : lo;
-      f[2 * i + 1] = isnan(hi) ? 0.0f : hi;
-    }
-    const uint32_t codes = f32x8_to_e2m1x8(f);
-    if (in_range && p < p_end) {
-      *reinterpret_cast<uint32_t *>(q + p * (K >> 1) + j * 8 + half * 4) = codes;
-      if (half == 0) {
-        if (kTiled) sf[sf_tiled_offset(p, j, nblk)] = (uint8_t)S;
-        else sf[p * nblk + j] = (uint8_t)S;
-      }
-    }
+    it.v = make_uint4(0, 0, 0, 0);
+    if (it.real) it.v = ldg_nc_v4(x + src * ld_x + it.j * 16 + half * 8);
+  };
+  uint64_t c = c0;
+  for (; c + 1 < c1; c += 2) {
+    EncodeItem a, b;
+    prepare(c, a);
+    prepare(c + 1, b);
+    encode_finish<kTiled>(a, half, nblk, K, gs, q, sf, bad);
+    encode_finish<kTiled>(b, half, nblk, K, gs, q, sf, bad);
+  }
+  if (c < c1) {
+    EncodeItem a;
+    prepare(c, a);
+    encode_finish<kTiled>(a, half, nblk, K, gs, q, sf, bad);
   }
   if (bad) report(dev_status, NVFP4_ERR_NONFINITE);
 }

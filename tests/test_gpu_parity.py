@@ -374,6 +374,44 @@ def test_gemm_grouped_ragged():
     assert ok.all(), (err.max(), (err / bound).max(), np.argwhere(~ok)[:5])
 
 
+@pytest.mark.parametrize("out_dtype", [0, 1])
+def test_gemm_grouped_chunk_edges(out_dtype):
+    """Expert sizes around every tile and chunk boundary (64-row chunk starts,
+    one or two scale row blocks, the 192-token tile limit)."""
+    counts = [1, 63, 64, 65, 127, 128, 129, 191, 192, 193, 255, 256, 257, 383, 384, 385, 577, 0, 2]
+    E, N, K = len(counts), 128, 256
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    R = int(offsets[-1])
+    x = synthetic.gaussian_bf16(12, synthetic.STREAMS["x"], (R, K), outlier_frac=0.001)
+    w = synthetic.gaussian_bf16(12, synthetic.STREAMS["w"], (E * N, K), sigma=0.02)
+    q, sf, gs, qs, ss = _packed_acts(x, None, offsets, E)
+    qw, sw, gw = _packed_weights(w, E, N, K)
+    y = _run_gemm(qs, ss, gs, qw, sw, gw, offsets, E, R, N, K, 0)
+    a = oracle.dequantize_f64(q, sf, oracle.rows_global_scale(gs, offsets, R))
+    bw = oracle.dequantize_f64(qw, sw, np.repeat(gw, N))
+    y_ref, s_ref = oracle.grouped_gemm_f64(a, bw.reshape(E, N, K), offsets)
+    ok, err, bound = gemm_tol(y, y_ref, s_ref)
+    assert ok.all(), (err.max(), (err / bound).max(), np.argwhere(~ok)[:5])
+    if out_dtype == 1:
+        y16 = _run_gemm(qs, ss, gs, qw, sw, gw, offsets, E, R, N, K, 1)
+        assert np.array_equal(y16, synthetic.f32_to_bf16_bits(y))
+
+
+def test_gemm_dense_many_tiles():
+    """Dense M = 1000 rows (6 token chunks, ragged last), N = 384, K = 1024."""
+    M, N, K = 1000, 384, 1024
+    x = synthetic.gaussian_bf16(13, synthetic.STREAMS["x"], (M, K), outlier_frac=0.001)
+    w = synthetic.gaussian_bf16(13, synthetic.STREAMS["w"], (N, K), sigma=0.02)
+    qx, sx, gx, _ = oracle.quantize(x)
+    qw, sw, gw = _packed_weights(w, 1, N, K)
+    y = _run_gemm(qx, sx, gx, qw, sw, gw, None, 1, M, N, K, 0)
+    a = oracle.dequantize_f64(qx, sx, np.full(M, gx[0], np.float32))
+    b = oracle.dequantize_f64(qw, sw, np.full(N, gw[0], np.float32))
+    y_ref, s_ref = oracle.gemm_f64(a, b)
+    ok, err, bound = gemm_tol(y, y_ref, s_ref)
+    assert ok.all(), (err.max(), (err / bound).max())
+
+
 def test_gemm_long_k_tolerance():
     """K = 17408 (the dense MLP's down projection) on a thin slice."""
     M, N, K = 64, 128, 17408
