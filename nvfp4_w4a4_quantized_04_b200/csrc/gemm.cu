@@ -56,7 +56,9 @@ constexpr int OFF_W = 0;
 constexpr int OFF_X = OFF_W + STAGES * W_STAGE;
 constexpr int OFF_SFW = OFF_X + STAGES * X_STAGE;
 constexpr int OFF_SFX = OFF_SFW + STAGES * SFW_STAGE;
-constexpr int OFF_BAR = OFF_SFX + STAGES * SFX_STAGE;        // 8-byte mbarriers
+constexpr int EPI_WARP_BYTES = 32 * 32 * 4;                   // 32 tokens x 32 columns, fp32
+constexpr int OFF_EPI = OFF_SFX + STAGES * SFX_STAGE;        // epilogue staging, one slab per warp
+constexpr int OFF_BAR = OFF_EPI + 4 * EPI_WARP_BYTES;        // 8-byte mbarriers
 // full[S], empty[S], sf_full[2], acc_full[2], acc_empty[2], drain
 constexpr int NUM_BARS = 2 * STAGES + 2 + 2 + 2 + 1;
 constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;              // tmem base, abort flag
@@ -490,6 +492,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(
     // ================================================================ epilogue
     const int quad = warp & 3;                    // TMEM lane quadrant of this warp
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
+    const uint32_t epi = sbase + OFF_EPI + (warp - 2) * EPI_WARP_BYTES;
     uint32_t titer = 0;
     for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++titer) {
       const Tile T = decode_tile(t, s_off, s_slot, s_tile, E, N);
@@ -497,7 +500,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(
       if (!mbar_wait_warp(bar_acc_full + 8 * ab, (titer >> 1) & 1, abort_flag, dev_status)) break;
       tc_fence_after();
       const float alpha = __fmul_rn(x_gs[T.e], w_gs[T.e]);
-      const int n_col = T.n_col0 + quad * 32 + lane;
       const uint32_t tacc = tmem_base + lane_base + ab * TMEM_ACC_STRIDE;
       for (int c0 = 0; c0 < T.n_valid; c0 += 64) {
         uint32_t r[64];
@@ -509,17 +511,49 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(
           tc_fence_before();
           mbar_arrive(bar_acc_empty + 8 * ab);
         }
-        const int lim = min(64, T.n_valid - c0);
-        if (kBf16Out) {
-          __nv_bfloat16 *yp = reinterpret_cast<__nv_bfloat16 *>(y) + (int64_t)(T.y_row0 + c0) * N + n_col;
+        // Stage each 32-token x 32-column block in shared memory (this lane
+        // owns one weight column), then write whole 64/128-byte row segments
+        // of Y with 16-byte vector stores.
 #pragma unroll
-          for (int i = 0; i < 64; ++i)
-            if (i < lim) yp[(int64_t)i * N] = __float2bfloat16_rn(__fmul_rn(__uint_as_float(r[i]), alpha));
-        } else {
-          float *yp = reinterpret_cast<float *>(y) + (int64_t)(T.y_row0 + c0) * N + n_col;
+        for (int sub = 0; sub < 2; ++sub) {
+          const int tok0 = c0 + sub * 32;
+          if (tok0 >= T.n_valid) break;
+          const int rows_here = min(32, T.n_valid - tok0);
+          if (kBf16Out) {
 #pragma unroll
-          for (int i = 0; i < 64; ++i)
-            if (i < lim) yp[(int64_t)i * N] = __fmul_rn(__uint_as_float(r[i]), alpha);
+            for (int i = 0; i < 32; ++i) {
+              const __nv_bfloat16 hv = __float2bfloat16_rn(__fmul_rn(__uint_as_float(r[sub * 32 + i]), alpha));
+              asm volatile("st.shared.b16 [%0], %1;" :: "r"(epi + i * 64 + lane * 2),
+                           "h"(*reinterpret_cast<const uint16_t *>(&hv)) : "memory");
+            }
+            __syncwarp();
+            __nv_bfloat16 *ybase = reinterpret_cast<__nv_bfloat16 *>(y) + (int64_t)(T.y_row0 + tok0) * N + T.n_col0 + quad * 32;
+#pragma unroll
+            for (int it = 0; it < 4; ++it) {
+              const int row = it * 8 + (lane >> 2), chunk = lane & 3;
+              if (row < rows_here) {
+                const uint4 v = lds128(epi + row * 64 + chunk * 16);
+                *reinterpret_cast<uint4 *>(ybase + (int64_t)row * N + chunk * 8) = v;
+              }
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const float fv = __fmul_rn(__uint_as_float(r[sub * 32 + i]), alpha);
+              asm volatile("st.shared.b32 [%0], %1;" :: "r"(epi + i * 128 + lane * 4), "f"(fv) : "memory");
+            }
+            __syncwarp();
+            float *ybase = reinterpret_cast<float *>(y) + (int64_t)(T.y_row0 + tok0) * N + T.n_col0 + quad * 32;
+#pragma unroll
+            for (int it = 0; it < 8; ++it) {
+              const int row = it * 4 + (lane >> 3), chunk = lane & 7;
+              if (row < rows_here) {
+                const uint4 v = lds128(epi + row * 128 + chunk * 16);
+                *reinterpret_cast<uint4 *>(ybase + (int64_t)row * N + chunk * 4) = v;
+              }
+            }
+          }
+          __syncwarp();
         }
       }
     }

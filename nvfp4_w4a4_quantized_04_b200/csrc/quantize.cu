@@ -192,63 +192,62 @@ __global__ void __launch_bounds__(256) quantize_kernel(
   if (group_offsets) load_groups(group_offsets, G, off, slot, scratch);
   const int lane = threadIdx.x & 31, half = lane & 1;
   const uint32_t K = (uint32_t)K64, nblk = K >> 4;
+  const uint32_t nsl = (nblk + 15) >> 4;                     // 16-block slices per row
   const uint32_t p_end = group_offsets ? (uint32_t)slot[G] : (uint32_t)P;
-  const uint64_t total = (uint64_t)p_end * nblk;             // blocks to write
-  const uint64_t nchunks = (total + 15) >> 4;
+  const uint64_t units = (uint64_t)p_end * nsl;              // (row, slice) work units, row-major
+  constexpr int U = 4;                                       // consecutive units per warp step
+  const uint64_t nchunks = (units + U - 1) / U;
   const uint64_t warp = ((uint64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const uint64_t nwarps = ((uint64_t)gridDim.x * blockDim.x) >> 5;
-  const uint64_t per = (nchunks + nwarps - 1) / nwarps;
-  const uint64_t c0 = warp * per, c1 = min(nchunks, c0 + per);
-  if (c0 >= c1) return;
+  const bool small = units < 0xFFFFFFF0ull;
+  // Warps stride over 4-unit chunks (2 KB of input per warp step, all warps
+  // moving through memory together).  Rows only move forward per lane, so the
+  // row -> (group, source row) lookup walks forward from the last group.
   int g = 0;
-  if (group_offsets) {
-    const uint64_t b0 = c0 * 16 + (lane >> 1);
-    g = upper_group(slot, G, (int64_t)(min(b0, total - 1) / nblk));
-  }
+  uint32_t cached_p = 0xFFFFFFFFu;
+  int64_t cached_src = -1;
+  bool cached_real = false;
   bool bad = false;
-  const bool small = total < 0xFFFFFFF0ull;
-  auto prepare = [&](uint64_t c, EncodeItem &it) {
-    const uint64_t b = c * 16 + (lane >> 1);
-    it.in_range = b < total;
-    if (small) {                       // 32-bit index math when it fits
-      const uint32_t b32 = it.in_range ? (uint32_t)b : 0u;
-      it.p = b32 / nblk;
-      it.j = b32 - it.p * nblk;
-    } else {
-      it.p = it.in_range ? (uint32_t)(b / nblk) : 0u;
-      it.j = it.in_range ? (uint32_t)(b - (uint64_t)it.p * nblk) : 0u;
-    }
-    it.real = false;
-    it.g = 0;
-    int64_t src = 0;
-    if (it.in_range) {
-      if (group_offsets) {
-        while (g + 1 < G && (uint32_t)slot[g + 1] <= it.p) ++g;
-        it.g = g;
-        const uint32_t local = it.p - (uint32_t)slot[g];
-        it.real = local < (uint32_t)(off[g + 1] - off[g]);
-        src = (int64_t)off[g] + local;
-      } else {
-        it.real = it.p < (uint64_t)rows;
-        src = it.p;
+  for (uint64_t c = warp; c < nchunks; c += nwarps) {
+    EncodeItem it[U];
+    int64_t src[U];
+#pragma unroll
+    for (int k = 0; k < U; ++k) {
+      const uint64_t unit = c * U + k;
+      uint32_t p = 0, sl = 0;
+      if (unit < units) {
+        if (small) { p = (uint32_t)unit / nsl; sl = (uint32_t)unit - p * nsl; }
+        else { p = (uint32_t)(unit / nsl); sl = (uint32_t)(unit - (uint64_t)p * nsl); }
       }
-      if (it.real && row_index) src = row_index[src];
+      const uint32_t j = sl * 16 + (lane >> 1);
+      it[k].in_range = unit < units && j < nblk;
+      it[k].p = p;
+      it[k].j = j;
+      if (unit < units && p != cached_p) {
+        cached_p = p;
+        if (group_offsets) {
+          if (g + 8 < G && (uint32_t)slot[g + 8] <= p) g = upper_group(slot, G, p);
+          while (g + 1 < G && (uint32_t)slot[g + 1] <= p) ++g;
+          const uint32_t local = p - (uint32_t)slot[g];
+          cached_real = local < (uint32_t)(off[g + 1] - off[g]);
+          cached_src = (int64_t)off[g] + local;
+        } else {
+          cached_real = p < (uint64_t)rows;
+          cached_src = p;
+        }
+        if (cached_real && row_index) cached_src = row_index[cached_src];
+      }
+      it[k].g = g;
+      it[k].real = it[k].in_range && cached_real;
+      src[k] = cached_src;
     }
-    it.v = make_uint4(0, 0, 0, 0);
-    if (it.real) it.v = ldg_nc_v4(x + src * ld_x + it.j * 16 + half * 8);
-  };
-  uint64_t c = c0;
-  for (; c + 1 < c1; c += 2) {
-    EncodeItem a, b;
-    prepare(c, a);
-    prepare(c + 1, b);
-    encode_finish<kTiled>(a, half, nblk, K, gs, q, sf, bad);
-    encode_finish<kTiled>(b, half, nblk, K, gs, q, sf, bad);
-  }
-  if (c < c1) {
-    EncodeItem a;
-    prepare(c, a);
-    encode_finish<kTiled>(a, half, nblk, K, gs, q, sf, bad);
+#pragma unroll
+    for (int k = 0; k < U; ++k) {
+      it[k].v = make_uint4(0, 0, 0, 0);
+      if (it[k].real) it[k].v = ldg_nc_v4(x + src[k] * ld_x + it[k].j * 16 + half * 8);
+    }
+#pragma unroll
+    for (int k = 0; k < U; ++k) encode_finish<kTiled>(it[k], half, nblk, K, gs, q, sf, bad);
   }
   if (bad) report(dev_status, NVFP4_ERR_NONFINITE);
 }
@@ -261,41 +260,43 @@ __global__ void __launch_bounds__(256) dequantize_kernel(
   extern __shared__ int32_t smem[];
   int32_t *off = smem, *slot = smem + (G + 1), *scratch = smem + 2 * (G + 1);
   if (group_offsets) load_groups(group_offsets, G, off, slot, scratch);
-  const int64_t nblk = K >> 4;
-  const int64_t total = rows * nblk;
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < total; b += stride) {
-    const int64_t r = b / nblk, j = b - r * nblk;
+  // one thread per 8 elements (a thread pair per 16-element block), so a warp
+  // writes 512 (bf16) or 1024 (fp32) contiguous bytes per step
+  const uint64_t nhalf = (uint64_t)(K >> 3);
+  const uint64_t total = (uint64_t)rows * nhalf;
+  const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
+  const uint64_t nblk = (uint64_t)(K >> 4);
+  for (uint64_t h = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; h < total; h += stride) {
+    const uint64_t r = h / nhalf, c = h - r * nhalf;
+    const uint64_t j = c >> 1;
     int g = 0;
-    int64_t p = r;
+    uint64_t p = r;
     if (group_offsets) {
-      g = upper_group(off, G, r);
-      p = slot[g] + (r - off[g]);
+      g = upper_group(off, G, (int64_t)r);
+      p = (uint64_t)slot[g] + (r - (uint64_t)off[g]);
     }
     const float s_g = gs[g];
     const float Sv = e4m3_to_f32(kTiled ? sf[sf_tiled_offset(p, j, nblk)] : sf[p * nblk + j]);
-    const uint2 cw = *reinterpret_cast<const uint2 *>(q + p * (K >> 1) + j * 8);
-    float out[16];
+    const uint32_t cw = *reinterpret_cast<const uint32_t *>(q + p * (K >> 1) + c * 4);
+    float out[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const uint32_t byte = ((i < 4 ? cw.x : cw.y) >> (8 * (i & 3))) & 0xFFu;
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t byte = (cw >> (8 * i)) & 0xFFu;
       out[2 * i] = __fmul_rn(__fmul_rn(e2m1_to_f32(byte & 15u), Sv), s_g);
       out[2 * i + 1] = __fmul_rn(__fmul_rn(e2m1_to_f32(byte >> 4), Sv), s_g);
     }
     if (kBf16) {
-      uint32_t h[8];
+      uint32_t hw[4];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
+      for (int i = 0; i < 4; ++i) {
         __nv_bfloat162 t = __floats2bfloat162_rn(out[2 * i], out[2 * i + 1]);
-        h[i] = *reinterpret_cast<uint32_t *>(&t);
+        hw[i] = *reinterpret_cast<uint32_t *>(&t);
       }
-      uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(y) + r * K + j * 16);
-      dst[0] = make_uint4(h[0], h[1], h[2], h[3]);
-      dst[1] = make_uint4(h[4], h[5], h[6], h[7]);
+      *reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(y) + r * K + c * 8) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
     } else {
-      float4 *dst = reinterpret_cast<float4 *>(reinterpret_cast<float *>(y) + r * K + j * 16);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) dst[i] = make_float4(out[4 * i], out[4 * i + 1], out[4 * i + 2], out[4 * i + 3]);
+      float4 *dst = reinterpret_cast<float4 *>(reinterpret_cast<float *>(y) + r * K + c * 8);
+      dst[0] = make_float4(out[0], out[1], out[2], out[3]);
+      dst[1] = make_float4(out[4], out[5], out[6], out[7]);
     }
   }
 }
@@ -513,7 +514,7 @@ nvfp4_status nvfp4_dequantize(const uint8_t *q, const uint8_t *sf, nvfp4_sf_layo
   if (rows == 0) return NVFP4_OK;
   if (!q || !sf || !global_scale || !y || !aligned16(q) || !aligned16(y)) return NVFP4_ERR_INVALID_ARG;
   const bool tiled = sf_layout == NVFP4_SF_MMA_TILED, bf = out_dtype == NVFP4_OUT_BF16;
-  const int64_t work = rows * (K / 16);
+  const int64_t work = rows * (K / 8);
   const unsigned grid = (unsigned)grid_for(work, 256, 8);
   const size_t sm = group_offsets ? sizeof(int32_t) * (2 * (G + 1) + 8) : 0;
 #define NVFP4_DQ(T, B) dequantize_kernel<T, B><<<grid, 256, sm, stream>>>(q, sf, global_scale, group_offsets, G, rows, K, y)
