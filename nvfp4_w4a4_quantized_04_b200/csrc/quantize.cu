@@ -137,48 +137,50 @@ __global__ void finalize_scales_kernel(const uint32_t *__restrict__ amax_bits, i
 }
 
 // ---------------------------------------------------------------- pass 2: encode
-// One thread pair per 16-element block (8 elements = one 16-byte load per
-// thread); a warp covers 16 consecutive blocks per chunk and owns a
-// contiguous range of chunks, so its output-row -> expert-group lookup only
-// ever moves forward and is kept across iterations.  The index space is the
-// padded output rows, so slot padding is zero-filled by the same pass.
-struct EncodeItem {
-  uint4 v;
-  uint32_t p, j;
-  int g;
-  bool in_range, real;
-};
+// One thread per 16-element block: one 32-byte load (two 16-byte loads when
+// the row stride is not 32-byte aligned), the block amax in integer SIMD,
+// one IEEE division for the scale and one IEEE reciprocal per block, the
+// 16 products as eight packed f32x2 multiplies, eight e2m1x2 conversions and
+// one 8-byte store.  A warp covers 32 consecutive blocks per step; warps
+// stride over 64-block chunks so the whole grid streams through memory
+// together.  Rows only move forward per lane, so the row -> (group, source
+// row) lookup walks forward from the last group.
+__device__ __forceinline__ uint2 load_block(const uint16_t *p, bool v8, uint4 &a, uint4 &b) {
+  if (v8) {
+    asm volatile("ld.global.nc.L1::no_allocate.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w), "=r"(b.x), "=r"(b.y), "=r"(b.z), "=r"(b.w)
+                 : "l"(p));
+  } else {
+    a = ldg_nc_v4(p);
+    b = ldg_nc_v4(p + 8);
+  }
+  return make_uint2(0, 0);
+}
 
-template <bool kTiled>
-__device__ __forceinline__ void encode_finish(const EncodeItem &it, int half, uint32_t nblk, uint32_t K,
-                                              const float *__restrict__ gs, uint8_t *__restrict__ q,
-                                              uint8_t *__restrict__ sf, bool &bad) {
-  uint32_t m = halves_max(absmax8_bits(it.v, 0));
-  m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
-  if (it.real && m >= 0x7F80u) bad = true;
-  const float s_g = it.real ? gs[it.g] : 1.0f;
-  const float a_b = __uint_as_float(m << 16);
-  uint32_t S = 0;
-  if (it.real) S = f32_to_e4m3_satfinite(__fdiv_rn(a_b, __fmul_rn(6.0f, s_g)));
-  const float e = __fmul_rn(e4m3_to_f32(S), s_g);
-  const float r = (e == 0.0f) ? 0.0f : __frcp_rn(e);
-  float f[8];
-  const uint32_t w[4] = {it.v.x, it.v.y, it.v.z, it.v.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float lo = __fmul_rn(bf16_bits_to_f32(w[i] & 0xFFFFu), r);
-    const float hi = __fmul_rn(bf16_bits_to_f32(w[i] >> 16), r);
-    f[2 * i] = isnan(lo) ? 0.0f : lo;
-    f[2 * i + 1] = isnan(hi) ? 0.0f : hi;
-  }
-  const uint32_t codes = f32x8_to_e2m1x8(f);
-  if (it.in_range) {
-    *reinterpret_cast<uint32_t *>(q + (uint64_t)it.p * (K >> 1) + it.j * 8 + half * 4) = codes;
-    if (half == 0) {
-      if (kTiled) sf[sf_tiled_offset(it.p, it.j, nblk)] = (uint8_t)S;
-      else sf[(uint64_t)it.p * nblk + it.j] = (uint8_t)S;
-    }
-  }
+// bf16 pair (lo in bits 0..15) times r, both products rounded to nearest even.
+__device__ __forceinline__ uint64_t mul_pair(uint32_t w, uint64_t rr) {
+  const uint64_t x = ((uint64_t)(w & 0xFFFF0000u) << 32) | (uint64_t)(w << 16);
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(x), "l"(rr));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t e2m1x4_from_pairs(uint64_t p0, uint64_t p1) {
+  uint32_t out;
+  asm("{\n.reg .b8 b0, b1;\n.reg .f32 l0, h0, l1, h1;\n"
+      "mov.b64 {l0, h0}, %1;\nmov.b64 {l1, h1}, %2;\n"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, h0, l0;\n"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, h1, l1;\n"
+      "mov.b32 %0, {b0, b1, b0, b1};\n}"
+      : "=r"(out) : "l"(p0), "l"(p1));
+  return out & 0xFFFFu;
+}
+
+__device__ __forceinline__ uint64_t sanitize_pair(uint64_t d) {
+  float lo = __uint_as_float((uint32_t)d), hi = __uint_as_float((uint32_t)(d >> 32));
+  lo = isnan(lo) ? 0.0f : lo;
+  hi = isnan(hi) ? 0.0f : hi;
+  return ((uint64_t)__float_as_uint(hi) << 32) | __float_as_uint(lo);
 }
 
 template <bool kTiled>
@@ -190,69 +192,112 @@ __global__ void __launch_bounds__(256) quantize_kernel(
   extern __shared__ int32_t smem[];
   int32_t *off = smem, *slot = smem + (G + 1), *scratch = smem + 2 * (G + 1);
   if (group_offsets) load_groups(group_offsets, G, off, slot, scratch);
-  const int lane = threadIdx.x & 31, half = lane & 1;
+  const int lane = threadIdx.x & 31;
   const uint32_t K = (uint32_t)K64, nblk = K >> 4;
-  const uint32_t nsl = (nblk + 15) >> 4;                     // 16-block slices per row
   const uint32_t p_end = group_offsets ? (uint32_t)slot[G] : (uint32_t)P;
-  const uint64_t units = (uint64_t)p_end * nsl;              // (row, slice) work units, row-major
-  constexpr int U = 4;                                       // consecutive units per warp step
-  const uint64_t nchunks = (units + U - 1) / U;
+  const uint64_t total = (uint64_t)p_end * nblk;             // blocks, row-major
+  constexpr int U = 2;                                       // 32-block steps per chunk
+  const uint64_t nchunks = (total + 32 * U - 1) / (32 * U);
   const uint64_t warp = ((uint64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const uint64_t nwarps = ((uint64_t)gridDim.x * blockDim.x) >> 5;
-  const bool small = units < 0xFFFFFFF0ull;
-  // Warps stride over 4-unit chunks (2 KB of input per warp step, all warps
-  // moving through memory together).  Rows only move forward per lane, so the
-  // row -> (group, source row) lookup walks forward from the last group.
+  const bool small = total < 0xFFFFFFF0ull;
+  const bool v8 = ((reinterpret_cast<uintptr_t>(x) & 31u) == 0) && ((ld_x & 15) == 0);
   int g = 0;
   uint32_t cached_p = 0xFFFFFFFFu;
   int64_t cached_src = -1;
   bool cached_real = false;
+  float s_g = 1.0f, t_g = 6.0f;
+  int g_for_scale = -1;
   bool bad = false;
   for (uint64_t c = warp; c < nchunks; c += nwarps) {
-    EncodeItem it[U];
-    int64_t src[U];
+    uint4 va[U], vb[U];
+    uint32_t pp[U], jj[U];
+    bool real[U], inr[U];
+    float sg[U], tg[U];
 #pragma unroll
     for (int k = 0; k < U; ++k) {
-      const uint64_t unit = c * U + k;
-      uint32_t p = 0, sl = 0;
-      if (unit < units) {
-        if (small) { p = (uint32_t)unit / nsl; sl = (uint32_t)unit - p * nsl; }
-        else { p = (uint32_t)(unit / nsl); sl = (uint32_t)(unit - (uint64_t)p * nsl); }
-      }
-      const uint32_t j = sl * 16 + (lane >> 1);
-      it[k].in_range = unit < units && j < nblk;
-      it[k].p = p;
-      it[k].j = j;
-      if (unit < units && p != cached_p) {
-        cached_p = p;
-        if (group_offsets) {
-          if (g + 8 < G && (uint32_t)slot[g + 8] <= p) g = upper_group(slot, G, p);
-          while (g + 1 < G && (uint32_t)slot[g + 1] <= p) ++g;
-          const uint32_t local = p - (uint32_t)slot[g];
-          cached_real = local < (uint32_t)(off[g + 1] - off[g]);
-          cached_src = (int64_t)off[g] + local;
-        } else {
-          cached_real = p < (uint64_t)rows;
-          cached_src = p;
+      const uint64_t b = c * (32 * U) + k * 32 + lane;
+      inr[k] = b < total;
+      uint32_t p = 0, j = 0;
+      if (inr[k]) {
+        if (small) { p = (uint32_t)b / nblk; j = (uint32_t)b - p * nblk; }
+        else { p = (uint32_t)(b / nblk); j = (uint32_t)(b - (uint64_t)p * nblk); }
+        if (p != cached_p) {
+          cached_p = p;
+          if (group_offsets) {
+            if (g + 8 < G && (uint32_t)slot[g + 8] <= p) g = upper_group(slot, G, p);
+            while (g + 1 < G && (uint32_t)slot[g + 1] <= p) ++g;
+            const uint32_t local = p - (uint32_t)slot[g];
+            cached_real = local < (uint32_t)(off[g + 1] - off[g]);
+            cached_src = (int64_t)off[g] + local;
+          } else {
+            cached_real = p < (uint64_t)rows;
+            cached_src = p;
+          }
+          if (cached_real && row_index) cached_src = row_index[cached_src];
+          if (g != g_for_scale) {
+            g_for_scale = g;
+            s_g = gs[g];
+            t_g = __fmul_rn(6.0f, s_g);
+          }
         }
-        if (cached_real && row_index) cached_src = row_index[cached_src];
       }
-      it[k].g = g;
-      it[k].real = it[k].in_range && cached_real;
-      src[k] = cached_src;
+      pp[k] = p;
+      jj[k] = j;
+      real[k] = inr[k] && cached_real;
+      sg[k] = s_g;
+      tg[k] = t_g;
+      va[k] = make_uint4(0, 0, 0, 0);
+      vb[k] = make_uint4(0, 0, 0, 0);
+      if (real[k]) load_block(x + cached_src * ld_x + (uint64_t)j * 16, v8, va[k], vb[k]);
     }
 #pragma unroll
     for (int k = 0; k < U; ++k) {
-      it[k].v = make_uint4(0, 0, 0, 0);
-      if (it[k].real) it[k].v = ldg_nc_v4(x + src[k] * ld_x + it[k].j * 16 + half * 8);
-    }
+      const uint32_t m2 = absmax8_bits(vb[k], absmax8_bits(va[k], 0));
+      const uint32_t m = halves_max(m2);
+      if (real[k] && m >= 0x7F80u) bad = true;
+      uint32_t S = 0;
+      if (real[k]) S = f32_to_e4m3_satfinite(__fdiv_rn(__uint_as_float(m << 16), tg[k]));
+      const float e = __fmul_rn(e4m3_to_f32(S), sg[k]);
+      const float r = (e == 0.0f) ? 0.0f : __frcp_rn(e);
+      const uint64_t rr = ((uint64_t)__float_as_uint(r) << 32) | __float_as_uint(r);
+      const uint32_t w[8] = {va[k].x, va[k].y, va[k].z, va[k].w, vb[k].x, vb[k].y, vb[k].z, vb[k].w};
+      uint64_t prod[8];
 #pragma unroll
-    for (int k = 0; k < U; ++k) encode_finish<kTiled>(it[k], half, nblk, K, gs, q, sf, bad);
+      for (int i = 0; i < 8; ++i) prod[i] = mul_pair(w[i], rr);
+      if (isinf(r)) {                     // 0 * inf: the NaN encodes as +0
+#pragma unroll
+        for (int i = 0; i < 8; ++i) prod[i] = sanitize_pair(prod[i]);
+      }
+      uint2 codes;
+      codes.x = e2m1x4_from_pairs(prod[0], prod[1]) | (e2m1x4_from_pairs(prod[2], prod[3]) << 16);
+      codes.y = e2m1x4_from_pairs(prod[4], prod[5]) | (e2m1x4_from_pairs(prod[6], prod[7]) << 16);
+      if (inr[k]) {
+        *reinterpret_cast<uint2 *>(q + (uint64_t)pp[k] * (K >> 1) + (uint64_t)jj[k] * 8) = codes;
+        if (kTiled) sf[sf_tiled_offset(pp[k], jj[k], nblk)] = (uint8_t)S;
+        else sf[(uint64_t)pp[k] * nblk + jj[k]] = (uint8_t)S;
+      }
+    }
   }
   if (bad) report(dev_status, NVFP4_ERR_NONFINITE);
 }
 
 // ---------------------------------------------------------------- dequantize
+// (code * S) in f16 is exact (at most 6 significant bits, |.| <= 2688), so the
+// hardware E2M1 -> f16 conversion times the f16 scale gives the exact product;
+// one fp32 multiply by s_g then rounds once, as the definition asks.
+__device__ __forceinline__ uint64_t dq_pair(uint32_t byte, uint32_t S2h, uint64_t gg) {
+  uint32_t h;
+  asm("{\n.reg .b8 b;\ncvt.u8.u32 b, %1;\ncvt.rn.f16x2.e2m1x2 %0, b;\n}" : "=r"(h) : "r"(byte));
+  asm("mul.rn.f16x2 %0, %0, %1;" : "+r"(h) : "r"(S2h));
+  float lo, hi;
+  asm("{\n.reg .f16 l, u;\nmov.b32 {l, u}, %2;\ncvt.f32.f16 %0, l;\ncvt.f32.f16 %1, u;\n}" : "=f"(lo), "=f"(hi) : "r"(h));
+  const uint64_t x = ((uint64_t)__float_as_uint(hi) << 32) | __float_as_uint(lo);
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(x), "l"(gg));
+  return d;
+}
+
 template <bool kTiled, bool kBf16>
 __global__ void __launch_bounds__(256) dequantize_kernel(
     const uint8_t *__restrict__ q, const uint8_t *__restrict__ sf, const float *__restrict__ gs,
@@ -266,8 +311,11 @@ __global__ void __launch_bounds__(256) dequantize_kernel(
   const uint64_t total = (uint64_t)rows * nhalf;
   const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
   const uint64_t nblk = (uint64_t)(K >> 4);
+  const bool small = total < 0xFFFFFFF0ull;
   for (uint64_t h = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; h < total; h += stride) {
-    const uint64_t r = h / nhalf, c = h - r * nhalf;
+    uint64_t r, c;
+    if (small) { const uint32_t r32 = (uint32_t)h / (uint32_t)nhalf; r = r32; c = (uint32_t)h - r32 * (uint32_t)nhalf; }
+    else { r = h / nhalf; c = h - r * nhalf; }
     const uint64_t j = c >> 1;
     int g = 0;
     uint64_t p = r;
@@ -276,27 +324,29 @@ __global__ void __launch_bounds__(256) dequantize_kernel(
       p = (uint64_t)slot[g] + (r - (uint64_t)off[g]);
     }
     const float s_g = gs[g];
-    const float Sv = e4m3_to_f32(kTiled ? sf[sf_tiled_offset(p, j, nblk)] : sf[p * nblk + j]);
-    const uint32_t cw = *reinterpret_cast<const uint32_t *>(q + p * (K >> 1) + c * 4);
-    float out[8];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint32_t byte = (cw >> (8 * i)) & 0xFFu;
-      out[2 * i] = __fmul_rn(__fmul_rn(e2m1_to_f32(byte & 15u), Sv), s_g);
-      out[2 * i + 1] = __fmul_rn(__fmul_rn(e2m1_to_f32(byte >> 4), Sv), s_g);
+    const uint32_t sb = kTiled ? sf[sf_tiled_offset(p, j, nblk)] : sf[p * nblk + j];
+    uint32_t S2h;
+    {
+      const uint16_t pair = (uint16_t)(sb | (sb << 8));
+      asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(S2h) : "h"(pair));
     }
+    const uint64_t gg = ((uint64_t)__float_as_uint(s_g) << 32) | __float_as_uint(s_g);
+    const uint32_t cw = *reinterpret_cast<const uint32_t *>(q + p * (K >> 1) + c * 4);
+    uint64_t d[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) d[i] = dq_pair((cw >> (8 * i)) & 0xFFu, S2h, gg);
     if (kBf16) {
       uint32_t hw[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        __nv_bfloat162 t = __floats2bfloat162_rn(out[2 * i], out[2 * i + 1]);
+        __nv_bfloat162 t = __floats2bfloat162_rn(__uint_as_float((uint32_t)d[i]), __uint_as_float((uint32_t)(d[i] >> 32)));
         hw[i] = *reinterpret_cast<uint32_t *>(&t);
       }
       *reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(y) + r * K + c * 8) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
     } else {
-      float4 *dst = reinterpret_cast<float4 *>(reinterpret_cast<float *>(y) + r * K + c * 8);
-      dst[0] = make_float4(out[0], out[1], out[2], out[3]);
-      dst[1] = make_float4(out[4], out[5], out[6], out[7]);
+      uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<float *>(y) + r * K + c * 8);
+      dst[0] = make_uint4((uint32_t)d[0], (uint32_t)(d[0] >> 32), (uint32_t)d[1], (uint32_t)(d[1] >> 32));
+      dst[1] = make_uint4((uint32_t)d[2], (uint32_t)(d[2] >> 32), (uint32_t)d[3], (uint32_t)(d[3] >> 32));
     }
   }
 }
@@ -398,6 +448,26 @@ int64_t grid_for(int64_t work_items, int threads, int per_sm) {
   return need < cap ? need : cap;
 }
 
+// Grid for a grid-stride kernel: at most one wave of resident blocks, so no
+// block starts late with a full share of the work.
+struct OccEntry { const void *fn; int threads; size_t smem; int per_sm; };
+OccEntry g_occ[64];
+int g_occ_n = 0;
+
+template <typename Kernel>
+int64_t grid_resident(Kernel kernel, int64_t work_items, int threads, size_t smem) {
+  const void *fn = reinterpret_cast<const void *>(kernel);
+  int per_sm = 0;
+  for (int i = 0; i < g_occ_n; ++i)
+    if (g_occ[i].fn == fn && g_occ[i].threads == threads && g_occ[i].smem == smem) per_sm = g_occ[i].per_sm;
+  if (per_sm == 0) {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem) != cudaSuccess || per_sm < 1)
+      per_sm = 1;
+    if (g_occ_n < 64) g_occ[g_occ_n++] = OccEntry{fn, threads, smem, per_sm};
+  }
+  return grid_for(work_items, threads, per_sm);
+}
+
 nvfp4_status launch_status() {
   return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
@@ -438,13 +508,15 @@ nvfp4_status run_encode(const uint16_t *x, int64_t rows, int64_t K, int64_t ld_x
   if (group_offsets) P = nvfp4_padded_rows_bound(rows, G);
   else P = tiled ? (rows + 127) / 128 * 128 : rows;
   if (P == 0) return NVFP4_OK;
-  const int64_t pairs = P * (K / 16);
+  const int64_t blocks = P * (K / 16);
   const size_t sm = group_offsets ? sizeof(int32_t) * (2 * (G + 1) + 8) : 0;
-  const unsigned grid = (unsigned)grid_for(pairs * 2, 256, 8);
-  if (tiled)
+  if (tiled) {
+    const unsigned grid = (unsigned)grid_resident(quantize_kernel<true>, (blocks + 1) / 2, 256, sm);
     quantize_kernel<true><<<grid, 256, sm, stream>>>(x, ld_x, K, rows, row_index, group_offsets, G, P, gs, q, sf, dev_status);
-  else
+  } else {
+    const unsigned grid = (unsigned)grid_resident(quantize_kernel<false>, (blocks + 1) / 2, 256, sm);
     quantize_kernel<false><<<grid, 256, sm, stream>>>(x, ld_x, K, rows, row_index, group_offsets, G, P, gs, q, sf, dev_status);
+  }
   return launch_status();
 }
 
@@ -542,11 +614,13 @@ nvfp4_status nvfp4_swiglu_quantize(const void *y, nvfp4_out_dtype y_dtype, int64
   if (cudaMemsetAsync(amax_bits, 0, sizeof(uint32_t) * G, stream) != cudaSuccess) return NVFP4_ERR_CUDA;
   if (rows > 0) {
     const size_t sm = group_offsets ? sizeof(int32_t) * (G + 1) : 0;
-    const unsigned grid = (unsigned)grid_for(rows * 32, 256, 8);
-    if (y_dtype == NVFP4_OUT_BF16)
+    if (y_dtype == NVFP4_OUT_BF16) {
+      const unsigned grid = (unsigned)grid_resident(swiglu_amax_kernel<true>, rows * 32, 256, sm);
       swiglu_amax_kernel<true><<<grid, 256, sm, stream>>>(y, rows, I, group_offsets, G, (uint16_t *)h, amax_bits);
-    else
+    } else {
+      const unsigned grid = (unsigned)grid_resident(swiglu_amax_kernel<false>, rows * 32, 256, sm);
       swiglu_amax_kernel<false><<<grid, 256, sm, stream>>>(y, rows, I, group_offsets, G, (uint16_t *)h, amax_bits);
+    }
     if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_CUDA;
   }
   finalize_scales_kernel<<<(G + 127) / 128, 128, 0, stream>>>(amax_bits, G, 0, global_scale, dev_status);

@@ -32,16 +32,28 @@ __global__ void __launch_bounds__(256) remap_scan_kernel(
   const uint8_t *et = e8 + t * blocks_per_tensor;
   uint32_t hi = 0, lo = 0;
   bool bad = false;
-  for (int64_t b = b0 + threadIdx.x; b < b1; b += blockDim.x) {
-    const uint4 c = __ldg(qt + b);          // the 32 codes of this block
-    const uint32_t u = et[b];
-    if (qo != qt) qo[b] = c;
-    if (u == 0xFFu) { bad = true; continue; }
+  const bool copy = qo != qt;
+  auto visit = [&](uint4 c, uint32_t u) {
+    if (u == 0xFFu) { bad = true; return; }
     const uint32_t nz = (c.x | c.y | c.z | c.w) & 0x77777777u;   // magnitude bits
     if (nz) {
       hi = max(hi, u + 1u);
       lo = max(lo, 256u - u);
     }
+  };
+  // four blocks (64 bytes of codes) in flight per thread
+  int64_t b = b0 + threadIdx.x;
+  const int64_t st = blockDim.x;
+  for (; b + 3 * st < b1; b += 4 * st) {
+    const uint4 c0 = __ldg(qt + b), c1 = __ldg(qt + b + st), c2 = __ldg(qt + b + 2 * st), c3 = __ldg(qt + b + 3 * st);
+    const uint32_t u0 = et[b], u1 = et[b + st], u2 = et[b + 2 * st], u3 = et[b + 3 * st];
+    if (copy) { qo[b] = c0; qo[b + st] = c1; qo[b + 2 * st] = c2; qo[b + 3 * st] = c3; }
+    visit(c0, u0); visit(c1, u1); visit(c2, u2); visit(c3, u3);
+  }
+  for (; b < b1; b += st) {
+    const uint4 c = __ldg(qt + b);
+    if (copy) qo[b] = c;
+    visit(c, et[b]);
   }
 #pragma unroll
   for (int d = 16; d > 0; d >>= 1) {
@@ -65,16 +77,23 @@ __global__ void __launch_bounds__(256) remap_scale_kernel(
     const uint8_t *__restrict__ e8, int64_t rows, int64_t K, int64_t n_tensors,
     const uint32_t *__restrict__ ws, uint8_t *__restrict__ sf, float *__restrict__ gs,
     int32_t *dev_status) {
-  const int64_t nb32_row = K >> 5;
-  const int64_t per_tensor = rows * nb32_row;
-  const int64_t total = n_tensors * per_tensor;
-  const int64_t nsf = K >> 4;
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += stride) {
-    const int64_t t = i / per_tensor;
+  const uint64_t nb32_row = (uint64_t)(K >> 5);
+  const uint64_t per_tensor = (uint64_t)rows * nb32_row;
+  const uint64_t total = (uint64_t)n_tensors * per_tensor;
+  const uint64_t nsf = (uint64_t)(K >> 4);
+  const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
+  const bool small = total < 0xFFFFFFF0ull;
+  for (uint64_t i = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += stride) {
+    uint64_t t, within, r, jb;
+    if (small) {
+      const uint32_t i32 = (uint32_t)i, t32 = i32 / (uint32_t)per_tensor;
+      const uint32_t w32 = i32 - t32 * (uint32_t)per_tensor, r32 = w32 / (uint32_t)nb32_row;
+      t = t32; within = w32; r = r32; jb = w32 - r32 * (uint32_t)nb32_row;
+    } else {
+      t = i / per_tensor; within = i - t * per_tensor; r = within / nb32_row; jb = within - r * nb32_row;
+    }
     const uint32_t hi = ws[2 * t], lo = ws[2 * t + 1];
     const int g = hi ? (int)hi - 1 - 127 - 8 : 0;
-    const int64_t within = i - t * per_tensor;
     if (within == 0) {
       gs[t] = ldexpf(1.0f, g);   // 2^g exactly, g in [-135, 119] (subnormal below -126)
       if (hi) {
@@ -85,13 +104,12 @@ __global__ void __launch_bounds__(256) remap_scale_kernel(
     const int e = (int)e8[i] - 127;
     const int p = max(-9, min(8, e - g));
     const uint32_t S = e4m3_pow2(p);
-    const int64_t r = t * rows + within / nb32_row;
-    const int64_t j = 2 * (within - (within / nb32_row) * nb32_row);
+    const uint64_t row = t * (uint64_t)rows + r, j = 2 * jb;
     if (kTiled) {
-      sf[sf_tiled_offset(r, j, nsf)] = (uint8_t)S;
-      sf[sf_tiled_offset(r, j + 1, nsf)] = (uint8_t)S;
+      // scales j and j+1 share one 4-scale group: two adjacent bytes
+      *reinterpret_cast<uint16_t *>(sf + sf_tiled_offset(row, j, nsf)) = (uint16_t)(S | (S << 8));
     } else {
-      *reinterpret_cast<uint16_t *>(sf + r * nsf + j) = (uint16_t)(S | (S << 8));
+      *reinterpret_cast<uint16_t *>(sf + row * nsf + j) = (uint16_t)(S | (S << 8));
     }
   }
 }
