@@ -183,6 +183,96 @@ __device__ __forceinline__ uint64_t sanitize_pair(uint64_t d) {
   return ((uint64_t)__float_as_uint(hi) << 32) | __float_as_uint(lo);
 }
 
+// The 16-element block math (see the definition in include/nvfp4.h): block
+// amax, S = e4m3(a_b / (6 s_g)), r = 1/(S s_g), codes = e2m1(x r).  Returns
+// the 8 packed code bytes and S; flags non-finite input.
+__device__ __forceinline__ uint2 encode_block16(const uint4 &va, const uint4 &vb, float s_g, float t_g, bool real,
+                                                uint32_t &S, bool &bad) {
+  const uint32_t m = halves_max(absmax8_bits(vb, absmax8_bits(va, 0)));
+  if (real && m >= 0x7F80u) bad = true;
+  S = 0;
+  if (real) S = f32_to_e4m3_satfinite(__fdiv_rn(__uint_as_float(m << 16), t_g));
+  const float e = __fmul_rn(e4m3_to_f32(S), s_g);
+  const float r = (e == 0.0f) ? 0.0f : __frcp_rn(e);
+  const uint64_t rr = ((uint64_t)__float_as_uint(r) << 32) | __float_as_uint(r);
+  const uint32_t w[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
+  uint64_t prod[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) prod[i] = mul_pair(w[i], rr);
+  if (isinf(r)) {                     // 0 * inf: the NaN encodes as +0
+#pragma unroll
+    for (int i = 0; i < 8; ++i) prod[i] = sanitize_pair(prod[i]);
+  }
+  uint2 codes;
+  codes.x = e2m1x4_from_pairs(prod[0], prod[1]) | (e2m1x4_from_pairs(prod[2], prod[3]) << 16);
+  codes.y = e2m1x4_from_pairs(prod[4], prod[5]) | (e2m1x4_from_pairs(prod[6], prod[7]) << 16);
+  return codes;
+}
+
+// Gathered long rows (row_index, K >= 2048): one warp per output row, the row's group and source
+// row looked up once, up to 8 blocks (256 bytes) in flight per lane; warps
+// stride over rows so the grid streams through the input together.
+template <bool kTiled>
+__global__ void __launch_bounds__(256) quantize_rows_kernel(
+    const uint16_t *__restrict__ x, int64_t ld_x, int64_t K64, int64_t rows,
+    const int32_t *__restrict__ row_index, const int32_t *__restrict__ group_offsets, int G,
+    int64_t P, const float *__restrict__ gs, uint8_t *__restrict__ q, uint8_t *__restrict__ sf,
+    int32_t *dev_status) {
+  extern __shared__ int32_t smem[];
+  int32_t *off = smem, *slot = smem + (G + 1), *scratch = smem + 2 * (G + 1);
+  if (group_offsets) load_groups(group_offsets, G, off, slot, scratch);
+  const int lane = threadIdx.x & 31;
+  const uint32_t K = (uint32_t)K64, nblk = K >> 4;
+  const uint32_t p_end = group_offsets ? (uint32_t)slot[G] : (uint32_t)P;
+  const uint32_t warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
+  const bool v8 = ((reinterpret_cast<uintptr_t>(x) & 31u) == 0) && ((ld_x & 15) == 0);
+  int g = 0;
+  bool bad = false;
+  constexpr int B = 8;
+  for (uint32_t p = warp; p < p_end; p += nwarps) {
+    bool real;
+    int64_t src;
+    if (group_offsets) {
+      if (g + 8 < G && (uint32_t)slot[g + 8] <= p) g = upper_group(slot, G, p);
+      while (g + 1 < G && (uint32_t)slot[g + 1] <= p) ++g;
+      const uint32_t local = p - (uint32_t)slot[g];
+      real = local < (uint32_t)(off[g + 1] - off[g]);
+      src = (int64_t)off[g] + local;
+    } else {
+      real = p < (uint64_t)rows;
+      src = p;
+    }
+    if (real && row_index) src = row_index[src];
+    const float s_g = real ? gs[g] : 1.0f;
+    const float t_g = __fmul_rn(6.0f, s_g);
+    const uint16_t *xr = x + src * ld_x;
+    uint8_t *qr = q + (uint64_t)p * (K >> 1);
+    for (uint32_t j0 = 0; j0 < nblk; j0 += 32 * B) {
+      uint4 va[B], vb[B];
+#pragma unroll
+      for (int k = 0; k < B; ++k) {
+        const uint32_t j = j0 + k * 32 + lane;
+        va[k] = make_uint4(0, 0, 0, 0);
+        vb[k] = make_uint4(0, 0, 0, 0);
+        if (real && j < nblk) load_block(xr + (uint64_t)j * 16, v8, va[k], vb[k]);
+      }
+#pragma unroll
+      for (int k = 0; k < B; ++k) {
+        const uint32_t j = j0 + k * 32 + lane;
+        uint32_t S;
+        const uint2 codes = encode_block16(va[k], vb[k], s_g, t_g, real && j < nblk, S, bad);
+        if (j < nblk) {
+          *reinterpret_cast<uint2 *>(qr + (uint64_t)j * 8) = codes;
+          if (kTiled) sf[sf_tiled_offset(p, j, nblk)] = (uint8_t)S;
+          else sf[(uint64_t)p * nblk + j] = (uint8_t)S;
+        }
+      }
+    }
+  }
+  if (bad) report(dev_status, NVFP4_ERR_NONFINITE);
+}
+
 template <bool kTiled>
 __global__ void __launch_bounds__(256) quantize_kernel(
     const uint16_t *__restrict__ x, int64_t ld_x, int64_t K64, int64_t rows,
@@ -253,25 +343,8 @@ __global__ void __launch_bounds__(256) quantize_kernel(
     }
 #pragma unroll
     for (int k = 0; k < U; ++k) {
-      const uint32_t m2 = absmax8_bits(vb[k], absmax8_bits(va[k], 0));
-      const uint32_t m = halves_max(m2);
-      if (real[k] && m >= 0x7F80u) bad = true;
-      uint32_t S = 0;
-      if (real[k]) S = f32_to_e4m3_satfinite(__fdiv_rn(__uint_as_float(m << 16), tg[k]));
-      const float e = __fmul_rn(e4m3_to_f32(S), sg[k]);
-      const float r = (e == 0.0f) ? 0.0f : __frcp_rn(e);
-      const uint64_t rr = ((uint64_t)__float_as_uint(r) << 32) | __float_as_uint(r);
-      const uint32_t w[8] = {va[k].x, va[k].y, va[k].z, va[k].w, vb[k].x, vb[k].y, vb[k].z, vb[k].w};
-      uint64_t prod[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) prod[i] = mul_pair(w[i], rr);
-      if (isinf(r)) {                     // 0 * inf: the NaN encodes as +0
-#pragma unroll
-        for (int i = 0; i < 8; ++i) prod[i] = sanitize_pair(prod[i]);
-      }
-      uint2 codes;
-      codes.x = e2m1x4_from_pairs(prod[0], prod[1]) | (e2m1x4_from_pairs(prod[2], prod[3]) << 16);
-      codes.y = e2m1x4_from_pairs(prod[4], prod[5]) | (e2m1x4_from_pairs(prod[6], prod[7]) << 16);
+      uint32_t S;
+      const uint2 codes = encode_block16(va[k], vb[k], sg[k], tg[k], real[k], S, bad);
       if (inr[k]) {
         *reinterpret_cast<uint2 *>(q + (uint64_t)pp[k] * (K >> 1) + (uint64_t)jj[k] * 8) = codes;
         if (kTiled) sf[sf_tiled_offset(pp[k], jj[k], nblk)] = (uint8_t)S;
@@ -510,6 +583,17 @@ nvfp4_status run_encode(const uint16_t *x, int64_t rows, int64_t K, int64_t ld_x
   if (P == 0) return NVFP4_OK;
   const int64_t blocks = P * (K / 16);
   const size_t sm = group_offsets ? sizeof(int32_t) * (2 * (G + 1) + 8) : 0;
+  if (row_index && K >= 2048 && P <= 0xFFFFFFFFll) {
+    // one warp per output row
+    if (tiled) {
+      const unsigned grid = (unsigned)grid_resident(quantize_rows_kernel<true>, P * 32, 256, sm);
+      quantize_rows_kernel<true><<<grid, 256, sm, stream>>>(x, ld_x, K, rows, row_index, group_offsets, G, P, gs, q, sf, dev_status);
+    } else {
+      const unsigned grid = (unsigned)grid_resident(quantize_rows_kernel<false>, P * 32, 256, sm);
+      quantize_rows_kernel<false><<<grid, 256, sm, stream>>>(x, ld_x, K, rows, row_index, group_offsets, G, P, gs, q, sf, dev_status);
+    }
+    return launch_status();
+  }
   if (tiled) {
     const unsigned grid = (unsigned)grid_resident(quantize_kernel<true>, (blocks + 1) / 2, 256, sm);
     quantize_kernel<true><<<grid, 256, sm, stream>>>(x, ld_x, K, rows, row_index, group_offsets, G, P, gs, q, sf, dev_status);
