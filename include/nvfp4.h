@@ -132,9 +132,10 @@ nvfp4_status nvfp4_dequantize(const uint8_t *q, const uint8_t *sf, nvfp4_sf_layo
 /*
  * mxfp4_to_nvfp4 -- lossless block-by-block MXFP4 -> NVFP4 weight remap.
  * [P2: MXFP4 uses 32-element blocks with UE8M0 (power-of-two) scales, NVFP4
- *  16-element blocks with a finer scale, and the weights "can be remapped
- *  block by block without loss"; the conversion script does the E2M1->E4M3
- *  remap.]
+ *  16-element blocks with a finer scale; because the finer format can express
+ *  every MXFP4 block exactly, the page converts the weights one block at a time
+ *  with no change to any dequantized value (its conversion script performs an
+ *  E2M1->E4M3 scale remap).]
  *   n_tensors tensors of [rows, K] laid back to back (K % 32 == 0).
  *   q_mx uint8 [n*rows, K/2]; ue8m0 uint8 [n*rows, K/32].
  *   q_nv uint8 [n*rows, K/2] (codes copied unchanged; may equal q_mx);
@@ -212,6 +213,36 @@ nvfp4_status nvfp4_kv_dequantize(const uint8_t *k_q, const uint8_t *k_sf, const 
                                  const uint8_t *v_q, const uint8_t *v_sf, const float *v_gs,
                                  int64_t tokens, int64_t heads, int64_t head_dim,
                                  void *k_out, void *v_out, cudaStream_t stream);
+
+/*
+ * nvfp4_quantize_noalloc -- nvfp4_quantize without a caller workspace.
+ *
+ * For callers that cannot hand the library a scratch buffer: code that must
+ * not call cudaMalloc or a caching allocator at this point (a host runtime
+ * whose device memory is owned and budgeted by another component, an
+ * allocator-free plug-in or interposer, a hot path that has to stay free of
+ * allocation-related synchronisation).  This entry point is not described by
+ * the pages; it exists for those callers.
+ *
+ * Same arguments, arithmetic and results as nvfp4_quantize, minus `workspace`.
+ * The scratch (per-group amax words) lives in one static device array inside
+ * the library, sized for NVFP4_NOALLOC_MAX_GROUPS groups (8.25 KB on every GPU
+ * that loads the library, held until process exit).  num_groups (or 1 without
+ * group_offsets) above NVFP4_NOALLOC_MAX_GROUPS returns
+ * NVFP4_ERR_UNSUPPORTED_SHAPE.  Nothing is allocated or freed: the first call
+ * on a device looks up that device's address of the array (a runtime symbol
+ * query, no allocation) and caches it, so make that first call before any
+ * stream capture on the device.  Every call shares the array and clears the
+ * words it needs before use; calls that can overlap on the GPU (different
+ * streams, or a second call enqueued before the first finished on another
+ * stream) race on it and must be serialised by the caller.
+ */
+#define NVFP4_NOALLOC_MAX_GROUPS 1024
+nvfp4_status nvfp4_quantize_noalloc(const void *x, int64_t rows, int64_t K, int64_t ld_x,
+                                    const int32_t *row_index, const int32_t *group_offsets,
+                                    int num_groups, nvfp4_gs_mode gs_mode, float *global_scale,
+                                    uint8_t *q, uint8_t *sf, nvfp4_sf_layout sf_layout,
+                                    int32_t *dev_status, cudaStream_t stream);
 
 #ifdef __cplusplus
 }

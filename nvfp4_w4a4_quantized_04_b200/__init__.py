@@ -39,8 +39,9 @@ EPI_NONE = 0
 EXPORTS = [
     "nvfp4_status_string", "nvfp4_workspace_size", "nvfp4_padded_rows_bound",
     "nvfp4_quantize", "nvfp4_dequantize", "mxfp4_to_nvfp4", "nvfp4_grouped_gemm",
-    "nvfp4_swiglu_quantize", "nvfp4_kv_quantize", "nvfp4_kv_dequantize",
+    "nvfp4_swiglu_quantize", "nvfp4_kv_quantize", "nvfp4_kv_dequantize", "nvfp4_quantize_noalloc",
 ]
+NOALLOC_MAX_GROUPS = 1024
 
 _lib = None
 
@@ -76,6 +77,8 @@ def load_library(path: str = LIB_PATH):
     L.nvfp4_swiglu_quantize.argtypes = [P, i32, i64, i64, P, i32, P, P, P, i32, P, P, P, P]
     L.nvfp4_kv_quantize.restype = i32
     L.nvfp4_kv_quantize.argtypes = [P, P, i64, i64, i64, i32, P, P, P, P, P, P, P, P, P]
+    L.nvfp4_quantize_noalloc.restype = i32
+    L.nvfp4_quantize_noalloc.argtypes = [P, i64, i64, i64, P, P, i32, i32, P, P, P, i32, P, P]
     L.nvfp4_kv_dequantize.restype = i32
     L.nvfp4_kv_dequantize.argtypes = [P, P, P, P, P, P, i64, i64, i64, P, P, P]
     _lib = L
@@ -117,6 +120,18 @@ def nvfp4_quantize(x, rows, K, ld_x, row_index, group_offsets, num_groups, gs_mo
         _ptr(global_scale), _ptr(q), _ptr(sf), sf_layout, _ptr(workspace), _ptr(dev_status), _stream(stream))
     if check:
         _check(st, "nvfp4_quantize")
+    return st
+
+
+def nvfp4_quantize_noalloc(x, rows, K, ld_x, row_index, group_offsets, num_groups, gs_mode, global_scale,
+                           q, sf, sf_layout, dev_status=None, stream=None, check=True) -> int:
+    """nvfp4_quantize with the library's own static scratch instead of a workspace
+    (for callers that cannot allocate; at most NOALLOC_MAX_GROUPS groups)."""
+    st = load_library().nvfp4_quantize_noalloc(
+        _ptr(x), rows, K, ld_x, _ptr(row_index), _ptr(group_offsets), num_groups, gs_mode,
+        _ptr(global_scale), _ptr(q), _ptr(sf), sf_layout, _ptr(dev_status), _stream(stream))
+    if check:
+        _check(st, "nvfp4_quantize_noalloc")
     return st
 
 

@@ -13,6 +13,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "common.cuh"
 
 namespace nvfp4 {
@@ -740,3 +742,39 @@ nvfp4_status nvfp4_kv_dequantize(const uint8_t *k_q, const uint8_t *k_sf, const 
 }
 
 }  // extern "C"
+
+// ======================================================= allocation-free variant
+// Scratch of nvfp4_quantize_noalloc: the per-group amax words (the same layout
+// nvfp4_quantize keeps in the caller's workspace), one copy per device.
+static __device__ __align__(256) uint32_t g_noalloc_scratch[2 * NVFP4_NOALLOC_MAX_GROUPS + 64];
+
+namespace {
+std::mutex g_noalloc_mu;
+void *g_noalloc_ptr[64] = {};       // per device ordinal, filled by the first call on that device
+}  // namespace
+
+extern "C" nvfp4_status nvfp4_quantize_noalloc(const void *x, int64_t rows, int64_t K, int64_t ld_x,
+                                               const int32_t *row_index, const int32_t *group_offsets,
+                                               int num_groups, nvfp4_gs_mode gs_mode, float *global_scale,
+                                               uint8_t *q, uint8_t *sf, nvfp4_sf_layout sf_layout,
+                                               int32_t *dev_status, cudaStream_t stream) {
+  const int G = group_offsets ? num_groups : 1;
+  if (G < 1) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (G > NVFP4_NOALLOC_MAX_GROUPS) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return NVFP4_ERR_CUDA;
+  void *scratch;
+  {
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+      // host code cannot use the array's name as a device address: ask the
+      // runtime for this device's address of it, once
+      void *ptr = nullptr;
+      if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return NVFP4_ERR_CUDA;
+      g_noalloc_ptr[dev] = ptr;
+    }
+    scratch = g_noalloc_ptr[dev];
+  }
+  return nvfp4_quantize(x, rows, K, ld_x, row_index, group_offsets, num_groups, gs_mode, global_scale, q, sf,
+                        sf_layout, scratch, dev_status, stream);
+}
