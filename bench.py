@@ -458,7 +458,34 @@ def comp_remap(device, iters, warmup, flush):
             "frac_hbm": round(gbs(b, ms) / HBM_PEAK, 4)}
 
 
-COMPONENTS = {"dense_mlp": comp_dense_mlp, "decode_moe": comp_decode_moe, "kv_cache": comp_kv,
+def comp_moe_full(device, iters, warmup, flush):
+    """The whole routed-expert block of the headline layer: on-device routing
+    order from the router's top-10 ids, the NVFP4 experts, and the weighted
+    combine back to [8192, 4096]."""
+    import torch
+
+    import synthetic
+    from nvfp4_w4a4_quantized_04_b200 import layer as L
+    E, T, H, I, k = 512, 8192, 4096, 1024, 10
+    moe, x, ri, off, r, R = setup_moe(device, 0, E, T, H, I, k)
+    full = L.MoELayer(moe, T, k, device)
+    ids = torch.from_numpy(r["experts"].astype(np.int32)).to(device)
+    w = torch.from_numpy(r["weights"].astype(np.float32)).to(device)
+    t_route = timed(lambda: L.route(ids, E), iters, warmup, flush)
+    y2 = moe.forward(x, ri, off)
+    t_comb = timed(lambda: L.combine(y2, full.slot[:T], w, out_dtype=1, out=full.out[:T]), iters, warmup, flush)
+    full.forward(x, ids, w)
+    t_full = timed(lambda: full.forward(x, ids, w), iters, warmup, flush)
+    flops = moe_flops(R, H, I)
+    comb_bytes = R * H * 2 + T * H * 2
+    return {"workload": f"moe_block_e{E}_top{k}_t{T}_h{H}_i{I}_route_experts_combine",
+            "block_ms": round(t_full, 4), "block_tflops": round(flops / (t_full * 1e-3) / 1e12, 1),
+            "route_ms": round(t_route, 4), "combine_ms": round(t_comb, 4),
+            "combine_gbs": round(gbs(comb_bytes, t_comb), 1),
+            "combine_frac_hbm": round(gbs(comb_bytes, t_comb) / HBM_PEAK, 4)}
+
+
+COMPONENTS = {"moe_full": comp_moe_full, "dense_mlp": comp_dense_mlp, "decode_moe": comp_decode_moe, "kv_cache": comp_kv,
               "act_quant_sweep": comp_act_sweep, "remap": comp_remap}
 
 

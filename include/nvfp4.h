@@ -64,7 +64,8 @@ typedef enum {
     /* data-dependent errors, written to *dev_status by the kernels */
     NVFP4_ERR_NONFINITE = 16,        /* an input element (or amax) is NaN or inf */
     NVFP4_ERR_NOT_REPRESENTABLE = 17,/* MXFP4 exponent byte 0xFF or spread > 17 */
-    NVFP4_ERR_TIMEOUT = 18           /* a bounded wait inside a kernel gave up */
+    NVFP4_ERR_TIMEOUT = 18,          /* a bounded wait inside a kernel gave up */
+    NVFP4_ERR_INDEX = 19             /* an index input (expert id) is out of range */
 } nvfp4_status;
 
 typedef enum { NVFP4_SF_ROWMAJOR = 0, NVFP4_SF_MMA_TILED = 1 } nvfp4_sf_layout;
@@ -213,6 +214,42 @@ nvfp4_status nvfp4_kv_dequantize(const uint8_t *k_q, const uint8_t *k_sf, const 
                                  const uint8_t *v_q, const uint8_t *v_sf, const float *v_gs,
                                  int64_t tokens, int64_t heads, int64_t head_dim,
                                  void *k_out, void *v_out, cudaStream_t stream);
+
+/*
+ * nvfp4_moe_route -- routed (token, choice) pairs -> expert-grouped row order.
+ * [P1 results section: each token goes to its top-10 of 512 routed experts;
+ *  the grouped GEMM consumes the routed rows of one expert contiguously.]
+ *   topk_ids        int32 [tokens, topk] expert ids (the router's choices;
+ *                   a token lists an expert at most once).
+ *   expert_offsets  int32 [num_experts+1] out: prefix sums of the per-expert
+ *                   row counts (the `group_offsets` / `expert_offsets` of the
+ *                   calls above).
+ *   row_index       int32 [tokens*topk] out: token id of every routed row;
+ *                   rows of an expert are in ascending token id.
+ *   slot            int32 [tokens, topk] out: routed row of each choice
+ *                   (-1 for an out-of-range id).
+ *   workspace       >= nvfp4_moe_route_workspace_size(tokens, num_experts).
+ *   num_experts <= 2048, topk <= 32.  Deterministic (no order-dependent
+ *   atomics decide any output).  dev_status: NVFP4_ERR_INDEX for an id
+ *   outside [0, num_experts) (that pair is dropped).
+ */
+size_t nvfp4_moe_route_workspace_size(int64_t tokens, int num_experts);
+nvfp4_status nvfp4_moe_route(const int32_t *topk_ids, int64_t tokens, int topk, int num_experts,
+                             int32_t *expert_offsets, int32_t *row_index, int32_t *slot,
+                             void *workspace, int32_t *dev_status, cudaStream_t stream);
+
+/*
+ * nvfp4_moe_combine -- out[t, :] = sum_j weights[t, j] * y[slot[t, j], :],
+ * accumulated in fp32 in choice order (the weighted sum of a token's expert
+ * outputs after the down projection).
+ *   y        fp32 or bf16 [routed rows, H] (the down GEMM output); H % 8 == 0.
+ *   slot     int32 [tokens, topk] from nvfp4_moe_route (-1 entries skipped).
+ *   weights  fp32 [tokens, topk] routing weights.
+ *   out      fp32 or bf16 [tokens, H].
+ */
+nvfp4_status nvfp4_moe_combine(const void *y, nvfp4_out_dtype y_dtype, const int32_t *slot,
+                               const float *weights, int64_t tokens, int topk, int64_t H, void *out,
+                               nvfp4_out_dtype out_dtype, cudaStream_t stream);
 
 /*
  * nvfp4_quantize_noalloc -- nvfp4_quantize without a caller workspace.

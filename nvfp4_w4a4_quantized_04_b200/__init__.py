@@ -27,6 +27,7 @@ ERR_CUDA = 3
 ERR_NONFINITE = 16
 ERR_NOT_REPRESENTABLE = 17
 ERR_TIMEOUT = 18
+ERR_INDEX = 19
 
 SF_ROWMAJOR = 0
 SF_MMA_TILED = 1
@@ -40,6 +41,7 @@ EXPORTS = [
     "nvfp4_status_string", "nvfp4_workspace_size", "nvfp4_padded_rows_bound",
     "nvfp4_quantize", "nvfp4_dequantize", "mxfp4_to_nvfp4", "nvfp4_grouped_gemm",
     "nvfp4_swiglu_quantize", "nvfp4_kv_quantize", "nvfp4_kv_dequantize", "nvfp4_quantize_noalloc",
+    "nvfp4_moe_route_workspace_size", "nvfp4_moe_route", "nvfp4_moe_combine",
 ]
 NOALLOC_MAX_GROUPS = 1024
 
@@ -79,6 +81,12 @@ def load_library(path: str = LIB_PATH):
     L.nvfp4_kv_quantize.argtypes = [P, P, i64, i64, i64, i32, P, P, P, P, P, P, P, P, P]
     L.nvfp4_quantize_noalloc.restype = i32
     L.nvfp4_quantize_noalloc.argtypes = [P, i64, i64, i64, P, P, i32, i32, P, P, P, i32, P, P]
+    L.nvfp4_moe_route_workspace_size.restype = ctypes.c_size_t
+    L.nvfp4_moe_route_workspace_size.argtypes = [i64, i32]
+    L.nvfp4_moe_route.restype = i32
+    L.nvfp4_moe_route.argtypes = [P, i64, i32, i32, P, P, P, P, P, P]
+    L.nvfp4_moe_combine.restype = i32
+    L.nvfp4_moe_combine.argtypes = [P, i32, P, P, i64, i32, i64, P, i32, P]
     L.nvfp4_kv_dequantize.restype = i32
     L.nvfp4_kv_dequantize.argtypes = [P, P, P, P, P, P, i64, i64, i64, P, P, P]
     _lib = L
@@ -192,4 +200,26 @@ def nvfp4_kv_dequantize(k_q, k_sf, k_gs, v_q, v_sf, v_gs, tokens, heads, head_di
         _ptr(k_out), _ptr(v_out), _stream(stream))
     if check:
         _check(st, "nvfp4_kv_dequantize")
+    return st
+
+
+def nvfp4_moe_route_workspace_size(tokens: int, num_experts: int) -> int:
+    return int(load_library().nvfp4_moe_route_workspace_size(tokens, num_experts))
+
+
+def nvfp4_moe_route(topk_ids, tokens, topk, num_experts, expert_offsets, row_index, slot, workspace,
+                    dev_status=None, stream=None, check=True) -> int:
+    st = load_library().nvfp4_moe_route(
+        _ptr(topk_ids), tokens, topk, num_experts, _ptr(expert_offsets), _ptr(row_index), _ptr(slot),
+        _ptr(workspace), _ptr(dev_status), _stream(stream))
+    if check:
+        _check(st, "nvfp4_moe_route")
+    return st
+
+
+def nvfp4_moe_combine(y, y_dtype, slot, weights, tokens, topk, H, out, out_dtype, stream=None, check=True) -> int:
+    st = load_library().nvfp4_moe_combine(
+        _ptr(y), y_dtype, _ptr(slot), _ptr(weights), tokens, topk, H, _ptr(out), out_dtype, _stream(stream))
+    if check:
+        _check(st, "nvfp4_moe_combine")
     return st

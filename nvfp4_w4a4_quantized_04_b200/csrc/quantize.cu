@@ -619,6 +619,7 @@ const char *nvfp4_status_string(int status) {
     case NVFP4_ERR_NONFINITE: return "non-finite input";
     case NVFP4_ERR_NOT_REPRESENTABLE: return "not representable";
     case NVFP4_ERR_TIMEOUT: return "bounded wait timed out";
+    case NVFP4_ERR_INDEX: return "index out of range";
     default: return "unknown status";
   }
 }

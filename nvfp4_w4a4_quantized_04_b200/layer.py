@@ -14,8 +14,9 @@ from typing import Optional
 import torch
 
 from . import (EPI_NONE, GS_FROM_AMAX, GS_GIVEN, OUT_BF16, OUT_F32, SF_MMA_TILED, SF_ROWMAJOR,
-               mxfp4_to_nvfp4, nvfp4_dequantize, nvfp4_grouped_gemm, nvfp4_padded_rows_bound,
-               nvfp4_quantize, nvfp4_swiglu_quantize, nvfp4_workspace_size)
+               mxfp4_to_nvfp4, nvfp4_dequantize, nvfp4_grouped_gemm, nvfp4_moe_combine, nvfp4_moe_route,
+               nvfp4_moe_route_workspace_size, nvfp4_padded_rows_bound, nvfp4_quantize, nvfp4_swiglu_quantize,
+               nvfp4_workspace_size)
 
 
 @dataclass
@@ -158,3 +159,57 @@ class MoEExperts:
         y2 = self.y2[:R]
         grouped_gemm(a2, self.w_down, H, self.out_dtype, y=y2, dev_status=dev_status)
         return y2
+
+
+def route(topk_ids: torch.Tensor, num_experts: int, dev_status=None):
+    """Expert-grouped order of routed rows: (offsets [E+1], row_index [T*k], slot [T, k])."""
+    T, k = topk_ids.shape
+    dev = topk_ids.device
+    off = torch.empty(num_experts + 1, dtype=torch.int32, device=dev)
+    ri = torch.empty(T * k, dtype=torch.int32, device=dev)
+    slot = torch.empty((T, k), dtype=torch.int32, device=dev)
+    ws = torch.empty(nvfp4_moe_route_workspace_size(T, num_experts), dtype=torch.uint8, device=dev)
+    nvfp4_moe_route(topk_ids, T, k, num_experts, off, ri, slot, ws, dev_status)
+    return off, ri, slot
+
+
+def combine(y: torch.Tensor, slot: torch.Tensor, weights: torch.Tensor, out_dtype=OUT_BF16, out=None):
+    """out[t] = sum_j weights[t, j] * y[slot[t, j]] (fp32 accumulation)."""
+    T, k = slot.shape
+    H = y.shape[1]
+    dt = torch.float32 if out_dtype == OUT_F32 else torch.bfloat16
+    if out is None:
+        out = torch.empty((T, H), dtype=dt, device=y.device)
+    ydt = OUT_F32 if y.dtype == torch.float32 else OUT_BF16
+    nvfp4_moe_combine(y, ydt, slot, weights, T, k, H, out, out_dtype)
+    return out
+
+
+class MoELayer:
+    """A whole routed-expert MoE block on one GPU: routing order, the NVFP4
+    W4A4 experts, and the weighted combine back to [T, H].
+
+    forward(x bf16 [T, H], topk_ids int32 [T, k], topk_weights fp32 [T, k]) -> bf16 [T, H].
+    The router itself (BF16 gate, top-k) stays outside, as on the pages.
+    """
+
+    def __init__(self, experts: MoEExperts, max_tokens: int, topk: int, device="cuda"):
+        self.experts = experts
+        E = experts.E
+        self.off = torch.empty(E + 1, dtype=torch.int32, device=device)
+        self.ri = torch.empty(max_tokens * topk, dtype=torch.int32, device=device)
+        self.slot = torch.empty((max_tokens, topk), dtype=torch.int32, device=device)
+        self.rws = torch.empty(nvfp4_moe_route_workspace_size(max_tokens, E), dtype=torch.uint8, device=device)
+        self.out = torch.empty((max_tokens, experts.H), dtype=torch.bfloat16, device=device)
+
+    def forward(self, x: torch.Tensor, topk_ids: torch.Tensor, topk_weights: torch.Tensor, dev_status=None):
+        T, k = topk_ids.shape
+        E = self.experts.E
+        slot = self.slot[:T]
+        ri = self.ri[:T * k]
+        nvfp4_moe_route(topk_ids, T, k, E, self.off, ri, slot, self.rws, dev_status)
+        y = self.experts.forward(x, ri, self.off, dev_status)
+        out = self.out[:T]
+        nvfp4_moe_combine(y, OUT_F32 if y.dtype == torch.float32 else OUT_BF16, slot, topk_weights, T, k,
+                          self.experts.H, out, OUT_BF16)
+        return out

@@ -89,6 +89,10 @@ def lib():
             L.orc_swiglu.argtypes = [P, i64, i64, P]
             L.orc_dot_f64.restype = None
             L.orc_dot_f64.argtypes = [P, P, i64, P, P]
+            L.orc_route.restype = ctypes.c_int
+            L.orc_route.argtypes = [P, i64, ctypes.c_int, ctypes.c_int, P, P, P]
+            L.orc_combine.restype = None
+            L.orc_combine.argtypes = [P, P, P, i64, ctypes.c_int, i64, P, P]
             for name in ("orc_e2m1_encode_array", "orc_e4m3_encode_array"):
                 getattr(L, name).restype = None
                 getattr(L, name).argtypes = [P, i64, P]
@@ -312,3 +316,31 @@ def dot_f64(a: np.ndarray, b: np.ndarray):
     s = ctypes.c_double()
     lib().orc_dot_f64(_p(a), _p(b), a.size, ctypes.byref(y), ctypes.byref(s))
     return y.value, s.value
+
+
+# ---------------------------------------------------------------- MoE plumbing
+def route(expert_ids: np.ndarray, num_experts: int):
+    """Group (token, choice) pairs by expert, tokens ascending inside a group
+    (the routed-row order the grouped GEMM consumes; P1: top-10 routing).
+    expert_ids: int32 [T, k].  Returns (offsets [E+1], row_index [T*k], slot [T, k], status)."""
+    ids = np.ascontiguousarray(expert_ids, dtype=np.int32)
+    T, k = ids.shape
+    off = np.empty(num_experts + 1, np.int32)
+    ri = np.empty(T * k, np.int32)
+    slot = np.empty((T, k), np.int32)
+    st = lib().orc_route(_p(ids), T, k, num_experts, _p(off), _p(ri), _p(slot))
+    return off, ri, slot, st
+
+
+def combine(y: np.ndarray, slot: np.ndarray, weights: np.ndarray):
+    """out[t] = sum_j w[t,j] * y[slot[t,j]] in fp64, and sum |w*y| (the weighted
+    sum of the k expert outputs of each token)."""
+    y = np.ascontiguousarray(y, dtype=np.float32)
+    slot = np.ascontiguousarray(slot, dtype=np.int32)
+    w = np.ascontiguousarray(weights, dtype=np.float32)
+    T, k = slot.shape
+    H = y.shape[1]
+    out = np.empty((T, H), np.float64)
+    sabs = np.empty((T, H), np.float64)
+    lib().orc_combine(_p(y), _p(slot), _p(w), T, k, H, _p(out), _p(sabs))
+    return out, sabs

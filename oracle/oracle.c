@@ -38,6 +38,7 @@
 #include <stdint.h>
 #include <stddef.h>
 #include <string.h>
+#include <stdlib.h>
 
 #define ORC_OK 0
 #define ORC_ERR_NONFINITE 16
@@ -409,4 +410,57 @@ void orc_e4m3_encode_bits_range(uint64_t lo, uint64_t hi, uint8_t *out) {
         memcpy(&f, &u, 4);
         out[i] = orc_e4m3_encode(f);
     }
+}
+
+/* ------------------------------------------------------------------ */
+/* MoE routing structure and combine (the steps on either side of the  */
+/* expert GEMMs; P1 results section: top-10 of 512 routed experts)     */
+/* ------------------------------------------------------------------ */
+
+/*
+ * Group routed (token, choice) pairs by expert: expert e's rows are the
+ * tokens that chose e, in ascending token id; offsets[E+1] are the prefix
+ * sums of the counts; slot[t*k + j] is the routed row of token t's j-th
+ * choice.  A plain counting sort in token order.  Returns 0, or 1 when an
+ * expert id is out of range.
+ */
+int orc_route(const int32_t *ids, int64_t T, int k, int E, int32_t *offsets, int32_t *row_index,
+              int32_t *slot) {
+    if (E <= 0 || k <= 0 || T < 0) return 1;
+    for (int e = 0; e <= E; ++e) offsets[e] = 0;
+    for (int64_t i = 0; i < T * k; ++i) {
+        if (ids[i] < 0 || ids[i] >= E) return 1;
+        offsets[ids[i] + 1] += 1;
+    }
+    for (int e = 0; e < E; ++e) offsets[e + 1] += offsets[e];
+    int32_t *fill = (int32_t *)malloc(sizeof(int32_t) * (size_t)(unsigned)E);
+    if (!fill) return 1;
+    for (int e = 0; e < E; ++e) fill[e] = offsets[e];
+    for (int64_t t = 0; t < T; ++t)
+        for (int j = 0; j < k; ++j) {
+            int e = ids[t * k + j];
+            int32_t r = fill[e]++;
+            row_index[r] = (int32_t)t;
+            slot[t * k + j] = r;
+        }
+    free(fill);
+    return 0;
+}
+
+/* out[t, :] = sum_j w[t, j] * y[slot[t, j], :], accumulated in fp64 in
+ * choice order; also |w*y| summed for the tolerance.  y is fp32. */
+void orc_combine(const float *y, const int32_t *slot, const float *w, int64_t T, int k, int64_t H,
+                 double *out, double *sabs) {
+    #pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t)
+        for (int64_t c = 0; c < H; ++c) {
+            double s = 0.0, a = 0.0;
+            for (int j = 0; j < k; ++j) {
+                double p = (double)w[t * k + j] * (double)y[(int64_t)slot[t * k + j] * H + c];
+                s += p;
+                a += fabs(p);
+            }
+            out[t * H + c] = s;
+            sabs[t * H + c] = a;
+        }
 }

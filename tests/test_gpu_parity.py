@@ -536,6 +536,83 @@ def test_moe_layer_small_stagewise():
     assert ok.all(), (err / bound).max()
 
 
+# --------------------------------------------------------------------------- routing / combine
+@pytest.mark.parametrize("T,E,k", [(1000, 64, 8), (8192, 512, 10), (3, 2048, 2), (257, 5, 5)])
+def test_route_bitexact(T, E, k):
+    L = layer()
+    if (T, E, k) == (8192, 512, 10):
+        ids = synthetic.route_topk_softmax(0, T, E, k)["experts"].astype(np.int32)
+    else:
+        rng = np.random.default_rng(T)
+        ids = np.stack([rng.choice(E, size=k, replace=False) for _ in range(T)]).astype(np.int32)
+    off_ref, ri_ref, slot_ref, st = oracle.route(ids, E)
+    s = status_word()
+    off, ri, slot = L.route(to_dev(ids), E, dev_status=s)
+    torch.cuda.synchronize()
+    assert int(s.item()) == 0
+    assert np.array_equal(to_np(off), off_ref)
+    assert np.array_equal(to_np(ri), ri_ref)
+    assert np.array_equal(to_np(slot), slot_ref)
+
+
+def test_route_bad_index_status():
+    L = layer()
+    ids = np.array([[0, 1], [2, 9], [1, 3]], dtype=np.int32)
+    s = status_word()
+    off, ri, slot = L.route(to_dev(ids), 4, dev_status=s)
+    torch.cuda.synchronize()
+    assert int(s.item()) == 19
+    assert to_np(slot)[1, 1] == -1 and to_np(off)[-1] == 5
+
+
+@pytest.mark.parametrize("ydt", [0, 1])
+def test_combine(ydt):
+    L = layer()
+    T, E, k, H = 300, 16, 4, 512
+    rng = np.random.default_rng(5)
+    ids = np.stack([rng.choice(E, size=k, replace=False) for _ in range(T)]).astype(np.int32)
+    off, ri, slot, _ = oracle.route(ids, E)
+    w = rng.random((T, k)).astype(np.float32)
+    w /= w.sum(1, keepdims=True)
+    yb = synthetic.gaussian_bf16(5, synthetic.STREAMS["x"], (T * k, H))
+    yf = synthetic.bf16_bits_to_f32(yb)
+    yd = bf16_dev(yb) if ydt == 1 else to_dev(yf)
+    out32 = to_np(L.combine(yd, to_dev(slot), to_dev(w), out_dtype=0))
+    out16 = to_np(L.combine(yd, to_dev(slot), to_dev(w), out_dtype=1))
+    torch.cuda.synchronize()
+    ref, sabs = oracle.combine(yf, slot, w)
+    assert (np.abs(out32 - ref) <= 1e-6 * sabs + 1e-30).all()
+    assert np.array_equal(out16, synthetic.f32_to_bf16_bits(out32))
+
+
+def test_moe_layer_full_small():
+    """route -> experts -> combine; the combine stage checked on the device's y."""
+    L = layer()
+    T, H, I, E, k = 64, 256, 256, 8, 3
+    r = synthetic.route_topk_softmax(6, T, E, k)
+    x = synthetic.gaussian_bf16(6, synthetic.STREAMS["x"], (T, H))
+    wgu = synthetic.gaussian_bf16(6, synthetic.STREAMS["w_gate_up"], (E * 2 * I, H), sigma=0.02)
+    wd = synthetic.gaussian_bf16(6, synthetic.STREAMS["w_down"], (E * H, I), sigma=0.02)
+    qg, sg, gg = _packed_weights(wgu, E, 2 * I, H)
+    qd, sd, gd = _packed_weights(wd, E, H, I)
+    Wgu = L.Packed(to_dev(qg), to_dev(tile(sg)), to_dev(gg), E * 2 * I, H, 1)
+    Wd = L.Packed(to_dev(qd), to_dev(tile(sd)), to_dev(gd), E * H, I, 1)
+    experts = L.MoEExperts(Wgu, Wd, E, H, I, max_rows=T * k, out_dtype=1, mid_dtype=1)
+    moe = L.MoELayer(experts, T, k)
+    s = status_word()
+    out = moe.forward(bf16_dev(x), to_dev(r["experts"].astype(np.int32)),
+                      to_dev(r["weights"].astype(np.float32)), dev_status=s)
+    torch.cuda.synchronize()
+    assert int(s.item()) == 0
+    off_ref, ri_ref, slot_ref, _ = oracle.route(r["experts"].astype(np.int32), E)
+    assert np.array_equal(to_np(moe.ri[:T * k]), ri_ref) and np.array_equal(to_np(moe.off), off_ref)
+    y2 = synthetic.bf16_bits_to_f32(to_np(experts.y2[:T * k]))
+    ref, sabs = oracle.combine(y2, slot_ref, r["weights"].astype(np.float32))
+    got = synthetic.bf16_bits_to_f32(to_np(out)).astype(np.float64)
+    # bf16 output: within one bf16 rounding of the fp32 result
+    assert (np.abs(got - ref) <= 1e-6 * sabs + np.abs(ref) * 2.0 ** -8 + 1e-30).all()
+
+
 def test_device_generator_matches_host():
     import synthetic.cuda as sc
     g = sc.gaussian_bf16(3, 5, (1000, 64), sigma=0.02, start=12345)

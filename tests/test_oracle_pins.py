@@ -441,3 +441,45 @@ def test_kv_cache_size_facts():
     bf16 = n * 2
     nvfp4 = n * FACTS["effective_bits"] / 8
     assert abs(nvfp4 / bf16 - FACTS["kv_nvfp4_over_bf16_approx"]) < 0.04
+
+
+# ------------------------------------------------------------------ routing / combine
+def test_route_matches_library_sort_and_invariants():
+    """Grouping by expert equals a stable lexicographic sort on (expert, token)
+    done by numpy, and every (token, choice) lands in its expert's rows."""
+    rng = np.random.default_rng(0)
+    T, E, k = 300, 37, 4
+    ids = np.stack([rng.choice(E, size=k, replace=False) for _ in range(T)]).astype(np.int32)
+    off, ri, slot, st = oracle.route(ids, E)
+    assert st == 0
+    flat_e = ids.reshape(-1)
+    flat_t = np.repeat(np.arange(T), k)
+    order = np.lexsort((flat_t, flat_e))
+    assert np.array_equal(ri, flat_t[order])
+    assert np.array_equal(off, np.concatenate([[0], np.cumsum(np.bincount(flat_e, minlength=E))]))
+    for t in range(T):
+        for j in range(k):
+            r = slot[t, j]
+            e = ids[t, j]
+            assert off[e] <= r < off[e + 1] and ri[r] == t
+    assert sorted(slot.reshape(-1).tolist()) == list(range(T * k))
+    bad = ids.copy()
+    bad[3, 1] = E
+    assert oracle.route(bad, E)[3] == 1
+
+
+def test_combine_closed_forms():
+    rng = np.random.default_rng(1)
+    T, k, H = 5, 3, 16
+    y = rng.standard_normal((T * k, H)).astype(np.float32)
+    slot = np.arange(T * k, dtype=np.int32).reshape(T, k)
+    onehot = np.zeros((T, k), np.float32)
+    onehot[:, 1] = 1.0
+    out, s = oracle.combine(y, slot, onehot)
+    assert np.array_equal(out, y[slot[:, 1]].astype(np.float64))
+    w = np.full((T, k), 0.25, np.float32)
+    out, s = oracle.combine(y, slot, w)
+    for t in range(T):
+        want = sum(0.25 * y[slot[t, j]].astype(np.float64) for j in range(k))
+        assert np.allclose(out[t], want, rtol=0, atol=1e-12)
+        assert np.allclose(s[t], sum(np.abs(0.25 * y[slot[t, j]].astype(np.float64)) for j in range(k)))
