@@ -148,7 +148,7 @@ def pack_weights(w_bf16, E, rows_per, ws):
 
 
 # --------------------------------------------------------------------------- headline: MoE layer
-def setup_moe(device, seed, E, T, H, I, topk):
+def setup_moe(device, seed, E, T, H, I, topk, fused=True):
     import torch
 
     import synthetic
@@ -165,7 +165,8 @@ def setup_moe(device, seed, E, T, H, I, topk):
         del w
     torch.cuda.synchronize()
     x = sc.gaussian_bf16(seed, synthetic.STREAMS["x"], (T, H))
-    moe = L.MoEExperts(packs[0], packs[1], E, H, I, max_rows=R, out_dtype=1, mid_dtype=1, device=device)
+    moe = L.MoEExperts(packs[0], packs[1], E, H, I, max_rows=R, out_dtype=1, mid_dtype=1, device=device,
+                       fused_swiglu=fused)
     ri = torch.from_numpy(r["row_index"]).to(device)
     off = torch.from_numpy(r["offsets"]).to(device)
     return moe, x, ri, off, r, R
@@ -177,20 +178,30 @@ def run_headline(args, rank, world, device):
     from nvfp4_w4a4_quantized_04_b200 import layer as L
 
     E, T, H, I, k = args.experts, args.tokens, 4096, 1024, 10
-    moe, x, ri, off, r, R = setup_moe(device, rank, E, T, H, I, k)
+    fused = not args.unfused
+    moe, x, ri, off, r, R = setup_moe(device, rank, E, T, H, I, k, fused=fused)
     flops = moe_flops(R, H, I)
     e_touched = int((np.diff(r["offsets"]) > 0).sum())
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream()
+
+    from nvfp4_w4a4_quantized_04_b200 import GS_AMAX_GIVEN, nvfp4_quantize
 
     def stages(evs=None):
         rec = (lambda i: evs[i].record(stream)) if evs else (lambda i: None)
         rec(0)
         a1 = L.quantize(x, ri, off, E, layout=1, out=moe.a1, ws=moe.ws, rows=R)
         rec(1)
-        L.grouped_gemm(a1, moe.w_gate_up, 2 * I, moe.mid_dtype, y=moe.y1[:R])
-        rec(2)
-        a2, _ = L.swiglu_quantize(moe.y1[:R], off, E, layout=1, out=moe.a2, h=moe.h[:R], ws=moe.ws)
+        if fused:
+            h, amax = L.grouped_gemm_swiglu(a1, moe.w_gate_up, 2 * I, h=moe.h[:R], amax=moe.amax)
+            rec(2)
+            a2 = moe.a2
+            a2.offsets, a2.num_groups, a2.rows, a2.gs = off, E, R, amax
+            nvfp4_quantize(h, R, I, I, None, off, E, GS_AMAX_GIVEN, amax, a2.q, a2.sf, 1, moe.ws)
+        else:
+            L.grouped_gemm(a1, moe.w_gate_up, 2 * I, moe.mid_dtype, y=moe.y1[:R])
+            rec(2)
+            a2, _ = L.swiglu_quantize(moe.y1[:R], off, E, layout=1, out=moe.a2, h=moe.h[:R], ws=moe.ws)
         rec(3)
         L.grouped_gemm(a2, moe.w_down, H, moe.out_dtype, y=moe.y2[:R])
         rec(4)
@@ -248,10 +259,13 @@ def run_headline(args, rank, world, device):
     med = np.median(per, axis=0)
     g1_ms, g2_ms = float(np.mean(per[:, 1])), float(np.mean(per[:, 3]))
     g1_bytes = gemm_bytes(R, e_touched, 2 * I, H)
+    if fused:
+        g1_bytes += R * I * 2 - R * 2 * I * 2          # the fused launch writes h [R, I], not [R, 2I]
     g1_flops = 2.0 * R * 2 * I * H
     g2_bytes = gemm_bytes(R, e_touched, H, I)
     g2_flops = 2.0 * R * H * I
-    roof = {"bound": "hbm", "kernel": "nvfp4::gemm::grouped_gemm_kernel (gate_up launch)",
+    roof = {"bound": "hbm", "kernel": ("nvfp4::gemm::grouped_gemm_kernel<swiglu> (gate_up + SwiGLU epilogue launch)"
+                                       if fused else "nvfp4::gemm::grouped_gemm_kernel (gate_up launch)"),
             "achieved": round(gbs(g1_bytes, g1_ms), 1), "peak": HBM_PEAK, "unit": "GB/s",
             "frac": round(gbs(g1_bytes, g1_ms) / HBM_PEAK, 4), "traffic": None,
             "peak_source": f"{PEAKS_KIND} hbm_gbs (burst copy)",
@@ -261,9 +275,10 @@ def run_headline(args, rank, world, device):
             "fp4_peak_tflops": round(FP4_PEAK, 1),
             "fp4_peak_source": f"{PEAKS_KIND} bf16_tflops x 4 (nominal fp4/bf16 ratio)"}
     breakdown = {
+        "pipeline": "gate_up GEMM with SwiGLU epilogue" if fused else "gate_up GEMM, then SwiGLU + requantize",
         "gather_quantize_ms": round(float(med[0]), 4),
-        "gate_up_gemm_ms": round(float(med[1]), 4),
-        "swiglu_requantize_ms": round(float(med[2]), 4),
+        ("gate_up_swiglu_gemm_ms" if fused else "gate_up_gemm_ms"): round(float(med[1]), 4),
+        ("requantize_ms" if fused else "swiglu_requantize_ms"): round(float(med[2]), 4),
         "down_gemm_ms": round(float(med[3]), 4),
         "gate_up_gbs": round(gbs(g1_bytes, g1_ms), 1), "gate_up_tflops": round(g1_flops / (g1_ms * 1e-3) / 1e12, 1),
         "down_gbs": round(gbs(g2_bytes, g2_ms), 1), "down_tflops": round(g2_flops / (g2_ms * 1e-3) / 1e12, 1),
@@ -284,7 +299,7 @@ def run_headline(args, rank, world, device):
         "breakdown": breakdown,
         "e2e": {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": round(e2e_ms, 3)},
-        "gpu_launches": 8 * args.steps,
+        "gpu_launches": (7 if fused else 8) * args.steps,
         "clocks": clk,
     }
 
@@ -370,7 +385,8 @@ def comp_decode_moe(device, iters, warmup, flush):
         packs.append(L.Packed(qn, sf, gs, E * rows_per, K, 1))
         del q, e8
     xb = sc.gaussian_bf16(7, synthetic.STREAMS["x"], (T, H))
-    moe = L.MoEExperts(packs[0], packs[1], E, H, I, max_rows=R, out_dtype=1, mid_dtype=1, device=device)
+    moe = L.MoEExperts(packs[0], packs[1], E, H, I, max_rows=R, out_dtype=1, mid_dtype=1, device=device,
+                       fused_swiglu=True)
     ri = torch.from_numpy(r["row_index"]).to(device)
     off = torch.from_numpy(r["offsets"]).to(device)
     ms = timed(lambda: moe.forward(xb, ri, off), iters, warmup, flush)
@@ -575,6 +591,8 @@ def main():
     ap.add_argument("--tokens", type=int, default=8192)
     ap.add_argument("--components", default="auto")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--unfused", action="store_true",
+                    help="run SwiGLU + requantize as separate kernels instead of the GEMM epilogue")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))

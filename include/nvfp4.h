@@ -69,9 +69,20 @@ typedef enum {
 } nvfp4_status;
 
 typedef enum { NVFP4_SF_ROWMAJOR = 0, NVFP4_SF_MMA_TILED = 1 } nvfp4_sf_layout;
-typedef enum { NVFP4_GS_FROM_AMAX = 0, NVFP4_GS_GIVEN = 1 } nvfp4_gs_mode;
+/* FROM_AMAX: s_g from the amax of the input (an extra read pass).
+ * GIVEN: s_g supplied (calibrated input scale, static KV scale).
+ * AMAX_GIVEN: global_scale holds the group amax on entry (e.g. produced by
+ *   the SwiGLU GEMM epilogue); it is replaced by s_g = amax/2688 (1 if 0). */
+typedef enum { NVFP4_GS_FROM_AMAX = 0, NVFP4_GS_GIVEN = 1, NVFP4_GS_AMAX_GIVEN = 2 } nvfp4_gs_mode;
 typedef enum { NVFP4_OUT_F32 = 0, NVFP4_OUT_BF16 = 1 } nvfp4_out_dtype;
-typedef enum { NVFP4_EPI_NONE = 0 } nvfp4_epilogue;
+/* NONE: y = alpha * A B^T.  SWIGLU: the weight is a fused gate_up [2I, K]
+ * (gate rows first); the epilogue writes h = bf16(silu(g) * u) with
+ * g = alpha*acc_gate, u = alpha*acc_up kept in fp32 (no bf16 rounding of the
+ * gate_up output in between; silu through the fast exp/divide intrinsics),
+ * y is bf16 [M_total, N/2], and amax_out[e]
+ * receives max |h| of expert e (fp32 bit pattern via integer max: the
+ * caller zeroes it). */
+typedef enum { NVFP4_EPI_NONE = 0, NVFP4_EPI_SWIGLU = 1 } nvfp4_epilogue;
 
 /* Human-readable name of a status code (static string). */
 const char *nvfp4_status_string(int status);
@@ -104,6 +115,8 @@ int64_t nvfp4_padded_rows_bound(int64_t rows, int num_groups);
  *               s_g = amax/2688 (2688 = 6*448: the block holding the amax gets
  *               scale 448), or 1 for an all-zero group.  GIVEN: read (a
  *               calibrated input scale or a static KV scale), must be > 0.
+ *               AMAX_GIVEN: holds the group amax on entry, replaced by s_g as
+ *               in FROM_AMAX (no amax pass over x).
  *   q           uint8 [packed rows, K/2]; sf uint8 scales in `sf_layout`.
  *   workspace   >= nvfp4_workspace_size(num_groups) bytes.
  *   dev_status  nullable int32: NVFP4_ERR_NONFINITE when an input element of a
@@ -167,7 +180,9 @@ nvfp4_status mxfp4_to_nvfp4(const uint8_t *q_mx, const uint8_t *ue8m0, int64_t n
  *               (offsets[E] == M_total).  NULL means one dense GEMM (E = 1).
  *   M_total, N, K   Y is [M_total, N]; N % 128 == 0, K % 256 == 0.
  *   y, out_dtype    fp32 or bf16 [M_total, N], rows in routed (unpadded) order.
- *   epi             NVFP4_EPI_NONE.
+ *   epi, amax_out   NVFP4_EPI_NONE (amax_out unused), or NVFP4_EPI_SWIGLU: y is
+ *                   bf16 h [M_total, N/2] (out_dtype must be BF16), amax_out
+ *                   fp32 [E] zeroed by the caller, N/2 % 64 == 0.
  *   workspace   >= nvfp4_workspace_size(E); dev_status: NVFP4_ERR_TIMEOUT if a
  *               pipeline wait gave up (the output is then incomplete).
  */
@@ -175,7 +190,7 @@ nvfp4_status nvfp4_grouped_gemm(const uint8_t *a_q, const uint8_t *a_sf, const f
                                 const uint8_t *b_q, const uint8_t *b_sf, const float *b_gs,
                                 const int32_t *expert_offsets, int num_experts,
                                 int64_t M_total, int64_t N, int64_t K, void *y,
-                                nvfp4_out_dtype out_dtype, nvfp4_epilogue epi,
+                                nvfp4_out_dtype out_dtype, nvfp4_epilogue epi, float *amax_out,
                                 void *workspace, int32_t *dev_status, cudaStream_t stream);
 
 /*

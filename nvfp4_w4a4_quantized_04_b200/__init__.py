@@ -36,6 +36,8 @@ GS_GIVEN = 1
 OUT_F32 = 0
 OUT_BF16 = 1
 EPI_NONE = 0
+EPI_SWIGLU = 1
+GS_AMAX_GIVEN = 2
 
 EXPORTS = [
     "nvfp4_status_string", "nvfp4_workspace_size", "nvfp4_padded_rows_bound",
@@ -74,7 +76,7 @@ def load_library(path: str = LIB_PATH):
     L.mxfp4_to_nvfp4.restype = i32
     L.mxfp4_to_nvfp4.argtypes = [P, P, i64, i64, i64, P, P, i32, P, P, P, P]
     L.nvfp4_grouped_gemm.restype = i32
-    L.nvfp4_grouped_gemm.argtypes = [P, P, P, P, P, P, P, i32, i64, i64, i64, P, i32, i32, P, P, P]
+    L.nvfp4_grouped_gemm.argtypes = [P, P, P, P, P, P, P, i32, i64, i64, i64, P, i32, i32, P, P, P, P]
     L.nvfp4_swiglu_quantize.restype = i32
     L.nvfp4_swiglu_quantize.argtypes = [P, i32, i64, i64, P, i32, P, P, P, i32, P, P, P, P]
     L.nvfp4_kv_quantize.restype = i32
@@ -164,10 +166,12 @@ def mxfp4_to_nvfp4(q_mx, ue8m0, n_tensors, rows, K, q_nv, sf_nv, sf_layout, glob
 
 
 def nvfp4_grouped_gemm(a_q, a_sf, a_gs, b_q, b_sf, b_gs, expert_offsets, num_experts, M_total, N, K, y,
-                       out_dtype, epi=EPI_NONE, workspace=None, dev_status=None, stream=None, check=True) -> int:
+                       out_dtype, epi=EPI_NONE, amax_out=None, workspace=None, dev_status=None, stream=None,
+                       check=True) -> int:
     st = load_library().nvfp4_grouped_gemm(
         _ptr(a_q), _ptr(a_sf), _ptr(a_gs), _ptr(b_q), _ptr(b_sf), _ptr(b_gs), _ptr(expert_offsets),
-        num_experts, M_total, N, K, _ptr(y), out_dtype, epi, _ptr(workspace), _ptr(dev_status), _stream(stream))
+        num_experts, M_total, N, K, _ptr(y), out_dtype, epi, _ptr(amax_out), _ptr(workspace), _ptr(dev_status),
+        _stream(stream))
     if check:
         _check(st, "nvfp4_grouped_gemm")
     return st

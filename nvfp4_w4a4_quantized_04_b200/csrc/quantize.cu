@@ -118,17 +118,18 @@ __global__ void __launch_bounds__(256) amax_flat_kernel(const uint4 *__restrict_
   }
 }
 
-// Global scales from the amax (FROM_AMAX) or a check of the given ones.
-__global__ void finalize_scales_kernel(const uint32_t *__restrict__ amax_bits, int G, int given,
+// Global scales from the amax (FROM_AMAX; AMAX_GIVEN reads the amax from gs
+// itself) or a check of the given ones (GIVEN).
+__global__ void finalize_scales_kernel(const uint32_t *__restrict__ amax_bits, int G, int mode,
                                        float *__restrict__ gs, int32_t *dev_status) {
   int g = blockIdx.x * blockDim.x + threadIdx.x;
   if (g >= G) return;
-  if (given) {
+  if (mode == NVFP4_GS_GIVEN) {
     float s = gs[g];
     if (!(s > 0.0f) || !isfinite(s)) report(dev_status, NVFP4_ERR_INVALID_ARG);
     return;
   }
-  uint32_t b = amax_bits[g];
+  uint32_t b = mode == NVFP4_GS_AMAX_GIVEN ? (__float_as_uint(gs[g]) & 0x7FFFFFFFu) : amax_bits[g];
   if (b >= 0x7F800000u) {
     gs[g] = __uint_as_float(0x7FC00000u);
     report(dev_status, NVFP4_ERR_NONFINITE);
@@ -553,8 +554,7 @@ nvfp4_status run_global_scales(const uint16_t *x, int64_t rows, int64_t K, int64
                                nvfp4_gs_mode gs_mode, float *global_scale, void *workspace,
                                int32_t *dev_status, cudaStream_t stream) {
   uint32_t *amax_bits = reinterpret_cast<uint32_t *>(workspace);
-  const int given = gs_mode == NVFP4_GS_GIVEN;
-  if (!given) {
+  if (gs_mode == NVFP4_GS_FROM_AMAX) {
     if (cudaMemsetAsync(amax_bits, 0, sizeof(uint32_t) * G, stream) != cudaSuccess) return NVFP4_ERR_CUDA;
     if (rows > 0) {
       if (!group_offsets && !row_index && ld_x == K) {
@@ -570,7 +570,7 @@ nvfp4_status run_global_scales(const uint16_t *x, int64_t rows, int64_t K, int64
       if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_CUDA;
     }
   }
-  finalize_scales_kernel<<<(G + 127) / 128, 128, 0, stream>>>(amax_bits, G, given, global_scale, dev_status);
+  finalize_scales_kernel<<<(G + 127) / 128, 128, 0, stream>>>(amax_bits, G, (int)gs_mode, global_scale, dev_status);
   return launch_status();
 }
 
@@ -646,7 +646,8 @@ nvfp4_status nvfp4_quantize(const void *x, int64_t rows, int64_t K, int64_t ld_x
   if (K % 16 != 0 || ld_x % 8 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   if (sf_layout != NVFP4_SF_ROWMAJOR && sf_layout != NVFP4_SF_MMA_TILED) return NVFP4_ERR_INVALID_ARG;
   if (sf_layout == NVFP4_SF_MMA_TILED && K % 64 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
-  if (gs_mode != NVFP4_GS_FROM_AMAX && gs_mode != NVFP4_GS_GIVEN) return NVFP4_ERR_INVALID_ARG;
+  if (gs_mode != NVFP4_GS_FROM_AMAX && gs_mode != NVFP4_GS_GIVEN && gs_mode != NVFP4_GS_AMAX_GIVEN)
+    return NVFP4_ERR_INVALID_ARG;
   const int G = group_offsets ? num_groups : 1;
   if (G < 1 || G > kMaxGroups) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   if (!global_scale || !workspace || !aligned16(workspace)) return NVFP4_ERR_INVALID_ARG;
@@ -710,7 +711,8 @@ nvfp4_status nvfp4_swiglu_quantize(const void *y, nvfp4_out_dtype y_dtype, int64
     }
     if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_CUDA;
   }
-  finalize_scales_kernel<<<(G + 127) / 128, 128, 0, stream>>>(amax_bits, G, 0, global_scale, dev_status);
+  finalize_scales_kernel<<<(G + 127) / 128, 128, 0, stream>>>(amax_bits, G, (int)NVFP4_GS_FROM_AMAX, global_scale,
+                                                              dev_status);
   if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_CUDA;
   return run_encode(reinterpret_cast<const uint16_t *>(h), rows, I, I, nullptr, group_offsets, G,
                     global_scale, q, sf, sf_layout, dev_status, stream);

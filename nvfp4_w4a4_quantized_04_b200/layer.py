@@ -13,7 +13,7 @@ from typing import Optional
 
 import torch
 
-from . import (EPI_NONE, GS_FROM_AMAX, GS_GIVEN, OUT_BF16, OUT_F32, SF_MMA_TILED, SF_ROWMAJOR,
+from . import (EPI_NONE, EPI_SWIGLU, GS_AMAX_GIVEN, GS_FROM_AMAX, GS_GIVEN, OUT_BF16, OUT_F32, SF_MMA_TILED, SF_ROWMAJOR,
                mxfp4_to_nvfp4, nvfp4_dequantize, nvfp4_grouped_gemm, nvfp4_moe_combine, nvfp4_moe_route,
                nvfp4_moe_route_workspace_size, nvfp4_padded_rows_bound, nvfp4_quantize, nvfp4_swiglu_quantize,
                nvfp4_workspace_size)
@@ -105,8 +105,25 @@ def grouped_gemm(a: Packed, w: Packed, N: int, out_dtype=OUT_BF16, y=None, dev_s
     if y is None:
         y = torch.empty((a.rows, N), dtype=dt, device=a.q.device)
     nvfp4_grouped_gemm(a.q, a.sf, a.gs, w.q, w.sf, w.gs, a.offsets, E, a.rows, N, a.K, y, out_dtype, EPI_NONE,
-                       None, dev_status)
+                       None, None, dev_status)
     return y
+
+
+def grouped_gemm_swiglu(a: Packed, w_gate_up: Packed, N: int, h=None, amax=None, dev_status=None):
+    """h [a.rows, N/2] = bf16(silu(g) * u) straight from the gate_up GEMM's
+    accumulators (g, u = the two halves of the fused weight), plus the
+    per-expert amax of h (fp32 [E])."""
+    assert a.layout == SF_MMA_TILED and w_gate_up.layout == SF_MMA_TILED
+    E = a.num_groups if a.offsets is not None else 1
+    if h is None:
+        h = torch.empty((a.rows, N // 2), dtype=torch.bfloat16, device=a.q.device)
+    if amax is None:
+        amax = torch.zeros(E, dtype=torch.float32, device=a.q.device)
+    else:
+        amax.zero_()
+    nvfp4_grouped_gemm(a.q, a.sf, a.gs, w_gate_up.q, w_gate_up.sf, w_gate_up.gs, a.offsets, E, a.rows, N, a.K, h,
+                       OUT_BF16, EPI_SWIGLU, amax, None, dev_status)
+    return h, amax
 
 
 def swiglu_quantize(y: torch.Tensor, offsets, num_groups: int, layout=SF_MMA_TILED, out: Optional[Packed] = None,
@@ -133,7 +150,9 @@ class MoEExperts:
     """
 
     def __init__(self, w_gate_up: Packed, w_down: Packed, E: int, H: int, I: int, max_rows: int,
-                 out_dtype=OUT_BF16, mid_dtype=OUT_BF16, device="cuda"):
+                 out_dtype=OUT_BF16, mid_dtype=OUT_BF16, device="cuda", fused_swiglu: bool = False):
+        self.fused_swiglu = fused_swiglu
+        self.amax = torch.zeros(E, dtype=torch.float32, device=device)
         self.w_gate_up, self.w_down = w_gate_up, w_down
         self.E, self.H, self.I = E, H, I
         self.out_dtype, self.mid_dtype = out_dtype, mid_dtype
@@ -152,10 +171,20 @@ class MoEExperts:
         assert R <= self.max_rows
         E, H, I = self.E, self.H, self.I
         a1 = quantize(x, row_index, offsets, E, SF_MMA_TILED, out=self.a1, ws=self.ws, dev_status=dev_status, rows=R)
-        y1 = self.y1[:R]
-        grouped_gemm(a1, self.w_gate_up, 2 * I, self.mid_dtype, y=y1, dev_status=dev_status)
-        a2, _ = swiglu_quantize(y1, offsets, E, SF_MMA_TILED, out=self.a2, h=self.h[:R], ws=self.ws,
-                                dev_status=dev_status)
+        if self.fused_swiglu:
+            # SwiGLU in the gate_up epilogue; its amax feeds the requantize directly
+            h, amax = grouped_gemm_swiglu(a1, self.w_gate_up, 2 * I, h=self.h[:R], amax=self.amax,
+                                          dev_status=dev_status)
+            a2 = self.a2
+            a2.offsets, a2.num_groups, a2.rows = offsets, E, R
+            nvfp4_quantize(h, R, I, I, None, offsets, E, GS_AMAX_GIVEN, amax, a2.q, a2.sf, SF_MMA_TILED, self.ws,
+                           dev_status)
+            a2.gs = amax
+        else:
+            y1 = self.y1[:R]
+            grouped_gemm(a1, self.w_gate_up, 2 * I, self.mid_dtype, y=y1, dev_status=dev_status)
+            a2, _ = swiglu_quantize(y1, offsets, E, SF_MMA_TILED, out=self.a2, h=self.h[:R], ws=self.ws,
+                                    dev_status=dev_status)
         y2 = self.y2[:R]
         grouped_gemm(a2, self.w_down, H, self.out_dtype, y=y2, dev_status=dev_status)
         return y2

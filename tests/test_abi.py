@@ -66,13 +66,18 @@ def test_host_validation_without_device(lib):
     # too many groups
     assert L.nvfp4_quantize(fake, 4, 32, 32, None, fake, 5000, 0, fake, fake, fake, 0, fake, None, None) == nv.ERR_UNSUPPORTED_SHAPE
     # GEMM shape limits
-    assert L.nvfp4_grouped_gemm(fake, fake, fake, fake, fake, fake, None, 1, 128, 100, 512, fake, 0, 0, None, None, None) == nv.ERR_UNSUPPORTED_SHAPE
-    assert L.nvfp4_grouped_gemm(fake, fake, fake, fake, fake, fake, None, 1, 128, 128, 320, fake, 0, 0, None, None, None) == nv.ERR_UNSUPPORTED_SHAPE
-    assert L.nvfp4_grouped_gemm(fake, fake, fake, fake, fake, fake, fake, 100000, 128, 128, 512, fake, 0, 0, None, None, None) == nv.ERR_UNSUPPORTED_SHAPE
-    assert L.nvfp4_grouped_gemm(fake, fake, fake, fake, fake, fake, None, 1, 128, 128, 512, fake, 0, 3, None, None, None) == nv.ERR_INVALID_ARG
-    assert L.nvfp4_grouped_gemm(None, fake, fake, fake, fake, fake, None, 1, 128, 128, 512, fake, 0, 0, None, None, None) == nv.ERR_INVALID_ARG
+    assert L.nvfp4_grouped_gemm(fake, fake, fake, fake, fake, fake, None, 1, 128, 100, 512, fake, 0, 0, None, None, None, None) == nv.ERR_UNSUPPORTED_SHAPE
+    assert L.nvfp4_grouped_gemm(fake, fake, fake, fake, fake, fake, None, 1, 128, 128, 320, fake, 0, 0, None, None, None, None) == nv.ERR_UNSUPPORTED_SHAPE
+    assert L.nvfp4_grouped_gemm(fake, fake, fake, fake, fake, fake, fake, 100000, 128, 128, 512, fake, 0, 0, None, None, None, None) == nv.ERR_UNSUPPORTED_SHAPE
+    assert L.nvfp4_grouped_gemm(fake, fake, fake, fake, fake, fake, None, 1, 128, 128, 512, fake, 0, 3, None, None, None, None) == nv.ERR_INVALID_ARG
+    assert L.nvfp4_grouped_gemm(None, fake, fake, fake, fake, fake, None, 1, 128, 128, 512, fake, 0, 0, None, None, None, None) == nv.ERR_INVALID_ARG
+    # SwiGLU epilogue: bf16 output and an amax buffer are required
+    assert L.nvfp4_grouped_gemm(fake, fake, fake, fake, fake, fake, None, 1, 128, 256, 512, fake, 0, 1, fake, None, None, None) == nv.ERR_INVALID_ARG
+    assert L.nvfp4_grouped_gemm(fake, fake, fake, fake, fake, fake, None, 1, 128, 256, 512, fake, 1, 1, None, None, None, None) == nv.ERR_INVALID_ARG
+    # AMAX_GIVEN is an accepted mode, an unknown one is not
+    assert L.nvfp4_quantize(fake, 4, 32, 32, None, None, 1, 3, fake, fake, fake, 0, fake, None, None) == nv.ERR_INVALID_ARG
     # empty problems are no-ops that touch nothing
-    assert L.nvfp4_grouped_gemm(None, None, None, None, None, None, None, 1, 0, 128, 512, None, 0, 0, None, None, None) == nv.OK
+    assert L.nvfp4_grouped_gemm(None, None, None, None, None, None, None, 1, 0, 128, 512, None, 0, 0, None, None, None, None) == nv.OK
     assert L.nvfp4_dequantize(None, None, 0, None, None, 1, 0, 32, None, 0, None) == nv.OK
     # remap shape limits
     assert L.mxfp4_to_nvfp4(fake, fake, 1, 4, 48, fake, fake, 0, fake, fake, None, None) == nv.ERR_UNSUPPORTED_SHAPE

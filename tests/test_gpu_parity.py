@@ -428,6 +428,72 @@ def test_gemm_long_k_tolerance():
     assert ok.all(), (err.max(), (err / bound).max())
 
 
+# --------------------------------------------------------------------------- fused SwiGLU epilogue
+def test_gemm_swiglu_epilogue():
+    """h = bf16(silu(g)*u) from the gate_up accumulators: compared with the
+    oracle SwiGLU of the same GEMM's fp32 output (one bf16 ulp), amax exact."""
+    L = layer()
+    nv = nvmod()
+    E, I, K = 5, 256, 512
+    N = 2 * I
+    counts = [3, 0, 200, 70, 129]
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    R = int(offsets[-1])
+    x = synthetic.gaussian_bf16(14, synthetic.STREAMS["x"], (R, K), outlier_frac=0.001)
+    w = synthetic.gaussian_bf16(14, synthetic.STREAMS["w_gate_up"], (E * N, K), sigma=0.02)
+    q, sf, gs, qs, ss = _packed_acts(x, None, offsets, E)
+    qw, sw, gw = _packed_weights(w, E, N, K)
+    y32 = _run_gemm(qs, ss, gs, qw, sw, gw, offsets, E, R, N, K, 0)
+    bound = nv.nvfp4_padded_rows_bound(R, E)
+    qa = np.zeros((bound, K // 2), np.uint8)
+    qa[:qs.shape[0]] = qs
+    sa = np.zeros((bound, K // 16), np.uint8)
+    sa[:ss.shape[0]] = ss
+    a = L.Packed(to_dev(qa), to_dev(tile(sa)), to_dev(gs), R, K, 1, to_dev(offsets), E)
+    wp = L.Packed(to_dev(qw), to_dev(tile(sw)), to_dev(gw), E * N, K, 1)
+    st = status_word()
+    h, amax = L.grouped_gemm_swiglu(a, wp, N, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    h_gpu = to_np(h)
+    h_ref = oracle.swiglu(y32)
+    d = np.abs(h_gpu.astype(np.int32) - h_ref.astype(np.int32))
+    assert (d <= 1).all() and (d == 0).mean() > 0.99
+    hf = np.abs(synthetic.bf16_bits_to_f32(h_gpu))
+    want = np.array([hf[offsets[e]:offsets[e + 1]].max() if counts[e] else 0.0 for e in range(E)], np.float32)
+    assert np.array_equal(to_np(amax), want)
+
+
+def test_moe_layer_fused_swiglu_stagewise():
+    L = layer()
+    T, H, I, E, k = 96, 256, 256, 8, 3
+    x = synthetic.gaussian_bf16(15, synthetic.STREAMS["x"], (T, H))
+    r = synthetic.route_topk_softmax(15, T, E, k)
+    off = r["offsets"]
+    R = len(r["row_index"])
+    wgu = synthetic.gaussian_bf16(15, synthetic.STREAMS["w_gate_up"], (E * 2 * I, H), sigma=0.02)
+    wd = synthetic.gaussian_bf16(15, synthetic.STREAMS["w_down"], (E * H, I), sigma=0.02)
+    qg, sg, gg = _packed_weights(wgu, E, 2 * I, H)
+    qd, sd, gd = _packed_weights(wd, E, H, I)
+    Wgu = L.Packed(to_dev(qg), to_dev(tile(sg)), to_dev(gg), E * 2 * I, H, 1)
+    Wd = L.Packed(to_dev(qd), to_dev(tile(sd)), to_dev(gd), E * H, I, 1)
+    moe = L.MoEExperts(Wgu, Wd, E, H, I, max_rows=R, out_dtype=0, mid_dtype=0, fused_swiglu=True)
+    s = status_word()
+    y2 = moe.forward(bf16_dev(x), to_dev(r["row_index"]), to_dev(off), dev_status=s)
+    torch.cuda.synchronize()
+    assert int(s.item()) == 0
+    rows, _ = slot_rows(off)
+    h = to_np(moe.h[:R])
+    q2, sf2, gs2, _ = oracle.quantize(h, None, off)          # requantize of the device's h: bit-exact
+    assert np.array_equal(to_np(moe.a2.gs), gs2)
+    assert np.array_equal(to_np(moe.a2.q)[rows], q2)
+    a2 = oracle.dequantize_f64(q2, sf2, oracle.rows_global_scale(gs2, off, R))
+    bd = oracle.dequantize_f64(qd, sd, np.repeat(gd, H)).reshape(E, H, I)
+    y2_ref, s2_ref = oracle.grouped_gemm_f64(a2, bd, off)
+    ok, err, bound = gemm_tol(to_np(y2), y2_ref, s2_ref)
+    assert ok.all(), (err / bound).max()
+
+
 # --------------------------------------------------------------------------- SwiGLU + requantize
 @pytest.mark.parametrize("ydt", [0, 1])
 def test_swiglu_requantize(ydt):
