@@ -137,16 +137,6 @@ def gemm_bytes(R, e_touched, N, K, out_bytes=2):
     return e_touched * N * K * 0.5625 + R * K * 0.5625 + R * N * out_bytes
 
 
-def pack_weights(w_bf16, E, rows_per, ws):
-    """Static NVFP4 quantization of [E*rows_per, K] weights, one global per expert."""
-    import torch
-    from nvfp4_w4a4_quantized_04_b200 import layer as L
-    offs = torch.arange(0, (E + 1) * rows_per, rows_per, dtype=torch.int32, device=w_bf16.device)
-    p = L.quantize(w_bf16, None, offs, E, layout=1, ws=ws)
-    p.offsets, p.num_groups, p.rows = None, 1, E * rows_per
-    return p
-
-
 # --------------------------------------------------------------------------- headline: MoE layer
 def setup_moe(device, seed, E, T, H, I, topk, fused=True):
     import torch
@@ -161,7 +151,8 @@ def setup_moe(device, seed, E, T, H, I, topk, fused=True):
     packs = []
     for name, rows_per, K in (("w_gate_up", 2 * I, H), ("w_down", H, I)):
         w = sc.gaussian_bf16(seed, synthetic.STREAMS[name], (E * rows_per, K), sigma=0.02)
-        packs.append(pack_weights(w, E, rows_per, ws))
+        ri = L.gate_up_interleave_index(E, I, device) if (fused and name == "w_gate_up") else None
+        packs.append(L.pack_weights(w, E, rows_per, ri, ws))
         del w
     torch.cuda.synchronize()
     x = sc.gaussian_bf16(seed, synthetic.STREAMS["x"], (T, H))
@@ -315,8 +306,8 @@ def comp_dense_mlp(device, iters, warmup, flush):
     from nvfp4_w4a4_quantized_04_b200 import layer as L
     M, H, I = 4096, 5120, 17408
     ws = L.workspace(1, device)
-    wgu = pack_weights(sc.gaussian_bf16(0, synthetic.STREAMS["w_gate_up"], (2 * I, H), sigma=0.02), 1, 2 * I, ws)
-    wd = pack_weights(sc.gaussian_bf16(0, synthetic.STREAMS["w_down"], (H, I), sigma=0.02), 1, H, ws)
+    wgu = L.pack_weights(sc.gaussian_bf16(0, synthetic.STREAMS["w_gate_up"], (2 * I, H), sigma=0.02), 1, 2 * I, None, ws)
+    wd = L.pack_weights(sc.gaussian_bf16(0, synthetic.STREAMS["w_down"], (H, I), sigma=0.02), 1, H, None, ws)
     xb = synthetic.gaussian_bf16(0, synthetic.STREAMS["x"], (M, H), outlier_frac=0.001)
     x = torch.from_numpy(xb.view(np.int16)).to(device).view(torch.bfloat16)
     a1 = L.empty_packed(M, H, 1, None, 1, device)
@@ -371,6 +362,11 @@ def comp_decode_moe(device, iters, warmup, flush):
         n = E * rows_per * K
         q = sc.mxfp4_codes(7, synthetic.STREAMS["mx_codes_" + name], n // 2).view(E * rows_per, K // 2)
         e8 = sc.mxfp4_exponents(7, synthetic.STREAMS["mx_exp_" + name], n // 32, lo=-10)
+        if name == "gate_up":
+            # checkpoint rows put in the SwiGLU epilogue's gate/up interleaved order
+            perm = L.gate_up_interleave_index(E, I, device).long()
+            q = q[perm].contiguous()
+            e8 = e8.view(E * rows_per, K // 32)[perm].reshape(-1).contiguous()
         qn = torch.empty_like(q)
         sf = torch.empty(n // 16, dtype=torch.uint8, device=device)
         gs = torch.empty(E, dtype=torch.float32, device=device)

@@ -76,7 +76,12 @@ typedef enum { NVFP4_SF_ROWMAJOR = 0, NVFP4_SF_MMA_TILED = 1 } nvfp4_sf_layout;
 typedef enum { NVFP4_GS_FROM_AMAX = 0, NVFP4_GS_GIVEN = 1, NVFP4_GS_AMAX_GIVEN = 2 } nvfp4_gs_mode;
 typedef enum { NVFP4_OUT_F32 = 0, NVFP4_OUT_BF16 = 1 } nvfp4_out_dtype;
 /* NONE: y = alpha * A B^T.  SWIGLU: the weight is a fused gate_up [2I, K]
- * (gate rows first); the epilogue writes h = bf16(silu(g) * u) with
+ * per expert stored gate/up interleaved in 32-row groups: packed rows
+ * 32j..32j+15 are gate rows 16j..16j+15 and packed rows 32j+16..32j+31 the
+ * up rows 16j..16j+15 (quantize the rows in that order, e.g. through the
+ * row_index of nvfp4_quantize: a row permutation commutes with NVFP4
+ * quantization, whose block scales are row-local and whose global scale is
+ * per expert).  The epilogue writes h = bf16(silu(g) * u) with
  * g = alpha*acc_gate, u = alpha*acc_up kept in fp32 (no bf16 rounding of the
  * gate_up output in between; silu through the fast exp/divide intrinsics),
  * y is bf16 [M_total, N/2], and amax_out[e]

@@ -50,7 +50,7 @@ constexpr int BK = 256;                 // K elements per stage = 128 bytes of c
 constexpr int STAGES = 4;
 constexpr int W_STAGE = BM * 128;       // 16 KB
 constexpr int X_STAGE = BN * 128;       // 24 KB
-constexpr int SFW_STAGE = 4096;         // 128 rows x 16 scales (4 atoms); SwiGLU tiles use two blocks
+constexpr int SFW_STAGE = 2048;         // 128 rows x 16 scales (4 atoms)
 constexpr int SFX_STAGE = 4096;         // up to 2 row blocks x 4 atoms
 constexpr int OFF_W = 0;
 constexpr int OFF_X = OFF_W + STAGES * W_STAGE;
@@ -233,9 +233,9 @@ struct Tile {
 
 __device__ __forceinline__ int chunks_of(int m) { return (m + BN - 1) / BN; }
 
-// With the SwiGLU epilogue a 128-row weight tile is the 64 gate rows
-// j0..j0+63 stacked on the matching 64 up rows I+j0..I+j0+63 (w_row0 is the
-// gate row; the up row is w_row0 + N/2), and n_col0 indexes h columns.
+// With the SwiGLU epilogue the fused gate_up weight is stored in 32-row
+// groups (16 gate rows, then the 16 matching up rows), so a 128-row weight
+// tile covers the 64 h columns starting at n_col0 = 64*mt.
 template <bool kSwiglu>
 __device__ __forceinline__ Tile decode_tile(int t, const int32_t *s_off, const int32_t *s_slot,
                                             const int32_t *s_tile, int E, int N) {
@@ -249,7 +249,7 @@ __device__ __forceinline__ Tile decode_tile(int t, const int32_t *s_off, const i
   const int start = ch * csz;
   T.e = e;
   T.n_col0 = kSwiglu ? mt * (BM / 2) : mt * BM;
-  T.w_row0 = e * N + (kSwiglu ? mt * (BM / 2) : mt * BM);
+  T.w_row0 = e * N + mt * BM;
   T.x_row0 = s_slot[e] + start;
   T.y_row0 = s_off[e] + start;
   T.n_valid = min(csz, m_e - start);
@@ -259,7 +259,7 @@ __device__ __forceinline__ Tile decode_tile(int t, const int32_t *s_off, const i
 // ------------------------------------------------------------------ kernel
 template <bool kSwiglu, bool kBf16Out>
 __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(
-    const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_w64,
+    const __grid_constant__ CUtensorMap tmap_w,
     const __grid_constant__ CUtensorMap tmap_x128,
     const __grid_constant__ CUtensorMap tmap_x64, const __grid_constant__ CUtensorMap tmap_x32,
     const uint8_t *__restrict__ w_sf, const uint8_t *__restrict__ x_sf,
@@ -376,11 +376,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(
         const int rows_ld = (T.n_valid + 31) & ~31;
         const int xr0 = T.x_row0 & ~127;                               // first scale row block
         const int nrb = ((T.x_row0 & 127) + T.n_valid + 127) >> 7;     // 1 or 2
-        const uint32_t bytes = is_w ? (uint32_t)(W_STAGE + (kSwiglu ? 4096 : 2048) + nrb * 2048)
+        const uint32_t bytes = is_w ? (uint32_t)(W_STAGE + SFW_STAGE + nrb * 2048)
                                     : (uint32_t)(rows_ld * 128);
         const uint8_t *sfw_tile = w_sf + (int64_t)(T.w_row0 >> 7) * sf_row_stride;
-        const int w_up0 = T.w_row0 + N / 2;                            // SwiGLU: matching up rows
-        const uint8_t *sfw_up = w_sf + (int64_t)(w_up0 >> 7) * sf_row_stride;
         const uint8_t *sfx_tile = x_sf + (int64_t)(xr0 >> 7) * sf_row_stride;
         for (int ks = 0; ks < ksteps; ++ks) {
           if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1, abort_flag, dev_status)) { ok = false; break; }
@@ -389,15 +387,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(
           armed[stage] = true;
           armed_parity[stage] = phase;
           if (is_w) {
-            if (kSwiglu) {
-              tma_load_2d(sbase + OFF_W + stage * W_STAGE, &tmap_w64, ks * 128, T.w_row0, fb, pol);
-              tma_load_2d(sbase + OFF_W + stage * W_STAGE + 8192, &tmap_w64, ks * 128, w_up0, fb, pol);
-              bulk_load(sbase + OFF_SFW + stage * SFW_STAGE, sfw_tile + ks * 2048, 2048, fb);
-              bulk_load(sbase + OFF_SFW + stage * SFW_STAGE + 2048, sfw_up + ks * 2048, 2048, fb);
-            } else {
-              tma_load_2d(sbase + OFF_W + stage * W_STAGE, &tmap_w, ks * 128, T.w_row0, fb, pol);
-              bulk_load(sbase + OFF_SFW + stage * SFW_STAGE, sfw_tile + ks * 2048, 2048, fb);
-            }
+            tma_load_2d(sbase + OFF_W + stage * W_STAGE, &tmap_w, ks * 128, T.w_row0, fb, pol);
+            bulk_load(sbase + OFF_SFW + stage * SFW_STAGE, sfw_tile + ks * 2048, 2048, fb);
             for (int rb = 0; rb < nrb; ++rb)
               bulk_load(sbase + OFF_SFX + stage * SFX_STAGE + rb * 2048, sfx_tile + rb * sf_row_stride + ks * 2048,
                         2048, fb);
@@ -445,20 +436,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(
         const uint32_t tcol = tmem_base + lane_base + TMEM_SF + sb * TMEM_SF_STRIDE;
         const uint32_t sfw_addr = sbase + OFF_SFW + stage * SFW_STAGE + lane * 16;
         const uint32_t sfx_addr = sbase + OFF_SFX + stage * SFX_STAGE + lane * 16;
-        if (kSwiglu) {
-          // tile rows 0..63 = gate rows of one half of a 128-row scale block,
-          // rows 64..127 = up rows: lane l takes the two 4-scale words of the
-          // right half from each atom row l
-          const int hg = (T.w_row0 & 127) >> 6, hu = ((T.w_row0 + N / 2) & 127) >> 6;
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint4 g = lds128(sfw_addr + kk * 512), u = lds128(sfw_addr + 2048 + kk * 512);
-            tc_st_x4(tcol + kk * 4, make_uint4(hg ? g.z : g.x, hg ? g.w : g.y, hu ? u.z : u.x, hu ? u.w : u.y));
-          }
-        } else {
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) tc_st_x4(tcol + kk * 4, lds128(sfw_addr + kk * 512));
-        }
+        for (int kk = 0; kk < 4; ++kk) tc_st_x4(tcol + kk * 4, lds128(sfw_addr + kk * 512));
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) tc_st_x4(tcol + 16 + kk * 8, lds128(sfx_addr + kk * 512));
         if (nrb > 1) {
@@ -542,52 +521,48 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(
           mbar_arrive(bar_acc_empty + 8 * ab);
         }
         if (kSwiglu) {
-          // lane quadrants 0,1 hold gate rows, 2,3 the matching up rows: the
-          // gate warps compute silu(g) of g = alpha*acc and park it in shared
-          // memory, the up warps form h = bf16(silu(g) * u), keep max|h|, and
-          // store h rows.  silu uses the fast exp and divide intrinsics (a
-          // few fp32 ulps, far below the bf16 rounding of h).
+          // TMEM lane l of quadrant q holds h column 16q + (l & 15): the gate
+          // row for l < 16, the matching up row for l >= 16.  One xor-16
+          // shuffle per token pair gives each lane both operands; the gate
+          // lane finishes tokens 0..15 of the 32, the up lane tokens 16..31.
+          // h = bf16(silu(g) * u) with g, u = alpha*acc in fp32 (silu through
+          // the fast exp and divide intrinsics: a few fp32 ulps, far below the
+          // bf16 rounding of h).  The 32x16 h block is staged in shared memory
+          // (the two token halves 576 bytes apart, so the halves' stores hit
+          // disjoint banks) and written as 32-byte row segments.
+          const bool gate_lane = lane < 16;
+          const uint32_t half = gate_lane ? 0u : 576u;
 #pragma unroll
           for (int sub = 0; sub < 2; ++sub) {
             const int tok0 = c0 + sub * 32;
             if (tok0 >= T.n_valid) break;
             const int rows_here = min(32, T.n_valid - tok0);
-            if (quad < 2) {
+            const int my0 = gate_lane ? 0 : 16;
 #pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                const float gv = __fmul_rn(__uint_as_float(r[sub * 32 + i]), alpha);
-                const float sv = __fdividef(gv, 1.0f + __expf(-gv));
-                asm volatile("st.shared.b32 [%0], %1;" :: "r"(epi + i * 128 + lane * 4), "f"(sv) : "memory");
+            for (int j = 0; j < 16; ++j) {
+              const uint32_t mine = gate_lane ? r[sub * 32 + 16 + j] : r[sub * 32 + j];
+              const uint32_t other = __shfl_xor_sync(0xffffffffu, mine, 16);
+              const float gv = __fmul_rn(__uint_as_float(gate_lane ? r[sub * 32 + j] : other), alpha);
+              const float uv = __fmul_rn(__uint_as_float(gate_lane ? other : r[sub * 32 + 16 + j]), alpha);
+              const float sv = __fdividef(gv, 1.0f + __expf(-gv));
+              const __nv_bfloat16 hv = __float2bfloat16_rn(__fmul_rn(sv, uv));
+              const uint16_t hb = *reinterpret_cast<const uint16_t *>(&hv);
+              if (my0 + j < rows_here) hmax = max(hmax, (uint32_t)(hb & 0x7FFFu));
+              asm volatile("st.shared.b16 [%0], %1;" :: "r"(epi + half + j * 32 + (lane & 15) * 2), "h"(hb) : "memory");
+            }
+            __syncwarp();
+            const int NH = N / 2;
+            __nv_bfloat16 *hbase = reinterpret_cast<__nv_bfloat16 *>(y) + (int64_t)(T.y_row0 + tok0) * NH +
+                                   T.n_col0 + quad * 16;
+#pragma unroll
+            for (int it = 0; it < 2; ++it) {
+              const int row = it * 16 + (lane >> 1), chunk = lane & 1;
+              if (row < rows_here) {
+                const uint4 v = lds128(epi + (row >> 4) * 576 + (row & 15) * 32 + chunk * 16);
+                *reinterpret_cast<uint4 *>(hbase + (int64_t)row * NH + chunk * 8) = v;
               }
             }
-            asm volatile("bar.sync 1, 128;" ::: "memory");
-            if (quad >= 2) {
-              const uint32_t gsl = sbase + OFF_EPI + quad * EPI_WARP_BYTES;   // slab of the gate partner
-#pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                float sv;
-                asm volatile("ld.shared.b32 %0, [%1];" : "=f"(sv) : "r"(gsl + i * 128 + lane * 4) : "memory");
-                const float uv = __fmul_rn(__uint_as_float(r[sub * 32 + i]), alpha);
-                const __nv_bfloat16 hv = __float2bfloat16_rn(__fmul_rn(sv, uv));
-                const uint16_t hb = *reinterpret_cast<const uint16_t *>(&hv);
-                if (i < rows_here) hmax = max(hmax, (uint32_t)(hb & 0x7FFFu));
-                asm volatile("st.shared.b16 [%0], %1;" :: "r"(epi + i * 64 + lane * 2), "h"(hb) : "memory");
-              }
-              __syncwarp();
-              const int NH = N / 2;
-              __nv_bfloat16 *hbase = reinterpret_cast<__nv_bfloat16 *>(y) + (int64_t)(T.y_row0 + tok0) * NH +
-                                     T.n_col0 + (quad - 2) * 32;
-#pragma unroll
-              for (int it = 0; it < 4; ++it) {
-                const int row = it * 8 + (lane >> 2), chunk = lane & 3;
-                if (row < rows_here) {
-                  const uint4 v = lds128(epi + row * 64 + chunk * 16);
-                  *reinterpret_cast<uint4 *>(hbase + (int64_t)row * NH + chunk * 8) = v;
-                }
-              }
-              __syncwarp();
-            }
-            asm volatile("bar.sync 1, 128;" ::: "memory");
+            __syncwarp();
           }
           continue;
         }
@@ -636,7 +611,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(
           __syncwarp();
         }
       }
-      if (kSwiglu && quad >= 2) {
+      if (kSwiglu) {
 #pragma unroll
         for (int d = 16; d > 0; d >>= 1) hmax = max(hmax, __shfl_xor_sync(0xffffffffu, hmax, d));
         if (lane == 0 && hmax) atomicMax(reinterpret_cast<uint32_t *>(amax_out) + T.e, hmax << 16);
@@ -713,9 +688,8 @@ extern "C" nvfp4_status nvfp4_grouped_gemm(const uint8_t *a_q, const uint8_t *a_
     return NVFP4_ERR_INVALID_ARG;
   if (!get_encoder()) return NVFP4_ERR_CUDA;
   const int64_t x_rows = nvfp4_padded_rows_bound(M_total, E);
-  CUtensorMap tw, tw64, tx128, tx64, tx32;
+  CUtensorMap tw, tx128, tx64, tx32;
   if (!make_map(&tw, b_q, (uint64_t)E * N, (uint64_t)K / 2, 128)) return NVFP4_ERR_CUDA;
-  if (!make_map(&tw64, b_q, (uint64_t)E * N, (uint64_t)K / 2, 64)) return NVFP4_ERR_CUDA;
   if (!make_map(&tx128, a_q, (uint64_t)x_rows, (uint64_t)K / 2, 128)) return NVFP4_ERR_CUDA;
   if (!make_map(&tx64, a_q, (uint64_t)x_rows, (uint64_t)K / 2, 64)) return NVFP4_ERR_CUDA;
   if (!make_map(&tx32, a_q, (uint64_t)x_rows, (uint64_t)K / 2, 32)) return NVFP4_ERR_CUDA;
@@ -733,7 +707,7 @@ extern "C" nvfp4_status nvfp4_grouped_gemm(const uint8_t *a_q, const uint8_t *a_
       return NVFP4_ERR_CUDA;
     g_attr_set[variant] = true;
   }
-  kern<<<g_sms, gemm::NUM_THREADS, gemm::SMEM_BYTES, stream>>>(tw, tw64, tx128, tx64, tx32, b_sf, a_sf, b_gs, a_gs,
+  kern<<<g_sms, gemm::NUM_THREADS, gemm::SMEM_BYTES, stream>>>(tw, tx128, tx64, tx32, b_sf, a_sf, b_gs, a_gs,
                                                                expert_offsets, E, (int)M_total, (int)N, (int)K, y,
                                                                amax_out, dev_status);
   return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;

@@ -109,10 +109,33 @@ def grouped_gemm(a: Packed, w: Packed, N: int, out_dtype=OUT_BF16, y=None, dev_s
     return y
 
 
+def gate_up_interleave_index(E: int, I: int, device="cuda") -> torch.Tensor:
+    """Source row of each packed row of a fused gate_up weight [E*2I, K] in the
+    order the SwiGLU epilogue reads: per expert, 32-row groups holding 16 gate
+    rows and then the 16 matching up rows (gate rows are 0..I-1 of the expert,
+    up rows I..2I-1 in the source).  int32 [E*2I]."""
+    assert I % 64 == 0
+    n = torch.arange(E * 2 * I, dtype=torch.int64)
+    e, m = n // (2 * I), n % (2 * I)
+    j, r = m // 32, m % 32
+    src = e * 2 * I + torch.where(r < 16, 16 * j + r, I + 16 * j + (r - 16))
+    return src.to(torch.int32).to(device)
+
+
+def pack_weights(w: torch.Tensor, E: int, rows_per: int, row_index=None, ws=None) -> Packed:
+    """Static NVFP4 quantization of per-expert weights [E*rows_per, K] (one global
+    scale per expert, MMA-tiled scales), optionally reordering rows within each
+    expert (``row_index``, e.g. ``gate_up_interleave_index``)."""
+    offs = torch.arange(0, (E + 1) * rows_per, rows_per, dtype=torch.int32, device=w.device)
+    p = quantize(w, row_index, offs, E, SF_MMA_TILED, ws=ws)
+    p.offsets, p.num_groups, p.rows = None, 1, E * rows_per
+    return p
+
+
 def grouped_gemm_swiglu(a: Packed, w_gate_up: Packed, N: int, h=None, amax=None, dev_status=None):
     """h [a.rows, N/2] = bf16(silu(g) * u) straight from the gate_up GEMM's
-    accumulators (g, u = the two halves of the fused weight), plus the
-    per-expert amax of h (fp32 [E])."""
+    accumulators, plus the per-expert amax of h (fp32 [E]).  ``w_gate_up`` is
+    packed in the interleaved row order of ``gate_up_interleave_index``."""
     assert a.layout == SF_MMA_TILED and w_gate_up.layout == SF_MMA_TILED
     E = a.num_groups if a.offsets is not None else 1
     if h is None:
@@ -143,8 +166,9 @@ def swiglu_quantize(y: torch.Tensor, offsets, num_groups: int, layout=SF_MMA_TIL
 class MoEExperts:
     """Routed experts of one MoE layer in NVFP4 W4A4.
 
-    w_gate_up: packed [E*2I, H] (rows 0..I-1 of each expert = gate, I..2I-1 = up),
-    one global scale per expert; w_down: packed [E*H, I].
+    w_gate_up: packed [E*2I, H], one global scale per expert: rows 0..I-1 of
+    each expert = gate, I..2I-1 = up; with ``fused_swiglu`` the rows are in the
+    order of ``gate_up_interleave_index`` instead.  w_down: packed [E*H, I].
     forward(x bf16 [T, H], row_index int32 [R], offsets int32 [E+1]) -> Y bf16 [R, H]
     in routed order (the weighted combine is outside this layer).
     """

@@ -450,7 +450,8 @@ def test_gemm_swiglu_epilogue():
     sa = np.zeros((bound, K // 16), np.uint8)
     sa[:ss.shape[0]] = ss
     a = L.Packed(to_dev(qa), to_dev(tile(sa)), to_dev(gs), R, K, 1, to_dev(offsets), E)
-    wp = L.Packed(to_dev(qw), to_dev(tile(sw)), to_dev(gw), E * N, K, 1)
+    il = L.gate_up_interleave_index(E, I, "cpu").numpy()
+    wp = L.Packed(to_dev(qw[il]), to_dev(tile(sw[il])), to_dev(gw), E * N, K, 1)
     st = status_word()
     h, amax = L.grouped_gemm_swiglu(a, wp, N, dev_status=st)
     torch.cuda.synchronize()
@@ -473,7 +474,8 @@ def test_moe_layer_fused_swiglu_stagewise():
     R = len(r["row_index"])
     wgu = synthetic.gaussian_bf16(15, synthetic.STREAMS["w_gate_up"], (E * 2 * I, H), sigma=0.02)
     wd = synthetic.gaussian_bf16(15, synthetic.STREAMS["w_down"], (E * H, I), sigma=0.02)
-    qg, sg, gg = _packed_weights(wgu, E, 2 * I, H)
+    il = L.gate_up_interleave_index(E, I, "cpu").numpy()
+    qg, sg, gg = _packed_weights(wgu[il], E, 2 * I, H)
     qd, sd, gd = _packed_weights(wd, E, H, I)
     Wgu = L.Packed(to_dev(qg), to_dev(tile(sg)), to_dev(gg), E * 2 * I, H, 1)
     Wd = L.Packed(to_dev(qd), to_dev(tile(sd)), to_dev(gd), E * H, I, 1)
@@ -484,6 +486,22 @@ def test_moe_layer_fused_swiglu_stagewise():
     assert int(s.item()) == 0
     rows, _ = slot_rows(off)
     h = to_np(moe.h[:R])
+    # stage 1+2: h against silu(g)*u of the fp64 gate_up GEMM on the oracle's
+    # quantized operands (gate/up rows put back in source order).  Bound: the
+    # GEMM tolerance on g and u carried through h (|dh/dg| <= 1.1|u|,
+    # |dh/du| = |silu g|) plus one bf16 rounding on each side.
+    q1, sf1, gs1, _ = oracle.quantize(x, r["row_index"], off)
+    a1 = oracle.dequantize_f64(q1, sf1, oracle.rows_global_scale(gs1, off, R))
+    b_il = oracle.dequantize_f64(qg, sg, np.repeat(gg, 2 * I))
+    b1 = np.empty_like(b_il)
+    b1[il] = b_il
+    y1, s1 = oracle.grouped_gemm_f64(a1, b1.reshape(E, 2 * I, H), off)
+    g, u, sg1, su1 = y1[:, :I], y1[:, I:], s1[:, :I], s1[:, I:]
+    silu = g / (1.0 + np.exp(-g))
+    h64 = silu * u
+    tol = 1.1 * np.abs(u) * (1e-5 * sg1 + 1e-6) + np.abs(silu) * (1e-5 * su1 + 1e-6) + 2.0 ** -7 * np.abs(h64) + 1e-30
+    hf = synthetic.bf16_bits_to_f32(h).astype(np.float64)
+    assert (np.abs(hf - h64) <= tol).all(), (np.abs(hf - h64) / tol).max()
     q2, sf2, gs2, _ = oracle.quantize(h, None, off)          # requantize of the device's h: bit-exact
     assert np.array_equal(to_np(moe.a2.gs), gs2)
     assert np.array_equal(to_np(moe.a2.q)[rows], q2)
