@@ -160,6 +160,7 @@ def setup_moe(device, seed, E, T, H, I, topk, fused=True):
                        fused_swiglu=fused)
     ri = torch.from_numpy(r["row_index"]).to(device)
     off = torch.from_numpy(r["offsets"]).to(device)
+    r["slot_dev"] = torch.from_numpy(r["slot"].astype(np.int32)).to(device)
     return moe, x, ri, off, r, R
 
 
@@ -171,6 +172,7 @@ def run_headline(args, rank, world, device):
     E, T, H, I, k = args.experts, args.tokens, 4096, 1024, 10
     fused = not args.unfused
     moe, x, ri, off, r, R = setup_moe(device, rank, E, T, H, I, k, fused=fused)
+    sl = r["slot_dev"]
     flops = moe_flops(R, H, I)
     e_touched = int((np.diff(r["offsets"]) > 0).sum())
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
@@ -181,7 +183,7 @@ def run_headline(args, rank, world, device):
     def stages(evs=None):
         rec = (lambda i: evs[i].record(stream)) if evs else (lambda i: None)
         rec(0)
-        a1 = L.quantize(x, ri, off, E, layout=1, out=moe.a1, ws=moe.ws, rows=R)
+        a1 = L.moe_quantize(x, sl, off, E, layout=1, out=moe.a1, ws=moe.ws, rows=R)
         rec(1)
         if fused:
             h, amax = L.grouped_gemm_swiglu(a1, moe.w_gate_up, 2 * I, h=moe.h[:R], amax=moe.amax)
@@ -225,8 +227,9 @@ def run_headline(args, rank, world, device):
     # e2e through the public API with host buffers: pinned H2D of the step's
     # inputs, the layer, D2H of its result, all inside the timed region
     x_host, ri_host, off_host = x.cpu().pin_memory(), ri.cpu().pin_memory(), off.cpu().pin_memory()
+    sl_host = sl.cpu().pin_memory()
     y_host = torch.empty((R, H), dtype=torch.bfloat16).pin_memory()
-    x_d, ri_d, off_d = torch.empty_like(x), torch.empty_like(ri), torch.empty_like(off)
+    x_d, ri_d, off_d, sl_d = torch.empty_like(x), torch.empty_like(ri), torch.empty_like(off), torch.empty_like(sl)
     n_e2e = max(2, min(args.steps, 5))
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -235,7 +238,8 @@ def run_headline(args, rank, world, device):
         x_d.copy_(x_host, non_blocking=True)
         ri_d.copy_(ri_host, non_blocking=True)
         off_d.copy_(off_host, non_blocking=True)
-        y = moe.forward(x_d, ri_d, off_d)
+        sl_d.copy_(sl_host, non_blocking=True)
+        y = moe.forward(x_d, ri_d, off_d, slot=sl_d)
         y_host.copy_(y, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
@@ -244,7 +248,7 @@ def run_headline(args, rank, world, device):
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     e2e_ms = float(t.item())
-    h2d = x.numel() * 2 + ri.numel() * 4 + off.numel() * 4
+    h2d = x.numel() * 2 + ri.numel() * 4 + off.numel() * 4 + sl.numel() * 4
     d2h = R * H * 2
 
     med = np.median(per, axis=0)
@@ -255,6 +259,11 @@ def run_headline(args, rank, world, device):
     g1_flops = 2.0 * R * 2 * I * H
     g2_bytes = gemm_bytes(R, e_touched, H, I)
     g2_flops = 2.0 * R * H * I
+    # the other two stages: x read once and R packed rows written; h read and
+    # its packed copy written
+    q1_bytes = T * H * 2 + R * H * (0.5 + 1 / 16)
+    q2_bytes = R * I * 2 + R * I * (0.5 + 1 / 16)
+    q1_ms, q2_ms = float(np.mean(per[:, 0])), float(np.mean(per[:, 2]))
     roof = {"bound": "hbm", "kernel": ("nvfp4::gemm::grouped_gemm_kernel<swiglu> (gate_up + SwiGLU epilogue launch)"
                                        if fused else "nvfp4::gemm::grouped_gemm_kernel (gate_up launch)"),
             "achieved": round(gbs(g1_bytes, g1_ms), 1), "peak": HBM_PEAK, "unit": "GB/s",
@@ -267,13 +276,15 @@ def run_headline(args, rank, world, device):
             "fp4_peak_source": f"{PEAKS_KIND} bf16_tflops x 4 (nominal fp4/bf16 ratio)"}
     breakdown = {
         "pipeline": "gate_up GEMM with SwiGLU epilogue" if fused else "gate_up GEMM, then SwiGLU + requantize",
-        "gather_quantize_ms": round(float(med[0]), 4),
+        "dispatch_quantize_ms": round(float(med[0]), 4),
+        "dispatch_quantize_gbs": round(gbs(q1_bytes, q1_ms), 1),
         ("gate_up_swiglu_gemm_ms" if fused else "gate_up_gemm_ms"): round(float(med[1]), 4),
         ("requantize_ms" if fused else "swiglu_requantize_ms"): round(float(med[2]), 4),
+        "requantize_gbs": round(gbs(q2_bytes, q2_ms), 1),
         "down_gemm_ms": round(float(med[3]), 4),
         "gate_up_gbs": round(gbs(g1_bytes, g1_ms), 1), "gate_up_tflops": round(g1_flops / (g1_ms * 1e-3) / 1e12, 1),
         "down_gbs": round(gbs(g2_bytes, g2_ms), 1), "down_tflops": round(g2_flops / (g2_ms * 1e-3) / 1e12, 1),
-        "layer_roofline_ms": round(1e3 * max((g1_bytes + g2_bytes) / (HBM_PEAK * 1e9),
+        "layer_roofline_ms": round(1e3 * max((q1_bytes + g1_bytes + q2_bytes + g2_bytes) / (HBM_PEAK * 1e9),
                                              flops / (FP4_PEAK * 1e12)), 4),
     }
     workload = f"moe_routed_experts_e{E}_top{k}_t{T}_h{H}_i{I}"

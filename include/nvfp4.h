@@ -114,7 +114,9 @@ int64_t nvfp4_padded_rows_bound(int64_t rows, int num_groups);
  *               rows (offsets[0] == 0, offsets[G] == rows).  Each group has
  *               its own global scale and its own 128-aligned slot in q/sf.
  *               NULL: one group, rows written contiguously (padded to 128 rows
- *               only for MMA_TILED).
+ *               only for MMA_TILED).  Padding rows (a slot's rows past its
+ *               group, a tile's rows past `rows`) are not written: the
+ *               grouped GEMM never stores the columns they feed.
  *   gs_mode, global_scale
  *               fp32 [max(1,num_groups)] device.  FROM_AMAX: written with
  *               s_g = amax/2688 (2688 = 6*448: the block holding the amax gets
@@ -135,6 +137,33 @@ nvfp4_status nvfp4_quantize(const void *x, int64_t rows, int64_t K, int64_t ld_x
                             int num_groups, nvfp4_gs_mode gs_mode, float *global_scale,
                             uint8_t *q, uint8_t *sf, nvfp4_sf_layout sf_layout,
                             void *workspace, int32_t *dev_status, cudaStream_t stream);
+
+/*
+ * nvfp4_moe_quantize -- the routed-expert activation quantize in token order.
+ * [P1: routed experts' inputs are quantized to NVFP4 on the fly, one global
+ *  scale per expert group as in nvfp4_quantize.]
+ * Same result, byte for byte in every routed row, as nvfp4_quantize with
+ * rows = group_offsets[num_groups] and row_index[slot[t*topk + c]] = t, but
+ * each token row of x is read once: its 16-element block amaxes are formed
+ * once and its topk copies are encoded with their experts' global scales.
+ *   x           bf16 [tokens, ld_x], ld_x >= K, ld_x % 8 == 0.
+ *   slot        int32 [tokens, topk] device: routed row of each (token,
+ *               choice), as nvfp4_moe_route writes it; -1 = not routed.  The
+ *               non-negative entries must be distinct and cover
+ *               [0, group_offsets[num_groups]); an entry beyond that range is
+ *               skipped and reported as NVFP4_ERR_INDEX.  1 <= topk <= 32.
+ *   group_offsets, num_groups   int32 [num_groups+1] prefix sums over routed
+ *               rows (required); each group has its own 128-aligned slot in
+ *               q/sf as in nvfp4_quantize.  Padding rows of a slot are left
+ *               unwritten (the grouped GEMM never stores their columns).
+ *   gs_mode, global_scale, q, sf, sf_layout, workspace, dev_status
+ *               as in nvfp4_quantize (FROM_AMAX takes the amax per expert over
+ *               the tokens routed to it).
+ */
+nvfp4_status nvfp4_moe_quantize(const void *x, int64_t tokens, int64_t K, int64_t ld_x, const int32_t *slot,
+                                int topk, const int32_t *group_offsets, int num_groups, nvfp4_gs_mode gs_mode,
+                                float *global_scale, uint8_t *q, uint8_t *sf, nvfp4_sf_layout sf_layout,
+                                void *workspace, int32_t *dev_status, cudaStream_t stream);
 
 /*
  * nvfp4_dequantize -- y = (e2m1(code) * e4m3(S)) * s_g, rounded once to the

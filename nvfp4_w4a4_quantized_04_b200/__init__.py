@@ -8,8 +8,10 @@ no CUDA device is present, the calls raise.
 
 Entry points (same names as the C ABI): ``nvfp4_quantize``,
 ``nvfp4_dequantize``, ``mxfp4_to_nvfp4``, ``nvfp4_grouped_gemm``,
-``nvfp4_swiglu_quantize``, ``nvfp4_kv_quantize``, ``nvfp4_kv_dequantize``, plus
-``nvfp4_workspace_size`` and ``nvfp4_padded_rows_bound``.
+``nvfp4_swiglu_quantize``, ``nvfp4_kv_quantize``, ``nvfp4_kv_dequantize``,
+``nvfp4_moe_quantize``, ``nvfp4_moe_route``, ``nvfp4_moe_combine``,
+``nvfp4_quantize_noalloc``, plus ``nvfp4_workspace_size``,
+``nvfp4_padded_rows_bound`` and ``nvfp4_moe_route_workspace_size``.
 """
 from __future__ import annotations
 
@@ -43,7 +45,7 @@ EXPORTS = [
     "nvfp4_status_string", "nvfp4_workspace_size", "nvfp4_padded_rows_bound",
     "nvfp4_quantize", "nvfp4_dequantize", "mxfp4_to_nvfp4", "nvfp4_grouped_gemm",
     "nvfp4_swiglu_quantize", "nvfp4_kv_quantize", "nvfp4_kv_dequantize", "nvfp4_quantize_noalloc",
-    "nvfp4_moe_route_workspace_size", "nvfp4_moe_route", "nvfp4_moe_combine",
+    "nvfp4_moe_route_workspace_size", "nvfp4_moe_route", "nvfp4_moe_combine", "nvfp4_moe_quantize",
 ]
 NOALLOC_MAX_GROUPS = 1024
 
@@ -71,6 +73,8 @@ def load_library(path: str = LIB_PATH):
     L.nvfp4_padded_rows_bound.argtypes = [i64, i32]
     L.nvfp4_quantize.restype = i32
     L.nvfp4_quantize.argtypes = [P, i64, i64, i64, P, P, i32, i32, P, P, P, i32, P, P, P]
+    L.nvfp4_moe_quantize.restype = i32
+    L.nvfp4_moe_quantize.argtypes = [P, i64, i64, i64, P, i32, P, i32, i32, P, P, P, i32, P, P, P]
     L.nvfp4_dequantize.restype = i32
     L.nvfp4_dequantize.argtypes = [P, P, i32, P, P, i32, i64, i64, P, i32, P]
     L.mxfp4_to_nvfp4.restype = i32
@@ -142,6 +146,17 @@ def nvfp4_quantize_noalloc(x, rows, K, ld_x, row_index, group_offsets, num_group
         _ptr(global_scale), _ptr(q), _ptr(sf), sf_layout, _ptr(dev_status), _stream(stream))
     if check:
         _check(st, "nvfp4_quantize_noalloc")
+    return st
+
+
+def nvfp4_moe_quantize(x, tokens, K, ld_x, slot, topk, group_offsets, num_groups, gs_mode, global_scale,
+                       q, sf, sf_layout, workspace, dev_status=None, stream=None, check=True) -> int:
+    """Routed-expert activation quantize in token order (each token row read once)."""
+    st = load_library().nvfp4_moe_quantize(
+        _ptr(x), tokens, K, ld_x, _ptr(slot), topk, _ptr(group_offsets), num_groups, gs_mode,
+        _ptr(global_scale), _ptr(q), _ptr(sf), sf_layout, _ptr(workspace), _ptr(dev_status), _stream(stream))
+    if check:
+        _check(st, "nvfp4_moe_quantize")
     return st
 
 

@@ -140,15 +140,10 @@ __global__ void finalize_scales_kernel(const uint32_t *__restrict__ amax_bits, i
 }
 
 // ---------------------------------------------------------------- pass 2: encode
-// One thread per 16-element block: one 32-byte load (two 16-byte loads when
-// the row stride is not 32-byte aligned), the block amax in integer SIMD,
-// one IEEE division for the scale and one IEEE reciprocal per block, the
-// 16 products as eight packed f32x2 multiplies, eight e2m1x2 conversions and
-// one 8-byte store.  A warp covers 32 consecutive blocks per step; warps
-// stride over 64-block chunks so the whole grid streams through memory
-// together.  Rows only move forward per lane, so the row -> (group, source
-// row) lookup walks forward from the last group.
-__device__ __forceinline__ uint2 load_block(const uint16_t *p, bool v8, uint4 &a, uint4 &b) {
+// Per 16-element block: the block amax in integer SIMD, one IEEE division
+// for the scale and one IEEE reciprocal, the 16 products as eight packed
+// f32x2 multiplies, eight e2m1x2 conversions and one 8-byte store.
+__device__ __forceinline__ void load_block(const uint16_t *p, bool v8, uint4 &a, uint4 &b) {
   if (v8) {
     asm volatile("ld.global.nc.L1::no_allocate.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
                  : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w), "=r"(b.x), "=r"(b.y), "=r"(b.z), "=r"(b.w)
@@ -157,26 +152,39 @@ __device__ __forceinline__ uint2 load_block(const uint16_t *p, bool v8, uint4 &a
     a = ldg_nc_v4(p);
     b = ldg_nc_v4(p + 8);
   }
-  return make_uint2(0, 0);
 }
 
-// bf16 pair (lo in bits 0..15) times r, both products rounded to nearest even.
-__device__ __forceinline__ uint64_t mul_pair(uint32_t w, uint64_t rr) {
-  const uint64_t x = ((uint64_t)(w & 0xFFFF0000u) << 32) | (uint64_t)(w << 16);
+// bf16 pair (element 2i in bits 0..15) -> fp32 pair (element 2i in the low word).
+__device__ __forceinline__ uint64_t bf16x2_to_f32x2(uint32_t w) {
+  return ((uint64_t)(w & 0xFFFF0000u) << 32) | (uint64_t)(w << 16);
+}
+
+__device__ __forceinline__ uint64_t mul_f32x2(uint64_t x, uint64_t rr) {
   uint64_t d;
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(x), "l"(rr));
   return d;
 }
 
-__device__ __forceinline__ uint32_t e2m1x4_from_pairs(uint64_t p0, uint64_t p1) {
+// Four fp32 pairs -> one word of eight E2M1 codes (element 2i in the low nibble
+// of byte i), round to nearest even, saturating at +-6.
+__device__ __forceinline__ uint32_t e2m1x8_from_pairs(uint64_t p0, uint64_t p1, uint64_t p2, uint64_t p3) {
   uint32_t out;
-  asm("{\n.reg .b8 b0, b1;\n.reg .f32 l0, h0, l1, h1;\n"
-      "mov.b64 {l0, h0}, %1;\nmov.b64 {l1, h1}, %2;\n"
-      "cvt.rn.satfinite.e2m1x2.f32 b0, h0, l0;\n"
-      "cvt.rn.satfinite.e2m1x2.f32 b1, h1, l1;\n"
-      "mov.b32 %0, {b0, b1, b0, b1};\n}"
-      : "=r"(out) : "l"(p0), "l"(p1));
-  return out & 0xFFFFu;
+  asm("{\n.reg .b8 b0, b1, b2, b3;\n.reg .f32 l0, h0, l1, h1, l2, h2, l3, h3;\n"
+      "mov.b64 {l0, h0}, %1;\nmov.b64 {l1, h1}, %2;\nmov.b64 {l2, h2}, %3;\nmov.b64 {l3, h3}, %4;\n"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, h0, l0;\ncvt.rn.satfinite.e2m1x2.f32 b1, h1, l1;\n"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, h2, l2;\ncvt.rn.satfinite.e2m1x2.f32 b3, h3, l3;\n"
+      "mov.b32 %0, {b0, b1, b2, b3};\n}"
+      : "=r"(out) : "l"(p0), "l"(p1), "l"(p2), "l"(p3));
+  return out;
+}
+
+// E4M3 byte -> fp32 through the hardware E4M3 -> f16 conversion (every E4M3
+// value is an f16 normal, so both steps are exact).
+__device__ __forceinline__ float e4m3_to_f32_hw(uint32_t s) {
+  float f;
+  asm("{\n.reg .b16 b, l, h;\n.reg .b32 w;\ncvt.u16.u32 b, %1;\ncvt.rn.f16x2.e4m3x2 w, b;\n"
+      "mov.b32 {l, h}, w;\ncvt.f32.f16 %0, l;\n}" : "=f"(f) : "r"(s));
+  return f;
 }
 
 __device__ __forceinline__ uint64_t sanitize_pair(uint64_t d) {
@@ -186,71 +194,94 @@ __device__ __forceinline__ uint64_t sanitize_pair(uint64_t d) {
   return ((uint64_t)__float_as_uint(hi) << 32) | __float_as_uint(lo);
 }
 
-// The 16-element block math (see the definition in include/nvfp4.h): block
-// amax, S = e4m3(a_b / (6 s_g)), r = 1/(S s_g), codes = e2m1(x r).  Returns
-// the 8 packed code bytes and S; flags non-finite input.
-__device__ __forceinline__ uint2 encode_block16(const uint4 &va, const uint4 &vb, float s_g, float t_g, bool real,
-                                                uint32_t &S, bool &bad) {
-  const uint32_t m = halves_max(absmax8_bits(vb, absmax8_bits(va, 0)));
-  if (real && m >= 0x7F80u) bad = true;
-  S = 0;
-  if (real) S = f32_to_e4m3_satfinite(__fdiv_rn(__uint_as_float(m << 16), t_g));
-  const float e = __fmul_rn(e4m3_to_f32(S), s_g);
+__device__ __forceinline__ uint32_t block_amax_bits(const uint4 &va, const uint4 &vb) {
+  return halves_max(absmax8_bits(vb, absmax8_bits(va, 0)));
+}
+
+// The block math (the definition in include/nvfp4.h) on a block already in
+// fp32 pairs with its amax a_b: S = e4m3(a_b / (6 s_g)), r = 1/(S s_g) (0 when
+// that product is 0), codes = e2m1(x r).
+__device__ __forceinline__ uint2 encode_f32x16(const uint64_t (&xf)[8], float a_b, float s_g, float t_g,
+                                               uint32_t &S) {
+  S = f32_to_e4m3_satfinite(__fdiv_rn(a_b, t_g));
+  const float e = __fmul_rn(e4m3_to_f32_hw(S), s_g);
   const float r = (e == 0.0f) ? 0.0f : __frcp_rn(e);
   const uint64_t rr = ((uint64_t)__float_as_uint(r) << 32) | __float_as_uint(r);
-  const uint32_t w[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
   uint64_t prod[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) prod[i] = mul_pair(w[i], rr);
+  for (int i = 0; i < 8; ++i) prod[i] = mul_f32x2(xf[i], rr);
   if (isinf(r)) {                     // 0 * inf: the NaN encodes as +0
 #pragma unroll
     for (int i = 0; i < 8; ++i) prod[i] = sanitize_pair(prod[i]);
   }
-  uint2 codes;
-  codes.x = e2m1x4_from_pairs(prod[0], prod[1]) | (e2m1x4_from_pairs(prod[2], prod[3]) << 16);
-  codes.y = e2m1x4_from_pairs(prod[4], prod[5]) | (e2m1x4_from_pairs(prod[6], prod[7]) << 16);
-  return codes;
+  return make_uint2(e2m1x8_from_pairs(prod[0], prod[1], prod[2], prod[3]),
+                    e2m1x8_from_pairs(prod[4], prod[5], prod[6], prod[7]));
 }
 
-// Gathered long rows (row_index, K >= 2048): one warp per output row, the row's group and source
-// row looked up once, up to 8 blocks (256 bytes) in flight per lane; warps
-// stride over rows so the grid streams through the input together.
+// Same, from the raw bf16 block; flags a non-finite element.
+__device__ __forceinline__ uint2 encode_block16(const uint4 &va, const uint4 &vb, float s_g, float t_g,
+                                                uint32_t &S, bool &bad) {
+  const uint32_t m = block_amax_bits(va, vb);
+  if (m >= 0x7F80u) bad = true;
+  const uint64_t xf[8] = {bf16x2_to_f32x2(va.x), bf16x2_to_f32x2(va.y), bf16x2_to_f32x2(va.z),
+                          bf16x2_to_f32x2(va.w), bf16x2_to_f32x2(vb.x), bf16x2_to_f32x2(vb.y),
+                          bf16x2_to_f32x2(vb.z), bf16x2_to_f32x2(vb.w)};
+  return encode_f32x16(xf, __uint_as_float(m << 16), s_g, t_g, S);
+}
+
+// Row part and block part of the MMA-tiled scale offset (they add up to
+// sf_tiled_offset(r, j, nsf)).
+__device__ __forceinline__ uint64_t sf_row_part(uint32_t r, uint32_t nsf) {
+  return (uint64_t)(r >> 7) * (nsf >> 2) * 512 + (r & 31) * 16 + ((r & 127) >> 5) * 4;
+}
+__device__ __forceinline__ uint32_t sf_blk_part(uint32_t j) { return (j >> 2) * 512 + (j & 3); }
+
+// n / d for 32-bit n by a multiply-high, with the constants of Granlund and
+// Montgomery, "Division by invariant integers using multiplication" (1994):
+// l = ceil(log2 d), m = floor(2^32 (2^l - d) / d) + 1, q = (mulhi(n, m) + n) >> l.
+struct FastDiv { uint32_t d, m, l; };
+FastDiv make_fastdiv(uint32_t d) {
+  uint32_t l = 0;
+  while (l < 32 && (1ull << l) < d) ++l;
+  const uint64_t m = (((1ull << 32) * ((1ull << l) - d)) / d) + 1;
+  return FastDiv{d, (uint32_t)m, l};
+}
+__device__ __forceinline__ uint32_t fast_div(uint32_t n, const FastDiv &f) {
+  return (uint32_t)(((uint64_t)__umulhi(n, f.m) + n) >> f.l);
+}
+
+// Gathered long rows (row_index, K >= 2048): one warp per result row, the
+// row's group and source row looked up once, up to 8 blocks (256 bytes) in
+// flight per lane; warps stride over rows so the grid streams through the
+// input together.  Only real rows are written (a slot's padding rows are not).
 template <bool kTiled>
 __global__ void __launch_bounds__(256) quantize_rows_kernel(
     const uint16_t *__restrict__ x, int64_t ld_x, int64_t K64, int64_t rows,
     const int32_t *__restrict__ row_index, const int32_t *__restrict__ group_offsets, int G,
-    int64_t P, const float *__restrict__ gs, uint8_t *__restrict__ q, uint8_t *__restrict__ sf,
-    int32_t *dev_status) {
+    const float *__restrict__ gs, uint8_t *__restrict__ q, uint8_t *__restrict__ sf, int32_t *dev_status) {
   extern __shared__ int32_t smem[];
   int32_t *off = smem, *slot = smem + (G + 1), *scratch = smem + 2 * (G + 1);
   if (group_offsets) load_groups(group_offsets, G, off, slot, scratch);
   const int lane = threadIdx.x & 31;
   const uint32_t K = (uint32_t)K64, nblk = K >> 4;
-  const uint32_t p_end = group_offsets ? (uint32_t)slot[G] : (uint32_t)P;
   const uint32_t warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
   const bool v8 = ((reinterpret_cast<uintptr_t>(x) & 31u) == 0) && ((ld_x & 15) == 0);
-  int g = 0;
   bool bad = false;
   constexpr int B = 8;
-  for (uint32_t p = warp; p < p_end; p += nwarps) {
-    bool real;
-    int64_t src;
+  for (uint32_t r = warp; r < (uint32_t)rows; r += nwarps) {
+    uint32_t p = r;
+    int g = 0;
     if (group_offsets) {
-      if (g + 8 < G && (uint32_t)slot[g + 8] <= p) g = upper_group(slot, G, p);
-      while (g + 1 < G && (uint32_t)slot[g + 1] <= p) ++g;
-      const uint32_t local = p - (uint32_t)slot[g];
-      real = local < (uint32_t)(off[g + 1] - off[g]);
-      src = (int64_t)off[g] + local;
-    } else {
-      real = p < (uint64_t)rows;
-      src = p;
+      g = upper_group(off, G, r);
+      p = (uint32_t)slot[g] + (r - (uint32_t)off[g]);
     }
-    if (real && row_index) src = row_index[src];
-    const float s_g = real ? gs[g] : 1.0f;
+    const int64_t src = row_index ? (int64_t)row_index[r] : (int64_t)r;
+    const float s_g = gs[g];
     const float t_g = __fmul_rn(6.0f, s_g);
     const uint16_t *xr = x + src * ld_x;
     uint8_t *qr = q + (uint64_t)p * (K >> 1);
+    const uint64_t rsf = kTiled ? sf_row_part(p, nblk) : (uint64_t)p * nblk;
     for (uint32_t j0 = 0; j0 < nblk; j0 += 32 * B) {
       uint4 va[B], vb[B];
 #pragma unroll
@@ -258,17 +289,16 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(
         const uint32_t j = j0 + k * 32 + lane;
         va[k] = make_uint4(0, 0, 0, 0);
         vb[k] = make_uint4(0, 0, 0, 0);
-        if (real && j < nblk) load_block(xr + (uint64_t)j * 16, v8, va[k], vb[k]);
+        if (j < nblk) load_block(xr + (uint64_t)j * 16, v8, va[k], vb[k]);
       }
 #pragma unroll
       for (int k = 0; k < B; ++k) {
         const uint32_t j = j0 + k * 32 + lane;
-        uint32_t S;
-        const uint2 codes = encode_block16(va[k], vb[k], s_g, t_g, real && j < nblk, S, bad);
         if (j < nblk) {
+          uint32_t S;
+          const uint2 codes = encode_block16(va[k], vb[k], s_g, t_g, S, bad);
           *reinterpret_cast<uint2 *>(qr + (uint64_t)j * 8) = codes;
-          if (kTiled) sf[sf_tiled_offset(p, j, nblk)] = (uint8_t)S;
-          else sf[(uint64_t)p * nblk + j] = (uint8_t)S;
+          sf[rsf + (kTiled ? sf_blk_part(j) : j)] = (uint8_t)S;
         }
       }
     }
@@ -276,82 +306,196 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(
   if (bad) report(dev_status, NVFP4_ERR_NONFINITE);
 }
 
+// General form: one thread per 16-element block of the real rows (routed
+// order), 64-block chunks, each warp a contiguous run of chunks so every
+// lane's row (and the row's group) only moves forward.  The block -> (row,
+// block) split is a multiply-high division; only real rows are written.
 template <bool kTiled>
 __global__ void __launch_bounds__(256) quantize_kernel(
     const uint16_t *__restrict__ x, int64_t ld_x, int64_t K64, int64_t rows,
     const int32_t *__restrict__ row_index, const int32_t *__restrict__ group_offsets, int G,
-    int64_t P, const float *__restrict__ gs, uint8_t *__restrict__ q, uint8_t *__restrict__ sf,
+    const float *__restrict__ gs, uint8_t *__restrict__ q, uint8_t *__restrict__ sf, FastDiv fd,
     int32_t *dev_status) {
   extern __shared__ int32_t smem[];
   int32_t *off = smem, *slot = smem + (G + 1), *scratch = smem + 2 * (G + 1);
   if (group_offsets) load_groups(group_offsets, G, off, slot, scratch);
   const int lane = threadIdx.x & 31;
   const uint32_t K = (uint32_t)K64, nblk = K >> 4;
-  const uint32_t p_end = group_offsets ? (uint32_t)slot[G] : (uint32_t)P;
-  const uint64_t total = (uint64_t)p_end * nblk;             // blocks, row-major
+  const uint32_t total = (uint32_t)rows * nblk;              // < 2^32 (host check)
   constexpr int U = 2;                                       // 32-block steps per chunk
-  const uint64_t nchunks = (total + 32 * U - 1) / (32 * U);
-  const uint64_t warp = ((uint64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const uint64_t nwarps = ((uint64_t)gridDim.x * blockDim.x) >> 5;
-  const bool small = total < 0xFFFFFFF0ull;
+  const uint32_t nchunks = (total + 32 * U - 1) / (32 * U);
+  const uint32_t warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
+  const uint32_t per = (nchunks + nwarps - 1) / nwarps;
+  const uint32_t c_begin = min(nchunks, warp * per), c_end = min(nchunks, c_begin + per);
+  if (c_begin >= c_end) return;
   const bool v8 = ((reinterpret_cast<uintptr_t>(x) & 31u) == 0) && ((ld_x & 15) == 0);
-  int g = 0;
-  uint32_t cached_p = 0xFFFFFFFFu;
-  int64_t cached_src = -1;
-  bool cached_real = false;
-  float s_g = 1.0f, t_g = 6.0f;
-  int g_for_scale = -1;
+  int g = group_offsets ? upper_group(off, G, fast_div(c_begin * (32 * U), fd)) : 0;
+  uint32_t cached_r = 0xFFFFFFFFu, p = 0;
+  int64_t src = 0;
+  uint64_t rsf = 0;
+  float s_g = gs[g], t_g = __fmul_rn(6.0f, s_g);
   bool bad = false;
-  for (uint64_t c = warp; c < nchunks; c += nwarps) {
+  for (uint32_t c = c_begin; c < c_end; ++c) {
     uint4 va[U], vb[U];
     uint32_t pp[U], jj[U];
-    bool real[U], inr[U];
+    uint64_t rs[U];
+    bool inr[U];
     float sg[U], tg[U];
 #pragma unroll
     for (int k = 0; k < U; ++k) {
-      const uint64_t b = c * (32 * U) + k * 32 + lane;
+      const uint32_t b = c * (32 * U) + k * 32 + lane;
       inr[k] = b < total;
-      uint32_t p = 0, j = 0;
+      uint32_t r = 0, j = 0;
       if (inr[k]) {
-        if (small) { p = (uint32_t)b / nblk; j = (uint32_t)b - p * nblk; }
-        else { p = (uint32_t)(b / nblk); j = (uint32_t)(b - (uint64_t)p * nblk); }
-        if (p != cached_p) {
-          cached_p = p;
+        r = fast_div(b, fd);
+        j = b - r * nblk;
+        if (r != cached_r) {
+          cached_r = r;
           if (group_offsets) {
-            if (g + 8 < G && (uint32_t)slot[g + 8] <= p) g = upper_group(slot, G, p);
-            while (g + 1 < G && (uint32_t)slot[g + 1] <= p) ++g;
-            const uint32_t local = p - (uint32_t)slot[g];
-            cached_real = local < (uint32_t)(off[g + 1] - off[g]);
-            cached_src = (int64_t)off[g] + local;
+            const int g0 = g;
+            while (g + 1 < G && off[g + 1] <= (int32_t)r) ++g;
+            p = (uint32_t)slot[g] + (r - (uint32_t)off[g]);
+            if (g != g0) { s_g = gs[g]; t_g = __fmul_rn(6.0f, s_g); }
           } else {
-            cached_real = p < (uint64_t)rows;
-            cached_src = p;
+            p = r;
           }
-          if (cached_real && row_index) cached_src = row_index[cached_src];
-          if (g != g_for_scale) {
-            g_for_scale = g;
-            s_g = gs[g];
-            t_g = __fmul_rn(6.0f, s_g);
-          }
+          src = row_index ? (int64_t)row_index[r] : (int64_t)r;
+          rsf = kTiled ? sf_row_part(p, nblk) : (uint64_t)p * nblk;
         }
       }
       pp[k] = p;
       jj[k] = j;
-      real[k] = inr[k] && cached_real;
+      rs[k] = rsf;
       sg[k] = s_g;
       tg[k] = t_g;
       va[k] = make_uint4(0, 0, 0, 0);
       vb[k] = make_uint4(0, 0, 0, 0);
-      if (real[k]) load_block(x + cached_src * ld_x + (uint64_t)j * 16, v8, va[k], vb[k]);
+      if (inr[k]) load_block(x + src * ld_x + (uint64_t)j * 16, v8, va[k], vb[k]);
     }
 #pragma unroll
     for (int k = 0; k < U; ++k) {
-      uint32_t S;
-      const uint2 codes = encode_block16(va[k], vb[k], sg[k], tg[k], real[k], S, bad);
       if (inr[k]) {
+        uint32_t S;
+        const uint2 codes = encode_block16(va[k], vb[k], sg[k], tg[k], S, bad);
         *reinterpret_cast<uint2 *>(q + (uint64_t)pp[k] * (K >> 1) + (uint64_t)jj[k] * 8) = codes;
-        if (kTiled) sf[sf_tiled_offset(pp[k], jj[k], nblk)] = (uint8_t)S;
-        else sf[(uint64_t)pp[k] * nblk + jj[k]] = (uint8_t)S;
+        sf[rs[k] + (kTiled ? sf_blk_part(jj[k]) : jj[k])] = (uint8_t)S;
+      }
+    }
+  }
+  if (bad) report(dev_status, NVFP4_ERR_NONFINITE);
+}
+
+// ---------------------------------------------------------------- MoE dispatch quantize
+// Token-major form of the gathered per-expert quantize.  A token routed to k
+// experts appears in k routed rows with the same 16-element blocks; only the
+// global scale differs.  So each token row is read once: the block amaxes and
+// the fp32 form of the block are taken once and each of the token's k copies
+// is encoded with its expert's s_g and written to its packed row.
+// slot[t*k + c] is the routed row of the token's c-th choice (-1: not routed);
+// a lane per choice holds its expert's packed row and global scale.
+
+// Pass 1: each warp takes a token, forms max|x| of the row (up to 8 32-byte
+// loads in flight per lane), and raises the amax of every expert the token is
+// routed to.
+__global__ void __launch_bounds__(256) moe_amax_kernel(
+    const uint16_t *__restrict__ x, int64_t ld_x, int64_t K, int64_t tokens, const int32_t *__restrict__ slot,
+    int topk, const int32_t *__restrict__ group_offsets, int G, uint32_t *__restrict__ amax_bits,
+    int32_t *dev_status) {
+  extern __shared__ int32_t smem[];
+  int32_t *off = smem;
+  for (int i = threadIdx.x; i <= G; i += blockDim.x) off[i] = group_offsets[i];
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const uint32_t nblk = (uint32_t)(K >> 4);
+  const bool v8 = ((reinterpret_cast<uintptr_t>(x) & 31u) == 0) && ((ld_x & 15) == 0);
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  constexpr int B = 8;
+  for (int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < tokens; t += nwarps) {
+    const uint16_t *row = x + t * ld_x;
+    uint32_t m = 0;
+    for (uint32_t j0 = 0; j0 < nblk; j0 += 32 * B) {
+      uint4 va[B], vb[B];
+#pragma unroll
+      for (int k = 0; k < B; ++k) {
+        const uint32_t j = j0 + k * 32 + lane;
+        va[k] = make_uint4(0, 0, 0, 0);
+        vb[k] = make_uint4(0, 0, 0, 0);
+        if (j < nblk) load_block(row + (uint64_t)j * 16, v8, va[k], vb[k]);
+      }
+#pragma unroll
+      for (int k = 0; k < B; ++k) m = absmax8_bits(vb[k], absmax8_bits(va[k], m));
+    }
+    const uint32_t mm = warp_max(halves_max(m));
+    if (lane < topk) {
+      const int32_t r = slot[t * topk + lane];
+      if (r >= off[G]) report(dev_status, NVFP4_ERR_INDEX);
+      else if (r >= 0 && mm) atomicMax(&amax_bits[upper_group(off, G, r)], mm << 16);
+    }
+  }
+}
+
+// Pass 2: a warp per token, 4 blocks in flight per lane, held as fp32 pairs
+// across the token's k encodes.
+template <bool kTiled>
+__global__ void __launch_bounds__(256, 2) moe_encode_kernel(
+    const uint16_t *__restrict__ x, int64_t ld_x, int64_t K64, int64_t tokens, const int32_t *__restrict__ slot,
+    int topk, const int32_t *__restrict__ group_offsets, int G, const float *__restrict__ gs,
+    uint8_t *__restrict__ q, uint8_t *__restrict__ sf, int32_t *dev_status) {
+  extern __shared__ int32_t smem[];
+  int32_t *off = smem, *pslot = smem + (G + 1), *scratch = smem + 2 * (G + 1);
+  load_groups(group_offsets, G, off, pslot, scratch);
+  const int lane = threadIdx.x & 31;
+  const uint32_t K = (uint32_t)K64, nblk = K >> 4;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  const bool v8 = ((reinterpret_cast<uintptr_t>(x) & 31u) == 0) && ((ld_x & 15) == 0);
+  bool bad = false;
+  constexpr int B = 4;
+  for (int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < tokens; t += nwarps) {
+    int32_t my_p = -1;
+    float my_sg = 1.0f;
+    if (lane < topk) {
+      const int32_t r = slot[t * topk + lane];
+      if (r >= 0 && r < off[G]) {
+        const int e = upper_group(off, G, r);
+        my_p = pslot[e] + (r - off[e]);
+        my_sg = gs[e];
+      }
+    }
+    const uint16_t *xr = x + t * ld_x;
+    for (uint32_t j0 = 0; j0 < nblk; j0 += 32 * B) {
+      uint64_t xf[B][8];
+      float amf[B];
+#pragma unroll
+      for (int k = 0; k < B; ++k) {
+        const uint32_t j = j0 + k * 32 + lane;
+        uint4 va = make_uint4(0, 0, 0, 0), vb = make_uint4(0, 0, 0, 0);
+        if (j < nblk) load_block(xr + (uint64_t)j * 16, v8, va, vb);
+        const uint32_t m = block_amax_bits(va, vb);
+        if (m >= 0x7F80u) bad = true;
+        amf[k] = __uint_as_float(m << 16);
+        xf[k][0] = bf16x2_to_f32x2(va.x); xf[k][1] = bf16x2_to_f32x2(va.y);
+        xf[k][2] = bf16x2_to_f32x2(va.z); xf[k][3] = bf16x2_to_f32x2(va.w);
+        xf[k][4] = bf16x2_to_f32x2(vb.x); xf[k][5] = bf16x2_to_f32x2(vb.y);
+        xf[k][6] = bf16x2_to_f32x2(vb.z); xf[k][7] = bf16x2_to_f32x2(vb.w);
+      }
+      for (int c = 0; c < topk; ++c) {
+        const int32_t p = __shfl_sync(0xffffffffu, my_p, c);
+        const float s_g = __shfl_sync(0xffffffffu, my_sg, c);
+        if (p < 0) continue;
+        const float t_g = __fmul_rn(6.0f, s_g);
+        uint8_t *qr = q + (uint64_t)p * (K >> 1);
+        const uint64_t rsf = kTiled ? sf_row_part((uint32_t)p, nblk) : (uint64_t)p * nblk;
+#pragma unroll
+        for (int k = 0; k < B; ++k) {
+          const uint32_t j = j0 + k * 32 + lane;
+          if (j < nblk) {
+            uint32_t S;
+            const uint2 codes = encode_f32x16(xf[k], amf[k], s_g, t_g, S);
+            *reinterpret_cast<uint2 *>(qr + (uint64_t)j * 8) = codes;
+            sf[rsf + (kTiled ? sf_blk_part(j) : j)] = (uint8_t)S;
+          }
+        }
       }
     }
   }
@@ -579,31 +723,41 @@ nvfp4_status run_encode(const uint16_t *x, int64_t rows, int64_t K, int64_t ld_x
                         const float *gs, uint8_t *q, uint8_t *sf, nvfp4_sf_layout layout,
                         int32_t *dev_status, cudaStream_t stream) {
   const bool tiled = layout == NVFP4_SF_MMA_TILED;
-  int64_t P;
-  if (group_offsets) P = nvfp4_padded_rows_bound(rows, G);
-  else P = tiled ? (rows + 127) / 128 * 128 : rows;
-  if (P == 0) return NVFP4_OK;
-  const int64_t blocks = P * (K / 16);
+  if (rows == 0) return NVFP4_OK;
   const size_t sm = group_offsets ? sizeof(int32_t) * (2 * (G + 1) + 8) : 0;
-  if (row_index && K >= 2048 && P <= 0xFFFFFFFFll) {
-    // one warp per output row
+  if (row_index && K >= 2048) {
+    // one warp per result row
     if (tiled) {
-      const unsigned grid = (unsigned)grid_resident(quantize_rows_kernel<true>, P * 32, 256, sm);
-      quantize_rows_kernel<true><<<grid, 256, sm, stream>>>(x, ld_x, K, rows, row_index, group_offsets, G, P, gs, q, sf, dev_status);
+      const unsigned grid = (unsigned)grid_resident(quantize_rows_kernel<true>, rows * 32, 256, sm);
+      quantize_rows_kernel<true><<<grid, 256, sm, stream>>>(x, ld_x, K, rows, row_index, group_offsets, G, gs, q, sf, dev_status);
     } else {
-      const unsigned grid = (unsigned)grid_resident(quantize_rows_kernel<false>, P * 32, 256, sm);
-      quantize_rows_kernel<false><<<grid, 256, sm, stream>>>(x, ld_x, K, rows, row_index, group_offsets, G, P, gs, q, sf, dev_status);
+      const unsigned grid = (unsigned)grid_resident(quantize_rows_kernel<false>, rows * 32, 256, sm);
+      quantize_rows_kernel<false><<<grid, 256, sm, stream>>>(x, ld_x, K, rows, row_index, group_offsets, G, gs, q, sf, dev_status);
     }
     return launch_status();
   }
-  if (tiled) {
-    const unsigned grid = (unsigned)grid_resident(quantize_kernel<true>, (blocks + 1) / 2, 256, sm);
-    quantize_kernel<true><<<grid, 256, sm, stream>>>(x, ld_x, K, rows, row_index, group_offsets, G, P, gs, q, sf, dev_status);
-  } else {
-    const unsigned grid = (unsigned)grid_resident(quantize_kernel<false>, (blocks + 1) / 2, 256, sm);
-    quantize_kernel<false><<<grid, 256, sm, stream>>>(x, ld_x, K, rows, row_index, group_offsets, G, P, gs, q, sf, dev_status);
+  const int64_t nblk = K / 16;
+  const FastDiv fd = make_fastdiv((uint32_t)nblk);
+  // the block index is 32-bit: one launch covers fewer than 2^32 - 64 blocks;
+  // a larger ungrouped tensor goes in pieces of whole 128-row tiles
+  const int64_t max_rows = ((int64_t)0xFFFFFFC0ll / nblk) / 128 * 128;
+  if (rows > max_rows && (group_offsets || row_index)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  for (int64_t r0 = 0; r0 < rows; r0 += max_rows) {
+    const int64_t n = rows - r0 < max_rows ? rows - r0 : max_rows;
+    const uint16_t *xp = x + r0 * ld_x;
+    uint8_t *qp = q + r0 * (K / 2);
+    uint8_t *sp = sf + (tiled ? (r0 / 128) * (nblk / 4) * 512 : r0 * nblk);
+    const int64_t work = (n * nblk + 1) / 2;
+    if (tiled) {
+      const unsigned grid = (unsigned)grid_resident(quantize_kernel<true>, work, 256, sm);
+      quantize_kernel<true><<<grid, 256, sm, stream>>>(xp, ld_x, K, n, row_index, group_offsets, G, gs, qp, sp, fd, dev_status);
+    } else {
+      const unsigned grid = (unsigned)grid_resident(quantize_kernel<false>, work, 256, sm);
+      quantize_kernel<false><<<grid, 256, sm, stream>>>(xp, ld_x, K, n, row_index, group_offsets, G, gs, qp, sp, fd, dev_status);
+    }
+    if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_CUDA;
   }
-  return launch_status();
+  return NVFP4_OK;
 }
 
 }  // namespace
@@ -659,6 +813,49 @@ nvfp4_status nvfp4_quantize(const void *x, int64_t rows, int64_t K, int64_t ld_x
   if (st != NVFP4_OK) return st;
   return run_encode(xb, rows, K, ld_x, row_index, group_offsets, G, global_scale, q, sf, sf_layout,
                     dev_status, stream);
+}
+
+nvfp4_status nvfp4_moe_quantize(const void *x, int64_t tokens, int64_t K, int64_t ld_x, const int32_t *slot,
+                                int topk, const int32_t *group_offsets, int num_groups, nvfp4_gs_mode gs_mode,
+                                float *global_scale, uint8_t *q, uint8_t *sf, nvfp4_sf_layout sf_layout,
+                                void *workspace, int32_t *dev_status, cudaStream_t stream) {
+  if (tokens < 0 || K <= 0 || ld_x < K || topk < 1 || topk > 32) return NVFP4_ERR_INVALID_ARG;
+  if (K % 16 != 0 || ld_x % 8 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (sf_layout != NVFP4_SF_ROWMAJOR && sf_layout != NVFP4_SF_MMA_TILED) return NVFP4_ERR_INVALID_ARG;
+  if (sf_layout == NVFP4_SF_MMA_TILED && K % 64 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (gs_mode != NVFP4_GS_FROM_AMAX && gs_mode != NVFP4_GS_GIVEN && gs_mode != NVFP4_GS_AMAX_GIVEN)
+    return NVFP4_ERR_INVALID_ARG;
+  const int G = num_groups;
+  if (!group_offsets || G < 1 || G > kMaxGroups) return NVFP4_ERR_INVALID_ARG;
+  if (!global_scale || !workspace || !aligned16(workspace)) return NVFP4_ERR_INVALID_ARG;
+  if (tokens > 0 && (!x || !slot || !q || !sf || !aligned16(x) || !aligned16(q))) return NVFP4_ERR_INVALID_ARG;
+  if (tokens * topk > ((int64_t)1 << 31)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  const uint16_t *xb = reinterpret_cast<const uint16_t *>(x);
+  uint32_t *amax_bits = reinterpret_cast<uint32_t *>(workspace);
+  if (gs_mode == NVFP4_GS_FROM_AMAX) {
+    if (cudaMemsetAsync(amax_bits, 0, sizeof(uint32_t) * G, stream) != cudaSuccess) return NVFP4_ERR_CUDA;
+    if (tokens > 0) {
+      const size_t sm = sizeof(int32_t) * (G + 1);
+      const unsigned grid = (unsigned)grid_resident(moe_amax_kernel, tokens * 32, 256, sm);
+      moe_amax_kernel<<<grid, 256, sm, stream>>>(xb, ld_x, K, tokens, slot, topk, group_offsets, G, amax_bits,
+                                                 dev_status);
+      if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_CUDA;
+    }
+  }
+  finalize_scales_kernel<<<(G + 127) / 128, 128, 0, stream>>>(amax_bits, G, (int)gs_mode, global_scale, dev_status);
+  if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_CUDA;
+  if (tokens == 0) return NVFP4_OK;
+  const size_t sm = sizeof(int32_t) * (2 * (G + 1) + 8);
+  if (sf_layout == NVFP4_SF_MMA_TILED) {
+    const unsigned grid = (unsigned)grid_resident(moe_encode_kernel<true>, tokens * 32, 256, sm);
+    moe_encode_kernel<true><<<grid, 256, sm, stream>>>(xb, ld_x, K, tokens, slot, topk, group_offsets, G,
+                                                       global_scale, q, sf, dev_status);
+  } else {
+    const unsigned grid = (unsigned)grid_resident(moe_encode_kernel<false>, tokens * 32, 256, sm);
+    moe_encode_kernel<false><<<grid, 256, sm, stream>>>(xb, ld_x, K, tokens, slot, topk, group_offsets, G,
+                                                        global_scale, q, sf, dev_status);
+  }
+  return launch_status();
 }
 
 nvfp4_status nvfp4_dequantize(const uint8_t *q, const uint8_t *sf, nvfp4_sf_layout sf_layout,

@@ -15,7 +15,8 @@ import torch
 
 from . import (EPI_NONE, EPI_SWIGLU, GS_AMAX_GIVEN, GS_FROM_AMAX, GS_GIVEN, OUT_BF16, OUT_F32, SF_MMA_TILED, SF_ROWMAJOR,
                mxfp4_to_nvfp4, nvfp4_dequantize, nvfp4_grouped_gemm, nvfp4_moe_combine, nvfp4_moe_route,
-               nvfp4_moe_route_workspace_size, nvfp4_padded_rows_bound, nvfp4_quantize, nvfp4_swiglu_quantize,
+               nvfp4_moe_quantize, nvfp4_moe_route_workspace_size, nvfp4_padded_rows_bound, nvfp4_quantize,
+               nvfp4_swiglu_quantize,
                nvfp4_workspace_size)
 
 
@@ -76,6 +77,23 @@ def quantize(x: torch.Tensor, row_index=None, offsets=None, num_groups: int = 1,
         mode = GS_GIVEN
     ws = ws if ws is not None else workspace(G, x.device)
     nvfp4_quantize(x, R, K, x.stride(0), row_index, offsets, G, mode, p.gs, p.q, p.sf, layout, ws, dev_status)
+    return p
+
+
+def moe_quantize(x: torch.Tensor, slot: torch.Tensor, offsets: torch.Tensor, num_groups: int, layout=SF_MMA_TILED,
+                 out: Optional[Packed] = None, ws=None, dev_status=None, rows=None) -> Packed:
+    """Routed-expert activations quantized in token order: the same packed rows
+    as ``quantize(x, row_index, offsets, ...)`` with row_index the inverse of
+    ``slot`` [T, k] (routed row of each token choice), each token read once."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and slot.dim() == 2
+    T, k = slot.shape
+    K = x.shape[1]
+    R = rows if rows is not None else T * k
+    p = out if out is not None else empty_packed(R, K, num_groups, offsets, layout, x.device)
+    p.offsets, p.num_groups, p.rows = offsets, num_groups, R
+    ws = ws if ws is not None else workspace(num_groups, x.device)
+    nvfp4_moe_quantize(x, T, K, x.stride(0), slot, k, offsets, num_groups, GS_FROM_AMAX, p.gs, p.q, p.sf, layout,
+                       ws, dev_status)
     return p
 
 
@@ -190,11 +208,19 @@ class MoEExperts:
         self.y2 = torch.empty((max_rows, H), dtype=odt, device=device)
         self.max_rows = max_rows
 
-    def forward(self, x: torch.Tensor, row_index: torch.Tensor, offsets: torch.Tensor, dev_status=None):
+    def forward(self, x: torch.Tensor, row_index: torch.Tensor, offsets: torch.Tensor, dev_status=None,
+                slot: Optional[torch.Tensor] = None):
+        """``slot`` [T, k] (routed row of each token choice), when given, selects
+        the token-order quantize that reads each token row once."""
         R = row_index.shape[0]
         assert R <= self.max_rows
         E, H, I = self.E, self.H, self.I
-        a1 = quantize(x, row_index, offsets, E, SF_MMA_TILED, out=self.a1, ws=self.ws, dev_status=dev_status, rows=R)
+        if slot is not None:
+            a1 = moe_quantize(x, slot, offsets, E, SF_MMA_TILED, out=self.a1, ws=self.ws, dev_status=dev_status,
+                              rows=R)
+        else:
+            a1 = quantize(x, row_index, offsets, E, SF_MMA_TILED, out=self.a1, ws=self.ws, dev_status=dev_status,
+                          rows=R)
         if self.fused_swiglu:
             # SwiGLU in the gate_up epilogue; its amax feeds the requantize directly
             h, amax = grouped_gemm_swiglu(a1, self.w_gate_up, 2 * I, h=self.h[:R], amax=self.amax,
@@ -261,7 +287,7 @@ class MoELayer:
         slot = self.slot[:T]
         ri = self.ri[:T * k]
         nvfp4_moe_route(topk_ids, T, k, E, self.off, ri, slot, self.rws, dev_status)
-        y = self.experts.forward(x, ri, self.off, dev_status)
+        y = self.experts.forward(x, ri, self.off, dev_status, slot=slot)
         out = self.out[:T]
         nvfp4_moe_combine(y, OUT_F32 if y.dtype == torch.float32 else OUT_BF16, slot, topk_weights, T, k,
                           self.experts.H, out, OUT_BF16)

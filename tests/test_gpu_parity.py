@@ -70,7 +70,10 @@ def test_quantize_grouped_gather_bitexact(layout, H):
     q_ref, sf_ref, gs_ref, st = oracle.quantize(x, r["row_index"], r["offsets"])
     assert st == 0
     off = to_dev(r["offsets"])
-    p = L.quantize(bf16_dev(x), to_dev(r["row_index"]), off, E, layout=layout)
+    out = L.empty_packed(T * k, H, E, off, layout)
+    out.q.fill_(0xAB)                       # padding rows must keep this: they are not written
+    out.sf.fill_(0xAB)
+    p = L.quantize(bf16_dev(x), to_dev(r["row_index"]), off, E, layout=layout, out=out)
     torch.cuda.synchronize()
     assert np.array_equal(to_np(p.gs), gs_ref)
     rows, starts = slot_rows(r["offsets"])
@@ -78,11 +81,85 @@ def test_quantize_grouped_gather_bitexact(layout, H):
     q = to_np(p.q)
     assert np.array_equal(q[rows], q_ref)
     pad = np.setdiff1d(np.arange(used), rows)
-    assert (q[pad] == 0).all()
+    assert (q[pad] == 0xAB).all()
     sf = to_np(p.sf)
     sfm = untile(sf, p.q.shape[0], H // 16) if layout == 1 else sf.reshape(-1, H // 16)
     assert np.array_equal(sfm[rows], sf_ref)
-    assert (sfm[pad] == 0).all()
+    assert (sfm[pad] == 0xAB).all()
+
+
+# --------------------------------------------------------------------------- token-order MoE quantize
+def _moe_quantize_check(x, slot, off, E, layout, x_dev=None):
+    """nvfp4_moe_quantize against the oracle's gathered per-expert quantize
+    (row_index = inverse of slot): bit-exact in every routed row."""
+    L = layer()
+    R = int(off[-1])
+    t, c = np.nonzero(slot >= 0)
+    ri = np.full(R, -1, np.int64)
+    ri[slot[t, c]] = t
+    assert (ri >= 0).all()
+    q_ref, sf_ref, gs_ref, st = oracle.quantize(x, ri.astype(np.int32), off)
+    assert st == 0
+    s = status_word()
+    K = x.shape[1]
+    out = L.empty_packed(R, K, E, to_dev(off), layout)
+    out.q.fill_(0xAB)
+    out.sf.fill_(0xAB)
+    p = L.moe_quantize(bf16_dev(x) if x_dev is None else x_dev, to_dev(slot.astype(np.int32)), to_dev(off), E,
+                       layout=layout, out=out, dev_status=s)
+    torch.cuda.synchronize()
+    assert int(s.item()) == 0
+    assert np.array_equal(to_np(p.gs), gs_ref)
+    rows, starts = slot_rows(off)
+    q = to_np(p.q)
+    assert np.array_equal(q[rows], q_ref)
+    pad = np.setdiff1d(np.arange(int(starts[-1])), rows)
+    assert (q[pad] == 0xAB).all()
+    sf = to_np(p.sf)
+    sfm = untile(sf, p.q.shape[0], K // 16) if layout == 1 else sf.reshape(-1, K // 16)
+    assert np.array_equal(sfm[rows], sf_ref)
+    assert (sfm[pad] == 0xAB).all()
+
+
+@pytest.mark.parametrize("layout,T,H,E,k", [(1, 1024, 512, 12, 2), (0, 1024, 2064, 12, 2), (1, 300, 7168, 40, 8),
+                                            (1, 2048, 4096, 64, 10), (0, 5, 64, 3, 3), (1, 8192, 4096, 512, 10)])
+def test_moe_quantize_bitexact(layout, T, H, E, k):
+    x = synthetic.gaussian_bf16(21, synthetic.STREAMS["x"], (T, H), outlier_frac=0.001)
+    r = synthetic.route_topk_softmax(21, T, E, k)
+    _moe_quantize_check(x, r["slot"], r["offsets"], E, layout)
+
+
+def test_moe_quantize_strided_rows():
+    """ld_x = K + 8 (rows not 32-byte aligned: the two 16-byte load path)."""
+    T, H, E, k = 333, 512, 7, 3
+    xw = synthetic.gaussian_bf16(22, synthetic.STREAMS["x"], (T, H + 8), outlier_frac=0.01)
+    r = synthetic.route_topk_softmax(22, T, E, k)
+    xd = bf16_dev(xw)[:, :H]
+    _moe_quantize_check(np.ascontiguousarray(xw[:, :H]), r["slot"], r["offsets"], E, 0, x_dev=xd)
+
+
+def test_moe_quantize_dropped_choices_and_bad_index():
+    """Choices with slot -1 are skipped; a slot beyond the routed rows is
+    reported as an index error and skipped."""
+    L = layer()
+    T, H, E, k = 200, 256, 6, 3
+    x = synthetic.gaussian_bf16(23, synthetic.STREAMS["x"], (T, H))
+    experts = synthetic.route_topk_softmax(23, T, E, k)["experts"].astype(np.int64)
+    rng = np.random.default_rng(23)
+    experts[rng.random((T, k)) < 0.15] = -1
+    t, c = np.nonzero(experts >= 0)
+    e = experts[t, c]
+    order = np.lexsort((c, t, e))
+    slot = np.full((T, k), -1, np.int64)
+    slot[t[order], c[order]] = np.arange(len(order))
+    off = np.concatenate([[0], np.cumsum(np.bincount(e, minlength=E))]).astype(np.int32)
+    _moe_quantize_check(x, slot, off, E, 1)
+    bad = slot.copy()
+    bad[0, np.argmax(bad[0] >= 0)] = int(off[-1]) + 3
+    s = status_word()
+    L.moe_quantize(bf16_dev(x), to_dev(bad.astype(np.int32)), to_dev(off), E, layout=1, dev_status=s)
+    torch.cuda.synchronize()
+    assert int(s.item()) == 19
 
 
 def test_quantize_groups_with_empty_experts():
@@ -481,10 +558,13 @@ def test_moe_layer_fused_swiglu_stagewise():
     Wd = L.Packed(to_dev(qd), to_dev(tile(sd)), to_dev(gd), E * H, I, 1)
     moe = L.MoEExperts(Wgu, Wd, E, H, I, max_rows=R, out_dtype=0, mid_dtype=0, fused_swiglu=True)
     s = status_word()
-    y2 = moe.forward(bf16_dev(x), to_dev(r["row_index"]), to_dev(off), dev_status=s)
+    y2 = moe.forward(bf16_dev(x), to_dev(r["row_index"]), to_dev(off), dev_status=s,
+                     slot=to_dev(r["slot"].astype(np.int32)))
     torch.cuda.synchronize()
     assert int(s.item()) == 0
     rows, _ = slot_rows(off)
+    q1_ref, _, gs1_ref, _ = oracle.quantize(x, r["row_index"], off)     # stage 1 (token-order quantize)
+    assert np.array_equal(to_np(moe.a1.gs), gs1_ref) and np.array_equal(to_np(moe.a1.q)[rows], q1_ref)
     h = to_np(moe.h[:R])
     # stage 1+2: h against silu(g)*u of the fp64 gate_up GEMM on the oracle's
     # quantized operands (gate/up rows put back in source order).  Bound: the
