@@ -228,6 +228,18 @@ nvfp4_status nvfp4_grouped_gemm(const uint8_t *a_q, const uint8_t *a_sf, const f
                                 void *workspace, int32_t *dev_status, cudaStream_t stream);
 
 /*
+ * nvfp4_gemm_select_kernel -- which grouped GEMM kernel nvfp4_grouped_gemm runs
+ * (process-wide; a tuning and testing switch, not part of the pages' method):
+ *   0  automatic (default): one CTA per 128-row weight tile (measured as fast
+ *      as or faster than the pair kernel on the MoE shapes);
+ *   1  one CTA per tile;  2  CTA pairs (tcgen05 cta_group::2, 256 weight rows
+ *      per tile; N % 256 != 0 is then NVFP4_ERR_UNSUPPORTED_SHAPE).
+ * Both give the same Y up to the fp32 accumulation order inside a tile.
+ * Returns NVFP4_ERR_INVALID_ARG for another mode.
+ */
+nvfp4_status nvfp4_gemm_select_kernel(int mode);
+
+/*
  * nvfp4_swiglu_quantize -- the step between the two expert projections:
  * h = bf16(silu(g) * u) with g = y[:, :I] (gate rows of the fused gate_up
  * weight come first) and u = y[:, I:], then h is NVFP4-quantized per expert

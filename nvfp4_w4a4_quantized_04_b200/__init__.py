@@ -46,6 +46,7 @@ EXPORTS = [
     "nvfp4_quantize", "nvfp4_dequantize", "mxfp4_to_nvfp4", "nvfp4_grouped_gemm",
     "nvfp4_swiglu_quantize", "nvfp4_kv_quantize", "nvfp4_kv_dequantize", "nvfp4_quantize_noalloc",
     "nvfp4_moe_route_workspace_size", "nvfp4_moe_route", "nvfp4_moe_combine", "nvfp4_moe_quantize",
+    "nvfp4_gemm_select_kernel",
 ]
 NOALLOC_MAX_GROUPS = 1024
 
@@ -73,6 +74,8 @@ def load_library(path: str = LIB_PATH):
     L.nvfp4_padded_rows_bound.argtypes = [i64, i32]
     L.nvfp4_quantize.restype = i32
     L.nvfp4_quantize.argtypes = [P, i64, i64, i64, P, P, i32, i32, P, P, P, i32, P, P, P]
+    L.nvfp4_gemm_select_kernel.restype = i32
+    L.nvfp4_gemm_select_kernel.argtypes = [i32]
     L.nvfp4_moe_quantize.restype = i32
     L.nvfp4_moe_quantize.argtypes = [P, i64, i64, i64, P, i32, P, i32, i32, P, P, P, i32, P, P, P]
     L.nvfp4_dequantize.restype = i32
@@ -146,6 +149,13 @@ def nvfp4_quantize_noalloc(x, rows, K, ld_x, row_index, group_offsets, num_group
         _ptr(global_scale), _ptr(q), _ptr(sf), sf_layout, _ptr(dev_status), _stream(stream))
     if check:
         _check(st, "nvfp4_quantize_noalloc")
+    return st
+
+
+def nvfp4_gemm_select_kernel(mode: int) -> int:
+    """0 automatic (one CTA per tile), 1 one CTA per tile, 2 CTA pairs (N % 256 == 0)."""
+    st = load_library().nvfp4_gemm_select_kernel(mode)
+    _check(st, "nvfp4_gemm_select_kernel")
     return st
 
 

@@ -1,0 +1,597 @@
+// Shared pieces of the block-scaled FP4 grouped GEMM kernels (sm_100a): the
+// tile constants, PTX wrappers for mbarriers, TMA and the tcgen05 tensor-core
+// instructions, the expert/tile tables, the scale-factor copy into tensor
+// memory and the accumulator epilogue.  Included by gemm.cu (one CTA per
+// tile) and gemm_pair.cu (a CTA pair per tile, cta_group::2).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace nvfp4 {
+namespace gemm {
+
+constexpr int BM = 128;                 // weight rows per CTA (MMA M of one CTA)
+constexpr int BN = 192;                 // max tokens per tile (MMA N)
+constexpr int BK = 256;                 // K elements per stage = 128 bytes of codes
+constexpr int W_STAGE = BM * 128;       // 16 KB
+constexpr int SFW_STAGE = 2048;         // 128 rows x 16 scales (4 atoms)
+constexpr int SFX_STAGE = 4096;         // up to 2 row blocks x 4 atoms
+constexpr int EPI_WARP_BYTES = 32 * 32 * 4;                   // 32 tokens x 32 columns, fp32
+constexpr int kMaxExperts = 1024;
+constexpr int NUM_WARPS = 11;
+constexpr int NUM_THREADS = NUM_WARPS * 32;
+constexpr int GROUP_TABLE_BYTES = 3 * (kMaxExperts + 1) * 4 + 2 * NUM_WARPS * 4;   // off / slot / tile + scan scratch
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t TMEM_ACC_STRIDE = BN;       // accumulator b at column b*192
+constexpr uint32_t TMEM_SF = 2 * BN;           // scale buffers at 384 and 448
+constexpr uint32_t TMEM_SF_STRIDE = 64;        // per buffer: W scales 16 cols, token scales 32 cols
+constexpr long long kWaitBudgetCycles = 4000000000LL;   // ~2 s at 2 GHz
+
+// warp roles (warps 2..5: epilogue, lane quadrants 2,3,0,1)
+constexpr int W_PRODUCER = 0;     // weight tiles + weight scales
+constexpr int W_MMA = 1;
+constexpr int W_SF0 = 6;          // 6..9: scale factors smem -> tensor memory (quadrants 2,3,0,1)
+constexpr int W_XLOAD = 10;       // token tiles + token scales
+
+static_assert(TMEM_SF + 2 * TMEM_SF_STRIDE <= TMEM_COLS, "tensor memory budget");
+
+// ------------------------------------------------------------------ PTX wrappers
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("{ .reg .b64 st; mbarrier.arrive.shared::cta.b64 st, [%0]; }" :: "r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("{ .reg .b64 st; mbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1; }"
+               :: "r"(bar), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile("{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+               : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+  return ok != 0;
+}
+
+// Same, with cluster-scope acquire: for barriers that the peer CTA of a pair
+// arrives on remotely.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{ .reg .pred p; mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+      : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+  return ok != 0;
+}
+
+// Store to a 32-bit word of another CTA of the cluster (address from mapa).
+__device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" :: "r"(addr), "r"(v) : "memory");
+}
+
+// Bounded wait.  Returns false (and raises the CTA abort flag plus a
+// TIMEOUT status) if the phase did not complete within the budget, or if
+// another role has already aborted.  peer_abort (a cluster address, 0 for
+// none) receives the abort flag too, so a paired CTA leaves its loops as well.
+template <bool kCluster = false>
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                          int32_t *dev_status, uint32_t peer_abort = 0) {
+  auto try_once = [&]() { return kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
+  if (try_once()) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (try_once()) return true;
+    if (*abort_flag) return false;
+    if (clock64() - t0 > kWaitBudgetCycles) {
+      *abort_flag = 1;
+      if (peer_abort) st_cluster_u32(peer_abort, 1u);
+      report(dev_status, NVFP4_ERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+// Warp-wide bounded wait: every lane waits, the verdict is made uniform so
+// that no .sync.aligned tcgen05 instruction ever runs on a partial warp.
+template <bool kCluster = false>
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                               int32_t *dev_status, uint32_t peer_abort = 0) {
+  const bool ok = mbar_wait<kCluster>(bar, parity, abort_flag, dev_status, peer_abort);
+  return __all_sync(0xffffffffu, ok) != 0;
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int32_t x, int32_t y,
+                                            uint32_t bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;"
+      :: "r"(dst), "l"(map), "r"(x), "r"(y), "r"(bar), "l"(policy) : "memory");
+}
+
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               :: "r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
+}
+
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// K-major operand tile, 128-byte swizzle: rows of 128 bytes, 8-row atoms
+// 1024 bytes apart (stride byte offset), version 1 descriptor.
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t addr) {
+  return (uint64_t)((addr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                       uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%5], [%6], p;\n}"
+      :: "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+               :: "r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void tc_ld32_nowait(uint32_t taddr, uint32_t *r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+
+// Instruction descriptor, kind::mxf4nvf4: E2M1 x E2M1, K-major both,
+// UE4M3 scales, M = m (128, or 256 for a CTA pair), N = n (multiple of 16).
+__device__ __forceinline__ uint32_t idesc_mxf4nvf4(uint32_t m, uint32_t n) {
+  return (1u << 7) | (1u << 10) | ((n >> 3) << 17) | ((m >> 4) << 24);
+}
+
+__device__ __forceinline__ void tc_st_x4(uint32_t taddr, uint4 v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};"
+               :: "r"(taddr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
+}
+
+__device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
+// 3-D tiled TMA load (no swizzle): the token scales of two 128-row blocks in
+// one copy.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, int32_t x, int32_t y, int32_t z,
+                                            uint32_t bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3, %4}], [%5], %6;"
+      :: "r"(dst), "l"(map), "r"(x), "r"(y), "r"(z), "r"(bar), "l"(policy) : "memory");
+}
+
+// ------------------------------------------------------------------ CTA pair (cta_group::2)
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_id_x() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t nclusters_x() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+  return r;
+}
+
+// Shared address of the same variable in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+
+// Arrive on an mbarrier of another CTA of the cluster (release at cluster scope).
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" :: "r"(cluster_addr) : "memory");
+}
+
+// Whole-cluster barrier (every thread of both CTAs).
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Tile load whose completion is counted on the mbarrier of the pair's leader
+// CTA (`bar` is a cluster address); the data lands in this CTA's shared memory.
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap *map, int32_t x, int32_t y,
+                                                 uint32_t bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;"
+      :: "r"(dst), "l"(map), "r"(x), "r"(y), "r"(bar), "l"(policy) : "memory");
+}
+
+// 3-D tiled TMA load counted on the pair leader's mbarrier (cluster address).
+__device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap *map, int32_t x, int32_t y, int32_t z,
+                                                 uint32_t bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3, %4}], [%5], %6;"
+      :: "r"(dst), "l"(map), "r"(x), "r"(y), "r"(z), "r"(bar), "l"(policy) : "memory");
+}
+
+// Shared-memory descriptor of one 512-byte scale atom for tcgen05.cp: 32 rows
+// x 16 bytes, no swizzle, 8-row core matrices 128 bytes apart.
+__device__ __forceinline__ uint64_t desc_sf_atom(uint32_t addr) {
+  return (uint64_t)((addr & 0x3FFFFu) >> 4) | ((uint64_t)(128 >> 4) << 32) | ((uint64_t)1 << 46);
+}
+
+// Scale atom -> tensor memory of both CTAs of the pair (each from its own
+// shared memory), replicated to the four lane quadrants (32x128b.warpx4).
+__device__ __forceinline__ void tc_cp_sf_pair(uint32_t taddr, uint64_t desc) {
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" :: "r"(taddr), "l"(desc) : "memory");
+}
+
+// One MMA over the pair: M = 256 (128 weight rows from each CTA's shared
+// memory and tensor memory), N tokens split N/2 + N/2 across the two CTAs.
+__device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
+      "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%5], [%6], p;\n}"
+      :: "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// Commit of the pair's MMAs to the mbarrier at `bar` in both CTAs (mask 0b11).
+__device__ __forceinline__ void tc_commit_pair_both(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+      :: "r"(bar), "h"((uint16_t)3) : "memory");
+}
+
+// Commit of the pair's MMAs to one local mbarrier.
+__device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+               :: "r"(bar) : "memory");
+}
+
+// ------------------------------------------------------------------ tile map
+// Tiles are (expert, weight block, token chunk), weight-block-major inside an
+// expert so that the chunks of one weight block run at the same time.  An
+// expert with m tokens is cut into ceil(m/192) chunks of equal size rounded up
+// to 64, so every chunk starts on a 64-row boundary of the expert's 128-aligned
+// slot: its scale atoms start at row (start & ~127) and the MMA reads them
+// from tensor-memory column offset (start & 127)/32 (0 or 2).
+struct Tile {
+  int e;          // expert
+  int w_row0;     // first weight row of this CTA (over E*N rows)
+  int n_col0;     // first output column of this CTA
+  int x_row0;     // first activation row of the tile (slot space)
+  int y_row0;     // first output row
+  int n_valid;    // tokens in this tile (1..192)
+};
+
+__device__ __forceinline__ int chunks_of(int m) { return (m + BN - 1) / BN; }
+
+// Tile t of a grid whose weight blocks are `wrows` rows (128 for one CTA, 256
+// for a pair); `sub` is the CTA's 128-row half of the block.  With the SwiGLU
+// epilogue the fused gate_up weight is stored in 32-row groups (16 gate rows,
+// then the 16 matching up rows), so 128 weight rows give 64 h columns.
+template <bool kSwiglu>
+__device__ __forceinline__ Tile decode_tile(int t, const int32_t *s_off, const int32_t *s_slot,
+                                            const int32_t *s_tile, int E, int N, int wrows, int sub) {
+  Tile T;
+  const int e = upper_group(s_tile, E, t);
+  const int m_e = s_off[e + 1] - s_off[e];
+  const int nch = chunks_of(m_e);
+  const int csz = ((m_e + nch - 1) / nch + 63) & ~63;
+  const int local = t - s_tile[e];
+  const int mt = local / nch, ch = local - mt * nch;
+  const int start = ch * csz;
+  const int row_in_e = mt * wrows + sub * BM;
+  T.e = e;
+  T.n_col0 = kSwiglu ? row_in_e / 2 : row_in_e;
+  T.w_row0 = e * N + row_in_e;
+  T.x_row0 = s_slot[e] + start;
+  T.y_row0 = s_off[e] + start;
+  T.n_valid = min(csz, m_e - start);
+  return T;
+}
+
+// Block-wide: s_off = expert offsets ({0, M_total} without offsets), s_slot =
+// 128-aligned slot starts, s_tile = first tile of each expert (n_mtiles weight
+// blocks x chunks per expert).  Every thread of the block calls it.
+__device__ inline void build_tile_tables(const int32_t *__restrict__ expert_offsets, int E, int M_total,
+                                         int n_mtiles, int32_t *s_off, int32_t *s_slot, int32_t *s_tile,
+                                         int32_t *s_scratch) {
+  if (expert_offsets) {
+    for (int i = threadIdx.x; i <= E; i += NUM_THREADS) s_off[i] = expert_offsets[i];
+  } else if (threadIdx.x == 0) {
+    s_off[0] = 0;
+    s_off[1] = M_total;
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int per = (E + NUM_THREADS - 1) / NUM_THREADS;
+  const int e0 = min(E, (int)threadIdx.x * per), e1 = min(E, e0 + per);
+  int32_t ls = 0, lt = 0;
+  for (int e = e0; e < e1; ++e) {
+    const int32_t m = s_off[e + 1] - s_off[e];
+    ls += (m + kSlotAlign - 1) / kSlotAlign * kSlotAlign;
+    lt += n_mtiles * chunks_of(m);
+  }
+  int32_t is = ls, it = lt;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int32_t a = __shfl_up_sync(0xffffffffu, is, d), b = __shfl_up_sync(0xffffffffu, it, d);
+    if (lane >= d) { is += a; it += b; }
+  }
+  if (lane == 31) { s_scratch[warp] = is; s_scratch[NUM_WARPS + warp] = it; }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int32_t as = 0, at = 0;
+    for (int w = 0; w < NUM_WARPS; ++w) {
+      const int32_t vs = s_scratch[w], vt = s_scratch[NUM_WARPS + w];
+      s_scratch[w] = as; s_scratch[NUM_WARPS + w] = at;
+      as += vs; at += vt;
+    }
+  }
+  __syncthreads();
+  int32_t rs = s_scratch[warp] + is - ls, rt = s_scratch[NUM_WARPS + warp] + it - lt;
+  for (int e = e0; e < e1; ++e) {
+    const int32_t m = s_off[e + 1] - s_off[e];
+    s_slot[e] = rs;
+    s_tile[e] = rt;
+    rs += (m + kSlotAlign - 1) / kSlotAlign * kSlotAlign;
+    rt += n_mtiles * chunks_of(m);
+  }
+  if (e1 == E && e0 < e1) { s_slot[E] = rs; s_tile[E] = rt; }
+  __syncthreads();
+}
+
+// One K stage of scale factors into tensor memory, written by one warp for its
+// lane quadrant: lane l gets the 16 bytes of atom row l (the scales of rows l,
+// l+32, l+64, l+96), i.e. the replicated 32x128b layout the block-scaled MMA
+// reads.  Weight scales go to columns 0..15 of the buffer, token scales of one
+// or two 128-row blocks to columns 16 + 8*kk + 4*rb.
+__device__ __forceinline__ void sf_stage_to_tmem(uint32_t tcol, uint32_t sfw_addr, uint32_t sfx_addr, int nrb) {
+#pragma unroll
+  for (int kk = 0; kk < 4; ++kk) tc_st_x4(tcol + kk * 4, lds128(sfw_addr + kk * 512));
+#pragma unroll
+  for (int kk = 0; kk < 4; ++kk) tc_st_x4(tcol + 16 + kk * 8, lds128(sfx_addr + kk * 512));
+  if (nrb > 1) {
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) tc_st_x4(tcol + 16 + kk * 8 + 4, lds128(sfx_addr + 2048 + kk * 512));
+  }
+  tc_wait_st();
+}
+
+// Epilogue of one tile for the calling warp (lane quadrant `quad`, 32
+// accumulator rows = 32 weight rows of this CTA): tcgen05.ld the accumulator
+// 64 columns (tokens) at a time, scale by alpha = a_gs[e] * b_gs[e], and store
+// Y (fp32 or bf16) or, with the SwiGLU epilogue, h = bf16(silu(g) * u) plus
+// the expert's max |h|.  Once the last columns are in registers the
+// accumulator is handed back by an arrive on `acc_empty` (in the pair's leader
+// CTA when release_remote).
+template <bool kSwiglu, bool kBf16Out>
+__device__ __forceinline__ void epilogue_tile(const Tile &T, uint32_t tacc, float alpha, uint32_t epi, int quad,
+                                              int lane, int N, void *__restrict__ y, float *__restrict__ amax_out,
+                                              uint32_t acc_empty, bool release_remote) {
+  uint32_t hmax = 0;                           // SwiGLU: max |h| bits of this lane
+  for (int c0 = 0; c0 < T.n_valid; c0 += 64) {
+    uint32_t r[64];
+    tc_ld32_nowait(tacc + (uint32_t)c0, r);
+    if (c0 + 32 < T.n_valid) tc_ld32_nowait(tacc + (uint32_t)c0 + 32, r + 32);
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+    if (c0 + 64 >= T.n_valid) {
+      // the whole accumulator has been read: hand it back to the MMA warp
+      tc_fence_before();
+      if (release_remote) mbar_arrive_remote(acc_empty);
+      else mbar_arrive(acc_empty);
+    }
+    if constexpr (kSwiglu) {
+      // TMEM lane l of quadrant q holds h column 16q + (l & 15): the gate
+      // row for l < 16, the matching up row for l >= 16.  One xor-16
+      // shuffle per token pair gives each lane both operands; the gate
+      // lane finishes tokens 0..15 of the 32, the up lane tokens 16..31.
+      // h = bf16(silu(g) * u) with g, u = alpha*acc in fp32 (silu through
+      // the fast exp and divide intrinsics: a few fp32 ulps, far below the
+      // bf16 rounding of h).  The 32x16 h block is staged in shared memory
+      // (the two token halves 576 bytes apart, so the halves' stores hit
+      // disjoint banks) and written as 32-byte row segments.
+      const bool gate_lane = lane < 16;
+      const uint32_t half = gate_lane ? 0u : 576u;
+#pragma unroll
+      for (int sub = 0; sub < 2; ++sub) {
+        const int tok0 = c0 + sub * 32;
+        if (tok0 >= T.n_valid) break;
+        const int rows_here = min(32, T.n_valid - tok0);
+        const int my0 = gate_lane ? 0 : 16;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const uint32_t mine = gate_lane ? r[sub * 32 + 16 + j] : r[sub * 32 + j];
+          const uint32_t other = __shfl_xor_sync(0xffffffffu, mine, 16);
+          const float gv = __fmul_rn(__uint_as_float(gate_lane ? r[sub * 32 + j] : other), alpha);
+          const float uv = __fmul_rn(__uint_as_float(gate_lane ? other : r[sub * 32 + 16 + j]), alpha);
+          const float sv = __fdividef(gv, 1.0f + __expf(-gv));
+          const __nv_bfloat16 hv = __float2bfloat16_rn(__fmul_rn(sv, uv));
+          const uint16_t hb = *reinterpret_cast<const uint16_t *>(&hv);
+          if (my0 + j < rows_here) hmax = max(hmax, (uint32_t)(hb & 0x7FFFu));
+          asm volatile("st.shared.b16 [%0], %1;" :: "r"(epi + half + j * 32 + (lane & 15) * 2), "h"(hb) : "memory");
+        }
+        __syncwarp();
+        const int NH = N / 2;
+        __nv_bfloat16 *hbase = reinterpret_cast<__nv_bfloat16 *>(y) + (int64_t)(T.y_row0 + tok0) * NH +
+                               T.n_col0 + quad * 16;
+#pragma unroll
+        for (int it = 0; it < 2; ++it) {
+          const int row = it * 16 + (lane >> 1), chunk = lane & 1;
+          if (row < rows_here) {
+            const uint4 v = lds128(epi + (row >> 4) * 576 + (row & 15) * 32 + chunk * 16);
+            *reinterpret_cast<uint4 *>(hbase + (int64_t)row * NH + chunk * 8) = v;
+          }
+        }
+        __syncwarp();
+      }
+    } else {
+      // Stage each 32-token x 32-column block in shared memory (this lane
+      // owns one weight column), then write whole 64/128-byte row segments
+      // of Y with 16-byte vector stores.
+#pragma unroll
+      for (int sub = 0; sub < 2; ++sub) {
+        const int tok0 = c0 + sub * 32;
+        if (tok0 >= T.n_valid) break;
+        const int rows_here = min(32, T.n_valid - tok0);
+        if (kBf16Out) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const __nv_bfloat16 hv = __float2bfloat16_rn(__fmul_rn(__uint_as_float(r[sub * 32 + i]), alpha));
+            asm volatile("st.shared.b16 [%0], %1;" :: "r"(epi + i * 64 + lane * 2),
+                         "h"(*reinterpret_cast<const uint16_t *>(&hv)) : "memory");
+          }
+          __syncwarp();
+          __nv_bfloat16 *ybase = reinterpret_cast<__nv_bfloat16 *>(y) + (int64_t)(T.y_row0 + tok0) * N + T.n_col0 + quad * 32;
+#pragma unroll
+          for (int it = 0; it < 4; ++it) {
+            const int row = it * 8 + (lane >> 2), chunk = lane & 3;
+            if (row < rows_here) {
+              const uint4 v = lds128(epi + row * 64 + chunk * 16);
+              *reinterpret_cast<uint4 *>(ybase + (int64_t)row * N + chunk * 8) = v;
+            }
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float fv = __fmul_rn(__uint_as_float(r[sub * 32 + i]), alpha);
+            asm volatile("st.shared.b32 [%0], %1;" :: "r"(epi + i * 128 + lane * 4), "f"(fv) : "memory");
+          }
+          __syncwarp();
+          float *ybase = reinterpret_cast<float *>(y) + (int64_t)(T.y_row0 + tok0) * N + T.n_col0 + quad * 32;
+#pragma unroll
+          for (int it = 0; it < 8; ++it) {
+            const int row = it * 4 + (lane >> 3), chunk = lane & 7;
+            if (row < rows_here) {
+              const uint4 v = lds128(epi + row * 128 + chunk * 16);
+              *reinterpret_cast<uint4 *>(ybase + (int64_t)row * N + chunk * 4) = v;
+            }
+          }
+        }
+        __syncwarp();
+      }
+    }
+  }
+  if (kSwiglu) {
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) hmax = max(hmax, __shfl_xor_sync(0xffffffffu, hmax, d));
+    if (lane == 0 && hmax) atomicMax(reinterpret_cast<uint32_t *>(amax_out) + T.e, hmax << 16);
+  }
+}
+
+}  // namespace gemm
+}  // namespace nvfp4
+
+// ====================================================================== host helpers
+namespace nvfp4 {
+namespace gemm {
+
+inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult qres;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qres) == cudaSuccess &&
+        qres == cudaDriverEntryPointSuccess && p)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 2-D uint8 view [rows, row_bytes] with a {128 bytes, box_rows} box, 128-byte swizzle.
+inline bool make_map(CUtensorMap *map, const void *base, uint64_t rows, uint64_t row_bytes, uint32_t box_rows) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {row_bytes, rows};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {128, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Token scales in the MMA-tiled layout viewed as [row block][K/32][256 bytes]:
+// one {256, 8, 2} box is the 2 KB of one K stage for two consecutive 128-row
+// blocks (a block past the end reads as zeros).
+inline bool make_map_sfx(CUtensorMap *map, const void *base, uint64_t row_blocks, uint64_t K) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {256, K / 32, row_blocks};
+  cuuint64_t strides[2] = {256, K * 8};
+  cuuint32_t box[3] = {256, 8, 2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Weight scales in the MMA-tiled layout viewed as [row block][K/32][256 bytes]:
+// one {256, 8, 1} box is the 2 KB of one K stage of one 128-row block.
+inline bool make_map_sfw(CUtensorMap *map, const void *base, uint64_t row_blocks, uint64_t K) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {256, K / 32, row_blocks};
+  cuuint64_t strides[2] = {256, K * 8};
+  cuuint32_t box[3] = {256, 8, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The pair kernel's launch (gemm_pair.cu).  Requires N % 256 == 0.
+nvfp4_status launch_grouped_gemm_pair(const uint8_t *a_q, const uint8_t *a_sf, const float *a_gs,
+                                      const uint8_t *b_q, const uint8_t *b_sf, const float *b_gs,
+                                      const int32_t *expert_offsets, int E, int64_t M_total, int64_t N, int64_t K,
+                                      void *y, nvfp4_out_dtype out_dtype, bool swiglu, float *amax_out,
+                                      int32_t *dev_status, cudaStream_t stream);
+
+}  // namespace gemm
+}  // namespace nvfp4

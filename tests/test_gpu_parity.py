@@ -36,6 +36,15 @@ def status_word():
     return torch.zeros(1, dtype=torch.int32, device="cuda")
 
 
+@pytest.fixture(params=[1, 2], ids=["one_cta", "cta_pair"])
+def gemm_kernel(request):
+    """Run the test on the one-CTA grouped GEMM and on the CTA-pair kernel."""
+    nv = nvmod()
+    nv.nvfp4_gemm_select_kernel(request.param)
+    yield request.param
+    nv.nvfp4_gemm_select_kernel(0)
+
+
 def gemm_tol(y, y_ref, s_ref):
     """|y - y_ref| <= 1e-5 * sum|a*b| + 1e-6 elementwise."""
     err = np.abs(y.astype(np.float64) - y_ref)
@@ -399,7 +408,7 @@ def _run_gemm(qs, ss, gs_a, qw, sfw, gs_w, offsets, E, R, N, K, out_dtype):
     return to_np(y)
 
 
-def test_gemm_closed_form_integer_case():
+def test_gemm_closed_form_integer_case(gemm_kernel):
     """All scales 1.0 and s_g = 1: every product is a multiple of 1/4 and the
     fp32 sum is exact, so the tensor-core result must equal the oracle exactly."""
     rng = np.random.default_rng(0)
@@ -417,7 +426,7 @@ def test_gemm_closed_form_integer_case():
 
 
 @pytest.mark.parametrize("out_dtype", [0, 1])
-def test_gemm_dense_config1(out_dtype):
+def test_gemm_dense_config1(out_dtype, gemm_kernel):
     M, N, K = 128, 256, 512
     x = synthetic.gaussian_bf16(0, synthetic.STREAMS["x"], (M, K), outlier_frac=0.001)
     w = synthetic.gaussian_bf16(0, synthetic.STREAMS["w"], (N, K), sigma=0.02)
@@ -435,7 +444,7 @@ def test_gemm_dense_config1(out_dtype):
         assert np.array_equal(y, synthetic.f32_to_bf16_bits(y32))
 
 
-def test_gemm_grouped_ragged():
+def test_gemm_grouped_ragged(gemm_kernel):
     E, N, K = 6, 256, 512
     counts = [0, 5, 130, 300, 16, 257]
     offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
@@ -453,11 +462,12 @@ def test_gemm_grouped_ragged():
 
 
 @pytest.mark.parametrize("out_dtype", [0, 1])
-def test_gemm_grouped_chunk_edges(out_dtype):
+def test_gemm_grouped_chunk_edges(out_dtype, gemm_kernel):
     """Expert sizes around every tile and chunk boundary (64-row chunk starts,
-    one or two scale row blocks, the 192-token tile limit)."""
-    counts = [1, 63, 64, 65, 127, 128, 129, 191, 192, 193, 255, 256, 257, 383, 384, 385, 577, 0, 2]
-    E, N, K = len(counts), 128, 256
+    one or two scale row blocks, the 192-token tile limit, token-tile halves of
+    8..96 rows on a CTA pair)."""
+    counts = [1, 63, 64, 65, 127, 128, 129, 191, 192, 193, 255, 256, 257, 383, 384, 385, 577, 0, 2, 17, 33]
+    E, N, K = len(counts), 256, 256
     offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
     R = int(offsets[-1])
     x = synthetic.gaussian_bf16(12, synthetic.STREAMS["x"], (R, K), outlier_frac=0.001)
@@ -475,9 +485,13 @@ def test_gemm_grouped_chunk_edges(out_dtype):
         assert np.array_equal(y16, synthetic.f32_to_bf16_bits(y))
 
 
-def test_gemm_dense_many_tiles():
-    """Dense M = 1000 rows (6 token chunks, ragged last), N = 384, K = 1024."""
-    M, N, K = 1000, 384, 1024
+@pytest.mark.parametrize("N", [384, 512])
+def test_gemm_dense_many_tiles(N, gemm_kernel):
+    """Dense M = 1000 rows (6 token chunks, ragged last), K = 1024; N = 384 is
+    not a multiple of the pair's 256 weight rows (one-CTA kernel only)."""
+    if gemm_kernel == 2 and N % 256:
+        pytest.skip("CTA pairs need N % 256 == 0")
+    M, K = 1000, 1024
     x = synthetic.gaussian_bf16(13, synthetic.STREAMS["x"], (M, K), outlier_frac=0.001)
     w = synthetic.gaussian_bf16(13, synthetic.STREAMS["w"], (N, K), sigma=0.02)
     qx, sx, gx, _ = oracle.quantize(x)
@@ -490,9 +504,9 @@ def test_gemm_dense_many_tiles():
     assert ok.all(), (err.max(), (err / bound).max())
 
 
-def test_gemm_long_k_tolerance():
+def test_gemm_long_k_tolerance(gemm_kernel):
     """K = 17408 (the dense MLP's down projection) on a thin slice."""
-    M, N, K = 64, 128, 17408
+    M, N, K = 64, 256, 17408
     x = synthetic.gaussian_bf16(9, synthetic.STREAMS["x"], (M, K), outlier_frac=0.001)
     w = synthetic.gaussian_bf16(9, synthetic.STREAMS["w"], (N, K), sigma=0.02)
     qx, sx, gx, _ = oracle.quantize(x)
@@ -506,7 +520,7 @@ def test_gemm_long_k_tolerance():
 
 
 # --------------------------------------------------------------------------- fused SwiGLU epilogue
-def test_gemm_swiglu_epilogue():
+def test_gemm_swiglu_epilogue(gemm_kernel):
     """h = bf16(silu(g)*u) from the gate_up accumulators: compared with the
     oracle SwiGLU of the same GEMM's fp32 output (one bf16 ulp), amax exact."""
     L = layer()
