@@ -496,7 +496,8 @@ def comp_moe_full(device, iters, warmup, flush):
     w = torch.from_numpy(r["weights"].astype(np.float32)).to(device)
     t_route = timed(lambda: L.route(ids, E), iters, warmup, flush)
     y2 = moe.forward(x, ri, off)
-    t_comb = timed(lambda: L.combine(y2, full.slot[:T], w, out_dtype=1, out=full.out[:T]), iters, warmup, flush)
+    sl = r["slot_dev"]                     # the slot map of the routing that ordered y2's rows
+    t_comb = timed(lambda: L.combine(y2, sl, w, out_dtype=1, out=full.out[:T]), iters, warmup, flush)
     full.forward(x, ids, w)
     t_full = timed(lambda: full.forward(x, ids, w), iters, warmup, flush)
     flops = moe_flops(R, H, I)

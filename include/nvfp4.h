@@ -303,14 +303,16 @@ nvfp4_status nvfp4_moe_route(const int32_t *topk_ids, int64_t tokens, int topk, 
  * nvfp4_moe_combine -- out[t, :] = sum_j weights[t, j] * y[slot[t, j], :],
  * accumulated in fp32 in choice order (the weighted sum of a token's expert
  * outputs after the down projection).
- *   y        fp32 or bf16 [routed rows, H] (the down GEMM output); H % 8 == 0.
- *   slot     int32 [tokens, topk] from nvfp4_moe_route (-1 entries skipped).
+ *   y, rows  fp32 or bf16 [rows, H] (the down GEMM output); H % 8 == 0.
+ *   slot     int32 [tokens, topk] from nvfp4_moe_route: -1 entries are
+ *            skipped; an entry >= rows is skipped and reported as
+ *            NVFP4_ERR_INDEX in dev_status (nullable), never read.
  *   weights  fp32 [tokens, topk] routing weights.
  *   out      fp32 or bf16 [tokens, H].
  */
-nvfp4_status nvfp4_moe_combine(const void *y, nvfp4_out_dtype y_dtype, const int32_t *slot,
+nvfp4_status nvfp4_moe_combine(const void *y, nvfp4_out_dtype y_dtype, int64_t rows, const int32_t *slot,
                                const float *weights, int64_t tokens, int topk, int64_t H, void *out,
-                               nvfp4_out_dtype out_dtype, cudaStream_t stream);
+                               nvfp4_out_dtype out_dtype, int32_t *dev_status, cudaStream_t stream);
 
 /*
  * nvfp4_quantize_noalloc -- nvfp4_quantize without a caller workspace.

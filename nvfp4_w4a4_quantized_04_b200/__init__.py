@@ -95,7 +95,7 @@ def load_library(path: str = LIB_PATH):
     L.nvfp4_moe_route.restype = i32
     L.nvfp4_moe_route.argtypes = [P, i64, i32, i32, P, P, P, P, P, P]
     L.nvfp4_moe_combine.restype = i32
-    L.nvfp4_moe_combine.argtypes = [P, i32, P, P, i64, i32, i64, P, i32, P]
+    L.nvfp4_moe_combine.argtypes = [P, i32, i64, P, P, i64, i32, i64, P, i32, P, P]
     L.nvfp4_kv_dequantize.restype = i32
     L.nvfp4_kv_dequantize.argtypes = [P, P, P, P, P, P, i64, i64, i64, P, P, P]
     _lib = L
@@ -246,9 +246,11 @@ def nvfp4_moe_route(topk_ids, tokens, topk, num_experts, expert_offsets, row_ind
     return st
 
 
-def nvfp4_moe_combine(y, y_dtype, slot, weights, tokens, topk, H, out, out_dtype, stream=None, check=True) -> int:
+def nvfp4_moe_combine(y, y_dtype, rows, slot, weights, tokens, topk, H, out, out_dtype, dev_status=None,
+                      stream=None, check=True) -> int:
     st = load_library().nvfp4_moe_combine(
-        _ptr(y), y_dtype, _ptr(slot), _ptr(weights), tokens, topk, H, _ptr(out), out_dtype, _stream(stream))
+        _ptr(y), y_dtype, rows, _ptr(slot), _ptr(weights), tokens, topk, H, _ptr(out), out_dtype, _ptr(dev_status),
+        _stream(stream))
     if check:
         _check(st, "nvfp4_moe_combine")
     return st

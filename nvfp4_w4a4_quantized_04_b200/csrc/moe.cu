@@ -137,9 +137,10 @@ __device__ __forceinline__ void load8(const void *y, bool bf16, int64_t idx, flo
 
 // One thread per (token, 8 columns): k loads of 16/32 bytes in flight.
 template <bool kBf16In, bool kBf16Out>
-__global__ void __launch_bounds__(256) combine_kernel(const void *__restrict__ y, const int32_t *__restrict__ slot,
+__global__ void __launch_bounds__(256) combine_kernel(const void *__restrict__ y, int64_t rows,
+                                                      const int32_t *__restrict__ slot,
                                                       const float *__restrict__ w, int64_t T, int k, int64_t H,
-                                                      void *__restrict__ out) {
+                                                      void *__restrict__ out, int32_t *dev_status) {
   const int64_t ncg = H >> 3;
   const int64_t total = T * ncg;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
@@ -149,6 +150,10 @@ __global__ void __launch_bounds__(256) combine_kernel(const void *__restrict__ y
     for (int j = 0; j < k; ++j) {
       const int32_t r = __ldg(slot + t * k + j);
       if (r < 0) continue;
+      if (r >= rows) {                      // never read past y: skip and report
+        if (c == 0) report(dev_status, NVFP4_ERR_INDEX);
+        continue;
+      }
       const float wj = __ldg(w + t * k + j);
       float v[8];
       load8(y, kBf16In, (int64_t)r * H + c, v);
@@ -215,16 +220,16 @@ extern "C" nvfp4_status nvfp4_moe_route(const int32_t *topk_ids, int64_t tokens,
   return NVFP4_OK;
 }
 
-extern "C" nvfp4_status nvfp4_moe_combine(const void *y, nvfp4_out_dtype y_dtype, const int32_t *slot,
+extern "C" nvfp4_status nvfp4_moe_combine(const void *y, nvfp4_out_dtype y_dtype, int64_t rows, const int32_t *slot,
                                           const float *weights, int64_t tokens, int topk, int64_t H, void *out,
-                                          nvfp4_out_dtype out_dtype, cudaStream_t stream) {
-  if (tokens < 0 || topk < 1 || topk > moe::kMaxTopk || H <= 0) return NVFP4_ERR_INVALID_ARG;
+                                          nvfp4_out_dtype out_dtype, int32_t *dev_status, cudaStream_t stream) {
+  if (tokens < 0 || rows < 0 || topk < 1 || topk > moe::kMaxTopk || H <= 0) return NVFP4_ERR_INVALID_ARG;
   if (H % 8 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   if ((y_dtype != NVFP4_OUT_F32 && y_dtype != NVFP4_OUT_BF16) ||
       (out_dtype != NVFP4_OUT_F32 && out_dtype != NVFP4_OUT_BF16))
     return NVFP4_ERR_INVALID_ARG;
   if (tokens == 0) return NVFP4_OK;
-  if (!y || !slot || !weights || !out) return NVFP4_ERR_INVALID_ARG;
+  if ((rows > 0 && !y) || !slot || !weights || !out) return NVFP4_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(y) | reinterpret_cast<uintptr_t>(out)) & 15u) return NVFP4_ERR_INVALID_ARG;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
@@ -233,7 +238,7 @@ extern "C" nvfp4_status nvfp4_moe_combine(const void *y, nvfp4_out_dtype y_dtype
   int64_t blocks = (work + 255) / 256;
   if (blocks > (int64_t)sms * 8) blocks = (int64_t)sms * 8;
   const bool bi = y_dtype == NVFP4_OUT_BF16, bo = out_dtype == NVFP4_OUT_BF16;
-#define NVFP4_CB(A, B) moe::combine_kernel<A, B><<<(unsigned)blocks, 256, 0, stream>>>(y, slot, weights, tokens, topk, H, out)
+#define NVFP4_CB(A, B) moe::combine_kernel<A, B><<<(unsigned)blocks, 256, 0, stream>>>(y, rows, slot, weights, tokens, topk, H, out, dev_status)
   if (bi && bo) NVFP4_CB(true, true);
   else if (bi) NVFP4_CB(true, false);
   else if (bo) NVFP4_CB(false, true);

@@ -252,15 +252,17 @@ def route(topk_ids: torch.Tensor, num_experts: int, dev_status=None):
     return off, ri, slot
 
 
-def combine(y: torch.Tensor, slot: torch.Tensor, weights: torch.Tensor, out_dtype=OUT_BF16, out=None):
-    """out[t] = sum_j weights[t, j] * y[slot[t, j]] (fp32 accumulation)."""
+def combine(y: torch.Tensor, slot: torch.Tensor, weights: torch.Tensor, out_dtype=OUT_BF16, out=None,
+            dev_status=None):
+    """out[t] = sum_j weights[t, j] * y[slot[t, j]] (fp32 accumulation); slots
+    outside y's rows are skipped and reported in dev_status."""
     T, k = slot.shape
     H = y.shape[1]
     dt = torch.float32 if out_dtype == OUT_F32 else torch.bfloat16
     if out is None:
         out = torch.empty((T, H), dtype=dt, device=y.device)
     ydt = OUT_F32 if y.dtype == torch.float32 else OUT_BF16
-    nvfp4_moe_combine(y, ydt, slot, weights, T, k, H, out, out_dtype)
+    nvfp4_moe_combine(y, ydt, y.shape[0], slot, weights, T, k, H, out, out_dtype, dev_status)
     return out
 
 
@@ -289,6 +291,6 @@ class MoELayer:
         nvfp4_moe_route(topk_ids, T, k, E, self.off, ri, slot, self.rws, dev_status)
         y = self.experts.forward(x, ri, self.off, dev_status, slot=slot)
         out = self.out[:T]
-        nvfp4_moe_combine(y, OUT_F32 if y.dtype == torch.float32 else OUT_BF16, slot, topk_weights, T, k,
-                          self.experts.H, out, OUT_BF16)
+        nvfp4_moe_combine(y, OUT_F32 if y.dtype == torch.float32 else OUT_BF16, y.shape[0], slot, topk_weights, T, k,
+                          self.experts.H, out, OUT_BF16, dev_status)
         return out

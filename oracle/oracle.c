@@ -448,7 +448,7 @@ int orc_route(const int32_t *ids, int64_t T, int k, int E, int32_t *offsets, int
 }
 
 /* out[t, :] = sum_j w[t, j] * y[slot[t, j], :], accumulated in fp64 in
- * choice order; also |w*y| summed for the tolerance.  y is fp32. */
+ * choice order, skipping slot -1; also |w*y| summed for the tolerance.  y is fp32. */
 void orc_combine(const float *y, const int32_t *slot, const float *w, int64_t T, int k, int64_t H,
                  double *out, double *sabs) {
     #pragma omp parallel for schedule(static)
@@ -456,6 +456,7 @@ void orc_combine(const float *y, const int32_t *slot, const float *w, int64_t T,
         for (int64_t c = 0; c < H; ++c) {
             double s = 0.0, a = 0.0;
             for (int j = 0; j < k; ++j) {
+                if (slot[t * k + j] < 0) continue;      /* a choice the routing dropped adds nothing */
                 double p = (double)w[t * k + j] * (double)y[(int64_t)slot[t * k + j] * H + c];
                 s += p;
                 a += fabs(p);

@@ -763,6 +763,24 @@ def test_combine(ydt):
     assert np.array_equal(out16, synthetic.f32_to_bf16_bits(out32))
 
 
+def test_combine_out_of_range_slot():
+    """A slot past y's rows is skipped (never read) and reported; -1 is skipped silently."""
+    L = layer()
+    T, k, H = 5, 2, 64
+    yb = synthetic.gaussian_bf16(6, synthetic.STREAMS["x"], (8, H))
+    yf = synthetic.bf16_bits_to_f32(yb)
+    slot = np.array([[0, 1], [2, -1], [3, 4], [5, 8], [6, 7]], dtype=np.int32)
+    w = np.full((T, k), 0.5, np.float32)
+    s = status_word()
+    out = to_np(L.combine(to_dev(yf), to_dev(slot), to_dev(w), out_dtype=0, dev_status=s))
+    torch.cuda.synchronize()
+    assert int(s.item()) == 19
+    ok = slot.copy()
+    ok[3, 1] = -1
+    ref, sabs = oracle.combine(yf, ok, w)
+    assert (np.abs(out - ref) <= 1e-6 * sabs + 1e-30).all()
+
+
 def test_moe_layer_full_small():
     """route -> experts -> combine; the combine stage checked on the device's y."""
     L = layer()

@@ -483,3 +483,11 @@ def test_combine_closed_forms():
         want = sum(0.25 * y[slot[t, j]].astype(np.float64) for j in range(k))
         assert np.allclose(out[t], want, rtol=0, atol=1e-12)
         assert np.allclose(s[t], sum(np.abs(0.25 * y[slot[t, j]].astype(np.float64)) for j in range(k)))
+    # a dropped choice (slot -1) contributes nothing: same as weight 0 on a real row
+    dropped = slot.copy()
+    dropped[:, 2] = -1
+    w0 = w.copy()
+    w0[:, 2] = 0.0
+    out_d, s_d = oracle.combine(y, dropped, w)
+    out_0, s_0 = oracle.combine(y, slot, w0)
+    assert np.array_equal(out_d, out_0) and np.array_equal(s_d, s_0)
