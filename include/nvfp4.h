@@ -85,8 +85,8 @@ typedef enum { NVFP4_OUT_F32 = 0, NVFP4_OUT_BF16 = 1 } nvfp4_out_dtype;
  * g = alpha*acc_gate, u = alpha*acc_up kept in fp32 (no bf16 rounding of the
  * gate_up output in between; silu through the fast exp/divide intrinsics),
  * y is bf16 [M_total, N/2], and amax_out[e]
- * receives max |h| of expert e (fp32 bit pattern via integer max: the
- * caller zeroes it). */
+ * receives max |h| of expert e (fp32 bit pattern via integer max; the call
+ * clears amax_out first). */
 typedef enum { NVFP4_EPI_NONE = 0, NVFP4_EPI_SWIGLU = 1 } nvfp4_epilogue;
 
 /* Human-readable name of a status code (static string). */
@@ -216,7 +216,7 @@ nvfp4_status mxfp4_to_nvfp4(const uint8_t *q_mx, const uint8_t *ue8m0, int64_t n
  *   y, out_dtype    fp32 or bf16 [M_total, N], rows in routed (unpadded) order.
  *   epi, amax_out   NVFP4_EPI_NONE (amax_out unused), or NVFP4_EPI_SWIGLU: y is
  *                   bf16 h [M_total, N/2] (out_dtype must be BF16), amax_out
- *                   fp32 [E] zeroed by the caller, N/2 % 64 == 0.
+ *                   fp32 [E] (cleared and written by the call), N/2 % 64 == 0.
  *   workspace   >= nvfp4_workspace_size(E); dev_status: NVFP4_ERR_TIMEOUT if a
  *               pipeline wait gave up (the output is then incomplete).
  */

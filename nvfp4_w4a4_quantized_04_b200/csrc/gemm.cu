@@ -306,6 +306,8 @@ extern "C" nvfp4_status nvfp4_grouped_gemm(const uint8_t *a_q, const uint8_t *a_
   if (M_total < 0 || N <= 0 || K <= 0) return NVFP4_ERR_INVALID_ARG;
   if (N % 128 != 0 || K % 256 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   if ((int64_t)E * N > ((int64_t)1 << 31) - 1 || M_total > ((int64_t)1 << 30)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  // the SwiGLU epilogue raises amax_out[e] with integer atomics: start from 0
+  if (swiglu && cudaMemsetAsync(amax_out, 0, sizeof(float) * (size_t)E, stream) != cudaSuccess) return NVFP4_ERR_CUDA;
   if (M_total == 0) return NVFP4_OK;
   if (!a_q || !a_sf || !a_gs || !b_q || !b_sf || !b_gs || !y) return NVFP4_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(a_q) | reinterpret_cast<uintptr_t>(b_q) | reinterpret_cast<uintptr_t>(a_sf) |

@@ -159,9 +159,7 @@ def grouped_gemm_swiglu(a: Packed, w_gate_up: Packed, N: int, h=None, amax=None,
     if h is None:
         h = torch.empty((a.rows, N // 2), dtype=torch.bfloat16, device=a.q.device)
     if amax is None:
-        amax = torch.zeros(E, dtype=torch.float32, device=a.q.device)
-    else:
-        amax.zero_()
+        amax = torch.empty(E, dtype=torch.float32, device=a.q.device)
     nvfp4_grouped_gemm(a.q, a.sf, a.gs, w_gate_up.q, w_gate_up.sf, w_gate_up.gs, a.offsets, E, a.rows, N, a.K, h,
                        OUT_BF16, EPI_SWIGLU, amax, None, dev_status)
     return h, amax
