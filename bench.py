@@ -125,6 +125,25 @@ def timed(fn, iters, warmup, flush=None):
     return statistics.median(ts)
 
 
+def max_over_ranks(value, world, device="cpu"):
+    """Largest per-rank value over all ranks of the process group (its own
+    backend: NCCL with CUDA tensors, gloo with CPU tensors); the value itself
+    when there is one rank."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank_step, world, steps, total_ms):
+    """Units per second of the whole job: every rank processes its own
+    units_per_rank_step each step (weak scaling), timed by the slowest rank."""
+    return world * units_per_rank_step * steps / (total_ms * 1e-3)
+
+
 def gbs(nbytes, ms):
     return nbytes / (ms * 1e-3) / 1e9
 
@@ -216,16 +235,14 @@ def run_headline(args, rank, world, device):
         flush.fill_(i & 0xFF)               # L2 flush between steps, outside the events
         stages(evs[i])
     torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
     time.sleep(0.15)
     clk = clocks.stop()
     per = np.array([[e[j].elapsed_time(e[j + 1]) for j in range(4)] for e in evs])
     step_ms = per.sum(axis=1)
-    total_ms = float(step_ms.sum())
-    t = torch.tensor([total_ms], dtype=torch.float64, device=device)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
-    value = world * flops * args.steps / (total_ms * 1e-3) / 1e12
+    total_ms = max_over_ranks(float(step_ms.sum()), world, device)
+    value = whole_job_rate(flops, world, args.steps, total_ms) / 1e12
 
     # e2e through the public API with host buffers: pinned H2D of the step's
     # inputs, the layer, D2H of its result, all inside the timed region
@@ -246,11 +263,8 @@ def run_headline(args, rank, world, device):
         y_host.copy_(y, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / n_e2e
-    t = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e, world, device)
+
     h2d = x.numel() * 2 + ri.numel() * 4 + off.numel() * 4 + sl.numel() * 4
     d2h = R * H * 2
 
@@ -306,7 +320,7 @@ def run_headline(args, rank, world, device):
                    "parallelism": f"{world} independent replicas" if world > 1 else "single GPU"},
         "roofline": roof,
         "breakdown": breakdown,
-        "e2e": {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+        "e2e": {"value": round(whole_job_rate(flops, world, 1, e2e_ms) / 1e12, 3), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": round(e2e_ms, 3)},
         "gpu_launches": (7 if fused else 8) * args.steps,
         "clocks": clk,
