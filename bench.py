@@ -427,6 +427,55 @@ def comp_decode_moe(device, iters, warmup, flush):
             "remap_ms": round(remap_ms, 4), "remap_gbs": round(gbs(remap_bytes, remap_ms), 1)}
 
 
+def comp_decode_w4a16(device, iters, warmup, flush):
+    """W4A16 (NVFP4 weights, bf16 activations) experts at decode size: 384
+    experts, 64 tokens, top-10 Zipf(1.1) routing (seed 7), hidden 7168,
+    intermediate 2048; gate_up with the SwiGLU epilogue, then down."""
+    import torch
+
+    import synthetic
+    import synthetic.cuda as sc
+    from nvfp4_w4a4_quantized_04_b200 import layer as L
+    from nvfp4_w4a4_quantized_04_b200 import mxfp4_to_nvfp4
+    E, T, H, I, k = 384, 64, 7168, 2048, 10
+    r = synthetic.route_zipf_gumbel(7, T, E, k)
+    R = len(r["row_index"])
+    ws = L.workspace(2 * E, device)
+    packs = []
+    for name, rows_per, K in (("gate_up", 2 * I, H), ("down", H, I)):
+        n = E * rows_per * K
+        q = sc.mxfp4_codes(7, synthetic.STREAMS["mx_codes_" + name], n // 2).view(E * rows_per, K // 2)
+        e8 = sc.mxfp4_exponents(7, synthetic.STREAMS["mx_exp_" + name], n // 32, lo=-10)
+        qn = torch.empty_like(q)
+        sf = torch.empty(n // 16, dtype=torch.uint8, device=device)
+        gs = torch.empty(E, dtype=torch.float32, device=device)
+        st = torch.zeros(1, dtype=torch.int32, device=device)
+        mxfp4_to_nvfp4(q, e8, E, rows_per, K, qn, sf, 0, gs, ws, st)   # row-major scales
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        packs.append(L.Packed(qn, sf, gs, E * rows_per, K, 0))
+        del q, e8
+    xb = sc.gaussian_bf16(7, synthetic.STREAMS["x"], (T, H))
+    ri = torch.from_numpy(r["row_index"]).to(device)
+    off = torch.from_numpy(r["offsets"]).to(device)
+    h = torch.empty((R, I), dtype=torch.bfloat16, device=device)
+    y = torch.empty((R, H), dtype=torch.bfloat16, device=device)
+
+    def layer():
+        L.grouped_gemm_w4a16(xb, packs[0], 2 * I, ri, off, E, rows=R, out_dtype=1, swiglu=True, y=h)
+        L.grouped_gemm_w4a16(h, packs[1], H, None, off, E, rows=R, out_dtype=1, y=y)
+    ms = timed(layer, iters, warmup, flush)
+    t_gu = timed(lambda: L.grouped_gemm_w4a16(xb, packs[0], 2 * I, ri, off, E, rows=R, out_dtype=1, swiglu=True,
+                                             y=h), iters, warmup, flush)
+    touched = int((np.diff(r["offsets"]) > 0).sum())
+    wbytes = touched * (2 * I * H + H * I) * 0.5625
+    gu_bytes = touched * 2 * I * H * 0.5625
+    return {"workload": "decode_w4a16_experts_e384_top10_zipf1.1_t64_h7168_i2048", "experts_touched": touched,
+            "routed_rows": R, "layer_ms": round(ms, 4), "touched_weight_gbs": round(gbs(wbytes, ms), 1),
+            "gate_up_swiglu_ms": round(t_gu, 4), "gate_up_gbs": round(gbs(gu_bytes, t_gu), 1),
+            "roofline": {"bound": "hbm", "frac": round(gbs(wbytes, ms) / HBM_PEAK, 4), "peak": HBM_PEAK}}
+
+
 def comp_kv(device, iters, warmup, flush):
     """NVFP4 KV cache for one full-attention layer: K, V [262144 tokens, 4, 256]."""
     import torch
@@ -530,7 +579,8 @@ def comp_moe_full(device, iters, warmup, flush):
             "combine_frac_hbm": round(gbs(comb_bytes, t_comb) / HBM_PEAK, 4)}
 
 
-COMPONENTS = {"moe_full": comp_moe_full, "dense_mlp": comp_dense_mlp, "decode_moe": comp_decode_moe, "kv_cache": comp_kv,
+COMPONENTS = {"moe_full": comp_moe_full, "dense_mlp": comp_dense_mlp, "decode_moe": comp_decode_moe,
+              "decode_w4a16": comp_decode_w4a16, "kv_cache": comp_kv,
               "act_quant_sweep": comp_act_sweep, "remap": comp_remap}
 
 

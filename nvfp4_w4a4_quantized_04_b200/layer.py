@@ -14,7 +14,8 @@ from typing import Optional
 import torch
 
 from . import (EPI_NONE, EPI_SWIGLU, GS_AMAX_GIVEN, GS_FROM_AMAX, GS_GIVEN, OUT_BF16, OUT_F32, SF_MMA_TILED, SF_ROWMAJOR,
-               mxfp4_to_nvfp4, nvfp4_dequantize, nvfp4_grouped_gemm, nvfp4_moe_combine, nvfp4_moe_route,
+               mxfp4_to_nvfp4, nvfp4_dequantize, nvfp4_grouped_gemm, nvfp4_grouped_gemm_w4a16, nvfp4_moe_combine,
+               nvfp4_moe_route,
                nvfp4_moe_quantize, nvfp4_moe_route_workspace_size, nvfp4_padded_rows_bound, nvfp4_quantize,
                nvfp4_swiglu_quantize,
                nvfp4_workspace_size)
@@ -163,6 +164,22 @@ def grouped_gemm_swiglu(a: Packed, w_gate_up: Packed, N: int, h=None, amax=None,
     nvfp4_grouped_gemm(a.q, a.sf, a.gs, w_gate_up.q, w_gate_up.sf, w_gate_up.gs, a.offsets, E, a.rows, N, a.K, h,
                        OUT_BF16, EPI_SWIGLU, amax, None, dev_status)
     return h, amax
+
+
+def grouped_gemm_w4a16(x: torch.Tensor, w: Packed, N: int, row_index=None, offsets=None, num_groups: int = 1,
+                       rows=None, out_dtype=OUT_BF16, swiglu=False, y=None, dev_status=None) -> torch.Tensor:
+    """Weight-only NVFP4 (row-major scales) x bf16 activations, per expert:
+    Y [rows, N] (or h [rows, N/2] with ``swiglu``; gate rows first)."""
+    assert x.dtype == torch.bfloat16 and w.layout == SF_ROWMAJOR
+    M = rows if rows is not None else (row_index.shape[0] if row_index is not None else x.shape[0])
+    G = num_groups if offsets is not None else 1
+    dt = torch.float32 if out_dtype == OUT_F32 else torch.bfloat16
+    cols = N // 2 if swiglu else N
+    if y is None:
+        y = torch.empty((M, cols), dtype=dt, device=x.device)
+    nvfp4_grouped_gemm_w4a16(x, x.stride(0), x.shape[0], row_index, w.q, w.sf, w.gs, offsets, G, M, N, w.K, y,
+                             out_dtype, EPI_SWIGLU if swiglu else EPI_NONE, dev_status)
+    return y
 
 
 def swiglu_quantize(y: torch.Tensor, offsets, num_groups: int, layout=SF_MMA_TILED, out: Optional[Packed] = None,

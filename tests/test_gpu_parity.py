@@ -820,3 +820,74 @@ def test_device_generator_matches_host():
     assert np.array_equal(to_np(c), synthetic.mxfp4_codes(1, 9, 4096, start_byte=64))
     e = sc.mxfp4_exponents(1, 10, 999, lo=-10, start=7)
     assert np.array_equal(to_np(e), synthetic.mxfp4_exponents(1, 10, 999, lo=-10, start=7))
+
+
+# --------------------------------------------------------------------------- W4A16 grouped GEMM
+def _w4a16_case(seed, counts, N, K, T):
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    R, E = int(offsets[-1]), len(counts)
+    rng = np.random.default_rng(seed)
+    ri = rng.integers(0, T, R).astype(np.int32)                 # gathered token rows
+    x = synthetic.gaussian_bf16(seed, synthetic.STREAMS["x"], (T, K), outlier_frac=0.001)
+    w = synthetic.gaussian_bf16(seed, synthetic.STREAMS["w"], (E * N, K), sigma=0.02)
+    qw, sw, gw = _packed_weights(w, E, N, K)
+    a = synthetic.bf16_bits_to_f32(x[ri]).astype(np.float64)
+    bw = oracle.dequantize_f64(qw, sw, np.repeat(gw, N)).reshape(E, N, K)
+    y_ref, s_ref = oracle.grouped_gemm_f64(a, bw, offsets)
+    L = layer()
+    wp = L.Packed(to_dev(qw), to_dev(sw), to_dev(gw), E * N, K, 0)
+    return L, x, ri, offsets, wp, y_ref, s_ref
+
+
+@pytest.mark.parametrize("K", [1024, 1088])
+def test_w4a16_grouped(K):
+    """bf16 activations x NVFP4 weights per expert vs fp64 on the exact
+    dequantized weights: groups of 0, 1, 3, 9, 17 and 64 tokens (several
+    8-token tiles), K an even and an odd number of 64-element chunks."""
+    counts = [0, 1, 3, 9, 17, 64]
+    N, T = 256, 40
+    L, x, ri, off, wp, y_ref, s_ref = _w4a16_case(30, counts, N, K, T)
+    s = status_word()
+    y = L.grouped_gemm_w4a16(bf16_dev(x), wp, N, to_dev(ri), to_dev(off), len(counts), out_dtype=0, dev_status=s)
+    y16 = L.grouped_gemm_w4a16(bf16_dev(x), wp, N, to_dev(ri), to_dev(off), len(counts), out_dtype=1)
+    torch.cuda.synchronize()
+    assert int(s.item()) == 0
+    ok, err, bound = gemm_tol(to_np(y), y_ref, s_ref)
+    assert ok.all(), (err / bound).max()
+    assert np.array_equal(to_np(y16), synthetic.f32_to_bf16_bits(to_np(y)))
+
+
+def test_w4a16_swiglu_epilogue():
+    """h = bf16(silu(g) * u) from the same g, u as the plain kernel's fp32
+    output: within one bf16 ulp of the oracle SwiGLU of that output."""
+    counts = [2, 0, 5, 11]
+    I, K, T = 128, 2048, 20
+    N = 2 * I
+    L, x, ri, off, wp, y_ref, s_ref = _w4a16_case(31, counts, N, K, T)
+    y32 = L.grouped_gemm_w4a16(bf16_dev(x), wp, N, to_dev(ri), to_dev(off), len(counts), out_dtype=0)
+    h = L.grouped_gemm_w4a16(bf16_dev(x), wp, N, to_dev(ri), to_dev(off), len(counts), out_dtype=1, swiglu=True)
+    torch.cuda.synchronize()
+    ok, err, bound = gemm_tol(to_np(y32), y_ref, s_ref)
+    assert ok.all()
+    d = np.abs(to_np(h).astype(np.int32) - oracle.swiglu(to_np(y32)).astype(np.int32))
+    assert (d <= 1).all() and (d == 0).mean() > 0.99
+
+
+def test_w4a16_dense_and_bad_row_index():
+    L = layer()
+    M, N, K = 5, 128, 4096
+    x = synthetic.gaussian_bf16(32, synthetic.STREAMS["x"], (M, K))
+    w = synthetic.gaussian_bf16(32, synthetic.STREAMS["w"], (N, K), sigma=0.02)
+    qw, sw, gw = _packed_weights(w, 1, N, K)
+    wp = L.Packed(to_dev(qw), to_dev(sw), to_dev(gw), N, K, 0)
+    y = to_np(L.grouped_gemm_w4a16(bf16_dev(x), wp, N, out_dtype=0))
+    a = synthetic.bf16_bits_to_f32(x).astype(np.float64)
+    b = oracle.dequantize_f64(qw, sw, np.full(N, gw[0], np.float32))
+    y_ref, s_ref = oracle.gemm_f64(a, b)
+    ok, err, bound = gemm_tol(y, y_ref, s_ref)
+    assert ok.all()
+    s = status_word()
+    bad = np.array([0, 1, 7, 2], dtype=np.int32)                 # 7 is past the 5 rows of x
+    L.grouped_gemm_w4a16(bf16_dev(x), wp, N, to_dev(bad), out_dtype=0, dev_status=s)
+    torch.cuda.synchronize()
+    assert int(s.item()) == 19
