@@ -377,6 +377,31 @@ def comp_dense_mlp(device, iters, warmup, flush):
                          "frac": round(tf / FP4_PEAK, 4)}}
 
 
+def comp_moe_static_h(device, iters, warmup, flush):
+    """The headline MoE layer with a calibrated (given) global for the down
+    projection's input: dispatch quantize -> gate_up whose SwiGLU epilogue
+    writes NVFP4 h -> down.  The scale comes from one dynamic forward."""
+    import torch
+
+    from nvfp4_w4a4_quantized_04_b200 import layer as L
+    E, T, H, I, k = 512, 8192, 4096, 1024, 10
+    moe, x, ri, off, r, R = setup_moe(device, 0, E, T, H, I, k)
+    sl = r["slot_dev"]
+    L.calibrate_h_scale(moe, x, ri, off, slot=sl)
+    ms = timed(lambda: moe.forward(x, ri, off, slot=sl), iters, warmup, flush)
+    a1 = L.moe_quantize(x, sl, off, E, out=moe.a1, ws=moe.ws, rows=R)
+    g1 = timed(lambda: L.grouped_gemm_swiglu_nvfp4(a1, moe.w_gate_up, 2 * I, moe.h_scale, out=moe.a2), iters,
+               warmup, flush)
+    flops = moe_flops(R, H, I)
+    e_t = int((np.diff(r["offsets"]) > 0).sum())
+    g1_bytes = gemm_bytes(R, e_t, 2 * I, H) - R * 2 * I * 2 + R * I * (0.5 + 1 / 16)
+    moe.h_scale = None
+    return {"workload": f"moe_routed_experts_e{E}_top{k}_t{T}_h{H}_i{I}_given_down_input_scale",
+            "layer_ms": round(ms, 4), "layer_tflops": round(flops / (ms * 1e-3) / 1e12, 1),
+            "gate_up_swiglu_nvfp4_ms": round(g1, 4), "gate_up_gbs": round(gbs(g1_bytes, g1), 1),
+            "gate_up_frac_hbm": round(gbs(g1_bytes, g1) / HBM_PEAK, 4)}
+
+
 def comp_decode_moe(device, iters, warmup, flush):
     """Decode MoE: 384 experts, 64 tokens, top-10 Zipf(1.1) routing (seed 7),
     hidden 7168, intermediate 2048, weights generated as MXFP4 and remapped."""
@@ -579,7 +604,8 @@ def comp_moe_full(device, iters, warmup, flush):
             "combine_frac_hbm": round(gbs(comb_bytes, t_comb) / HBM_PEAK, 4)}
 
 
-COMPONENTS = {"moe_full": comp_moe_full, "dense_mlp": comp_dense_mlp, "decode_moe": comp_decode_moe,
+COMPONENTS = {"moe_full": comp_moe_full, "moe_static_h": comp_moe_static_h, "dense_mlp": comp_dense_mlp,
+              "decode_moe": comp_decode_moe,
               "decode_w4a16": comp_decode_w4a16, "kv_cache": comp_kv,
               "act_quant_sweep": comp_act_sweep, "remap": comp_remap}
 

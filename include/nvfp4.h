@@ -228,6 +228,30 @@ nvfp4_status nvfp4_grouped_gemm(const uint8_t *a_q, const uint8_t *a_sf, const f
                                 void *workspace, int32_t *dev_status, cudaStream_t stream);
 
 /*
+ * nvfp4_grouped_gemm_swiglu_nvfp4 -- the gate_up grouped GEMM with the SwiGLU
+ * epilogue emitting NVFP4 h directly, for a down projection whose input
+ * global scale is given (calibrated).
+ * [P1: activation scales from calibration, the checkpoints' input_scale;
+ *  the same two-level NVFP4 block encoding as nvfp4_quantize.]
+ * h = bf16(silu(g) * u) exactly as with NVFP4_EPI_SWIGLU, then every 16
+ * columns of a routed row are quantized with the expert's h_gs[e]: the bytes
+ * nvfp4_quantize would write for that bf16 h in GIVEN mode, grouped by
+ * expert, MMA_TILED.  h itself never reaches memory.
+ *   a_*, b_*, expert_offsets, num_experts, M_total, N, K  as nvfp4_grouped_gemm
+ *               (b is the gate/up-interleaved fused weight of NVFP4_EPI_SWIGLU).
+ *   h_gs        fp32 [E], > 0 and finite (else NVFP4_ERR_INVALID_ARG in dev_status).
+ *   h_q, h_sf   uint8 [nvfp4_padded_rows_bound(M_total, E), N/4] codes and their
+ *               MMA-tiled scales, in the expert slots of the gate_up input;
+ *               padding rows are not written.  16-byte aligned h_q.
+ *   dev_status  also NVFP4_ERR_NONFINITE (non-finite h), NVFP4_ERR_TIMEOUT.
+ */
+nvfp4_status nvfp4_grouped_gemm_swiglu_nvfp4(const uint8_t *a_q, const uint8_t *a_sf, const float *a_gs,
+                                             const uint8_t *b_q, const uint8_t *b_sf, const float *b_gs,
+                                             const int32_t *expert_offsets, int num_experts, int64_t M_total,
+                                             int64_t N, int64_t K, const float *h_gs, uint8_t *h_q, uint8_t *h_sf,
+                                             void *workspace, int32_t *dev_status, cudaStream_t stream);
+
+/*
  * nvfp4_grouped_gemm_w4a16 -- weight-only NVFP4 grouped GEMM with bf16
  * activations: Y_e = X_e (b_gs[e] * W_e)^T for every expert e, fp32 accumulate.
  * [P5: the MTP layer's experts are W4A16_NVFP4 -- NVFP4 weights, BF16

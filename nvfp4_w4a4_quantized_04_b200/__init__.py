@@ -46,7 +46,7 @@ EXPORTS = [
     "nvfp4_quantize", "nvfp4_dequantize", "mxfp4_to_nvfp4", "nvfp4_grouped_gemm",
     "nvfp4_swiglu_quantize", "nvfp4_kv_quantize", "nvfp4_kv_dequantize", "nvfp4_quantize_noalloc",
     "nvfp4_moe_route_workspace_size", "nvfp4_moe_route", "nvfp4_moe_combine", "nvfp4_moe_quantize",
-    "nvfp4_gemm_select_kernel", "nvfp4_grouped_gemm_w4a16",
+    "nvfp4_gemm_select_kernel", "nvfp4_grouped_gemm_w4a16", "nvfp4_grouped_gemm_swiglu_nvfp4",
 ]
 NOALLOC_MAX_GROUPS = 1024
 
@@ -74,6 +74,8 @@ def load_library(path: str = LIB_PATH):
     L.nvfp4_padded_rows_bound.argtypes = [i64, i32]
     L.nvfp4_quantize.restype = i32
     L.nvfp4_quantize.argtypes = [P, i64, i64, i64, P, P, i32, i32, P, P, P, i32, P, P, P]
+    L.nvfp4_grouped_gemm_swiglu_nvfp4.restype = i32
+    L.nvfp4_grouped_gemm_swiglu_nvfp4.argtypes = [P, P, P, P, P, P, P, i32, i64, i64, i64, P, P, P, P, P, P]
     L.nvfp4_grouped_gemm_w4a16.restype = i32
     L.nvfp4_grouped_gemm_w4a16.argtypes = [P, i64, i64, P, P, P, P, P, i32, i64, i64, i64, P, i32, i32, P, P]
     L.nvfp4_gemm_select_kernel.restype = i32
@@ -151,6 +153,17 @@ def nvfp4_quantize_noalloc(x, rows, K, ld_x, row_index, group_offsets, num_group
         _ptr(global_scale), _ptr(q), _ptr(sf), sf_layout, _ptr(dev_status), _stream(stream))
     if check:
         _check(st, "nvfp4_quantize_noalloc")
+    return st
+
+
+def nvfp4_grouped_gemm_swiglu_nvfp4(a_q, a_sf, a_gs, b_q, b_sf, b_gs, expert_offsets, num_experts, M_total, N, K,
+                                    h_gs, h_q, h_sf, workspace=None, dev_status=None, stream=None, check=True) -> int:
+    """gate_up GEMM whose SwiGLU epilogue writes NVFP4 h with a given global per expert."""
+    st = load_library().nvfp4_grouped_gemm_swiglu_nvfp4(
+        _ptr(a_q), _ptr(a_sf), _ptr(a_gs), _ptr(b_q), _ptr(b_sf), _ptr(b_gs), _ptr(expert_offsets), num_experts,
+        M_total, N, K, _ptr(h_gs), _ptr(h_q), _ptr(h_sf), _ptr(workspace), _ptr(dev_status), _stream(stream))
+    if check:
+        _check(st, "nvfp4_grouped_gemm_swiglu_nvfp4")
     return st
 
 

@@ -58,7 +58,7 @@ constexpr int SMEM_BYTES = OFF_GROUPS + GROUP_TABLE_BYTES + 1024;   // +1024 for
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
 // ------------------------------------------------------------------ kernel
-template <bool kSwiglu, bool kBf16Out>
+template <bool kSwiglu, bool kBf16Out, bool kQuantH = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(
     const __grid_constant__ CUtensorMap tmap_w,
     const __grid_constant__ CUtensorMap tmap_x128,
@@ -66,7 +66,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(
     const uint8_t *__restrict__ w_sf, const uint8_t *__restrict__ x_sf,
     const float *__restrict__ w_gs, const float *__restrict__ x_gs,
     const int32_t *__restrict__ expert_offsets, int E, int M_total, int N, int K,
-    void *__restrict__ y, float *__restrict__ amax_out, int32_t *dev_status) {
+    void *__restrict__ y, float *__restrict__ amax_out, int32_t *dev_status, HQuantOut hq) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   const uint32_t sbase = smem_u32(smem);
@@ -263,8 +263,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(
       if (!mbar_wait_warp(bar_acc_full + 8 * ab, (titer >> 1) & 1, abort_flag, dev_status)) break;
       tc_fence_after();
       const float alpha = __fmul_rn(x_gs[T.e], w_gs[T.e]);
-      epilogue_tile<kSwiglu, kBf16Out>(T, tmem_base + lane_base + ab * TMEM_ACC_STRIDE, alpha, epi, quad, lane, N, y,
-                                       amax_out, bar_acc_empty + 8 * ab, false);
+      epilogue_tile<kSwiglu, kBf16Out, kQuantH>(T, tmem_base + lane_base + ab * TMEM_ACC_STRIDE, alpha, epi, quad,
+                                                lane, N, y, amax_out, bar_acc_empty + 8 * ab, false, hq, dev_status);
     }
   }
 
@@ -286,7 +286,7 @@ namespace {
 
 int g_sms = 0;
 int g_gemm_kernel = 0;      // 0 automatic (one CTA per tile), 1 one CTA per tile, 2 CTA pairs
-bool g_attr_set[3] = {false, false, false};
+bool g_attr_set[4] = {false, false, false, false};
 
 }  // namespace
 
@@ -338,7 +338,7 @@ extern "C" nvfp4_status nvfp4_grouped_gemm(const uint8_t *a_q, const uint8_t *a_
   }
   kern<<<g_sms, gemm::NUM_THREADS, gemm::SMEM_BYTES, stream>>>(tw, tx128, tx64, tx32, b_sf, a_sf, b_gs, a_gs,
                                                                expert_offsets, E, (int)M_total, (int)N, (int)K, y,
-                                                               amax_out, dev_status);
+                                                               amax_out, dev_status, gemm::HQuantOut{});
   return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 
@@ -346,4 +346,49 @@ extern "C" nvfp4_status nvfp4_gemm_select_kernel(int mode) {
   if (mode < 0 || mode > 2) return NVFP4_ERR_INVALID_ARG;
   g_gemm_kernel = mode;
   return NVFP4_OK;
+}
+
+extern "C" nvfp4_status nvfp4_grouped_gemm_swiglu_nvfp4(const uint8_t *a_q, const uint8_t *a_sf, const float *a_gs,
+                                                      const uint8_t *b_q, const uint8_t *b_sf, const float *b_gs,
+                                                      const int32_t *expert_offsets, int num_experts, int64_t M_total,
+                                                      int64_t N, int64_t K, const float *h_gs, uint8_t *h_q,
+                                                      uint8_t *h_sf, void *workspace, int32_t *dev_status,
+                                                      cudaStream_t stream) {
+  (void)workspace;
+  const int E = expert_offsets ? num_experts : 1;
+  if (E < 1 || E > gemm::kMaxExperts) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (M_total < 0 || N <= 0 || K <= 0) return NVFP4_ERR_INVALID_ARG;
+  if (N % 128 != 0 || K % 256 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if ((int64_t)E * N > ((int64_t)1 << 31) - 1 || M_total > ((int64_t)1 << 30)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (M_total == 0) return NVFP4_OK;
+  if (!a_q || !a_sf || !a_gs || !b_q || !b_sf || !b_gs || !h_gs || !h_q || !h_sf) return NVFP4_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(a_q) | reinterpret_cast<uintptr_t>(b_q) | reinterpret_cast<uintptr_t>(a_sf) |
+       reinterpret_cast<uintptr_t>(b_sf) | reinterpret_cast<uintptr_t>(h_q)) & 15u)
+    return NVFP4_ERR_INVALID_ARG;
+  const int64_t x_rows = nvfp4_padded_rows_bound(M_total, E);
+  CUtensorMap tw, tx128, tx64, tx32;
+  if (!gemm::make_map(&tw, b_q, (uint64_t)E * N, (uint64_t)K / 2, 128)) return NVFP4_ERR_CUDA;
+  if (!gemm::make_map(&tx128, a_q, (uint64_t)x_rows, (uint64_t)K / 2, 128)) return NVFP4_ERR_CUDA;
+  if (!gemm::make_map(&tx64, a_q, (uint64_t)x_rows, (uint64_t)K / 2, 64)) return NVFP4_ERR_CUDA;
+  if (!gemm::make_map(&tx32, a_q, (uint64_t)x_rows, (uint64_t)K / 2, 32)) return NVFP4_ERR_CUDA;
+  if (g_sms == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&g_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (g_sms <= 0) g_sms = 148;
+  }
+  auto kern = gemm::grouped_gemm_kernel<true, true, true>;
+  if (!g_attr_set[3]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::SMEM_BYTES) != cudaSuccess)
+      return NVFP4_ERR_CUDA;
+    g_attr_set[3] = true;
+  }
+  gemm::HQuantOut hq;
+  hq.gs = h_gs;
+  hq.q = h_q;
+  hq.sf = h_sf;
+  kern<<<g_sms, gemm::NUM_THREADS, gemm::SMEM_BYTES, stream>>>(tw, tx128, tx64, tx32, b_sf, a_sf, b_gs, a_gs,
+                                                               expert_offsets, E, (int)M_total, (int)N, (int)K, nullptr,
+                                                               nullptr, dev_status, hq);
+  return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }

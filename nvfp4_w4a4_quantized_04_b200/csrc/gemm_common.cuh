@@ -404,6 +404,47 @@ __device__ __forceinline__ void sf_stage_to_tmem(uint32_t tcol, uint32_t sfw_add
   tc_wait_st();
 }
 
+// One 16-element block of bf16 values encoded with a given global s_g
+// (t_g = 6 s_g): the block amax, S = e4m3(a_b / t_g), e = S * s_g,
+// r = 1/e (0 when e is 0), codes = e2m1(x * r), each step one IEEE
+// round-to-nearest-even fp32 operation; a NaN product (0 * inf) encodes as +0.
+__device__ __forceinline__ uint2 encode16_given(const uint4 &va, const uint4 &vb, float s_g, float t_g, uint32_t &S,
+                                                bool &nonfinite) {
+  const uint32_t w[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
+  uint32_t m2 = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) m2 = __vmaxu2(m2, w[i] & 0x7FFF7FFFu);
+  const uint32_t m = max(m2 & 0xFFFFu, m2 >> 16);
+  nonfinite = m >= 0x7F80u;
+  S = f32_to_e4m3_satfinite(__fdiv_rn(__uint_as_float(m << 16), t_g));
+  const float e = __fmul_rn(e4m3_to_f32(S), s_g);
+  const float r = (e == 0.0f) ? 0.0f : __frcp_rn(e);
+  uint32_t out[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    float v[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t x = w[4 * h + i];
+      v[2 * i] = __fmul_rn(__uint_as_float(x << 16), r);
+      v[2 * i + 1] = __fmul_rn(__uint_as_float(x & 0xFFFF0000u), r);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = isnan(v[i]) ? 0.0f : v[i];
+    out[h] = f32x8_to_e2m1x8(v);
+  }
+  return make_uint2(out[0], out[1]);
+}
+
+// NVFP4 output of the SwiGLU epilogue (h quantized with a given global per
+// expert): codes [slot rows, I/2] and MMA-tiled scales in the activation slot
+// layout of the gate_up input.
+struct HQuantOut {
+  const float *gs = nullptr;    // [E] given global scale of h
+  uint8_t *q = nullptr;
+  uint8_t *sf = nullptr;
+};
+
 // Epilogue of one tile for the calling warp (lane quadrant `quad`, 32
 // accumulator rows = 32 weight rows of this CTA): tcgen05.ld the accumulator
 // 64 columns (tokens) at a time, scale by alpha = a_gs[e] * b_gs[e], and store
@@ -411,11 +452,23 @@ __device__ __forceinline__ void sf_stage_to_tmem(uint32_t tcol, uint32_t sfw_add
 // the expert's max |h|.  Once the last columns are in registers the
 // accumulator is handed back by an arrive on `acc_empty` (in the pair's leader
 // CTA when release_remote).
-template <bool kSwiglu, bool kBf16Out>
+// With kQuantH (SwiGLU only) h is not stored: each 16-column block of a
+// token (one warp's 16 columns) is quantized on the spot with the expert's
+// given global, exactly as nvfp4_quantize in GIVEN mode would quantize the
+// bf16 h, and the codes and the E4M3 scale are written to hq.
+template <bool kSwiglu, bool kBf16Out, bool kQuantH = false>
 __device__ __forceinline__ void epilogue_tile(const Tile &T, uint32_t tacc, float alpha, uint32_t epi, int quad,
                                               int lane, int N, void *__restrict__ y, float *__restrict__ amax_out,
-                                              uint32_t acc_empty, bool release_remote) {
+                                              uint32_t acc_empty, bool release_remote,
+                                              const HQuantOut &hq = HQuantOut{}, int32_t *dev_status = nullptr) {
   uint32_t hmax = 0;                           // SwiGLU: max |h| bits of this lane
+  float q_sg = 1.0f, q_tg = 6.0f;
+  bool q_bad = false, q_gs_bad = false;
+  if constexpr (kQuantH) {
+    q_sg = hq.gs[T.e];
+    q_tg = __fmul_rn(6.0f, q_sg);
+    if (!(q_sg > 0.0f) || !isfinite(q_sg)) q_gs_bad = true;
+  }
   for (int c0 = 0; c0 < T.n_valid; c0 += 64) {
     uint32_t r[64];
     tc_ld32_nowait(tacc + (uint32_t)c0, r);
@@ -454,10 +507,28 @@ __device__ __forceinline__ void epilogue_tile(const Tile &T, uint32_t tacc, floa
           const float sv = __fdividef(gv, 1.0f + __expf(-gv));
           const __nv_bfloat16 hv = __float2bfloat16_rn(__fmul_rn(sv, uv));
           const uint16_t hb = *reinterpret_cast<const uint16_t *>(&hv);
-          if (my0 + j < rows_here) hmax = max(hmax, (uint32_t)(hb & 0x7FFFu));
+          if (!kQuantH && my0 + j < rows_here) hmax = max(hmax, (uint32_t)(hb & 0x7FFFu));
           asm volatile("st.shared.b16 [%0], %1;" :: "r"(epi + half + j * 32 + (lane & 15) * 2), "h"(hb) : "memory");
         }
         __syncwarp();
+        if constexpr (kQuantH) {
+          // lane L encodes token row L of this sub: its 16 columns are one block
+          if (lane < rows_here) {
+            const uint32_t ra = epi + (lane >> 4) * 576 + (lane & 15) * 32;
+            const uint4 va = lds128(ra), vb = lds128(ra + 16);
+            uint32_t S;
+            bool nonfinite;
+            const uint2 codes = encode16_given(va, vb, q_sg, q_tg, S, nonfinite);
+            q_bad |= nonfinite;
+            const int NH = N / 2;
+            const int64_t p = (int64_t)T.x_row0 + tok0 + lane;             // slot row of this token
+            const int col0 = T.n_col0 + quad * 16;
+            *reinterpret_cast<uint2 *>(hq.q + p * (NH / 2) + col0 / 2) = codes;
+            hq.sf[sf_tiled_offset(p, col0 / 16, NH / 16)] = (uint8_t)S;
+          }
+          __syncwarp();
+          continue;
+        }
         const int NH = N / 2;
         __nv_bfloat16 *hbase = reinterpret_cast<__nv_bfloat16 *>(y) + (int64_t)(T.y_row0 + tok0) * NH +
                                T.n_col0 + quad * 16;
@@ -518,7 +589,10 @@ __device__ __forceinline__ void epilogue_tile(const Tile &T, uint32_t tacc, floa
       }
     }
   }
-  if (kSwiglu) {
+  if constexpr (kQuantH) {
+    if (q_gs_bad) report(dev_status, NVFP4_ERR_INVALID_ARG);
+    if (q_bad) report(dev_status, NVFP4_ERR_NONFINITE);
+  } else if (kSwiglu) {
 #pragma unroll
     for (int d = 16; d > 0; d >>= 1) hmax = max(hmax, __shfl_xor_sync(0xffffffffu, hmax, d));
     if (lane == 0 && hmax) atomicMax(reinterpret_cast<uint32_t *>(amax_out) + T.e, hmax << 16);

@@ -14,7 +14,8 @@ from typing import Optional
 import torch
 
 from . import (EPI_NONE, EPI_SWIGLU, GS_AMAX_GIVEN, GS_FROM_AMAX, GS_GIVEN, OUT_BF16, OUT_F32, SF_MMA_TILED, SF_ROWMAJOR,
-               mxfp4_to_nvfp4, nvfp4_dequantize, nvfp4_grouped_gemm, nvfp4_grouped_gemm_w4a16, nvfp4_moe_combine,
+               mxfp4_to_nvfp4, nvfp4_dequantize, nvfp4_grouped_gemm, nvfp4_grouped_gemm_swiglu_nvfp4,
+               nvfp4_grouped_gemm_w4a16, nvfp4_moe_combine,
                nvfp4_moe_route,
                nvfp4_moe_quantize, nvfp4_moe_route_workspace_size, nvfp4_padded_rows_bound, nvfp4_quantize,
                nvfp4_swiglu_quantize,
@@ -166,6 +167,22 @@ def grouped_gemm_swiglu(a: Packed, w_gate_up: Packed, N: int, h=None, amax=None,
     return h, amax
 
 
+def grouped_gemm_swiglu_nvfp4(a: Packed, w_gate_up: Packed, N: int, h_gs: torch.Tensor, out: Optional[Packed] = None,
+                              dev_status=None) -> Packed:
+    """gate_up GEMM + SwiGLU whose epilogue quantizes h with the given per-expert
+    global ``h_gs`` (the down projection's calibrated input scale): the packed
+    down-GEMM input, with no bf16 h in memory."""
+    assert a.layout == SF_MMA_TILED and w_gate_up.layout == SF_MMA_TILED
+    E = a.num_groups if a.offsets is not None else 1
+    I = N // 2
+    p = out if out is not None else empty_packed(a.rows, I, E, a.offsets, SF_MMA_TILED, a.q.device)
+    p.offsets, p.num_groups, p.rows = a.offsets, E, a.rows
+    p.gs = h_gs
+    nvfp4_grouped_gemm_swiglu_nvfp4(a.q, a.sf, a.gs, w_gate_up.q, w_gate_up.sf, w_gate_up.gs, a.offsets, E, a.rows,
+                                    N, a.K, h_gs, p.q, p.sf, None, dev_status)
+    return p
+
+
 def grouped_gemm_w4a16(x: torch.Tensor, w: Packed, N: int, row_index=None, offsets=None, num_groups: int = 1,
                        rows=None, out_dtype=OUT_BF16, swiglu=False, y=None, dev_status=None) -> torch.Tensor:
     """Weight-only NVFP4 (row-major scales) x bf16 activations, per expert:
@@ -203,12 +220,15 @@ class MoEExperts:
     each expert = gate, I..2I-1 = up; with ``fused_swiglu`` the rows are in the
     order of ``gate_up_interleave_index`` instead.  w_down: packed [E*H, I].
     forward(x bf16 [T, H], row_index int32 [R], offsets int32 [E+1]) -> Y bf16 [R, H]
-    in routed order (the weighted combine is outside this layer).
+    in routed order (the weighted combine is outside this layer).  With
+    ``h_scale`` set (a given down-input global per expert, see
+    ``calibrate_h_scale``) the gate_up epilogue writes NVFP4 h directly.
     """
 
     def __init__(self, w_gate_up: Packed, w_down: Packed, E: int, H: int, I: int, max_rows: int,
                  out_dtype=OUT_BF16, mid_dtype=OUT_BF16, device="cuda", fused_swiglu: bool = False):
         self.fused_swiglu = fused_swiglu
+        self.h_scale: Optional[torch.Tensor] = None   # given down-input global per expert (fp32 [E])
         self.amax = torch.zeros(E, dtype=torch.float32, device=device)
         self.w_gate_up, self.w_down = w_gate_up, w_down
         self.E, self.H, self.I = E, H, I
@@ -236,7 +256,11 @@ class MoEExperts:
         else:
             a1 = quantize(x, row_index, offsets, E, SF_MMA_TILED, out=self.a1, ws=self.ws, dev_status=dev_status,
                           rows=R)
-        if self.fused_swiglu:
+        if self.h_scale is not None:
+            # calibrated down-input global: the gate_up epilogue writes NVFP4 h itself
+            a2 = grouped_gemm_swiglu_nvfp4(a1, self.w_gate_up, 2 * I, self.h_scale, out=self.a2,
+                                           dev_status=dev_status)
+        elif self.fused_swiglu:
             # SwiGLU in the gate_up epilogue; its amax feeds the requantize directly
             h, amax = grouped_gemm_swiglu(a1, self.w_gate_up, 2 * I, h=self.h[:R], amax=self.amax,
                                           dev_status=dev_status)
@@ -253,6 +277,19 @@ class MoEExperts:
         y2 = self.y2[:R]
         grouped_gemm(a2, self.w_down, H, self.out_dtype, y=y2, dev_status=dev_status)
         return y2
+
+
+def calibrate_h_scale(experts: "MoEExperts", x, row_index, offsets, slot=None, margin: float = 1.0) -> torch.Tensor:
+    """A down-input global per expert from one dynamic forward (s_g = margin *
+    max|h| / 2688, 1 for an expert without tokens), as a calibration pass would
+    set the checkpoint's input_scale; installs it on ``experts``."""
+    assert experts.fused_swiglu
+    experts.h_scale = None
+    experts.forward(x, row_index, offsets, slot=slot)
+    gs = experts.amax.clone() * (margin / 2688.0)
+    gs[gs == 0] = 1.0
+    experts.h_scale = gs
+    return gs
 
 
 def route(topk_ids: torch.Tensor, num_experts: int, dev_status=None):

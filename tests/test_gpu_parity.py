@@ -556,6 +556,60 @@ def test_gemm_swiglu_epilogue(gemm_kernel):
     assert np.array_equal(to_np(amax), want)
 
 
+def test_gemm_swiglu_nvfp4_epilogue():
+    """The epilogue that quantizes h with a given global per expert writes the
+    bytes the oracle's GIVEN-mode quantize writes for the device's bf16 h
+    (taken from the SwiGLU epilogue of the same GEMM); padding rows untouched.
+    One expert's global is tiny, so its block scales saturate at 448."""
+    L = layer()
+    E, I, K = 5, 256, 512
+    N = 2 * I
+    counts = [3, 0, 200, 70, 129]
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    R = int(offsets[-1])
+    x = synthetic.gaussian_bf16(16, synthetic.STREAMS["x"], (R, K), outlier_frac=0.001)
+    w = synthetic.gaussian_bf16(16, synthetic.STREAMS["w_gate_up"], (E * N, K), sigma=0.02)
+    q, sf, gs, qs, ss = _packed_acts(x, None, offsets, E)
+    il = L.gate_up_interleave_index(E, I, "cpu").numpy()
+    qw, sw, gw = _packed_weights(w[il], E, N, K)
+    nv = nvmod()
+    bound = nv.nvfp4_padded_rows_bound(R, E)
+    qa = np.zeros((bound, K // 2), np.uint8)
+    qa[:qs.shape[0]] = qs
+    sa = np.zeros((bound, K // 16), np.uint8)
+    sa[:ss.shape[0]] = ss
+    a = L.Packed(to_dev(qa), to_dev(tile(sa)), to_dev(gs), R, K, 1, to_dev(offsets), E)
+    wp = L.Packed(to_dev(qw), to_dev(tile(sw)), to_dev(gw), E * N, K, 1)
+    h, amax = L.grouped_gemm_swiglu(a, wp, N)
+    torch.cuda.synchronize()
+    h_gs = (to_np(amax) / 2688.0 * 1.3).astype(np.float32)
+    h_gs[h_gs == 0] = 1.0
+    h_gs[4] = np.float32(to_np(amax)[4] / 2688.0 / 50.0)        # block scales clip at 448
+    out = L.empty_packed(R, I, E, to_dev(offsets), 1)
+    out.q.fill_(0xAB)
+    out.sf.fill_(0xAB)
+    st = status_word()
+    p = L.grouped_gemm_swiglu_nvfp4(a, wp, N, to_dev(h_gs), out=out, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    q_ref, sf_ref, _, ost = oracle.quantize(to_np(h), None, offsets, global_scale=h_gs)
+    assert ost == 0
+    rows, starts = slot_rows(offsets)
+    qd = to_np(p.q)
+    assert np.array_equal(qd[rows], q_ref)
+    sfm = untile(to_np(p.sf), qd.shape[0], I // 16)
+    assert np.array_equal(sfm[rows], sf_ref)
+    assert (sfm[rows[offsets[4]:]] == 0x7E).any()                  # saturated scales on expert 4
+    pad = np.setdiff1d(np.arange(int(starts[-1])), rows)
+    assert (qd[pad] == 0xAB).all() and (sfm[pad] == 0xAB).all()
+    bad = h_gs.copy()
+    bad[2] = 0.0
+    st2 = status_word()
+    L.grouped_gemm_swiglu_nvfp4(a, wp, N, to_dev(bad), dev_status=st2)
+    torch.cuda.synchronize()
+    assert int(st2.item()) == 1
+
+
 def test_moe_layer_fused_swiglu_stagewise():
     L = layer()
     T, H, I, E, k = 96, 256, 256, 8, 3
@@ -600,6 +654,42 @@ def test_moe_layer_fused_swiglu_stagewise():
     assert np.array_equal(to_np(moe.a2.gs), gs2)
     assert np.array_equal(to_np(moe.a2.q)[rows], q2)
     a2 = oracle.dequantize_f64(q2, sf2, oracle.rows_global_scale(gs2, off, R))
+    bd = oracle.dequantize_f64(qd, sd, np.repeat(gd, H)).reshape(E, H, I)
+    y2_ref, s2_ref = oracle.grouped_gemm_f64(a2, bd, off)
+    ok, err, bound = gemm_tol(to_np(y2), y2_ref, s2_ref)
+    assert ok.all(), (err / bound).max()
+
+
+def test_moe_layer_given_down_input_scale():
+    """MoEExperts with a calibrated down-input global: the packed h equals the
+    oracle's GIVEN-mode quantize of the dynamic path's h, and the down GEMM
+    meets the tolerance on it."""
+    L = layer()
+    T, H, I, E, k = 96, 256, 256, 8, 3
+    x = synthetic.gaussian_bf16(17, synthetic.STREAMS["x"], (T, H))
+    r = synthetic.route_topk_softmax(17, T, E, k)
+    off = r["offsets"]
+    R = len(r["row_index"])
+    wgu = synthetic.gaussian_bf16(17, synthetic.STREAMS["w_gate_up"], (E * 2 * I, H), sigma=0.02)
+    wd = synthetic.gaussian_bf16(17, synthetic.STREAMS["w_down"], (E * H, I), sigma=0.02)
+    il = L.gate_up_interleave_index(E, I, "cpu").numpy()
+    qg, sg, gg = _packed_weights(wgu[il], E, 2 * I, H)
+    qd, sd, gd = _packed_weights(wd, E, H, I)
+    Wgu = L.Packed(to_dev(qg), to_dev(tile(sg)), to_dev(gg), E * 2 * I, H, 1)
+    Wd = L.Packed(to_dev(qd), to_dev(tile(sd)), to_dev(gd), E * H, I, 1)
+    moe = L.MoEExperts(Wgu, Wd, E, H, I, max_rows=R, out_dtype=0, mid_dtype=0, fused_swiglu=True)
+    xd, rid, offd, sld = bf16_dev(x), to_dev(r["row_index"]), to_dev(off), to_dev(r["slot"].astype(np.int32))
+    gs_h = to_np(L.calibrate_h_scale(moe, xd, rid, offd, slot=sld, margin=1.25))
+    h_dyn = to_np(moe.h[:R]).copy()
+    s = status_word()
+    y2 = moe.forward(xd, rid, offd, dev_status=s, slot=sld)
+    torch.cuda.synchronize()
+    assert int(s.item()) == 0
+    rows, _ = slot_rows(off)
+    q2, sf2, _, st = oracle.quantize(h_dyn, None, off, global_scale=gs_h)
+    assert st == 0
+    assert np.array_equal(to_np(moe.a2.q)[rows], q2)
+    a2 = oracle.dequantize_f64(q2, sf2, oracle.rows_global_scale(gs_h, off, R))
     bd = oracle.dequantize_f64(qd, sd, np.repeat(gd, H)).reshape(E, H, I)
     y2_ref, s2_ref = oracle.grouped_gemm_f64(a2, bd, off)
     ok, err, bound = gemm_tol(to_np(y2), y2_ref, s2_ref)
