@@ -1,7 +1,7 @@
 """NVFP4 oracle -- TEST INFRASTRUCTURE ONLY.
 
 Plain CPU reference for the NVFP4 W4A4 path: E2M1 / E4M3 codecs, quantize,
-dequantize, the MXFP4 -> NVFP4 remap, SwiGLU and an fp64 GEMM of dequantized
+dequantize, the MXFP4 encoder and the MXFP4 -> NVFP4 remap, SwiGLU and an fp64 GEMM of dequantized
 operands.  The arithmetic lives in ``oracle.c`` (scalar C, no FMA
 contraction, no fast-math); this module only loads it and adds the fp64
 matrix products, for which ``numpy.matmul`` in float64 is the library step.
@@ -83,6 +83,8 @@ def lib():
             L.orc_dequantize_f64.argtypes = [P, P, P, i64, i64, P]
             L.orc_remap_mxfp4.restype = ctypes.c_int
             L.orc_remap_mxfp4.argtypes = [P, P, i64, i64, i64, P, P, P]
+            L.orc_quantize_mxfp4.restype = ctypes.c_int
+            L.orc_quantize_mxfp4.argtypes = [P, i64, i64, i64, P, P]
             L.orc_dequantize_mxfp4_f64.restype = None
             L.orc_dequantize_mxfp4_f64.argtypes = [P, P, i64, i64, P]
             L.orc_swiglu.restype = None
@@ -250,6 +252,21 @@ def remap_mxfp4(q_mx: np.ndarray, e8: np.ndarray, n_tensors: int, rows: int, K: 
     gs = np.empty(n_tensors, dtype=np.float32)
     st = lib().orc_remap_mxfp4(_p(q_mx), _p(e8), n_tensors, rows, K, _p(q_nv), _p(sf), _p(gs))
     return q_nv, sf, gs, st
+
+
+def quantize_mxfp4(x_bf16: np.ndarray):
+    """MXFP4 encode of a bf16 matrix [rows, K] (P2, the FP8 -> MXFP4 step of
+    the which-layers section; rule read as the OCP MX v1.0 conversion, see
+    ``orc_quantize_mxfp4``).  Returns (q uint8 [rows, K/2], e8 uint8 UE8M0
+    [rows, K/32], status)."""
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    R, K = x.shape
+    if K % 32:
+        raise ValueError("K must be a multiple of 32")
+    q = np.empty((R, K // 2), dtype=np.uint8)
+    e8 = np.empty((R, K // 32), dtype=np.uint8)
+    st = lib().orc_quantize_mxfp4(_p(x), R, K, K, _p(q), _p(e8))
+    return q, e8, st
 
 
 def dequantize_mxfp4_f64(q: np.ndarray, e8: np.ndarray) -> np.ndarray:

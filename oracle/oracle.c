@@ -29,7 +29,10 @@
  *    6 (also for +-inf), sign kept (a negative value rounding to 0 gives -0),
  *    NaN encodes as +0;
  *  - element 2j in bits [3:0] and element 2j+1 in bits [7:4] of byte j;
- *  - remap: g = e_max - 8 over the blocks that are not all zero.
+ *  - remap: g = e_max - 8 over the blocks that are not all zero;
+ *  - MXFP4 encode: the OCP MX v1.0 exponent rule E = floor(log2 amax) - 2,
+ *    clamped to the UE8M0 range, byte 0 for an all-zero block, 0xFF for a
+ *    block with a non-finite element.
  *
  * Compiled with -O2 -ffp-contract=off and no fast-math, so every float
  * expression below is evaluated as written.
@@ -345,6 +348,60 @@ void orc_dequantize_mxfp4_f64(const uint8_t *q, const uint8_t *e8, int64_t rows,
             uint8_t code = (k & 1) ? (byte >> 4) : (byte & 15);
             out[r * K + k] = ldexp(orc_e2m1_decode(code), (int)e8[r * (K / 32) + k / 32] - 127);
         }
+}
+
+/* ------------------------------------------------------------------ */
+/* MXFP4 encode  [P2, section 三 (which layers): the FP8 -> MXFP4 step, */
+/* one UE8M0 scale per 32 elements, lossy; format table of section 二] */
+/* ------------------------------------------------------------------ */
+
+/* The page fixes the block (32 elements) and the scale type (UE8M0, a power
+ * of two) but not how the exponent is chosen.  Reading taken: the OCP
+ * Microscaling v1.0 conversion.  Per 32-block of a row,
+ *   E = floor(log2(amax)) - 2          (2 = exponent of 6, the largest E2M1),
+ *   E clamped to [-127, 127]           (UE8M0 byte u = E + 127; 0xFF is NaN),
+ *   code_k = e2m1(x_k / 2^E)           (round to nearest even, saturating at 6).
+ * An all-zero block takes u = 0 and zero codes (signs kept).  A block holding
+ * a NaN or an infinity takes u = 0xFF and all codes 0, and the call returns
+ * ORC_ERR_NONFINITE.  The input is bf16, which holds every FP8 E4M3 value
+ * exactly, so an FP8 source is covered by passing its values as bf16.
+ * x: [rows, ld_x] bf16, K % 32 == 0; q: [rows, K/2]; e8: [rows, K/32]. */
+int orc_quantize_mxfp4(const uint16_t *x, int64_t rows, int64_t K, int64_t ld_x,
+                       uint8_t *q, uint8_t *e8) {
+    int status = ORC_OK;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t b = 0; b < K / 32; ++b) {
+            const uint16_t *xb = x + r * ld_x + b * 32;
+            uint8_t *qb = q + r * (K / 2) + b * 16;
+            double amax = 0.0;
+            int finite = 1;
+            for (int k = 0; k < 32; ++k) {
+                double v = bf16_to_f32(xb[k]);
+                if (!isfinite(v)) finite = 0;
+                else if (fabs(v) > amax) amax = fabs(v);
+            }
+            if (!finite) {
+                status = ORC_ERR_NONFINITE;
+                e8[r * (K / 32) + b] = 0xFF;
+                memset(qb, 0, 16);
+                continue;
+            }
+            int E = -127;
+            if (amax > 0.0) {
+                int e2;
+                frexp(amax, &e2);          /* amax = m * 2^e2, m in [0.5, 1) */
+                E = (e2 - 1) - 2;          /* floor(log2 amax) - 2 */
+                if (E < -127) E = -127;
+                if (E > 127) E = 127;
+            }
+            e8[r * (K / 32) + b] = (uint8_t)(E + 127);
+            for (int k = 0; k < 32; k += 2) {
+                uint8_t c0 = orc_e2m1_encode((float)ldexp(bf16_to_f32(xb[k]), -E));
+                uint8_t c1 = orc_e2m1_encode((float)ldexp(bf16_to_f32(xb[k + 1]), -E));
+                qb[k / 2] = (uint8_t)(c0 | (c1 << 4));
+            }
+        }
+    return status;
 }
 
 /* ------------------------------------------------------------------ */

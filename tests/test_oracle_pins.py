@@ -368,6 +368,120 @@ def test_remap_zero_blocks_exempt():
                           oracle.dequantize_mxfp4_f64(q, e))
 
 
+# ------------------------------------------------------------------ MXFP4 encode
+def _bf16(vals):
+    return synthetic.f32_to_bf16_bits(np.asarray(vals, dtype=np.float32))
+
+
+def _mx_block(vals):
+    x = np.zeros(32, dtype=np.float32)
+    x[:len(vals)] = vals
+    return _bf16(x).reshape(1, 32)
+
+
+def _codes(q):
+    return np.stack([q & 15, q >> 4], axis=-1).reshape(q.shape[0], -1)
+
+
+@pytest.mark.parametrize("vals, byte, first_codes", [
+    # amax 6 = 1.5 * 2^2: E = 2 - 2 = 0, the block is already on the E2M1 grid
+    ([6.0, -3.0, 0.5], 127, [7, 8 + 5, 1]),
+    # amax 7: floor(log2 7) = 2, E = 0; 7 saturates to 6 and 5 ties to 4 (even)
+    ([7.0, 5.0, -1.25], 127, [7, 6, 8 + 2]),
+    # amax 8: E = 1, so every value is halved before rounding: 3 -> 1.5, and
+    # 0.5 -> 0.25 ties to 0 (even)
+    ([8.0, 3.0, 0.5], 128, [6, 3, 0]),
+    # amax 1: E = -2, so every value is quadrupled: 0.75 -> 3, -0.25 -> -1,
+    # bf16(0.3) = 0.30078125 -> 1.203 -> 1.0
+    ([1.0, 0.75, -0.25, 0.3], 125, [6, 5, 8 + 2, 2]),
+])
+def test_mxfp4_encode_worked_blocks(vals, byte, first_codes):
+    """Blocks worked by hand from the OCP MX v1.0 rule (E = floor(log2 amax) - 2)."""
+    q, e, st = oracle.quantize_mxfp4(_mx_block(vals))
+    assert st == oracle.OK and int(e[0, 0]) == byte
+    c = _codes(q)[0]
+    assert list(c[:len(first_codes)]) == first_codes
+    assert (c[len(vals):] == 0).all()
+
+
+def test_mxfp4_encode_vs_log2_and_library_codec():
+    """Scale byte = floor(log2 amax) + 125 (numpy log2), codes = ml_dtypes E2M1
+    of x / 2^E, over blocks whose amax spans the bf16 normal and subnormal range."""
+    rows, K = 64, 256
+    x = synthetic.bf16_bits_to_f32(synthetic.gaussian_bf16(21, 1, (rows, K))).astype(np.float64)
+    mag = np.ldexp(1.0, (synthetic.words(21, 2, 0, rows * K // 32) % 250).astype(np.int64) - 130)
+    x = x * np.repeat(mag, 32).reshape(rows, K)
+    xb = synthetic.f32_to_bf16_bits(x.astype(np.float32))
+    q, e, st = oracle.quantize_mxfp4(xb)
+    assert st == oracle.OK
+    xf = synthetic.bf16_bits_to_f32(xb).astype(np.float64).reshape(rows, K // 32, 32)
+    amax = np.abs(xf).max(axis=2)
+    E = np.clip(np.floor(np.log2(np.where(amax > 0, amax, 1.0))) - 2, -127, 127).astype(np.int64)
+    E = np.where(amax > 0, E, -127)
+    assert np.array_equal(e.astype(np.int64), E + 127)
+    scaled = (xf / np.ldexp(1.0, E)[..., None]).astype(np.float32).reshape(rows, K)
+    lib = scaled.astype(ml_dtypes.float4_e2m1fn).view(np.uint8)
+    assert np.array_equal(_codes(q), lib)
+    # the subnormal and clamped end of the range is exercised
+    assert (e == 0).any() and (e > 200).any()
+
+
+def test_mxfp4_encode_error_bound_and_exact_powers():
+    """|x - deq| <= 2^E on the unsaturated grid, < 2^(E+1) where x / 2^E in (6, 8);
+    a block whose amax is a power of two reproduces its amax exactly."""
+    x = synthetic.gaussian_bf16(22, 1, (32, 512), sigma=3.0)
+    q, e, st = oracle.quantize_mxfp4(x)
+    assert st == oracle.OK
+    xf = synthetic.bf16_bits_to_f32(x).astype(np.float64)
+    y = oracle.dequantize_mxfp4_f64(q, e)
+    X = np.repeat(np.ldexp(1.0, e.astype(np.int64) - 127), 32, axis=1)
+    err = np.abs(xf - y)
+    small = np.abs(xf) <= 6 * X
+    assert (err[small] <= X[small]).all() and (err[~small] < 2 * X[~small]).all()
+    assert (~small).any()                                   # saturation happens on Gaussian data
+    xp = _mx_block([2.0 ** -5, 0.01, -0.02])
+    qp, ep, _ = oracle.quantize_mxfp4(xp)
+    assert oracle.dequantize_mxfp4_f64(qp, ep)[0, 0] == 2.0 ** -5
+
+
+def test_mxfp4_encode_zero_and_nonfinite_blocks():
+    x = np.zeros((2, 96), dtype=np.uint16)
+    x[0, 40] = 0x8000                                     # -0 in block 1
+    x[1, 5] = 0x7F80                                      # +inf in block 0
+    x[1, 70] = _bf16([1.5])[0]                            # block 2 stays encodable
+    q, e, st = oracle.quantize_mxfp4(x)
+    assert st == oracle.ERR_NONFINITE
+    assert list(e[0]) == [0, 0, 0]
+    assert _codes(q)[0, 40] == 8 and (np.delete(_codes(q)[0], 40) == 0).all()
+    assert e[1, 0] == 0xFF and (q[1, :16] == 0).all()
+    assert e[1, 2] == 125 and _codes(q)[1, 70] == 7     # 1.5 / 2^-2 = 6
+
+
+def test_mxfp4_encode_then_remap_is_lossless():
+    """The encoder's output is a valid remap input: its NVFP4 remap dequantizes
+    to the same values (the lossless remap of the format section)."""
+    rows, K = 48, 512
+    x = synthetic.gaussian_bf16(23, 1, (rows, K))
+    q, e, _ = oracle.quantize_mxfp4(x)
+    qn, sfn, gs, st = oracle.remap_mxfp4(q, e, 1, rows, K)
+    assert st == oracle.OK
+    assert np.array_equal(oracle.dequantize_f64(qn, sfn, np.full(rows, gs[0], np.float32)),
+                          oracle.dequantize_mxfp4_f64(q, e))
+
+
+def test_mxfp4_from_fp8_relative_error_matches_page():
+    """FP8 (E4M3) Gaussian weights through the encoder lose about 12 % in
+    relative L2, the figure the page prints for its FP8 -> MXFP4 step."""
+    want = FACTS["mxfp4_from_fp8_rel_l2_error_approx"]
+    x = synthetic.bf16_bits_to_f32(synthetic.gaussian_bf16(24, 1, (256, 1024)))
+    x8 = x.astype(ml_dtypes.float8_e4m3fn).astype(np.float32)
+    q, e, st = oracle.quantize_mxfp4(synthetic.f32_to_bf16_bits(x8))
+    assert st == oracle.OK
+    y = oracle.dequantize_mxfp4_f64(q, e)
+    rel = np.linalg.norm(y - x8) / np.linalg.norm(x8)
+    assert abs(rel - want) < 0.015
+
+
 # ------------------------------------------------------------------ GEMM
 def test_gemm_closed_form_integer_case():
     """All S = 1 (0x38), s_g = 1: values are multiples of 0.5, so 4*y is an
