@@ -576,6 +576,71 @@ def comp_remap(device, iters, warmup, flush):
             "frac_hbm": round(gbs(b, ms) / HBM_PEAK, 4)}
 
 
+def comp_mxfp4_encode(device, iters, warmup, flush):
+    """MXFP4 encode (one UE8M0 scale per 32 elements) of 2^28 bf16 elements as
+    [65536, 4096], tensor-core scale layout."""
+    import synthetic
+    import synthetic.cuda as sc
+    from nvfp4_w4a4_quantized_04_b200 import layer as L
+    rows, K = 65536, 4096
+    x = sc.gaussian_bf16(0, synthetic.STREAMS["x_sweep"], (rows, K))
+    q, e8 = L.mxfp4_quantize(x, layout=1)
+    ms = timed(lambda: L.mxfp4_quantize(x, layout=1), iters, warmup, flush)
+    n = rows * K
+    b = n * (2 + 0.5 + 1 / 32)
+    return {"workload": "mxfp4_encode_2^28_as_65536x4096", "ms": round(ms, 4), "gbs": round(gbs(b, ms), 1),
+            "frac_hbm": round(gbs(b, ms) / HBM_PEAK, 4), "bytes_per_element": 2 + 0.5 + 1 / 32}
+
+
+def comp_mx_gemm_routes(device, iters, warmup, flush):
+    """MXFP4 weights two ways on the headline gate_up GEMM (512 experts, 81,920
+    routed rows, N = 2048, K = 4096): the direct kind::mxf4 grouped GEMM on
+    MXFP4 activations, and the NVFP4 grouped GEMM on the losslessly remapped
+    weights with NVFP4 activations.  Operands are prepared outside the events;
+    only the GEMM launches are timed."""
+    import torch
+
+    import synthetic
+    import synthetic.cuda as sc
+    from nvfp4_w4a4_quantized_04_b200 import layer as L, nvfp4_padded_rows_bound
+    E, T, k, N, K = 512, 8192, 10, 2048, 4096
+    r = synthetic.route_topk_softmax(0, T, E, k)
+    R = len(r["row_index"])
+    off = torch.from_numpy(r["offsets"]).to(device)
+    bound = nvfp4_padded_rows_bound(R, E)
+    # activations already in their 128-aligned expert slots (padding rows hold data too)
+    xs = sc.gaussian_bf16(0, synthetic.STREAMS["x"], (bound, K))
+    w = sc.gaussian_bf16(0, synthetic.STREAMS["w_gate_up"], (E * N, K), sigma=0.02)
+    wq, we_tiled = L.mxfp4_quantize(w, layout=1)
+    _, we_rm = L.mxfp4_quantize(w, layout=0)
+    del w
+    xq, xe = L.mxfp4_quantize(xs, layout=1)
+    ws = L.workspace(E, device)
+    w_nv = L.remap_mxfp4(wq, we_rm, E, N, K, layout=1, ws=ws)
+    a_nv = L.quantize(xs, layout=1, ws=ws)
+    a_nv = L.Packed(a_nv.q, a_nv.sf, a_nv.gs.repeat(E), R, K, 1, off, E)
+    w_nv = L.Packed(w_nv.q, w_nv.sf, w_nv.gs, E * N, K, 1)
+    del xs
+    y = torch.empty((R, N), dtype=torch.bfloat16, device=device)
+    t_mx = timed(lambda: L.mx_grouped_gemm(xq, xe, wq, we_tiled, N, K, R, off, E, out_dtype=1, y=y),
+                 iters, warmup, flush)
+    t_nv = timed(lambda: L.grouped_gemm(a_nv, w_nv, N, 1, y=y), iters, warmup, flush)
+    touched = int((np.diff(r["offsets"]) > 0).sum())
+    w_mx_bytes = touched * N * K * (0.5 + 1 / 32)
+    w_nv_bytes = touched * N * K * (0.5 + 1 / 16)
+    a_mx, a_nvb = R * K * (0.5 + 1 / 32), R * K * (0.5 + 1 / 16)
+    out_b = R * N * 2
+    flops = 2.0 * R * N * K
+    b_mx, b_nv = w_mx_bytes + a_mx + out_b, w_nv_bytes + a_nvb + out_b
+    return {"workload": f"gate_up_e{E}_top{k}_t{T}_n{N}_k{K}",
+            "mxfp4_gemm_ms": round(t_mx, 4), "mxfp4_gbs": round(gbs(b_mx, t_mx), 1),
+            "mxfp4_frac_hbm": round(gbs(b_mx, t_mx) / HBM_PEAK, 4),
+            "mxfp4_tflops": round(flops / (t_mx * 1e-3) / 1e12, 1),
+            "remap_nvfp4_gemm_ms": round(t_nv, 4), "remap_nvfp4_gbs": round(gbs(b_nv, t_nv), 1),
+            "remap_nvfp4_frac_hbm": round(gbs(b_nv, t_nv) / HBM_PEAK, 4),
+            "remap_nvfp4_tflops": round(flops / (t_nv * 1e-3) / 1e12, 1)}
+
+
 def comp_moe_full(device, iters, warmup, flush):
     """The whole routed-expert block of the headline layer: on-device routing
     order from the router's top-10 ids, the NVFP4 experts, and the weighted
@@ -607,7 +672,8 @@ def comp_moe_full(device, iters, warmup, flush):
 COMPONENTS = {"moe_full": comp_moe_full, "moe_static_h": comp_moe_static_h, "dense_mlp": comp_dense_mlp,
               "decode_moe": comp_decode_moe,
               "decode_w4a16": comp_decode_w4a16, "kv_cache": comp_kv,
-              "act_quant_sweep": comp_act_sweep, "remap": comp_remap}
+              "act_quant_sweep": comp_act_sweep, "remap": comp_remap, "mxfp4_encode": comp_mxfp4_encode,
+              "mx_gemm_routes": comp_mx_gemm_routes}
 
 
 # --------------------------------------------------------------------------- CPU oracle baseline

@@ -201,6 +201,32 @@ nvfp4_status mxfp4_to_nvfp4(const uint8_t *q_mx, const uint8_t *ue8m0, int64_t n
                             int32_t *dev_status, cudaStream_t stream);
 
 /*
+ * mxfp4_quantize -- MXFP4 encode: E2M1 codes with one UE8M0 (power-of-two)
+ * scale per 32 elements.
+ * [P2, format table: MXFP4 = 32-element blocks with UE8M0 scales; P2,
+ *  which-layers section: an FP8 table is converted to MXFP4, a lossy step.
+ *  The page gives no exponent rule; this follows the OCP Microscaling v1.0
+ *  conversion.]
+ *   x        bf16 [rows, ld_x], ld_x >= K, ld_x % 8 == 0, 16-byte aligned.
+ *            (bf16 holds every FP8 E4M3 value exactly, so an FP8 source is
+ *            encoded by passing its values widened to bf16.)
+ *   rows, K  K % 32 == 0 (K % 128 == 0 for MMA_TILED); rows * K/32 < 2^31;
+ *            rows == 0 is a no-op.
+ *   q        uint8 [rows, K/2], 16-byte aligned, same nibble order as NVFP4.
+ *   ue8m0    uint8 scales, ROWMAJOR [rows, K/32] or MMA_TILED (the NVFP4 atom
+ *            layout with one scale per 32 elements: 128-row blocks, 4 scales =
+ *            128 elements per 512-byte atom; the tensor holds roundup(rows,128)
+ *            rows, padding rows not written).
+ *   dev_status  NVFP4_ERR_NONFINITE when a block holds a NaN or inf (that
+ *            block gets byte 0xFF and zero codes).
+ * Per 32-block with amax a: E = floor(log2 a) - 2 clamped to [-127, 127]
+ * (byte E + 127; an all-zero block gets 0), codes = e2m1_rne_satfinite(x * 2^-E).
+ */
+nvfp4_status mxfp4_quantize(const void *x, int64_t rows, int64_t K, int64_t ld_x, uint8_t *q,
+                            uint8_t *ue8m0, nvfp4_sf_layout sf_layout, int32_t *dev_status,
+                            cudaStream_t stream);
+
+/*
  * nvfp4_grouped_gemm -- Y_e = (a_gs[e] * b_gs[e]) * A_e B_e^T for every expert e,
  * block-scaled FP4 x FP4 on the tcgen05 tensor cores, fp32 accumulation.
  * [P2 "why NVFP4": Blackwell tensor cores multiply 4-bit operands natively;
@@ -250,6 +276,27 @@ nvfp4_status nvfp4_grouped_gemm_swiglu_nvfp4(const uint8_t *a_q, const uint8_t *
                                              const int32_t *expert_offsets, int num_experts, int64_t M_total,
                                              int64_t N, int64_t K, const float *h_gs, uint8_t *h_q, uint8_t *h_sf,
                                              void *workspace, int32_t *dev_status, cudaStream_t stream);
+
+/*
+ * mxfp4_grouped_gemm -- Y_e = A_e B_e^T for every expert e with MXFP4 operands
+ * (E2M1 codes, one UE8M0 scale per 32 elements, no global scale) on the
+ * tcgen05 tensor cores (kind::mxf4, block-scaled), fp32 accumulation.
+ * [P2, format table: MXFP4 blocks of 32 with power-of-two scales, the
+ *  checkpoint's source format before the NVFP4 remap; this is the direct
+ *  MXFP4 GEMM to set against the remap-then-NVFP4 route.]
+ *   a_q, a_sf   activations in 128-aligned expert slots (as for
+ *               nvfp4_grouped_gemm), scales from mxfp4_quantize in MMA_TILED
+ *               layout over nvfp4_padded_rows_bound(M_total, E) rows.
+ *   b_q, b_sf   weights [E, N, K/2], MMA_TILED UE8M0 scales over E*N rows.
+ *   expert_offsets, num_experts, M_total, N, K, y, out_dtype, workspace,
+ *   dev_status  as for nvfp4_grouped_gemm (N % 128 == 0, K % 256 == 0; no
+ *               epilogue option).
+ */
+nvfp4_status mxfp4_grouped_gemm(const uint8_t *a_q, const uint8_t *a_sf, const uint8_t *b_q,
+                                const uint8_t *b_sf, const int32_t *expert_offsets, int num_experts,
+                                int64_t M_total, int64_t N, int64_t K, void *y,
+                                nvfp4_out_dtype out_dtype, void *workspace, int32_t *dev_status,
+                                cudaStream_t stream);
 
 /*
  * nvfp4_grouped_gemm_w4a16 -- weight-only NVFP4 grouped GEMM with bf16

@@ -7,7 +7,8 @@ library's kernels.  There is no CPU fallback: if the library is missing or
 no CUDA device is present, the calls raise.
 
 Entry points (same names as the C ABI): ``nvfp4_quantize``,
-``nvfp4_dequantize``, ``mxfp4_to_nvfp4``, ``nvfp4_grouped_gemm``,
+``nvfp4_dequantize``, ``mxfp4_to_nvfp4``, ``mxfp4_quantize``, ``mxfp4_grouped_gemm``,
+``nvfp4_grouped_gemm``,
 ``nvfp4_swiglu_quantize``, ``nvfp4_kv_quantize``, ``nvfp4_kv_dequantize``,
 ``nvfp4_moe_quantize``, ``nvfp4_moe_route``, ``nvfp4_moe_combine``,
 ``nvfp4_quantize_noalloc``, plus ``nvfp4_workspace_size``,
@@ -47,6 +48,7 @@ EXPORTS = [
     "nvfp4_swiglu_quantize", "nvfp4_kv_quantize", "nvfp4_kv_dequantize", "nvfp4_quantize_noalloc",
     "nvfp4_moe_route_workspace_size", "nvfp4_moe_route", "nvfp4_moe_combine", "nvfp4_moe_quantize",
     "nvfp4_gemm_select_kernel", "nvfp4_grouped_gemm_w4a16", "nvfp4_grouped_gemm_swiglu_nvfp4",
+    "mxfp4_quantize", "mxfp4_grouped_gemm",
 ]
 NOALLOC_MAX_GROUPS = 1024
 
@@ -85,6 +87,10 @@ def load_library(path: str = LIB_PATH):
     L.nvfp4_dequantize.restype = i32
     L.nvfp4_dequantize.argtypes = [P, P, i32, P, P, i32, i64, i64, P, i32, P]
     L.mxfp4_to_nvfp4.restype = i32
+    L.mxfp4_quantize.restype = i32
+    L.mxfp4_grouped_gemm.restype = i32
+    L.mxfp4_grouped_gemm.argtypes = [P, P, P, P, P, i32, i64, i64, i64, P, i32, P, P, P]
+    L.mxfp4_quantize.argtypes = [P, i64, i64, i64, P, P, i32, P, P]
     L.mxfp4_to_nvfp4.argtypes = [P, P, i64, i64, i64, P, P, i32, P, P, P, P]
     L.nvfp4_grouped_gemm.restype = i32
     L.nvfp4_grouped_gemm.argtypes = [P, P, P, P, P, P, P, i32, i64, i64, i64, P, i32, i32, P, P, P, P]
@@ -213,6 +219,24 @@ def mxfp4_to_nvfp4(q_mx, ue8m0, n_tensors, rows, K, q_nv, sf_nv, sf_layout, glob
         _ptr(global_scale), _ptr(workspace), _ptr(dev_status), _stream(stream))
     if check:
         _check(st, "mxfp4_to_nvfp4")
+    return st
+
+
+def mxfp4_quantize(x, rows, K, ld_x, q, ue8m0, sf_layout, dev_status=None, stream=None, check=True) -> int:
+    st = load_library().mxfp4_quantize(_ptr(x), rows, K, ld_x, _ptr(q), _ptr(ue8m0), sf_layout, _ptr(dev_status),
+                                       _stream(stream))
+    if check:
+        _check(st, "mxfp4_quantize")
+    return st
+
+
+def mxfp4_grouped_gemm(a_q, a_sf, b_q, b_sf, expert_offsets, num_experts, M_total, N, K, y, out_dtype,
+                       workspace=None, dev_status=None, stream=None, check=True) -> int:
+    st = load_library().mxfp4_grouped_gemm(
+        _ptr(a_q), _ptr(a_sf), _ptr(b_q), _ptr(b_sf), _ptr(expert_offsets), num_experts, M_total, N, K, _ptr(y),
+        out_dtype, _ptr(workspace), _ptr(dev_status), _stream(stream))
+    if check:
+        _check(st, "mxfp4_grouped_gemm")
     return st
 
 

@@ -58,7 +58,9 @@ constexpr int SMEM_BYTES = OFF_GROUPS + GROUP_TABLE_BYTES + 1024;   // +1024 for
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
 // ------------------------------------------------------------------ kernel
-template <bool kSwiglu, bool kBf16Out, bool kQuantH = false>
+// kMx: MXFP4 operands (kind::mxf4, one UE8M0 scale per 32 elements, no
+// global scales); otherwise NVFP4 (kind::mxf4nvf4, E4M3 per 16 elements).
+template <bool kSwiglu, bool kBf16Out, bool kQuantH = false, bool kMx = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(
     const __grid_constant__ CUtensorMap tmap_w,
     const __grid_constant__ CUtensorMap tmap_x128,
@@ -119,7 +121,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
   const int total_tiles = s_tile[E];
-  const int64_t sf_row_stride = (int64_t)(K / 64) * 512;   // bytes per 128-row block of scales
+  // bytes per 128-row block of scales, and scale bytes per K stage of one row block
+  const int64_t sf_row_stride = (int64_t)(K / (kMx ? 128 : 64)) * 512;
+  constexpr uint32_t kSfStage = kMx ? 1024u : 2048u;
 
   if (warp == W_PRODUCER || warp == W_XLOAD) {
     // ================================================================ TMA producers
@@ -142,7 +146,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(
         const int rows_ld = (T.n_valid + 31) & ~31;
         const int xr0 = T.x_row0 & ~127;                               // first scale row block
         const int nrb = ((T.x_row0 & 127) + T.n_valid + 127) >> 7;     // 1 or 2
-        const uint32_t bytes = is_w ? (uint32_t)(W_STAGE + SFW_STAGE) : (uint32_t)(rows_ld * 128 + nrb * 2048);
+        const uint32_t bytes = is_w ? (uint32_t)(W_STAGE + kSfStage) : (uint32_t)(rows_ld * 128 + nrb * kSfStage);
         const uint8_t *sfw_tile = w_sf + (int64_t)(T.w_row0 >> 7) * sf_row_stride;
         const uint8_t *sfx_tile = x_sf + (int64_t)(xr0 >> 7) * sf_row_stride;
         for (int ks = 0; ks < ksteps; ++ks) {
@@ -153,11 +157,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(
           armed_parity[stage] = phase;
           if (is_w) {
             tma_load_2d(sbase + OFF_W + stage * W_STAGE, &tmap_w, ks * 128, T.w_row0, fb, pol);
-            bulk_load(sbase + OFF_SFW + stage * SFW_STAGE, sfw_tile + ks * 2048, 2048, fb);
+            bulk_load(sbase + OFF_SFW + stage * SFW_STAGE, sfw_tile + ks * kSfStage, kSfStage, fb);
           } else {
             for (int rb = 0; rb < nrb; ++rb)
-              bulk_load(sbase + OFF_SFX + stage * SFX_STAGE + rb * 2048, sfx_tile + rb * sf_row_stride + ks * 2048,
-                        2048, fb);
+              bulk_load(sbase + OFF_SFX + stage * SFX_STAGE + rb * 2048, sfx_tile + rb * sf_row_stride + ks * kSfStage,
+                        kSfStage, fb);
             uint32_t dst = sbase + OFF_X + stage * X_STAGE;
             int row = T.x_row0, left = rows_ld;
             if (left >= 128) { tma_load_2d(dst, &tmap_x128, ks * 128, row, fb, pol); dst += 16384; row += 128; left -= 128; }
@@ -199,8 +203,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(
         if (!mbar_wait_warp(bar_xfull + 8 * sx, (kiter / X_STAGES) & 1, abort_flag, dev_status)) { ok = false; break; }
         tc_fence_after();
         const uint32_t tcol = tmem_base + lane_base + TMEM_SF + sb * TMEM_SF_STRIDE;
-        sf_stage_to_tmem(tcol, sbase + OFF_SFW + sw * SFW_STAGE + lane * 16, sbase + OFF_SFX + sx * SFX_STAGE + lane * 16,
-                         nrb);
+        if constexpr (kMx)
+          sf_stage_to_tmem_mx(tcol, sbase + OFF_SFW + sw * SFW_STAGE + lane * 16,
+                              sbase + OFF_SFX + sx * SFX_STAGE + lane * 16, nrb);
+        else
+          sf_stage_to_tmem(tcol, sbase + OFF_SFW + sw * SFW_STAGE + lane * 16, sbase + OFF_SFX + sx * SFX_STAGE + lane * 16,
+                           nrb);
         tc_fence_before();
         mbar_arrive(bar_sf_full + 8 * sb);
       }
@@ -212,7 +220,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(
     for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++titer) {
       const Tile T = decode_tile<kSwiglu>(t, s_off, s_slot, s_tile, E, N, BM, 0);
       const uint32_t n_mma = (T.n_valid + 15) & ~15;
-      const uint32_t idesc = idesc_mxf4nvf4(BM, n_mma);
+      const uint32_t idesc = kMx ? idesc_mxf4_ue8m0(BM, n_mma) : idesc_mxf4nvf4(BM, n_mma);
       const uint32_t xoff = (uint32_t)(T.x_row0 & 127) >> 5;      // 0 or 2 columns
       const uint32_t ab = titer & 1;
       const uint32_t t_acc = tmem_base + ab * TMEM_ACC_STRIDE;
@@ -232,8 +240,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             // +32 bytes of K per MMA: +2 in the descriptor's 16-byte address field
-            tc_mma(t_acc, dw + 2 * kk, dx + 2 * kk, idesc, t_sf + kk * 4, t_sf + 16 + kk * 8 + xoff,
-                   (ks > 0 || kk > 0) ? 1u : 0u);
+            if constexpr (kMx)
+              tc_mma_mx(t_acc, dw + 2 * kk, dx + 2 * kk, idesc, t_sf + kk * 4, t_sf + 16 + kk * 8 + xoff,
+                        (ks > 0 || kk > 0) ? 1u : 0u);
+            else
+              tc_mma(t_acc, dw + 2 * kk, dx + 2 * kk, idesc, t_sf + kk * 4, t_sf + 16 + kk * 8 + xoff,
+                     (ks > 0 || kk > 0) ? 1u : 0u);
           }
           tc_commit(bar_wempty + 8 * sw);
           tc_commit(bar_xempty + 8 * sx);
@@ -262,7 +274,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(
       const uint32_t ab = titer & 1;
       if (!mbar_wait_warp(bar_acc_full + 8 * ab, (titer >> 1) & 1, abort_flag, dev_status)) break;
       tc_fence_after();
-      const float alpha = __fmul_rn(x_gs[T.e], w_gs[T.e]);
+      const float alpha = kMx ? 1.0f : __fmul_rn(x_gs[T.e], w_gs[T.e]);
       epilogue_tile<kSwiglu, kBf16Out, kQuantH>(T, tmem_base + lane_base + ab * TMEM_ACC_STRIDE, alpha, epi, quad,
                                                 lane, N, y, amax_out, bar_acc_empty + 8 * ab, false, hq, dev_status);
     }
@@ -286,7 +298,7 @@ namespace {
 
 int g_sms = 0;
 int g_gemm_kernel = 0;      // 0 automatic (one CTA per tile), 1 one CTA per tile, 2 CTA pairs
-bool g_attr_set[4] = {false, false, false, false};
+bool g_attr_set[6] = {false, false, false, false, false, false};
 
 }  // namespace
 
@@ -390,5 +402,50 @@ extern "C" nvfp4_status nvfp4_grouped_gemm_swiglu_nvfp4(const uint8_t *a_q, cons
   kern<<<g_sms, gemm::NUM_THREADS, gemm::SMEM_BYTES, stream>>>(tw, tx128, tx64, tx32, b_sf, a_sf, b_gs, a_gs,
                                                                expert_offsets, E, (int)M_total, (int)N, (int)K, nullptr,
                                                                nullptr, dev_status, hq);
+  return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
+// MXFP4 x MXFP4 grouped GEMM (kind::mxf4): the same persistent pipeline with
+// UE8M0 scales per 32 elements and no global scales.
+extern "C" nvfp4_status mxfp4_grouped_gemm(const uint8_t *a_q, const uint8_t *a_sf, const uint8_t *b_q,
+                                           const uint8_t *b_sf, const int32_t *expert_offsets, int num_experts,
+                                           int64_t M_total, int64_t N, int64_t K, void *y,
+                                           nvfp4_out_dtype out_dtype, void *workspace, int32_t *dev_status,
+                                           cudaStream_t stream) {
+  (void)workspace;
+  if (out_dtype != NVFP4_OUT_F32 && out_dtype != NVFP4_OUT_BF16) return NVFP4_ERR_INVALID_ARG;
+  const int E = expert_offsets ? num_experts : 1;
+  if (E < 1 || E > gemm::kMaxExperts) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (M_total < 0 || N <= 0 || K <= 0) return NVFP4_ERR_INVALID_ARG;
+  if (N % 128 != 0 || K % 256 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if ((int64_t)E * N > ((int64_t)1 << 31) - 1 || M_total > ((int64_t)1 << 30)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (M_total == 0) return NVFP4_OK;
+  if (!a_q || !a_sf || !b_q || !b_sf || !y) return NVFP4_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(a_q) | reinterpret_cast<uintptr_t>(b_q) | reinterpret_cast<uintptr_t>(a_sf) |
+       reinterpret_cast<uintptr_t>(b_sf) | reinterpret_cast<uintptr_t>(y)) & 15u)
+    return NVFP4_ERR_INVALID_ARG;
+  const int64_t x_rows = nvfp4_padded_rows_bound(M_total, E);
+  CUtensorMap tw, tx128, tx64, tx32;
+  if (!gemm::make_map(&tw, b_q, (uint64_t)E * N, (uint64_t)K / 2, 128)) return NVFP4_ERR_CUDA;
+  if (!gemm::make_map(&tx128, a_q, (uint64_t)x_rows, (uint64_t)K / 2, 128)) return NVFP4_ERR_CUDA;
+  if (!gemm::make_map(&tx64, a_q, (uint64_t)x_rows, (uint64_t)K / 2, 64)) return NVFP4_ERR_CUDA;
+  if (!gemm::make_map(&tx32, a_q, (uint64_t)x_rows, (uint64_t)K / 2, 32)) return NVFP4_ERR_CUDA;
+  if (g_sms == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&g_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (g_sms <= 0) g_sms = 148;
+  }
+  const int variant = out_dtype == NVFP4_OUT_BF16 ? 5 : 4;
+  auto kern = variant == 5 ? gemm::grouped_gemm_kernel<false, true, false, true>
+                           : gemm::grouped_gemm_kernel<false, false, false, true>;
+  if (!g_attr_set[variant]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::SMEM_BYTES) != cudaSuccess)
+      return NVFP4_ERR_CUDA;
+    g_attr_set[variant] = true;
+  }
+  kern<<<g_sms, gemm::NUM_THREADS, gemm::SMEM_BYTES, stream>>>(tw, tx128, tx64, tx32, b_sf, a_sf, nullptr, nullptr,
+                                                               expert_offsets, E, (int)M_total, (int)N, (int)K, y,
+                                                               nullptr, dev_status, gemm::HQuantOut{});
   return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }

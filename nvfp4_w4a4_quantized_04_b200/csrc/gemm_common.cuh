@@ -159,6 +159,17 @@ __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_
       : "memory");
 }
 
+// MXFP4 x MXFP4: UE8M0 scales, two per row per MMA (K = 64 in 32-element blocks),
+// read from bytes 0 and 1 of the row's tensor-memory word (scale id 0).
+__device__ __forceinline__ void tc_mma_mx(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
+      "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.scale_vec::2X [%0], %1, %2, %3, [%5], [%6], p;\n}"
+      :: "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
 __device__ __forceinline__ void tc_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
                :: "r"(bar) : "memory");
@@ -179,6 +190,11 @@ __device__ __forceinline__ void tc_ld32_nowait(uint32_t taddr, uint32_t *r) {
 // UE4M3 scales, M = m (128, or 256 for a CTA pair), N = n (multiple of 16).
 __device__ __forceinline__ uint32_t idesc_mxf4nvf4(uint32_t m, uint32_t n) {
   return (1u << 7) | (1u << 10) | ((n >> 3) << 17) | ((m >> 4) << 24);
+}
+
+// Same fields with the scale type set to UE8M0 (bit 23), for kind::mxf4.
+__device__ __forceinline__ uint32_t idesc_mxf4_ue8m0(uint32_t m, uint32_t n) {
+  return idesc_mxf4nvf4(m, n) | (1u << 23);
 }
 
 __device__ __forceinline__ void tc_st_x4(uint32_t taddr, uint4 v) {
@@ -400,6 +416,40 @@ __device__ __forceinline__ void sf_stage_to_tmem(uint32_t tcol, uint32_t sfw_add
   if (nrb > 1) {
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk) tc_st_x4(tcol + 16 + kk * 8 + 4, lds128(sfx_addr + 2048 + kk * 512));
+  }
+  tc_wait_st();
+}
+
+// MXFP4 form of the same: a 512-byte atom now holds 4 UE8M0 scales per row =
+// 128 elements = two MMAs, so one K stage has two atoms per row block.  Each
+// MMA gets its own 4 columns (the NVFP4 column map) with its two scales in
+// bytes 0 and 1 of the row's word: the low half-word of the atom word for the
+// first MMA of the pair, the high half-word for the second.
+__device__ __forceinline__ uint4 lo16x4(uint4 v) {
+  return make_uint4(v.x & 0xFFFFu, v.y & 0xFFFFu, v.z & 0xFFFFu, v.w & 0xFFFFu);
+}
+__device__ __forceinline__ uint4 hi16x4(uint4 v) { return make_uint4(v.x >> 16, v.y >> 16, v.z >> 16, v.w >> 16); }
+
+__device__ __forceinline__ void sf_stage_to_tmem_mx(uint32_t tcol, uint32_t sfw_addr, uint32_t sfx_addr, int nrb) {
+#pragma unroll
+  for (int a = 0; a < 2; ++a) {
+    const uint4 w = lds128(sfw_addr + a * 512);
+    tc_st_x4(tcol + (2 * a) * 4, lo16x4(w));
+    tc_st_x4(tcol + (2 * a + 1) * 4, hi16x4(w));
+  }
+#pragma unroll
+  for (int a = 0; a < 2; ++a) {
+    const uint4 x = lds128(sfx_addr + a * 512);
+    tc_st_x4(tcol + 16 + (2 * a) * 8, lo16x4(x));
+    tc_st_x4(tcol + 16 + (2 * a + 1) * 8, hi16x4(x));
+  }
+  if (nrb > 1) {
+#pragma unroll
+    for (int a = 0; a < 2; ++a) {
+      const uint4 x = lds128(sfx_addr + 2048 + a * 512);
+      tc_st_x4(tcol + 16 + (2 * a) * 8 + 4, lo16x4(x));
+      tc_st_x4(tcol + 16 + (2 * a + 1) * 8 + 4, hi16x4(x));
+    }
   }
   tc_wait_st();
 }

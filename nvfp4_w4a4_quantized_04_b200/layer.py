@@ -14,7 +14,7 @@ from typing import Optional
 import torch
 
 from . import (EPI_NONE, EPI_SWIGLU, GS_AMAX_GIVEN, GS_FROM_AMAX, GS_GIVEN, OUT_BF16, OUT_F32, SF_MMA_TILED, SF_ROWMAJOR,
-               mxfp4_to_nvfp4, nvfp4_dequantize, nvfp4_grouped_gemm, nvfp4_grouped_gemm_swiglu_nvfp4,
+               mxfp4_grouped_gemm as _mxfp4_grouped_gemm, mxfp4_quantize as _mxfp4_quantize, mxfp4_to_nvfp4, nvfp4_dequantize, nvfp4_grouped_gemm, nvfp4_grouped_gemm_swiglu_nvfp4,
                nvfp4_grouped_gemm_w4a16, nvfp4_moe_combine,
                nvfp4_moe_route,
                nvfp4_moe_quantize, nvfp4_moe_route_workspace_size, nvfp4_padded_rows_bound, nvfp4_quantize,
@@ -115,6 +115,33 @@ def remap_mxfp4(q_mx: torch.Tensor, e8: torch.Tensor, n_tensors: int, rows: int,
     ws = ws if ws is not None else workspace(n_tensors, q_mx.device)
     mxfp4_to_nvfp4(q_mx, e8, n_tensors, rows, K, q_nv, sf, layout, gs, ws, dev_status)
     return Packed(q_nv, sf, gs, n_tensors * rows, K, layout, None, n_tensors)
+
+
+def mxfp4_quantize(x: torch.Tensor, layout=SF_ROWMAJOR, dev_status=None):
+    """MXFP4 encode of bf16 rows [rows, K]: (codes uint8 [rows, K/2], UE8M0
+    scales, one per 32 elements, in `layout`)."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    rows, K = x.shape
+    q = torch.empty((rows, K // 2), dtype=torch.uint8, device=x.device)
+    if layout == SF_MMA_TILED:
+        e8 = torch.empty(((rows + 127) // 128 * 128) * (K // 32), dtype=torch.uint8, device=x.device)
+    else:
+        e8 = torch.empty((rows, K // 32), dtype=torch.uint8, device=x.device)
+    _mxfp4_quantize(x, rows, K, x.stride(0), q, e8, layout, dev_status)
+    return q, e8
+
+
+def mx_grouped_gemm(a_q: torch.Tensor, a_sf: torch.Tensor, w_q: torch.Tensor, w_sf: torch.Tensor, N: int, K: int,
+                    rows: int, offsets: Optional[torch.Tensor] = None, num_experts: int = 1, out_dtype=OUT_BF16,
+                    y=None, dev_status=None) -> torch.Tensor:
+    """MXFP4 x MXFP4 grouped GEMM: Y [rows, N] = per expert A_e W_e^T
+    (activations in 128-aligned expert slots, tensor-core scale layout)."""
+    dt = torch.float32 if out_dtype == OUT_F32 else torch.bfloat16
+    if y is None:
+        y = torch.empty((rows, N), dtype=dt, device=a_q.device)
+    E = num_experts if offsets is not None else 1
+    _mxfp4_grouped_gemm(a_q, a_sf, w_q, w_sf, offsets, E, rows, N, K, y, out_dtype, None, dev_status)
+    return y
 
 
 def grouped_gemm(a: Packed, w: Packed, N: int, out_dtype=OUT_BF16, y=None, dev_status=None) -> torch.Tensor:

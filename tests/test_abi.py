@@ -93,6 +93,13 @@ def test_host_validation_without_device(lib):
     assert L.nvfp4_moe_quantize(fake, 4, 64, 64, fake, 0, fake, 2, 0, fake, fake, fake, 1, fake, None, None) == nv.ERR_INVALID_ARG
     assert L.nvfp4_moe_quantize(fake, 4, 64, 64, fake, 2, None, 2, 0, fake, fake, fake, 1, fake, None, None) == nv.ERR_INVALID_ARG
     assert L.nvfp4_moe_quantize(fake, 4, 48, 48, fake, 2, fake, 2, 0, fake, fake, fake, 1, fake, None, None) == nv.ERR_UNSUPPORTED_SHAPE
+    # MXFP4 encode: K % 32, K % 128 for tiled scales, aligned pointers, rows == 0 a no-op
+    assert L.mxfp4_quantize(fake, 4, 48, 48, fake, fake, 0, None, None) == nv.ERR_UNSUPPORTED_SHAPE
+    assert L.mxfp4_quantize(fake, 4, 64, 64, fake, fake, 1, None, None) == nv.ERR_UNSUPPORTED_SHAPE
+    assert L.mxfp4_quantize(fake, 4, 64, 60, fake, fake, 0, None, None) == nv.ERR_INVALID_ARG
+    assert L.mxfp4_quantize(P((1 << 20) + 2), 4, 64, 64, fake, fake, 0, None, None) == nv.ERR_INVALID_ARG
+    assert L.mxfp4_quantize(fake, 4, 64, 64, fake, fake, 2, None, None) == nv.ERR_INVALID_ARG
+    assert L.mxfp4_quantize(None, 0, 64, 64, None, None, 0, None, None) == nv.OK
 
 
 def test_product_path_has_no_oracle_or_cpu_fallback():

@@ -337,6 +337,194 @@ def test_remap_bitexact(layout):
         assert np.array_equal(dq, oracle.dequantize_mxfp4_f64(q[sl], e[sl]))
 
 
+# --------------------------------------------------------------------------- MXFP4 encode
+def _mx_input(seed, rows, K, ld=None):
+    """Gaussian rows, each 32-block scaled by its own power of two over the
+    bf16 range (subnormal amax to ~2^120), plus hand-placed edge blocks."""
+    ld = ld or K
+    lp = (ld + 31) // 32 * 32
+    z = synthetic.bf16_bits_to_f32(synthetic.gaussian_bf16(seed, 1, (rows, lp))).astype(np.float64)
+    mag = np.ldexp(1.0, (synthetic.words(seed, 2, 0, rows * lp // 32) % 250).astype(np.int64) - 130)
+    x = synthetic.f32_to_bf16_bits((z * np.repeat(mag, 32).reshape(rows, lp)).astype(np.float32))
+    x = np.ascontiguousarray(x[:, :ld])
+    x[0, :32] = 0                                             # all-zero block
+    x[0, 32:64] = 0x8000                                      # all -0 block
+    x[1, :32] = synthetic.f32_to_bf16_bits(np.float32([1e30] + [-1e-30] * 31))   # products underflow to -0
+    x[1, 32:64] = synthetic.f32_to_bf16_bits(np.float32([4.0, 5.0, 2.5, -1.75, 0.25] + [0.0] * 27))  # ties
+    x[2, :32] = np.arange(1, 33, dtype=np.uint16)             # subnormal-only block
+    return x
+
+
+@pytest.mark.parametrize("rows, K, ld, layout", [(300, 1024, 1024, 0), (300, 1024, 1024, 1),
+                                                  (7, 96, 104, 0), (129, 384, 400, 1)])
+def test_mxfp4_quantize_bitexact(rows, K, ld, layout):
+    L = layer()
+    xw = _mx_input(31, rows, K, ld)
+    q_ref, e_ref, st = oracle.quantize_mxfp4(np.ascontiguousarray(xw[:, :K]))
+    assert st == 0
+    s = status_word()
+    xd = bf16_dev(xw)[:, :K]
+    q, e = L.mxfp4_quantize(xd, layout=layout, dev_status=s)
+    torch.cuda.synchronize()
+    assert int(s.item()) == 0
+    assert np.array_equal(to_np(q), q_ref)
+    e = to_np(e)
+    e = untile(e, (rows + 127) // 128 * 128, K // 32)[:rows] if layout == 1 else e
+    assert np.array_equal(e, e_ref)
+
+
+def test_mxfp4_quantize_nonfinite_blocks():
+    L = layer()
+    rows, K = 64, 256
+    x = _mx_input(32, rows, K)
+    x[3, 40] = 0x7F80                                        # +inf
+    x[9, 200] = 0xFFC1                                       # NaN
+    q_ref, e_ref, st = oracle.quantize_mxfp4(x)
+    assert st == oracle.ERR_NONFINITE
+    s = status_word()
+    q, e = L.mxfp4_quantize(bf16_dev(x), dev_status=s)
+    torch.cuda.synchronize()
+    assert int(s.item()) == oracle.ERR_NONFINITE
+    assert np.array_equal(to_np(q), q_ref) and np.array_equal(to_np(e), e_ref)
+    assert to_np(e)[3, 1] == 0xFF and to_np(e)[9, 6] == 0xFF
+
+
+def test_mxfp4_quantize_then_remap_lossless_on_device():
+    """Both device kernels in a row: MXFP4 encode, then the NVFP4 remap, which
+    must dequantize to the oracle's MXFP4 values exactly."""
+    L = layer()
+    rows, K = 256, 512
+    x = synthetic.gaussian_bf16(33, 1, (rows, K))
+    q_ref, e_ref, _ = oracle.quantize_mxfp4(x)
+    q, e = L.mxfp4_quantize(bf16_dev(x))
+    s = status_word()
+    p = L.remap_mxfp4(q, e, 1, rows, K, layout=0, dev_status=s)
+    torch.cuda.synchronize()
+    assert int(s.item()) == 0
+    got = oracle.dequantize_f64(to_np(p.q), to_np(p.sf).reshape(rows, K // 16), np.full(rows, to_np(p.gs)[0], np.float32))
+    assert np.array_equal(got, oracle.dequantize_mxfp4_f64(q_ref, e_ref))
+
+
+def test_mxfp4_quantize_full_size_sampled_rows():
+    """The bench's workload (65,536 x 4,096 bf16, 2^28 elements, tiled scales):
+    sampled rows against the oracle."""
+    import synthetic.cuda as sc
+    L = layer()
+    rows, K = 65536, 4096
+    xd = sc.gaussian_bf16(34, 1, (rows, K))
+    q, e = L.mxfp4_quantize(xd, layout=1)
+    torch.cuda.synchronize()
+    pick = np.array([0, 1, 127, 128, 4097, 33333, rows - 129, rows - 1])
+    xs = to_np(xd[torch.from_numpy(pick).cuda()])
+    q_ref, e_ref, _ = oracle.quantize_mxfp4(xs)
+    assert np.array_equal(to_np(q)[pick], q_ref)
+    e_rm = untile(to_np(e), rows, K // 32)
+    assert np.array_equal(e_rm[pick], e_ref)
+
+
+def _run_mx_gemm(x_bits, w_bits, offsets, E, N, K, out_dtype):
+    """MXFP4 GEMM on oracle-encoded operands; returns (y, y_ref, s_ref)."""
+    L = layer()
+    nv = nvmod()
+    R = x_bits.shape[0]
+    qa, ea, st = oracle.quantize_mxfp4(x_bits)
+    qw, ew, st2 = oracle.quantize_mxfp4(w_bits)
+    assert st == 0 and st2 == 0
+    bound = nv.nvfp4_padded_rows_bound(R, E)
+    qs = np.zeros((bound, K // 2), np.uint8)
+    es = np.zeros((bound, K // 32), np.uint8)
+    if offsets is not None:
+        rows, _ = slot_rows(offsets)
+    else:
+        rows = np.arange(R)
+    qs[rows] = qa
+    es[rows] = ea
+    s = status_word()
+    y = L.mx_grouped_gemm(to_dev(qs), to_dev(tile(es)), to_dev(qw), to_dev(tile(ew)), N, K, R,
+                          to_dev(offsets) if offsets is not None else None, E, out_dtype, dev_status=s)
+    torch.cuda.synchronize()
+    assert int(s.item()) == 0
+    a = oracle.dequantize_mxfp4_f64(qa, ea)
+    b = oracle.dequantize_mxfp4_f64(qw, ew)
+    if offsets is None:
+        y_ref, s_ref = oracle.gemm_f64(a, b)
+    else:
+        y_ref, s_ref = oracle.grouped_gemm_f64(a, b.reshape(E, N, K), offsets)
+    return to_np(y), y_ref, s_ref
+
+
+def test_mx_gemm_closed_form_integer_case():
+    """All UE8M0 scales 1: every product is a multiple of 1/4 and the fp32 sum
+    is exact, so the kind::mxf4 result must equal the oracle exactly."""
+    L = layer()
+    rng = np.random.default_rng(1)
+    M, N, K = 128, 256, 512
+    qa = rng.integers(0, 256, (M, K // 2), dtype=np.uint8)
+    qw = rng.integers(0, 256, (N, K // 2), dtype=np.uint8)
+    ea = np.full((M, K // 32), 127, np.uint8)
+    ew = np.full((N, K // 32), 127, np.uint8)
+    ea[5, 3] = 129                                   # a few non-unit scales (still exact sums)
+    ew[7, 0] = 125
+    s = status_word()
+    y = L.mx_grouped_gemm(to_dev(qa), to_dev(tile(ea)), to_dev(qw), to_dev(tile(ew)), N, K, M, out_dtype=0,
+                          dev_status=s)
+    torch.cuda.synchronize()
+    assert int(s.item()) == 0
+    y_ref, _ = oracle.gemm_f64(oracle.dequantize_mxfp4_f64(qa, ea), oracle.dequantize_mxfp4_f64(qw, ew))
+    assert np.array_equal(to_np(y).astype(np.float64), y_ref)
+
+
+@pytest.mark.parametrize("out_dtype", [0, 1])
+def test_mx_gemm_dense_many_tiles(out_dtype):
+    M, N, K = 1000, 384, 1024
+    x = synthetic.gaussian_bf16(41, synthetic.STREAMS["x"], (M, K), outlier_frac=0.001)
+    w = synthetic.gaussian_bf16(41, synthetic.STREAMS["w"], (N, K), sigma=0.02)
+    y, y_ref, s_ref = _run_mx_gemm(x, w, None, 1, N, K, 0)
+    ok, err, bound = gemm_tol(y, y_ref, s_ref)
+    assert ok.all(), (err.max(), (err / bound).max())
+    if out_dtype == 1:
+        y16, _, _ = _run_mx_gemm(x, w, None, 1, N, K, 1)
+        assert np.array_equal(y16, synthetic.f32_to_bf16_bits(y))
+
+
+def test_mx_gemm_grouped_chunk_edges():
+    counts = [1, 63, 64, 65, 127, 128, 129, 191, 192, 193, 257, 385, 0, 2, 17, 33]
+    E, N, K = len(counts), 256, 512
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    R = int(offsets[-1])
+    x = synthetic.gaussian_bf16(42, synthetic.STREAMS["x"], (R, K), outlier_frac=0.001)
+    w = synthetic.gaussian_bf16(42, synthetic.STREAMS["w"], (E * N, K), sigma=0.02)
+    y, y_ref, s_ref = _run_mx_gemm(x, w, offsets, E, N, K, 0)
+    ok, err, bound = gemm_tol(y, y_ref, s_ref)
+    assert ok.all(), (err.max(), (err / bound).max(), np.argwhere(~ok)[:5])
+
+
+def test_mx_gemm_matches_remapped_nvfp4_gemm():
+    """The two routes for MXFP4 weights: the direct kind::mxf4 GEMM, and the
+    lossless NVFP4 remap followed by the NVFP4 GEMM.  Both multiply the same
+    values, so both sit within the fp32 accumulation bound of one fp64 result."""
+    L = layer()
+    M, N, K = 256, 256, 1024
+    x = synthetic.gaussian_bf16(43, synthetic.STREAMS["x"], (M, K))
+    w = synthetic.gaussian_bf16(43, synthetic.STREAMS["w"], (N, K), sigma=0.02)
+    y_mx, y_ref, s_ref = _run_mx_gemm(x, w, None, 1, N, K, 0)
+    qa, ea, _ = oracle.quantize_mxfp4(x)
+    qw, ew, _ = oracle.quantize_mxfp4(w)
+    pa = L.remap_mxfp4(to_dev(qa), to_dev(ea), 1, M, K, layout=1)
+    pw = L.remap_mxfp4(to_dev(qw), to_dev(ew), 1, N, K, layout=1)
+    # the GEMM's token operand spans nvfp4_padded_rows_bound rows: pad the remapped copy
+    bound = nvmod().nvfp4_padded_rows_bound(M, 1)
+    qpad = torch.zeros((bound, K // 2), dtype=torch.uint8, device="cuda")
+    qpad[:M] = pa.q
+    spad = torch.zeros(bound * (K // 16), dtype=torch.uint8, device="cuda")
+    spad[:pa.sf.numel()] = pa.sf
+    a_nv = L.Packed(qpad, spad, pa.gs, M, K, 1, None, 1)
+    y_nv = to_np(L.grouped_gemm(a_nv, pw, N, 0))
+    for y in (y_mx, y_nv):
+        ok, err, bound = gemm_tol(y, y_ref, s_ref)
+        assert ok.all(), (err.max(), (err / bound).max())
+
+
 def test_remap_errors_and_inplace():
     L = layer()
     rows, K = 128, 64
