@@ -435,67 +435,120 @@ __global__ void __launch_bounds__(256) moe_amax_kernel(
   }
 }
 
-// Pass 2: a warp per token, 4 blocks in flight per lane, held as fp32 pairs
-// across the token's k encodes.
+// Per-group constants of the dispatch encode, computed once per call with the
+// same IEEE operations the per-block path would use: rtab[g][S] = 1/(S*s_g)
+// (0 when that product is 0) for every E4M3 byte S < 128, and
+// ytab[g] = RN(1/(6*s_g)).
+__global__ void encode_tables_kernel(const float *__restrict__ gs, float *__restrict__ rtab,
+                                     float *__restrict__ ytab) {
+  const int g = blockIdx.x;
+  const uint32_t S = threadIdx.x;
+  const float s_g = gs[g];
+  const float e = __fmul_rn(e4m3_to_f32_hw(S), s_g);
+  rtab[g * 128 + S] = (e == 0.0f) ? 0.0f : __frcp_rn(e);
+  if (S == 0) ytab[g] = __frcp_rn(__fmul_rn(6.0f, s_g));
+}
+
+// S = e4m3_rne_satfinite(RN(a_b / t_g)) without the division in the common
+// case.  q = RN(a_b * y) with y = RN(1/t_g) is within 3 * 2^-24 (relative) of
+// the exact quotient, and so is RN(a_b / t_g); the bracket [q(1-2^-21),
+// q(1+2^-21)], each end rounded, holds RN(a_b / t_g) (below the fp32 normal
+// range both ends and the quotient encode to 0).  E4M3 rounding is monotone, so
+// when both ends give the same byte that byte is the IEEE path's S; otherwise
+// (a quotient within 2^-21 of an E4M3 rounding boundary, or y = inf) the
+// division is done.
+__device__ __forceinline__ uint32_t block_scale_fast(float a_b, float t_g, float y, bool exact) {
+  const float q = __fmul_rn(a_b, y);
+  const uint32_t lo = f32_to_e4m3_satfinite(__fmul_rn(q, 0.99999952316284180f));   // 1 - 2^-21
+  const uint32_t hi = f32_to_e4m3_satfinite(__fmul_rn(q, 1.00000047683715820f));   // 1 + 2^-21
+  if (lo == hi && !exact) return lo;
+  return f32_to_e4m3_satfinite(__fdiv_rn(a_b, t_g));
+}
+
+// Codes of a block in fp32 pairs for a given r (a NaN product 0 * inf encodes as +0).
+__device__ __forceinline__ uint2 encode_codes(const uint64_t (&xf)[8], float r) {
+  const uint64_t rr = ((uint64_t)__float_as_uint(r) << 32) | __float_as_uint(r);
+  uint64_t prod[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) prod[i] = mul_f32x2(xf[i], rr);
+  if (isinf(r)) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) prod[i] = sanitize_pair(prod[i]);
+  }
+  return make_uint2(e2m1x8_from_pairs(prod[0], prod[1], prod[2], prod[3]),
+                    e2m1x8_from_pairs(prod[4], prod[5], prod[6], prod[7]));
+}
+
+// Pass 2: a warp takes 64 consecutive 16-element blocks of one token row (two
+// per lane, so the token's routing is warp-uniform), holds them as fp32 pairs
+// and encodes them once per routed copy, with the scale byte from
+// block_scale_fast and r from the group's table.  The block loads are issued
+// before the routing lookups so the two latencies overlap.
 template <bool kTiled>
-__global__ void __launch_bounds__(256, 2) moe_encode_kernel(
+__global__ void __launch_bounds__(256, 3) moe_encode_blocks_kernel(
     const uint16_t *__restrict__ x, int64_t ld_x, int64_t K64, int64_t tokens, const int32_t *__restrict__ slot,
     int topk, const int32_t *__restrict__ group_offsets, int G, const float *__restrict__ gs,
-    uint8_t *__restrict__ q, uint8_t *__restrict__ sf, int32_t *dev_status) {
+    const float *__restrict__ rtab, const float *__restrict__ ytab, uint8_t *__restrict__ q,
+    uint8_t *__restrict__ sf, int32_t *dev_status) {
   extern __shared__ int32_t smem[];
   int32_t *off = smem, *pslot = smem + (G + 1), *scratch = smem + 2 * (G + 1);
   load_groups(group_offsets, G, off, pslot, scratch);
   const int lane = threadIdx.x & 31;
   const uint32_t K = (uint32_t)K64, nblk = K >> 4;
-  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  const uint32_t cpr = (nblk + 63) >> 6;                     // 64-block chunks per row
+  const uint64_t nwork = (uint64_t)tokens * cpr;
+  const uint64_t nwarps = ((uint64_t)gridDim.x * blockDim.x) >> 5;
   const bool v8 = ((reinterpret_cast<uintptr_t>(x) & 31u) == 0) && ((ld_x & 15) == 0);
   bool bad = false;
-  constexpr int B = 4;
-  for (int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < tokens; t += nwarps) {
-    int32_t my_p = -1;
-    float my_sg = 1.0f;
+  for (uint64_t w = ((uint64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; w < nwork; w += nwarps) {
+    const uint64_t t = w / cpr;
+    const uint32_t j0 = (uint32_t)(w - t * cpr) * 64 + lane, j1 = j0 + 32;
+    const uint16_t *xr = x + t * ld_x;
+    uint4 a0 = make_uint4(0, 0, 0, 0), b0 = a0, a1 = a0, b1 = a0;
+    if (j0 < nblk) load_block(xr + (uint64_t)j0 * 16, v8, a0, b0);
+    if (j1 < nblk) load_block(xr + (uint64_t)j1 * 16, v8, a1, b1);
+    int32_t my_p = -1, my_e = 0;
+    float my_sg = 1.0f, my_y = 0.0f;
     if (lane < topk) {
       const int32_t r = slot[t * topk + lane];
       if (r >= 0 && r < off[G]) {
         const int e = upper_group(off, G, r);
         my_p = pslot[e] + (r - off[e]);
+        my_e = e;
         my_sg = gs[e];
+        my_y = ytab[e];
       }
     }
-    const uint16_t *xr = x + t * ld_x;
-    for (uint32_t j0 = 0; j0 < nblk; j0 += 32 * B) {
-      uint64_t xf[B][8];
-      float amf[B];
-#pragma unroll
-      for (int k = 0; k < B; ++k) {
-        const uint32_t j = j0 + k * 32 + lane;
-        uint4 va = make_uint4(0, 0, 0, 0), vb = make_uint4(0, 0, 0, 0);
-        if (j < nblk) load_block(xr + (uint64_t)j * 16, v8, va, vb);
-        const uint32_t m = block_amax_bits(va, vb);
-        if (m >= 0x7F80u) bad = true;
-        amf[k] = __uint_as_float(m << 16);
-        xf[k][0] = bf16x2_to_f32x2(va.x); xf[k][1] = bf16x2_to_f32x2(va.y);
-        xf[k][2] = bf16x2_to_f32x2(va.z); xf[k][3] = bf16x2_to_f32x2(va.w);
-        xf[k][4] = bf16x2_to_f32x2(vb.x); xf[k][5] = bf16x2_to_f32x2(vb.y);
-        xf[k][6] = bf16x2_to_f32x2(vb.z); xf[k][7] = bf16x2_to_f32x2(vb.w);
+    const uint32_t m0 = block_amax_bits(a0, b0), m1 = block_amax_bits(a1, b1);
+    if (max(m0, m1) >= 0x7F80u) bad = true;
+    const float am0 = __uint_as_float(m0 << 16), am1 = __uint_as_float(m1 << 16);
+    const uint64_t x0[8] = {bf16x2_to_f32x2(a0.x), bf16x2_to_f32x2(a0.y), bf16x2_to_f32x2(a0.z),
+                            bf16x2_to_f32x2(a0.w), bf16x2_to_f32x2(b0.x), bf16x2_to_f32x2(b0.y),
+                            bf16x2_to_f32x2(b0.z), bf16x2_to_f32x2(b0.w)};
+    const uint64_t x1[8] = {bf16x2_to_f32x2(a1.x), bf16x2_to_f32x2(a1.y), bf16x2_to_f32x2(a1.z),
+                            bf16x2_to_f32x2(a1.w), bf16x2_to_f32x2(b1.x), bf16x2_to_f32x2(b1.y),
+                            bf16x2_to_f32x2(b1.z), bf16x2_to_f32x2(b1.w)};
+    const uint32_t jb0 = kTiled ? sf_blk_part(j0) : j0, jb1 = kTiled ? sf_blk_part(j1) : j1;
+    for (int c = 0; c < topk; ++c) {
+      const int32_t p = __shfl_sync(0xffffffffu, my_p, c);
+      if (p < 0) continue;
+      const int32_t e = __shfl_sync(0xffffffffu, my_e, c);
+      const float s_g = __shfl_sync(0xffffffffu, my_sg, c);
+      const float y = __shfl_sync(0xffffffffu, my_y, c);
+      const float t_g = __fmul_rn(6.0f, s_g);
+      const bool exact = !(y <= 3.402823466e38f);             // y = inf (or NaN): always divide
+      const float *rt = rtab + (int64_t)e * 128;
+      uint8_t *qr = q + (uint64_t)p * (K >> 1);
+      const uint64_t rsf = kTiled ? sf_row_part((uint32_t)p, nblk) : (uint64_t)p * nblk;
+      if (j0 < nblk) {
+        const uint32_t S = block_scale_fast(am0, t_g, y, exact);
+        *reinterpret_cast<uint2 *>(qr + (uint64_t)j0 * 8) = encode_codes(x0, __ldg(rt + S));
+        sf[rsf + jb0] = (uint8_t)S;
       }
-      for (int c = 0; c < topk; ++c) {
-        const int32_t p = __shfl_sync(0xffffffffu, my_p, c);
-        const float s_g = __shfl_sync(0xffffffffu, my_sg, c);
-        if (p < 0) continue;
-        const float t_g = __fmul_rn(6.0f, s_g);
-        uint8_t *qr = q + (uint64_t)p * (K >> 1);
-        const uint64_t rsf = kTiled ? sf_row_part((uint32_t)p, nblk) : (uint64_t)p * nblk;
-#pragma unroll
-        for (int k = 0; k < B; ++k) {
-          const uint32_t j = j0 + k * 32 + lane;
-          if (j < nblk) {
-            uint32_t S;
-            const uint2 codes = encode_f32x16(xf[k], amf[k], s_g, t_g, S);
-            *reinterpret_cast<uint2 *>(qr + (uint64_t)j * 8) = codes;
-            sf[rsf + (kTiled ? sf_blk_part(j) : j)] = (uint8_t)S;
-          }
-        }
+      if (j1 < nblk) {
+        const uint32_t S = block_scale_fast(am1, t_g, y, exact);
+        *reinterpret_cast<uint2 *>(qr + (uint64_t)j1 * 8) = encode_codes(x1, __ldg(rt + S));
+        sf[rsf + jb1] = (uint8_t)S;
       }
     }
   }
@@ -647,6 +700,16 @@ using namespace nvfp4;
 
 namespace {
 
+// Workspace: amax / exponent-range words (2 per group) and room for kernel
+// bookkeeping, then the per-group encode tables of the dispatch quantize
+// (128 reciprocals + 1 per group).
+size_t workspace_words_bytes(int num_groups) {
+  return (sizeof(uint32_t) * 2 * (size_t)num_groups + 256 + 255) / 256 * 256;
+}
+float *workspace_tables(void *workspace, int num_groups) {
+  return reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(workspace) + workspace_words_bytes(num_groups));
+}
+
 int g_num_sms = 0;
 
 int num_sms() {
@@ -780,8 +843,7 @@ const char *nvfp4_status_string(int status) {
 
 size_t nvfp4_workspace_size(int num_groups) {
   if (num_groups < 1) num_groups = 1;
-  // amax / exponent-range words (2 per group) plus room for kernel bookkeeping
-  size_t bytes = sizeof(uint32_t) * 2 * (size_t)num_groups + 256;
+  size_t bytes = workspace_words_bytes(num_groups) + sizeof(float) * 129 * (size_t)num_groups;
   return (bytes + 255) / 256 * 256;
 }
 
@@ -846,14 +908,18 @@ nvfp4_status nvfp4_moe_quantize(const void *x, int64_t tokens, int64_t K, int64_
   if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_CUDA;
   if (tokens == 0) return NVFP4_OK;
   const size_t sm = sizeof(int32_t) * (2 * (G + 1) + 8);
+  float *rtab = workspace_tables(workspace, G), *ytab = rtab + (size_t)G * 128;
+  encode_tables_kernel<<<G, 128, 0, stream>>>(global_scale, rtab, ytab);
+  if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_CUDA;
+  const int64_t work = tokens * ((K / 16 + 63) / 64) * 32;       // one warp per 64 blocks of a row
   if (sf_layout == NVFP4_SF_MMA_TILED) {
-    const unsigned grid = (unsigned)grid_resident(moe_encode_kernel<true>, tokens * 32, 256, sm);
-    moe_encode_kernel<true><<<grid, 256, sm, stream>>>(xb, ld_x, K, tokens, slot, topk, group_offsets, G,
-                                                       global_scale, q, sf, dev_status);
+    const unsigned grid = (unsigned)grid_resident(moe_encode_blocks_kernel<true>, work, 256, sm);
+    moe_encode_blocks_kernel<true><<<grid, 256, sm, stream>>>(xb, ld_x, K, tokens, slot, topk, group_offsets, G,
+                                                              global_scale, rtab, ytab, q, sf, dev_status);
   } else {
-    const unsigned grid = (unsigned)grid_resident(moe_encode_kernel<false>, tokens * 32, 256, sm);
-    moe_encode_kernel<false><<<grid, 256, sm, stream>>>(xb, ld_x, K, tokens, slot, topk, group_offsets, G,
-                                                        global_scale, q, sf, dev_status);
+    const unsigned grid = (unsigned)grid_resident(moe_encode_blocks_kernel<false>, work, 256, sm);
+    moe_encode_blocks_kernel<false><<<grid, 256, sm, stream>>>(xb, ld_x, K, tokens, slot, topk, group_offsets, G,
+                                                               global_scale, rtab, ytab, q, sf, dev_status);
   }
   return launch_status();
 }
