@@ -322,7 +322,9 @@ def run_headline(args, rank, world, device):
         "breakdown": breakdown,
         "e2e": {"value": round(whole_job_rate(flops, world, 1, e2e_ms) / 1e12, 3), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": round(e2e_ms, 3)},
-        "gpu_launches": (7 if fused else 8) * args.steps,
+        # per step: dispatch (amax, finalize, tables, encode), gate_up, then either
+        # requantize (finalize, encode) or SwiGLU + quantize (amax, finalize, encode), down
+        "gpu_launches": (8 if fused else 9) * args.steps,
         "clocks": clk,
     }
 

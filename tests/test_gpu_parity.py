@@ -147,6 +147,36 @@ def test_moe_quantize_strided_rows():
     _moe_quantize_check(np.ascontiguousarray(xw[:, :H]), r["slot"], r["offsets"], E, 0, x_dev=xd)
 
 
+def test_moe_quantize_scale_ties_and_near_ties():
+    """Blocks whose amax over 6*s_g is exactly an E4M3 rounding midpoint (ties
+    to even) or one bf16 step from it.  With s_g = 2^-4 (the expert amax is
+    2688 * 2^-4 = 168) each quotient is exact, so the division the kernel may
+    skip in the common case must be taken here and must round like the oracle."""
+    import ml_dtypes
+    codes = np.arange(0, 126, dtype=np.uint8)
+    v = codes.view(ml_dtypes.float8_e4m3fn).astype(np.float64)
+    w = (codes + 1).view(ml_dtypes.float8_e4m3fn).astype(np.float64)
+    mids = (v + w) / 2                                        # 126 midpoints, at most 5 significant bits
+    a = synthetic.f32_to_bf16_bits((mids * 6 * 2.0 ** -4).astype(np.float32))
+    assert np.array_equal(synthetic.bf16_bits_to_f32(a).astype(np.float64), mids * 6 * 2.0 ** -4)
+    amaxes = np.concatenate([a, a + 1, a - 1])               # ties, one bf16 step above and below
+    amaxes = amaxes[synthetic.bf16_bits_to_f32(amaxes) > 0]
+    T, H = 64, 512
+    x = np.zeros((T, H), np.uint16)
+    x[0, 0] = synthetic.f32_to_bf16_bits(np.float32([168.0]))[0]            # expert amax -> s_g = 2^-4
+    blocks = x.reshape(T, H // 16, 16)
+    flat = blocks.reshape(-1, 16)
+    n = min(len(amaxes), flat.shape[0] - 1)
+    flat[1:1 + n, 3] = amaxes[:n]                                            # the block amax
+    flat[1:1 + n, 7] = synthetic.f32_to_bf16_bits(-0.5 * synthetic.bf16_bits_to_f32(amaxes[:n]))  # exact halves
+    x = flat.reshape(T, H)
+    slot = np.arange(T, dtype=np.int64).reshape(T, 1)
+    off = np.array([0, T], dtype=np.int32)
+    _moe_quantize_check(x, slot, off, 1, 1)
+    _, _, gs_ref, _ = oracle.quantize(x, None, off)
+    assert gs_ref[0] == np.float32(2.0 ** -4)
+
+
 def test_moe_quantize_dropped_choices_and_bad_index():
     """Choices with slot -1 are skipped; a slot beyond the routed rows is
     reported as an index error and skipped."""
