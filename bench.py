@@ -488,12 +488,14 @@ def comp_decode_w4a16(device, iters, warmup, flush):
     h = torch.empty((R, I), dtype=torch.bfloat16, device=device)
     y = torch.empty((R, H), dtype=torch.bfloat16, device=device)
 
+    ws = L.w4a16_workspace(R, E, max(H, I), device)
+
     def layer():
-        L.grouped_gemm_w4a16(xb, packs[0], 2 * I, ri, off, E, rows=R, out_dtype=1, swiglu=True, y=h)
-        L.grouped_gemm_w4a16(h, packs[1], H, None, off, E, rows=R, out_dtype=1, y=y)
+        L.grouped_gemm_w4a16(xb, packs[0], 2 * I, ri, off, E, rows=R, out_dtype=1, swiglu=True, y=h, ws=ws)
+        L.grouped_gemm_w4a16(h, packs[1], H, None, off, E, rows=R, out_dtype=1, y=y, ws=ws)
     ms = timed(layer, iters, warmup, flush)
     t_gu = timed(lambda: L.grouped_gemm_w4a16(xb, packs[0], 2 * I, ri, off, E, rows=R, out_dtype=1, swiglu=True,
-                                             y=h), iters, warmup, flush)
+                                             y=h, ws=ws), iters, warmup, flush)
     touched = int((np.diff(r["offsets"]) > 0).sum())
     wbytes = touched * (2 * I * H + H * I) * 0.5625
     gu_bytes = touched * 2 * I * H * 0.5625

@@ -301,28 +301,39 @@ nvfp4_status mxfp4_grouped_gemm(const uint8_t *a_q, const uint8_t *a_sf, const u
 /*
  * nvfp4_grouped_gemm_w4a16 -- weight-only NVFP4 grouped GEMM with bf16
  * activations: Y_e = X_e (b_gs[e] * W_e)^T for every expert e, fp32 accumulate.
- * [P5: the MTP layer's experts are W4A16_NVFP4 -- NVFP4 weights, BF16
+ * [P5: the MTP layer's experts are W4A16_NVFP4 -- NVFP4 weights, 16-bit
  *  activations; P1/P2: the weight format and its dequantisation.]
- * A streaming kernel for decode-sized groups: each weight row is read once
- * per 8 tokens of its expert.
- *   x, ld_x, x_rows  bf16 [x_rows, ld_x] activations (ld_x >= K, % 8 == 0).
+ * A streaming kernel for decode-sized groups (8 tokens per weight pass).  The
+ * tensor-core operands are f16: the weights exactly (e2m1 * e4m3 fits f16),
+ * the activations after a per-row power-of-two scaling 2^-k that puts the row's
+ * max |x| in [2^14, 2^15) -- exact for every element within 2^29 of the row
+ * max, smaller ones rounded to f16's subnormal grid (error < 2^-25 * max|x|);
+ * the epilogue multiplies by 2^k again.
+ *   x, ld_x, x_rows  bf16 [x_rows, ld_x] activations (ld_x >= K, % 8 == 0,
+ *               16-byte aligned).
  *   row_index   nullable int32 [M_total]: routed row r reads x[row_index[r]]
  *               (an entry outside [0, x_rows) reads row 0 and reports
  *               NVFP4_ERR_INDEX); NULL: row r reads x[r] (x_rows >= M_total).
  *   b_q, b_sf, b_gs  packed weights [E, N, K/2], ROW-MAJOR E4M3 scales
- *               [E*N, K/16], fp32 global per expert.
+ *               [E*N, K/16] (16-byte aligned), fp32 global per expert.
  *   expert_offsets, num_experts  int32 [E+1] prefix sums over routed rows
- *               (NULL: one dense GEMM).
- *   M_total, N, K    K % 64 == 0; N % 32 == 0 (N % 64 == 0 with SwiGLU).
+ *               (NULL: one dense GEMM); num_experts <= 1024.
+ *   M_total, N, K    K % 256 == 0; N % 128 == 0.
  *   y, out_dtype     fp32 or bf16 [M_total, N] (routed order); with
  *               NVFP4_EPI_SWIGLU the weight is a fused gate_up [2I, K] (gate
  *               rows first) and y is h = silu(g) * u, [M_total, N/2].
+ *   workspace   >= nvfp4_w4a16_workspace_size(M_total, num_experts, K) bytes,
+ *               16-byte aligned (the scaled f16 activations and their scales).
+ *   dev_status  NVFP4_ERR_INDEX, NVFP4_ERR_NONFINITE (a non-finite activation
+ *               row), NVFP4_ERR_TIMEOUT.
  */
+size_t nvfp4_w4a16_workspace_size(int64_t M_total, int num_experts, int64_t K);
 nvfp4_status nvfp4_grouped_gemm_w4a16(const void *x, int64_t ld_x, int64_t x_rows, const int32_t *row_index,
                                       const uint8_t *b_q, const uint8_t *b_sf, const float *b_gs,
                                       const int32_t *expert_offsets, int num_experts, int64_t M_total,
                                       int64_t N, int64_t K, void *y, nvfp4_out_dtype out_dtype,
-                                      nvfp4_epilogue epi, int32_t *dev_status, cudaStream_t stream);
+                                      nvfp4_epilogue epi, void *workspace, int32_t *dev_status,
+                                      cudaStream_t stream);
 
 /*
  * nvfp4_gemm_select_kernel -- which grouped GEMM kernel nvfp4_grouped_gemm runs

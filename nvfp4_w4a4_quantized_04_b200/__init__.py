@@ -48,7 +48,7 @@ EXPORTS = [
     "nvfp4_swiglu_quantize", "nvfp4_kv_quantize", "nvfp4_kv_dequantize", "nvfp4_quantize_noalloc",
     "nvfp4_moe_route_workspace_size", "nvfp4_moe_route", "nvfp4_moe_combine", "nvfp4_moe_quantize",
     "nvfp4_gemm_select_kernel", "nvfp4_grouped_gemm_w4a16", "nvfp4_grouped_gemm_swiglu_nvfp4",
-    "mxfp4_quantize", "mxfp4_grouped_gemm",
+    "mxfp4_quantize", "mxfp4_grouped_gemm", "nvfp4_w4a16_workspace_size",
 ]
 NOALLOC_MAX_GROUPS = 1024
 
@@ -79,7 +79,9 @@ def load_library(path: str = LIB_PATH):
     L.nvfp4_grouped_gemm_swiglu_nvfp4.restype = i32
     L.nvfp4_grouped_gemm_swiglu_nvfp4.argtypes = [P, P, P, P, P, P, P, i32, i64, i64, i64, P, P, P, P, P, P]
     L.nvfp4_grouped_gemm_w4a16.restype = i32
-    L.nvfp4_grouped_gemm_w4a16.argtypes = [P, i64, i64, P, P, P, P, P, i32, i64, i64, i64, P, i32, i32, P, P]
+    L.nvfp4_grouped_gemm_w4a16.argtypes = [P, i64, i64, P, P, P, P, P, i32, i64, i64, i64, P, i32, i32, P, P, P]
+    L.nvfp4_w4a16_workspace_size.restype = ctypes.c_size_t
+    L.nvfp4_w4a16_workspace_size.argtypes = [i64, i32, i64]
     L.nvfp4_gemm_select_kernel.restype = i32
     L.nvfp4_gemm_select_kernel.argtypes = [i32]
     L.nvfp4_moe_quantize.restype = i32
@@ -173,12 +175,16 @@ def nvfp4_grouped_gemm_swiglu_nvfp4(a_q, a_sf, a_gs, b_q, b_sf, b_gs, expert_off
     return st
 
 
+def nvfp4_w4a16_workspace_size(M_total: int, num_experts: int, K: int) -> int:
+    return int(load_library().nvfp4_w4a16_workspace_size(M_total, num_experts, K))
+
+
 def nvfp4_grouped_gemm_w4a16(x, ld_x, x_rows, row_index, b_q, b_sf, b_gs, expert_offsets, num_experts, M_total,
-                             N, K, y, out_dtype, epi, dev_status=None, stream=None, check=True) -> int:
+                             N, K, y, out_dtype, epi, workspace, dev_status=None, stream=None, check=True) -> int:
     """Weight-only NVFP4 grouped GEMM, bf16 activations (row-major weight scales)."""
     st = load_library().nvfp4_grouped_gemm_w4a16(
         _ptr(x), ld_x, x_rows, _ptr(row_index), _ptr(b_q), _ptr(b_sf), _ptr(b_gs), _ptr(expert_offsets),
-        num_experts, M_total, N, K, _ptr(y), out_dtype, epi, _ptr(dev_status), _stream(stream))
+        num_experts, M_total, N, K, _ptr(y), out_dtype, epi, _ptr(workspace), _ptr(dev_status), _stream(stream))
     if check:
         _check(st, "nvfp4_grouped_gemm_w4a16")
     return st

@@ -1,245 +1,478 @@
-// Weight-only NVFP4 grouped GEMM, bf16 activations (W4A16), sm_100a.
+// Weight-only NVFP4 grouped GEMM with 16-bit activations (W4A16), sm_100a.
 //
 // The "DeepSeek-V4.1-Flash-NVFP4" page lists the MTP layer's experts as
 // W4A16_NVFP4: the weights are NVFP4 (E2M1 codes, E4M3 scale per 16, FP32
-// global) and the activations stay bf16.  For every routed expert e:
+// global) and the activations stay 16-bit.  For every routed expert e:
 //   Y_e = X_e (s_g[e] * W_e)^T,   W_e[n, k] = e2m1(code) * e4m3(S[n, k/16]),
 // accumulated in fp32.  With the SwiGLU epilogue the weight is a fused gate_up
 // [2I, K] (gate rows 0..I-1, up rows I..2I-1) and the output is
-// h = bf16(silu(g) * u).
+// h = silu(g) * u.
 //
 // Built for decode-sized expert groups (a few tokens per expert), where the
-// weight bytes dominate: a warp owns 32 weight rows x 8 tokens and runs
-// mma.sync m16n8k16 (bf16 in, fp32 accumulate) over K, every weight byte read
-// once per 8 tokens.  The 16-element K slices of the instruction are mapped to
-// memory so that each lane's A elements are 16 consecutive codes of a row (one
-// 8-byte load, one E4M3 scale) and its B elements 16 consecutive bf16 of a
-// token; the same permutation on both sides leaves the dot products unchanged.
-// E2M1 -> bf16 and the product with the scale in bf16 are exact (at most 6
-// significant bits); s_g multiplies the accumulated sum once.
-#include <cuda_runtime.h>
-#include <cuda_bf16.h>
-#include <cuda_fp16.h>
-#include <stdint.h>
+// weight bytes dominate and the kernel must stream them at HBM rate:
+//  * Tensor-core operands in f16.  E2M1 -> f16 is one hardware conversion per
+//    two codes, and e2m1 * e4m3 is exact in f16 (at most 6 significant bits,
+//    |.| in [2^-10, 2688]), so each weight element costs one conversion and
+//    one f16x2 multiply per pair.  The bf16 activations are converted once per
+//    call by a prep kernel: each routed row is scaled by a power of two 2^-k
+//    that puts its max |x| in [2^14, 2^15), then rounded to f16.  Every
+//    element within 2^29 of the row's max is exact; smaller ones land on f16's
+//    subnormal grid (error below 2^-25 of the row max).  The epilogue
+//    multiplies by 2^k again, which is exact.
+//  * Pipeline.  One producer warp streams, per 256-element K stage, the
+//    128-row weight tile and its scales by TMA (128-byte swizzle) and the
+//    item's 8 activation rows (4 KB, pre-arranged by the prep kernel in
+//    fragment order) by one bulk copy, into an 8-stage ring of 22 KB stages.
+//    Sixteen consumer warps run mma.sync m16n8k16 (f16 in, fp32 accumulate):
+//    warp w owns weight rows 16 (w%8) .. +16 (x 8 tokens) and the K half w/8
+//    of every stage; the two halves are added through shared memory at the
+//    end of the item.  Two warps per row tile hide the latency of the
+//    conversion -> multiply -> MMA chain.
+//  * K permutation.  Within a stage, lane t of a quad holds K range
+//    [64t, 64t+64) of its rows: MMA slice s takes physical K 64t + 4s + {0..3},
+//    the same on both operands, which leaves the dot products unchanged and
+//    gives each lane two 16-byte weight loads and one scale word per row.
+//  * Work item = (expert, 128-row weight block, chunk of 8 tokens); an expert
+//    with more than 8 tokens re-reads its weight block per chunk, and those
+//    reads follow each other so they hit L2.
+//  * Every mbarrier wait is bounded (NVFP4_ERR_TIMEOUT, then all roles leave).
+#include "gemm_common.cuh"
 
-#include "common.cuh"
+#include <cuda_fp16.h>
 
 namespace nvfp4 {
 namespace w4a16 {
 
-constexpr int kTokChunk = 8;       // tokens per warp tile (MMA N)
-constexpr int kRows = 32;          // weight rows per warp: two MMA tiles of 16 sharing the B fragment
-constexpr int kThreads = 256;
+using gemm::kWaitBudgetCycles;
+using gemm::mbar_arrive;
+using gemm::mbar_arrive_expect_tx;
+using gemm::mbar_init;
+using gemm::mbar_try_wait;
+using gemm::mbar_wait;
+using gemm::smem_u32;
 
-// Two E2M1 codes (one byte, element 2i in the low nibble) times a bf16x2 scale
-// -> one bf16x2 register (low half = even element), exact.
-__device__ __forceinline__ uint32_t e2m1x2_bf16x2(uint32_t byte, uint32_t s2) {
-  uint32_t h, r;
-  asm("{\n.reg .b8 b;\n.reg .f16 l, u;\n.reg .f32 fl, fu;\ncvt.u8.u32 b, %1;\ncvt.rn.f16x2.e2m1x2 %0, b;\n}"
-      : "=r"(h) : "r"(byte));
-  asm("{\n.reg .f16 l, u;\n.reg .f32 fl, fu;\nmov.b32 {l, u}, %1;\ncvt.f32.f16 fl, l;\ncvt.f32.f16 fu, u;\n"
-      "cvt.rn.bf16x2.f32 %0, fu, fl;\n}" : "=r"(r) : "r"(h));
-  asm("mul.rn.bf16x2 %0, %0, %1;" : "+r"(r) : "r"(s2));
-  return r;
+constexpr int kTok = 8;                      // tokens per item (MMA N)
+constexpr int kConsumers = 16;               // consumer warps: 8 row tiles x 2 K halves
+constexpr int kThreads = (kConsumers + 1) * 32;
+constexpr int kStages = 8;
+constexpr int kWBytes = 128 * 128;           // 128 rows x 256 codes
+constexpr int kSBytes = 128 * 16;            // 128 rows x 16 scales
+constexpr int kXBytes = kTok * 256 * 2;      // 8 tokens x 256 f16
+constexpr int kStageBytes = kWBytes + kSBytes + kXBytes;
+constexpr int OFF_BAR = kStages * kStageBytes;
+constexpr int OFF_MISC = OFF_BAR + 2 * kStages * 8;
+constexpr int OFF_RED = OFF_MISC + 16;       // K-half partial sums: 8 warps x 32 lanes x 4 floats
+constexpr int OFF_TABLES = OFF_RED + 8 * 32 * 16;
+constexpr int kMaxExperts = 1024;
+constexpr int TABLE_BYTES = 3 * (kMaxExperts + 1) * 4 + 32 * 4;
+constexpr int SMEM_BYTES = OFF_TABLES + TABLE_BYTES + 1024;
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+
+// Block-wide exclusive prefix sums over e < E of f(e), into out[0..E].
+template <typename F>
+__device__ void block_prefix(int E, int32_t *out, int32_t *scratch, F f) {
+  const int nt = blockDim.x, t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int per = (E + nt - 1) / nt;
+  const int e0 = min(E, t * per), e1 = min(E, e0 + per);
+  int32_t local = 0;
+  for (int e = e0; e < e1; ++e) local += f(e);
+  int32_t incl = local;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int32_t v = __shfl_up_sync(0xffffffffu, incl, d);
+    if (lane >= d) incl += v;
+  }
+  if (lane == 31) scratch[warp] = incl;
+  __syncthreads();
+  if (t == 0) {
+    int32_t a = 0;
+    for (int w = 0; w < nt / 32; ++w) { const int32_t v = scratch[w]; scratch[w] = a; a += v; }
+  }
+  __syncthreads();
+  int32_t run = scratch[warp] + incl - local;
+  for (int e = e0; e < e1; ++e) { out[e] = run; run += f(e); }
+  if (e1 == E && e0 < e1) out[E] = run;
+  if (E == 0 && t == 0) out[0] = 0;
+  __syncthreads();
 }
 
-// E4M3 byte -> bf16 in both halves (exact: every E4M3 value is a bf16).
-__device__ __forceinline__ uint32_t e4m3_bf16x2(uint32_t s) {
-  uint32_t h, r;
-  asm("{\n.reg .b16 b;\ncvt.u16.u32 b, %1;\ncvt.rn.f16x2.e4m3x2 %0, b;\n}" : "=r"(h) : "r"(s & 0xFFu));
-  asm("{\n.reg .f16 l, u;\n.reg .f32 fl;\nmov.b32 {l, u}, %1;\ncvt.f32.f16 fl, l;\ncvt.rn.bf16x2.f32 %0, fl, fl;\n}"
-      : "=r"(r) : "r"(h));
-  return r;
+// ------------------------------------------------------------------ prep
+// Activation layout in the workspace: the tokens of expert e form
+// ceil(n_e/8) chunks of 8 rows, chunk index C = cslot[e] + c.  For chunk C and
+// K stage st the 4 KB block at ((C * nst + st) * 2048) halves holds, at
+// 16-byte piece (i * 32 + L), token g = L/4 at K = 256 st + 64 (L%4) + 8 i ..
+// +8: lane L of a consumer warp reads its pieces i = 0..7 with conflict-free
+// 16-byte shared loads.  xscale[C * 8 + g] = 2^k of that token.
+__global__ void __launch_bounds__(256) w4a16_prep_kernel(
+    const uint16_t *__restrict__ x, int64_t ld_x, int64_t x_rows, const int32_t *__restrict__ row_index,
+    const int32_t *__restrict__ offsets, int E, int64_t M_total, int K, uint16_t *__restrict__ x16,
+    float *__restrict__ xscale, int32_t *dev_status) {
+  extern __shared__ int32_t smem[];
+  int32_t *off = smem, *cslot = smem + (E + 1), *scratch = smem + 2 * (E + 1);
+  for (int i = threadIdx.x; i <= E; i += blockDim.x)
+    off[i] = offsets ? offsets[i] : (i == 0 ? 0 : (int32_t)M_total);
+  __syncthreads();
+  block_prefix(E, cslot, scratch, [&](int e) { return (off[e + 1] - off[e] + kTok - 1) / kTok; });
+  const int lane = threadIdx.x & 31;
+  const int nst = K / 256;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  bool bad_index = false, bad_value = false;
+  for (int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < M_total; r += nwarps) {
+    const int e = upper_group(off, E, r);
+    const int i = (int)(r - off[e]);
+    const int64_t C = cslot[e] + i / kTok;
+    const int g = i % kTok;
+    int64_t src = row_index ? (int64_t)row_index[r] : r;
+    if (src < 0 || src >= x_rows) { src = 0; bad_index = true; }
+    const uint16_t *xr = x + src * ld_x;
+    uint32_t m = 0;
+    for (int k = lane * 8; k < K; k += 256) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4 *>(xr + k));
+      m = __vmaxu2(m, v.x & 0x7FFF7FFFu);
+      m = __vmaxu2(m, v.y & 0x7FFF7FFFu);
+      m = __vmaxu2(m, v.z & 0x7FFF7FFFu);
+      m = __vmaxu2(m, v.w & 0x7FFF7FFFu);
+    }
+    m = max(m & 0xFFFFu, m >> 16);
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, d));
+    if (m >= 0x7F80u) bad_value = true;
+    // k = floor(log2 max) - 14, kept where 2^k and 2^-k are fp32 normals
+    int k = (m == 0 || m >= 0x7F80u) ? 0 : (int)(m >> 7) - 127 - 14;
+    k = max(-126, min(k, 113));
+    const float sc = __uint_as_float((uint32_t)(127 - k) << 23);
+    if (lane == 0) xscale[C * kTok + g] = __uint_as_float((uint32_t)(127 + k) << 23);
+    uint16_t *dst = x16 + C * (int64_t)nst * 2048;
+    for (int p = lane; p < K / 8; p += 32) {
+      const int st = p >> 5, rest = p & 31, t = rest >> 3, i8 = rest & 7;
+      const int kk = st * 256 + 64 * t + 8 * i8;
+      const uint4 v = __ldg(reinterpret_cast<const uint4 *>(xr + kk));
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+      uint32_t o[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float lo = __fmul_rn(__uint_as_float(w[j] << 16), sc);
+        const float hi = __fmul_rn(__uint_as_float(w[j] & 0xFFFF0000u), sc);
+        const __half2 h = __floats2half2_rn(lo, hi);
+        o[j] = *reinterpret_cast<const uint32_t *>(&h);
+      }
+      *reinterpret_cast<uint4 *>(dst + (int64_t)st * 2048 + (i8 * 32 + g * 4 + t) * 8) =
+          make_uint4(o[0], o[1], o[2], o[3]);
+    }
+  }
+  if (bad_index) report(dev_status, NVFP4_ERR_INDEX);
+  if (bad_value) report(dev_status, NVFP4_ERR_NONFINITE);
 }
 
-__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                         uint32_t b0, uint32_t b1) {
-  asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+// ------------------------------------------------------------------ GEMM
+// Two E2M1 codes (one byte, element 2i in the low nibble) -> f16x2, exact.
+__device__ __forceinline__ uint32_t e2m1x2_f16x2(uint32_t byte) {
+  uint32_t h;
+  asm("{\n.reg .b8 b;\ncvt.u8.u32 b, %1;\ncvt.rn.f16x2.e2m1x2 %0, b;\n}" : "=r"(h) : "r"(byte));
+  return h;
+}
+
+// Two E4M3 bytes (low 16 bits) -> f16x2 (low half = low byte), exact.
+__device__ __forceinline__ uint32_t e4m3x2_f16x2(uint32_t two) {
+  uint32_t h;
+  asm("{\n.reg .b16 b;\ncvt.u16.u32 b, %1;\ncvt.rn.f16x2.e4m3x2 %0, b;\n}" : "=r"(h) : "r"(two & 0xFFFFu));
+  return h;
+}
+
+__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+__device__ __forceinline__ void mma_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                        uint32_t b0, uint32_t b1) {
+  asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
                "{%0,%1,%2,%3};"
                : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
                : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// One 64-element K chunk of a 16-row weight tile against the B fragment:
-// lane (g = lane/4, t = lane%4) holds codes 16t..16t+15 of the chunk for rows
-// g and g+8 (wlo, whi) with their scales (slo, shi).
-__device__ __forceinline__ void chunk_mma(float (&d)[4], uint2 wlo, uint2 whi, uint32_t slo, uint32_t shi,
-                                          const uint32_t (&b)[8]) {
-  const uint32_t s_lo = e4m3_bf16x2(slo), s_hi = e4m3_bf16x2(shi);
-  const uint32_t lo[2] = {wlo.x, wlo.y}, hi[2] = {whi.x, whi.y};
-#pragma unroll
-  for (int s = 0; s < 4; ++s) {
-    // k-step s: elements 4s..4s+3 of the lane's 16 = bytes 2s, 2s+1
-    const uint32_t wl = lo[s >> 1] >> (16 * (s & 1)), wh = hi[s >> 1] >> (16 * (s & 1));
-    mma_bf16(d, e2m1x2_bf16x2(wl & 0xFFu, s_lo), e2m1x2_bf16x2(wh & 0xFFu, s_hi),
-             e2m1x2_bf16x2((wl >> 8) & 0xFFu, s_lo), e2m1x2_bf16x2((wh >> 8) & 0xFFu, s_hi), b[2 * s], b[2 * s + 1]);
-  }
+// The four block scales of a lane's 64 K elements, each broadcast to both halves.
+__device__ __forceinline__ void scales4(uint32_t word, uint32_t (&s)[4]) {
+  const uint32_t lo = e4m3x2_f16x2(word), hi = e4m3x2_f16x2(word >> 16);
+  s[0] = __byte_perm(lo, 0, 0x1010);
+  s[1] = __byte_perm(lo, 0, 0x3232);
+  s[2] = __byte_perm(hi, 0, 0x1010);
+  s[3] = __byte_perm(hi, 0, 0x3232);
 }
 
-// Work item = (expert, 16-row block (gate rows with SwiGLU), 8-token chunk).
+struct Item { int e, rb, c; };
+
+__device__ __forceinline__ Item decode_item(int64_t it, const int32_t *items, const int32_t *off, int E) {
+  Item I;
+  I.e = upper_group(items, E, it);
+  const int nch = (off[I.e + 1] - off[I.e] + kTok - 1) / kTok;
+  const int rem = (int)(it - items[I.e]);
+  I.rb = rem / nch;                       // weight block major: the chunks of one block follow each other
+  I.c = rem % nch;
+  return I;
+}
+
 template <bool kSwiglu, bool kBf16Out>
-__global__ void __launch_bounds__(kThreads) w4a16_kernel(
-    const uint16_t *__restrict__ x, int64_t ld_x, int64_t x_rows, const int32_t *__restrict__ row_index,
-    const uint8_t *__restrict__ wq, const uint8_t *__restrict__ wsf, const float *__restrict__ w_gs,
-    const int32_t *__restrict__ expert_offsets, int E, int64_t M_total, int N, int K, void *__restrict__ y,
+__global__ void __launch_bounds__(kThreads, 1) w4a16_kernel(
+    const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_s,
+    const uint16_t *__restrict__ x16, const float *__restrict__ xscale, const float *__restrict__ w_gs,
+    const int32_t *__restrict__ offsets, int E, int64_t M_total, int N, int K, void *__restrict__ y,
     int32_t *dev_status) {
-  extern __shared__ int32_t smem[];
-  int32_t *off = smem, *items = smem + (E + 1);       // items[e] = first work item of expert e
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar_full = sbase + OFF_BAR, bar_empty = bar_full + 8 * kStages;
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC);
+  volatile int *stop_word = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
+  int32_t *off = reinterpret_cast<int32_t *>(smem + OFF_TABLES);
+  int32_t *cslot = off + (kMaxExperts + 1), *items = cslot + (kMaxExperts + 1), *scratch = items + (kMaxExperts + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rows_out = kSwiglu ? N / 2 : N;
-  const int row_blocks = rows_out / kRows;
-  __shared__ int32_t scratch[kThreads / 32];
-  for (int i = threadIdx.x; i <= E; i += blockDim.x)
-    off[i] = expert_offsets ? expert_offsets[i] : (i == 0 ? 0 : (int32_t)M_total);
-  __syncthreads();
-  {
-    // items[e] = exclusive prefix sum of row_blocks * chunks(e): block-wide scan
-    const int per = (E + kThreads - 1) / kThreads;
-    const int e0 = min(E, (int)threadIdx.x * per), e1 = min(E, e0 + per);
-    int32_t local = 0;
-    for (int e = e0; e < e1; ++e) local += row_blocks * ((off[e + 1] - off[e] + kTokChunk - 1) / kTokChunk);
-    const int ln = threadIdx.x & 31, wp = threadIdx.x >> 5;
-    int32_t incl = local;
-#pragma unroll
-    for (int dd = 1; dd < 32; dd <<= 1) {
-      const int32_t v = __shfl_up_sync(0xffffffffu, incl, dd);
-      if (ln >= dd) incl += v;
+  const int row_blocks = kSwiglu ? rows_out / 64 : N / 128;
+  const int nst = K / 256;
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_empty + 8 * s, kConsumers);
     }
-    if (ln == 31) scratch[wp] = incl;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      int32_t a = 0;
-      for (int w = 0; w < kThreads / 32; ++w) { const int32_t v = scratch[w]; scratch[w] = a; a += v; }
-    }
-    __syncthreads();
-    int32_t run = scratch[wp] + incl - local;
-    for (int e = e0; e < e1; ++e) {
-      items[e] = run;
-      run += row_blocks * ((off[e + 1] - off[e] + kTokChunk - 1) / kTokChunk);
-    }
-    if (e1 == E && e0 < e1) items[E] = run;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
+  for (int i = threadIdx.x; i <= E; i += blockDim.x)
+    off[i] = offsets ? offsets[i] : (i == 0 ? 0 : (int32_t)M_total);
   __syncthreads();
-  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-  const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  block_prefix(E, cslot, scratch, [&](int e) { return (off[e + 1] - off[e] + kTok - 1) / kTok; });
+  block_prefix(E, items, scratch, [&](int e) { return row_blocks * ((off[e + 1] - off[e] + kTok - 1) / kTok); });
   const int64_t total = items[E];
-  const int64_t row_bytes = K / 2, sf_bytes = K / 16;
-  const int nchunks = K / 64;
-  bool bad_index = false;
-  for (int64_t it = warp; it < total; it += nwarps) {
-    const int e = upper_group(items, E, it);
-    const int64_t local = it - items[e];
-    const int rb = (int)(local % row_blocks);
-    const int chunk = (int)(local / row_blocks);
-    const int32_t r0 = off[e] + chunk * kTokChunk;
-    const int ntok = min(kTokChunk, off[e + 1] - r0);
-    // B rows: token g of the chunk (a missing token reads a valid row; its column is not stored)
-    int64_t src = r0 + min(g, ntok - 1);
-    if (row_index) {
-      src = row_index[src];
-      if (src < 0 || src >= x_rows) { src = 0; bad_index = true; }
-    }
-    const uint16_t *xr = x + src * ld_x + 16 * t;
-    const int64_t n0 = (int64_t)e * N + (int64_t)rb * kRows;
-    // lane rows g, g+8 (tile 0) and g+16, g+24 (tile 1); with SwiGLU the
-    // matching up rows N/2 further
-    const uint8_t *qrow = wq + (n0 + g) * row_bytes + 8 * t;
-    const uint8_t *frow = wsf + (n0 + g) * sf_bytes + t;
-    const int64_t up = (int64_t)(N / 2) * row_bytes, upf = (int64_t)(N / 2) * sf_bytes;
-    constexpr int NW = kSwiglu ? 8 : 4;               // weight rows per lane
-    float d[NW / 2][4] = {};
-    auto load = [&](int c, uint4 &x0, uint4 &x1, uint2 (&w)[NW], uint32_t (&sc)[NW]) {
-      x0 = __ldg(reinterpret_cast<const uint4 *>(xr + 64 * c));
-      x1 = __ldg(reinterpret_cast<const uint4 *>(xr + 64 * c + 8));
-#pragma unroll
-      for (int i = 0; i < NW; ++i) {
-        const int64_t ro = (int64_t)(i & 3) * 8;           // rows g, g+8, g+16, g+24
-        const int64_t qo = ro * row_bytes + (i >= 4 ? up : 0), fo = ro * sf_bytes + (i >= 4 ? upf : 0);
-        w[i] = __ldg(reinterpret_cast<const uint2 *>(qrow + qo + 32 * c));
-        sc[i] = __ldg(frow + fo + 4 * c);
+
+  if (warp == kConsumers) {
+    // ================================================================ producer
+    if (lane == 0) {
+      const uint64_t pol = gemm::policy_evict_first();
+      int stage = 0;
+      uint32_t phase = 0;
+      bool armed[kStages] = {};
+      uint32_t armed_parity[kStages] = {};
+      bool ok = true;
+      for (int64_t it = blockIdx.x; it < total && ok; it += gridDim.x) {
+        const Item I = decode_item(it, items, off, E);
+        const int64_t C = cslot[I.e] + I.c;
+        const int32_t row0 = I.e * N + I.rb * (kSwiglu ? 64 : 128);
+        const int32_t uprow0 = row0 + N / 2;
+        for (int st = 0; st < nst; ++st) {
+          if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1, abort_flag, dev_status)) { ok = false; break; }
+          const uint32_t fb = bar_full + 8 * stage;
+          mbar_arrive_expect_tx(fb, kStageBytes);
+          armed[stage] = true;
+          armed_parity[stage] = phase;
+          const uint32_t base = sbase + stage * kStageBytes;
+          if (kSwiglu) {
+            gemm::tma_load_2d(base, &tmap_w, st * 128, row0, fb, pol);
+            gemm::tma_load_2d(base + kWBytes / 2, &tmap_w, st * 128, uprow0, fb, pol);
+            gemm::tma_load_2d(base + kWBytes, &tmap_s, st * 16, row0, fb, pol);
+            gemm::tma_load_2d(base + kWBytes + kSBytes / 2, &tmap_s, st * 16, uprow0, fb, pol);
+          } else {
+            gemm::tma_load_2d(base, &tmap_w, st * 128, row0, fb, pol);
+            gemm::tma_load_2d(base + kWBytes, &tmap_s, st * 16, row0, fb, pol);
+          }
+          gemm::bulk_load(base + kWBytes + kSBytes, x16 + (C * nst + st) * 2048, kXBytes, fb);
+          if (++stage == kStages) { stage = 0; phase ^= 1; }
+        }
       }
-    };
-    uint4 x0, x1;
-    uint2 w[NW];
-    uint32_t sc[NW];
-    load(0, x0, x1, w, sc);
-    for (int c = 0; c < nchunks; ++c) {
-      uint4 nx0 = x0, nx1 = x1;
-      uint2 nw[NW];
-      uint32_t nsc[NW];
-#pragma unroll
-      for (int i = 0; i < NW; ++i) { nw[i] = w[i]; nsc[i] = sc[i]; }
-      if (c + 1 < nchunks) load(c + 1, nx0, nx1, nw, nsc);     // next chunk in flight during this one
-      const uint32_t b[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-#pragma unroll
-      for (int m = 0; m < NW / 2; ++m) chunk_mma(d[m], w[2 * m], w[2 * m + 1], sc[2 * m], sc[2 * m + 1], b);
-      x0 = nx0; x1 = nx1;
-#pragma unroll
-      for (int i = 0; i < NW; ++i) { w[i] = nw[i]; sc[i] = nsc[i]; }
+      // every armed stage's copies land before the CTA exits
+      for (int s = 0; s < kStages; ++s) {
+        if (!armed[s]) continue;
+        const long long t0 = clock64();
+        while (!mbar_try_wait(bar_full + 8 * s, armed_parity[s]) && clock64() - t0 < kWaitBudgetCycles) {}
+      }
     }
-    // tile m (0, 1): d[m][0..1] row 16m+g, d[m][2..3] row 16m+g+8, tokens 2t, 2t+1;
-    // with SwiGLU d[2+m] holds the matching up rows
-    const float gs = w_gs[e];
+  } else {
+    // ================================================================ consumers
+    const int g = lane >> 2, t = lane & 3;
+    const int tile = warp & 7, half = warp >> 3;                      // row tile, K half of each stage
+    const int rowA = kSwiglu ? 8 * tile + g : 16 * tile + g;          // MMA rows g and g + 8
+    const int rowB = kSwiglu ? 64 + 8 * tile + g : 16 * tile + 8 + g;
+    // the lane's 16 code bytes of this half: 16-byte chunk 2t + half of the row (128-byte swizzle)
+    const uint32_t offA = rowA * 128 + (((2 * t + half) ^ (rowA & 7)) << 4);
+    const uint32_t offB = rowB * 128 + (((2 * t + half) ^ (rowB & 7)) << 4);
+    float *red = reinterpret_cast<float *>(smem + OFF_RED) + (tile * 32 + lane) * 4;
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int64_t it = blockIdx.x; it < total; it += gridDim.x) {
+      const Item I = decode_item(it, items, off, E);
+      float d[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int st = 0; st < nst; ++st) {
+        if (!gemm::mbar_wait_warp(bar_full + 8 * stage, phase, abort_flag, dev_status)) break;
+        const uint8_t *base = smem + stage * kStageBytes;
+        const uint4 wa = *reinterpret_cast<const uint4 *>(base + offA);
+        const uint4 wb = *reinterpret_cast<const uint4 *>(base + offB);
+        // scales of K blocks 4t + 2 half .. +1 (two bytes of the lane's word)
+        const uint32_t sa = *reinterpret_cast<const uint16_t *>(base + kWBytes + rowA * 16 + 4 * t + 2 * half);
+        const uint32_t sb = *reinterpret_cast<const uint16_t *>(base + kWBytes + rowB * 16 + 4 * t + 2 * half);
+        uint4 xp[4];
 #pragma unroll
-    for (int m = 0; m < 2; ++m) {
+        for (int i = 0; i < 4; ++i)
+          xp[i] = *reinterpret_cast<const uint4 *>(base + kWBytes + kSBytes + ((4 * half + i) * 32 + lane) * 16);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_empty + 8 * stage);     // release: the loads above are ordered before it
+        if (++stage == kStages) { stage = 0; phase ^= 1; }
+        const uint32_t hA = e4m3x2_f16x2(sa), hB = e4m3x2_f16x2(sb);
+        const uint32_t sA[2] = {__byte_perm(hA, 0, 0x1010), __byte_perm(hA, 0, 0x3232)};
+        const uint32_t sB[2] = {__byte_perm(hB, 0, 0x1010), __byte_perm(hB, 0, 0x3232)};
+        const uint32_t wA[4] = {wa.x, wa.y, wa.z, wa.w};
+        const uint32_t wB[4] = {wb.x, wb.y, wb.z, wb.w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int tok = 2 * t + (i & 1);
-        const int row = rb * kRows + 16 * m + g + 8 * (i >> 1);
-        if (tok < ntok) {
-          const float gv = __fmul_rn(d[m][i], gs);
-          float v = gv;
-          if constexpr (kSwiglu) v = __fmul_rn(__fdividef(gv, 1.0f + __expf(-gv)), __fmul_rn(d[2 + m][i], gs));
-          const int64_t o = (int64_t)(r0 + tok) * rows_out + row;
-          if (kBf16Out) reinterpret_cast<__nv_bfloat16 *>(y)[o] = __float2bfloat16_rn(v);
-          else reinterpret_cast<float *>(y)[o] = v;
+        for (int s = 0; s < 8; ++s) {
+          // slice 8 half + s: physical K 64t + 4 (8 half + s) .. +3, bytes 2s, 2s+1 of the lane's 16
+          const uint32_t ca = wA[s >> 1] >> (16 * (s & 1)), cb = wB[s >> 1] >> (16 * (s & 1));
+          const uint32_t a0 = hmul2(e2m1x2_f16x2(ca & 0xFFu), sA[s >> 2]);
+          const uint32_t a2 = hmul2(e2m1x2_f16x2((ca >> 8) & 0xFFu), sA[s >> 2]);
+          const uint32_t a1 = hmul2(e2m1x2_f16x2(cb & 0xFFu), sB[s >> 2]);
+          const uint32_t a3 = hmul2(e2m1x2_f16x2((cb >> 8) & 0xFFu), sB[s >> 2]);
+          const uint4 xv = xp[s >> 1];
+          const uint32_t b0 = (s & 1) ? xv.z : xv.x, b1 = (s & 1) ? xv.w : xv.y;
+          mma_f16(d, a0, a1, a2, a3, b0, b1);
+        }
+      }
+      // The second K half hands its partial sums to the first.  Every consumer
+      // warp reaches both barriers of every item it starts (a wait that gave
+      // up only ends the stage loop), and the decision to stop is read from
+      // one shared word after the second barrier, so all warps leave together.
+      if (half == 1) *reinterpret_cast<float4 *>(red) = make_float4(d[0], d[1], d[2], d[3]);
+      asm volatile("bar.sync 1, %0;" :: "n"(kConsumers * 32) : "memory");
+      if (half == 0) {
+        const float4 p = *reinterpret_cast<const float4 *>(red);
+        d[0] += p.x; d[1] += p.y; d[2] += p.z; d[3] += p.w;
+      }
+      if (warp == 0 && lane == 0) *stop_word = *abort_flag;
+      asm volatile("bar.sync 1, %0;" :: "n"(kConsumers * 32) : "memory");
+      if (*stop_word) break;
+      if (half == 1) continue;
+      // d[0], d[1]: row A, tokens 2t, 2t+1; d[2], d[3]: row B
+      const int32_t r0 = off[I.e] + I.c * kTok;
+      const int ntok = min(kTok, off[I.e + 1] - r0);
+      const int64_t C = cslot[I.e] + I.c;
+      const float gs = w_gs[I.e];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int tok = 2 * t + j;
+        if (tok >= ntok) continue;
+        const float xs = xscale[C * kTok + tok];
+        const float va = __fmul_rn(__fmul_rn(d[j], gs), xs);
+        const float vb = __fmul_rn(__fmul_rn(d[2 + j], gs), xs);
+        if constexpr (kSwiglu) {
+          const float h = __fmul_rn(__fdividef(va, 1.0f + __expf(-va)), vb);
+          const int64_t o = (int64_t)(r0 + tok) * rows_out + I.rb * 64 + 8 * tile + g;
+          if (kBf16Out) reinterpret_cast<__nv_bfloat16 *>(y)[o] = __float2bfloat16_rn(h);
+          else reinterpret_cast<float *>(y)[o] = h;
+        } else {
+          const int64_t o = (int64_t)(r0 + tok) * rows_out + I.rb * 128 + 16 * tile + g;
+          if (kBf16Out) {
+            reinterpret_cast<__nv_bfloat16 *>(y)[o] = __float2bfloat16_rn(va);
+            reinterpret_cast<__nv_bfloat16 *>(y)[o + 8] = __float2bfloat16_rn(vb);
+          } else {
+            reinterpret_cast<float *>(y)[o] = va;
+            reinterpret_cast<float *>(y)[o + 8] = vb;
+          }
         }
       }
     }
   }
-  if (bad_index) report(dev_status, NVFP4_ERR_INDEX);
+  __syncthreads();
 }
 
 }  // namespace w4a16
 }  // namespace nvfp4
 
+// ====================================================================== host side
 using namespace nvfp4;
+
+namespace {
+
+// 2-D uint8 view [rows, row_bytes] with a {16 bytes, box_rows} box, no swizzle
+// (row-major E4M3 scales: 16 per 256-element K stage).
+bool make_map_scales16(CUtensorMap *map, const void *base, uint64_t rows, uint64_t row_bytes, uint32_t box_rows) {
+  auto enc = gemm::tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {row_bytes, rows};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {16, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Upper bound on the 8-token chunks of all experts: sum ceil(n_e / 8).
+int64_t w4a16_chunks_bound(int64_t M_total, int E) { return (M_total + 7 * (int64_t)E) / 8 + 1; }
+
+size_t w4a16_x16_bytes(int64_t M_total, int E, int64_t K) {
+  return ((size_t)w4a16_chunks_bound(M_total, E) * 8 * (size_t)K * 2 + 255) / 256 * 256;
+}
+
+bool g_w4a16_attr[4] = {false, false, false, false};
+
+}  // namespace
+
+extern "C" size_t nvfp4_w4a16_workspace_size(int64_t M_total, int num_experts, int64_t K) {
+  if (M_total < 0 || K <= 0) return 0;
+  const int E = num_experts < 1 ? 1 : num_experts;
+  return w4a16_x16_bytes(M_total, E, K) + (size_t)w4a16_chunks_bound(M_total, E) * 8 * sizeof(float) + 256;
+}
 
 extern "C" nvfp4_status nvfp4_grouped_gemm_w4a16(const void *x, int64_t ld_x, int64_t x_rows, const int32_t *row_index,
                                                  const uint8_t *b_q, const uint8_t *b_sf, const float *b_gs,
                                                  const int32_t *expert_offsets, int num_experts, int64_t M_total,
                                                  int64_t N, int64_t K, void *y, nvfp4_out_dtype out_dtype,
-                                                 nvfp4_epilogue epi, int32_t *dev_status, cudaStream_t stream) {
+                                                 nvfp4_epilogue epi, void *workspace, int32_t *dev_status,
+                                                 cudaStream_t stream) {
   if (epi != NVFP4_EPI_NONE && epi != NVFP4_EPI_SWIGLU) return NVFP4_ERR_INVALID_ARG;
   if (out_dtype != NVFP4_OUT_F32 && out_dtype != NVFP4_OUT_BF16) return NVFP4_ERR_INVALID_ARG;
   const bool swiglu = epi == NVFP4_EPI_SWIGLU;
   const int E = expert_offsets ? num_experts : 1;
-  if (E < 1 || E > kMaxGroups) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (E < 1 || E > w4a16::kMaxExperts) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   if (M_total < 0 || N <= 0 || K <= 0 || ld_x < K || x_rows < 0) return NVFP4_ERR_INVALID_ARG;
   if (!row_index && x_rows < M_total) return NVFP4_ERR_INVALID_ARG;
-  if (K % 64 != 0 || ld_x % 8 != 0 || N % (swiglu ? 64 : 32) != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
-  if ((int64_t)E * N > ((int64_t)1 << 31) - 1 || M_total > ((int64_t)1 << 31) - 1 || N > (1 << 30))
+  if (K % 256 != 0 || ld_x % 8 != 0 || N % 128 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if ((int64_t)E * N > ((int64_t)1 << 31) - 1 || M_total > ((int64_t)1 << 30) || K > (1 << 24))
     return NVFP4_ERR_UNSUPPORTED_SHAPE;
   if (M_total == 0) return NVFP4_OK;
-  if (!x || x_rows == 0 || !b_q || !b_sf || !b_gs || !y) return NVFP4_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(b_q)) & 15u) return NVFP4_ERR_INVALID_ARG;
-  if (reinterpret_cast<uintptr_t>(b_sf) & 1u) return NVFP4_ERR_INVALID_ARG;
+  if (!x || x_rows == 0 || !b_q || !b_sf || !b_gs || !y || !workspace) return NVFP4_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(b_q) | reinterpret_cast<uintptr_t>(b_sf) |
+       reinterpret_cast<uintptr_t>(workspace)) & 15u)
+    return NVFP4_ERR_INVALID_ARG;
+  uint16_t *x16 = reinterpret_cast<uint16_t *>(workspace);
+  float *xscale = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(workspace) + w4a16_x16_bytes(M_total, E, K));
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const size_t sm = sizeof(int32_t) * 2 * (size_t)(E + 1);
-  const int blocks = sms * 8;
-  const uint16_t *xb = reinterpret_cast<const uint16_t *>(x);
-#define NVFP4_W4(S, B)                                                                                      \
-  w4a16::w4a16_kernel<S, B><<<blocks, w4a16::kThreads, sm, stream>>>(xb, ld_x, x_rows, row_index, b_q, b_sf, b_gs, \
-                                                                     expert_offsets, E, M_total, (int)N, (int)K, y, \
-                                                                     dev_status)
-  if (sm > 48 * 1024) return NVFP4_ERR_UNSUPPORTED_SHAPE;
-  const bool bo = out_dtype == NVFP4_OUT_BF16;
-  if (swiglu && bo) NVFP4_W4(true, true);
-  else if (swiglu) NVFP4_W4(true, false);
-  else if (bo) NVFP4_W4(false, true);
-  else NVFP4_W4(false, false);
-#undef NVFP4_W4
+  // prep: the routed rows, as scaled f16 in fragment order
+  {
+    const size_t sm = sizeof(int32_t) * (2 * (size_t)(E + 1) + 8);
+    int64_t grid = (M_total + 7) / 8;
+    if (grid > (int64_t)sms * 8) grid = (int64_t)sms * 8;
+    w4a16::w4a16_prep_kernel<<<(unsigned)grid, 256, sm, stream>>>(
+        reinterpret_cast<const uint16_t *>(x), ld_x, x_rows, row_index, expert_offsets, E, M_total, (int)K, x16, xscale,
+        dev_status);
+    if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_CUDA;
+  }
+  CUtensorMap tw, ts;
+  const uint32_t box_rows = swiglu ? 64 : 128;
+  if (!gemm::make_map(&tw, b_q, (uint64_t)E * N, (uint64_t)K / 2, box_rows)) return NVFP4_ERR_CUDA;
+  if (!make_map_scales16(&ts, b_sf, (uint64_t)E * N, (uint64_t)K / 16, box_rows)) return NVFP4_ERR_CUDA;
+  const int variant = (swiglu ? 2 : 0) + (out_dtype == NVFP4_OUT_BF16 ? 1 : 0);
+  auto kern = variant == 3 ? w4a16::w4a16_kernel<true, true>
+            : variant == 2 ? w4a16::w4a16_kernel<true, false>
+            : variant == 1 ? w4a16::w4a16_kernel<false, true> : w4a16::w4a16_kernel<false, false>;
+  if (!g_w4a16_attr[variant]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, w4a16::SMEM_BYTES) != cudaSuccess)
+      return NVFP4_ERR_CUDA;
+    g_w4a16_attr[variant] = true;
+  }
+  kern<<<sms, w4a16::kThreads, w4a16::SMEM_BYTES, stream>>>(tw, ts, x16, xscale, b_gs, expert_offsets, E, M_total,
+                                                            (int)N, (int)K, y, dev_status);
   return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }

@@ -15,7 +15,7 @@ import torch
 
 from . import (EPI_NONE, EPI_SWIGLU, GS_AMAX_GIVEN, GS_FROM_AMAX, GS_GIVEN, OUT_BF16, OUT_F32, SF_MMA_TILED, SF_ROWMAJOR,
                mxfp4_grouped_gemm as _mxfp4_grouped_gemm, mxfp4_quantize as _mxfp4_quantize, mxfp4_to_nvfp4, nvfp4_dequantize, nvfp4_grouped_gemm, nvfp4_grouped_gemm_swiglu_nvfp4,
-               nvfp4_grouped_gemm_w4a16, nvfp4_moe_combine,
+               nvfp4_grouped_gemm_w4a16, nvfp4_moe_combine, nvfp4_w4a16_workspace_size,
                nvfp4_moe_route,
                nvfp4_moe_quantize, nvfp4_moe_route_workspace_size, nvfp4_padded_rows_bound, nvfp4_quantize,
                nvfp4_swiglu_quantize,
@@ -210,8 +210,12 @@ def grouped_gemm_swiglu_nvfp4(a: Packed, w_gate_up: Packed, N: int, h_gs: torch.
     return p
 
 
+def w4a16_workspace(rows: int, num_groups: int, K: int, device="cuda") -> torch.Tensor:
+    return torch.empty(nvfp4_w4a16_workspace_size(rows, num_groups, K), dtype=torch.uint8, device=device)
+
+
 def grouped_gemm_w4a16(x: torch.Tensor, w: Packed, N: int, row_index=None, offsets=None, num_groups: int = 1,
-                       rows=None, out_dtype=OUT_BF16, swiglu=False, y=None, dev_status=None) -> torch.Tensor:
+                       rows=None, out_dtype=OUT_BF16, swiglu=False, y=None, ws=None, dev_status=None) -> torch.Tensor:
     """Weight-only NVFP4 (row-major scales) x bf16 activations, per expert:
     Y [rows, N] (or h [rows, N/2] with ``swiglu``; gate rows first)."""
     assert x.dtype == torch.bfloat16 and w.layout == SF_ROWMAJOR
@@ -221,8 +225,10 @@ def grouped_gemm_w4a16(x: torch.Tensor, w: Packed, N: int, row_index=None, offse
     cols = N // 2 if swiglu else N
     if y is None:
         y = torch.empty((M, cols), dtype=dt, device=x.device)
+    if ws is None:
+        ws = w4a16_workspace(M, G, w.K, x.device)
     nvfp4_grouped_gemm_w4a16(x, x.stride(0), x.shape[0], row_index, w.q, w.sf, w.gs, offsets, G, M, N, w.K, y,
-                             out_dtype, EPI_SWIGLU if swiglu else EPI_NONE, dev_status)
+                             out_dtype, EPI_SWIGLU if swiglu else EPI_NONE, ws, dev_status)
     return y
 
 

@@ -93,6 +93,12 @@ def test_host_validation_without_device(lib):
     assert L.nvfp4_moe_quantize(fake, 4, 64, 64, fake, 0, fake, 2, 0, fake, fake, fake, 1, fake, None, None) == nv.ERR_INVALID_ARG
     assert L.nvfp4_moe_quantize(fake, 4, 64, 64, fake, 2, None, 2, 0, fake, fake, fake, 1, fake, None, None) == nv.ERR_INVALID_ARG
     assert L.nvfp4_moe_quantize(fake, 4, 48, 48, fake, 2, fake, 2, 0, fake, fake, fake, 1, fake, None, None) == nv.ERR_UNSUPPORTED_SHAPE
+    # W4A16: K % 256, N % 128, a workspace is required
+    ws = fake
+    assert L.nvfp4_grouped_gemm_w4a16(fake, 1088, 8, None, fake, fake, fake, None, 1, 8, 128, 1088, fake, 0, 0, ws, None, None) == nv.ERR_UNSUPPORTED_SHAPE
+    assert L.nvfp4_grouped_gemm_w4a16(fake, 1024, 8, None, fake, fake, fake, None, 1, 8, 96, 1024, fake, 0, 0, ws, None, None) == nv.ERR_UNSUPPORTED_SHAPE
+    assert L.nvfp4_grouped_gemm_w4a16(fake, 1024, 8, None, fake, fake, fake, None, 1, 8, 128, 1024, fake, 0, 0, None, None, None) == nv.ERR_INVALID_ARG
+    assert L.nvfp4_w4a16_workspace_size(640, 384, 7168) >= 640 * 7168 * 2
     # MXFP4 encode: K % 32, K % 128 for tiled scales, aligned pointers, rows == 0 a no-op
     assert L.mxfp4_quantize(fake, 4, 48, 48, fake, fake, 0, None, None) == nv.ERR_UNSUPPORTED_SHAPE
     assert L.mxfp4_quantize(fake, 4, 64, 64, fake, fake, 1, None, None) == nv.ERR_UNSUPPORTED_SHAPE

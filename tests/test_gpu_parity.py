@@ -1147,11 +1147,11 @@ def _w4a16_case(seed, counts, N, K, T):
     return L, x, ri, offsets, wp, y_ref, s_ref
 
 
-@pytest.mark.parametrize("K", [1024, 1088])
+@pytest.mark.parametrize("K", [1024, 1280])
 def test_w4a16_grouped(K):
     """bf16 activations x NVFP4 weights per expert vs fp64 on the exact
     dequantized weights: groups of 0, 1, 3, 9, 17 and 64 tokens (several
-    8-token tiles), K an even and an odd number of 64-element chunks."""
+    8-token chunks), K an even and an odd number of 256-element stages."""
     counts = [0, 1, 3, 9, 17, 64]
     N, T = 256, 40
     L, x, ri, off, wp, y_ref, s_ref = _w4a16_case(30, counts, N, K, T)
@@ -1167,7 +1167,8 @@ def test_w4a16_grouped(K):
 
 def test_w4a16_swiglu_epilogue():
     """h = bf16(silu(g) * u) from the same g, u as the plain kernel's fp32
-    output: within one bf16 ulp of the oracle SwiGLU of that output."""
+    output (each output element sums its K terms in the same order in both
+    variants): within one bf16 ulp of the oracle SwiGLU of that output."""
     counts = [2, 0, 5, 11]
     I, K, T = 128, 2048, 20
     N = 2 * I
@@ -1199,3 +1200,35 @@ def test_w4a16_dense_and_bad_row_index():
     L.grouped_gemm_w4a16(bf16_dev(x), wp, N, to_dev(bad), out_dtype=0, dev_status=s)
     torch.cuda.synchronize()
     assert int(s.item()) == 19
+
+
+def test_w4a16_activation_range():
+    """Rows whose magnitudes sit far from 1 (1e30, 1e-30) and a row spanning
+    about 2^40 of dynamic range: the per-row power-of-two scaling into f16
+    keeps every row within the GEMM tolerance; a row holding an inf is
+    reported as non-finite."""
+    L = layer()
+    M, N, K = 6, 128, 1024
+    z = synthetic.bf16_bits_to_f32(synthetic.gaussian_bf16(33, synthetic.STREAMS["x"], (M, K))).astype(np.float64)
+    z[0] *= 1e30
+    z[1] *= 1e-30
+    z[2] *= np.ldexp(1.0, (np.arange(K) % 41) - 20)             # 2^-20 .. 2^20 across the row
+    z[3, ::7] = 0.0
+    x = synthetic.f32_to_bf16_bits(z.astype(np.float32))
+    w = synthetic.gaussian_bf16(33, synthetic.STREAMS["w"], (N, K), sigma=0.02)
+    qw, sw, gw = _packed_weights(w, 1, N, K)
+    wp = L.Packed(to_dev(qw), to_dev(sw), to_dev(gw), N, K, 0)
+    s = status_word()
+    y = to_np(L.grouped_gemm_w4a16(bf16_dev(x), wp, N, out_dtype=0, dev_status=s))
+    torch.cuda.synchronize()
+    assert int(s.item()) == 0
+    a = synthetic.bf16_bits_to_f32(x).astype(np.float64)
+    b = oracle.dequantize_f64(qw, sw, np.full(N, gw[0], np.float32))
+    y_ref, s_ref = oracle.gemm_f64(a, b)
+    ok, err, bound = gemm_tol(y, y_ref, s_ref)
+    assert ok.all(), (err / bound).max()
+    x[4, 17] = 0x7F80                                            # +inf
+    s = status_word()
+    L.grouped_gemm_w4a16(bf16_dev(x), wp, N, out_dtype=0, dev_status=s)
+    torch.cuda.synchronize()
+    assert int(s.item()) == 16
