@@ -165,18 +165,19 @@ __global__ void __launch_bounds__(256) w4a16_prep_kernel(
 }
 
 // ------------------------------------------------------------------ GEMM
-// Two E2M1 codes (one byte, element 2i in the low nibble) -> f16x2, exact.
-__device__ __forceinline__ uint32_t e2m1x2_f16x2(uint32_t byte) {
-  uint32_t h;
-  asm("{\n.reg .b8 b;\ncvt.u8.u32 b, %1;\ncvt.rn.f16x2.e2m1x2 %0, b;\n}" : "=r"(h) : "r"(byte));
-  return h;
-}
-
 // Two E4M3 bytes (low 16 bits) -> f16x2 (low half = low byte), exact.
 __device__ __forceinline__ uint32_t e4m3x2_f16x2(uint32_t two) {
   uint32_t h;
   asm("{\n.reg .b16 b;\ncvt.u16.u32 b, %1;\ncvt.rn.f16x2.e4m3x2 %0, b;\n}" : "=r"(h) : "r"(two & 0xFFFFu));
   return h;
+}
+
+// The four bytes of a word (8 codes) -> four f16x2 (byte j -> o[j]), exact.
+__device__ __forceinline__ void e2m1x8_f16x2(uint32_t w, uint32_t (&o)[4]) {
+  asm("{\n.reg .b8 b0, b1, b2, b3;\nmov.b32 {b0, b1, b2, b3}, %4;\n"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\ncvt.rn.f16x2.e2m1x2 %1, b1;\n"
+      "cvt.rn.f16x2.e2m1x2 %2, b2;\ncvt.rn.f16x2.e2m1x2 %3, b3;\n}"
+      : "=r"(o[0]), "=r"(o[1]), "=r"(o[2]), "=r"(o[3]) : "r"(w));
 }
 
 __device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
@@ -325,16 +326,16 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_kernel(
         const uint32_t wA[4] = {wa.x, wa.y, wa.z, wa.w};
         const uint32_t wB[4] = {wb.x, wb.y, wb.z, wb.w};
 #pragma unroll
-        for (int s = 0; s < 8; ++s) {
-          // slice 8 half + s: physical K 64t + 4 (8 half + s) .. +3, bytes 2s, 2s+1 of the lane's 16
-          const uint32_t ca = wA[s >> 1] >> (16 * (s & 1)), cb = wB[s >> 1] >> (16 * (s & 1));
-          const uint32_t a0 = hmul2(e2m1x2_f16x2(ca & 0xFFu), sA[s >> 2]);
-          const uint32_t a2 = hmul2(e2m1x2_f16x2((ca >> 8) & 0xFFu), sA[s >> 2]);
-          const uint32_t a1 = hmul2(e2m1x2_f16x2(cb & 0xFFu), sB[s >> 2]);
-          const uint32_t a3 = hmul2(e2m1x2_f16x2((cb >> 8) & 0xFFu), sB[s >> 2]);
-          const uint4 xv = xp[s >> 1];
-          const uint32_t b0 = (s & 1) ? xv.z : xv.x, b1 = (s & 1) ? xv.w : xv.y;
-          mma_f16(d, a0, a1, a2, a3, b0, b1);
+        for (int j = 0; j < 4; ++j) {
+          // word j = slices 8 half + 2j, +1 (physical K 64t + 4 (8 half + 2j) .. +7):
+          // bytes 0, 1 feed the first slice, bytes 2, 3 the second
+          uint32_t fa[4], fb[4];
+          e2m1x8_f16x2(wA[j], fa);
+          e2m1x8_f16x2(wB[j], fb);
+          const uint32_t sa2 = sA[j >> 1], sb2 = sB[j >> 1];
+          const uint4 xv = xp[j];
+          mma_f16(d, hmul2(fa[0], sa2), hmul2(fb[0], sb2), hmul2(fa[1], sa2), hmul2(fb[1], sb2), xv.x, xv.y);
+          mma_f16(d, hmul2(fa[2], sa2), hmul2(fb[2], sb2), hmul2(fa[3], sa2), hmul2(fb[3], sb2), xv.z, xv.w);
         }
       }
       // The second K half hands its partial sums to the first.  Every consumer
