@@ -21,8 +21,9 @@
 //    multiplies by 2^k again, which is exact.
 //  * Pipeline.  One producer warp streams, per 256-element K stage, the
 //    128-row weight tile and its scales by TMA (128-byte swizzle) and the
-//    item's 8 activation rows (4 KB, pre-arranged by the prep kernel in
-//    fragment order) by one bulk copy, into an 8-stage ring of 22 KB stages.
+//    item's activation rows (4 KB per 8 tokens, pre-arranged by the prep
+//    kernel in fragment order) by bulk copies, into a 7-stage ring of 26 KB
+//    stages.
 //    Sixteen consumer warps run mma.sync m16n8k16 (f16 in, fp32 accumulate):
 //    warp w owns weight rows 16 (w%8) .. +16 (x 8 tokens) and the K half w/8
 //    of every stage; the two halves are added through shared memory at the
@@ -32,13 +33,16 @@
 //    [64t, 64t+64) of its rows: MMA slice s takes physical K 64t + 4s + {0..3},
 //    the same on both operands, which leaves the dot products unchanged and
 //    gives each lane two 16-byte weight loads and one scale word per row.
-//  * Work item = (expert, 128-row weight block, chunk of 8 tokens); an expert
-//    with more than 8 tokens re-reads its weight block per chunk, and those
-//    reads follow each other so they hit L2.
+//  * Work item = (expert, 128-row weight block, up to two 8-token chunks):
+//    the converted weight fragments feed one MMA per chunk.  An expert with
+//    more than 16 tokens re-reads its weight block per item, and those reads
+//    follow each other so they hit L2.
 //  * Every mbarrier wait is bounded (NVFP4_ERR_TIMEOUT, then all roles leave).
 #include "gemm_common.cuh"
 
 #include <cuda_fp16.h>
+
+#include <type_traits>
 
 namespace nvfp4 {
 namespace w4a16 {
@@ -51,18 +55,19 @@ using gemm::mbar_try_wait;
 using gemm::mbar_wait;
 using gemm::smem_u32;
 
-constexpr int kTok = 8;                      // tokens per item (MMA N)
+constexpr int kTok = 8;                      // tokens per chunk (MMA N)
+constexpr int kChunks = 2;                   // chunks per item: both share one weight conversion
 constexpr int kConsumers = 16;               // consumer warps: 8 row tiles x 2 K halves
 constexpr int kThreads = (kConsumers + 1) * 32;
-constexpr int kStages = 8;
+constexpr int kStages = 7;
 constexpr int kWBytes = 128 * 128;           // 128 rows x 256 codes
 constexpr int kSBytes = 128 * 16;            // 128 rows x 16 scales
-constexpr int kXBytes = kTok * 256 * 2;      // 8 tokens x 256 f16
-constexpr int kStageBytes = kWBytes + kSBytes + kXBytes;
+constexpr int kXChunk = kTok * 256 * 2;      // 8 tokens x 256 f16
+constexpr int kStageBytes = kWBytes + kSBytes + kChunks * kXChunk;
 constexpr int OFF_BAR = kStages * kStageBytes;
 constexpr int OFF_MISC = OFF_BAR + 2 * kStages * 8;
-constexpr int OFF_RED = OFF_MISC + 16;       // K-half partial sums: 8 warps x 32 lanes x 4 floats
-constexpr int OFF_TABLES = OFF_RED + 8 * 32 * 16;
+constexpr int OFF_RED = OFF_MISC + 16;       // K-half partial sums: 8 warps x 32 lanes x 8 floats
+constexpr int OFF_TABLES = OFF_RED + 8 * 32 * 32;
 constexpr int kMaxExperts = 1024;
 constexpr int TABLE_BYTES = 3 * (kMaxExperts + 1) * 4 + 32 * 4;
 constexpr int SMEM_BYTES = OFF_TABLES + TABLE_BYTES + 1024;
@@ -203,15 +208,19 @@ __device__ __forceinline__ void scales4(uint32_t word, uint32_t (&s)[4]) {
   s[3] = __byte_perm(hi, 0, 0x3232);
 }
 
-struct Item { int e, rb, c; };
+struct Item { int e, rb, c, nc; };      // expert, weight block, first chunk, chunks (1 or 2)
+
+__device__ __forceinline__ int chunks_of(const int32_t *off, int e) { return (off[e + 1] - off[e] + kTok - 1) / kTok; }
+__device__ __forceinline__ int groups_of(const int32_t *off, int e) { return (chunks_of(off, e) + kChunks - 1) / kChunks; }
 
 __device__ __forceinline__ Item decode_item(int64_t it, const int32_t *items, const int32_t *off, int E) {
   Item I;
   I.e = upper_group(items, E, it);
-  const int nch = (off[I.e + 1] - off[I.e] + kTok - 1) / kTok;
+  const int ng = groups_of(off, I.e);
   const int rem = (int)(it - items[I.e]);
-  I.rb = rem / nch;                       // weight block major: the chunks of one block follow each other
-  I.c = rem % nch;
+  I.rb = rem / ng;                        // weight block major: the groups of one block follow each other
+  I.c = (rem % ng) * kChunks;
+  I.nc = min(kChunks, chunks_of(off, I.e) - I.c);
   return I;
 }
 
@@ -246,7 +255,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_kernel(
     off[i] = offsets ? offsets[i] : (i == 0 ? 0 : (int32_t)M_total);
   __syncthreads();
   block_prefix(E, cslot, scratch, [&](int e) { return (off[e + 1] - off[e] + kTok - 1) / kTok; });
-  block_prefix(E, items, scratch, [&](int e) { return row_blocks * ((off[e + 1] - off[e] + kTok - 1) / kTok); });
+  block_prefix(E, items, scratch, [&](int e) { return row_blocks * groups_of(off, e); });
   const int64_t total = items[E];
 
   if (warp == kConsumers) {
@@ -261,12 +270,13 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_kernel(
       for (int64_t it = blockIdx.x; it < total && ok; it += gridDim.x) {
         const Item I = decode_item(it, items, off, E);
         const int64_t C = cslot[I.e] + I.c;
+        const uint32_t bytes = kWBytes + kSBytes + I.nc * kXChunk;
         const int32_t row0 = I.e * N + I.rb * (kSwiglu ? 64 : 128);
         const int32_t uprow0 = row0 + N / 2;
         for (int st = 0; st < nst; ++st) {
           if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1, abort_flag, dev_status)) { ok = false; break; }
           const uint32_t fb = bar_full + 8 * stage;
-          mbar_arrive_expect_tx(fb, kStageBytes);
+          mbar_arrive_expect_tx(fb, bytes);
           armed[stage] = true;
           armed_parity[stage] = phase;
           const uint32_t base = sbase + stage * kStageBytes;
@@ -279,7 +289,8 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_kernel(
             gemm::tma_load_2d(base, &tmap_w, st * 128, row0, fb, pol);
             gemm::tma_load_2d(base + kWBytes, &tmap_s, st * 16, row0, fb, pol);
           }
-          gemm::bulk_load(base + kWBytes + kSBytes, x16 + (C * nst + st) * 2048, kXBytes, fb);
+          for (int cc = 0; cc < I.nc; ++cc)
+            gemm::bulk_load(base + kWBytes + kSBytes + cc * kXChunk, x16 + ((C + cc) * nst + st) * 2048, kXChunk, fb);
           if (++stage == kStages) { stage = 0; phase ^= 1; }
         }
       }
@@ -299,12 +310,15 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_kernel(
     // the lane's 16 code bytes of this half: 16-byte chunk 2t + half of the row (128-byte swizzle)
     const uint32_t offA = rowA * 128 + (((2 * t + half) ^ (rowA & 7)) << 4);
     const uint32_t offB = rowB * 128 + (((2 * t + half) ^ (rowB & 7)) << 4);
-    float *red = reinterpret_cast<float *>(smem + OFF_RED) + (tile * 32 + lane) * 4;
+    float *red = reinterpret_cast<float *>(smem + OFF_RED) + (tile * 32 + lane) * 8;
     int stage = 0;
     uint32_t phase = 0;
     for (int64_t it = blockIdx.x; it < total; it += gridDim.x) {
       const Item I = decode_item(it, items, off, E);
-      float d[4] = {0.f, 0.f, 0.f, 0.f};
+      float d[kChunks][4] = {};
+      // the K loop, compiled once per chunk count (I.nc is warp-uniform)
+      auto kloop = [&](auto nc_tag) {
+      constexpr bool two = decltype(nc_tag)::value == 2;
       for (int st = 0; st < nst; ++st) {
         if (!gemm::mbar_wait_warp(bar_full + 8 * stage, phase, abort_flag, dev_status)) break;
         const uint8_t *base = smem + stage * kStageBytes;
@@ -313,10 +327,13 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_kernel(
         // scales of K blocks 4t + 2 half .. +1 (two bytes of the lane's word)
         const uint32_t sa = *reinterpret_cast<const uint16_t *>(base + kWBytes + rowA * 16 + 4 * t + 2 * half);
         const uint32_t sb = *reinterpret_cast<const uint16_t *>(base + kWBytes + rowB * 16 + 4 * t + 2 * half);
-        uint4 xp[4];
+        const uint8_t *xb = base + kWBytes + kSBytes;
+        uint4 xp[kChunks][4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-          xp[i] = *reinterpret_cast<const uint4 *>(base + kWBytes + kSBytes + ((4 * half + i) * 32 + lane) * 16);
+        for (int i = 0; i < 4; ++i) {
+          xp[0][i] = *reinterpret_cast<const uint4 *>(xb + ((4 * half + i) * 32 + lane) * 16);
+          if constexpr (two) xp[1][i] = *reinterpret_cast<const uint4 *>(xb + kXChunk + ((4 * half + i) * 32 + lane) * 16);
+        }
         __syncwarp();
         if (lane == 0) mbar_arrive(bar_empty + 8 * stage);     // release: the loads above are ordered before it
         if (++stage == kStages) { stage = 0; phase ^= 1; }
@@ -333,50 +350,66 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_kernel(
           e2m1x8_f16x2(wA[j], fa);
           e2m1x8_f16x2(wB[j], fb);
           const uint32_t sa2 = sA[j >> 1], sb2 = sB[j >> 1];
-          const uint4 xv = xp[j];
-          mma_f16(d, hmul2(fa[0], sa2), hmul2(fb[0], sb2), hmul2(fa[1], sa2), hmul2(fb[1], sb2), xv.x, xv.y);
-          mma_f16(d, hmul2(fa[2], sa2), hmul2(fb[2], sb2), hmul2(fa[3], sa2), hmul2(fb[3], sb2), xv.z, xv.w);
+          const uint32_t a0 = hmul2(fa[0], sa2), a1 = hmul2(fb[0], sb2), a2 = hmul2(fa[1], sa2), a3 = hmul2(fb[1], sb2);
+          const uint32_t c0 = hmul2(fa[2], sa2), c1 = hmul2(fb[2], sb2), c2 = hmul2(fa[3], sa2), c3 = hmul2(fb[3], sb2);
+          mma_f16(d[0], a0, a1, a2, a3, xp[0][j].x, xp[0][j].y);
+          mma_f16(d[0], c0, c1, c2, c3, xp[0][j].z, xp[0][j].w);
+          if constexpr (two) {
+            mma_f16(d[1], a0, a1, a2, a3, xp[1][j].x, xp[1][j].y);
+            mma_f16(d[1], c0, c1, c2, c3, xp[1][j].z, xp[1][j].w);
+          }
         }
       }
+      };
+      if (I.nc == 2) kloop(std::integral_constant<int, 2>{});
+      else kloop(std::integral_constant<int, 1>{});
       // The second K half hands its partial sums to the first.  Every consumer
       // warp reaches both barriers of every item it starts (a wait that gave
       // up only ends the stage loop), and the decision to stop is read from
       // one shared word after the second barrier, so all warps leave together.
-      if (half == 1) *reinterpret_cast<float4 *>(red) = make_float4(d[0], d[1], d[2], d[3]);
+      if (half == 1) {
+        reinterpret_cast<float4 *>(red)[0] = make_float4(d[0][0], d[0][1], d[0][2], d[0][3]);
+        reinterpret_cast<float4 *>(red)[1] = make_float4(d[1][0], d[1][1], d[1][2], d[1][3]);
+      }
       asm volatile("bar.sync 1, %0;" :: "n"(kConsumers * 32) : "memory");
       if (half == 0) {
-        const float4 p = *reinterpret_cast<const float4 *>(red);
-        d[0] += p.x; d[1] += p.y; d[2] += p.z; d[3] += p.w;
+        const float4 p0 = reinterpret_cast<const float4 *>(red)[0], p1 = reinterpret_cast<const float4 *>(red)[1];
+        d[0][0] += p0.x; d[0][1] += p0.y; d[0][2] += p0.z; d[0][3] += p0.w;
+        d[1][0] += p1.x; d[1][1] += p1.y; d[1][2] += p1.z; d[1][3] += p1.w;
       }
       if (warp == 0 && lane == 0) *stop_word = *abort_flag;
       asm volatile("bar.sync 1, %0;" :: "n"(kConsumers * 32) : "memory");
       if (*stop_word) break;
       if (half == 1) continue;
-      // d[0], d[1]: row A, tokens 2t, 2t+1; d[2], d[3]: row B
-      const int32_t r0 = off[I.e] + I.c * kTok;
-      const int ntok = min(kTok, off[I.e + 1] - r0);
-      const int64_t C = cslot[I.e] + I.c;
+      // per chunk: d[cc][0], d[cc][1]: row A, tokens 2t, 2t+1; d[cc][2], d[cc][3]: row B
       const float gs = w_gs[I.e];
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const int tok = 2 * t + j;
-        if (tok >= ntok) continue;
-        const float xs = xscale[C * kTok + tok];
-        const float va = __fmul_rn(__fmul_rn(d[j], gs), xs);
-        const float vb = __fmul_rn(__fmul_rn(d[2 + j], gs), xs);
-        if constexpr (kSwiglu) {
-          const float h = __fmul_rn(__fdividef(va, 1.0f + __expf(-va)), vb);
-          const int64_t o = (int64_t)(r0 + tok) * rows_out + I.rb * 64 + 8 * tile + g;
-          if (kBf16Out) reinterpret_cast<__nv_bfloat16 *>(y)[o] = __float2bfloat16_rn(h);
-          else reinterpret_cast<float *>(y)[o] = h;
-        } else {
-          const int64_t o = (int64_t)(r0 + tok) * rows_out + I.rb * 128 + 16 * tile + g;
-          if (kBf16Out) {
-            reinterpret_cast<__nv_bfloat16 *>(y)[o] = __float2bfloat16_rn(va);
-            reinterpret_cast<__nv_bfloat16 *>(y)[o + 8] = __float2bfloat16_rn(vb);
+      for (int cc = 0; cc < kChunks; ++cc) {
+        if (cc >= I.nc) break;
+        const int32_t r0 = off[I.e] + (I.c + cc) * kTok;
+        const int ntok = min(kTok, off[I.e + 1] - r0);
+        const int64_t C = cslot[I.e] + I.c + cc;
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int tok = 2 * t + j;
+          if (tok >= ntok) continue;
+          const float xs = xscale[C * kTok + tok];
+          const float va = __fmul_rn(__fmul_rn(d[cc][j], gs), xs);
+          const float vb = __fmul_rn(__fmul_rn(d[cc][2 + j], gs), xs);
+          if constexpr (kSwiglu) {
+            const float h = __fmul_rn(__fdividef(va, 1.0f + __expf(-va)), vb);
+            const int64_t o = (int64_t)(r0 + tok) * rows_out + I.rb * 64 + 8 * tile + g;
+            if (kBf16Out) reinterpret_cast<__nv_bfloat16 *>(y)[o] = __float2bfloat16_rn(h);
+            else reinterpret_cast<float *>(y)[o] = h;
           } else {
-            reinterpret_cast<float *>(y)[o] = va;
-            reinterpret_cast<float *>(y)[o + 8] = vb;
+            const int64_t o = (int64_t)(r0 + tok) * rows_out + I.rb * 128 + 16 * tile + g;
+            if (kBf16Out) {
+              reinterpret_cast<__nv_bfloat16 *>(y)[o] = __float2bfloat16_rn(va);
+              reinterpret_cast<__nv_bfloat16 *>(y)[o + 8] = __float2bfloat16_rn(vb);
+            } else {
+              reinterpret_cast<float *>(y)[o] = va;
+              reinterpret_cast<float *>(y)[o + 8] = vb;
+            }
           }
         }
       }
