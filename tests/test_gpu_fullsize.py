@@ -1,0 +1,329 @@
+"""Parity at the benchmark configurations' full sizes (GPU, through the C ABI).
+
+The GPU runs each configuration whole, in the launch configuration the bench
+times; the oracle recomputes what it can in seconds:
+- GEMMs: every output row of a strided sample of experts (every 16th or 8th,
+  plus the largest, the smallest and the last group), or every token against
+  a sample of weight rows, in fp64 on the oracle's own quantization of the
+  same seeded inputs, within |y - y_ref| <= 1e-5 * sum|a*b| + 1e-6;
+- quantize, KV cache, remap: every byte.
+
+All oracle inputs are regenerated on the host from the seeded generators
+(counter-based, so any slice of a device tensor can be regenerated alone);
+nothing the CUDA path computes is fed to the oracle.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import synthetic
+from tests._util import bf16_dev, slot_rows, to_dev, to_np, untile
+
+torch = pytest.importorskip("torch")
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not torch.cuda.is_available(), reason="no CUDA device")]
+
+
+def layer():
+    from nvfp4_w4a4_quantized_04_b200 import layer as L
+    return L
+
+
+def nvmod():
+    import nvfp4_w4a4_quantized_04_b200 as nv
+    return nv
+
+
+def status_word():
+    return torch.zeros(1, dtype=torch.int32, device="cuda")
+
+
+def gemm_tol(y, y_ref, s_ref):
+    err = np.abs(y.astype(np.float64) - y_ref)
+    bound = 1e-5 * s_ref + 1e-6
+    return err <= bound, err, bound
+
+
+def tiled_rows_host(sf_flat, row0, nrows, K):
+    """Row-major scales of rows [row0, row0 + nrows) of a tensor-core-tiled
+    scale tensor already on the host (row0 a multiple of 128)."""
+    nsf = K // 16
+    per_block = (nsf // 4) * 512
+    b0, nb = row0 // 128, (nrows + 127) // 128
+    return untile(sf_flat.reshape(-1)[b0 * per_block:(b0 + nb) * per_block], nb * 128, nsf)[:nrows]
+
+
+def tiled_rows(sf_dev, row0, nrows, K):
+    """Row-major scales of rows [row0, row0 + nrows) of a tensor-core-tiled scale
+    tensor (row0 and nrows multiples of 128), copied from the device."""
+    nsf = K // 16
+    per_block = (nsf // 4) * 512
+    b0, nb = row0 // 128, (nrows + 127) // 128
+    flat = to_np(sf_dev.reshape(-1)[b0 * per_block:(b0 + nb) * per_block])
+    return untile(flat, nb * 128, nsf)[:nrows]
+
+
+def sample_experts(counts, stride, seed):
+    """Every stride-th non-empty expert from a seeded offset, plus the largest,
+    the smallest and the last non-empty group."""
+    nz = np.nonzero(counts)[0]
+    j = int(np.random.default_rng(seed).integers(stride))
+    pick = {int(e) for e in nz[j::stride]}
+    pick.update((int(np.argmax(counts)), int(nz[np.argmin(counts[nz])]), int(nz[-1])))
+    return sorted(pick)
+
+
+def check_expert_gemm(x_rows_bits, w_bits, a_gpu, w_gpu, y_gpu_rows, a_gs, w_gs):
+    """Oracle-quantize both operands of one expert, check the GPU's packed bytes
+    against them, then the GPU's fp32 output rows against the fp64 product."""
+    qa, sfa, gsa, st = oracle.quantize(x_rows_bits)
+    assert st == 0
+    qw, sfw, gsw, st = oracle.quantize(w_bits)
+    assert st == 0
+    assert np.array_equal(a_gpu[0], qa) and np.array_equal(a_gpu[1], sfa) and a_gs == gsa[0]
+    assert np.array_equal(w_gpu[0], qw) and np.array_equal(w_gpu[1], sfw) and w_gs == gsw[0]
+    a = oracle.dequantize_f64(qa, sfa, np.full(qa.shape[0], gsa[0], np.float32))
+    b = oracle.dequantize_f64(qw, sfw, np.full(qw.shape[0], gsw[0], np.float32))
+    y_ref, s_ref = oracle.gemm_f64(a, b)
+    ok, err, bound = gemm_tol(y_gpu_rows, y_ref, s_ref)
+    assert ok.all(), (err.max(), (err / bound).max())
+
+
+def test_config3_moe_gemms_full_size():
+    """512 experts, top-10 of 8192 tokens, H 4096, I 1024: the dispatch quantize
+    and both grouped GEMMs run whole; a strided sample of experts (one in 16)
+    is checked, bytes and rows."""
+    import synthetic.cuda as sc
+    L = layer()
+    E, T, H, I, k = 512, 8192, 4096, 1024, 10
+    r = synthetic.route_topk_softmax(0, T, E, k)
+    off = r["offsets"].astype(np.int64)
+    R = int(off[-1])
+    counts = np.diff(off)
+    _, starts = slot_rows(off)
+    ws = L.workspace(E, "cuda")
+    offd = to_dev(r["offsets"])
+    s = status_word()
+    # gate_up: token-order dispatch quantize, then the grouped GEMM (fp32 out)
+    x = sc.gaussian_bf16(0, synthetic.STREAMS["x"], (T, H))
+    w = sc.gaussian_bf16(0, synthetic.STREAMS["w_gate_up"], (E * 2 * I, H), sigma=0.02)
+    wp = L.pack_weights(w, E, 2 * I, None, ws)
+    del w
+    a1 = L.moe_quantize(x, to_dev(r["slot"].astype(np.int32)), offd, E, layout=1, ws=ws, rows=R, dev_status=s)
+    y1 = L.grouped_gemm(a1, wp, 2 * I, 0, dev_status=s)
+    # down: an independent seeded h [R, I] in routed order
+    h = sc.gaussian_bf16(1, synthetic.STREAMS["x"], (R, I))
+    wd = sc.gaussian_bf16(0, synthetic.STREAMS["w_down"], (E * H, I), sigma=0.02)
+    wdp = L.pack_weights(wd, E, H, None, ws)
+    del wd
+    a2 = L.quantize(h, None, offd, E, layout=1, ws=ws, dev_status=s)
+    y2 = L.grouped_gemm(a2, wdp, H, 0, dev_status=s)
+    torch.cuda.synchronize()
+    assert int(s.item()) == 0
+    xh = synthetic.gaussian_bf16(0, synthetic.STREAMS["x"], (T, H))
+    # device results to the host once
+    a1q, a1s, a1g = to_np(a1.q), to_np(a1.sf), to_np(a1.gs)
+    a2q, a2s, a2g = to_np(a2.q), to_np(a2.sf), to_np(a2.gs)
+    y1h, y2h = to_np(y1), to_np(y2)
+    wq, wsf, wg = to_np(wp.q), to_np(wp.sf), to_np(wp.gs)
+    wdq, wdsf, wdg = to_np(wdp.q), to_np(wdp.sf), to_np(wdp.gs)
+    for e in sample_experts(counts, 16, 3):
+        m, r0, p0 = int(counts[e]), int(off[e]), int(starts[e])
+        rows = r["row_index"][r0:r0 + m]
+        # gate_up
+        a_gpu = (a1q[p0:p0 + m], tiled_rows_host(a1s, p0, m, H))
+        w_gpu = (wq[e * 2 * I:(e + 1) * 2 * I], tiled_rows_host(wsf, e * 2 * I, 2 * I, H))
+        wbits = synthetic.gaussian_bf16(0, synthetic.STREAMS["w_gate_up"], (2 * I, H), sigma=0.02, start=e * 2 * I * H)
+        check_expert_gemm(xh[rows], wbits, a_gpu, w_gpu, y1h[r0:r0 + m], a1g[e], wg[e])
+        # down
+        hbits = synthetic.gaussian_bf16(1, synthetic.STREAMS["x"], (m, I), start=r0 * I)
+        a_gpu = (a2q[p0:p0 + m], tiled_rows_host(a2s, p0, m, I))
+        w_gpu = (wdq[e * H:(e + 1) * H], tiled_rows_host(wdsf, e * H, H, I))
+        wbits = synthetic.gaussian_bf16(0, synthetic.STREAMS["w_down"], (H, I), sigma=0.02, start=e * H * I)
+        check_expert_gemm(hbits, wbits, a_gpu, w_gpu, y2h[r0:r0 + m], a2g[e], wdg[e])
+
+
+def test_config4_decode_full_size():
+    """384 experts, 64 tokens, top-10 Zipf routing, H 7168, I 2048, weights
+    generated as MXFP4 and remapped on the device: the remap and both grouped
+    GEMMs run whole; one touched expert in 8 is checked (remap bytes, then GEMM
+    rows), and four untouched experts' remap bytes."""
+    import synthetic.cuda as sc
+    L = layer()
+    nv = nvmod()
+    E, T, H, I, k = 384, 64, 7168, 2048, 10
+    r = synthetic.route_zipf_gumbel(7, T, E, k)
+    off = r["offsets"].astype(np.int64)
+    R = int(off[-1])
+    counts = np.diff(off)
+    _, starts = slot_rows(off)
+    ws = L.workspace(E, "cuda")
+    offd = to_dev(r["offsets"])
+    s = status_word()
+    packs = []
+    for name, rows_per, K in (("gate_up", 2 * I, H), ("down", H, I)):
+        n = E * rows_per * K
+        q = sc.mxfp4_codes(7, synthetic.STREAMS["mx_codes_" + name], n // 2).view(E * rows_per, K // 2)
+        e8 = sc.mxfp4_exponents(7, synthetic.STREAMS["mx_exp_" + name], n // 32, lo=-10)
+        qn = torch.empty_like(q)
+        sf = torch.empty(n // 16, dtype=torch.uint8, device="cuda")
+        gs = torch.empty(E, dtype=torch.float32, device="cuda")
+        nv.mxfp4_to_nvfp4(q, e8, E, rows_per, K, qn, sf, 1, gs, ws, s)
+        del q, e8
+        packs.append(L.Packed(qn, sf, gs, E * rows_per, K, 1))
+    x = sc.gaussian_bf16(7, synthetic.STREAMS["x"], (T, H))
+    a1 = L.moe_quantize(x, to_dev(r["slot"].astype(np.int32)), offd, E, layout=1, ws=ws, rows=R, dev_status=s)
+    y1 = L.grouped_gemm(a1, packs[0], 2 * I, 0, dev_status=s)
+    h = sc.gaussian_bf16(8, synthetic.STREAMS["x"], (R, I))
+    a2 = L.quantize(h, None, offd, E, layout=1, ws=ws, dev_status=s)
+    y2 = L.grouped_gemm(a2, packs[1], H, 0, dev_status=s)
+    torch.cuda.synchronize()
+    assert int(s.item()) == 0
+    xh = synthetic.gaussian_bf16(7, synthetic.STREAMS["x"], (T, H))
+    untouched = [int(e) for e in np.nonzero(counts == 0)[0][:4]]
+    for e in sample_experts(counts, 8, 4) + untouched:
+        m, r0, p0 = int(counts[e]), int(off[e]), int(starts[e])
+        for proj, (rows_per, K, a, y, gpu_w) in enumerate(((2 * I, H, a1, y1, packs[0]), (H, I, a2, y2, packs[1]))):
+            name = ("gate_up", "down")[proj]
+            nb = rows_per * K // 2
+            qm = synthetic.mxfp4_codes(7, synthetic.STREAMS["mx_codes_" + name], nb, start_byte=e * nb).reshape(rows_per, K // 2)
+            em = synthetic.mxfp4_exponents(7, synthetic.STREAMS["mx_exp_" + name], rows_per * K // 32, lo=-10,
+                                           start=e * rows_per * K // 32).reshape(rows_per, K // 32)
+            qn, sfn, gsn, st = oracle.remap_mxfp4(qm, em, 1, rows_per, K)
+            assert st == 0
+            assert np.array_equal(to_np(gpu_w.q[e * rows_per:(e + 1) * rows_per]), qn)
+            assert np.array_equal(tiled_rows(gpu_w.sf, e * rows_per, rows_per, K), sfn)
+            assert to_np(gpu_w.gs)[e] == gsn[0]
+            if m == 0:
+                continue
+            if proj == 0:
+                xr = xh[r["row_index"][r0:r0 + m]]
+            else:
+                xr = synthetic.gaussian_bf16(8, synthetic.STREAMS["x"], (m, I), start=r0 * I)
+            qa, sfa, gsa, st = oracle.quantize(xr)
+            assert st == 0
+            assert np.array_equal(to_np(a.q[p0:p0 + m]), qa) and np.array_equal(tiled_rows(a.sf, p0, m, K), sfa)
+            assert to_np(a.gs)[e] == gsa[0]
+            y_ref, s_ref = oracle.gemm_f64(oracle.dequantize_f64(qa, sfa, np.full(m, gsa[0], np.float32)),
+                                           oracle.dequantize_f64(qn, sfn, np.full(rows_per, gsn[0], np.float32)))
+            ok, err, bound = gemm_tol(to_np(y[r0:r0 + m]), y_ref, s_ref)
+            assert ok.all(), (name, e, err.max(), (err / bound).max())
+
+
+def test_config5_kv_cache_full_size_bitexact():
+    """K and V [262144 tokens x 4 heads, 256] (2^28 elements each): K with the
+    global from its amax, V with a given (static) global; every code and scale
+    byte, the globals and the bf16 dequantized values are compared."""
+    import synthetic.cuda as sc
+    L = layer()
+    nv = nvmod()
+    T, Hh, D = 262144, 4, 256
+    rows = T * Hh
+    kd = sc.gaussian_bf16(0, synthetic.STREAMS["kv_k"], (rows, D))
+    vd = sc.gaussian_bf16(0, synthetic.STREAMS["kv_v"], (rows, D))
+    kq = torch.empty((rows, D // 2), dtype=torch.uint8, device="cuda")
+    vq = torch.empty_like(kq)
+    ks = torch.empty(rows * D // 16, dtype=torch.uint8, device="cuda")
+    vs = torch.empty_like(ks)
+    kgs = torch.empty(1, dtype=torch.float32, device="cuda")
+    vgs = torch.tensor([0.0019], dtype=torch.float32, device="cuda")
+    s = status_word()
+    # K: global from the amax; V: a given global
+    nv.nvfp4_quantize(kd, rows, D, D, None, None, 1, 0, kgs, kq, ks, 0, L.workspace(1), s)
+    nv.nvfp4_quantize(vd, rows, D, D, None, None, 1, 1, vgs, vq, vs, 0, L.workspace(1), s)
+    ko = torch.empty((rows, D), dtype=torch.bfloat16, device="cuda")
+    vo = torch.empty_like(ko)
+    nv.nvfp4_kv_dequantize(kq, ks, kgs, vq, vs, vgs, T, Hh, D, ko, vo)
+    torch.cuda.synchronize()
+    assert int(s.item()) == 0
+    for stream, given, qg, sg, gg, og in ((synthetic.STREAMS["kv_k"], None, kq, ks, kgs, ko),
+                                          (synthetic.STREAMS["kv_v"], np.float32(0.0019), vq, vs, vgs, vo)):
+        xh = synthetic.gaussian_bf16(0, stream, (rows, D))
+        qr, sr, gr, st = oracle.quantize(xh, global_scale=None if given is None else np.array([given], np.float32))
+        assert st == 0
+        assert to_np(gg)[0] == gr[0]
+        assert np.array_equal(to_np(qg), qr)
+        assert np.array_equal(to_np(sg).reshape(rows, D // 16), sr)
+        ref = oracle.dequantize(qr, sr, np.full(rows, gr[0], np.float32), out="bf16")
+        assert np.array_equal(to_np(og), ref)
+        del xh, qr, sr, ref
+
+
+def test_config5_activation_quantize_full_size_bitexact():
+    """The largest activation sweep point, [131072, 5120] bf16 (671 M elements),
+    dynamic global, tensor-core scale layout: every byte and the global."""
+    import synthetic.cuda as sc
+    L = layer()
+    T, H = 131072, 5120
+    xd = sc.gaussian_bf16(0, synthetic.STREAMS["x_sweep"], (T, H))
+    s = status_word()
+    p = L.quantize(xd, layout=1, dev_status=s)
+    torch.cuda.synchronize()
+    assert int(s.item()) == 0
+    del xd
+    xh = synthetic.gaussian_bf16(0, synthetic.STREAMS["x_sweep"], (T, H))
+    qr, sr, gr, st = oracle.quantize(xh)
+    assert st == 0
+    del xh
+    assert to_np(p.gs)[0] == gr[0]
+    assert np.array_equal(to_np(p.q[:T]), qr)
+    assert np.array_equal(tiled_rows(p.sf, 0, T, H), sr)
+
+
+def test_config5_remap_full_size_bitexact():
+    """2^28 MXFP4 elements as 1024 tensors [512, 512], remapped to NVFP4 with
+    tensor-core scales: codes, scale bytes and the 1024 globals."""
+    import synthetic.cuda as sc
+    L = layer()
+    nt, rows, K = 1024, 512, 512
+    n = nt * rows * K
+    q = sc.mxfp4_codes(0, synthetic.STREAMS["mx_codes"], n // 2).view(nt * rows, K // 2)
+    e8 = sc.mxfp4_exponents(0, synthetic.STREAMS["mx_exp"], n // 32)
+    s = status_word()
+    p = L.remap_mxfp4(q, e8, nt, rows, K, layout=1, dev_status=s)
+    torch.cuda.synchronize()
+    assert int(s.item()) == 0
+    qh = synthetic.mxfp4_codes(0, synthetic.STREAMS["mx_codes"], n // 2).reshape(nt * rows, K // 2)
+    eh = synthetic.mxfp4_exponents(0, synthetic.STREAMS["mx_exp"], n // 32).reshape(nt * rows, K // 32)
+    qn, sfn, gsn, st = oracle.remap_mxfp4(qh, eh, nt, rows, K)
+    assert st == 0
+    assert np.array_equal(to_np(p.q), qn)
+    assert np.array_equal(to_np(p.gs), gsn)
+    assert np.array_equal(tiled_rows(p.sf, 0, nt * rows, K), sfn)
+
+
+def test_config2_dense_mlp_full_size_sampled_columns():
+    """Dense MLP, 4096 tokens, hidden 5120, intermediate 17408, X with 0.1 %
+    outliers x50: the activation quantize in full; both GEMMs run whole and
+    every token is checked against a seeded sample of 256 weight rows."""
+    import synthetic.cuda as sc
+    L = layer()
+    M, H, I = 4096, 5120, 17408
+    ws = L.workspace(1, "cuda")
+    s = status_word()
+    wgu = L.pack_weights(sc.gaussian_bf16(0, synthetic.STREAMS["w_gate_up"], (2 * I, H), sigma=0.02), 1, 2 * I, None, ws)
+    wd = L.pack_weights(sc.gaussian_bf16(0, synthetic.STREAMS["w_down"], (H, I), sigma=0.02), 1, H, None, ws)
+    xb = synthetic.gaussian_bf16(0, synthetic.STREAMS["x"], (M, H), outlier_frac=0.001)
+    a1 = L.quantize(bf16_dev(xb), layout=1, ws=ws, dev_status=s)
+    y1 = L.grouped_gemm(a1, wgu, 2 * I, 0, dev_status=s)
+    hb = synthetic.gaussian_bf16(2, synthetic.STREAMS["x"], (M, I))
+    a2 = L.quantize(bf16_dev(hb), layout=1, ws=ws, dev_status=s)
+    y2 = L.grouped_gemm(a2, wd, H, 0, dev_status=s)
+    torch.cuda.synchronize()
+    assert int(s.item()) == 0
+    rng = np.random.default_rng(11)
+    for (abits, a, w, N, K, stream, y) in ((xb, a1, wgu, 2 * I, H, "w_gate_up", y1), (hb, a2, wd, H, I, "w_down", y2)):
+        qa, sfa, gsa, st = oracle.quantize(abits)
+        assert st == 0
+        assert np.array_equal(to_np(a.q[:M]), qa) and np.array_equal(tiled_rows(a.sf, 0, M, K), sfa)
+        assert to_np(a.gs)[0] == gsa[0]
+        wbits = synthetic.gaussian_bf16(0, synthetic.STREAMS[stream], (N, K), sigma=0.02)
+        qw, sfw, gsw, st = oracle.quantize(wbits)
+        assert st == 0 and to_np(w.gs)[0] == gsw[0]
+        cols = np.sort(rng.choice(N, 256, replace=False))
+        assert np.array_equal(to_np(w.q[torch.from_numpy(cols).cuda()]), qw[cols])
+        aref = oracle.dequantize_f64(qa, sfa, np.full(M, gsa[0], np.float32))
+        bref = oracle.dequantize_f64(qw[cols], sfw[cols], np.full(len(cols), gsw[0], np.float32))
+        y_ref, s_ref = oracle.gemm_f64(aref, bref)
+        ok, err, bound = gemm_tol(to_np(y[:, torch.from_numpy(cols).cuda()]), y_ref, s_ref)
+        assert ok.all(), (stream, err.max(), (err / bound).max())
