@@ -119,24 +119,30 @@ __global__ void __launch_bounds__(256) amax_flat_kernel(const uint4 *__restrict_
 }
 
 // Global scales from the amax (FROM_AMAX; AMAX_GIVEN reads the amax from gs
-// itself) or a check of the given ones (GIVEN).
-__global__ void finalize_scales_kernel(const uint32_t *__restrict__ amax_bits, int G, int mode,
-                                       float *__restrict__ gs, int32_t *dev_status) {
-  int g = blockIdx.x * blockDim.x + threadIdx.x;
-  if (g >= G) return;
+// itself) or a check of the given ones (GIVEN).  Returns the group's s_g.
+__device__ __forceinline__ float finalize_one(const uint32_t *__restrict__ amax_bits, int g, int mode, float *gs,
+                                              int32_t *dev_status) {
   if (mode == NVFP4_GS_GIVEN) {
-    float s = gs[g];
+    const float s = gs[g];
     if (!(s > 0.0f) || !isfinite(s)) report(dev_status, NVFP4_ERR_INVALID_ARG);
-    return;
+    return s;
   }
-  uint32_t b = mode == NVFP4_GS_AMAX_GIVEN ? (__float_as_uint(gs[g]) & 0x7FFFFFFFu) : amax_bits[g];
+  const uint32_t b = mode == NVFP4_GS_AMAX_GIVEN ? (__float_as_uint(gs[g]) & 0x7FFFFFFFu) : amax_bits[g];
   if (b >= 0x7F800000u) {
     gs[g] = __uint_as_float(0x7FC00000u);
     report(dev_status, NVFP4_ERR_NONFINITE);
-    return;
+    return __uint_as_float(0x7FC00000u);
   }
-  float a = __uint_as_float(b);
-  gs[g] = (a == 0.0f) ? 1.0f : __fdiv_rn(a, 2688.0f);   // 2688 = 6 * 448
+  const float a = __uint_as_float(b);
+  const float s = (a == 0.0f) ? 1.0f : __fdiv_rn(a, 2688.0f);   // 2688 = 6 * 448
+  gs[g] = s;
+  return s;
+}
+
+__global__ void finalize_scales_kernel(const uint32_t *__restrict__ amax_bits, int G, int mode,
+                                       float *__restrict__ gs, int32_t *dev_status) {
+  const int g = blockIdx.x * blockDim.x + threadIdx.x;
+  if (g < G) finalize_one(amax_bits, g, mode, gs, dev_status);
 }
 
 // ---------------------------------------------------------------- pass 2: encode
@@ -395,55 +401,77 @@ __global__ void __launch_bounds__(256) quantize_kernel(
 // slot[t*k + c] is the routed row of the token's c-th choice (-1: not routed);
 // a lane per choice holds its expert's packed row and global scale.
 
-// Pass 1: each warp takes a token, forms max|x| of the row (up to 8 32-byte
-// loads in flight per lane), and raises the amax of every expert the token is
-// routed to.
-__global__ void __launch_bounds__(256) moe_amax_kernel(
+// Pass 1: the rows are cut into 1024-element pieces, one per warp, eight
+// consecutive pieces per CTA (a CTA covers one or more whole tokens when a row
+// holds 1, 2, 4 or 8 pieces).  Each lane keeps two 32-byte loads in flight;
+// the warp's max|x| goes to shared memory, and after one barrier a thread per
+// (token, choice) pair of the CTA raises the expert's amax.  A token whose
+// pieces straddle two CTAs is raised by both, which atomicMax makes harmless.
+// CTAs are short and not persistent, so the last wave is small.
+constexpr int kAmaxWarps = 8;
+
+__global__ void __launch_bounds__(kAmaxWarps * 32) moe_amax_kernel(
     const uint16_t *__restrict__ x, int64_t ld_x, int64_t K, int64_t tokens, const int32_t *__restrict__ slot,
     int topk, const int32_t *__restrict__ group_offsets, int G, uint32_t *__restrict__ amax_bits,
     int32_t *dev_status) {
   extern __shared__ int32_t smem[];
   int32_t *off = smem;
+  __shared__ uint32_t piece_max[kAmaxWarps];
   for (int i = threadIdx.x; i <= G; i += blockDim.x) off[i] = group_offsets[i];
-  __syncthreads();
-  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t nblk = (uint32_t)(K >> 4);
+  const int64_t pieces = (nblk + 63) >> 6;                 // 64 blocks of 16 per piece
   const bool v8 = ((reinterpret_cast<uintptr_t>(x) & 31u) == 0) && ((ld_x & 15) == 0);
-  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-  constexpr int B = 8;
-  for (int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < tokens; t += nwarps) {
+  const int64_t u0 = (int64_t)blockIdx.x * kAmaxWarps;     // first piece of the CTA
+  const int64_t u = u0 + warp;
+  uint32_t m = 0;
+  if (u < tokens * pieces) {
+    const int64_t t = u / pieces;
+    const uint32_t j0 = (uint32_t)(u - t * pieces) << 6;
     const uint16_t *row = x + t * ld_x;
-    uint32_t m = 0;
-    for (uint32_t j0 = 0; j0 < nblk; j0 += 32 * B) {
-      uint4 va[B], vb[B];
+    uint4 va[2], vb[2];
 #pragma unroll
-      for (int k = 0; k < B; ++k) {
-        const uint32_t j = j0 + k * 32 + lane;
-        va[k] = make_uint4(0, 0, 0, 0);
-        vb[k] = make_uint4(0, 0, 0, 0);
-        if (j < nblk) load_block(row + (uint64_t)j * 16, v8, va[k], vb[k]);
-      }
+    for (int k = 0; k < 2; ++k) {
+      const uint32_t j = j0 + k * 32 + lane;
+      va[k] = make_uint4(0, 0, 0, 0);
+      vb[k] = make_uint4(0, 0, 0, 0);
+      if (j < nblk) load_block(row + (uint64_t)j * 16, v8, va[k], vb[k]);
+    }
 #pragma unroll
-      for (int k = 0; k < B; ++k) m = absmax8_bits(vb[k], absmax8_bits(va[k], m));
-    }
-    const uint32_t mm = warp_max(halves_max(m));
-    if (lane < topk) {
-      const int32_t r = slot[t * topk + lane];
-      if (r >= off[G]) report(dev_status, NVFP4_ERR_INDEX);
-      else if (r >= 0 && mm) atomicMax(&amax_bits[upper_group(off, G, r)], mm << 16);
-    }
+    for (int k = 0; k < 2; ++k) m = absmax8_bits(vb[k], absmax8_bits(va[k], m));
   }
+  m = warp_max(halves_max(m));
+  if (lane == 0) piece_max[warp] = m;
+  __syncthreads();
+  // tokens touched by this CTA: t_first .. t_last
+  const int64_t u_last = min(u0 + kAmaxWarps, tokens * pieces) - 1;
+  if (u_last < u0) return;
+  const int64_t t_first = u0 / pieces, t_last = u_last / pieces;
+  const int64_t i = threadIdx.x / topk, c = threadIdx.x - i * topk;
+  if (t_first + i > t_last) return;
+  const int64_t t = t_first + i;
+  // max over this CTA's pieces of token t
+  const int64_t a = max(t * pieces, u0) - u0, b = min((t + 1) * pieces, u_last + 1) - u0;
+  uint32_t mm = 0;
+  for (int64_t w = a; w < b; ++w) mm = max(mm, piece_max[w]);
+  const int32_t r = slot[t * topk + c];
+  if (r >= off[G]) report(dev_status, NVFP4_ERR_INDEX);
+  else if (r >= 0 && mm) atomicMax(&amax_bits[upper_group(off, G, r)], mm << 16);
 }
 
 // Per-group constants of the dispatch encode, computed once per call with the
 // same IEEE operations the per-block path would use: rtab[g][S] = 1/(S*s_g)
 // (0 when that product is 0) for every E4M3 byte S < 128, and
-// ytab[g] = RN(1/(6*s_g)).
-__global__ void encode_tables_kernel(const float *__restrict__ gs, float *__restrict__ rtab,
-                                     float *__restrict__ ytab) {
+// ytab[g] = RN(1/(6*s_g)).  One block per group; thread 0 first settles the
+// group's s_g (finalize_one), which the block then reads from shared memory.
+__global__ void finalize_tables_kernel(const uint32_t *__restrict__ amax_bits, int mode, float *gs,
+                                       float *__restrict__ rtab, float *__restrict__ ytab, int32_t *dev_status) {
+  __shared__ float s_sg;
   const int g = blockIdx.x;
   const uint32_t S = threadIdx.x;
-  const float s_g = gs[g];
+  if (S == 0) s_sg = finalize_one(amax_bits, g, mode, gs, dev_status);
+  __syncthreads();
+  const float s_g = s_sg;
   const float e = __fmul_rn(e4m3_to_f32_hw(S), s_g);
   rtab[g * 128 + S] = (e == 0.0f) ? 0.0f : __frcp_rn(e);
   if (S == 0) ytab[g] = __frcp_rn(__fmul_rn(6.0f, s_g));
@@ -894,23 +922,23 @@ nvfp4_status nvfp4_moe_quantize(const void *x, int64_t tokens, int64_t K, int64_
   if (tokens * topk > ((int64_t)1 << 31)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   const uint16_t *xb = reinterpret_cast<const uint16_t *>(x);
   uint32_t *amax_bits = reinterpret_cast<uint32_t *>(workspace);
+  const int64_t pieces = tokens * ((K / 16 + 63) / 64);         // amax pass: 1024-element pieces
+  if ((pieces + kAmaxWarps - 1) / kAmaxWarps > 0x7FFFFFFF) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   if (gs_mode == NVFP4_GS_FROM_AMAX) {
     if (cudaMemsetAsync(amax_bits, 0, sizeof(uint32_t) * G, stream) != cudaSuccess) return NVFP4_ERR_CUDA;
     if (tokens > 0) {
       const size_t sm = sizeof(int32_t) * (G + 1);
-      const unsigned grid = (unsigned)grid_resident(moe_amax_kernel, tokens * 32, 256, sm);
-      moe_amax_kernel<<<grid, 256, sm, stream>>>(xb, ld_x, K, tokens, slot, topk, group_offsets, G, amax_bits,
-                                                 dev_status);
+      const unsigned grid = (unsigned)((pieces + kAmaxWarps - 1) / kAmaxWarps);
+      moe_amax_kernel<<<grid, kAmaxWarps * 32, sm, stream>>>(xb, ld_x, K, tokens, slot, topk, group_offsets, G,
+                                                             amax_bits, dev_status);
       if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_CUDA;
     }
   }
-  finalize_scales_kernel<<<(G + 127) / 128, 128, 0, stream>>>(amax_bits, G, (int)gs_mode, global_scale, dev_status);
+  float *rtab = workspace_tables(workspace, G), *ytab = rtab + (size_t)G * 128;
+  finalize_tables_kernel<<<G, 128, 0, stream>>>(amax_bits, (int)gs_mode, global_scale, rtab, ytab, dev_status);
   if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_CUDA;
   if (tokens == 0) return NVFP4_OK;
   const size_t sm = sizeof(int32_t) * (2 * (G + 1) + 8);
-  float *rtab = workspace_tables(workspace, G), *ytab = rtab + (size_t)G * 128;
-  encode_tables_kernel<<<G, 128, 0, stream>>>(global_scale, rtab, ytab);
-  if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_CUDA;
   const int64_t work = tokens * ((K / 16 + 63) / 64) * 32;       // one warp per 64 blocks of a row
   if (sf_layout == NVFP4_SF_MMA_TILED) {
     const unsigned grid = (unsigned)grid_resident(moe_encode_blocks_kernel<true>, work, 256, sm);
