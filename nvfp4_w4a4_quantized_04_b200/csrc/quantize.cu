@@ -493,6 +493,20 @@ __device__ __forceinline__ uint32_t block_scale_fast(float a_b, float t_g, float
   return f32_to_e4m3_satfinite(__fdiv_rn(a_b, t_g));
 }
 
+// Both ends of the bracket of block_scale_fast in one packed multiply and one
+// two-way E4M3 conversion: returns the byte of q(1-2^-21) and sets `same` when
+// q(1+2^-21) rounds to the same byte.  Each end is rounded exactly as
+// f32_to_e4m3_satfinite rounds it alone.
+__device__ __forceinline__ uint32_t bracket_e4m3(float q, bool &same) {
+  const uint64_t qq = ((uint64_t)__float_as_uint(q) << 32) | __float_as_uint(q);
+  const uint64_t ends = mul_f32x2(qq, 0x3F8000043F7FFFF8ull);    // (1 - 2^-21, 1 + 2^-21)
+  uint16_t d;
+  asm("{\n.reg .f32 l, h;\nmov.b64 {l, h}, %1;\ncvt.rn.satfinite.e4m3x2.f32 %0, h, l;\n}" : "=h"(d) : "l"(ends));
+  const uint32_t lo = d & 0xFFu;
+  same = lo == (uint32_t)(d >> 8);
+  return lo;
+}
+
 // Codes of a block in fp32 pairs for a given r (a NaN product 0 * inf encodes as +0).
 __device__ __forceinline__ uint2 encode_codes(const uint64_t (&xf)[8], float r) {
   const uint64_t rr = ((uint64_t)__float_as_uint(r) << 32) | __float_as_uint(r);
@@ -568,15 +582,26 @@ __global__ void __launch_bounds__(256, 3) moe_encode_blocks_kernel(
       const float *rt = rtab + (int64_t)e * 128;
       uint8_t *qr = q + (uint64_t)p * (K >> 1);
       const uint64_t rsf = kTiled ? sf_row_part((uint32_t)p, nblk) : (uint64_t)p * nblk;
-      if (j0 < nblk) {
+      if (j1 < nblk) {
+        // both blocks (every chunk of a row whose K is a multiple of 1024):
+        // straight-line code, so the two blocks' chains interleave
+        const uint64_t qv = mul_f32x2(((uint64_t)__float_as_uint(am1) << 32) | __float_as_uint(am0),
+                                      ((uint64_t)__float_as_uint(y) << 32) | __float_as_uint(y));
+        bool same0, same1;
+        uint32_t S0 = bracket_e4m3(__uint_as_float((uint32_t)qv), same0);
+        uint32_t S1 = bracket_e4m3(__uint_as_float((uint32_t)(qv >> 32)), same1);
+        if (!same0 || exact) S0 = f32_to_e4m3_satfinite(__fdiv_rn(am0, t_g));
+        if (!same1 || exact) S1 = f32_to_e4m3_satfinite(__fdiv_rn(am1, t_g));
+        const float r0 = __ldg(rt + S0), r1 = __ldg(rt + S1);
+        const uint2 c0 = encode_codes(x0, r0), c1 = encode_codes(x1, r1);
+        *reinterpret_cast<uint2 *>(qr + (uint64_t)j0 * 8) = c0;
+        *reinterpret_cast<uint2 *>(qr + (uint64_t)j1 * 8) = c1;
+        sf[rsf + jb0] = (uint8_t)S0;
+        sf[rsf + jb1] = (uint8_t)S1;
+      } else if (j0 < nblk) {
         const uint32_t S = block_scale_fast(am0, t_g, y, exact);
         *reinterpret_cast<uint2 *>(qr + (uint64_t)j0 * 8) = encode_codes(x0, __ldg(rt + S));
         sf[rsf + jb0] = (uint8_t)S;
-      }
-      if (j1 < nblk) {
-        const uint32_t S = block_scale_fast(am1, t_g, y, exact);
-        *reinterpret_cast<uint2 *>(qr + (uint64_t)j1 * 8) = encode_codes(x1, __ldg(rt + S));
-        sf[rsf + jb1] = (uint8_t)S;
       }
     }
   }
