@@ -42,8 +42,9 @@
  *    prefix sums of the rows of each expert group, on the device), packed
  *    rows of group g start at the 128-aligned slot
  *    slot[g] = sum_{h<g} roundup(rows_h, 128); rows of a slot past the
- *    group's rows are written as zero codes and zero scales.  Size packed
- *    buffers with nvfp4_padded_rows_bound().
+ *    group's rows are left unwritten (the grouped GEMM reads them as padding
+ *    MMA rows whose outputs it never stores).  Size packed buffers with
+ *    nvfp4_padded_rows_bound().
  */
 #ifndef NVFP4_H_
 #define NVFP4_H_
@@ -176,6 +177,30 @@ nvfp4_status nvfp4_dequantize(const uint8_t *q, const uint8_t *sf, nvfp4_sf_layo
                               const float *global_scale, const int32_t *group_offsets,
                               int num_groups, int64_t rows, int64_t K, void *y,
                               nvfp4_out_dtype out_dtype, cudaStream_t stream);
+
+/*
+ * nvfp4_e2m1_encode -- the element-wise FP32 -> E2M1 step of every quantize
+ * call on its own.  [P2: the E2M1 value set {0, 0.5, 1, 1.5, 2, 3, 4, 6} with
+ *  a sign bit, two codes per byte.]  Round to nearest, ties to the even
+ * mantissa bit; magnitudes above 6 (and +-inf) saturate to 6; the sign is
+ * kept, so -0 and small negatives give 0x8; NaN gives +0 (the quantize
+ * kernels' rule for the product 0 * inf).
+ *   x   fp32 [n] device, 16-byte aligned; n % 8 == 0 (else UNSUPPORTED_SHAPE).
+ *   q   uint8 [n/2] device, 16-byte aligned: element 2i in bits [3:0] of byte
+ *       i, element 2i+1 in bits [7:4].
+ */
+nvfp4_status nvfp4_e2m1_encode(const float *x, int64_t n, uint8_t *q, cudaStream_t stream);
+
+/*
+ * nvfp4_e4m3_encode -- the element-wise FP32 -> E4M3 step of the block
+ * scales on its own.  [P1: the per-16 block scale is an FP8 E4M3 value, at
+ *  most 448.]  Round to nearest even, subnormals kept (2^-9 is the smallest),
+ * magnitudes from 464 up (and +-inf) saturate to +-448 (0x7E / 0xFE); NaN
+ * gives 0x7F.
+ *   x    fp32 [n] device, 16-byte aligned; n % 4 == 0 (else UNSUPPORTED_SHAPE).
+ *   out  uint8 [n] device, 16-byte aligned.
+ */
+nvfp4_status nvfp4_e4m3_encode(const float *x, int64_t n, uint8_t *out, cudaStream_t stream);
 
 /*
  * mxfp4_to_nvfp4 -- lossless block-by-block MXFP4 -> NVFP4 weight remap.

@@ -49,6 +49,7 @@ EXPORTS = [
     "nvfp4_moe_route_workspace_size", "nvfp4_moe_route", "nvfp4_moe_combine", "nvfp4_moe_quantize",
     "nvfp4_gemm_select_kernel", "nvfp4_grouped_gemm_w4a16", "nvfp4_grouped_gemm_swiglu_nvfp4",
     "mxfp4_quantize", "mxfp4_grouped_gemm", "nvfp4_w4a16_workspace_size",
+    "nvfp4_e2m1_encode", "nvfp4_e4m3_encode",
 ]
 NOALLOC_MAX_GROUPS = 1024
 
@@ -110,6 +111,10 @@ def load_library(path: str = LIB_PATH):
     L.nvfp4_moe_combine.argtypes = [P, i32, i64, P, P, i64, i32, i64, P, i32, P, P]
     L.nvfp4_kv_dequantize.restype = i32
     L.nvfp4_kv_dequantize.argtypes = [P, P, P, P, P, P, i64, i64, i64, P, P, P]
+    L.nvfp4_e2m1_encode.restype = i32
+    L.nvfp4_e2m1_encode.argtypes = [P, i64, P, P]
+    L.nvfp4_e4m3_encode.restype = i32
+    L.nvfp4_e4m3_encode.argtypes = [P, i64, P, P]
     _lib = L
     return L
 
@@ -215,6 +220,22 @@ def nvfp4_dequantize(q, sf, sf_layout, global_scale, group_offsets, num_groups, 
         _ptr(y), out_dtype, _stream(stream))
     if check:
         _check(st, "nvfp4_dequantize")
+    return st
+
+
+def nvfp4_e2m1_encode(x, n, q, stream=None, check=True) -> int:
+    """fp32 [n] -> packed E2M1 codes [n/2] (the quantize kernels' code step)."""
+    st = load_library().nvfp4_e2m1_encode(_ptr(x), n, _ptr(q), _stream(stream))
+    if check:
+        _check(st, "nvfp4_e2m1_encode")
+    return st
+
+
+def nvfp4_e4m3_encode(x, n, out, stream=None, check=True) -> int:
+    """fp32 [n] -> E4M3 bytes [n] (the block-scale step)."""
+    st = load_library().nvfp4_e4m3_encode(_ptr(x), n, _ptr(out), _stream(stream))
+    if check:
+        _check(st, "nvfp4_e4m3_encode")
     return st
 
 

@@ -608,6 +608,31 @@ __global__ void __launch_bounds__(256, 3) moe_encode_blocks_kernel(
   if (bad) report(dev_status, NVFP4_ERR_NONFINITE);
 }
 
+// ---------------------------------------------------------------- element-wise codecs
+// The two conversions of the encode path on their own, for any fp32 input:
+// E2M1 through e2m1x8_from_pairs (the code step of every quantize kernel; a
+// NaN input encodes as +0, as the product 0 * inf does there), E4M3 through
+// f32_to_e4m3_satfinite (the block-scale step; NaN gives 0x7F).
+__global__ void e2m1_encode_kernel(const float4 *__restrict__ x, int64_t n8, uint32_t *__restrict__ q) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += stride) {
+    const float4 a = x[2 * i], b = x[2 * i + 1];
+    auto pair = [](float lo, float hi) {
+      return sanitize_pair(((uint64_t)__float_as_uint(hi) << 32) | __float_as_uint(lo));
+    };
+    q[i] = e2m1x8_from_pairs(pair(a.x, a.y), pair(a.z, a.w), pair(b.x, b.y), pair(b.z, b.w));
+  }
+}
+
+__global__ void e4m3_encode_kernel(const float4 *__restrict__ x, int64_t n4, uint32_t *__restrict__ out) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += stride) {
+    const float4 v = x[i];
+    auto enc = [](float f) { return isnan(f) ? 0x7Fu : f32_to_e4m3_satfinite(f); };
+    out[i] = enc(v.x) | (enc(v.y) << 8) | (enc(v.z) << 16) | (enc(v.w) << 24);
+  }
+}
+
 // ---------------------------------------------------------------- dequantize
 // (code * S) in f16 is exact (at most 6 significant bits, |.| <= 2688), so the
 // hardware E2M1 -> f16 conversion times the f16 scale gives the exact product;
@@ -974,6 +999,28 @@ nvfp4_status nvfp4_moe_quantize(const void *x, int64_t tokens, int64_t K, int64_
     moe_encode_blocks_kernel<false><<<grid, 256, sm, stream>>>(xb, ld_x, K, tokens, slot, topk, group_offsets, G,
                                                                global_scale, rtab, ytab, q, sf, dev_status);
   }
+  return launch_status();
+}
+
+nvfp4_status nvfp4_e2m1_encode(const float *x, int64_t n, uint8_t *q, cudaStream_t stream) {
+  if (n < 0) return NVFP4_ERR_INVALID_ARG;
+  if (n % 8 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (n == 0) return NVFP4_OK;
+  if (!x || !q || !aligned16(x) || !aligned16(q)) return NVFP4_ERR_INVALID_ARG;
+  const int64_t n8 = n / 8;
+  e2m1_encode_kernel<<<(unsigned)grid_for(n8, 256, 8), 256, 0, stream>>>(reinterpret_cast<const float4 *>(x), n8,
+                                                                        reinterpret_cast<uint32_t *>(q));
+  return launch_status();
+}
+
+nvfp4_status nvfp4_e4m3_encode(const float *x, int64_t n, uint8_t *out, cudaStream_t stream) {
+  if (n < 0) return NVFP4_ERR_INVALID_ARG;
+  if (n % 4 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (n == 0) return NVFP4_OK;
+  if (!x || !out || !aligned16(x) || !aligned16(out)) return NVFP4_ERR_INVALID_ARG;
+  const int64_t n4 = n / 4;
+  e4m3_encode_kernel<<<(unsigned)grid_for(n4, 256, 8), 256, 0, stream>>>(reinterpret_cast<const float4 *>(x), n4,
+                                                                        reinterpret_cast<uint32_t *>(out));
   return launch_status();
 }
 

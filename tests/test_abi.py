@@ -78,6 +78,14 @@ def test_host_validation_without_device(lib):
     assert L.nvfp4_quantize(fake, 4, 32, 32, None, None, 1, 3, fake, fake, fake, 0, fake, None, None) == nv.ERR_INVALID_ARG
     # empty problems are no-ops that touch nothing
     assert L.nvfp4_grouped_gemm(None, None, None, None, None, None, None, 1, 0, 128, 512, None, 0, 0, None, None, None, None) == nv.OK
+    # element-wise codecs: length multiple of 8 (E2M1) or 4 (E4M3), aligned pointers
+    assert L.nvfp4_e2m1_encode(fake, 12, fake, None) == nv.ERR_UNSUPPORTED_SHAPE
+    assert L.nvfp4_e2m1_encode(fake, -8, fake, None) == nv.ERR_INVALID_ARG
+    assert L.nvfp4_e2m1_encode(fake, 16, P((1 << 20) + 4), None) == nv.ERR_INVALID_ARG
+    assert L.nvfp4_e2m1_encode(None, 0, None, None) == nv.OK
+    assert L.nvfp4_e4m3_encode(fake, 6, fake, None) == nv.ERR_UNSUPPORTED_SHAPE
+    assert L.nvfp4_e4m3_encode(None, 8, fake, None) == nv.ERR_INVALID_ARG
+    assert L.nvfp4_e4m3_encode(None, 0, None, None) == nv.OK
     assert L.nvfp4_dequantize(None, None, 0, None, None, 1, 0, 32, None, 0, None) == nv.OK
     # remap shape limits
     assert L.mxfp4_to_nvfp4(fake, fake, 1, 4, 48, fake, fake, 0, fake, fake, None, None) == nv.ERR_UNSUPPORTED_SHAPE
