@@ -10,7 +10,9 @@ The other rows of the path are measured in the same run as "components":
 the dense MLP (4096 tokens, 5120 -> 2x17408 -> 5120), the decode MoE (384
 experts, 64 tokens, Zipf routing, MXFP4 weights remapped to NVFP4), the
 NVFP4 KV cache (4 heads x 256 x 262144 tokens, K and V), the activation
-quantize sweep [T, 5120] and the MXFP4 -> NVFP4 remap of 2^28 elements.
+quantize sweep [T, 5120], the MXFP4 -> NVFP4 remap of 2^28 elements, the
+W4A16 decode layer, the MXFP4 encoder and GEMM, the whole MoE block (route,
+experts, combine), and the smallest GEMM [128 x 256 x 512] in microseconds.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
        [--experts E --tokens T] [--components all|none|<name,...>] [--no-cpu-baseline]
@@ -51,7 +53,7 @@ PEAKS, PEAKS_KIND = load_peaks()
 HBM_PEAK = PEAKS.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
 # DRAM traffic / algorithmic bytes of the gate_up + SwiGLU grouped GEMM launch,
 # from one ncu capture of this kernel (706.6 MB / 693.1 MB at 128 experts).
-GATE_UP_TRAFFIC_RATIO = 706575616 / 693108736
+GATE_UP_TRAFFIC_RATIO = 707430400 / 693108736
 FP4_PEAK = PEAKS.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]) * FP4_OVER_BF16
 
 
@@ -337,7 +339,7 @@ def run_headline(args, rank, world, device):
             "traffic": (int(GATE_UP_TRAFFIC_RATIO * g1_bytes) if fused else None),
             "traffic_source": ("ncu dram__bytes_read.sum + dram__bytes_write.sum of the gate_up + SwiGLU launch at "
                                "128 experts / 2048 tokens (profiles/grouped_gemm_moe_e128_t2048.md), ratio to "
-                               "algorithmic bytes 1.019, scaled by the units processed" if fused else None),
+                               "algorithmic bytes 1.021, scaled by the units processed" if fused else None),
             "peak_source": f"{PEAKS_KIND} hbm_gbs (burst copy)",
             "algorithmic_bytes_per_launch": int(g1_bytes), "avg_launch_ms": round(g1_ms, 4),
             "tensor_tflops": round(g1_flops / (g1_ms * 1e-3) / 1e12, 1),
@@ -613,6 +615,34 @@ def comp_act_sweep(device, iters, warmup, flush):
     return out
 
 
+def comp_gemm_small(device, iters, warmup, flush):
+    """The smallest GEMM case, X [128, 512] x W [256, 512] -> fp32 [128, 256]:
+    launch- and latency-bound, reported in microseconds (dynamic quantize of X,
+    the GEMM, and both back to back)."""
+    import torch
+
+    import synthetic
+    import synthetic.cuda as sc
+    from nvfp4_w4a4_quantized_04_b200 import layer as L
+    M, N, K = 128, 256, 512
+    ws = L.workspace(1, device)
+    w = L.pack_weights(sc.gaussian_bf16(0, synthetic.STREAMS["w_gate_up"], (N, K), sigma=0.02), 1, N, None, ws)
+    x = sc.gaussian_bf16(0, synthetic.STREAMS["x"], (M, K))
+    a = L.empty_packed(M, K, 1, None, 1, device)
+    y = torch.empty((M, N), dtype=torch.float32, device=device)
+    t_q = timed(lambda: L.quantize(x, layout=1, out=a, ws=ws), iters, warmup, flush)
+    t_g = timed(lambda: L.grouped_gemm(a, w, N, 0, y=y), iters, warmup, flush)
+
+    def both():
+        L.quantize(x, layout=1, out=a, ws=ws)
+        L.grouped_gemm(a, w, N, 0, y=y)
+    t_b = timed(both, iters, warmup, flush)
+    flop = 2.0 * M * N * K
+    return {"workload": "gemm_m128_n256_k512_fp32_out", "quantize_us": round(t_q * 1e3, 2),
+            "gemm_us": round(t_g * 1e3, 2), "quantize_and_gemm_us": round(t_b * 1e3, 2),
+            "gemm_tflops": round(flop / (t_g * 1e-3) / 1e12, 3), "bound": "launch latency"}
+
+
 def comp_remap(device, iters, warmup, flush):
     """MXFP4 -> NVFP4 remap of 2^28 elements as 1024 tensors of [512, 512]."""
     import torch
@@ -731,7 +761,7 @@ COMPONENTS = {"moe_full": comp_moe_full, "moe_static_h": comp_moe_static_h, "den
               "decode_moe": comp_decode_moe,
               "decode_w4a16": comp_decode_w4a16, "kv_cache": comp_kv,
               "act_quant_sweep": comp_act_sweep, "remap": comp_remap, "mxfp4_encode": comp_mxfp4_encode,
-              "mx_gemm_routes": comp_mx_gemm_routes}
+              "mx_gemm_routes": comp_mx_gemm_routes, "gemm_small": comp_gemm_small}
 
 
 # --------------------------------------------------------------------------- CPU oracle baseline
