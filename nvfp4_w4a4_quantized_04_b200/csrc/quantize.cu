@@ -93,20 +93,41 @@ __global__ void __launch_bounds__(256) amax_rows_kernel(
   if (lane == 0 && mm) atomicMax(&amax_bits[g], mm << 16);
 }
 
-// Dense contiguous tensor: flat grid-stride over 16-byte vectors.
-__global__ void __launch_bounds__(256) amax_flat_kernel(const uint4 *__restrict__ x, int64_t nvec,
-                                                        uint32_t *__restrict__ amax_bits) {
+// One 16-element bf16 block: a 32-byte load when v8 (32-byte aligned), else two 16-byte loads.
+__device__ __forceinline__ void load_block(const uint16_t *p, bool v8, uint4 &a, uint4 &b) {
+  if (v8) {
+    asm volatile("ld.global.nc.L1::no_allocate.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w), "=r"(b.x), "=r"(b.y), "=r"(b.z), "=r"(b.w)
+                 : "l"(p));
+  } else {
+    a = ldg_nc_v4(p);
+    b = ldg_nc_v4(p + 8);
+  }
+}
+
+// Dense contiguous tensor: flat grid-stride over 16-element blocks (32 bytes,
+// one 32-byte load when x is 32-byte aligned).  Four blocks, 128 bytes, are in
+// flight per thread and at least four CTAs of 256 threads fit on an SM, so
+// each SM keeps 128 KB of loads outstanding; the grid is one resident wave.
+template <bool kV8>
+__global__ void __launch_bounds__(256, 4) amax_flat_kernel(const uint16_t *__restrict__ x, int64_t nblk,
+                                                           uint32_t *__restrict__ amax_bits) {
   const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   uint32_t m = 0;
   int64_t i = tid;
-  for (; i + 3 * stride < nvec; i += 4 * stride) {
-    uint4 a = ldg_nc_v4(x + i), b = ldg_nc_v4(x + i + stride);
-    uint4 c = ldg_nc_v4(x + i + 2 * stride), d = ldg_nc_v4(x + i + 3 * stride);
-    m = absmax8_bits(a, m); m = absmax8_bits(b, m);
-    m = absmax8_bits(c, m); m = absmax8_bits(d, m);
+  for (; i + 3 * stride < nblk; i += 4 * stride) {
+    uint4 a[4], b[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) load_block(x + (uint64_t)(i + k * stride) * 16, kV8, a[k], b[k]);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) m = absmax8_bits(b[k], absmax8_bits(a[k], m));
   }
-  for (; i < nvec; i += stride) m = absmax8_bits(ldg_nc_v4(x + i), m);
+  for (; i < nblk; i += stride) {
+    uint4 a, b;
+    load_block(x + (uint64_t)i * 16, kV8, a, b);
+    m = absmax8_bits(b, absmax8_bits(a, m));
+  }
   m = warp_max(halves_max(m));
   __shared__ uint32_t red[8];
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
@@ -149,16 +170,6 @@ __global__ void finalize_scales_kernel(const uint32_t *__restrict__ amax_bits, i
 // Per 16-element block: the block amax in integer SIMD, one IEEE division
 // for the scale and one IEEE reciprocal, the 16 products as eight packed
 // f32x2 multiplies, eight e2m1x2 conversions and one 8-byte store.
-__device__ __forceinline__ void load_block(const uint16_t *p, bool v8, uint4 &a, uint4 &b) {
-  if (v8) {
-    asm volatile("ld.global.nc.L1::no_allocate.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-                 : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w), "=r"(b.x), "=r"(b.y), "=r"(b.z), "=r"(b.w)
-                 : "l"(p));
-  } else {
-    a = ldg_nc_v4(p);
-    b = ldg_nc_v4(p + 8);
-  }
-}
 
 // bf16 pair (element 2i in bits 0..15) -> fp32 pair (element 2i in the low word).
 __device__ __forceinline__ uint64_t bf16x2_to_f32x2(uint32_t w) {
@@ -843,9 +854,14 @@ nvfp4_status run_global_scales(const uint16_t *x, int64_t rows, int64_t K, int64
     if (cudaMemsetAsync(amax_bits, 0, sizeof(uint32_t) * G, stream) != cudaSuccess) return NVFP4_ERR_CUDA;
     if (rows > 0) {
       if (!group_offsets && !row_index && ld_x == K) {
-        int64_t nvec = rows * K / 8;
-        amax_flat_kernel<<<(unsigned)grid_for(nvec / 4, 256, 8), 256, 0, stream>>>(
-            reinterpret_cast<const uint4 *>(x), nvec, amax_bits);
+        const int64_t nblk = rows * K / 16;
+        if ((reinterpret_cast<uintptr_t>(x) & 31u) == 0) {
+          const unsigned grid = (unsigned)grid_resident(amax_flat_kernel<true>, (nblk + 3) / 4, 256, 0);
+          amax_flat_kernel<true><<<grid, 256, 0, stream>>>(x, nblk, amax_bits);
+        } else {
+          const unsigned grid = (unsigned)grid_resident(amax_flat_kernel<false>, (nblk + 3) / 4, 256, 0);
+          amax_flat_kernel<false><<<grid, 256, 0, stream>>>(x, nblk, amax_bits);
+        }
       } else {
         size_t sm = group_offsets ? sizeof(int32_t) * (G + 1) : 0;
         int64_t warps_needed = rows;
