@@ -11,7 +11,8 @@
 //
 // Pass 1 (reads codes + exponents, writes the code copy): per tensor, the
 // largest and smallest exponent over blocks that are not all +-0, and the
-// 0xFF check.  Pass 2 (reads exponents only): the scale bytes and s_g.
+// 0xFF check.  Pass 2 (reads exponents only): the scale bytes and s_g, a warp
+// per 512-byte scale atom in the tensor-core layout.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -20,13 +21,18 @@
 namespace nvfp4 {
 
 // ws[2t] = max(u+1), ws[2t+1] = max(256-u) over non-zero blocks of tensor t
-// (0 = no such block), via atomicMax on zero-initialised words.
+// (0 = no such block), via atomicMax on zero-initialised words.  A CTA takes
+// kScanChunk consecutive blocks of one tensor, eight per thread (128 bytes of
+// codes in flight per thread); CTAs are short and not persistent.
+constexpr int kScanUnroll = 8;
+constexpr int64_t kScanChunk = 256 * kScanUnroll;
+
 __global__ void __launch_bounds__(256) remap_scan_kernel(
     const uint8_t *__restrict__ q_mx, const uint8_t *__restrict__ e8, int64_t blocks_per_tensor,
-    int64_t chunk, uint8_t *__restrict__ q_nv, uint32_t *__restrict__ ws, int32_t *dev_status) {
+    uint8_t *__restrict__ q_nv, uint32_t *__restrict__ ws, int32_t *dev_status) {
   const int64_t t = blockIdx.y;
-  const int64_t b0 = (int64_t)blockIdx.x * chunk;
-  const int64_t b1 = min(blocks_per_tensor, b0 + chunk);
+  const int64_t b0 = (int64_t)blockIdx.x * kScanChunk;
+  const int64_t b1 = min(blocks_per_tensor, b0 + kScanChunk);
   const uint4 *qt = reinterpret_cast<const uint4 *>(q_mx) + t * blocks_per_tensor;
   uint4 *qo = reinterpret_cast<uint4 *>(q_nv) + t * blocks_per_tensor;
   const uint8_t *et = e8 + t * blocks_per_tensor;
@@ -41,28 +47,50 @@ __global__ void __launch_bounds__(256) remap_scan_kernel(
       lo = max(lo, 256u - u);
     }
   };
-  // four blocks (64 bytes of codes) in flight per thread
-  int64_t b = b0 + threadIdx.x;
   const int64_t st = blockDim.x;
-  for (; b + 3 * st < b1; b += 4 * st) {
-    const uint4 c0 = __ldg(qt + b), c1 = __ldg(qt + b + st), c2 = __ldg(qt + b + 2 * st), c3 = __ldg(qt + b + 3 * st);
-    const uint32_t u0 = et[b], u1 = et[b + st], u2 = et[b + 2 * st], u3 = et[b + 3 * st];
-    if (copy) { qo[b] = c0; qo[b + st] = c1; qo[b + 2 * st] = c2; qo[b + 3 * st] = c3; }
-    visit(c0, u0); visit(c1, u1); visit(c2, u2); visit(c3, u3);
-  }
-  for (; b < b1; b += st) {
-    const uint4 c = __ldg(qt + b);
-    if (copy) qo[b] = c;
-    visit(c, et[b]);
+  int64_t b = b0 + threadIdx.x;
+  if (b0 + kScanChunk <= blocks_per_tensor) {
+    uint4 c[kScanUnroll];
+    uint32_t u[kScanUnroll];
+#pragma unroll
+    for (int k = 0; k < kScanUnroll; ++k) c[k] = __ldg(qt + b + k * st);
+#pragma unroll
+    for (int k = 0; k < kScanUnroll; ++k) u[k] = et[b + k * st];
+    if (copy) {
+#pragma unroll
+      for (int k = 0; k < kScanUnroll; ++k) qo[b + k * st] = c[k];
+    }
+#pragma unroll
+    for (int k = 0; k < kScanUnroll; ++k) visit(c[k], u[k]);
+  } else {
+    for (; b < b1; b += st) {
+      const uint4 c = __ldg(qt + b);
+      if (copy) qo[b] = c;
+      visit(c, et[b]);
+    }
   }
 #pragma unroll
   for (int d = 16; d > 0; d >>= 1) {
     hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, d));
     lo = max(lo, __shfl_xor_sync(0xffffffffu, lo, d));
   }
-  if ((threadIdx.x & 31) == 0 && hi) {
-    atomicMax(&ws[2 * t], hi);
-    atomicMax(&ws[2 * t + 1], lo);
+  // one pair of atomics per CTA: the words of a tensor are shared by all of
+  // its CTAs, so same-address atomics are what this pass must keep few
+  __shared__ uint32_t red[2][8];
+  if ((threadIdx.x & 31) == 0) {
+    red[0][threadIdx.x >> 5] = hi;
+    red[1][threadIdx.x >> 5] = lo;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < (int)(blockDim.x >> 5); ++w) {
+      hi = max(hi, red[0][w]);
+      lo = max(lo, red[1][w]);
+    }
+    if (hi) {
+      atomicMax(&ws[2 * t], hi);
+      atomicMax(&ws[2 * t + 1], lo);
+    }
   }
   if (bad) report(dev_status, NVFP4_ERR_NOT_REPRESENTABLE);
 }
@@ -72,45 +100,75 @@ __device__ __forceinline__ uint32_t e4m3_pow2(int p) {
   return p >= -6 ? (uint32_t)((p + 7) << 3) : (1u << (p + 9));
 }
 
-template <bool kTiled>
-__global__ void __launch_bounds__(256) remap_scale_kernel(
+// Tensor-core scale layout: a warp writes 512-byte atoms (row block, group of
+// four 16-element scales), up to kAtomRun consecutive groups of one row block
+// per work unit, so the 32-byte sectors of UE8M0 bytes it reads (16 groups of
+// a row) come from L2 once and are reused from L1.  In an atom, lane l covers
+// rows l, l+32, l+64 and l+96 of the row block: for each it reads the two
+// UE8M0 bytes of the group's 64 elements and writes the four scale bytes
+// (each 32-block's byte twice) as one 16-byte line.  Lane 0 of a tensor's
+// first unit also writes s_g and checks the exponent spread.
+constexpr int64_t kAtomRun = 16;
+
+__device__ __forceinline__ int remap_global_exp(const uint32_t *__restrict__ ws, int64_t t, uint32_t &hi,
+                                                uint32_t &lo) {
+  hi = ws[2 * t];
+  lo = ws[2 * t + 1];
+  return hi ? (int)hi - 1 - 127 - 8 : 0;
+}
+
+__global__ void __launch_bounds__(256) remap_scale_atoms_kernel(
     const uint8_t *__restrict__ e8, int64_t rows, int64_t K, int64_t n_tensors,
-    const uint32_t *__restrict__ ws, uint8_t *__restrict__ sf, float *__restrict__ gs,
-    int32_t *dev_status) {
-  const uint64_t nb32_row = (uint64_t)(K >> 5);
-  const uint64_t per_tensor = (uint64_t)rows * nb32_row;
-  const uint64_t total = (uint64_t)n_tensors * per_tensor;
-  const uint64_t nsf = (uint64_t)(K >> 4);
-  const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
-  const bool small = total < 0xFFFFFFF0ull;
-  for (uint64_t i = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += stride) {
-    uint64_t t, within, r, jb;
-    if (small) {
-      const uint32_t i32 = (uint32_t)i, t32 = i32 / (uint32_t)per_tensor;
-      const uint32_t w32 = i32 - t32 * (uint32_t)per_tensor, r32 = w32 / (uint32_t)nb32_row;
-      t = t32; within = w32; r = r32; jb = w32 - r32 * (uint32_t)nb32_row;
-    } else {
-      t = i / per_tensor; within = i - t * per_tensor; r = within / nb32_row; jb = within - r * nb32_row;
+    const uint32_t *__restrict__ ws, uint8_t *__restrict__ sf, float *__restrict__ gs, int32_t *dev_status) {
+  const int lane = threadIdx.x & 31;
+  const int64_t rb_per_t = rows >> 7, kg_per_row = K >> 6, nb32 = K >> 5;
+  const int64_t runs_per_rb = (kg_per_row + kAtomRun - 1) / kAtomRun;
+  const int64_t units_per_t = rb_per_t * runs_per_rb;
+  const int64_t total = n_tensors * units_per_t;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t u = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; u < total; u += nwarps) {
+    const int64_t t = u / units_per_t, w = u - t * units_per_t;
+    const int64_t rb = w / runs_per_rb, kg0 = (w - rb * runs_per_rb) * kAtomRun;
+    const int64_t kg1 = min(kg_per_row, kg0 + kAtomRun);
+    uint32_t hi, lo;
+    const int g = remap_global_exp(ws, t, hi, lo);
+    if (w == 0 && lane == 0) {
+      gs[t] = ldexpf(1.0f, g);   // 2^g exactly, g in [-135, 119] (subnormal below -126)
+      if (hi && (256 - (int)lo - 127) - g < -9) report(dev_status, NVFP4_ERR_NOT_REPRESENTABLE);
     }
-    const uint32_t hi = ws[2 * t], lo = ws[2 * t + 1];
-    const int g = hi ? (int)hi - 1 - 127 - 8 : 0;
+    const uint8_t *rows0 = e8 + (t * rows + rb * 128 + lane) * nb32;
+    uint8_t *atom = sf + (t * rb_per_t + rb) * kg_per_row * 512 + lane * 16;
+    for (int64_t kg = kg0; kg < kg1; ++kg) {
+      uint32_t words[4];
+#pragma unroll
+      for (int qd = 0; qd < 4; ++qd) {
+        const uint8_t *er = rows0 + qd * 32 * nb32 + 2 * kg;
+        const uint32_t S0 = e4m3_pow2(max(-9, min(8, (int)er[0] - 127 - g)));
+        const uint32_t S1 = e4m3_pow2(max(-9, min(8, (int)er[1] - 127 - g)));
+        words[qd] = S0 * 0x0101u | S1 * 0x01010000u;
+      }
+      *reinterpret_cast<uint4 *>(atom + kg * 512) = make_uint4(words[0], words[1], words[2], words[3]);
+    }
+  }
+}
+
+// Row-major scale layout: MX block i (over all tensors) gives scales 2i and
+// 2i+1, written as one 2-byte store.
+__global__ void __launch_bounds__(256) remap_scale_rows_kernel(
+    const uint8_t *__restrict__ e8, int64_t per_tensor, int64_t n_tensors, const uint32_t *__restrict__ ws,
+    uint8_t *__restrict__ sf, float *__restrict__ gs, int32_t *dev_status) {
+  const uint64_t total = (uint64_t)n_tensors * (uint64_t)per_tensor;
+  const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
+  for (uint64_t i = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += stride) {
+    const uint64_t t = i / (uint64_t)per_tensor, within = i - t * (uint64_t)per_tensor;
+    uint32_t hi, lo;
+    const int g = remap_global_exp(ws, (int64_t)t, hi, lo);
     if (within == 0) {
       gs[t] = ldexpf(1.0f, g);   // 2^g exactly, g in [-135, 119] (subnormal below -126)
-      if (hi) {
-        const int emin = 256 - (int)lo - 127;
-        if (emin - g < -9) report(dev_status, NVFP4_ERR_NOT_REPRESENTABLE);
-      }
+      if (hi && (256 - (int)lo - 127) - g < -9) report(dev_status, NVFP4_ERR_NOT_REPRESENTABLE);
     }
-    const int e = (int)e8[i] - 127;
-    const int p = max(-9, min(8, e - g));
-    const uint32_t S = e4m3_pow2(p);
-    const uint64_t row = t * (uint64_t)rows + r, j = 2 * jb;
-    if (kTiled) {
-      // scales j and j+1 share one 4-scale group: two adjacent bytes
-      *reinterpret_cast<uint16_t *>(sf + sf_tiled_offset(row, j, nsf)) = (uint16_t)(S | (S << 8));
-    } else {
-      *reinterpret_cast<uint16_t *>(sf + row * nsf + j) = (uint16_t)(S | (S << 8));
-    }
+    const uint32_t S = e4m3_pow2(max(-9, min(8, (int)e8[i] - 127 - g)));
+    *reinterpret_cast<uint16_t *>(sf + 2 * i) = (uint16_t)(S | (S << 8));
   }
 }
 
@@ -135,20 +193,27 @@ extern "C" nvfp4_status mxfp4_to_nvfp4(const uint8_t *q_mx, const uint8_t *ue8m0
   uint32_t *ws = reinterpret_cast<uint32_t *>(workspace);
   if (cudaMemsetAsync(ws, 0, sizeof(uint32_t) * 2 * n_tensors, stream) != cudaSuccess) return NVFP4_ERR_CUDA;
   const int64_t bpt = rows * (K / 32);
-  const int64_t chunk = 8192;
-  dim3 grid1((unsigned)((bpt + chunk - 1) / chunk), (unsigned)n_tensors);
+  const int64_t xblocks = (bpt + kScanChunk - 1) / kScanChunk;
+  if (xblocks > 0x7FFFFFFF) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  dim3 grid1((unsigned)xblocks, (unsigned)n_tensors);
   if (grid1.y > 65535) return NVFP4_ERR_UNSUPPORTED_SHAPE;
-  remap_scan_kernel<<<grid1, 256, 0, stream>>>(q_mx, ue8m0, bpt, chunk, q_nv, ws, dev_status);
+  remap_scan_kernel<<<grid1, 256, 0, stream>>>(q_mx, ue8m0, bpt, q_nv, ws, dev_status);
   if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_CUDA;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t total = n_tensors * bpt;
-  int64_t blocks = (total + 255) / 256;
-  if (blocks > (int64_t)sms * 8) blocks = (int64_t)sms * 8;
-  if (sf_layout == NVFP4_SF_MMA_TILED)
-    remap_scale_kernel<true><<<(unsigned)blocks, 256, 0, stream>>>(ue8m0, rows, K, n_tensors, ws, sf_nv, global_scale, dev_status);
-  else
-    remap_scale_kernel<false><<<(unsigned)blocks, 256, 0, stream>>>(ue8m0, rows, K, n_tensors, ws, sf_nv, global_scale, dev_status);
+  if (sf_layout == NVFP4_SF_MMA_TILED) {
+    const int64_t units = n_tensors * (rows / 128) * ((K / 64 + kAtomRun - 1) / kAtomRun);
+    int64_t blocks = (units + 7) / 8;                      // a warp per unit, 8 warps per CTA
+    if (blocks > (int64_t)sms * 8) blocks = (int64_t)sms * 8;
+    remap_scale_atoms_kernel<<<(unsigned)blocks, 256, 0, stream>>>(ue8m0, rows, K, n_tensors, ws, sf_nv, global_scale,
+                                                                   dev_status);
+  } else {
+    const int64_t total = n_tensors * bpt;
+    int64_t blocks = (total + 255) / 256;
+    if (blocks > (int64_t)sms * 8) blocks = (int64_t)sms * 8;
+    remap_scale_rows_kernel<<<(unsigned)blocks, 256, 0, stream>>>(ue8m0, bpt, n_tensors, ws, sf_nv, global_scale,
+                                                                   dev_status);
+  }
   return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
