@@ -886,7 +886,16 @@ def main():
         flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
         out["components"] = {}
         for n in names:
+            # an NVTX range per component, so a profiler can select one
+            # component's launches (ncu --nvtx --nvtx-include "<name>/")
+            nvtx = getattr(torch.cuda, "nvtx", None)
+            try:
+                nvtx.range_push(n)
+            except Exception:
+                nvtx = None
             out["components"][n] = COMPONENTS[n](device, 7, 3, flush)
+            if nvtx is not None:
+                nvtx.range_pop()
             torch.cuda.empty_cache()
 
     if rank == 0 and not args.no_cpu_baseline:

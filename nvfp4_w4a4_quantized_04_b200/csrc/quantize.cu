@@ -343,8 +343,25 @@ __global__ void __launch_bounds__(256) quantize_kernel(
   const uint32_t nchunks = (total + 32 * U - 1) / (32 * U);
   const uint32_t warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
-  const uint32_t per = (nchunks + nwarps - 1) / nwarps;
-  const uint32_t c_begin = min(nchunks, warp * per), c_end = min(nchunks, c_begin + per);
+  // Ungrouped tensors: chunks are dealt round-robin, so all warps work on one
+  // narrow band of rows at a time and the scale bytes of a 32-byte sector
+  // (rows r, r+1, r+32, ..., r+97 in the tiled layout) are written close
+  // together in time; the sector is complete before L2 evicts it.  Contiguous
+  // ranges per warp left rows r and r+32 far apart in time when rows are long,
+  // and the partial sectors cost a read-modify-write in DRAM.  Grouped calls
+  // keep contiguous ranges, so a warp's group index walks forward one group at
+  // a time (their rows are short and their ranges a few rows long).
+  uint32_t c_begin, c_end, c_step;
+  if (!group_offsets) {
+    c_begin = warp;
+    c_end = nchunks;
+    c_step = nwarps;
+  } else {
+    const uint32_t per = (nchunks + nwarps - 1) / nwarps;
+    c_begin = min(nchunks, warp * per);
+    c_end = min(nchunks, c_begin + per);
+    c_step = 1;
+  }
   if (c_begin >= c_end) return;
   const bool v8 = ((reinterpret_cast<uintptr_t>(x) & 31u) == 0) && ((ld_x & 15) == 0);
   int g = group_offsets ? upper_group(off, G, fast_div(c_begin * (32 * U), fd)) : 0;
@@ -353,7 +370,7 @@ __global__ void __launch_bounds__(256) quantize_kernel(
   uint64_t rsf = 0;
   float s_g = gs[g], t_g = __fmul_rn(6.0f, s_g);
   bool bad = false;
-  for (uint32_t c = c_begin; c < c_end; ++c) {
+  for (uint32_t c = c_begin; c < c_end; c += c_step) {
     uint4 va[U], vb[U];
     uint32_t pp[U], jj[U];
     uint64_t rs[U];

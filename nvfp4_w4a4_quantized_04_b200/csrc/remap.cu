@@ -119,7 +119,8 @@ __device__ __forceinline__ int remap_global_exp(const uint32_t *__restrict__ ws,
 
 __global__ void __launch_bounds__(256) remap_scale_atoms_kernel(
     const uint8_t *__restrict__ e8, int64_t rows, int64_t K, int64_t n_tensors,
-    const uint32_t *__restrict__ ws, uint8_t *__restrict__ sf, float *__restrict__ gs, int32_t *dev_status) {
+    const uint32_t *__restrict__ ws, uint8_t *__restrict__ sf, float *__restrict__ gs, bool vec,
+    int32_t *dev_status) {
   const int lane = threadIdx.x & 31;
   const int64_t rb_per_t = rows >> 7, kg_per_row = K >> 6, nb32 = K >> 5;
   const int64_t runs_per_rb = (kg_per_row + kAtomRun - 1) / kAtomRun;
@@ -138,16 +139,43 @@ __global__ void __launch_bounds__(256) remap_scale_atoms_kernel(
     }
     const uint8_t *rows0 = e8 + (t * rows + rb * 128 + lane) * nb32;
     uint8_t *atom = sf + (t * rb_per_t + rb) * kg_per_row * 512 + lane * 16;
-    for (int64_t kg = kg0; kg < kg1; ++kg) {
-      uint32_t words[4];
+    const int kr = (int)(kg1 - kg0);
+    // the run's UE8M0 bytes of this lane's four rows, loaded up front: one or
+    // two 16-byte loads per row when they are aligned and the run is 8 or 16
+    // groups long (then they end inside the run), single bytes otherwise
+    uint32_t ew[4][8];
 #pragma unroll
-      for (int qd = 0; qd < 4; ++qd) {
-        const uint8_t *er = rows0 + qd * 32 * nb32 + 2 * kg;
-        const uint32_t S0 = e4m3_pow2(max(-9, min(8, (int)er[0] - 127 - g)));
-        const uint32_t S1 = e4m3_pow2(max(-9, min(8, (int)er[1] - 127 - g)));
-        words[qd] = S0 * 0x0101u | S1 * 0x01010000u;
+    for (int qd = 0; qd < 4; ++qd) {
+      const uint8_t *er = rows0 + qd * 32 * nb32 + 2 * kg0;
+      if (vec && (kr == 8 || kr == 16)) {
+        const uint4 a = __ldg(reinterpret_cast<const uint4 *>(er));
+        const uint4 b = kr == 16 ? __ldg(reinterpret_cast<const uint4 *>(er) + 1) : make_uint4(0, 0, 0, 0);
+        ew[qd][0] = a.x; ew[qd][1] = a.y; ew[qd][2] = a.z; ew[qd][3] = a.w;
+        ew[qd][4] = b.x; ew[qd][5] = b.y; ew[qd][6] = b.z; ew[qd][7] = b.w;
+      } else {
+#pragma unroll
+        for (int w8 = 0; w8 < 8; ++w8) {
+          uint32_t v = 0;
+#pragma unroll
+          for (int by = 0; by < 4; ++by)
+            if (4 * w8 + by < 2 * kr) v |= (uint32_t)er[4 * w8 + by] << (8 * by);
+          ew[qd][w8] = v;
+        }
       }
-      *reinterpret_cast<uint4 *>(atom + kg * 512) = make_uint4(words[0], words[1], words[2], words[3]);
+    }
+#pragma unroll
+    for (int i = 0; i < (int)kAtomRun; ++i) {
+      if (i < kr) {
+        uint32_t words[4];
+#pragma unroll
+        for (int qd = 0; qd < 4; ++qd) {
+          const uint32_t pair = ew[qd][i >> 1] >> (16 * (i & 1));     // UE8M0 bytes of blocks 2(kg0+i), +1
+          const uint32_t S0 = e4m3_pow2(max(-9, min(8, (int)(pair & 0xFFu) - 127 - g)));
+          const uint32_t S1 = e4m3_pow2(max(-9, min(8, (int)((pair >> 8) & 0xFFu) - 127 - g)));
+          words[qd] = S0 * 0x0101u | S1 * 0x01010000u;
+        }
+        *reinterpret_cast<uint4 *>(atom + (kg0 + i) * 512) = make_uint4(words[0], words[1], words[2], words[3]);
+      }
     }
   }
 }
@@ -206,8 +234,10 @@ extern "C" nvfp4_status mxfp4_to_nvfp4(const uint8_t *q_mx, const uint8_t *ue8m0
     const int64_t units = n_tensors * (rows / 128) * ((K / 64 + kAtomRun - 1) / kAtomRun);
     int64_t blocks = (units + 7) / 8;                      // a warp per unit, 8 warps per CTA
     if (blocks > (int64_t)sms * 8) blocks = (int64_t)sms * 8;
+    // 16-byte exponent loads need 16-byte aligned rows of exponents
+    const bool vec = (reinterpret_cast<uintptr_t>(ue8m0) & 15u) == 0 && (K / 32) % 16 == 0;
     remap_scale_atoms_kernel<<<(unsigned)blocks, 256, 0, stream>>>(ue8m0, rows, K, n_tensors, ws, sf_nv, global_scale,
-                                                                   dev_status);
+                                                                   vec, dev_status);
   } else {
     const int64_t total = n_tensors * bpt;
     int64_t blocks = (total + 255) / 256;

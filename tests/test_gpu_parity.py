@@ -342,17 +342,27 @@ def _mx(seed, n, rows, K, lo=-10):
     return q, e
 
 
+# Shapes for the scale pass's paths: 16-byte exponent loads with runs of 8 or
+# 16 scale groups (K = 512, 1024), byte loads (K/32 not a multiple of 16:
+# K = 128, 1152, 2112) with partial runs (1152: 16 + 2 groups, 2112: 16+16+1),
+# and an exponent pointer that is not 16-byte aligned.
 @pytest.mark.parametrize("layout", [0, 1])
-def test_remap_bitexact(layout):
+@pytest.mark.parametrize("n,rows,K,e_offset", [(3, 128, 512, 0), (2, 256, 128, 0), (1, 128, 1024, 0),
+                                               (2, 128, 1152, 0), (1, 256, 2112, 0), (1, 128, 1024, 1)])
+def test_remap_bitexact(layout, n, rows, K, e_offset):
     L = layer()
-    n, rows, K = 3, 128, 512
     q, e = _mx(0, n, rows, K)
     q[5, :16] = 0x88                            # one all -0 block (exempt)
     e[5, 0] = 3
     q_ref, sf_ref, gs_ref, st = oracle.remap_mxfp4(q, e, n, rows, K)
     assert st == 0
     s = status_word()
-    p = L.remap_mxfp4(to_dev(q), to_dev(e), n, rows, K, layout=layout, dev_status=s)
+    e_dev = to_dev(e)
+    if e_offset:
+        buf = torch.empty(e.size + 16, dtype=torch.uint8, device="cuda")
+        e_dev = buf[e_offset:e_offset + e.size].view(e.shape)
+        e_dev.copy_(to_dev(e))
+    p = L.remap_mxfp4(to_dev(q), e_dev, n, rows, K, layout=layout, dev_status=s)
     torch.cuda.synchronize()
     assert int(s.item()) == 0
     assert np.array_equal(to_np(p.gs), gs_ref)
