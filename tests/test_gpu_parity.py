@@ -68,6 +68,32 @@ def test_quantize_dense_config1_bitexact(layout):
     assert np.array_equal(sf, sf_ref)
 
 
+@pytest.mark.parametrize("layout", [0, 1])
+def test_quantize_dense_16byte_aligned_input(layout):
+    """A dense input that is 16-byte but not 32-byte aligned takes the 16-byte
+    load forms of the amax pass and the encode; many chunks per warp and a
+    ragged last chunk (rows * K/16 not a multiple of 64) in the round-robin
+    deal of the encode."""
+    L = layer()
+    rows, K = 3001, 1088
+    x = synthetic.gaussian_bf16(2, synthetic.STREAMS["x"], (rows, K), outlier_frac=0.001)
+    q_ref, sf_ref, gs_ref, st = oracle.quantize(x)
+    assert st == 0
+    buf = torch.empty(rows * K + 64, dtype=torch.bfloat16, device="cuda")
+    base = (buf.data_ptr() // 2) % 16                          # elements past a 32-byte boundary
+    start = (16 - base) % 16 + 8                                # 16 bytes past a 32-byte boundary
+    xd = buf[start:start + rows * K].view(rows, K)
+    assert xd.data_ptr() % 32 == 16
+    xd.copy_(bf16_dev(x))
+    p = L.quantize(xd, layout=layout)
+    torch.cuda.synchronize()
+    assert to_np(p.gs)[0] == gs_ref[0]
+    assert np.array_equal(to_np(p.q)[:rows], q_ref)
+    sf = to_np(p.sf)
+    sf = untile(sf, rows, K // 16) if layout == 1 else sf.reshape(-1, K // 16)[:rows]
+    assert np.array_equal(sf, sf_ref)
+
+
 @pytest.mark.parametrize("layout,H", [(0, 512), (1, 512), (1, 4096), (0, 2048), (0, 2064)])
 def test_quantize_grouped_gather_bitexact(layout, H):
     L = layer()
