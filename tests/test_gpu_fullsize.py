@@ -311,8 +311,9 @@ def test_config5_remap_full_size_bitexact():
 def test_config2_dense_mlp_full_size():
     """Dense MLP, 4096 tokens, hidden 5120, intermediate 17408, X with 0.1 %
     outliers x50: both activation quantizes and both weight packings are
-    compared byte for byte, and every output element of both GEMMs is checked
-    (in chunks of 1024 weight rows)."""
+    compared byte for byte, every output element of both GEMMs is checked (in
+    chunks of 1024 weight rows), and the fused SwiGLU epilogue plus the
+    requantize of its h are checked against the same GEMM."""
     import synthetic.cuda as sc
     L = layer()
     M, H, I = 4096, 5120, 17408
@@ -350,4 +351,30 @@ def test_config2_dense_mlp_full_size():
             assert ok.all(), (stream, c0, err.max(), (err / bound).max())
 
         pool_map(check, range(0, N, 1024))
-        del aref, yh, qw, sfw
+        del aref, qw, sfw
+        if stream == "w_gate_up":
+            y1h = yh
+        del yh
+    # the fused form the bench times: SwiGLU in the gate_up epilogue (one group,
+    # interleaved gate/up rows), then h requantized from the epilogue's amax.
+    # The accumulators are the GEMM's above, so h is checked against the
+    # oracle SwiGLU of that fp32 output (one bf16 ulp), the amax exactly, and
+    # the requantized bytes against the oracle's quantize of the device's h.
+    from nvfp4_w4a4_quantized_04_b200 import GS_AMAX_GIVEN, nvfp4_quantize
+    wil = L.pack_weights(sc.gaussian_bf16(0, synthetic.STREAMS["w_gate_up"], (2 * I, H), sigma=0.02), 1, 2 * I,
+                         L.gate_up_interleave_index(1, I, "cuda"), ws)
+    h, amax = L.grouped_gemm_swiglu(a1, wil, 2 * I, dev_status=s)
+    torch.cuda.synchronize()
+    assert int(s.item()) == 0
+    h_gpu = to_np(h)
+    h_ref = oracle.swiglu(y1h)
+    d = np.abs(h_gpu.astype(np.int32) - h_ref.astype(np.int32))
+    assert (d <= 1).all() and (d == 0).mean() > 0.99
+    assert to_np(amax)[0] == np.abs(synthetic.bf16_bits_to_f32(h_gpu)).max()
+    a3 = L.empty_packed(M, I, 1, None, 1, "cuda")
+    nvfp4_quantize(h, M, I, I, None, None, 1, GS_AMAX_GIVEN, amax, a3.q, a3.sf, 1, ws, s)
+    torch.cuda.synchronize()
+    assert int(s.item()) == 0
+    qh, sfh, gsh, st = oracle.quantize(h_gpu)
+    assert st == 0 and to_np(amax)[0] == gsh[0]
+    assert np.array_equal(to_np(a3.q[:M]), qh) and np.array_equal(tiled_rows(a3.sf, 0, M, I), sfh)
