@@ -373,6 +373,20 @@ nvfp4_status nvfp4_grouped_gemm_w4a16(const void *x, int64_t ld_x, int64_t x_row
 nvfp4_status nvfp4_gemm_select_kernel(int mode);
 
 /*
+ * nvfp4_gemm_set_wait_budget -- a testing switch for the failure path of the
+ * one-CTA grouped GEMM (nvfp4_gemm_select_kernel modes 0 and 1; not part of
+ * the pages' method).  Every wait of the kernel's main loop on a ring,
+ * scale or accumulator barrier gives up after this many SM clock cycles: it
+ * raises the CTA's abort flag, writes NVFP4_ERR_TIMEOUT to dev_status, and
+ * every role leaves its loop.  The closing waits for copies and MMAs still in
+ * flight keep the full budget, so the kernel ends cleanly and the context
+ * stays usable.  cycles = 0 restores the default (4e9 cycles, about 2 s); a
+ * test sets 1 to force the timeout.  Process-wide, synchronous; call it
+ * between launches.  Returns NVFP4_ERR_INVALID_ARG for cycles < 0.
+ */
+nvfp4_status nvfp4_gemm_set_wait_budget(int64_t cycles);
+
+/*
  * nvfp4_swiglu_quantize -- the step between the two expert projections:
  * h = bf16(silu(g) * u) with g = y[:, :I] (gate rows of the fused gate_up
  * weight come first) and u = y[:, I:], then h is NVFP4-quantized per expert

@@ -49,7 +49,7 @@ EXPORTS = [
     "nvfp4_moe_route_workspace_size", "nvfp4_moe_route", "nvfp4_moe_combine", "nvfp4_moe_quantize",
     "nvfp4_gemm_select_kernel", "nvfp4_grouped_gemm_w4a16", "nvfp4_grouped_gemm_swiglu_nvfp4",
     "mxfp4_quantize", "mxfp4_grouped_gemm", "nvfp4_w4a16_workspace_size",
-    "nvfp4_e2m1_encode", "nvfp4_e4m3_encode",
+    "nvfp4_e2m1_encode", "nvfp4_e4m3_encode", "nvfp4_gemm_set_wait_budget",
 ]
 NOALLOC_MAX_GROUPS = 1024
 
@@ -111,6 +111,8 @@ def load_library(path: str = LIB_PATH):
     L.nvfp4_moe_combine.argtypes = [P, i32, i64, P, P, i64, i32, i64, P, i32, P, P]
     L.nvfp4_kv_dequantize.restype = i32
     L.nvfp4_kv_dequantize.argtypes = [P, P, P, P, P, P, i64, i64, i64, P, P, P]
+    L.nvfp4_gemm_set_wait_budget.restype = i32
+    L.nvfp4_gemm_set_wait_budget.argtypes = [i64]
     L.nvfp4_e2m1_encode.restype = i32
     L.nvfp4_e2m1_encode.argtypes = [P, i64, P, P]
     L.nvfp4_e4m3_encode.restype = i32
@@ -192,6 +194,14 @@ def nvfp4_grouped_gemm_w4a16(x, ld_x, x_rows, row_index, b_q, b_sf, b_gs, expert
         num_experts, M_total, N, K, _ptr(y), out_dtype, epi, _ptr(workspace), _ptr(dev_status), _stream(stream))
     if check:
         _check(st, "nvfp4_grouped_gemm_w4a16")
+    return st
+
+
+def nvfp4_gemm_set_wait_budget(cycles: int) -> int:
+    """Main-loop wait budget of the one-CTA grouped GEMM in SM cycles (0 = default);
+    a switch for testing the timeout path."""
+    st = load_library().nvfp4_gemm_set_wait_budget(cycles)
+    _check(st, "nvfp4_gemm_set_wait_budget")
     return st
 
 

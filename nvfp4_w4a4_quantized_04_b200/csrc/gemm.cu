@@ -354,6 +354,12 @@ extern "C" nvfp4_status nvfp4_grouped_gemm(const uint8_t *a_q, const uint8_t *a_
   return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 
+extern "C" nvfp4_status nvfp4_gemm_set_wait_budget(int64_t cycles) {
+  if (cycles < 0) return NVFP4_ERR_INVALID_ARG;
+  const long long v = cycles == 0 ? gemm::kWaitBudgetCycles : (long long)cycles;
+  return cudaMemcpyToSymbol(gemm::c_wait_budget, &v, sizeof(v)) == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
 extern "C" nvfp4_status nvfp4_gemm_select_kernel(int mode) {
   if (mode < 0 || mode > 2) return NVFP4_ERR_INVALID_ARG;
   g_gemm_kernel = mode;

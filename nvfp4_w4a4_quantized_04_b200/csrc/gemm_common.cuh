@@ -32,6 +32,11 @@ constexpr uint32_t TMEM_ACC_STRIDE = BN;       // accumulator b at column b*192
 constexpr uint32_t TMEM_SF = 2 * BN;           // scale buffers at 384 and 448
 constexpr uint32_t TMEM_SF_STRIDE = 64;        // per buffer: W scales 16 cols, token scales 32 cols
 constexpr long long kWaitBudgetCycles = 4000000000LL;   // ~2 s at 2 GHz
+// Budget of the main-loop waits (mbar_wait), one copy per translation unit.
+// Only a test lowers it (nvfp4_gemm_set_wait_budget, one-CTA kernel) to force
+// the timeout path; the drains at the end of a kernel always use
+// kWaitBudgetCycles, so no copy or MMA is ever left in flight.
+static __constant__ long long c_wait_budget = kWaitBudgetCycles;
 
 // warp roles (warps 2..5: epilogue, lane quadrants 2,3,0,1)
 constexpr int W_PRODUCER = 0;     // weight tiles + weight scales
@@ -66,6 +71,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking form: returns at once whether the phase has completed.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile("{ .reg .pred p; mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+               : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+  return ok != 0;
+}
+
 // Same, with cluster-scope acquire: for barriers that the peer CTA of a pair
 // arrives on remotely.
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
@@ -88,13 +101,19 @@ __device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v) {
 template <bool kCluster = false>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
                                           int32_t *dev_status, uint32_t peer_abort = 0) {
-  auto try_once = [&]() { return kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
+  // try_wait may suspend the thread inside the instruction until the phase
+  // completes, so a lowered (test) budget polls with test_wait instead
+  const bool poll = !kCluster && c_wait_budget < kWaitBudgetCycles;
+  auto try_once = [&]() {
+    if (poll) return mbar_test_wait(bar, parity);
+    return kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity);
+  };
   if (try_once()) return true;
   const long long t0 = clock64();
   while (true) {
     if (try_once()) return true;
     if (*abort_flag) return false;
-    if (clock64() - t0 > kWaitBudgetCycles) {
+    if (clock64() - t0 > c_wait_budget) {
       *abort_flag = 1;
       if (peer_abort) st_cluster_u32(peer_abort, 1u);
       report(dev_status, NVFP4_ERR_TIMEOUT);

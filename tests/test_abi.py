@@ -78,6 +78,8 @@ def test_host_validation_without_device(lib):
     assert L.nvfp4_quantize(fake, 4, 32, 32, None, None, 1, 3, fake, fake, fake, 0, fake, None, None) == nv.ERR_INVALID_ARG
     # empty problems are no-ops that touch nothing
     assert L.nvfp4_grouped_gemm(None, None, None, None, None, None, None, 1, 0, 128, 512, None, 0, 0, None, None, None, None) == nv.OK
+    # the wait-budget switch rejects a negative budget before touching the device
+    assert L.nvfp4_gemm_set_wait_budget(-1) == nv.ERR_INVALID_ARG
     # element-wise codecs: length multiple of 8 (E2M1) or 4 (E4M3), aligned pointers
     assert L.nvfp4_e2m1_encode(fake, 12, fake, None) == nv.ERR_UNSUPPORTED_SHAPE
     assert L.nvfp4_e2m1_encode(fake, -8, fake, None) == nv.ERR_INVALID_ARG

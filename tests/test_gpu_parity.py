@@ -698,6 +698,45 @@ def test_gemm_dense_config1(out_dtype, gemm_kernel):
         assert np.array_equal(y, synthetic.f32_to_bf16_bits(y32))
 
 
+def test_gemm_wait_timeout_reports_and_recovers():
+    """The failure path of the one-CTA GEMM without any GPU fault: with a
+    1-cycle budget on its main-loop waits, the first wait that is not already
+    complete gives up, the kernel writes NVFP4_ERR_TIMEOUT to the status word
+    and ends (its closing waits for copies and MMAs in flight keep the full
+    budget).  With the budget restored, the same context runs the same GEMM
+    again and gets the result of a run made before the timeout, bit for bit."""
+    L = layer()
+    nv = nvmod()
+    E, N, K = 6, 256, 1024
+    counts = [0, 5, 130, 300, 16, 257]
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    R = int(offsets[-1])
+    x = synthetic.gaussian_bf16(21, synthetic.STREAMS["x"], (R, K))
+    w = synthetic.gaussian_bf16(21, synthetic.STREAMS["w"], (E * N, K), sigma=0.02)
+    q, sf, gs, qs, ss = _packed_acts(x, None, offsets, E)
+    qw, sw, gw = _packed_weights(w, E, N, K)
+    nv.nvfp4_gemm_select_kernel(1)
+    try:
+        y_before = _run_gemm(qs, ss, gs, qw, sw, gw, offsets, E, R, N, K, 0)
+        bound = nv.nvfp4_padded_rows_bound(R, E)
+        qa = np.zeros((bound, K // 2), np.uint8)
+        qa[:qs.shape[0]] = qs
+        sa = np.zeros((((bound + 127) // 128) * 128, K // 16), np.uint8)
+        sa[:ss.shape[0]] = ss
+        a = L.Packed(to_dev(qa), to_dev(tile(sa)), to_dev(gs), R, K, 1, to_dev(offsets), E)
+        wp = L.Packed(to_dev(qw), to_dev(tile(sw)), to_dev(gw), qw.shape[0], K, 1)
+        nv.nvfp4_gemm_set_wait_budget(1)
+        s = status_word()
+        L.grouped_gemm(a, wp, N, 0, dev_status=s)
+        torch.cuda.synchronize()
+        assert int(s.item()) == nv.ERR_TIMEOUT
+    finally:
+        nv.nvfp4_gemm_set_wait_budget(0)
+        nv.nvfp4_gemm_select_kernel(0)
+    y_after = _run_gemm(qs, ss, gs, qw, sw, gw, offsets, E, R, N, K, 0)
+    assert np.array_equal(y_after, y_before)
+
+
 def test_gemm_grouped_ragged(gemm_kernel):
     E, N, K = 6, 256, 512
     counts = [0, 5, 130, 300, 16, 257]
