@@ -328,6 +328,27 @@ def test_quantize_given_scale_and_nonfinite_status():
             assert int(s.item()) == oracle.ERR_NONFINITE == 16
 
 
+def test_status_word_first_error_wins():
+    """The device status word keeps the first error: a word already holding an
+    error (here NOT_REPRESENTABLE, as if a remap had failed) is not overwritten
+    by a quantize that meets a NaN, and a word holding NONFINITE is not
+    overwritten by a routing call that meets an expert id out of range."""
+    L = layer()
+    x = synthetic.gaussian_bf16(3, synthetic.STREAMS["x"], (64, 256))
+    x[7, 9] = 0x7FC0                                       # NaN
+    s = torch.full((1,), 17, dtype=torch.int32, device="cuda")
+    L.quantize(bf16_dev(x), layout=0, dev_status=s)
+    torch.cuda.synchronize()
+    assert int(s.item()) == 17
+    s = status_word()
+    L.quantize(bf16_dev(x), layout=0, dev_status=s)
+    torch.cuda.synchronize()
+    assert int(s.item()) == 16
+    L.route(to_dev(np.array([[0, 1], [2, 9]], dtype=np.int32)), 4, dev_status=s)
+    torch.cuda.synchronize()
+    assert int(s.item()) == 16
+
+
 # --------------------------------------------------------------------------- dequantize
 @pytest.mark.parametrize("layout", [0, 1])
 def test_dequantize_bitexact(layout):
