@@ -363,10 +363,12 @@ nvfp4_status nvfp4_grouped_gemm_w4a16(const void *x, int64_t ld_x, int64_t x_row
 /*
  * nvfp4_gemm_select_kernel -- which grouped GEMM kernel nvfp4_grouped_gemm runs
  * (process-wide; a tuning and testing switch, not part of the pages' method):
- *   0  automatic (default): one CTA per 128-row weight tile (measured as fast
- *      as or faster than the pair kernel on the MoE shapes);
- *   1  one CTA per tile;  2  CTA pairs (tcgen05 cta_group::2, 256 weight rows
- *      per tile; N % 256 != 0 is then NVFP4_ERR_UNSUPPORTED_SHAPE).
+ *   0  automatic (default): one CTA per 128-row weight tile, with 512-element
+ *      K stages when K % 512 == 0 (NVFP4 operands) and 256-element stages
+ *      otherwise;
+ *   1  one CTA per tile, 256-element K stages;  2  CTA pairs (tcgen05
+ *      cta_group::2, 256 weight rows per tile; N % 256 != 0 is then
+ *      NVFP4_ERR_UNSUPPORTED_SHAPE).
  * Both give the same Y up to the fp32 accumulation order inside a tile.
  * Returns NVFP4_ERR_INVALID_ARG for another mode.
  */
@@ -374,8 +376,8 @@ nvfp4_status nvfp4_gemm_select_kernel(int mode);
 
 /*
  * nvfp4_gemm_set_wait_budget -- a testing switch for the failure path of the
- * one-CTA grouped GEMM (nvfp4_gemm_select_kernel modes 0 and 1; not part of
- * the pages' method).  Every wait of the kernel's main loop on a ring,
+ * one-CTA grouped GEMM kernels (nvfp4_gemm_select_kernel modes 0 and 1, both
+ * K-stage sizes; not part of the pages' method).  Every wait of the kernel's main loop on a ring,
  * scale or accumulator barrier gives up after this many SM clock cycles: it
  * raises the CTA's abort flag, writes NVFP4_ERR_TIMEOUT to dev_status, and
  * every role leaves its loop.  The closing waits for copies and MMAs still in

@@ -297,7 +297,9 @@ using namespace nvfp4;
 namespace {
 
 int g_sms = 0;
-int g_gemm_kernel = 0;      // 0 automatic (one CTA per tile), 1 one CTA per tile, 2 CTA pairs
+// 0 automatic (512-element stages when K % 512 == 0, else one CTA per tile with
+// 256-element stages), 1 one CTA per tile with 256-element stages, 2 CTA pairs
+int g_gemm_kernel = 0;
 bool g_attr_set[6] = {false, false, false, false, false, false};
 
 }  // namespace
@@ -328,6 +330,9 @@ extern "C" nvfp4_status nvfp4_grouped_gemm(const uint8_t *a_q, const uint8_t *a_
   if (g_gemm_kernel == 2)
     return gemm::launch_grouped_gemm_pair(a_q, a_sf, a_gs, b_q, b_sf, b_gs, expert_offsets, E, M_total, N, K, y,
                                           out_dtype, swiglu, amax_out, dev_status, stream);
+  if (g_gemm_kernel == 0 && K % 512 == 0)
+    return gemm::launch_grouped_gemm_k512(a_q, a_sf, a_gs, b_q, b_sf, b_gs, expert_offsets, E, M_total, N, K, y,
+                                          out_dtype, swiglu, amax_out, nullptr, dev_status, stream);
   const int64_t x_rows = nvfp4_padded_rows_bound(M_total, E);
   CUtensorMap tw, tx128, tx64, tx32;
   if (!gemm::make_map(&tw, b_q, (uint64_t)E * N, (uint64_t)K / 2, 128)) return NVFP4_ERR_CUDA;
@@ -357,7 +362,8 @@ extern "C" nvfp4_status nvfp4_grouped_gemm(const uint8_t *a_q, const uint8_t *a_
 extern "C" nvfp4_status nvfp4_gemm_set_wait_budget(int64_t cycles) {
   if (cycles < 0) return NVFP4_ERR_INVALID_ARG;
   const long long v = cycles == 0 ? gemm::kWaitBudgetCycles : (long long)cycles;
-  return cudaMemcpyToSymbol(gemm::c_wait_budget, &v, sizeof(v)) == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+  if (cudaMemcpyToSymbol(gemm::c_wait_budget, &v, sizeof(v)) != cudaSuccess) return NVFP4_ERR_CUDA;
+  return gemm::set_wait_budget_k512(v);
 }
 
 extern "C" nvfp4_status nvfp4_gemm_select_kernel(int mode) {
@@ -383,6 +389,13 @@ extern "C" nvfp4_status nvfp4_grouped_gemm_swiglu_nvfp4(const uint8_t *a_q, cons
   if ((reinterpret_cast<uintptr_t>(a_q) | reinterpret_cast<uintptr_t>(b_q) | reinterpret_cast<uintptr_t>(a_sf) |
        reinterpret_cast<uintptr_t>(b_sf) | reinterpret_cast<uintptr_t>(h_q)) & 15u)
     return NVFP4_ERR_INVALID_ARG;
+  gemm::HQuantOut hq;
+  hq.gs = h_gs;
+  hq.q = h_q;
+  hq.sf = h_sf;
+  if (g_gemm_kernel == 0 && K % 512 == 0)
+    return gemm::launch_grouped_gemm_k512(a_q, a_sf, a_gs, b_q, b_sf, b_gs, expert_offsets, E, M_total, N, K, nullptr,
+                                          NVFP4_OUT_BF16, true, nullptr, &hq, dev_status, stream);
   const int64_t x_rows = nvfp4_padded_rows_bound(M_total, E);
   CUtensorMap tw, tx128, tx64, tx32;
   if (!gemm::make_map(&tw, b_q, (uint64_t)E * N, (uint64_t)K / 2, 128)) return NVFP4_ERR_CUDA;
@@ -401,10 +414,6 @@ extern "C" nvfp4_status nvfp4_grouped_gemm_swiglu_nvfp4(const uint8_t *a_q, cons
       return NVFP4_ERR_CUDA;
     g_attr_set[3] = true;
   }
-  gemm::HQuantOut hq;
-  hq.gs = h_gs;
-  hq.q = h_q;
-  hq.sf = h_sf;
   kern<<<g_sms, gemm::NUM_THREADS, gemm::SMEM_BYTES, stream>>>(tw, tx128, tx64, tx32, b_sf, a_sf, b_gs, a_gs,
                                                                expert_offsets, E, (int)M_total, (int)N, (int)K, nullptr,
                                                                nullptr, dev_status, hq);

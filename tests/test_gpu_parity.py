@@ -36,9 +36,11 @@ def status_word():
     return torch.zeros(1, dtype=torch.int32, device="cuda")
 
 
-@pytest.fixture(params=[1, 2], ids=["one_cta", "cta_pair"])
+@pytest.fixture(params=[0, 1, 2], ids=["auto", "one_cta", "cta_pair"])
 def gemm_kernel(request):
-    """Run the test on the one-CTA grouped GEMM and on the CTA-pair kernel."""
+    """Run the test on each grouped GEMM kernel: automatic (512-element K
+    stages when K % 512 == 0), one CTA per tile with 256-element stages, and
+    the CTA-pair kernel."""
     nv = nvmod()
     nv.nvfp4_gemm_select_kernel(request.param)
     yield request.param
@@ -719,7 +721,8 @@ def test_gemm_dense_config1(out_dtype, gemm_kernel):
         assert np.array_equal(y, synthetic.f32_to_bf16_bits(y32))
 
 
-def test_gemm_wait_timeout_reports_and_recovers():
+@pytest.mark.parametrize("mode", [0, 1], ids=["k512", "k256"])
+def test_gemm_wait_timeout_reports_and_recovers(mode):
     """The failure path of the one-CTA GEMM without any GPU fault: with a
     1-cycle budget on its main-loop waits, the first wait that is not already
     complete gives up, the kernel writes NVFP4_ERR_TIMEOUT to the status word
@@ -736,7 +739,7 @@ def test_gemm_wait_timeout_reports_and_recovers():
     w = synthetic.gaussian_bf16(21, synthetic.STREAMS["w"], (E * N, K), sigma=0.02)
     q, sf, gs, qs, ss = _packed_acts(x, None, offsets, E)
     qw, sw, gw = _packed_weights(w, E, N, K)
-    nv.nvfp4_gemm_select_kernel(1)
+    nv.nvfp4_gemm_select_kernel(mode)
     try:
         y_before = _run_gemm(qs, ss, gs, qw, sw, gw, offsets, E, R, N, K, 0)
         bound = nv.nvfp4_padded_rows_bound(R, E)
@@ -751,11 +754,35 @@ def test_gemm_wait_timeout_reports_and_recovers():
         L.grouped_gemm(a, wp, N, 0, dev_status=s)
         torch.cuda.synchronize()
         assert int(s.item()) == nv.ERR_TIMEOUT
+        nv.nvfp4_gemm_set_wait_budget(0)
+        y_after = _run_gemm(qs, ss, gs, qw, sw, gw, offsets, E, R, N, K, 0)
     finally:
         nv.nvfp4_gemm_set_wait_budget(0)
         nv.nvfp4_gemm_select_kernel(0)
-    y_after = _run_gemm(qs, ss, gs, qw, sw, gw, offsets, E, R, N, K, 0)
     assert np.array_equal(y_after, y_before)
+
+
+def test_gemm_k_not_multiple_of_512():
+    """K = 1280 (a multiple of 256, not of 512): the automatic choice falls back
+    to the 256-element-stage kernel; ragged groups, fp32 out, within the bound."""
+    E, N, K = 3, 256, 1280
+    counts = [77, 0, 190]
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    R = int(offsets[-1])
+    x = synthetic.gaussian_bf16(22, synthetic.STREAMS["x"], (R, K))
+    w = synthetic.gaussian_bf16(22, synthetic.STREAMS["w"], (E * N, K), sigma=0.02)
+    q, sf, gs, qs, ss = _packed_acts(x, None, offsets, E)
+    qw, sw, gw = _packed_weights(w, E, N, K)
+    y = _run_gemm(qs, ss, gs, qw, sw, gw, offsets, E, R, N, K, 0)
+    for e in range(E):
+        r0, r1 = int(offsets[e]), int(offsets[e + 1])
+        if r0 == r1:
+            continue
+        a = oracle.dequantize_f64(q[r0:r1], sf[r0:r1], np.full(r1 - r0, gs[e], np.float32))
+        b = oracle.dequantize_f64(qw[e * N:(e + 1) * N], sw[e * N:(e + 1) * N], np.full(N, gw[e], np.float32))
+        y_ref, s_ref = oracle.gemm_f64(a, b)
+        ok, err, bound = gemm_tol(y[r0:r1], y_ref, s_ref)
+        assert ok.all(), (e, err.max(), (err / bound).max())
 
 
 def test_gemm_grouped_ragged(gemm_kernel):
