@@ -332,7 +332,7 @@ extern "C" nvfp4_status nvfp4_grouped_gemm(const uint8_t *a_q, const uint8_t *a_
                                           out_dtype, swiglu, amax_out, dev_status, stream);
   if (g_gemm_kernel == 0 && K % 512 == 0)
     return gemm::launch_grouped_gemm_k512(a_q, a_sf, a_gs, b_q, b_sf, b_gs, expert_offsets, E, M_total, N, K, y,
-                                          out_dtype, swiglu, amax_out, nullptr, dev_status, stream);
+                                          out_dtype, swiglu, amax_out, nullptr, false, dev_status, stream);
   const int64_t x_rows = nvfp4_padded_rows_bound(M_total, E);
   CUtensorMap tw, tx128, tx64, tx32;
   if (!gemm::make_map(&tw, b_q, (uint64_t)E * N, (uint64_t)K / 2, 128)) return NVFP4_ERR_CUDA;
@@ -395,7 +395,7 @@ extern "C" nvfp4_status nvfp4_grouped_gemm_swiglu_nvfp4(const uint8_t *a_q, cons
   hq.sf = h_sf;
   if (g_gemm_kernel == 0 && K % 512 == 0)
     return gemm::launch_grouped_gemm_k512(a_q, a_sf, a_gs, b_q, b_sf, b_gs, expert_offsets, E, M_total, N, K, nullptr,
-                                          NVFP4_OUT_BF16, true, nullptr, &hq, dev_status, stream);
+                                          NVFP4_OUT_BF16, true, nullptr, &hq, false, dev_status, stream);
   const int64_t x_rows = nvfp4_padded_rows_bound(M_total, E);
   CUtensorMap tw, tx128, tx64, tx32;
   if (!gemm::make_map(&tw, b_q, (uint64_t)E * N, (uint64_t)K / 2, 128)) return NVFP4_ERR_CUDA;
@@ -439,6 +439,9 @@ extern "C" nvfp4_status mxfp4_grouped_gemm(const uint8_t *a_q, const uint8_t *a_
   if ((reinterpret_cast<uintptr_t>(a_q) | reinterpret_cast<uintptr_t>(b_q) | reinterpret_cast<uintptr_t>(a_sf) |
        reinterpret_cast<uintptr_t>(b_sf) | reinterpret_cast<uintptr_t>(y)) & 15u)
     return NVFP4_ERR_INVALID_ARG;
+  if (g_gemm_kernel == 0 && K % 512 == 0)
+    return gemm::launch_grouped_gemm_k512(a_q, a_sf, nullptr, b_q, b_sf, nullptr, expert_offsets, E, M_total, N, K, y,
+                                          out_dtype, false, nullptr, nullptr, true, dev_status, stream);
   const int64_t x_rows = nvfp4_padded_rows_bound(M_total, E);
   CUtensorMap tw, tx128, tx64, tx32;
   if (!gemm::make_map(&tw, b_q, (uint64_t)E * N, (uint64_t)K / 2, 128)) return NVFP4_ERR_CUDA;

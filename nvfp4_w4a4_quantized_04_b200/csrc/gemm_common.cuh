@@ -729,13 +729,14 @@ inline bool make_map_sfw(CUtensorMap *map, const void *base, uint64_t row_blocks
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// The 512-element-stage kernel's launch (gemm_k512.cu), NVFP4 operands,
-// K % 512 == 0; hq != nullptr selects the SwiGLU epilogue that writes NVFP4 h.
+// The 512-element-stage kernel's launch (gemm_k512.cu), K % 512 == 0;
+// hq != nullptr selects the SwiGLU epilogue that writes NVFP4 h; mx selects
+// MXFP4 operands (no global scales: a_gs and b_gs are not read).
 nvfp4_status launch_grouped_gemm_k512(const uint8_t *a_q, const uint8_t *a_sf, const float *a_gs,
                                       const uint8_t *b_q, const uint8_t *b_sf, const float *b_gs,
                                       const int32_t *expert_offsets, int E, int64_t M_total, int64_t N, int64_t K,
                                       void *y, nvfp4_out_dtype out_dtype, bool swiglu, float *amax_out,
-                                      const HQuantOut *hq, int32_t *dev_status, cudaStream_t stream);
+                                      const HQuantOut *hq, bool mx, int32_t *dev_status, cudaStream_t stream);
 // Its copy of the main-loop wait budget (see c_wait_budget).
 nvfp4_status set_wait_budget_k512(long long cycles);
 

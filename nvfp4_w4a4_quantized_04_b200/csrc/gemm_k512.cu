@@ -17,7 +17,8 @@
 // the smallest that holds the tile's tokens.  Measured against the 256-element
 // kernel, bit-identical: 2.5-3 % faster on the 512-expert MoE shapes and 8-12 %
 // on decode (1-3 tokens per expert), where a stage is mostly weight bytes.
-// Used when K % 512 == 0 (nvfp4_gemm_select_kernel mode 0).
+// Used when K % 512 == 0 (nvfp4_gemm_select_kernel mode 0), for NVFP4 and for
+// MXFP4 operands (kind::mxf4, UE8M0 scales per 32 elements, no global scales).
 #include "gemm_common.cuh"
 
 namespace nvfp4 {
@@ -61,7 +62,37 @@ __device__ __forceinline__ void sf_half_to_tmem(uint32_t tcol, uint32_t sfw_addr
   tc_wait_st();
 }
 
-template <bool kSwiglu, bool kBf16Out, bool kQuantH>
+// MXFP4 form: a 512-byte atom holds 4 UE8M0 scales per row = 128 elements =
+// two MMAs, so a 256-element half has two atoms per row block; each MMA gets
+// its own 4 tensor-memory columns with its two scales in bytes 0 and 1 (the
+// 256-element kernel's sf_stage_to_tmem_mx, second row block 4 KB on).
+__device__ __forceinline__ void sf_half_to_tmem_mx(uint32_t tcol, uint32_t sfw_addr, uint32_t sfx_addr, int nrb) {
+#pragma unroll
+  for (int a = 0; a < 2; ++a) {
+    const uint4 w = lds128(sfw_addr + a * 512);
+    tc_st_x4(tcol + (2 * a) * 4, lo16x4(w));
+    tc_st_x4(tcol + (2 * a + 1) * 4, hi16x4(w));
+  }
+#pragma unroll
+  for (int a = 0; a < 2; ++a) {
+    const uint4 x = lds128(sfx_addr + a * 512);
+    tc_st_x4(tcol + 16 + (2 * a) * 8, lo16x4(x));
+    tc_st_x4(tcol + 16 + (2 * a + 1) * 8, hi16x4(x));
+  }
+  if (nrb > 1) {
+#pragma unroll
+    for (int a = 0; a < 2; ++a) {
+      const uint4 x = lds128(sfx_addr + 4096 + a * 512);
+      tc_st_x4(tcol + 16 + (2 * a) * 8 + 4, lo16x4(x));
+      tc_st_x4(tcol + 16 + (2 * a + 1) * 8 + 4, hi16x4(x));
+    }
+  }
+  tc_wait_st();
+}
+
+// kMx: MXFP4 operands (kind::mxf4, one UE8M0 scale per 32 elements, no global
+// scales); otherwise NVFP4 (kind::mxf4nvf4, E4M3 per 16 elements).
+template <bool kSwiglu, bool kBf16Out, bool kQuantH, bool kMx>
 __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_k512_kernel(
     const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x32,
     const __grid_constant__ CUtensorMap tmap_x64, const __grid_constant__ CUtensorMap tmap_x128,
@@ -117,7 +148,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_k512_kernel(
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
   const int total_tiles = s_tile[E];
-  const int64_t sf_row_stride = (int64_t)(K / 64) * 512;
+  // bytes per 128-row block of scales, and per 256-element half of one row block
+  const int64_t sf_row_stride = (int64_t)(K / (kMx ? 128 : 64)) * 512;
+  constexpr uint32_t kHalfSf = kMx ? 1024u : 2048u;
 
   if (warp == W_PRODUCER || warp == W_XLOAD) {
     if (lane == 0) {
@@ -134,7 +167,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_k512_kernel(
         const int nrb = ((T.x_row0 & 127) + T.n_valid + 127) >> 7;
         const int xbox = token_box_rows(T.n_valid);
         const CUtensorMap *xmap = xbox == 32 ? &tmap_x32 : xbox == 64 ? &tmap_x64 : xbox == 128 ? &tmap_x128 : &tmap_x192;
-        const uint32_t bytes = is_w ? (uint32_t)(W_STAGE2 + SFW_STAGE2) : (uint32_t)(2 * xbox * 128 + nrb * 4096);
+        const uint32_t bytes = is_w ? (uint32_t)(W_STAGE2 + 2 * kHalfSf) : (uint32_t)(2 * xbox * 128 + nrb * 2 * kHalfSf);
         const uint8_t *sfw_tile = w_sf + (int64_t)(T.w_row0 >> 7) * sf_row_stride;
         const uint8_t *sfx_tile = x_sf + (int64_t)(xr0 >> 7) * sf_row_stride;
         for (int ks = 0; ks < ksteps; ++ks) {
@@ -144,11 +177,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_k512_kernel(
           armed[stage] = true; armed_parity[stage] = phase;
           if (is_w) {
             tma_load_3d(sbase + OFF_W + stage * W_STAGE2, &tmap_w, 0, T.w_row0, 2 * ks, fb, pol);
-            bulk_load(sbase + OFF_SFW + stage * SFW_STAGE2, sfw_tile + ks * 4096, 4096, fb);
+            bulk_load(sbase + OFF_SFW + stage * SFW_STAGE2, sfw_tile + ks * 2 * kHalfSf, 2 * kHalfSf, fb);
           } else {
             for (int rb = 0; rb < nrb; ++rb)
-              bulk_load(sbase + OFF_SFX + stage * SFX_STAGE2 + rb * 4096, sfx_tile + rb * sf_row_stride + ks * 4096,
-                        4096, fb);
+              bulk_load(sbase + OFF_SFX + stage * SFX_STAGE2 + rb * 4096, sfx_tile + rb * sf_row_stride + ks * 2 * kHalfSf,
+                        2 * kHalfSf, fb);
             tma_load_3d(sbase + OFF_X + stage * X_STAGE2, xmap, 0, T.x_row0, 2 * ks, fb, pol);
           }
           if (++stage == 2) { stage = 0; phase ^= 1; }
@@ -178,8 +211,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_k512_kernel(
           }
           tc_fence_after();
           const uint32_t tcol = tmem_base + lane_base + TMEM_SF + sb * TMEM_SF_STRIDE;
-          sf_half_to_tmem(tcol, sbase + OFF_SFW + s2 * SFW_STAGE2 + h * 2048 + lane * 16,
-                          sbase + OFF_SFX + s2 * SFX_STAGE2 + h * 2048 + lane * 16, nrb);
+          if constexpr (kMx)
+            sf_half_to_tmem_mx(tcol, sbase + OFF_SFW + s2 * SFW_STAGE2 + h * kHalfSf + lane * 16,
+                               sbase + OFF_SFX + s2 * SFX_STAGE2 + h * kHalfSf + lane * 16, nrb);
+          else
+            sf_half_to_tmem(tcol, sbase + OFF_SFW + s2 * SFW_STAGE2 + h * kHalfSf + lane * 16,
+                            sbase + OFF_SFX + s2 * SFX_STAGE2 + h * kHalfSf + lane * 16, nrb);
           tc_fence_before();
           mbar_arrive(bar_sf_full + 8 * sb);
         }
@@ -191,7 +228,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_k512_kernel(
     for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++titer) {
       const Tile T = decode_tile<kSwiglu>(t, s_off, s_slot, s_tile, E, N, BM, 0);
       const uint32_t n_mma = (T.n_valid + 15) & ~15;
-      const uint32_t idesc = idesc_mxf4nvf4(BM, n_mma);
+      const uint32_t idesc = kMx ? idesc_mxf4_ue8m0(BM, n_mma) : idesc_mxf4nvf4(BM, n_mma);
       const uint32_t x_half = (uint32_t)token_box_rows(T.n_valid) * 128;   // bytes of one K half of the token tile
       const uint32_t xoff = (uint32_t)(T.x_row0 & 127) >> 5;
       const uint32_t ab = titer & 1;
@@ -212,8 +249,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_k512_kernel(
             const uint64_t dx = desc_sw128(sbase + OFF_X + s2 * X_STAGE2 + h * x_half);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-              tc_mma(t_acc, dw + 2 * kk, dx + 2 * kk, idesc, t_sf + kk * 4, t_sf + 16 + kk * 8 + xoff,
-                     (ks > 0 || h > 0 || kk > 0) ? 1u : 0u);
+              if constexpr (kMx)
+                tc_mma_mx(t_acc, dw + 2 * kk, dx + 2 * kk, idesc, t_sf + kk * 4, t_sf + 16 + kk * 8 + xoff,
+                          (ks > 0 || h > 0 || kk > 0) ? 1u : 0u);
+              else
+                tc_mma(t_acc, dw + 2 * kk, dx + 2 * kk, idesc, t_sf + kk * 4, t_sf + 16 + kk * 8 + xoff,
+                       (ks > 0 || h > 0 || kk > 0) ? 1u : 0u);
             tc_commit(bar_sf_free + 8 * sb);
           }
           __syncwarp();
@@ -242,7 +283,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_k512_kernel(
       const uint32_t ab = titer & 1;
       if (!mbar_wait_warp(bar_acc_full + 8 * ab, (titer >> 1) & 1, abort_flag, dev_status)) break;
       tc_fence_after();
-      const float alpha = __fmul_rn(x_gs[T.e], w_gs[T.e]);
+      const float alpha = kMx ? 1.0f : __fmul_rn(x_gs[T.e], w_gs[T.e]);
       epilogue_tile<kSwiglu, kBf16Out, kQuantH>(T, tmem_base + lane_base + ab * TMEM_ACC_STRIDE, alpha, epi, quad,
                                                 lane, N, y, amax_out, bar_acc_empty + 8 * ab, false, hq, dev_status);
     }
@@ -282,9 +323,9 @@ nvfp4_status launch_grouped_gemm_k512(const uint8_t *a_q, const uint8_t *a_sf, c
                                       const uint8_t *b_q, const uint8_t *b_sf, const float *b_gs,
                                       const int32_t *expert_offsets, int E, int64_t M_total, int64_t N, int64_t K,
                                       void *y, nvfp4_out_dtype out_dtype, bool swiglu, float *amax_out,
-                                      const HQuantOut *hq, int32_t *dev_status, cudaStream_t stream) {
+                                      const HQuantOut *hq, bool mx, int32_t *dev_status, cudaStream_t stream) {
   static int sms = 0;
-  static bool attr_set[4] = {false, false, false, false};
+  static bool attr_set[6] = {false, false, false, false, false, false};
   const int64_t x_rows = nvfp4_padded_rows_bound(M_total, E);
   CUtensorMap tw, tx32, tx64, tx128, tx192;
   if (!make_map_k512(&tw, b_q, (uint64_t)E * N, (uint64_t)K / 2, 128)) return NVFP4_ERR_CUDA;
@@ -298,11 +339,14 @@ nvfp4_status launch_grouped_gemm_k512(const uint8_t *a_q, const uint8_t *a_sf, c
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (sms <= 0) sms = 148;
   }
-  const int variant = hq ? 3 : swiglu ? 2 : (out_dtype == NVFP4_OUT_BF16 ? 1 : 0);
-  auto kern = variant == 3   ? grouped_gemm_k512_kernel<true, true, true>
-              : variant == 2 ? grouped_gemm_k512_kernel<true, true, false>
-              : variant == 1 ? grouped_gemm_k512_kernel<false, true, false>
-                             : grouped_gemm_k512_kernel<false, false, false>;
+  const bool bf = out_dtype == NVFP4_OUT_BF16;
+  const int variant = mx ? (bf ? 5 : 4) : hq ? 3 : swiglu ? 2 : (bf ? 1 : 0);
+  auto kern = variant == 5   ? grouped_gemm_k512_kernel<false, true, false, true>
+              : variant == 4 ? grouped_gemm_k512_kernel<false, false, false, true>
+              : variant == 3 ? grouped_gemm_k512_kernel<true, true, true, false>
+              : variant == 2 ? grouped_gemm_k512_kernel<true, true, false, false>
+              : variant == 1 ? grouped_gemm_k512_kernel<false, true, false, false>
+                             : grouped_gemm_k512_kernel<false, false, false, false>;
   if (!attr_set[variant]) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess)
       return NVFP4_ERR_CUDA;

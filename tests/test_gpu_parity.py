@@ -47,6 +47,16 @@ def gemm_kernel(request):
     nv.nvfp4_gemm_select_kernel(0)
 
 
+@pytest.fixture(params=[0, 1], ids=["auto", "k256"])
+def mx_kernel(request):
+    """Run an MXFP4 GEMM test on both kernels that take MXFP4 operands: 512-element
+    K stages (automatic when K % 512 == 0) and 256-element stages."""
+    nv = nvmod()
+    nv.nvfp4_gemm_select_kernel(request.param)
+    yield request.param
+    nv.nvfp4_gemm_select_kernel(0)
+
+
 def gemm_tol(y, y_ref, s_ref):
     """|y - y_ref| <= 1e-5 * sum|a*b| + 1e-6 elementwise."""
     err = np.abs(y.astype(np.float64) - y_ref)
@@ -542,7 +552,7 @@ def _run_mx_gemm(x_bits, w_bits, offsets, E, N, K, out_dtype):
     return to_np(y), y_ref, s_ref
 
 
-def test_mx_gemm_closed_form_integer_case():
+def test_mx_gemm_closed_form_integer_case(mx_kernel):
     """All UE8M0 scales 1: every product is a multiple of 1/4 and the fp32 sum
     is exact, so the kind::mxf4 result must equal the oracle exactly."""
     L = layer()
@@ -564,7 +574,7 @@ def test_mx_gemm_closed_form_integer_case():
 
 
 @pytest.mark.parametrize("out_dtype", [0, 1])
-def test_mx_gemm_dense_many_tiles(out_dtype):
+def test_mx_gemm_dense_many_tiles(out_dtype, mx_kernel):
     M, N, K = 1000, 384, 1024
     x = synthetic.gaussian_bf16(41, synthetic.STREAMS["x"], (M, K), outlier_frac=0.001)
     w = synthetic.gaussian_bf16(41, synthetic.STREAMS["w"], (N, K), sigma=0.02)
@@ -576,7 +586,7 @@ def test_mx_gemm_dense_many_tiles(out_dtype):
         assert np.array_equal(y16, synthetic.f32_to_bf16_bits(y))
 
 
-def test_mx_gemm_grouped_chunk_edges():
+def test_mx_gemm_grouped_chunk_edges(mx_kernel):
     counts = [1, 63, 64, 65, 127, 128, 129, 191, 192, 193, 257, 385, 0, 2, 17, 33]
     E, N, K = len(counts), 256, 512
     offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
