@@ -772,6 +772,29 @@ def test_gemm_wait_timeout_reports_and_recovers(mode):
     assert np.array_equal(y_after, y_before)
 
 
+def test_gemm_max_experts(gemm_kernel):
+    """1024 experts, the most the GEMM's shared-memory tile tables hold: mostly
+    empty groups, a few with 1-3 rows and one with 200 (two token chunks)."""
+    rng = np.random.default_rng(23)
+    E, N, K = 1024, 256, 512
+    counts = np.where(rng.random(E) < 0.8, 0, rng.integers(1, 4, E))
+    counts[517] = 200
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    R = int(offsets[-1])
+    x = synthetic.gaussian_bf16(23, synthetic.STREAMS["x"], (R, K))
+    w = synthetic.gaussian_bf16(23, synthetic.STREAMS["w"], (E * N, K), sigma=0.02)
+    q, sf, gs, qs, ss = _packed_acts(x, None, offsets, E)
+    qw, sw, gw = _packed_weights(w, E, N, K)
+    y = _run_gemm(qs, ss, gs, qw, sw, gw, offsets, E, R, N, K, 0)
+    for e in np.nonzero(counts)[0]:
+        r0, r1 = int(offsets[e]), int(offsets[e + 1])
+        a = oracle.dequantize_f64(q[r0:r1], sf[r0:r1], np.full(r1 - r0, gs[e], np.float32))
+        b = oracle.dequantize_f64(qw[e * N:(e + 1) * N], sw[e * N:(e + 1) * N], np.full(N, gw[e], np.float32))
+        y_ref, s_ref = oracle.gemm_f64(a, b)
+        ok, err, bound = gemm_tol(y[r0:r1], y_ref, s_ref)
+        assert ok.all(), (int(e), err.max(), (err / bound).max())
+
+
 def test_gemm_k_not_multiple_of_512():
     """K = 1280 (a multiple of 256, not of 512): the automatic choice falls back
     to the 256-element-stage kernel; ragged groups, fp32 out, within the bound."""
