@@ -266,7 +266,7 @@ def run_headline(args, rank, world, device):
         lay.forward(x, ids_host.to(device), w_host.to(device))
     torch.cuda.synchronize()
     s_up, s_down = torch.cuda.Stream(device), torch.cuda.Stream(device)
-    n_e2e = max(4, min(3 * args.steps, 30))       # long enough that pipeline fill and drain amortise
+    n_e2e = max(4, min(6 * args.steps, 60))       # long enough that pipeline fill and drain amortise
     up_done = [torch.cuda.Event() for _ in range(n_e2e)]
     comp_done = [torch.cuda.Event() for _ in range(n_e2e)]
     down_done = [torch.cuda.Event() for _ in range(n_e2e)]
