@@ -795,6 +795,40 @@ def test_gemm_max_experts(gemm_kernel):
         assert ok.all(), (int(e), err.max(), (err / bound).max())
 
 
+def test_gemm_scale_bytes_over_the_whole_e4m3_range(gemm_kernel):
+    """Random E2M1 codes with block-scale bytes drawn from every non-negative
+    finite E4M3 value (0, the subnormals 2^-9 ... 7*2^-9, up to 448) on both
+    operands, and globals far from 1: the tensor core's reading of each scale
+    byte is checked against the fp64 oracle of the same packed operands."""
+    rng = np.random.default_rng(24)
+    E, N, K = 3, 256, 1024
+    counts = [130, 7, 64]
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    R = int(offsets[-1])
+    q = rng.integers(0, 256, (R, K // 2), dtype=np.uint8)
+    sf = rng.integers(0, 0x7F, (R, K // 16), dtype=np.uint8)          # 0x00 .. 0x7E
+    qw = rng.integers(0, 256, (E * N, K // 2), dtype=np.uint8)
+    sw = rng.integers(0, 0x7F, (E * N, K // 16), dtype=np.uint8)
+    sf[0, :8] = np.arange(8)                                           # zero and every subnormal
+    sw[1, :8] = 0x7E                                                   # 448
+    gs = np.array([2.0 ** -20, 3.5e-3, 1.25e2], dtype=np.float32)
+    gw = np.array([7.0e-4, 2.0 ** 10, 1.0], dtype=np.float32)
+    rows, starts = slot_rows(offsets)
+    alloc = (max(int(starts[-1]), 128) + 127) // 128 * 128
+    qs = np.zeros((alloc, K // 2), np.uint8)
+    ss = np.zeros((alloc, K // 16), np.uint8)
+    qs[rows] = q
+    ss[rows] = sf
+    y = _run_gemm(qs, ss, gs, qw, sw, gw, offsets, E, R, N, K, 0)
+    for e in range(E):
+        r0, r1 = int(offsets[e]), int(offsets[e + 1])
+        a = oracle.dequantize_f64(q[r0:r1], sf[r0:r1], np.full(r1 - r0, gs[e], np.float32))
+        b = oracle.dequantize_f64(qw[e * N:(e + 1) * N], sw[e * N:(e + 1) * N], np.full(N, gw[e], np.float32))
+        y_ref, s_ref = oracle.gemm_f64(a, b)
+        ok, err, bound = gemm_tol(y[r0:r1], y_ref, s_ref)
+        assert ok.all(), (e, err.max(), (err / bound).max())
+
+
 def test_gemm_k_not_multiple_of_512():
     """K = 1280 (a multiple of 256, not of 512): the automatic choice falls back
     to the 256-element-stage kernel; ragged groups, fp32 out, within the bound."""
