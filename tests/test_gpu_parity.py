@@ -552,6 +552,41 @@ def _run_mx_gemm(x_bits, w_bits, offsets, E, N, K, out_dtype):
     return to_np(y), y_ref, s_ref
 
 
+def test_mx_gemm_wide_exponent_range(mx_kernel):
+    """Random E2M1 codes with UE8M0 bytes spread over 2^-57 ... 2^53 on both
+    operands (products stay finite in fp32), some blocks at 2^-127: the
+    tensor core's reading of each exponent byte against the fp64 oracle."""
+    L = layer()
+    nv = nvmod()
+    rng = np.random.default_rng(25)
+    E, N, K = 2, 256, 1024
+    counts = [90, 150]
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    R = int(offsets[-1])
+    qa = rng.integers(0, 256, (R, K // 2), dtype=np.uint8)
+    ea = rng.integers(70, 181, (R, K // 32), dtype=np.uint8)
+    qw = rng.integers(0, 256, (E * N, K // 2), dtype=np.uint8)
+    ew = rng.integers(70, 181, (E * N, K // 32), dtype=np.uint8)
+    ea[3, :5] = 0                                                   # 2^-127
+    ew[7, :5] = 0
+    bound = nv.nvfp4_padded_rows_bound(R, E)
+    qs = np.zeros((bound, K // 2), np.uint8)
+    es = np.zeros((bound, K // 32), np.uint8)
+    rows, _ = slot_rows(offsets)
+    qs[rows] = qa
+    es[rows] = ea
+    s = status_word()
+    y = L.mx_grouped_gemm(to_dev(qs), to_dev(tile(es)), to_dev(qw), to_dev(tile(ew)), N, K, R,
+                          to_dev(offsets), E, 0, dev_status=s)
+    torch.cuda.synchronize()
+    assert int(s.item()) == 0
+    a = oracle.dequantize_mxfp4_f64(qa, ea)
+    b = oracle.dequantize_mxfp4_f64(qw, ew)
+    y_ref, s_ref = oracle.grouped_gemm_f64(a, b.reshape(E, N, K), offsets)
+    ok, err, bnd = gemm_tol(to_np(y), y_ref, s_ref)
+    assert ok.all(), (err.max(), (err / bnd).max())
+
+
 def test_mx_gemm_closed_form_integer_case(mx_kernel):
     """All UE8M0 scales 1: every product is a multiple of 1/4 and the fp32 sum
     is exact, so the kind::mxf4 result must equal the oracle exactly."""
