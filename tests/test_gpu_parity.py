@@ -1390,6 +1390,36 @@ def test_w4a16_grouped(K):
     assert np.array_equal(to_np(y16), synthetic.f32_to_bf16_bits(to_np(y)))
 
 
+def test_w4a16_scale_bytes_over_the_whole_e4m3_range():
+    """Weights with random codes and block-scale bytes over every non-negative
+    finite E4M3 value (zero, the subnormals, up to 448) and globals far from 1:
+    the kernel's f16 code x scale products must be exact over the whole range
+    (within the fp64 oracle's bound after accumulation)."""
+    L = layer()
+    rng = np.random.default_rng(33)
+    counts = [5, 12, 0, 30]
+    N, K, T = 256, 1024, 24
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    R, E = int(offsets[-1]), len(counts)
+    ri = rng.integers(0, T, R).astype(np.int32)
+    x = synthetic.gaussian_bf16(33, synthetic.STREAMS["x"], (T, K))
+    qw = rng.integers(0, 256, (E * N, K // 2), dtype=np.uint8)
+    sw = rng.integers(0, 0x7F, (E * N, K // 16), dtype=np.uint8)
+    sw[0, :8] = np.arange(8)
+    sw[1, :8] = 0x7E
+    gw = np.array([2.0 ** -20, 3.0e-3, 1.0, 2.0 ** 9], dtype=np.float32)
+    a = synthetic.bf16_bits_to_f32(x[ri]).astype(np.float64)
+    bw = oracle.dequantize_f64(qw, sw, np.repeat(gw, N)).reshape(E, N, K)
+    y_ref, s_ref = oracle.grouped_gemm_f64(a, bw, offsets)
+    wp = L.Packed(to_dev(qw), to_dev(sw), to_dev(gw), E * N, K, 0)
+    s = status_word()
+    y = L.grouped_gemm_w4a16(bf16_dev(x), wp, N, to_dev(ri), to_dev(offsets), E, out_dtype=0, dev_status=s)
+    torch.cuda.synchronize()
+    assert int(s.item()) == 0
+    ok, err, bound = gemm_tol(to_np(y), y_ref, s_ref)
+    assert ok.all(), (err.max(), (err / bound).max())
+
+
 def test_w4a16_swiglu_epilogue():
     """h = bf16(silu(g) * u) from the same g, u as the plain kernel's fp32
     output (each output element sums its K terms in the same order in both
