@@ -429,14 +429,15 @@ __global__ void __launch_bounds__(256) quantize_kernel(
 // slot[t*k + c] is the routed row of the token's c-th choice (-1: not routed);
 // a lane per choice holds its expert's packed row and global scale.
 
-// Pass 1: the rows are cut into 1024-element pieces, one per warp, eight
+// Pass 1: the rows are cut into 2048-element pieces, one per warp, eight
 // consecutive pieces per CTA (a CTA covers one or more whole tokens when a row
-// holds 1, 2, 4 or 8 pieces).  Each lane keeps two 32-byte loads in flight;
+// holds 1, 2, 4 or 8 pieces).  Each lane keeps four 32-byte loads in flight;
 // the warp's max|x| goes to shared memory, and after one barrier a thread per
 // (token, choice) pair of the CTA raises the expert's amax.  A token whose
 // pieces straddle two CTAs is raised by both, which atomicMax makes harmless.
 // CTAs are short and not persistent, so the last wave is small.
 constexpr int kAmaxWarps = 8;
+constexpr int kAmaxPieceBlocks = 128;                      // 16-element blocks per piece (2048 elements)
 
 __global__ void __launch_bounds__(kAmaxWarps * 32) moe_amax_kernel(
     const uint16_t *__restrict__ x, int64_t ld_x, int64_t K, int64_t tokens, const int32_t *__restrict__ slot,
@@ -448,25 +449,26 @@ __global__ void __launch_bounds__(kAmaxWarps * 32) moe_amax_kernel(
   for (int i = threadIdx.x; i <= G; i += blockDim.x) off[i] = group_offsets[i];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t nblk = (uint32_t)(K >> 4);
-  const int64_t pieces = (nblk + 63) >> 6;                 // 64 blocks of 16 per piece
+  const int64_t pieces = (nblk + kAmaxPieceBlocks - 1) / kAmaxPieceBlocks;
   const bool v8 = ((reinterpret_cast<uintptr_t>(x) & 31u) == 0) && ((ld_x & 15) == 0);
   const int64_t u0 = (int64_t)blockIdx.x * kAmaxWarps;     // first piece of the CTA
   const int64_t u = u0 + warp;
   uint32_t m = 0;
   if (u < tokens * pieces) {
     const int64_t t = u / pieces;
-    const uint32_t j0 = (uint32_t)(u - t * pieces) << 6;
+    const uint32_t j0 = (uint32_t)(u - t * pieces) * kAmaxPieceBlocks;
     const uint16_t *row = x + t * ld_x;
-    uint4 va[2], vb[2];
+    constexpr int kLoads = kAmaxPieceBlocks / 32;           // 32-byte loads per lane
+    uint4 va[kLoads], vb[kLoads];
 #pragma unroll
-    for (int k = 0; k < 2; ++k) {
+    for (int k = 0; k < kLoads; ++k) {
       const uint32_t j = j0 + k * 32 + lane;
       va[k] = make_uint4(0, 0, 0, 0);
       vb[k] = make_uint4(0, 0, 0, 0);
       if (j < nblk) load_block(row + (uint64_t)j * 16, v8, va[k], vb[k]);
     }
 #pragma unroll
-    for (int k = 0; k < 2; ++k) m = absmax8_bits(vb[k], absmax8_bits(va[k], m));
+    for (int k = 0; k < kLoads; ++k) m = absmax8_bits(vb[k], absmax8_bits(va[k], m));
   }
   m = warp_max(halves_max(m));
   if (lane == 0) piece_max[warp] = m;
@@ -1005,7 +1007,7 @@ nvfp4_status nvfp4_moe_quantize(const void *x, int64_t tokens, int64_t K, int64_
   if (tokens * topk > ((int64_t)1 << 31)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   const uint16_t *xb = reinterpret_cast<const uint16_t *>(x);
   uint32_t *amax_bits = reinterpret_cast<uint32_t *>(workspace);
-  const int64_t pieces = tokens * ((K / 16 + 63) / 64);         // amax pass: 1024-element pieces
+  const int64_t pieces = tokens * ((K / 16 + kAmaxPieceBlocks - 1) / kAmaxPieceBlocks);   // amax pass pieces
   if ((pieces + kAmaxWarps - 1) / kAmaxWarps > 0x7FFFFFFF) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   if (gs_mode == NVFP4_GS_FROM_AMAX) {
     if (cudaMemsetAsync(amax_bits, 0, sizeof(uint32_t) * G, stream) != cudaSuccess) return NVFP4_ERR_CUDA;
