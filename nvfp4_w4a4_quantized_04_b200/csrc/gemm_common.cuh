@@ -122,7 +122,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   }
 }
 
-// Warp-wide bounded wait: every lane waits, the verdict is made uniform so
+// Warp-wide bounded wait: every lane waits, the result is made uniform so
 // that no .sync.aligned tcgen05 instruction ever runs on a partial warp.
 template <bool kCluster = false>
 __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, volatile int *abort_flag,

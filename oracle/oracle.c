@@ -21,7 +21,7 @@
  *  [P3] "Qwen3.8-2.4T-A95B-NVFP4 ..." (hnwysp.cn/news/107543), section "为什么值得开
  *       NVFP4 KV 缓存": NVFP4 KV cache, group size 16.
  *
- * Readings taken where the pages are silent (each listed in the design doc):
+ * Readings taken where the pages are silent:
  *  - global scale s_g = amax / (6 * 448); s_g = 1 for an all-zero tensor;
  *  - every fp32 step is one IEEE round-to-nearest-even operation;
  *  - E4M3 block scale: round-to-nearest-even, saturate to 448, subnormals kept;
