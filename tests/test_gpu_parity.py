@@ -169,7 +169,8 @@ def _moe_quantize_check(x, slot, off, E, layout, x_dev=None):
 
 
 @pytest.mark.parametrize("layout,T,H,E,k", [(1, 1024, 512, 12, 2), (0, 1024, 2064, 12, 2), (1, 300, 7168, 40, 8),
-                                            (1, 2048, 4096, 64, 10), (0, 5, 64, 3, 3), (1, 8192, 4096, 512, 10)])
+                                            (1, 2048, 4096, 64, 10), (0, 5, 64, 3, 3), (1, 8192, 4096, 512, 10),
+                                            (1, 777, 1024, 9, 1), (1, 64, 10240, 16, 32)])
 def test_moe_quantize_bitexact(layout, T, H, E, k):
     x = synthetic.gaussian_bf16(21, synthetic.STREAMS["x"], (T, H), outlier_frac=0.001)
     r = synthetic.route_topk_softmax(21, T, E, k)
