@@ -254,6 +254,31 @@ def test_quantize_groups_with_empty_experts():
     assert np.array_equal(untile(to_np(p.sf), p.q.shape[0] // 128 * 128, H // 16)[rows], sf_ref)
 
 
+def test_quantize_and_dispatch_with_4096_groups():
+    """4096 groups, the most the quantizers take (their group tables sit in
+    shared memory): mostly empty, a few with 1-5 rows.  The grouped quantize and
+    the token-order dispatch (top-2) are both bit-exact to the oracle."""
+    rng = np.random.default_rng(26)
+    G, H = 4096, 256
+    counts = np.where(rng.random(G) < 0.9, 0, rng.integers(1, 6, G))
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    R = int(offsets[-1])
+    L = layer()
+    x = synthetic.gaussian_bf16(26, synthetic.STREAMS["x"], (R, H))
+    q_ref, sf_ref, gs_ref, st = oracle.quantize(x, None, offsets)
+    assert st == 0
+    p = L.quantize(bf16_dev(x), None, to_dev(offsets), G, layout=1)
+    torch.cuda.synchronize()
+    assert np.array_equal(to_np(p.gs), gs_ref)
+    rows, _ = slot_rows(offsets)
+    assert np.array_equal(to_np(p.q)[rows], q_ref)
+    assert np.array_equal(untile(to_np(p.sf), p.q.shape[0] // 128 * 128, H // 16)[rows], sf_ref)
+    T = 700
+    xt = synthetic.gaussian_bf16(27, synthetic.STREAMS["x"], (T, H))
+    r = synthetic.route_topk_softmax(27, T, G, 2)
+    _moe_quantize_check(xt, r["slot"], r["offsets"], G, 1)
+
+
 @pytest.mark.parametrize("shape", [(1, 16), (5, 48), (3, 208), (0, 64), (1000, 16), (7, 1040), (33, 5120),
                                    (2, 17408)])
 def test_quantize_ragged_shapes(shape):
