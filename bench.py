@@ -513,10 +513,20 @@ def comp_decode_moe(device, iters, warmup, flush):
     ms = timed(lambda: moe.forward(xb, ri, off), iters, warmup, flush)
     touched = int((np.diff(r["offsets"]) > 0).sum())
     wbytes = touched * (2 * I * H + H * I) * 0.5625
+    # the whole decode block (routing order, experts, weighted combine) through
+    # MoELayer, launched eagerly and as one captured CUDA graph
+    block = L.MoELayer(moe, T, k, device)
+    ids = torch.from_numpy(r["experts"].astype(np.int32)).to(device)
+    wts = torch.from_numpy(r["weights"].astype(np.float32)).to(device)
+    block_ms = timed(lambda: block.forward(xb, ids, wts), iters, warmup, flush)
+    graph, _ = block.capture(xb, ids, wts)
+    graph_ms = timed(graph.replay, iters, warmup, flush)
+    del graph
     return {"workload": "decode_moe_e384_top10_zipf1.1_t64_h7168_i2048", "experts_touched": touched,
             "routed_rows": R, "layer_ms": round(ms, 4),
             "touched_weight_gbs": round(gbs(wbytes, ms), 1),
             "roofline": {"bound": "hbm", "frac": round(gbs(wbytes, ms) / HBM_PEAK, 4), "peak": HBM_PEAK},
+            "block_ms": round(block_ms, 4), "block_graph_ms": round(graph_ms, 4),
             "remap_ms": round(remap_ms, 4), "remap_gbs": round(gbs(remap_bytes, remap_ms), 1)}
 
 

@@ -379,3 +379,19 @@ class MoELayer:
         nvfp4_moe_combine(y, OUT_F32 if y.dtype == torch.float32 else OUT_BF16, y.shape[0], slot, topk_weights, T, k,
                           self.experts.H, out, OUT_BF16, dev_status)
         return out
+
+    def capture(self, x: torch.Tensor, topk_ids: torch.Tensor, topk_weights: torch.Tensor, dev_status=None):
+        """Record forward() on these input tensors as a CUDA graph.
+
+        Returns (graph, out): graph.replay() reruns the whole block (routing
+        order, experts, combine: about ten kernel launches and memsets) on the
+        current contents of x, topk_ids and topk_weights, which keep their
+        shapes and addresses, and leaves the result in out.  forward() issues
+        no host synchronisation and allocates nothing, so it captures as is;
+        one eager call first sets the kernels' launch attributes."""
+        self.forward(x, topk_ids, topk_weights, dev_status)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            out = self.forward(x, topk_ids, topk_weights, dev_status)
+        return graph, out

@@ -1368,6 +1368,50 @@ def test_moe_layer_full_small():
     assert (np.abs(got - ref) <= 1e-6 * sabs + np.abs(ref) * 2.0 ** -8 + 1e-30).all()
 
 
+@pytest.mark.parametrize("H,I,fused", [(256, 256, False), (512, 1024, True)])
+def test_moe_layer_graph_replay(H, I, fused):
+    """The whole block captured as a CUDA graph: a replay gives the eager
+    forward's output bit for bit.  After new inputs are copied into the same
+    tensors (new tokens, new routing, new weights), a replay matches an eager
+    forward on them.  K = 256 takes the 256-element-stage GEMM, K = 512 and
+    1024 the 512-element one."""
+    L = layer()
+    T, E, k = 96, 8, 3
+    wgu = synthetic.gaussian_bf16(8, synthetic.STREAMS["w_gate_up"], (E * 2 * I, H), sigma=0.02)
+    wd = synthetic.gaussian_bf16(8, synthetic.STREAMS["w_down"], (E * H, I), sigma=0.02)
+    il = L.gate_up_interleave_index(E, I, "cpu").numpy() if fused else np.arange(E * 2 * I)
+    qg, sg, gg = _packed_weights(wgu, E, 2 * I, H)
+    qd, sd, gd = _packed_weights(wd, E, H, I)
+    Wgu = L.Packed(to_dev(qg[il]), to_dev(tile(sg[il])), to_dev(gg), E * 2 * I, H, 1)
+    Wd = L.Packed(to_dev(qd), to_dev(tile(sd)), to_dev(gd), E * H, I, 1)
+    experts = L.MoEExperts(Wgu, Wd, E, H, I, max_rows=T * k, out_dtype=1, mid_dtype=1, fused_swiglu=fused)
+    moe = L.MoELayer(experts, T, k)
+
+    def inputs(seed):
+        r = synthetic.route_topk_softmax(seed, T, E, k)
+        return (synthetic.gaussian_bf16(seed, synthetic.STREAMS["x"], (T, H)), r["experts"].astype(np.int32),
+                r["weights"].astype(np.float32))
+    xb, ids, wts = inputs(9)
+    x, idd, wd_ = bf16_dev(xb), to_dev(ids), to_dev(wts)
+    eager = moe.forward(x, idd, wd_).clone()
+    graph, out = moe.capture(x, idd, wd_)
+    out.zero_()
+    graph.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out, eager)
+    xb2, ids2, wts2 = inputs(10)
+    x.copy_(bf16_dev(xb2))
+    idd.copy_(to_dev(ids2))
+    wd_.copy_(to_dev(wts2))
+    graph.replay()
+    torch.cuda.synchronize()
+    replayed = out.clone()
+    eager2 = moe.forward(bf16_dev(xb2), to_dev(ids2), to_dev(wts2))
+    torch.cuda.synchronize()
+    assert torch.equal(replayed, eager2)
+    assert not torch.equal(replayed, eager)
+
+
 def test_device_generator_matches_host():
     import synthetic.cuda as sc
     g = sc.gaussian_bf16(3, 5, (1000, 64), sigma=0.02, start=12345)
