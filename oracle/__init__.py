@@ -339,14 +339,17 @@ def dot_f64(a: np.ndarray, b: np.ndarray):
 def route(expert_ids: np.ndarray, num_experts: int):
     """Group (token, choice) pairs by expert, tokens ascending inside a group
     (the routed-row order the grouped GEMM consumes; P1: top-10 routing).
-    expert_ids: int32 [T, k].  Returns (offsets [E+1], row_index [T*k], slot [T, k], status)."""
+    expert_ids: int32 [T, k].  A choice with an id outside [0, E) is dropped:
+    slot -1, not counted in the offsets, no routed row.
+    Returns (offsets [E+1], row_index [offsets[E]], slot [T, k], status) with
+    status 0, 1 (some choice dropped) or 2 (no routing: E or k <= 0)."""
     ids = np.ascontiguousarray(expert_ids, dtype=np.int32)
     T, k = ids.shape
-    off = np.empty(num_experts + 1, np.int32)
-    ri = np.empty(T * k, np.int32)
-    slot = np.empty((T, k), np.int32)
+    off = np.zeros(max(num_experts, 0) + 1, np.int32)
+    ri = np.full(T * k, -1, np.int32)
+    slot = np.full((T, k), -1, np.int32)
     st = lib().orc_route(_p(ids), T, k, num_experts, _p(off), _p(ri), _p(slot))
-    return off, ri, slot, st
+    return off, ri[:int(off[-1])], slot, st
 
 
 def combine(y: np.ndarray, slot: np.ndarray, weights: np.ndarray):

@@ -478,30 +478,37 @@ void orc_e4m3_encode_bits_range(uint64_t lo, uint64_t hi, uint8_t *out) {
  * Group routed (token, choice) pairs by expert: expert e's rows are the
  * tokens that chose e, in ascending token id; offsets[E+1] are the prefix
  * sums of the counts; slot[t*k + j] is the routed row of token t's j-th
- * choice.  A plain counting sort in token order.  Returns 0, or 1 when an
- * expert id is out of range.
+ * choice.  A plain counting sort in token order.
+ * A choice whose expert id is outside [0, E) is dropped (reading taken: the
+ * pages route each token to experts of the model only, so an id past the
+ * table names no expert): it gets slot -1, is not counted in the offsets and
+ * gets no routed row, so row_index holds offsets[E] entries and its tail is
+ * left untouched.  Returns 0, 1 when some choice was dropped, or 2 for
+ * arguments that describe no routing at all (E, k <= 0 or T < 0).
  */
 int orc_route(const int32_t *ids, int64_t T, int k, int E, int32_t *offsets, int32_t *row_index,
               int32_t *slot) {
-    if (E <= 0 || k <= 0 || T < 0) return 1;
+    if (E <= 0 || k <= 0 || T < 0) return 2;
+    int dropped = 0;
     for (int e = 0; e <= E; ++e) offsets[e] = 0;
     for (int64_t i = 0; i < T * k; ++i) {
-        if (ids[i] < 0 || ids[i] >= E) return 1;
+        if (ids[i] < 0 || ids[i] >= E) { dropped = 1; continue; }
         offsets[ids[i] + 1] += 1;
     }
     for (int e = 0; e < E; ++e) offsets[e + 1] += offsets[e];
     int32_t *fill = (int32_t *)malloc(sizeof(int32_t) * (size_t)(unsigned)E);
-    if (!fill) return 1;
+    if (!fill) return 2;
     for (int e = 0; e < E; ++e) fill[e] = offsets[e];
     for (int64_t t = 0; t < T; ++t)
         for (int j = 0; j < k; ++j) {
             int e = ids[t * k + j];
+            if (e < 0 || e >= E) { slot[t * k + j] = -1; continue; }
             int32_t r = fill[e]++;
             row_index[r] = (int32_t)t;
             slot[t * k + j] = r;
         }
     free(fill);
-    return 0;
+    return dropped;
 }
 
 /* out[t, :] = sum_j w[t, j] * y[slot[t, j], :], accumulated in fp64 in

@@ -220,6 +220,82 @@ def test_scale_audit_invariants(shape, sigma, outl):
     assert (sf[big] > 0).all()
 
 
+def _wide_range_blocks(seed, rows, K):
+    """N(0,1) rows whose 16-element blocks are each scaled by their own power
+    of two 2^-26 .. 2^3, plus a few all-zero blocks: beside the normal E4M3
+    block scales this reaches every subnormal scale and the zero scale."""
+    x = synthetic.bf16_bits_to_f32(synthetic.gaussian_bf16(seed, 1, (rows, K))).reshape(rows, K // 16, 16)
+    rng = np.random.default_rng(seed)
+    p = rng.integers(-26, 4, size=(rows, K // 16, 1)).astype(np.float32)
+    x = x * np.exp2(p)
+    x[rng.random((rows, K // 16)) < 0.01] = 0.0
+    return synthetic.f32_to_bf16_bits(x.reshape(rows, K).astype(np.float32))
+
+
+@pytest.mark.parametrize("case", ["gauss_outliers", "weights", "wide_range"])
+def test_block_scale_pulls_each_group_into_pm6(case):
+    """The page's rule for the block scale: it maps the group's values back into
+    [-6, 6], i.e. the group's largest |x| lands on 6, the top of the E2M1 grid
+    (golden fact block_scale_target_magnitude).  With S an E4M3 value:
+      - S normal: S is within half an E4M3 step of the exact quotient, at
+        most 2^-4 of S (the bound is reached just below 2^-6, where the
+        subnormal grid's step equals the lowest binade's), so
+        max|x| / (S s_g) lies in [6 (1-2^-4), 6 (1+2^-4)] = [5.625, 6.375] and
+        the block's largest code is +-6 (code 7);
+      - S = m 2^-9 subnormal (m = 1..7): S is within 2^-10 of the quotient, so
+        max|x| / (S s_g) lies in [6 (m - 1/2)/m, 6 (m + 1/2)/m] and the largest
+        code is at least the library's E2M1 rounding of the lower end;
+      - S = 0: the quotient is at most 2^-10 and every code is +-0.
+    A divisor other than 6 (or a product where the rule divides) fails the
+    normal-scale interval on every block but the amax one."""
+    top = FACTS["block_scale_target_magnitude"]
+    if case == "gauss_outliers":
+        x = synthetic.gaussian_bf16(11, 1, (256, 1024), outlier_frac=0.001)
+    elif case == "weights":
+        x = synthetic.gaussian_bf16(12, 2, (512, 512), sigma=0.02)
+    else:
+        x = _wide_range_blocks(13, 256, 1024)
+    q, sf, gs = _quant(x)
+    s_g = float(gs[0])
+    xf = synthetic.bf16_bits_to_f32(x).astype(np.float64)
+    rows, K = xf.shape
+    a_b = np.abs(xf).reshape(rows, K // 16, 16).max(axis=2)
+    S = ml_dtypes_e4m3(sf)
+    codes = np.empty((rows, K), dtype=np.int64)
+    codes[:, 0::2] = q & 15
+    codes[:, 1::2] = q >> 4
+    cmax = (codes & 7).reshape(rows, K // 16, 16).max(axis=2)
+    exp_field = (sf >> 3) & 15
+    normal = exp_field > 0
+    sub = (exp_field == 0) & (sf != 0)
+    zero = sf == 0
+    slack = 1e-6
+    ratio = np.where(S > 0, a_b / np.where(S > 0, S * s_g, 1.0), 0.0)
+    assert normal.any()
+    lo, hi = top * (1 - 2.0 ** -4), top * (1 + 2.0 ** -4)
+    assert (ratio[normal] >= lo * (1 - slack)).all() and (ratio[normal] <= hi * (1 + slack)).all()
+    assert (cmax[normal] == 7).all()
+    if case == "wide_range":
+        m = (sf & 7).astype(np.float64)
+        assert set(np.unique(m[sub]).astype(int)) == set(range(1, 8))
+        assert zero.any() and (a_b[zero] > 0).any()
+    if sub.any():
+        m = (sf[sub] & 7).astype(np.float64)
+        r = ratio[sub]
+        assert (r >= top * (m - 0.5) / m * (1 - slack)).all() and (r <= top * (m + 0.5) / m * (1 + slack)).all()
+        e2m1 = np.array([oracle.e2m1_decode(c) for c in range(8)])
+        least = np.abs((top * (m - 0.5) / m).astype(np.float32).astype(ml_dtypes.float4_e2m1fn).astype(np.float64))
+        assert (e2m1[cmax[sub]] >= least).all()
+    if zero.any():
+        assert (a_b[zero] / (6.0 * s_g) <= 2.0 ** -10 * (1 + slack)).all()
+        assert (cmax[zero] == 0).all()
+
+
+def ml_dtypes_e4m3(sf):
+    """E4M3 bytes -> float64 through the library codec (independent of the oracle)."""
+    return np.asarray(sf, np.uint8).view(ml_dtypes.float8_e4m3fn).astype(np.float64)
+
+
 def test_quantize_rne_error_bound():
     """|x/(S s_g) - code| <= half the local E2M1 spacing, unless clipped at 6."""
     x = synthetic.gaussian_bf16(5, 1, (256, 1024), outlier_frac=0.001)
@@ -577,9 +653,39 @@ def test_route_matches_library_sort_and_invariants():
             e = ids[t, j]
             assert off[e] <= r < off[e + 1] and ri[r] == t
     assert sorted(slot.reshape(-1).tolist()) == list(range(T * k))
-    bad = ids.copy()
-    bad[3, 1] = E
-    assert oracle.route(bad, E)[3] == 1
+
+
+def test_route_drops_out_of_range_choices():
+    """An id outside [0, E) names no expert of the model (the pages route each
+    token to its top-10 of the model's 512 experts): that choice is dropped.
+    The rest must be exactly numpy's stable (expert, token) sort of the valid
+    pairs alone, the dropped ones get slot -1 and the offsets count only valid
+    choices."""
+    rng = np.random.default_rng(3)
+    T, E, k = 257, 19, 5
+    ids = np.stack([rng.choice(E, size=k, replace=False) for _ in range(T)]).astype(np.int32)
+    bad_pos = rng.choice(T * k, size=40, replace=False)
+    flat = ids.reshape(-1)
+    flat[bad_pos[:20]] = E + rng.integers(0, 1000, 20)
+    flat[bad_pos[20:]] = -1 - rng.integers(0, 1000, 20)
+    ids = flat.reshape(T, k)
+    off, ri, slot, st = oracle.route(ids, E)
+    assert st == 1
+    flat_t = np.repeat(np.arange(T), k)
+    valid = (flat >= 0) & (flat < E)
+    order = np.lexsort((flat_t[valid], flat[valid]))
+    assert np.array_equal(ri, flat_t[valid][order])
+    assert np.array_equal(off, np.concatenate([[0], np.cumsum(np.bincount(flat[valid], minlength=E))]))
+    sl = slot.reshape(-1)
+    assert (sl[~valid] == -1).all()
+    want = np.empty(valid.sum(), np.int64)
+    want[order] = np.arange(valid.sum())
+    assert np.array_equal(sl[valid], want)
+    # all choices dropped: empty routing, every slot -1
+    off0, ri0, slot0, st0 = oracle.route(np.full((4, 2), E, np.int32), E)
+    assert st0 == 1 and (off0 == 0).all() and ri0.size == 0 and (slot0 == -1).all()
+    # no routing at all
+    assert oracle.route(ids, 0)[3] == 2
 
 
 def test_combine_closed_forms():
