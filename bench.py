@@ -23,6 +23,7 @@ Rank 0 prints one JSON line.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -51,9 +52,28 @@ def load_peaks():
 
 PEAKS, PEAKS_KIND = load_peaks()
 HBM_PEAK = PEAKS.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
-# DRAM traffic / algorithmic bytes of the gate_up + SwiGLU grouped GEMM launch,
-# from one ncu capture of this kernel (706.6 MB / 693.1 MB at 128 experts).
-GATE_UP_TRAFFIC_RATIO = 689016320 / 693108736
+# DRAM traffic / algorithmic bytes of the gate_up + SwiGLU grouped GEMM launch
+# (dram__bytes_read.sum + dram__bytes_write.sum over the bench's algorithmic
+# bytes), from one ncu capture at 128 experts / 2048 tokens of the kernel built
+# from the sources whose digest is recorded beside it.  Once those sources
+# change the figure no longer describes the kernel that runs, and the bench
+# reports the traffic as null until a new capture is recorded here.
+GATE_UP_TRAFFIC = {"ratio": 689016320 / 693108736, "capture": "128 experts, 2048 tokens",
+                   "sources_sha256": "452800defec16ce0bb6b4529b494fa6606f90d832a0cfb1286f23a1348bd8f8e"}
+GEMM_KERNEL_SOURCES = ("gemm_k512.cu", "gemm_common.cuh", "common.cuh")
+
+
+def gemm_sources_digest() -> str:
+    h = hashlib.sha256()
+    for name in GEMM_KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "nvfp4_w4a4_quantized_04_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def gate_up_traffic_ratio():
+    """The recorded DRAM/algorithmic ratio, or None when the kernel changed since its capture."""
+    return GATE_UP_TRAFFIC["ratio"] if gemm_sources_digest() == GATE_UP_TRAFFIC["sources_sha256"] else None
 FP4_PEAK = PEAKS.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]) * FP4_OVER_BF16
 
 
@@ -332,14 +352,16 @@ def run_headline(args, rank, world, device):
     q1_bytes = T * H * 2 + R * H * (0.5 + 1 / 16)
     q2_bytes = R * I * 2 + R * I * (0.5 + 1 / 16)
     q1_ms, q2_ms = float(np.mean(per[:, 0])), float(np.mean(per[:, 2]))
+    traffic_ratio = gate_up_traffic_ratio()
     roof = {"bound": "hbm", "kernel": ("nvfp4::gemm::grouped_gemm_k512_kernel<swiglu> (gate_up + SwiGLU epilogue launch)"
                                        if fused else "nvfp4::gemm::grouped_gemm_k512_kernel (gate_up launch)"),
             "achieved": round(gbs(g1_bytes, g1_ms), 1), "peak": HBM_PEAK, "unit": "GB/s",
             "frac": round(gbs(g1_bytes, g1_ms) / HBM_PEAK, 4),
-            "traffic": (int(GATE_UP_TRAFFIC_RATIO * g1_bytes) if fused else None),
-            "traffic_source": ("ncu dram__bytes_read.sum + dram__bytes_write.sum of the gate_up + SwiGLU launch at "
-                               "128 experts / 2048 tokens (profiles/grouped_gemm_moe_e128_t2048.md), ratio to "
-                               "algorithmic bytes 0.994, scaled by the units processed" if fused else None),
+            "traffic": (int(traffic_ratio * g1_bytes) if fused and traffic_ratio else None),
+            "traffic_source": (("ncu dram__bytes_read.sum + dram__bytes_write.sum of the gate_up + SwiGLU launch at "
+                                f"{GATE_UP_TRAFFIC['capture']}, ratio to algorithmic bytes {traffic_ratio:.3f}, "
+                                "scaled by the units processed") if fused and traffic_ratio else
+                               "null: no ncu capture of the kernel as built" if fused else None),
             "peak_source": f"{PEAKS_KIND} hbm_gbs (burst copy)",
             "algorithmic_bytes_per_launch": int(g1_bytes), "avg_launch_ms": round(g1_ms, 4),
             "tensor_tflops": round(g1_flops / (g1_ms * 1e-3) / 1e12, 1),

@@ -179,6 +179,27 @@ nvfp4_status nvfp4_dequantize(const uint8_t *q, const uint8_t *sf, nvfp4_sf_layo
                               nvfp4_out_dtype out_dtype, cudaStream_t stream);
 
 /*
+ * nvfp4_global_scale_from_amax -- the global-scale rule on its own, for a
+ * calibration pass that fixes a static scale (the checkpoints' input_scale)
+ * from observed amaxes.  [P1 two-level scaling: one FP32 global scale per
+ * tensor; calibrated activation scales.]
+ *   global_scale[i] = a_i / 2688 (1 when a_i == 0), a_i = |amax[i]| * margin:
+ *   the multiply is one IEEE fp32 round-to-nearest-even operation and is
+ *   skipped when margin == 1, the division is one IEEE operation -- with
+ *   margin 1 exactly the s_g that FROM_AMAX mode derives from that amax.
+ *   amax          fp32 [n] device (max |x| per tensor or group); may alias
+ *                 global_scale.
+ *   n             >= 0 (0 is a no-op), at most 2^30.
+ *   margin        finite and > 0, else NVFP4_ERR_INVALID_ARG (> 1 leaves
+ *                 headroom for activations larger than the calibration saw).
+ *   global_scale  fp32 [n] device, written.
+ *   dev_status    nullable: NVFP4_ERR_NONFINITE when some a_i is NaN or inf
+ *                 (that entry is written as NaN).
+ */
+nvfp4_status nvfp4_global_scale_from_amax(const float *amax, int64_t n, float margin, float *global_scale,
+                                          int32_t *dev_status, cudaStream_t stream);
+
+/*
  * nvfp4_e2m1_encode -- the element-wise FP32 -> E2M1 step of every quantize
  * call on its own.  [P2: the E2M1 value set {0, 0.5, 1, 1.5, 2, 3, 4, 6} with
  *  a sign bit, two codes per byte.]  Round to nearest, ties to the even

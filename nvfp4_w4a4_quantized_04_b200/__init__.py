@@ -11,7 +11,7 @@ Entry points (same names as the C ABI): ``nvfp4_quantize``,
 ``nvfp4_grouped_gemm``,
 ``nvfp4_swiglu_quantize``, ``nvfp4_kv_quantize``, ``nvfp4_kv_dequantize``,
 ``nvfp4_moe_quantize``, ``nvfp4_moe_route``, ``nvfp4_moe_combine``,
-``nvfp4_quantize_noalloc``, plus ``nvfp4_workspace_size``,
+``nvfp4_quantize_noalloc``, ``nvfp4_global_scale_from_amax``, plus ``nvfp4_workspace_size``,
 ``nvfp4_padded_rows_bound`` and ``nvfp4_moe_route_workspace_size``.
 """
 from __future__ import annotations
@@ -49,7 +49,7 @@ EXPORTS = [
     "nvfp4_moe_route_workspace_size", "nvfp4_moe_route", "nvfp4_moe_combine", "nvfp4_moe_quantize",
     "nvfp4_gemm_select_kernel", "nvfp4_grouped_gemm_w4a16", "nvfp4_grouped_gemm_swiglu_nvfp4",
     "mxfp4_quantize", "mxfp4_grouped_gemm", "nvfp4_w4a16_workspace_size",
-    "nvfp4_e2m1_encode", "nvfp4_e4m3_encode", "nvfp4_gemm_set_wait_budget",
+    "nvfp4_e2m1_encode", "nvfp4_e4m3_encode", "nvfp4_gemm_set_wait_budget", "nvfp4_global_scale_from_amax",
 ]
 NOALLOC_MAX_GROUPS = 1024
 
@@ -117,6 +117,8 @@ def load_library(path: str = LIB_PATH):
     L.nvfp4_e2m1_encode.argtypes = [P, i64, P, P]
     L.nvfp4_e4m3_encode.restype = i32
     L.nvfp4_e4m3_encode.argtypes = [P, i64, P, P]
+    L.nvfp4_global_scale_from_amax.restype = i32
+    L.nvfp4_global_scale_from_amax.argtypes = [P, i64, ctypes.c_float, P, P, P]
     _lib = L
     return L
 
@@ -230,6 +232,15 @@ def nvfp4_dequantize(q, sf, sf_layout, global_scale, group_offsets, num_groups, 
         _ptr(y), out_dtype, _stream(stream))
     if check:
         _check(st, "nvfp4_dequantize")
+    return st
+
+
+def nvfp4_global_scale_from_amax(amax, n, margin, global_scale, dev_status=None, stream=None, check=True) -> int:
+    """fp32 amax [n] -> fp32 s_g [n] with the library's global-scale rule (times ``margin``)."""
+    st = load_library().nvfp4_global_scale_from_amax(_ptr(amax), n, float(margin), _ptr(global_scale),
+                                                     _ptr(dev_status), _stream(stream))
+    if check:
+        _check(st, "nvfp4_global_scale_from_amax")
     return st
 
 

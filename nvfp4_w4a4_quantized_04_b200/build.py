@@ -54,8 +54,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
         if p.returncode != 0:
             raise RuntimeError("nvcc failed: " + " ".join(cmd))
     tmp = LIB + f".tmp{os.getpid()}"
-    subprocess.check_call([NVCC, *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs, "-lcuda"]
-                          if False else [NVCC, *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs])
+    subprocess.check_call([NVCC, *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs])
     os.replace(tmp, LIB)
     return LIB
 

@@ -81,10 +81,17 @@ __device__ __host__ __forceinline__ int64_t sf_tiled_offset(int64_t r, int64_t j
 // Block-wide: off[0..G] = group_offsets and slot[0..G] = exclusive prefix sums
 // of the 128-aligned group sizes (the slot starts), both in smem.  `scratch`
 // holds blockDim.x/32 ints.  blockDim.x must be a multiple of 32.
-__device__ inline void load_groups(const int32_t *__restrict__ group_offsets, int G,
-                                   int32_t *off, int32_t *slot, int32_t *scratch) {
+// Returns false (uniformly over the block, tables not built) unless the
+// offsets start at 0, never decrease and end at `total` (exact) or at most at
+// `total`: every output row a kernel writes is derived from them.
+__device__ inline bool load_groups(const int32_t *__restrict__ group_offsets, int G,
+                                   int32_t *off, int32_t *slot, int32_t *scratch, int64_t total, bool exact) {
   for (int i = threadIdx.x; i <= G; i += blockDim.x) off[i] = group_offsets[i];
   __syncthreads();
+  bool bad = false;
+  for (int i = threadIdx.x; i < G; i += blockDim.x) bad |= off[i + 1] < off[i];
+  if (threadIdx.x == 0) bad |= off[0] != 0 || (exact ? (int64_t)off[G] != total : (int64_t)off[G] > total);
+  if (__syncthreads_or(bad)) return false;
   const int nt = blockDim.x, t = threadIdx.x;
   const int per = (G + nt - 1) / nt;
   const int g0 = min(G, t * per), g1 = min(G, g0 + per);
@@ -117,6 +124,7 @@ __device__ inline void load_groups(const int32_t *__restrict__ group_offsets, in
   if (g1 == G && g0 < g1) slot[G] = run;
   if (G == 0 && t == 0) slot[0] = 0;
   __syncthreads();
+  return true;
 }
 
 // Largest g in [0, G) with a[g] <= x (a non-decreasing, a[0] <= x).

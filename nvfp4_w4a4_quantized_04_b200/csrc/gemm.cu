@@ -34,7 +34,10 @@
 //    NVFP4_ERR_TIMEOUT, every role leaves its loop, outstanding copies and
 //    MMAs are drained (again bounded) and tensor memory is freed.
 //  * No cluster multicast anywhere.
+#include <atomic>
+
 #include "gemm_common.cuh"
+#include "host_util.cuh"
 
 namespace nvfp4 {
 namespace gemm {
@@ -115,7 +118,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(
                  :: "r"(smem_u32((const void *)tmem_holder)), "r"(TMEM_COLS) : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
-  build_tile_tables(expert_offsets, E, M_total, n_mtiles, s_off, s_slot, s_tile, s_scratch);
+  build_tile_tables(expert_offsets, E, M_total, n_mtiles, s_off, s_slot, s_tile, s_scratch, dev_status);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -296,11 +299,9 @@ using namespace nvfp4;
 
 namespace {
 
-int g_sms = 0;
 // 0 automatic (512-element stages when K % 512 == 0, else one CTA per tile with
 // 256-element stages), 1 one CTA per tile with 256-element stages, 2 CTA pairs
-int g_gemm_kernel = 0;
-bool g_attr_set[6] = {false, false, false, false, false, false};
+std::atomic<int> g_gemm_kernel{0};
 
 }  // namespace
 
@@ -339,21 +340,11 @@ extern "C" nvfp4_status nvfp4_grouped_gemm(const uint8_t *a_q, const uint8_t *a_
   if (!gemm::make_map(&tx128, a_q, (uint64_t)x_rows, (uint64_t)K / 2, 128)) return NVFP4_ERR_CUDA;
   if (!gemm::make_map(&tx64, a_q, (uint64_t)x_rows, (uint64_t)K / 2, 64)) return NVFP4_ERR_CUDA;
   if (!gemm::make_map(&tx32, a_q, (uint64_t)x_rows, (uint64_t)K / 2, 32)) return NVFP4_ERR_CUDA;
-  if (g_sms == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&g_sms, cudaDevAttrMultiProcessorCount, dev);
-    if (g_sms <= 0) g_sms = 148;
-  }
   const int variant = swiglu ? 2 : (out_dtype == NVFP4_OUT_BF16 ? 1 : 0);
   auto kern = variant == 2 ? gemm::grouped_gemm_kernel<true, true>
                            : (variant == 1 ? gemm::grouped_gemm_kernel<false, true> : gemm::grouped_gemm_kernel<false, false>);
-  if (!g_attr_set[variant]) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::SMEM_BYTES) != cudaSuccess)
-      return NVFP4_ERR_CUDA;
-    g_attr_set[variant] = true;
-  }
-  kern<<<g_sms, gemm::NUM_THREADS, gemm::SMEM_BYTES, stream>>>(tw, tx128, tx64, tx32, b_sf, a_sf, b_gs, a_gs,
+  if (!host::set_max_dynamic_smem(reinterpret_cast<const void *>(kern), gemm::SMEM_BYTES)) return NVFP4_ERR_CUDA;
+  kern<<<host::sm_count(), gemm::NUM_THREADS, gemm::SMEM_BYTES, stream>>>(tw, tx128, tx64, tx32, b_sf, a_sf, b_gs, a_gs,
                                                                expert_offsets, E, (int)M_total, (int)N, (int)K, y,
                                                                amax_out, dev_status, gemm::HQuantOut{});
   return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
@@ -402,19 +393,9 @@ extern "C" nvfp4_status nvfp4_grouped_gemm_swiglu_nvfp4(const uint8_t *a_q, cons
   if (!gemm::make_map(&tx128, a_q, (uint64_t)x_rows, (uint64_t)K / 2, 128)) return NVFP4_ERR_CUDA;
   if (!gemm::make_map(&tx64, a_q, (uint64_t)x_rows, (uint64_t)K / 2, 64)) return NVFP4_ERR_CUDA;
   if (!gemm::make_map(&tx32, a_q, (uint64_t)x_rows, (uint64_t)K / 2, 32)) return NVFP4_ERR_CUDA;
-  if (g_sms == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&g_sms, cudaDevAttrMultiProcessorCount, dev);
-    if (g_sms <= 0) g_sms = 148;
-  }
   auto kern = gemm::grouped_gemm_kernel<true, true, true>;
-  if (!g_attr_set[3]) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::SMEM_BYTES) != cudaSuccess)
-      return NVFP4_ERR_CUDA;
-    g_attr_set[3] = true;
-  }
-  kern<<<g_sms, gemm::NUM_THREADS, gemm::SMEM_BYTES, stream>>>(tw, tx128, tx64, tx32, b_sf, a_sf, b_gs, a_gs,
+  if (!host::set_max_dynamic_smem(reinterpret_cast<const void *>(kern), gemm::SMEM_BYTES)) return NVFP4_ERR_CUDA;
+  kern<<<host::sm_count(), gemm::NUM_THREADS, gemm::SMEM_BYTES, stream>>>(tw, tx128, tx64, tx32, b_sf, a_sf, b_gs, a_gs,
                                                                expert_offsets, E, (int)M_total, (int)N, (int)K, nullptr,
                                                                nullptr, dev_status, hq);
   return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
@@ -448,21 +429,11 @@ extern "C" nvfp4_status mxfp4_grouped_gemm(const uint8_t *a_q, const uint8_t *a_
   if (!gemm::make_map(&tx128, a_q, (uint64_t)x_rows, (uint64_t)K / 2, 128)) return NVFP4_ERR_CUDA;
   if (!gemm::make_map(&tx64, a_q, (uint64_t)x_rows, (uint64_t)K / 2, 64)) return NVFP4_ERR_CUDA;
   if (!gemm::make_map(&tx32, a_q, (uint64_t)x_rows, (uint64_t)K / 2, 32)) return NVFP4_ERR_CUDA;
-  if (g_sms == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&g_sms, cudaDevAttrMultiProcessorCount, dev);
-    if (g_sms <= 0) g_sms = 148;
-  }
   const int variant = out_dtype == NVFP4_OUT_BF16 ? 5 : 4;
   auto kern = variant == 5 ? gemm::grouped_gemm_kernel<false, true, false, true>
                            : gemm::grouped_gemm_kernel<false, false, false, true>;
-  if (!g_attr_set[variant]) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::SMEM_BYTES) != cudaSuccess)
-      return NVFP4_ERR_CUDA;
-    g_attr_set[variant] = true;
-  }
-  kern<<<g_sms, gemm::NUM_THREADS, gemm::SMEM_BYTES, stream>>>(tw, tx128, tx64, tx32, b_sf, a_sf, nullptr, nullptr,
+  if (!host::set_max_dynamic_smem(reinterpret_cast<const void *>(kern), gemm::SMEM_BYTES)) return NVFP4_ERR_CUDA;
+  kern<<<host::sm_count(), gemm::NUM_THREADS, gemm::SMEM_BYTES, stream>>>(tw, tx128, tx64, tx32, b_sf, a_sf, nullptr, nullptr,
                                                                expert_offsets, E, (int)M_total, (int)N, (int)K, y,
                                                                nullptr, dev_status, gemm::HQuantOut{});
   return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;

@@ -374,9 +374,13 @@ __device__ __forceinline__ Tile decode_tile(int t, const int32_t *s_off, const i
 // Block-wide: s_off = expert offsets ({0, M_total} without offsets), s_slot =
 // 128-aligned slot starts, s_tile = first tile of each expert (n_mtiles weight
 // blocks x chunks per expert).  Every thread of the block calls it.
+// Every tile's rows, and so every output row the epilogue stores, come from
+// the offsets: unless they start at 0, never decrease and end at M_total, the
+// call reports NVFP4_ERR_INDEX and leaves s_tile[E] = 0, so the kernel runs no
+// tile (no copy, no MMA, no store).
 __device__ inline void build_tile_tables(const int32_t *__restrict__ expert_offsets, int E, int M_total,
                                          int n_mtiles, int32_t *s_off, int32_t *s_slot, int32_t *s_tile,
-                                         int32_t *s_scratch) {
+                                         int32_t *s_scratch, int32_t *dev_status) {
   if (expert_offsets) {
     for (int i = threadIdx.x; i <= E; i += NUM_THREADS) s_off[i] = expert_offsets[i];
   } else if (threadIdx.x == 0) {
@@ -384,6 +388,17 @@ __device__ inline void build_tile_tables(const int32_t *__restrict__ expert_offs
     s_off[1] = M_total;
   }
   __syncthreads();
+  bool bad = false;
+  for (int i = threadIdx.x; i < E; i += NUM_THREADS) bad |= s_off[i + 1] < s_off[i];
+  if (threadIdx.x == 0) bad |= s_off[0] != 0 || s_off[E] != M_total;
+  if (__syncthreads_or(bad)) {
+    if (threadIdx.x == 0) {
+      s_tile[E] = 0;
+      report(dev_status, NVFP4_ERR_INDEX);
+    }
+    __syncthreads();
+    return;
+  }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int per = (E + NUM_THREADS - 1) / NUM_THREADS;
   const int e0 = min(E, (int)threadIdx.x * per), e1 = min(E, e0 + per);

@@ -20,6 +20,7 @@
 // Used when K % 512 == 0 (nvfp4_gemm_select_kernel mode 0), for NVFP4 and for
 // MXFP4 operands (kind::mxf4, UE8M0 scales per 32 elements, no global scales).
 #include "gemm_common.cuh"
+#include "host_util.cuh"
 
 namespace nvfp4 {
 namespace gemm {
@@ -142,7 +143,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_k512_kernel(
                  :: "r"(smem_u32((const void *)tmem_holder)), "r"(TMEM_COLS) : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
-  build_tile_tables(expert_offsets, E, M_total, n_mtiles, s_off, s_slot, s_tile, s_scratch);
+  build_tile_tables(expert_offsets, E, M_total, n_mtiles, s_off, s_slot, s_tile, s_scratch, dev_status);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -324,8 +325,6 @@ nvfp4_status launch_grouped_gemm_k512(const uint8_t *a_q, const uint8_t *a_sf, c
                                       const int32_t *expert_offsets, int E, int64_t M_total, int64_t N, int64_t K,
                                       void *y, nvfp4_out_dtype out_dtype, bool swiglu, float *amax_out,
                                       const HQuantOut *hq, bool mx, int32_t *dev_status, cudaStream_t stream) {
-  static int sms = 0;
-  static bool attr_set[6] = {false, false, false, false, false, false};
   const int64_t x_rows = nvfp4_padded_rows_bound(M_total, E);
   CUtensorMap tw, tx32, tx64, tx128, tx192;
   if (!make_map_k512(&tw, b_q, (uint64_t)E * N, (uint64_t)K / 2, 128)) return NVFP4_ERR_CUDA;
@@ -333,12 +332,6 @@ nvfp4_status launch_grouped_gemm_k512(const uint8_t *a_q, const uint8_t *a_sf, c
   if (!make_map_k512(&tx64, a_q, (uint64_t)x_rows, (uint64_t)K / 2, 64)) return NVFP4_ERR_CUDA;
   if (!make_map_k512(&tx128, a_q, (uint64_t)x_rows, (uint64_t)K / 2, 128)) return NVFP4_ERR_CUDA;
   if (!make_map_k512(&tx192, a_q, (uint64_t)x_rows, (uint64_t)K / 2, 192)) return NVFP4_ERR_CUDA;
-  if (sms == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (sms <= 0) sms = 148;
-  }
   const bool bf = out_dtype == NVFP4_OUT_BF16;
   const int variant = mx ? (bf ? 5 : 4) : hq ? 3 : swiglu ? 2 : (bf ? 1 : 0);
   auto kern = variant == 5   ? grouped_gemm_k512_kernel<false, true, false, true>
@@ -347,12 +340,8 @@ nvfp4_status launch_grouped_gemm_k512(const uint8_t *a_q, const uint8_t *a_sf, c
               : variant == 2 ? grouped_gemm_k512_kernel<true, true, false, false>
               : variant == 1 ? grouped_gemm_k512_kernel<false, true, false, false>
                              : grouped_gemm_k512_kernel<false, false, false, false>;
-  if (!attr_set[variant]) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess)
-      return NVFP4_ERR_CUDA;
-    attr_set[variant] = true;
-  }
-  kern<<<sms, NUM_THREADS, SMEM_BYTES, stream>>>(tw, tx32, tx64, tx128, tx192, b_sf, a_sf, b_gs, a_gs,
+  if (!host::set_max_dynamic_smem(reinterpret_cast<const void *>(kern), SMEM_BYTES)) return NVFP4_ERR_CUDA;
+  kern<<<host::sm_count(), NUM_THREADS, SMEM_BYTES, stream>>>(tw, tx32, tx64, tx128, tx192, b_sf, a_sf, b_gs, a_gs,
                                                  expert_offsets, E, (int)M_total, (int)N, (int)K, y, amax_out,
                                                  dev_status, hq ? *hq : HQuantOut{});
   return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;

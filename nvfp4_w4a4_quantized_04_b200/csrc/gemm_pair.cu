@@ -25,7 +25,10 @@
 //    epilogue warps of both CTAs drain their own accumulators and release
 //    them to the leader.
 //  * Every wait is bounded; a timeout raises the abort flag of both CTAs.
+#include <mutex>
+
 #include "gemm_common.cuh"
+#include "host_util.cuh"
 
 namespace nvfp4 {
 namespace gemm {
@@ -109,7 +112,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_pair_kernel(
                  :: "r"(smem_u32((const void *)tmem_holder)), "r"(TMEM_COLS) : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
   }
-  build_tile_tables(expert_offsets, E, M_total, n_mtiles, s_off, s_slot, s_tile, s_scratch);
+  build_tile_tables(expert_offsets, E, M_total, n_mtiles, s_off, s_slot, s_tile, s_scratch, dev_status);
   tc_fence_before();
   __syncthreads();
   cluster_sync_all();              // both CTAs' barriers exist before any remote arrive or pair copy
@@ -299,8 +302,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_pair_kernel(
 
 // ====================================================================== host side
 namespace {
-bool g_pair_attr_set[3] = {false, false, false};
-int g_pair_clusters[3] = {0, 0, 0};
+// Resident CTA pairs per variant and device, from the occupancy query (0 = not asked yet).
+std::mutex g_pair_mu;
+int g_pair_clusters[host::kMaxDevices][3] = {};
 }  // namespace
 
 nvfp4_status launch_grouped_gemm_pair(const uint8_t *a_q, const uint8_t *a_sf, const float *a_gs,
@@ -322,11 +326,9 @@ nvfp4_status launch_grouped_gemm_pair(const uint8_t *a_q, const uint8_t *a_sf, c
   auto kern = variant == 2 ? pair::grouped_gemm_pair_kernel<true, true>
                            : (variant == 1 ? pair::grouped_gemm_pair_kernel<false, true>
                                            : pair::grouped_gemm_pair_kernel<false, false>);
-  if (!g_pair_attr_set[variant]) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, pair::SMEM_BYTES) != cudaSuccess)
-      return NVFP4_ERR_CUDA;
-    g_pair_attr_set[variant] = true;
-  }
+  if (!host::set_max_dynamic_smem(reinterpret_cast<const void *>(kern), pair::SMEM_BYTES)) return NVFP4_ERR_CUDA;
+  const int dev = host::current_device();
+  if (dev < 0) return NVFP4_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -338,19 +340,24 @@ nvfp4_status launch_grouped_gemm_pair(const uint8_t *a_q, const uint8_t *a_sf, c
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (g_pair_clusters[variant] == 0) {
-    int sms = 0, dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int clusters;
+  {
+    std::lock_guard<std::mutex> lock(g_pair_mu);
+    clusters = g_pair_clusters[dev][variant];
+  }
+  if (clusters == 0) {
+    const int sms = host::sm_count();
     cfg.gridDim = dim3(2 * (sms / 2 > 0 ? sms / 2 : 1), 1, 1);
     int n = 0;
     if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) {
       (void)cudaGetLastError();
       n = sms / 2 > 0 ? sms / 2 : 1;
     }
-    g_pair_clusters[variant] = n;
+    clusters = n;
+    std::lock_guard<std::mutex> lock(g_pair_mu);
+    g_pair_clusters[dev][variant] = n;
   }
-  cfg.gridDim = dim3(2 * g_pair_clusters[variant], 1, 1);
+  cfg.gridDim = dim3(2 * clusters, 1, 1);
   const cudaError_t err = cudaLaunchKernelEx(&cfg, kern, tw, tx96, tx64, tx32, tsfx, tsfw, b_gs, a_gs, expert_offsets,
                                              E, (int)M_total, (int)N, (int)K, y, amax_out, dev_status);
   return err == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;

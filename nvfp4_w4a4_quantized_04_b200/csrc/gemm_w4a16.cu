@@ -39,6 +39,7 @@
 //    follow each other so they hit L2.
 //  * Every mbarrier wait is bounded (NVFP4_ERR_TIMEOUT, then all roles leave).
 #include "gemm_common.cuh"
+#include "host_util.cuh"
 
 #include <cuda_fp16.h>
 
@@ -447,7 +448,6 @@ size_t w4a16_x16_bytes(int64_t M_total, int E, int64_t K) {
   return ((size_t)w4a16_chunks_bound(M_total, E) * 8 * (size_t)K * 2 + 255) / 256 * 256;
 }
 
-bool g_w4a16_attr[4] = {false, false, false, false};
 
 }  // namespace
 
@@ -480,9 +480,7 @@ extern "C" nvfp4_status nvfp4_grouped_gemm_w4a16(const void *x, int64_t ld_x, in
     return NVFP4_ERR_INVALID_ARG;
   uint16_t *x16 = reinterpret_cast<uint16_t *>(workspace);
   float *xscale = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(workspace) + w4a16_x16_bytes(M_total, E, K));
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int sms = host::sm_count();
   // prep: the routed rows, as scaled f16 in fragment order
   {
     const size_t sm = sizeof(int32_t) * (2 * (size_t)(E + 1) + 8);
@@ -501,11 +499,7 @@ extern "C" nvfp4_status nvfp4_grouped_gemm_w4a16(const void *x, int64_t ld_x, in
   auto kern = variant == 3 ? w4a16::w4a16_kernel<true, true>
             : variant == 2 ? w4a16::w4a16_kernel<true, false>
             : variant == 1 ? w4a16::w4a16_kernel<false, true> : w4a16::w4a16_kernel<false, false>;
-  if (!g_w4a16_attr[variant]) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, w4a16::SMEM_BYTES) != cudaSuccess)
-      return NVFP4_ERR_CUDA;
-    g_w4a16_attr[variant] = true;
-  }
+  if (!host::set_max_dynamic_smem(reinterpret_cast<const void *>(kern), w4a16::SMEM_BYTES)) return NVFP4_ERR_CUDA;
   kern<<<sms, w4a16::kThreads, w4a16::SMEM_BYTES, stream>>>(tw, ts, x16, xscale, b_gs, expert_offsets, E, M_total,
                                                             (int)N, (int)K, y, dev_status);
   return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;

@@ -19,6 +19,7 @@
 #include <stdint.h>
 
 #include "common.cuh"
+#include "host_util.cuh"
 
 namespace nvfp4 {
 namespace moe {
@@ -208,11 +209,9 @@ extern "C" nvfp4_status nvfp4_moe_route(const int32_t *topk_ids, int64_t tokens,
   if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_CUDA;
   if (n_chunks > 0) {
     const size_t sm = sizeof(uint32_t) * 8 * (size_t)num_experts;
-    if (sm > 48 * 1024) {
-      if (cudaFuncSetAttribute(moe::route_place_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) !=
-          cudaSuccess)
-        return NVFP4_ERR_CUDA;
-    }
+    if (sm > 48 * 1024 &&
+        !host::set_max_dynamic_smem(reinterpret_cast<const void *>(moe::route_place_kernel), (int)sm))
+      return NVFP4_ERR_CUDA;
     moe::route_place_kernel<<<(unsigned)n_chunks, moe::kChunk, sm, stream>>>(topk_ids, tokens, topk, num_experts,
                                                                               counts, row_index, slot);
     if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_CUDA;
@@ -231,9 +230,7 @@ extern "C" nvfp4_status nvfp4_moe_combine(const void *y, nvfp4_out_dtype y_dtype
   if (tokens == 0) return NVFP4_OK;
   if ((rows > 0 && !y) || !slot || !weights || !out) return NVFP4_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(y) | reinterpret_cast<uintptr_t>(out)) & 15u) return NVFP4_ERR_INVALID_ARG;
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int sms = host::sm_count();
   const int64_t work = tokens * (H / 8);
   int64_t blocks = (work + 255) / 256;
   if (blocks > (int64_t)sms * 8) blocks = (int64_t)sms * 8;

@@ -20,6 +20,7 @@
 #include <stdint.h>
 
 #include "common.cuh"
+#include "host_util.cuh"
 
 namespace nvfp4 {
 namespace {
@@ -101,8 +102,6 @@ __global__ void __launch_bounds__(256) mxfp4_quantize_kernel(
   if (bad) report(dev_status, NVFP4_ERR_NONFINITE);
 }
 
-int g_sms_mx = 0;
-
 }  // namespace
 }  // namespace nvfp4
 
@@ -125,15 +124,9 @@ extern "C" nvfp4_status mxfp4_quantize(const void *x, int64_t rows, int64_t K, i
   uint32_t l = 0;
   while (l < 32 && (1ull << l) < nb) ++l;
   const uint32_t m = (uint32_t)((((1ull << 32) * ((1ull << l) - nb)) / nb) + 1);
-  if (g_sms_mx == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&g_sms_mx, cudaDevAttrMultiProcessorCount, dev);
-    if (g_sms_mx <= 0) g_sms_mx = 148;
-  }
   // one wave of resident 256-thread blocks (8 per SM) at most
   uint64_t grid = (total + 255) / 256;
-  const uint64_t cap = (uint64_t)g_sms_mx * 8;
+  const uint64_t cap = (uint64_t)host::sm_count() * 8;
   if (grid > cap) grid = cap;
   const uint16_t *xb = reinterpret_cast<const uint16_t *>(x);
   if (sf_layout == NVFP4_SF_MMA_TILED)

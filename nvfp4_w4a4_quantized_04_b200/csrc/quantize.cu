@@ -16,6 +16,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "host_util.cuh"
 
 namespace nvfp4 {
 
@@ -139,6 +140,18 @@ __global__ void __launch_bounds__(256, 4) amax_flat_kernel(const uint16_t *__res
   }
 }
 
+// s_g from the bit pattern of a non-negative amax: amax / 2688 in one IEEE
+// division (2688 = 6 * 448, so the block holding the amax gets the E4M3 scale
+// 448), 1 for an amax of 0, NaN (reported) for inf or NaN.
+__device__ __forceinline__ float gs_from_amax_bits(uint32_t b, int32_t *dev_status) {
+  if (b >= 0x7F800000u) {
+    report(dev_status, NVFP4_ERR_NONFINITE);
+    return __uint_as_float(0x7FC00000u);
+  }
+  const float a = __uint_as_float(b);
+  return (a == 0.0f) ? 1.0f : __fdiv_rn(a, 2688.0f);
+}
+
 // Global scales from the amax (FROM_AMAX; AMAX_GIVEN reads the amax from gs
 // itself) or a check of the given ones (GIVEN).  Returns the group's s_g.
 __device__ __forceinline__ float finalize_one(const uint32_t *__restrict__ amax_bits, int g, int mode, float *gs,
@@ -149,15 +162,20 @@ __device__ __forceinline__ float finalize_one(const uint32_t *__restrict__ amax_
     return s;
   }
   const uint32_t b = mode == NVFP4_GS_AMAX_GIVEN ? (__float_as_uint(gs[g]) & 0x7FFFFFFFu) : amax_bits[g];
-  if (b >= 0x7F800000u) {
-    gs[g] = __uint_as_float(0x7FC00000u);
-    report(dev_status, NVFP4_ERR_NONFINITE);
-    return __uint_as_float(0x7FC00000u);
-  }
-  const float a = __uint_as_float(b);
-  const float s = (a == 0.0f) ? 1.0f : __fdiv_rn(a, 2688.0f);   // 2688 = 6 * 448
+  const float s = gs_from_amax_bits(b, dev_status);
   gs[g] = s;
   return s;
+}
+
+// nvfp4_global_scale_from_amax: a = |amax[i]| (times the margin, one IEEE
+// multiply, unless it is 1), then the rule above.
+__global__ void gs_from_amax_kernel(const float *__restrict__ amax, int n, float margin, float *__restrict__ gs,
+                                    int32_t *dev_status) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  float a = fabsf(amax[i]);
+  if (margin != 1.0f) a = __fmul_rn(a, margin);
+  gs[i] = gs_from_amax_bits(__float_as_uint(a) & 0x7FFFFFFFu, dev_status);
 }
 
 __global__ void finalize_scales_kernel(const uint32_t *__restrict__ amax_bits, int G, int mode,
@@ -278,7 +296,10 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(
     const float *__restrict__ gs, uint8_t *__restrict__ q, uint8_t *__restrict__ sf, int32_t *dev_status) {
   extern __shared__ int32_t smem[];
   int32_t *off = smem, *slot = smem + (G + 1), *scratch = smem + 2 * (G + 1);
-  if (group_offsets) load_groups(group_offsets, G, off, slot, scratch);
+  if (group_offsets && !load_groups(group_offsets, G, off, slot, scratch, rows, true)) {
+    if (threadIdx.x == 0) report(dev_status, NVFP4_ERR_INDEX);
+    return;
+  }
   const int lane = threadIdx.x & 31;
   const uint32_t K = (uint32_t)K64, nblk = K >> 4;
   const uint32_t warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -335,7 +356,10 @@ __global__ void __launch_bounds__(256) quantize_kernel(
     int32_t *dev_status) {
   extern __shared__ int32_t smem[];
   int32_t *off = smem, *slot = smem + (G + 1), *scratch = smem + 2 * (G + 1);
-  if (group_offsets) load_groups(group_offsets, G, off, slot, scratch);
+  if (group_offsets && !load_groups(group_offsets, G, off, slot, scratch, rows, true)) {
+    if (threadIdx.x == 0) report(dev_status, NVFP4_ERR_INDEX);
+    return;
+  }
   const int lane = threadIdx.x & 31;
   const uint32_t K = (uint32_t)K64, nblk = K >> 4;
   const uint32_t total = (uint32_t)rows * nblk;              // < 2^32 (host check)
@@ -564,7 +588,10 @@ __global__ void __launch_bounds__(256, 3) moe_encode_blocks_kernel(
     uint8_t *__restrict__ sf, int32_t *dev_status) {
   extern __shared__ int32_t smem[];
   int32_t *off = smem, *pslot = smem + (G + 1), *scratch = smem + 2 * (G + 1);
-  load_groups(group_offsets, G, off, pslot, scratch);
+  if (!load_groups(group_offsets, G, off, pslot, scratch, tokens * topk, false)) {
+    if (threadIdx.x == 0) report(dev_status, NVFP4_ERR_INDEX);
+    return;
+  }
   const int lane = threadIdx.x & 31;
   const uint32_t K = (uint32_t)K64, nblk = K >> 4;
   const uint32_t cpr = (nblk + 63) >> 6;                     // 64-block chunks per row
@@ -685,7 +712,7 @@ __global__ void __launch_bounds__(256) dequantize_kernel(
     const int32_t *__restrict__ group_offsets, int G, int64_t rows, int64_t K, void *__restrict__ y) {
   extern __shared__ int32_t smem[];
   int32_t *off = smem, *slot = smem + (G + 1), *scratch = smem + 2 * (G + 1);
-  if (group_offsets) load_groups(group_offsets, G, off, slot, scratch);
+  if (group_offsets && !load_groups(group_offsets, G, off, slot, scratch, rows, true)) return;   // nothing written
   // one thread per 8 elements (a thread pair per 16-element block), so a warp
   // writes 512 (bf16) or 1024 (fp32) contiguous bytes per step
   const uint64_t nhalf = (uint64_t)(K >> 3);
@@ -818,17 +845,7 @@ float *workspace_tables(void *workspace, int num_groups) {
   return reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(workspace) + workspace_words_bytes(num_groups));
 }
 
-int g_num_sms = 0;
-
-int num_sms() {
-  if (g_num_sms == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
-    if (g_num_sms <= 0) g_num_sms = 148;
-  }
-  return g_num_sms;
-}
+int num_sms() { return host::sm_count(); }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -841,22 +858,9 @@ int64_t grid_for(int64_t work_items, int threads, int per_sm) {
 
 // Grid for a grid-stride kernel: at most one wave of resident blocks, so no
 // block starts late with a full share of the work.
-struct OccEntry { const void *fn; int threads; size_t smem; int per_sm; };
-OccEntry g_occ[64];
-int g_occ_n = 0;
-
 template <typename Kernel>
 int64_t grid_resident(Kernel kernel, int64_t work_items, int threads, size_t smem) {
-  const void *fn = reinterpret_cast<const void *>(kernel);
-  int per_sm = 0;
-  for (int i = 0; i < g_occ_n; ++i)
-    if (g_occ[i].fn == fn && g_occ[i].threads == threads && g_occ[i].smem == smem) per_sm = g_occ[i].per_sm;
-  if (per_sm == 0) {
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem) != cudaSuccess || per_sm < 1)
-      per_sm = 1;
-    if (g_occ_n < 64) g_occ[g_occ_n++] = OccEntry{fn, threads, smem, per_sm};
-  }
-  return grid_for(work_items, threads, per_sm);
+  return grid_for(work_items, threads, host::blocks_per_sm(reinterpret_cast<const void *>(kernel), threads, smem));
 }
 
 nvfp4_status launch_status() {
@@ -1034,6 +1038,17 @@ nvfp4_status nvfp4_moe_quantize(const void *x, int64_t tokens, int64_t K, int64_
     moe_encode_blocks_kernel<false><<<grid, 256, sm, stream>>>(xb, ld_x, K, tokens, slot, topk, group_offsets, G,
                                                                global_scale, rtab, ytab, q, sf, dev_status);
   }
+  return launch_status();
+}
+
+nvfp4_status nvfp4_global_scale_from_amax(const float *amax, int64_t n, float margin, float *global_scale,
+                                          int32_t *dev_status, cudaStream_t stream) {
+  if (n < 0 || !(margin > 0.0f) || !isfinite(margin)) return NVFP4_ERR_INVALID_ARG;
+  if (n > ((int64_t)1 << 30)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (n == 0) return NVFP4_OK;
+  if (!amax || !global_scale) return NVFP4_ERR_INVALID_ARG;
+  gs_from_amax_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(amax, (int)n, margin, global_scale,
+                                                                      dev_status);
   return launch_status();
 }
 

@@ -17,6 +17,7 @@
 #include <stdint.h>
 
 #include "common.cuh"
+#include "host_util.cuh"
 
 namespace nvfp4 {
 
@@ -227,9 +228,7 @@ extern "C" nvfp4_status mxfp4_to_nvfp4(const uint8_t *q_mx, const uint8_t *ue8m0
   if (grid1.y > 65535) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   remap_scan_kernel<<<grid1, 256, 0, stream>>>(q_mx, ue8m0, bpt, q_nv, ws, dev_status);
   if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_CUDA;
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int sms = host::sm_count();
   if (sf_layout == NVFP4_SF_MMA_TILED) {
     const int64_t units = n_tensors * (rows / 128) * ((K / 64 + kAtomRun - 1) / kAtomRun);
     int64_t blocks = (units + 7) / 8;                      // a warp per unit, 8 warps per CTA

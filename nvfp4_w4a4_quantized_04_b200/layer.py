@@ -15,7 +15,8 @@ import torch
 
 from . import (EPI_NONE, EPI_SWIGLU, GS_AMAX_GIVEN, GS_FROM_AMAX, GS_GIVEN, OUT_BF16, OUT_F32, SF_MMA_TILED, SF_ROWMAJOR,
                mxfp4_grouped_gemm as _mxfp4_grouped_gemm, mxfp4_quantize as _mxfp4_quantize, mxfp4_to_nvfp4, nvfp4_dequantize, nvfp4_grouped_gemm, nvfp4_grouped_gemm_swiglu_nvfp4,
-               nvfp4_grouped_gemm_w4a16, nvfp4_moe_combine, nvfp4_w4a16_workspace_size,
+               nvfp4_global_scale_from_amax, nvfp4_grouped_gemm_w4a16, nvfp4_moe_combine,
+               nvfp4_w4a16_workspace_size,
                nvfp4_moe_route,
                nvfp4_moe_quantize, nvfp4_moe_route_workspace_size, nvfp4_padded_rows_bound, nvfp4_quantize,
                nvfp4_swiglu_quantize,
@@ -276,6 +277,14 @@ class MoEExperts:
         self.y2 = torch.empty((max_rows, H), dtype=odt, device=device)
         self.max_rows = max_rows
 
+    def _quantize_input(self, x, row_index, offsets, slot, dev_status):
+        R = row_index.shape[0]
+        if slot is not None:
+            return moe_quantize(x, slot, offsets, self.E, SF_MMA_TILED, out=self.a1, ws=self.ws,
+                                dev_status=dev_status, rows=R)
+        return quantize(x, row_index, offsets, self.E, SF_MMA_TILED, out=self.a1, ws=self.ws,
+                        dev_status=dev_status, rows=R)
+
     def forward(self, x: torch.Tensor, row_index: torch.Tensor, offsets: torch.Tensor, dev_status=None,
                 slot: Optional[torch.Tensor] = None):
         """``slot`` [T, k] (routed row of each token choice), when given, selects
@@ -283,12 +292,7 @@ class MoEExperts:
         R = row_index.shape[0]
         assert R <= self.max_rows
         E, H, I = self.E, self.H, self.I
-        if slot is not None:
-            a1 = moe_quantize(x, slot, offsets, E, SF_MMA_TILED, out=self.a1, ws=self.ws, dev_status=dev_status,
-                              rows=R)
-        else:
-            a1 = quantize(x, row_index, offsets, E, SF_MMA_TILED, out=self.a1, ws=self.ws, dev_status=dev_status,
-                          rows=R)
+        a1 = self._quantize_input(x, row_index, offsets, slot, dev_status)
         if self.h_scale is not None:
             # calibrated down-input global: the gate_up epilogue writes NVFP4 h itself
             a2 = grouped_gemm_swiglu_nvfp4(a1, self.w_gate_up, 2 * I, self.h_scale, out=self.a2,
@@ -312,15 +316,23 @@ class MoEExperts:
         return y2
 
 
-def calibrate_h_scale(experts: "MoEExperts", x, row_index, offsets, slot=None, margin: float = 1.0) -> torch.Tensor:
-    """A down-input global per expert from one dynamic forward (s_g = margin *
-    max|h| / 2688, 1 for an expert without tokens), as a calibration pass would
-    set the checkpoint's input_scale; installs it on ``experts``."""
+def calibrate_h_scale(experts: "MoEExperts", x, row_index, offsets, slot=None, margin: float = 1.0,
+                      dev_status=None) -> torch.Tensor:
+    """A down-input global per expert from one calibration batch, as a
+    calibration pass would set the checkpoint's input_scale, installed on
+    ``experts``: the dynamic path's first two stages give the per-expert max |h|
+    (SwiGLU epilogue), and the library turns it into s_g = margin * max|h| / 2688
+    (1 for an expert without tokens) with the same arithmetic as the dynamic
+    global scale.  With margin 1 the result is exactly the s_g a dynamic forward
+    derives for the same batch."""
     assert experts.fused_swiglu
     experts.h_scale = None
-    experts.forward(x, row_index, offsets, slot=slot)
-    gs = experts.amax.clone() * (margin / 2688.0)
-    gs[gs == 0] = 1.0
+    R = row_index.shape[0]
+    a1 = experts._quantize_input(x, row_index, offsets, slot, dev_status)
+    _, amax = grouped_gemm_swiglu(a1, experts.w_gate_up, 2 * experts.I, h=experts.h[:R], amax=experts.amax,
+                                  dev_status=dev_status)
+    gs = torch.empty(experts.E, dtype=torch.float32, device=amax.device)
+    nvfp4_global_scale_from_amax(amax, experts.E, margin, gs, dev_status)
     experts.h_scale = gs
     return gs
 
@@ -388,7 +400,11 @@ class MoELayer:
         current contents of x, topk_ids and topk_weights, which keep their
         shapes and addresses, and leaves the result in out.  forward() issues
         no host synchronisation and allocates nothing, so it captures as is;
-        one eager call first sets the kernels' launch attributes."""
+        one eager call first sets the kernels' launch attributes.
+
+        ``out`` is a view of this layer's own output buffer, not a copy: a
+        later eager forward(), or the replay of another graph captured on this
+        layer, overwrites it.  Copy it out (or read it) before either runs."""
         self.forward(x, topk_ids, topk_weights, dev_status)
         torch.cuda.synchronize()
         graph = torch.cuda.CUDAGraph()

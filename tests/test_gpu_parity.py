@@ -833,6 +833,68 @@ def test_gemm_wait_timeout_reports_and_recovers(mode):
     assert np.array_equal(y_after, y_before)
 
 
+@pytest.mark.parametrize("bad", ["decreasing", "end_past_rows", "end_short", "nonzero_start"])
+def test_gemm_rejects_bad_offsets(gemm_kernel, bad):
+    """Expert offsets that do not start at 0, decrease, or end elsewhere than
+    at M_total: every CTA reports NVFP4_ERR_INDEX and runs no tile, so y keeps
+    its sentinel.  The buffers are sized so that even a kernel that trusted
+    the offsets would stay inside them (the slots of the largest offsets fit)."""
+    L = layer()
+    nv = nvmod()
+    E, N, K, M = 3, 256, 1024, 300
+    offsets = {"decreasing": [0, 200, 120, 300], "end_past_rows": [0, 100, 200, 380],
+               "end_short": [0, 100, 200, 250], "nonzero_start": [7, 100, 200, 300]}[bad]
+    offsets = np.array(offsets, np.int32)
+    rows_alloc = 2048
+    rng = np.random.default_rng(1)
+    qa = rng.integers(0, 256, (rows_alloc, K // 2), dtype=np.uint8)
+    sa = np.full((rows_alloc, K // 16), 0x38, np.uint8)
+    qw = rng.integers(0, 256, (E * N, K // 2), dtype=np.uint8)
+    sw = np.full((E * N, K // 16), 0x38, np.uint8)
+    one = np.ones(E, np.float32)
+    a = L.Packed(to_dev(qa), to_dev(tile(sa)), to_dev(one), M, K, 1, to_dev(offsets), E)
+    w = L.Packed(to_dev(qw), to_dev(tile(sw)), to_dev(one), E * N, K, 1)
+    y = torch.full((rows_alloc, N), 12345.0, dtype=torch.float32, device="cuda")
+    s = status_word()
+    L.grouped_gemm(a, w, N, 0, y=y[:M], dev_status=s)
+    torch.cuda.synchronize()
+    assert int(s.item()) == nv.ERR_INDEX
+    assert (to_np(y) == np.float32(12345.0)).all()
+
+
+def test_quantize_rejects_bad_group_offsets():
+    """The grouped quantize and the dispatch quantize check their group offsets
+    the same way: NVFP4_ERR_INDEX and no packed byte written."""
+    L = layer()
+    nv = nvmod()
+    T, K, E = 64, 256, 4
+    x = synthetic.gaussian_bf16(3, synthetic.STREAMS["x"], (T, K))
+    xd = bf16_dev(x)
+    for offs in ([0, 10, 5, 64], [0, 10, 20, 60], [3, 10, 20, 64]):
+        off = to_dev(np.array(offs, np.int32))
+        q = torch.full((2048, K // 2), 0xAB, dtype=torch.uint8, device="cuda")
+        sf = torch.full((2048 * K // 16,), 0xAB, dtype=torch.uint8, device="cuda")
+        gs = torch.ones(E - 1, dtype=torch.float32, device="cuda")
+        ws = L.workspace(E - 1)
+        for layout in (0, 1):
+            s = status_word()
+            nv.nvfp4_quantize(xd, T, K, K, None, off, E - 1, nv.GS_GIVEN, gs, q, sf, layout, ws, s)
+            torch.cuda.synchronize()
+            assert int(s.item()) == nv.ERR_INDEX, (offs, layout)
+            assert (to_np(q) == 0xAB).all() and (to_np(sf) == 0xAB).all()
+    # the dispatch quantize: offsets past the routed rows of T tokens x top-1
+    slot = to_dev(np.arange(T, dtype=np.int32).reshape(T, 1))
+    off = to_dev(np.array([0, 30, 20, 64], np.int32))
+    q = torch.full((2048, K // 2), 0xAB, dtype=torch.uint8, device="cuda")
+    sf = torch.full((2048 * K // 16,), 0xAB, dtype=torch.uint8, device="cuda")
+    gs = torch.ones(E - 1, dtype=torch.float32, device="cuda")
+    s = status_word()
+    nv.nvfp4_moe_quantize(xd, T, K, K, slot, 1, off, E - 1, nv.GS_GIVEN, gs, q, sf, 1, L.workspace(E - 1), s)
+    torch.cuda.synchronize()
+    assert int(s.item()) == nv.ERR_INDEX
+    assert (to_np(q) == 0xAB).all() and (to_np(sf) == 0xAB).all()
+
+
 def test_gemm_max_experts(gemm_kernel):
     """1024 experts, the most the GEMM's shared-memory tile tables hold: mostly
     empty groups, a few with 1-3 rows and one with 200 (two token chunks)."""
@@ -1148,8 +1210,20 @@ def test_moe_layer_given_down_input_scale():
     Wd = L.Packed(to_dev(qd), to_dev(tile(sd)), to_dev(gd), E * H, I, 1)
     moe = L.MoEExperts(Wgu, Wd, E, H, I, max_rows=R, out_dtype=0, mid_dtype=0, fused_swiglu=True)
     xd, rid, offd, sld = bf16_dev(x), to_dev(r["row_index"]), to_dev(off), to_dev(r["slot"].astype(np.int32))
-    gs_h = to_np(L.calibrate_h_scale(moe, xd, rid, offd, slot=sld, margin=1.25))
+    # a dynamic forward first: its requantize leaves s_g of each expert's max |h| in moe.amax
+    moe.forward(xd, rid, offd, slot=sld)
+    gs_dyn = to_np(moe.amax).copy()
     h_dyn = to_np(moe.h[:R]).copy()
+    # margin 1: the calibrated global is the dynamic one, bit for bit
+    gs_1 = to_np(L.calibrate_h_scale(moe, xd, rid, offd, slot=sld, margin=1.0))
+    assert np.array_equal(gs_1.view(np.uint32), gs_dyn.view(np.uint32))
+    gs_h = to_np(L.calibrate_h_scale(moe, xd, rid, offd, slot=sld, margin=1.25))
+    assert np.array_equal(to_np(moe.h[:R]), h_dyn)
+    hf = synthetic.bf16_bits_to_f32(h_dyn)
+    for e in range(E):
+        a = float(np.abs(hf[off[e]:off[e + 1]]).max()) if off[e + 1] > off[e] else 0.0
+        assert gs_1[e] == np.float32(oracle.global_scale_from_amax(a))
+        assert gs_h[e] == np.float32(oracle.global_scale_from_amax(float(np.float32(a) * np.float32(1.25))))
     s = status_word()
     y2 = moe.forward(xd, rid, offd, dev_status=s, slot=sld)
     torch.cuda.synchronize()
@@ -1158,11 +1232,50 @@ def test_moe_layer_given_down_input_scale():
     q2, sf2, _, st = oracle.quantize(h_dyn, None, off, global_scale=gs_h)
     assert st == 0
     assert np.array_equal(to_np(moe.a2.q)[rows], q2)
+    # with 25 % headroom no block scale of h saturates
+    assert (sf2 < 0x7E).all() and (sf2.max() >> 3) >= 14
     a2 = oracle.dequantize_f64(q2, sf2, oracle.rows_global_scale(gs_h, off, R))
     bd = oracle.dequantize_f64(qd, sd, np.repeat(gd, H)).reshape(E, H, I)
     y2_ref, s2_ref = oracle.grouped_gemm_f64(a2, bd, off)
     ok, err, bound = gemm_tol(to_np(y2), y2_ref, s2_ref)
     assert ok.all(), (err / bound).max()
+
+
+def test_global_scale_from_amax_entry_point():
+    """The global-scale rule as its own call equals the oracle's rule on amaxes
+    over the whole fp32 range, with and without a margin; zero gives 1, a
+    non-finite amax gives NaN and NVFP4_ERR_NONFINITE; negative amaxes count by
+    magnitude; in place works."""
+    nv = nvmod()
+    rng = np.random.default_rng(9)
+    vals = np.concatenate([
+        [0.0, -0.0, 1.0, 2688.0, 448.0, 6.0, 3.0e38, 1e-45, 1.17549435e-38, -7.5],
+        np.exp2(rng.uniform(-140, 127, 4000)),
+        rng.standard_normal(1000) * 100,
+    ]).astype(np.float32)
+    for margin in (1.0, 1.25, 0.75):
+        a = to_dev(vals)
+        out = torch.empty_like(a)
+        s = status_word()
+        nv.nvfp4_global_scale_from_amax(a, vals.size, margin, out, s)
+        torch.cuda.synchronize()
+        got = to_np(out)
+        m = np.float32(margin)
+        want = np.array([oracle.global_scale_from_amax(float(abs(v) if margin == 1.0 else np.float32(abs(v)) * m))
+                         for v in vals], np.float32)
+        fin = np.isfinite(want)
+        assert np.array_equal(got[fin].view(np.uint32), want[fin].view(np.uint32))
+        assert np.isnan(got[~fin]).all()
+        assert int(s.item()) == (16 if (~fin).any() else 0)
+    bad = to_dev(np.array([1.0, np.inf, np.nan, 5.0], np.float32))
+    s = status_word()
+    nv.nvfp4_global_scale_from_amax(bad, 4, 1.0, bad, s)        # in place
+    torch.cuda.synchronize()
+    g = to_np(bad)
+    assert int(s.item()) == 16 and np.isnan(g[1]) and np.isnan(g[2])
+    assert g[0] == np.float32(1.0) / np.float32(2688.0) and g[3] == np.float32(5.0) / np.float32(2688.0)
+    for margin in (0.0, -1.0, float("inf"), float("nan")):
+        assert nv.nvfp4_global_scale_from_amax(bad, 4, margin, bad, None, check=False) == nv.ERR_INVALID_ARG
 
 
 # --------------------------------------------------------------------------- SwiGLU + requantize
@@ -1292,14 +1405,26 @@ def test_route_bitexact(T, E, k):
     assert np.array_equal(to_np(slot), slot_ref)
 
 
-def test_route_bad_index_status():
+@pytest.mark.parametrize("T,E,k,nbad", [(3, 4, 2, 1), (1000, 64, 8, 300), (600, 2048, 3, 17), (5, 7, 2, 10)])
+def test_route_bad_index_status(T, E, k, nbad):
+    """Out-of-range expert ids: the device drops those choices exactly as the
+    oracle's routing does (slot -1, not counted, no routed row), reports
+    NVFP4_ERR_INDEX, and every other output equals the oracle's in full."""
     L = layer()
-    ids = np.array([[0, 1], [2, 9], [1, 3]], dtype=np.int32)
+    rng = np.random.default_rng(T + nbad)
+    ids = np.stack([rng.choice(E, size=k, replace=False) for _ in range(T)]).astype(np.int32)
+    flat = ids.reshape(-1)
+    pos = rng.choice(T * k, size=nbad, replace=False)
+    flat[pos] = np.where(rng.random(nbad) < 0.5, E + rng.integers(0, 1 << 20, nbad), -1 - rng.integers(0, 1 << 20, nbad))
+    off_ref, ri_ref, slot_ref, st = oracle.route(ids, E)
+    assert st == 1
     s = status_word()
-    off, ri, slot = L.route(to_dev(ids), 4, dev_status=s)
+    off, ri, slot = L.route(to_dev(ids), E, dev_status=s)
     torch.cuda.synchronize()
     assert int(s.item()) == 19
-    assert to_np(slot)[1, 1] == -1 and to_np(off)[-1] == 5
+    assert np.array_equal(to_np(off), off_ref)
+    assert np.array_equal(to_np(ri)[:int(off_ref[-1])], ri_ref)
+    assert np.array_equal(to_np(slot), slot_ref)
 
 
 @pytest.mark.parametrize("ydt", [0, 1])

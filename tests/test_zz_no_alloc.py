@@ -88,6 +88,27 @@ def test_noalloc_matches_workspace_path_twice(lib):
         assert np.array_equal(u, v)
 
 
+def test_noalloc_at_the_group_limit(lib):
+    """The static array's edge: NOALLOC_MAX_GROUPS groups, most of them empty and
+    a few ragged, twice in a row with different magnitudes."""
+    import nvfp4_w4a4_quantized_04_b200 as nv
+    G = nv.NOALLOC_MAX_GROUPS
+    rng = np.random.default_rng(5)
+    counts = np.zeros(G, np.int64)
+    busy = rng.choice(G, size=40, replace=False)
+    busy[:2] = [0, G - 1]                        # the first and the last group hold rows
+    counts[busy] = rng.integers(1, 300, size=busy.size)
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    R = int(offsets[-1])
+    T = 700
+    ri = rng.integers(0, T, size=R).astype(np.int32)
+    for seed, sigma in ((31, 1.0), (32, 1e-4)):
+        x = synthetic.gaussian_bf16(seed, synthetic.STREAMS["x"], (T, 256), sigma=sigma, outlier_frac=0.002)
+        a, b = _quantize_both(lib, x, ri, offsets, G, 1)
+        for u, v in zip(a, b):
+            assert np.array_equal(u, v)
+
+
 def test_noalloc_rejects_too_many_groups(lib):
     import nvfp4_w4a4_quantized_04_b200 as nv
     fake = ctypes.c_void_p(1 << 20)
