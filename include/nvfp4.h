@@ -385,11 +385,14 @@ nvfp4_status nvfp4_grouped_gemm_w4a16(const void *x, int64_t ld_x, int64_t x_row
  * nvfp4_gemm_select_kernel -- which grouped GEMM kernel nvfp4_grouped_gemm runs
  * (process-wide; a tuning and testing switch, not part of the pages' method):
  *   0  automatic (default): one CTA per 128-row weight tile, with 512-element
- *      K stages when K % 512 == 0 (NVFP4 operands) and 256-element stages
- *      otherwise;
+ *      K stages when K % 512 == 0 and 256-element stages otherwise; the
+ *      512-element kernel takes tiles of at most 64 tokens in a ring of three
+ *      slots when the experts average at most 16 routed rows (M_total <=
+ *      16 * num_experts), of at most 192 tokens in two slots otherwise;
  *   1  one CTA per tile, 256-element K stages;  2  CTA pairs (tcgen05
  *      cta_group::2, 256 weight rows per tile; N % 256 != 0 is then
- *      NVFP4_ERR_UNSUPPORTED_SHAPE).
+ *      NVFP4_ERR_UNSUPPORTED_SHAPE);  3  the three-slot, 64-token ring
+ *      whenever K % 512 == 0 (256-element stages otherwise).
  * Both give the same Y up to the fp32 accumulation order inside a tile.
  * Returns NVFP4_ERR_INVALID_ARG for another mode.
  */

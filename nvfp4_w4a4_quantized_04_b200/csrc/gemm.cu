@@ -299,11 +299,28 @@ using namespace nvfp4;
 
 namespace {
 
-// 0 automatic (512-element stages when K % 512 == 0, else one CTA per tile with
-// 256-element stages), 1 one CTA per tile with 256-element stages, 2 CTA pairs
+// 0 automatic (512-element stages when K % 512 == 0, with the deep ring when
+// the groups average at most 16 rows; else one CTA per tile with 256-element
+// stages), 1 one CTA per tile with 256-element stages, 2 CTA pairs, 3 the
+// deep 512-element ring whenever K % 512 == 0
 std::atomic<int> g_gemm_kernel{0};
 
 }  // namespace
+
+// One CTA per SM, but no more CTAs than tiles can exist: each expert has at
+// most ceil(m_e / BN) <= m_e / BN + 1 token chunks per 128-row weight block.
+int persistent_grid(int64_t M_total, int E, int64_t N) {
+  const int64_t bound = (N / gemm::BM) * ((M_total + gemm::BN - 1) / gemm::BN + E);
+  const int sms = host::sm_count();
+  return (int)(bound < sms ? bound : sms);
+}
+
+// The deep ring (64-token tiles, three slots) in mode 3, and in mode 0 for
+// problems of few tokens per expert.
+bool deep_ring(int64_t M_total, int E) {
+  const int mode = g_gemm_kernel.load();
+  return mode == 3 || (mode == 0 && M_total <= gemm::kDeepRingMaxRowsPerExpert * (int64_t)E);
+}
 
 extern "C" nvfp4_status nvfp4_grouped_gemm(const uint8_t *a_q, const uint8_t *a_sf, const float *a_gs,
                                            const uint8_t *b_q, const uint8_t *b_sf, const float *b_gs,
@@ -331,9 +348,9 @@ extern "C" nvfp4_status nvfp4_grouped_gemm(const uint8_t *a_q, const uint8_t *a_
   if (g_gemm_kernel == 2)
     return gemm::launch_grouped_gemm_pair(a_q, a_sf, a_gs, b_q, b_sf, b_gs, expert_offsets, E, M_total, N, K, y,
                                           out_dtype, swiglu, amax_out, dev_status, stream);
-  if (g_gemm_kernel == 0 && K % 512 == 0)
+  if ((g_gemm_kernel == 0 || g_gemm_kernel == 3) && K % 512 == 0)
     return gemm::launch_grouped_gemm_k512(a_q, a_sf, a_gs, b_q, b_sf, b_gs, expert_offsets, E, M_total, N, K, y,
-                                          out_dtype, swiglu, amax_out, nullptr, false, dev_status, stream);
+                                          out_dtype, swiglu, amax_out, nullptr, false, deep_ring(M_total, E), dev_status, stream);
   const int64_t x_rows = nvfp4_padded_rows_bound(M_total, E);
   CUtensorMap tw, tx128, tx64, tx32;
   if (!gemm::make_map(&tw, b_q, (uint64_t)E * N, (uint64_t)K / 2, 128)) return NVFP4_ERR_CUDA;
@@ -344,7 +361,7 @@ extern "C" nvfp4_status nvfp4_grouped_gemm(const uint8_t *a_q, const uint8_t *a_
   auto kern = variant == 2 ? gemm::grouped_gemm_kernel<true, true>
                            : (variant == 1 ? gemm::grouped_gemm_kernel<false, true> : gemm::grouped_gemm_kernel<false, false>);
   if (!host::set_max_dynamic_smem(reinterpret_cast<const void *>(kern), gemm::SMEM_BYTES)) return NVFP4_ERR_CUDA;
-  kern<<<host::sm_count(), gemm::NUM_THREADS, gemm::SMEM_BYTES, stream>>>(tw, tx128, tx64, tx32, b_sf, a_sf, b_gs, a_gs,
+  kern<<<persistent_grid(M_total, E, N), gemm::NUM_THREADS, gemm::SMEM_BYTES, stream>>>(tw, tx128, tx64, tx32, b_sf, a_sf, b_gs, a_gs,
                                                                expert_offsets, E, (int)M_total, (int)N, (int)K, y,
                                                                amax_out, dev_status, gemm::HQuantOut{});
   return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
@@ -358,7 +375,7 @@ extern "C" nvfp4_status nvfp4_gemm_set_wait_budget(int64_t cycles) {
 }
 
 extern "C" nvfp4_status nvfp4_gemm_select_kernel(int mode) {
-  if (mode < 0 || mode > 2) return NVFP4_ERR_INVALID_ARG;
+  if (mode < 0 || mode > 3) return NVFP4_ERR_INVALID_ARG;
   g_gemm_kernel = mode;
   return NVFP4_OK;
 }
@@ -384,9 +401,9 @@ extern "C" nvfp4_status nvfp4_grouped_gemm_swiglu_nvfp4(const uint8_t *a_q, cons
   hq.gs = h_gs;
   hq.q = h_q;
   hq.sf = h_sf;
-  if (g_gemm_kernel == 0 && K % 512 == 0)
+  if ((g_gemm_kernel == 0 || g_gemm_kernel == 3) && K % 512 == 0)
     return gemm::launch_grouped_gemm_k512(a_q, a_sf, a_gs, b_q, b_sf, b_gs, expert_offsets, E, M_total, N, K, nullptr,
-                                          NVFP4_OUT_BF16, true, nullptr, &hq, false, dev_status, stream);
+                                          NVFP4_OUT_BF16, true, nullptr, &hq, false, deep_ring(M_total, E), dev_status, stream);
   const int64_t x_rows = nvfp4_padded_rows_bound(M_total, E);
   CUtensorMap tw, tx128, tx64, tx32;
   if (!gemm::make_map(&tw, b_q, (uint64_t)E * N, (uint64_t)K / 2, 128)) return NVFP4_ERR_CUDA;
@@ -395,7 +412,7 @@ extern "C" nvfp4_status nvfp4_grouped_gemm_swiglu_nvfp4(const uint8_t *a_q, cons
   if (!gemm::make_map(&tx32, a_q, (uint64_t)x_rows, (uint64_t)K / 2, 32)) return NVFP4_ERR_CUDA;
   auto kern = gemm::grouped_gemm_kernel<true, true, true>;
   if (!host::set_max_dynamic_smem(reinterpret_cast<const void *>(kern), gemm::SMEM_BYTES)) return NVFP4_ERR_CUDA;
-  kern<<<host::sm_count(), gemm::NUM_THREADS, gemm::SMEM_BYTES, stream>>>(tw, tx128, tx64, tx32, b_sf, a_sf, b_gs, a_gs,
+  kern<<<persistent_grid(M_total, E, N), gemm::NUM_THREADS, gemm::SMEM_BYTES, stream>>>(tw, tx128, tx64, tx32, b_sf, a_sf, b_gs, a_gs,
                                                                expert_offsets, E, (int)M_total, (int)N, (int)K, nullptr,
                                                                nullptr, dev_status, hq);
   return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
@@ -420,9 +437,9 @@ extern "C" nvfp4_status mxfp4_grouped_gemm(const uint8_t *a_q, const uint8_t *a_
   if ((reinterpret_cast<uintptr_t>(a_q) | reinterpret_cast<uintptr_t>(b_q) | reinterpret_cast<uintptr_t>(a_sf) |
        reinterpret_cast<uintptr_t>(b_sf) | reinterpret_cast<uintptr_t>(y)) & 15u)
     return NVFP4_ERR_INVALID_ARG;
-  if (g_gemm_kernel == 0 && K % 512 == 0)
+  if ((g_gemm_kernel == 0 || g_gemm_kernel == 3) && K % 512 == 0)
     return gemm::launch_grouped_gemm_k512(a_q, a_sf, nullptr, b_q, b_sf, nullptr, expert_offsets, E, M_total, N, K, y,
-                                          out_dtype, false, nullptr, nullptr, true, dev_status, stream);
+                                          out_dtype, false, nullptr, nullptr, true, deep_ring(M_total, E), dev_status, stream);
   const int64_t x_rows = nvfp4_padded_rows_bound(M_total, E);
   CUtensorMap tw, tx128, tx64, tx32;
   if (!gemm::make_map(&tw, b_q, (uint64_t)E * N, (uint64_t)K / 2, 128)) return NVFP4_ERR_CUDA;
@@ -433,7 +450,7 @@ extern "C" nvfp4_status mxfp4_grouped_gemm(const uint8_t *a_q, const uint8_t *a_
   auto kern = variant == 5 ? gemm::grouped_gemm_kernel<false, true, false, true>
                            : gemm::grouped_gemm_kernel<false, false, false, true>;
   if (!host::set_max_dynamic_smem(reinterpret_cast<const void *>(kern), gemm::SMEM_BYTES)) return NVFP4_ERR_CUDA;
-  kern<<<host::sm_count(), gemm::NUM_THREADS, gemm::SMEM_BYTES, stream>>>(tw, tx128, tx64, tx32, b_sf, a_sf, nullptr, nullptr,
+  kern<<<persistent_grid(M_total, E, N), gemm::NUM_THREADS, gemm::SMEM_BYTES, stream>>>(tw, tx128, tx64, tx32, b_sf, a_sf, nullptr, nullptr,
                                                                expert_offsets, E, (int)M_total, (int)N, (int)K, y,
                                                                nullptr, dev_status, gemm::HQuantOut{});
   return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;

@@ -11,6 +11,8 @@
 #include <cudaTypedefs.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "common.cuh"
 
 namespace nvfp4 {
@@ -137,6 +139,12 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
       " [%0], [%1, {%2, %3}], [%4], %5;"
       :: "r"(dst), "l"(map), "r"(x), "r"(y), "r"(bar), "l"(policy) : "memory");
+}
+
+// Fetch a tensor map (a __grid_constant__ kernel parameter) into the TMA
+// descriptor cache ahead of its first copy.
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
+  asm volatile("prefetch.tensormap [%0];" :: "l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
@@ -344,19 +352,23 @@ struct Tile {
   int n_valid;    // tokens in this tile (1..192)
 };
 
-__device__ __forceinline__ int chunks_of(int m) { return (m + BN - 1) / BN; }
+// kCap: the most tokens one tile takes (192, or 64 for the deep-ring kernel
+// of decode-sized groups); chunks start on 64-row boundaries either way.
+template <int kCap = BN>
+__device__ __forceinline__ int chunks_of(int m) { return (m + kCap - 1) / kCap; }
 
 // Tile t of a grid whose weight blocks are `wrows` rows (128 for one CTA, 256
 // for a pair); `sub` is the CTA's 128-row half of the block.  With the SwiGLU
 // epilogue the fused gate_up weight is stored in 32-row groups (16 gate rows,
 // then the 16 matching up rows), so 128 weight rows give 64 h columns.
-template <bool kSwiglu>
+template <bool kSwiglu, int kCap = BN>
 __device__ __forceinline__ Tile decode_tile(int t, const int32_t *s_off, const int32_t *s_slot,
                                             const int32_t *s_tile, int E, int N, int wrows, int sub) {
+  static_assert(kCap % 64 == 0 && kCap <= BN, "tiles start on 64-row boundaries and fit the accumulator");
   Tile T;
   const int e = upper_group(s_tile, E, t);
   const int m_e = s_off[e + 1] - s_off[e];
-  const int nch = chunks_of(m_e);
+  const int nch = chunks_of<kCap>(m_e);
   const int csz = ((m_e + nch - 1) / nch + 63) & ~63;
   const int local = t - s_tile[e];
   const int mt = local / nch, ch = local - mt * nch;
@@ -378,6 +390,7 @@ __device__ __forceinline__ Tile decode_tile(int t, const int32_t *s_off, const i
 // the offsets: unless they start at 0, never decrease and end at M_total, the
 // call reports NVFP4_ERR_INDEX and leaves s_tile[E] = 0, so the kernel runs no
 // tile (no copy, no MMA, no store).
+template <int kCap = BN>
 __device__ inline void build_tile_tables(const int32_t *__restrict__ expert_offsets, int E, int M_total,
                                          int n_mtiles, int32_t *s_off, int32_t *s_slot, int32_t *s_tile,
                                          int32_t *s_scratch, int32_t *dev_status) {
@@ -406,7 +419,7 @@ __device__ inline void build_tile_tables(const int32_t *__restrict__ expert_offs
   for (int e = e0; e < e1; ++e) {
     const int32_t m = s_off[e + 1] - s_off[e];
     ls += (m + kSlotAlign - 1) / kSlotAlign * kSlotAlign;
-    lt += n_mtiles * chunks_of(m);
+    lt += n_mtiles * chunks_of<kCap>(m);
   }
   int32_t is = ls, it = lt;
 #pragma unroll
@@ -431,7 +444,7 @@ __device__ inline void build_tile_tables(const int32_t *__restrict__ expert_offs
     s_slot[e] = rs;
     s_tile[e] = rt;
     rs += (m + kSlotAlign - 1) / kSlotAlign * kSlotAlign;
-    rt += n_mtiles * chunks_of(m);
+    rt += n_mtiles * chunks_of<kCap>(m);
   }
   if (e1 == E && e0 < e1) { s_slot[E] = rs; s_tile[E] = rt; }
   __syncthreads();
@@ -702,56 +715,99 @@ inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// 2-D uint8 view [rows, row_bytes] with a {128 bytes, box_rows} box, 128-byte swizzle.
-inline bool make_map(CUtensorMap *map, const void *base, uint64_t rows, uint64_t row_bytes, uint32_t box_rows) {
+// A uint8 tensor map of rank 2 or 3, from a process-wide cache keyed by its
+// arguments.  Encoding is several microseconds of host work per map, which
+// would otherwise dominate the call of a small GEMM.  A map holds only an
+// address and a shape, never ownership, so an entry stays valid for whatever
+// buffer later sits at the same address.
+inline bool encode_u8_map(CUtensorMap *map, int rank, const void *base, const cuuint64_t *dims,
+                          const cuuint64_t *strides, const cuuint32_t *box, CUtensorMapSwizzle swizzle) {
+  struct Entry {
+    bool used;
+    int rank, swizzle;
+    const void *base;
+    cuuint64_t dims[3], strides[2];
+    cuuint32_t box[3];
+    CUtensorMap map;
+  };
+  static std::mutex mu;
+  static Entry cache[64];
+  static int next = 0;
+  auto same = [&](const Entry &e) {
+    if (!e.used || e.rank != rank || e.swizzle != (int)swizzle || e.base != base) return false;
+    for (int i = 0; i < rank; ++i)
+      if (e.dims[i] != dims[i] || e.box[i] != box[i] || (i < rank - 1 && e.strides[i] != strides[i])) return false;
+    return true;
+  };
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    for (const Entry &e : cache)
+      if (same(e)) { *map = e.map; return true; }
+  }
   auto enc = tensor_map_encoder();
   if (!enc) return false;
+  cuuint32_t estr[3] = {1, 1, 1};
+  if (enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, (cuuint32_t)rank, const_cast<void *>(base), dims, strides, box, estr,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  std::lock_guard<std::mutex> lock(mu);
+  Entry &e = cache[next];
+  next = (next + 1) % 64;
+  e.used = true;
+  e.rank = rank;
+  e.swizzle = (int)swizzle;
+  e.base = base;
+  for (int i = 0; i < rank; ++i) {
+    e.dims[i] = dims[i];
+    e.box[i] = box[i];
+    if (i < rank - 1) e.strides[i] = strides[i];
+  }
+  e.map = *map;
+  return true;
+}
+
+// 2-D uint8 view [rows, row_bytes] with a {128 bytes, box_rows} box, 128-byte swizzle.
+inline bool make_map(CUtensorMap *map, const void *base, uint64_t rows, uint64_t row_bytes, uint32_t box_rows) {
   cuuint64_t dims[2] = {row_bytes, rows};
   cuuint64_t strides[1] = {row_bytes};
   cuuint32_t box[2] = {128, box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return encode_u8_map(map, 2, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 // Token scales in the MMA-tiled layout viewed as [row block][K/32][256 bytes]:
 // one {256, 8, 2} box is the 2 KB of one K stage for two consecutive 128-row
 // blocks (a block past the end reads as zeros).
 inline bool make_map_sfx(CUtensorMap *map, const void *base, uint64_t row_blocks, uint64_t K) {
-  auto enc = tensor_map_encoder();
-  if (!enc) return false;
   cuuint64_t dims[3] = {256, K / 32, row_blocks};
   cuuint64_t strides[2] = {256, K * 8};
   cuuint32_t box[3] = {256, 8, 2};
-  cuuint32_t estr[3] = {1, 1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return encode_u8_map(map, 3, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
 // Weight scales in the MMA-tiled layout viewed as [row block][K/32][256 bytes]:
 // one {256, 8, 1} box is the 2 KB of one K stage of one 128-row block.
 inline bool make_map_sfw(CUtensorMap *map, const void *base, uint64_t row_blocks, uint64_t K) {
-  auto enc = tensor_map_encoder();
-  if (!enc) return false;
   cuuint64_t dims[3] = {256, K / 32, row_blocks};
   cuuint64_t strides[2] = {256, K * 8};
   cuuint32_t box[3] = {256, 8, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return encode_u8_map(map, 3, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
 // The 512-element-stage kernel's launch (gemm_k512.cu), K % 512 == 0;
 // hq != nullptr selects the SwiGLU epilogue that writes NVFP4 h; mx selects
-// MXFP4 operands (no global scales: a_gs and b_gs are not read).
+// MXFP4 operands (no global scales: a_gs and b_gs are not read); deep selects
+// the ring of three slots for tiles of at most 64 tokens (few tokens per
+// expert) instead of two slots for up to 192.
 nvfp4_status launch_grouped_gemm_k512(const uint8_t *a_q, const uint8_t *a_sf, const float *a_gs,
                                       const uint8_t *b_q, const uint8_t *b_sf, const float *b_gs,
                                       const int32_t *expert_offsets, int E, int64_t M_total, int64_t N, int64_t K,
                                       void *y, nvfp4_out_dtype out_dtype, bool swiglu, float *amax_out,
-                                      const HQuantOut *hq, bool mx, int32_t *dev_status, cudaStream_t stream);
+                                      const HQuantOut *hq, bool mx, bool deep, int32_t *dev_status,
+                                      cudaStream_t stream);
+// Rows per expert on average at or below which the automatic choice takes the
+// deep ring (the decode regime: 640 routed rows over 384 experts).
+constexpr int64_t kDeepRingMaxRowsPerExpert = 16;
 // Its copy of the main-loop wait budget (see c_wait_budget).
 nvfp4_status set_wait_budget_k512(long long cycles);
 

@@ -430,15 +430,10 @@ namespace {
 // 2-D uint8 view [rows, row_bytes] with a {16 bytes, box_rows} box, no swizzle
 // (row-major E4M3 scales: 16 per 256-element K stage).
 bool make_map_scales16(CUtensorMap *map, const void *base, uint64_t rows, uint64_t row_bytes, uint32_t box_rows) {
-  auto enc = gemm::tensor_map_encoder();
-  if (!enc) return false;
   cuuint64_t dims[2] = {row_bytes, rows};
   cuuint64_t strides[1] = {row_bytes};
   cuuint32_t box[2] = {16, box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return gemm::encode_u8_map(map, 2, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
 // Upper bound on the 8-token chunks of all experts: sum ceil(n_e / 8).

@@ -36,21 +36,23 @@ def status_word():
     return torch.zeros(1, dtype=torch.int32, device="cuda")
 
 
-@pytest.fixture(params=[0, 1, 2], ids=["auto", "one_cta", "cta_pair"])
+@pytest.fixture(params=[0, 1, 2, 3], ids=["auto", "one_cta", "cta_pair", "deep_ring"])
 def gemm_kernel(request):
     """Run the test on each grouped GEMM kernel: automatic (512-element K
-    stages when K % 512 == 0), one CTA per tile with 256-element stages, and
-    the CTA-pair kernel."""
+    stages when K % 512 == 0), one CTA per tile with 256-element stages, the
+    CTA-pair kernel, and the 512-element kernel's deep ring (tiles of at most
+    64 tokens, three slots)."""
     nv = nvmod()
     nv.nvfp4_gemm_select_kernel(request.param)
     yield request.param
     nv.nvfp4_gemm_select_kernel(0)
 
 
-@pytest.fixture(params=[0, 1], ids=["auto", "k256"])
+@pytest.fixture(params=[0, 1, 3], ids=["auto", "k256", "deep_ring"])
 def mx_kernel(request):
-    """Run an MXFP4 GEMM test on both kernels that take MXFP4 operands: 512-element
-    K stages (automatic when K % 512 == 0) and 256-element stages."""
+    """Run an MXFP4 GEMM test on the kernels that take MXFP4 operands: 512-element
+    K stages (automatic when K % 512 == 0; also with the deep ring) and
+    256-element stages."""
     nv = nvmod()
     nv.nvfp4_gemm_select_kernel(request.param)
     yield request.param
@@ -405,6 +407,38 @@ def test_dequantize_bitexact(layout):
     torch.cuda.synchronize()
     assert np.array_equal(to_np(y32).view(np.uint32), ref32.view(np.uint32))
     assert np.array_equal(to_np(y16), ref16)
+
+
+@pytest.mark.parametrize("R,K", [(333, 1088), (1, 64), (7, 48), (4099, 256)])
+@pytest.mark.parametrize("y_offset", [0, 16])
+def test_dequantize_ragged_and_alignments(R, K, y_offset):
+    """Ungrouped dequantize: block counts that are not a multiple of the
+    kernel's per-warp step, every layout and output type, and an output that is
+    16 but not 32 bytes aligned (the per-thread kernel then runs instead of the
+    flat one).  Bit-exact either way."""
+    nv = nvmod()
+    rng = np.random.default_rng(R + K)
+    q = rng.integers(0, 256, (R, K // 2), dtype=np.uint8)
+    sf = rng.integers(0, 0x7F, (R, K // 16), dtype=np.uint8)
+    gs = np.array([2.0 ** -7 * 1.375], dtype=np.float32)
+    ref32 = oracle.dequantize(q, sf, np.full(R, gs[0], np.float32))
+    ref16 = oracle.dequantize(q, sf, np.full(R, gs[0], np.float32), out="bf16")
+    layouts = [0, 1] if K % 64 == 0 else [0]
+    for layout in layouts:
+        if layout == 1:
+            sfa = np.zeros(((R + 127) // 128 * 128, K // 16), np.uint8)
+            sfa[:R] = sf
+            sfd = to_dev(tile(sfa))
+        else:
+            sfd = to_dev(sf.reshape(-1))
+        for out_dtype, ref, esz in ((0, ref32.view(np.uint32), 4), (1, ref16, 2)):
+            buf = torch.zeros(R * K * esz + 64, dtype=torch.uint8, device="cuda")
+            base = (-buf.data_ptr()) % 32 + y_offset
+            yv = buf[base:base + R * K * esz]
+            nv.nvfp4_dequantize(to_dev(q), sfd, layout, to_dev(gs), None, 1, R, K, yv, out_dtype)
+            torch.cuda.synchronize()
+            got = to_np(yv).view(np.uint32 if esz == 4 else np.uint16).reshape(R, K)
+            assert np.array_equal(got, ref), (layout, out_dtype)
 
 
 def test_dequantize_grouped_slots():
@@ -792,7 +826,7 @@ def test_gemm_dense_config1(out_dtype, gemm_kernel):
         assert np.array_equal(y, synthetic.f32_to_bf16_bits(y32))
 
 
-@pytest.mark.parametrize("mode", [0, 1], ids=["k512", "k256"])
+@pytest.mark.parametrize("mode", [0, 1, 3], ids=["k512", "k256", "k512_deep"])
 def test_gemm_wait_timeout_reports_and_recovers(mode):
     """The failure path of the one-CTA GEMM without any GPU fault: with a
     1-cycle budget on its main-loop waits, the first wait that is not already
