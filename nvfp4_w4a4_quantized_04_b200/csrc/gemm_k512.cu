@@ -43,8 +43,9 @@ struct Ring {
   static constexpr int OFF_SFX = OFF_SFW + kSlots * SFW_STAGE2;
   static constexpr int OFF_EPI = OFF_SFX + kSlots * SFX_STAGE2;
   static constexpr int OFF_BAR = OFF_EPI + 4 * EPI_WARP_BYTES;
-  // wfull[S], wempty[S], xfull[S], xempty[S], sf_full[2], sf_free[2], acc_full[2], acc_empty[2], drain
-  static constexpr int NUM_BARS = 4 * kSlots + 2 + 2 + 2 + 2 + 1;
+  // wfull[S], wempty[S], xfull[S], xempty[S], sf_full[2], sf_free[2], acc_full[2], acc_empty[2], drain,
+  // sfw_data[S], sfx_data[S]
+  static constexpr int NUM_BARS = 4 * kSlots + 2 + 2 + 2 + 2 + 1 + 2 * kSlots;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int OFF_GROUPS = OFF_MISC + 16;
   static constexpr int SMEM_BYTES = OFF_GROUPS + GROUP_TABLE_BYTES + 1024;
@@ -132,6 +133,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_k512_kernel(
   const uint32_t bar_acc_full = bar_sf_free + 16;
   const uint32_t bar_acc_empty = bar_acc_full + 16;
   const uint32_t bar_drain = bar_acc_empty + 16;
+  // A slot's scale bytes land on barriers of their own (weight and token
+  // scales, one per producer), so the scale warps can stage them into tensor
+  // memory while the slot's large weight and token copies are still arriving.
+  const uint32_t bar_sfw_data = bar_drain + 8;            // [S_W], count 1
+  const uint32_t bar_sfx_data = bar_sfw_data + 8 * S_W;   // [S_X], count 1
   volatile uint32_t *tmem_holder = reinterpret_cast<volatile uint32_t *>(smem + OFF_MISC);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
   int32_t *s_off = reinterpret_cast<int32_t *>(smem + OFF_GROUPS);
@@ -145,8 +151,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_k512_kernel(
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
-    for (int s = 0; s < S_W; ++s) { mbar_init(bar_wfull + 8 * s, 1); mbar_init(bar_wempty + 8 * s, 1); }
-    for (int s = 0; s < S_X; ++s) { mbar_init(bar_xfull + 8 * s, 1); mbar_init(bar_xempty + 8 * s, 1); }
+    for (int s = 0; s < S_W; ++s) {
+      mbar_init(bar_wfull + 8 * s, 1);
+      mbar_init(bar_wempty + 8 * s, 1);
+      mbar_init(bar_sfw_data + 8 * s, 1);
+    }
+    for (int s = 0; s < S_X; ++s) {
+      mbar_init(bar_xfull + 8 * s, 1);
+      mbar_init(bar_xempty + 8 * s, 1);
+      mbar_init(bar_sfx_data + 8 * s, 1);
+    }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar_sf_full + 8 * b, 128);
       mbar_init(bar_sf_free + 8 * b, 1);
@@ -185,6 +199,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_k512_kernel(
       }
       const uint64_t pol = is_w ? policy_evict_first() : policy_evict_last();
       const uint32_t bar_full = is_w ? bar_wfull : bar_xfull, bar_empty = is_w ? bar_wempty : bar_xempty;
+      const uint32_t bar_sfd = is_w ? bar_sfw_data : bar_sfx_data;
       int stage = 0;
       uint32_t phase = 0;
       bool armed[S_W] = {}; uint32_t armed_parity[S_W] = {};
@@ -195,21 +210,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_k512_kernel(
         const int nrb = ((T.x_row0 & 127) + T.n_valid + 127) >> 7;
         const int xbox = token_box_rows(T.n_valid);
         const CUtensorMap *xmap = xbox == 32 ? &tmap_x32 : xbox == 64 ? &tmap_x64 : xbox == 128 ? &tmap_x128 : &tmap_x192;
-        const uint32_t bytes = is_w ? (uint32_t)(W_STAGE2 + 2 * kHalfSf) : (uint32_t)(2 * xbox * 128 + nrb * 2 * kHalfSf);
+        const uint32_t bytes = is_w ? (uint32_t)W_STAGE2 : (uint32_t)(2 * xbox * 128);
+        const uint32_t sf_bytes = is_w ? 2 * kHalfSf : (uint32_t)nrb * 2 * kHalfSf;
         const uint8_t *sfw_tile = w_sf + (int64_t)(T.w_row0 >> 7) * sf_row_stride;
         const uint8_t *sfx_tile = x_sf + (int64_t)(xr0 >> 7) * sf_row_stride;
         for (int ks = 0; ks < ksteps; ++ks) {
           if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1, abort_flag, dev_status)) { ok = false; break; }
-          const uint32_t fb = bar_full + 8 * stage;
+          const uint32_t fb = bar_full + 8 * stage, sb = bar_sfd + 8 * stage;
+          // the scale bytes first, on their own barrier, then the large copy
+          mbar_arrive_expect_tx(sb, sf_bytes);
           mbar_arrive_expect_tx(fb, bytes);
           armed[stage] = true; armed_parity[stage] = phase;
           if (is_w) {
+            bulk_load(sbase + OFF_SFW + stage * SFW_STAGE2, sfw_tile + ks * 2 * kHalfSf, 2 * kHalfSf, sb);
             tma_load_3d(sbase + OFF_W + stage * W_STAGE2, &tmap_w, 0, T.w_row0, 2 * ks, fb, pol);
-            bulk_load(sbase + OFF_SFW + stage * SFW_STAGE2, sfw_tile + ks * 2 * kHalfSf, 2 * kHalfSf, fb);
           } else {
             for (int rb = 0; rb < nrb; ++rb)
               bulk_load(sbase + OFF_SFX + stage * SFX_STAGE2 + rb * 4096, sfx_tile + rb * sf_row_stride + ks * 2 * kHalfSf,
-                        2 * kHalfSf, fb);
+                        2 * kHalfSf, sb);
             tma_load_3d(sbase + OFF_X + stage * X_STAGE2, xmap, 0, T.x_row0, 2 * ks, fb, pol);
           }
           if (++stage == S_W) { stage = 0; phase ^= 1; }
@@ -217,8 +235,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_k512_kernel(
       }
       for (int s = 0; s < S_W; ++s) {
         if (!armed[s]) continue;
-        const long long t0 = clock64();
+        long long t0 = clock64();
         while (!mbar_try_wait(bar_full + 8 * s, armed_parity[s]) && clock64() - t0 < kWaitBudgetCycles) {}
+        t0 = clock64();
+        while (!mbar_try_wait(bar_sfd + 8 * s, armed_parity[s]) && clock64() - t0 < kWaitBudgetCycles) {}
       }
     }
   } else if (warp >= W_SF0 && warp < W_SF0 + 4) {
@@ -230,8 +250,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_k512_kernel(
       const int nrb = ((T.x_row0 & 127) + T.n_valid + 127) >> 7;
       for (int ks = 0; ks < ksteps && ok; ++ks, ++kst) {
         const uint32_t s2 = kst % S_W, par = (kst / S_W) & 1;
-        if (!mbar_wait_warp(bar_wfull + 8 * s2, par, abort_flag, dev_status)) { ok = false; break; }
-        if (!mbar_wait_warp(bar_xfull + 8 * s2, par, abort_flag, dev_status)) { ok = false; break; }
+        if (!mbar_wait_warp(bar_sfw_data + 8 * s2, par, abort_flag, dev_status)) { ok = false; break; }
+        if (!mbar_wait_warp(bar_sfx_data + 8 * s2, par, abort_flag, dev_status)) { ok = false; break; }
         for (int h = 0; h < 2; ++h, ++hk) {
           const uint32_t sb = hk & 1;
           if (hk >= 2 && !mbar_wait_warp(bar_sf_free + 8 * sb, ((hk - 2) >> 1) & 1, abort_flag, dev_status)) {
