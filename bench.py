@@ -533,6 +533,9 @@ def comp_decode_moe(device, iters, warmup, flush):
     ri = torch.from_numpy(r["row_index"]).to(device)
     off = torch.from_numpy(r["offsets"]).to(device)
     ms = timed(lambda: moe.forward(xb, ri, off), iters, warmup, flush)
+    # the activation quantize on its own: the most that folding it into the
+    # GEMM's prologue could save
+    q_ms = timed(lambda: moe._quantize_input(xb, ri, off, None, None), iters, warmup, flush)
     touched = int((np.diff(r["offsets"]) > 0).sum())
     wbytes = touched * (2 * I * H + H * I) * 0.5625
     # the whole decode block (routing order, experts, weighted combine) through
@@ -545,7 +548,7 @@ def comp_decode_moe(device, iters, warmup, flush):
     graph_ms = timed(graph.replay, iters, warmup, flush)
     del graph
     return {"workload": "decode_moe_e384_top10_zipf1.1_t64_h7168_i2048", "experts_touched": touched,
-            "routed_rows": R, "layer_ms": round(ms, 4),
+            "routed_rows": R, "layer_ms": round(ms, 4), "activation_quantize_ms": round(q_ms, 4),
             "touched_weight_gbs": round(gbs(wbytes, ms), 1),
             "roofline": {"bound": "hbm", "frac": round(gbs(wbytes, ms) / HBM_PEAK, 4), "peak": HBM_PEAK},
             "block_ms": round(block_ms, 4), "block_graph_ms": round(graph_ms, 4),

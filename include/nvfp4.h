@@ -349,8 +349,9 @@ nvfp4_status mxfp4_grouped_gemm(const uint8_t *a_q, const uint8_t *a_sf, const u
  * activations: Y_e = X_e (b_gs[e] * W_e)^T for every expert e, fp32 accumulate.
  * [P5: the MTP layer's experts are W4A16_NVFP4 -- NVFP4 weights, 16-bit
  *  activations; P1/P2: the weight format and its dequantisation.]
- * A streaming kernel for decode-sized groups (8 tokens per weight pass).  The
- * tensor-core operands are f16: the weights exactly (e2m1 * e4m3 fits f16),
+ * Two kernels (nvfp4_w4a16_select_kernel): a warp-MMA one for decode-sized
+ * groups and a tcgen05 one (dequantized weights as the A operand in tensor
+ * memory) for larger groups.  The tensor-core operands are f16: the weights exactly (e2m1 * e4m3 fits f16),
  * the activations after a per-row power-of-two scaling 2^-k that puts the row's
  * max |x| in [2^14, 2^15) -- exact for every element within 2^29 of the row
  * max, smaller ones rounded to f16's subnormal grid (error < 2^-25 * max|x|);
@@ -374,6 +375,18 @@ nvfp4_status mxfp4_grouped_gemm(const uint8_t *a_q, const uint8_t *a_sf, const u
  *               row), NVFP4_ERR_TIMEOUT.
  */
 size_t nvfp4_w4a16_workspace_size(int64_t M_total, int num_experts, int64_t K);
+/*
+ * nvfp4_w4a16_select_kernel -- which kernel nvfp4_grouped_gemm_w4a16 runs
+ * (process-wide; a tuning and testing switch, not part of the pages' method):
+ *   0  automatic (default): the warp-MMA kernel (mma.sync, 16 tokens per
+ *      weight pass) when the experts average at most 16 routed rows
+ *      (M_total <= 16 * num_experts), the tcgen05 kernel otherwise;
+ *   1  the warp-MMA kernel;  2  the tcgen05 kernel (dequantized weights as the
+ *      MMA's A operand in tensor memory, up to 64 tokens per weight pass).
+ * Both compute the same products; sums may differ in rounding order.
+ * Returns NVFP4_ERR_INVALID_ARG for another mode.
+ */
+nvfp4_status nvfp4_w4a16_select_kernel(int mode);
 nvfp4_status nvfp4_grouped_gemm_w4a16(const void *x, int64_t ld_x, int64_t x_rows, const int32_t *row_index,
                                       const uint8_t *b_q, const uint8_t *b_sf, const float *b_gs,
                                       const int32_t *expert_offsets, int num_experts, int64_t M_total,

@@ -50,6 +50,7 @@ EXPORTS = [
     "nvfp4_gemm_select_kernel", "nvfp4_grouped_gemm_w4a16", "nvfp4_grouped_gemm_swiglu_nvfp4",
     "mxfp4_quantize", "mxfp4_grouped_gemm", "nvfp4_w4a16_workspace_size",
     "nvfp4_e2m1_encode", "nvfp4_e4m3_encode", "nvfp4_gemm_set_wait_budget", "nvfp4_global_scale_from_amax",
+    "nvfp4_w4a16_select_kernel",
 ]
 NOALLOC_MAX_GROUPS = 1024
 
@@ -85,6 +86,8 @@ def load_library(path: str = LIB_PATH):
     L.nvfp4_w4a16_workspace_size.argtypes = [i64, i32, i64]
     L.nvfp4_gemm_select_kernel.restype = i32
     L.nvfp4_gemm_select_kernel.argtypes = [i32]
+    L.nvfp4_w4a16_select_kernel.restype = i32
+    L.nvfp4_w4a16_select_kernel.argtypes = [i32]
     L.nvfp4_moe_quantize.restype = i32
     L.nvfp4_moe_quantize.argtypes = [P, i64, i64, i64, P, i32, P, i32, i32, P, P, P, i32, P, P, P]
     L.nvfp4_dequantize.restype = i32
@@ -211,6 +214,13 @@ def nvfp4_gemm_select_kernel(mode: int) -> int:
     """0 automatic (one CTA per tile), 1 one CTA per tile, 2 CTA pairs (N % 256 == 0)."""
     st = load_library().nvfp4_gemm_select_kernel(mode)
     _check(st, "nvfp4_gemm_select_kernel")
+    return st
+
+
+def nvfp4_w4a16_select_kernel(mode: int) -> int:
+    """0 automatic, 1 the warp-MMA kernel (small groups), 2 the tcgen05 kernel."""
+    st = load_library().nvfp4_w4a16_select_kernel(mode)
+    _check(st, "nvfp4_w4a16_select_kernel")
     return st
 
 

@@ -1585,6 +1585,16 @@ def test_device_generator_matches_host():
 
 
 # --------------------------------------------------------------------------- W4A16 grouped GEMM
+@pytest.fixture(params=[1, 2], ids=["warp_mma", "tcgen05"], autouse=False)
+def w4a16_kernel(request):
+    """Run a W4A16 test on both kernels: the warp-MMA one (small groups) and the
+    tcgen05 one (weights as the A operand in tensor memory)."""
+    nv = nvmod()
+    nv.nvfp4_w4a16_select_kernel(request.param)
+    yield request.param
+    nv.nvfp4_w4a16_select_kernel(0)
+
+
 def _w4a16_case(seed, counts, N, K, T):
     offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
     R, E = int(offsets[-1]), len(counts)
@@ -1602,11 +1612,13 @@ def _w4a16_case(seed, counts, N, K, T):
 
 
 @pytest.mark.parametrize("K", [1024, 1280])
-def test_w4a16_grouped(K):
+def test_w4a16_grouped(K, w4a16_kernel):
     """bf16 activations x NVFP4 weights per expert vs fp64 on the exact
-    dequantized weights: groups of 0, 1, 3, 9, 17 and 64 tokens (several
-    8-token chunks), K an even and an odd number of 256-element stages."""
-    counts = [0, 1, 3, 9, 17, 64]
+    dequantized weights: groups of 0, 1, 3, 9, 17, 64, 65 and 200 tokens
+    (several 16-token chunks for the warp-MMA kernel, several 64-token items
+    and partial 16-row groups for the tcgen05 one), K an even and an odd
+    number of 256-element stages."""
+    counts = [0, 1, 3, 9, 17, 64, 65, 200]
     N, T = 256, 40
     L, x, ri, off, wp, y_ref, s_ref = _w4a16_case(30, counts, N, K, T)
     s = status_word()
@@ -1619,7 +1631,7 @@ def test_w4a16_grouped(K):
     assert np.array_equal(to_np(y16), synthetic.f32_to_bf16_bits(to_np(y)))
 
 
-def test_w4a16_scale_bytes_over_the_whole_e4m3_range():
+def test_w4a16_scale_bytes_over_the_whole_e4m3_range(w4a16_kernel):
     """Weights with random codes and block-scale bytes over every non-negative
     finite E4M3 value (zero, the subnormals, up to 448) and globals far from 1:
     the kernel's f16 code x scale products must be exact over the whole range
@@ -1649,7 +1661,7 @@ def test_w4a16_scale_bytes_over_the_whole_e4m3_range():
     assert ok.all(), (err.max(), (err / bound).max())
 
 
-def test_w4a16_swiglu_epilogue():
+def test_w4a16_swiglu_epilogue(w4a16_kernel):
     """h = bf16(silu(g) * u) from the same g, u as the plain kernel's fp32
     output (each output element sums its K terms in the same order in both
     variants): within one bf16 ulp of the oracle SwiGLU of that output."""
@@ -1666,7 +1678,7 @@ def test_w4a16_swiglu_epilogue():
     assert (d <= 1).all() and (d == 0).mean() > 0.99
 
 
-def test_w4a16_dense_and_bad_row_index():
+def test_w4a16_dense_and_bad_row_index(w4a16_kernel):
     L = layer()
     M, N, K = 5, 128, 4096
     x = synthetic.gaussian_bf16(32, synthetic.STREAMS["x"], (M, K))
@@ -1686,7 +1698,7 @@ def test_w4a16_dense_and_bad_row_index():
     assert int(s.item()) == 19
 
 
-def test_w4a16_activation_range():
+def test_w4a16_activation_range(w4a16_kernel):
     """Rows whose magnitudes sit far from 1 (1e30, 1e-30) and a row spanning
     about 2^40 of dynamic range: the per-row power-of-two scaling into f16
     keeps every row within the GEMM tolerance; a row holding an inf is
