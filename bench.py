@@ -58,9 +58,8 @@ HBM_PEAK = PEAKS.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
 # from the sources whose digest is recorded beside it.  Once those sources
 # change the figure no longer describes the kernel that runs, and the bench
 # reports the traffic as null until a new capture is recorded here.
-GATE_UP_TRAFFIC = {"ratio": 689016320 / 693108736, "capture": "128 experts, 2048 tokens",
-                   "sources_sha256": "452800defec16ce0bb6b4529b494fa6606f90d832a0cfb1286f23a1348bd8f8e"}
-GEMM_KERNEL_SOURCES = ("gemm_k512.cu", "gemm_common.cuh", "common.cuh")
+GATE_UP_TRAFFIC = {"ratio": None, "capture": "128 experts, 2048 tokens", "sources_sha256": None}
+GEMM_KERNEL_SOURCES = ("gemm.cu", "gemm_w2.cu", "gemm_common.cuh", "common.cuh")
 
 
 def gemm_sources_digest() -> str:
@@ -73,7 +72,20 @@ def gemm_sources_digest() -> str:
 
 def gate_up_traffic_ratio():
     """The recorded DRAM/algorithmic ratio, or None when the kernel changed since its capture."""
+    if GATE_UP_TRAFFIC["ratio"] is None:
+        return None
     return GATE_UP_TRAFFIC["ratio"] if gemm_sources_digest() == GATE_UP_TRAFFIC["sources_sha256"] else None
+
+
+def grouped_gemm_kernel_name(R, E, N, K, bf16_out, swiglu):
+    """The kernel nvfp4_grouped_gemm's automatic choice launches for this
+    problem (its rule, restated for the bench line's label only)."""
+    tag = "<swiglu>" if swiglu else ""
+    if R <= 16 * E:
+        return f"nvfp4::gemm::grouped_gemm_k512_kernel{tag} (deep ring)"
+    if N % 256 == 0 and bf16_out and K >= 1024:
+        return f"nvfp4::gemm::w2::grouped_gemm_w2_kernel{tag} (two weight blocks per tile)"
+    return f"nvfp4::gemm::grouped_gemm_k512_kernel{tag}" if K % 512 == 0 else f"nvfp4::gemm::grouped_gemm_kernel{tag}"
 FP4_PEAK = PEAKS.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]) * FP4_OVER_BF16
 
 
@@ -353,8 +365,8 @@ def run_headline(args, rank, world, device):
     q2_bytes = R * I * 2 + R * I * (0.5 + 1 / 16)
     q1_ms, q2_ms = float(np.mean(per[:, 0])), float(np.mean(per[:, 2]))
     traffic_ratio = gate_up_traffic_ratio()
-    roof = {"bound": "hbm", "kernel": ("nvfp4::gemm::grouped_gemm_k512_kernel<swiglu> (gate_up + SwiGLU epilogue launch)"
-                                       if fused else "nvfp4::gemm::grouped_gemm_k512_kernel (gate_up launch)"),
+    kname = grouped_gemm_kernel_name(R, E, 2 * I, H, fused or moe.mid_dtype == 1, fused)
+    roof = {"bound": "hbm", "kernel": kname + (": gate_up + SwiGLU epilogue launch" if fused else ": gate_up launch"),
             "achieved": round(gbs(g1_bytes, g1_ms), 1), "peak": HBM_PEAK, "unit": "GB/s",
             "frac": round(gbs(g1_bytes, g1_ms) / HBM_PEAK, 4),
             "traffic": (int(traffic_ratio * g1_bytes) if fused and traffic_ratio else None),
@@ -600,10 +612,43 @@ def comp_decode_w4a16(device, iters, warmup, flush):
     touched = int((np.diff(r["offsets"]) > 0).sum())
     wbytes = touched * (2 * I * H + H * I) * 0.5625
     gu_bytes = touched * 2 * I * H * 0.5625
+    del packs, ws, h, y
+    # Larger groups, where the automatic choice takes the tcgen05 kernel: the
+    # same gate_up shape for 64 experts, 2048 tokens top-8 (about 256 tokens
+    # per expert), timed on both kernels.
+    from nvfp4_w4a4_quantized_04_b200 import nvfp4_w4a16_select_kernel
+    nvtx = getattr(torch.cuda, "nvtx", None)
+    if nvtx is not None:
+        nvtx.range_push("w4a16_groups256")
+    E2, T2, k2 = 64, 2048, 8
+    r2 = synthetic.route_topk_softmax(5, T2, E2, k2)
+    R2 = len(r2["row_index"])
+    w2 = sc.gaussian_bf16(5, synthetic.STREAMS["w_gate_up"], (E2 * 2 * I, H), sigma=0.02)
+    offs2 = torch.arange(0, (E2 + 1) * 2 * I, 2 * I, dtype=torch.int32, device=device)
+    wp2 = L.quantize(w2, None, offs2, E2, 0)
+    wp2.offsets, wp2.num_groups, wp2.rows = None, 1, E2 * 2 * I
+    del w2
+    x2 = sc.gaussian_bf16(5, synthetic.STREAMS["x"], (T2, H))
+    ri2 = torch.from_numpy(r2["row_index"]).to(device)
+    off2 = torch.from_numpy(r2["offsets"]).to(device)
+    h2 = torch.empty((R2, I), dtype=torch.bfloat16, device=device)
+    ws2 = L.w4a16_workspace(R2, E2, H, device)
+    big = {}
+    for mode, name in ((2, "tcgen05"), (1, "warp_mma")):
+        nvfp4_w4a16_select_kernel(mode)
+        t = timed(lambda: L.grouped_gemm_w4a16(x2, wp2, 2 * I, ri2, off2, E2, rows=R2, out_dtype=1, swiglu=True,
+                                               y=h2, ws=ws2), iters, warmup, flush)
+        big[name + "_ms"] = round(t, 4)
+        big[name + "_tflops"] = round(2.0 * R2 * 2 * I * H / (t * 1e-3) / 1e12, 1)
+    nvfp4_w4a16_select_kernel(0)
+    if nvtx is not None:
+        nvtx.range_pop()
     return {"workload": "decode_w4a16_experts_e384_top10_zipf1.1_t64_h7168_i2048", "experts_touched": touched,
             "routed_rows": R, "layer_ms": round(ms, 4), "touched_weight_gbs": round(gbs(wbytes, ms), 1),
             "gate_up_swiglu_ms": round(t_gu, 4), "gate_up_gbs": round(gbs(gu_bytes, t_gu), 1),
-            "roofline": {"bound": "hbm", "frac": round(gbs(wbytes, ms) / HBM_PEAK, 4), "peak": HBM_PEAK}}
+            "kernel": "warp-MMA (automatic choice: at most 16 rows per expert)",
+            "roofline": {"bound": "hbm", "frac": round(gbs(wbytes, ms) / HBM_PEAK, 4), "peak": HBM_PEAK},
+            "groups256_gate_up": dict(workload="w4a16_gate_up_e64_top8_t2048_h7168_i2048", rows=R2, **big)}
 
 
 def comp_kv(device, iters, warmup, flush):

@@ -397,24 +397,31 @@ nvfp4_status nvfp4_grouped_gemm_w4a16(const void *x, int64_t ld_x, int64_t x_row
 /*
  * nvfp4_gemm_select_kernel -- which grouped GEMM kernel nvfp4_grouped_gemm runs
  * (process-wide; a tuning and testing switch, not part of the pages' method):
- *   0  automatic (default): one CTA per 128-row weight tile, with 512-element
- *      K stages when K % 512 == 0 and 256-element stages otherwise; the
- *      512-element kernel takes tiles of at most 64 tokens in a ring of three
- *      slots when the experts average at most 16 routed rows (M_total <=
- *      16 * num_experts), of at most 192 tokens in two slots otherwise;
+ *   0  automatic (default): when the experts average at most 16 routed rows
+ *      (M_total <= 16 * num_experts), one CTA per 128-row weight tile with
+ *      512-element K stages and tiles of at most 64 tokens in a ring of three
+ *      slots; otherwise, for a bf16 output with N % 256 == 0 and K >= 1024,
+ *      the kernel of mode 4; otherwise one CTA per 128-row weight tile with
+ *      512-element K stages (tiles of at most 192 tokens, two slots) when
+ *      K % 512 == 0 and 256-element stages when not;
  *   1  one CTA per tile, 256-element K stages;  2  CTA pairs (tcgen05
  *      cta_group::2, 256 weight rows per tile; N % 256 != 0 is then
  *      NVFP4_ERR_UNSUPPORTED_SHAPE);  3  the three-slot, 64-token ring
- *      whenever K % 512 == 0 (256-element stages otherwise).
- * Both give the same Y up to the fp32 accumulation order inside a tile.
+ *      whenever K % 512 == 0 (256-element stages otherwise);  4  two
+ *      128-row weight blocks per tile sharing one token tile, three
+ *      256-element K stages, whenever N % 256 == 0 and the output is bf16
+ *      (plain Y, SwiGLU h, or NVFP4 h from nvfp4_grouped_gemm_swiglu_nvfp4);
+ *      other calls run as in mode 0 (mxfp4_grouped_gemm always does).
+ *      The modes apply to nvfp4_grouped_gemm_swiglu_nvfp4 too.
+ * All give the same Y up to the fp32 accumulation order inside a tile.
  * Returns NVFP4_ERR_INVALID_ARG for another mode.
  */
 nvfp4_status nvfp4_gemm_select_kernel(int mode);
 
 /*
  * nvfp4_gemm_set_wait_budget -- a testing switch for the failure path of the
- * one-CTA grouped GEMM kernels (nvfp4_gemm_select_kernel modes 0 and 1, both
- * K-stage sizes; not part of the pages' method).  Every wait of the kernel's main loop on a ring,
+ * one-CTA grouped GEMM kernels (nvfp4_gemm_select_kernel modes 0, 1, 3 and
+ * 4; not part of the pages' method).  Every wait of the kernel's main loop on a ring,
  * scale or accumulator barrier gives up after this many SM clock cycles: it
  * raises the CTA's abort flag, writes NVFP4_ERR_TIMEOUT to dev_status, and
  * every role leaves its loop.  The closing waits for copies and MMAs still in

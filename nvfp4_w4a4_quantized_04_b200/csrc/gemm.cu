@@ -299,13 +299,33 @@ using namespace nvfp4;
 
 namespace {
 
-// 0 automatic (512-element stages when K % 512 == 0, with the deep ring when
-// the groups average at most 16 rows; else one CTA per tile with 256-element
-// stages), 1 one CTA per tile with 256-element stages, 2 CTA pairs, 3 the
-// deep 512-element ring whenever K % 512 == 0
+// 0 automatic (the deep 512-element ring when the groups average at most 16
+// rows; else two weight blocks per tile for bf16 outputs with N % 256 == 0 and
+// K >= 1024; else 512-element stages when K % 512 == 0; else one CTA per tile
+// with 256-element stages), 1 one CTA per tile with 256-element stages, 2 CTA
+// pairs, 3 the deep 512-element ring whenever K % 512 == 0, 4 two weight
+// blocks per tile whenever N % 256 == 0 and the output is bf16 (else as 0)
 std::atomic<int> g_gemm_kernel{0};
 
 }  // namespace
+
+// The deep ring (64-token tiles, three slots) in mode 3, and in mode 0 for
+// problems of few tokens per expert.
+bool deep_ring(int64_t M_total, int E) {
+  const int mode = g_gemm_kernel.load();
+  return mode == 3 || (mode == 0 && M_total <= gemm::kDeepRingMaxRowsPerExpert * (int64_t)E);
+}
+
+// The two-weight-block kernel (gemm_w2.cu) serves NVFP4 operands with a bf16
+// output (plain, SwiGLU h or NVFP4 h) and N % 256 == 0: always in mode 4, and
+// in mode 0 outside the deep ring's regime when K >= 1024 (its single
+// accumulator pair drains between tiles, which a K loop of at least four
+// stages hides behind the ring's loads).
+bool use_w2(int64_t M_total, int E, int64_t N, int64_t K, bool bf16_out) {
+  if (N % 256 != 0 || !bf16_out) return false;
+  const int mode = g_gemm_kernel.load();
+  return mode == 4 || (mode == 0 && K >= 1024 && !deep_ring(M_total, E));
+}
 
 // One CTA per SM, but no more CTAs than tiles can exist: each expert has at
 // most ceil(m_e / BN) <= m_e / BN + 1 token chunks per 128-row weight block.
@@ -313,13 +333,6 @@ int persistent_grid(int64_t M_total, int E, int64_t N) {
   const int64_t bound = (N / gemm::BM) * ((M_total + gemm::BN - 1) / gemm::BN + E);
   const int sms = host::sm_count();
   return (int)(bound < sms ? bound : sms);
-}
-
-// The deep ring (64-token tiles, three slots) in mode 3, and in mode 0 for
-// problems of few tokens per expert.
-bool deep_ring(int64_t M_total, int E) {
-  const int mode = g_gemm_kernel.load();
-  return mode == 3 || (mode == 0 && M_total <= gemm::kDeepRingMaxRowsPerExpert * (int64_t)E);
 }
 
 extern "C" nvfp4_status nvfp4_grouped_gemm(const uint8_t *a_q, const uint8_t *a_sf, const float *a_gs,
@@ -345,6 +358,9 @@ extern "C" nvfp4_status nvfp4_grouped_gemm(const uint8_t *a_q, const uint8_t *a_
   if ((reinterpret_cast<uintptr_t>(a_q) | reinterpret_cast<uintptr_t>(b_q) | reinterpret_cast<uintptr_t>(a_sf) |
        reinterpret_cast<uintptr_t>(b_sf) | reinterpret_cast<uintptr_t>(y)) & 15u)
     return NVFP4_ERR_INVALID_ARG;
+  if (use_w2(M_total, E, N, K, out_dtype == NVFP4_OUT_BF16))
+    return gemm::launch_grouped_gemm_w2(a_q, a_sf, a_gs, b_q, b_sf, b_gs, expert_offsets, E, M_total, N, K, y, swiglu,
+                                        amax_out, nullptr, dev_status, stream);
   if (g_gemm_kernel == 2)
     return gemm::launch_grouped_gemm_pair(a_q, a_sf, a_gs, b_q, b_sf, b_gs, expert_offsets, E, M_total, N, K, y,
                                           out_dtype, swiglu, amax_out, dev_status, stream);
@@ -371,11 +387,12 @@ extern "C" nvfp4_status nvfp4_gemm_set_wait_budget(int64_t cycles) {
   if (cycles < 0) return NVFP4_ERR_INVALID_ARG;
   const long long v = cycles == 0 ? gemm::kWaitBudgetCycles : (long long)cycles;
   if (cudaMemcpyToSymbol(gemm::c_wait_budget, &v, sizeof(v)) != cudaSuccess) return NVFP4_ERR_CUDA;
-  return gemm::set_wait_budget_k512(v);
+  if (gemm::set_wait_budget_k512(v) != NVFP4_OK) return NVFP4_ERR_CUDA;
+  return gemm::set_wait_budget_w2(v);
 }
 
 extern "C" nvfp4_status nvfp4_gemm_select_kernel(int mode) {
-  if (mode < 0 || mode > 3) return NVFP4_ERR_INVALID_ARG;
+  if (mode < 0 || mode > 4) return NVFP4_ERR_INVALID_ARG;
   g_gemm_kernel = mode;
   return NVFP4_OK;
 }
@@ -401,6 +418,9 @@ extern "C" nvfp4_status nvfp4_grouped_gemm_swiglu_nvfp4(const uint8_t *a_q, cons
   hq.gs = h_gs;
   hq.q = h_q;
   hq.sf = h_sf;
+  if (use_w2(M_total, E, N, K, true))
+    return gemm::launch_grouped_gemm_w2(a_q, a_sf, a_gs, b_q, b_sf, b_gs, expert_offsets, E, M_total, N, K, nullptr,
+                                        true, nullptr, &hq, dev_status, stream);
   if ((g_gemm_kernel == 0 || g_gemm_kernel == 3) && K % 512 == 0)
     return gemm::launch_grouped_gemm_k512(a_q, a_sf, a_gs, b_q, b_sf, b_gs, expert_offsets, E, M_total, N, K, nullptr,
                                           NVFP4_OUT_BF16, true, nullptr, &hq, false, deep_ring(M_total, E), dev_status, stream);

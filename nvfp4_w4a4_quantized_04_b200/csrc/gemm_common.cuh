@@ -385,24 +385,25 @@ __device__ __forceinline__ Tile decode_tile(int t, const int32_t *s_off, const i
 
 // Block-wide: s_off = expert offsets ({0, M_total} without offsets), s_slot =
 // 128-aligned slot starts, s_tile = first tile of each expert (n_mtiles weight
-// blocks x chunks per expert).  Every thread of the block calls it.
+// blocks x chunks per expert).  Every thread of the block (kThreadsT threads)
+// calls it; s_scratch holds 2 * kThreadsT / 32 ints.
 // Every tile's rows, and so every output row the epilogue stores, come from
 // the offsets: unless they start at 0, never decrease and end at M_total, the
 // call reports NVFP4_ERR_INDEX and leaves s_tile[E] = 0, so the kernel runs no
 // tile (no copy, no MMA, no store).
-template <int kCap = BN>
+template <int kCap = BN, int kThreadsT = NUM_THREADS>
 __device__ inline void build_tile_tables(const int32_t *__restrict__ expert_offsets, int E, int M_total,
                                          int n_mtiles, int32_t *s_off, int32_t *s_slot, int32_t *s_tile,
                                          int32_t *s_scratch, int32_t *dev_status) {
   if (expert_offsets) {
-    for (int i = threadIdx.x; i <= E; i += NUM_THREADS) s_off[i] = expert_offsets[i];
+    for (int i = threadIdx.x; i <= E; i += kThreadsT) s_off[i] = expert_offsets[i];
   } else if (threadIdx.x == 0) {
     s_off[0] = 0;
     s_off[1] = M_total;
   }
   __syncthreads();
   bool bad = false;
-  for (int i = threadIdx.x; i < E; i += NUM_THREADS) bad |= s_off[i + 1] < s_off[i];
+  for (int i = threadIdx.x; i < E; i += kThreadsT) bad |= s_off[i + 1] < s_off[i];
   if (threadIdx.x == 0) bad |= s_off[0] != 0 || s_off[E] != M_total;
   if (__syncthreads_or(bad)) {
     if (threadIdx.x == 0) {
@@ -412,8 +413,9 @@ __device__ inline void build_tile_tables(const int32_t *__restrict__ expert_offs
     __syncthreads();
     return;
   }
+  constexpr int kWarpsT = kThreadsT / 32;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int per = (E + NUM_THREADS - 1) / NUM_THREADS;
+  const int per = (E + kThreadsT - 1) / kThreadsT;
   const int e0 = min(E, (int)threadIdx.x * per), e1 = min(E, e0 + per);
   int32_t ls = 0, lt = 0;
   for (int e = e0; e < e1; ++e) {
@@ -427,18 +429,18 @@ __device__ inline void build_tile_tables(const int32_t *__restrict__ expert_offs
     const int32_t a = __shfl_up_sync(0xffffffffu, is, d), b = __shfl_up_sync(0xffffffffu, it, d);
     if (lane >= d) { is += a; it += b; }
   }
-  if (lane == 31) { s_scratch[warp] = is; s_scratch[NUM_WARPS + warp] = it; }
+  if (lane == 31) { s_scratch[warp] = is; s_scratch[kWarpsT + warp] = it; }
   __syncthreads();
   if (threadIdx.x == 0) {
     int32_t as = 0, at = 0;
-    for (int w = 0; w < NUM_WARPS; ++w) {
-      const int32_t vs = s_scratch[w], vt = s_scratch[NUM_WARPS + w];
-      s_scratch[w] = as; s_scratch[NUM_WARPS + w] = at;
+    for (int w = 0; w < kWarpsT; ++w) {
+      const int32_t vs = s_scratch[w], vt = s_scratch[kWarpsT + w];
+      s_scratch[w] = as; s_scratch[kWarpsT + w] = at;
       as += vs; at += vt;
     }
   }
   __syncthreads();
-  int32_t rs = s_scratch[warp] + is - ls, rt = s_scratch[NUM_WARPS + warp] + it - lt;
+  int32_t rs = s_scratch[warp] + is - ls, rt = s_scratch[kWarpsT + warp] + it - lt;
   for (int e = e0; e < e1; ++e) {
     const int32_t m = s_off[e + 1] - s_off[e];
     s_slot[e] = rs;
@@ -810,6 +812,14 @@ nvfp4_status launch_grouped_gemm_k512(const uint8_t *a_q, const uint8_t *a_sf, c
 constexpr int64_t kDeepRingMaxRowsPerExpert = 16;
 // Its copy of the main-loop wait budget (see c_wait_budget).
 nvfp4_status set_wait_budget_k512(long long cycles);
+
+// The two-weight-block kernel's launch (gemm_w2.cu): N % 256 == 0, bf16
+// output (SwiGLU h when swiglu, NVFP4 h when hq != nullptr), NVFP4 operands.
+nvfp4_status launch_grouped_gemm_w2(const uint8_t *a_q, const uint8_t *a_sf, const float *a_gs, const uint8_t *b_q,
+                                    const uint8_t *b_sf, const float *b_gs, const int32_t *expert_offsets, int E,
+                                    int64_t M_total, int64_t N, int64_t K, void *y, bool swiglu, float *amax_out,
+                                    const HQuantOut *hq, int32_t *dev_status, cudaStream_t stream);
+nvfp4_status set_wait_budget_w2(long long cycles);
 
 // The pair kernel's launch (gemm_pair.cu).  Requires N % 256 == 0.
 nvfp4_status launch_grouped_gemm_pair(const uint8_t *a_q, const uint8_t *a_sf, const float *a_gs,

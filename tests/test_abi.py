@@ -94,8 +94,8 @@ def test_host_validation_without_device(lib):
     assert L.mxfp4_to_nvfp4(fake, fake, 1, 100, 64, fake, fake, 1, fake, fake, None, None) == nv.ERR_UNSUPPORTED_SHAPE
     # swiglu
     assert L.nvfp4_swiglu_quantize(fake, 0, 4, 24, None, 1, fake, fake, fake, 0, fake, fake, None, None) == nv.ERR_UNSUPPORTED_SHAPE
-    # GEMM kernel switch: modes 0..3; CTA pairs cannot take N % 256 != 0
-    assert L.nvfp4_gemm_select_kernel(4) == nv.ERR_INVALID_ARG
+    # GEMM kernel switch: modes 0..4; CTA pairs cannot take N % 256 != 0
+    assert L.nvfp4_gemm_select_kernel(5) == nv.ERR_INVALID_ARG
     assert L.nvfp4_gemm_select_kernel(-1) == nv.ERR_INVALID_ARG
     assert L.nvfp4_gemm_select_kernel(2) == nv.OK
     assert L.nvfp4_grouped_gemm(fake, fake, fake, fake, fake, fake, None, 1, 128, 384, 512, fake, 0, 0, None, None, None, None) == nv.ERR_UNSUPPORTED_SHAPE

@@ -36,12 +36,14 @@ def status_word():
     return torch.zeros(1, dtype=torch.int32, device="cuda")
 
 
-@pytest.fixture(params=[0, 1, 2, 3], ids=["auto", "one_cta", "cta_pair", "deep_ring"])
+@pytest.fixture(params=[0, 1, 2, 3, 4], ids=["auto", "one_cta", "cta_pair", "deep_ring", "two_blocks"])
 def gemm_kernel(request):
-    """Run the test on each grouped GEMM kernel: automatic (512-element K
+    """Run the test on each grouped GEMM kernel: automatic (the two-block
+    kernel for bf16 outputs with N % 256 == 0 and K >= 1024, else 512-element K
     stages when K % 512 == 0), one CTA per tile with 256-element stages, the
-    CTA-pair kernel, and the 512-element kernel's deep ring (tiles of at most
-    64 tokens, three slots)."""
+    CTA-pair kernel, the 512-element kernel's deep ring (tiles of at most
+    64 tokens, three slots), and two weight blocks per tile (bf16 outputs with
+    N % 256 == 0; other calls of that mode run the automatic choice)."""
     nv = nvmod()
     nv.nvfp4_gemm_select_kernel(request.param)
     yield request.param
@@ -826,17 +828,19 @@ def test_gemm_dense_config1(out_dtype, gemm_kernel):
         assert np.array_equal(y, synthetic.f32_to_bf16_bits(y32))
 
 
-@pytest.mark.parametrize("mode", [0, 1, 3], ids=["k512", "k256", "k512_deep"])
+@pytest.mark.parametrize("mode", [0, 1, 3, 4], ids=["k512", "k256", "k512_deep", "two_blocks"])
 def test_gemm_wait_timeout_reports_and_recovers(mode):
     """The failure path of the one-CTA GEMM without any GPU fault: with a
     1-cycle budget on its main-loop waits, the first wait that is not already
     complete gives up, the kernel writes NVFP4_ERR_TIMEOUT to the status word
     and ends (its closing waits for copies and MMAs in flight keep the full
     budget).  With the budget restored, the same context runs the same GEMM
-    again and gets the result of a run made before the timeout, bit for bit."""
+    again and gets the result of a run made before the timeout, bit for bit.
+    The two-block kernel takes bf16 outputs only, so its case writes bf16."""
     L = layer()
     nv = nvmod()
     E, N, K = 6, 256, 1024
+    od = 1 if mode == 4 else 0
     counts = [0, 5, 130, 300, 16, 257]
     offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
     R = int(offsets[-1])
@@ -846,7 +850,7 @@ def test_gemm_wait_timeout_reports_and_recovers(mode):
     qw, sw, gw = _packed_weights(w, E, N, K)
     nv.nvfp4_gemm_select_kernel(mode)
     try:
-        y_before = _run_gemm(qs, ss, gs, qw, sw, gw, offsets, E, R, N, K, 0)
+        y_before = _run_gemm(qs, ss, gs, qw, sw, gw, offsets, E, R, N, K, od)
         bound = nv.nvfp4_padded_rows_bound(R, E)
         qa = np.zeros((bound, K // 2), np.uint8)
         qa[:qs.shape[0]] = qs
@@ -856,11 +860,11 @@ def test_gemm_wait_timeout_reports_and_recovers(mode):
         wp = L.Packed(to_dev(qw), to_dev(tile(sw)), to_dev(gw), qw.shape[0], K, 1)
         nv.nvfp4_gemm_set_wait_budget(1)
         s = status_word()
-        L.grouped_gemm(a, wp, N, 0, dev_status=s)
+        L.grouped_gemm(a, wp, N, od, dev_status=s)
         torch.cuda.synchronize()
         assert int(s.item()) == nv.ERR_TIMEOUT
         nv.nvfp4_gemm_set_wait_budget(0)
-        y_after = _run_gemm(qs, ss, gs, qw, sw, gw, offsets, E, R, N, K, 0)
+        y_after = _run_gemm(qs, ss, gs, qw, sw, gw, offsets, E, R, N, K, od)
     finally:
         nv.nvfp4_gemm_set_wait_budget(0)
         nv.nvfp4_gemm_select_kernel(0)
@@ -872,7 +876,8 @@ def test_gemm_rejects_bad_offsets(gemm_kernel, bad):
     """Expert offsets that do not start at 0, decrease, or end elsewhere than
     at M_total: every CTA reports NVFP4_ERR_INDEX and runs no tile, so y keeps
     its sentinel.  The buffers are sized so that even a kernel that trusted
-    the offsets would stay inside them (the slots of the largest offsets fit)."""
+    the offsets would stay inside them (the slots of the largest offsets fit).
+    fp32 and bf16 outputs (the two-block kernel writes bf16 only)."""
     L = layer()
     nv = nvmod()
     E, N, K, M = 3, 256, 1024, 300
@@ -888,12 +893,13 @@ def test_gemm_rejects_bad_offsets(gemm_kernel, bad):
     one = np.ones(E, np.float32)
     a = L.Packed(to_dev(qa), to_dev(tile(sa)), to_dev(one), M, K, 1, to_dev(offsets), E)
     w = L.Packed(to_dev(qw), to_dev(tile(sw)), to_dev(one), E * N, K, 1)
-    y = torch.full((rows_alloc, N), 12345.0, dtype=torch.float32, device="cuda")
-    s = status_word()
-    L.grouped_gemm(a, w, N, 0, y=y[:M], dev_status=s)
-    torch.cuda.synchronize()
-    assert int(s.item()) == nv.ERR_INDEX
-    assert (to_np(y) == np.float32(12345.0)).all()
+    for od, dt in ((0, torch.float32), (1, torch.bfloat16)):
+        y = torch.full((rows_alloc, N), 12345.0, dtype=dt, device="cuda")
+        s = status_word()
+        L.grouped_gemm(a, w, N, od, y=y[:M], dev_status=s)
+        torch.cuda.synchronize()
+        assert int(s.item()) == nv.ERR_INDEX
+        assert (y == 12345.0).all().item()
 
 
 def test_quantize_rejects_bad_group_offsets():
@@ -1084,6 +1090,38 @@ def test_gemm_long_k_tolerance(gemm_kernel):
     assert ok.all(), (err.max(), (err / bound).max())
 
 
+def test_gemm_two_blocks_long_k_bf16():
+    """The two-weight-block kernel on ragged groups with K = 4096 (16 turns of
+    its three-slot ring per tile) and 4 weight-block pairs per expert: bf16 Y
+    within the GEMM bound plus bf16 rounding of the oracle, and bit for bit the
+    bf16 Y of the one-CTA kernel with 256-element stages (same MMAs in the same
+    K order)."""
+    nv = nvmod()
+    E, N, K = 5, 1024, 4096
+    counts = [1, 70, 0, 200, 385]
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    R = int(offsets[-1])
+    x = synthetic.gaussian_bf16(31, synthetic.STREAMS["x"], (R, K), outlier_frac=0.001)
+    w = synthetic.gaussian_bf16(31, synthetic.STREAMS["w"], (E * N, K), sigma=0.02)
+    q, sf, gs, qs, ss = _packed_acts(x, None, offsets, E)
+    qw, sw, gw = _packed_weights(w, E, N, K)
+    try:
+        nv.nvfp4_gemm_select_kernel(4)
+        y16 = _run_gemm(qs, ss, gs, qw, sw, gw, offsets, E, R, N, K, 1)
+        nv.nvfp4_gemm_select_kernel(1)
+        y16_k256 = _run_gemm(qs, ss, gs, qw, sw, gw, offsets, E, R, N, K, 1)
+    finally:
+        nv.nvfp4_gemm_select_kernel(0)
+    assert np.array_equal(y16, y16_k256)
+    a = oracle.dequantize_f64(q, sf, oracle.rows_global_scale(gs, offsets, R))
+    bw = oracle.dequantize_f64(qw, sw, np.repeat(gw, N))
+    y_ref, s_ref = oracle.grouped_gemm_f64(a, bw.reshape(E, N, K), offsets)
+    y = synthetic.bf16_bits_to_f32(y16).astype(np.float64)
+    err = np.abs(y - y_ref)
+    bound = (1e-5 * s_ref + 1e-6) * (1 + 2.0 ** -8) + 2.0 ** -8 * np.abs(y_ref)
+    assert (err <= bound).all(), (err.max(), (err / bound).max())
+
+
 # --------------------------------------------------------------------------- fused SwiGLU epilogue
 def test_gemm_swiglu_epilogue(gemm_kernel):
     """h = bf16(silu(g)*u) from the gate_up accumulators: compared with the
@@ -1121,7 +1159,7 @@ def test_gemm_swiglu_epilogue(gemm_kernel):
     assert np.array_equal(to_np(amax), want)
 
 
-def test_gemm_swiglu_nvfp4_epilogue():
+def test_gemm_swiglu_nvfp4_epilogue(gemm_kernel):
     """The epilogue that quantizes h with a given global per expert writes the
     bytes the oracle's GIVEN-mode quantize writes for the device's bf16 h
     (taken from the SwiGLU epilogue of the same GEMM); padding rows untouched.
