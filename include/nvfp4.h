@@ -129,6 +129,12 @@ int64_t nvfp4_padded_rows_bound(int64_t rows, int num_groups);
  *   workspace   >= nvfp4_workspace_size(num_groups) bytes.
  *   dev_status  nullable int32: NVFP4_ERR_NONFINITE when an input element of a
  *               group is NaN/inf (that group's outputs are unspecified).
+ * Launches: FROM_AMAX without row_index and group_offsets runs as one
+ * cooperative launch (amax, global scale, encode; its CTAs wait for each other
+ * with a bounded wait, NVFP4_ERR_TIMEOUT if it ever ran out), after clearing
+ * two words of the workspace; if the runtime refuses a cooperative launch, or
+ * rows * K/16 >= 2^32 - 64, the separate passes run instead.  Other calls run
+ * an amax pass (FROM_AMAX), a scale finalisation and the encode.
  * Arithmetic (each step one IEEE fp32 round-to-nearest-even operation):
  *   block amax a_b; S = e4m3_rne_satfinite(a_b / (6*s_g));
  *   r = 1/(S*s_g) (0 when S*s_g == 0); code_i = e2m1_rne_satfinite(x_i * r).

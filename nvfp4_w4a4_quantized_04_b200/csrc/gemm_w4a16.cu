@@ -79,7 +79,7 @@ constexpr int kConverters = 8;               // warps 6.., kConverters / 4 per T
 constexpr int kConvSplit = kConverters / 4;  // K pieces of a stage per weight row
 constexpr int kConvCodes = 256 / kConvSplit; // codes per converter thread per stage
 static_assert(kConverters % 4 == 0 && kConvCodes % 64 == 0, "whole 32-column stores per converter");
-constexpr int W_PRODUCER = 0, W_MMA = 1, W_EPI0 = 2, W_CONV0 = 6;
+constexpr int W_PRODUCER = 0, W_MMA = 1, W_CONV0 = 6;   // warps 2..5: epilogue
 constexpr int kWarps = W_CONV0 + kConverters;
 constexpr int kThreads = kWarps * 32;
 constexpr int OFF_BAR = kStages * kStageBytes;
@@ -144,7 +144,6 @@ __global__ void __launch_bounds__(256) w4a16_prep_kernel(
   block_prefix(E, gslot, scratch, [&](int e) { return (off[e + 1] - off[e] + kGrp - 1) / kGrp; });
   const int64_t Gt = gslot[E];
   const int lane = threadIdx.x & 31;
-  const int nst = K / 256;
   const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
   bool bad_index = false, bad_value = false;
   for (int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < M_total; r += nwarps) {

@@ -344,25 +344,100 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(
   if (bad) report(dev_status, NVFP4_ERR_NONFINITE);
 }
 
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t *p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// One-launch dynamic quantize of a whole ungrouped tensor (FROM_AMAX, no row
+// index), the first phase of quantize_kernel<kTiled, true>: every CTA reduces
+// its grid-stride share of max|x| into words[0] (atomicMax on the fp32 bit
+// pattern, as the amax pass does), counts itself in words[1], and waits until
+// all gridDim.x CTAs have (the launch is cooperative, so every CTA is
+// resident; the wait is bounded and reports NVFP4_ERR_TIMEOUT, after which the
+// CTA writes nothing).  Then each CTA derives s_g from the amax with the
+// finalisation's arithmetic; CTA 0 stores it to gs[0].  words[0..1] are zero
+// at launch (the host clears them).  Returns false when the CTA must stop.
+__device__ __forceinline__ bool fused_global_scale(const uint16_t *__restrict__ x, int64_t ld_x, uint32_t nblk,
+                                                   uint32_t total, const FastDiv &fd, uint32_t *words,
+                                                   float *gs, float &s_g, int32_t *dev_status) {
+  __shared__ uint32_t red[8];
+  __shared__ int s_ok;
+  const bool v8 = ((reinterpret_cast<uintptr_t>(x) & 31u) == 0) && ((ld_x & 15) == 0);
+  // 64-bit indices: total is below 2^32, but b + 4 * nthr need not be
+  const uint64_t nthr = (uint64_t)gridDim.x * blockDim.x;
+  uint64_t b = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  uint32_t m = 0;
+  for (; b + 3 * nthr < total; b += 4 * nthr) {
+    uint4 a[4], c[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint32_t bb = (uint32_t)(b + k * nthr), r = fast_div(bb, fd);
+      load_block(x + (int64_t)r * ld_x + (uint64_t)(bb - r * nblk) * 16, v8, a[k], c[k]);
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) m = absmax8_bits(c[k], absmax8_bits(a[k], m));
+  }
+  for (; b < total; b += nthr) {
+    uint4 a, c;
+    const uint32_t bb = (uint32_t)b, r = fast_div(bb, fd);
+    load_block(x + (int64_t)r * ld_x + (uint64_t)(bb - r * nblk) * 16, v8, a, c);
+    m = absmax8_bits(c, absmax8_bits(a, m));
+  }
+  m = warp_max(halves_max(m));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t bm = 0;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) bm = max(bm, red[w]);
+    if (bm) atomicMax(&words[0], bm << 16);
+    __threadfence();
+    atomicAdd(&words[1], 1u);
+    int ok = 1;
+    const long long t0 = clock64();
+    while (ld_acquire_u32(&words[1]) < gridDim.x) {
+      if (clock64() - t0 > 4000000000LL) {                   // about 2 s
+        ok = 0;
+        report(dev_status, NVFP4_ERR_TIMEOUT);
+        break;
+      }
+    }
+    s_ok = ok;
+  }
+  __syncthreads();
+  if (!s_ok) return false;
+  const uint32_t amax_bits = ld_acquire_u32(&words[0]);
+  s_g = gs_from_amax_bits(amax_bits, blockIdx.x == 0 ? dev_status : nullptr);
+  if (blockIdx.x == 0 && threadIdx.x == 0) gs[0] = s_g;
+  return true;
+}
+
 // General form: one thread per 16-element block of the real rows (routed
 // order), 64-block chunks, each warp a contiguous run of chunks so every
 // lane's row (and the row's group) only moves forward.  The block -> (row,
 // block) split is a multiply-high division; only real rows are written.
-template <bool kTiled>
+// kFused: an ungrouped tensor whose global scale comes from its amax, in one
+// cooperative launch (fused_global_scale first, then the encode).
+template <bool kTiled, bool kFused = false>
 __global__ void __launch_bounds__(256) quantize_kernel(
     const uint16_t *__restrict__ x, int64_t ld_x, int64_t K64, int64_t rows,
     const int32_t *__restrict__ row_index, const int32_t *__restrict__ group_offsets, int G,
-    const float *__restrict__ gs, uint8_t *__restrict__ q, uint8_t *__restrict__ sf, FastDiv fd,
+    float *gs, uint8_t *__restrict__ q, uint8_t *__restrict__ sf, FastDiv fd, uint32_t *fuse_words,
     int32_t *dev_status) {
   extern __shared__ int32_t smem[];
   int32_t *off = smem, *slot = smem + (G + 1), *scratch = smem + 2 * (G + 1);
-  if (group_offsets && !load_groups(group_offsets, G, off, slot, scratch, rows, true)) {
+  if (!kFused && group_offsets && !load_groups(group_offsets, G, off, slot, scratch, rows, true)) {
     if (threadIdx.x == 0) report(dev_status, NVFP4_ERR_INDEX);
     return;
   }
   const int lane = threadIdx.x & 31;
   const uint32_t K = (uint32_t)K64, nblk = K >> 4;
   const uint32_t total = (uint32_t)rows * nblk;              // < 2^32 (host check)
+  float fused_sg = 0.0f;
+  if constexpr (kFused) {
+    if (!fused_global_scale(x, ld_x, nblk, total, fd, fuse_words, gs, fused_sg, dev_status)) return;
+  }
   constexpr int U = 2;                                       // 32-block steps per chunk
   const uint32_t nchunks = (total + 32 * U - 1) / (32 * U);
   const uint32_t warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -392,7 +467,7 @@ __global__ void __launch_bounds__(256) quantize_kernel(
   uint32_t cached_r = 0xFFFFFFFFu, p = 0;
   int64_t src = 0;
   uint64_t rsf = 0;
-  float s_g = gs[g], t_g = __fmul_rn(6.0f, s_g);
+  float s_g = kFused ? fused_sg : gs[g], t_g = __fmul_rn(6.0f, s_g);
   bool bad = false;
   for (uint32_t ci = c_begin; ci < c_end; ci += c_step) {
     // Ungrouped tensors are walked from the end: the amax pass just streamed
@@ -1011,13 +1086,55 @@ nvfp4_status run_encode(const uint16_t *x, int64_t rows, int64_t K, int64_t ld_x
     const int64_t work = (n * nblk + 1) / 2;
     if (tiled) {
       const unsigned grid = (unsigned)grid_resident(quantize_kernel<true>, work, 256, sm);
-      quantize_kernel<true><<<grid, 256, sm, stream>>>(xp, ld_x, K, n, row_index, group_offsets, G, gs, qp, sp, fd, dev_status);
+      quantize_kernel<true><<<grid, 256, sm, stream>>>(xp, ld_x, K, n, row_index, group_offsets, G, const_cast<float *>(gs), qp, sp, fd, nullptr, dev_status);
     } else {
       const unsigned grid = (unsigned)grid_resident(quantize_kernel<false>, work, 256, sm);
-      quantize_kernel<false><<<grid, 256, sm, stream>>>(xp, ld_x, K, n, row_index, group_offsets, G, gs, qp, sp, fd, dev_status);
+      quantize_kernel<false><<<grid, 256, sm, stream>>>(xp, ld_x, K, n, row_index, group_offsets, G, const_cast<float *>(gs), qp, sp, fd, nullptr, dev_status);
     }
     if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_CUDA;
   }
+  return NVFP4_OK;
+}
+
+// The dynamic quantize of an ungrouped tensor in one cooperative launch
+// (quantize_kernel<tiled, true>): the amax pass, the global scale and the
+// encode without the two extra launches and their gaps.  The grid is at most
+// one resident wave, so every CTA can wait for the others.  *launched is false
+// (and nothing was enqueued but the clearing of the two workspace words) when
+// the runtime refuses the cooperative launch; the caller then runs the
+// separate passes.
+nvfp4_status run_fused_dense(const uint16_t *x, int64_t rows, int64_t K, int64_t ld_x, float *global_scale,
+                             uint8_t *q, uint8_t *sf, nvfp4_sf_layout layout, void *workspace,
+                             int32_t *dev_status, cudaStream_t stream, bool *launched) {
+  *launched = false;
+  const bool tiled = layout == NVFP4_SF_MMA_TILED;
+  const int64_t nblk = K / 16, total = rows * nblk;
+  uint32_t *words = reinterpret_cast<uint32_t *>(workspace);
+  if (cudaMemsetAsync(words, 0, 2 * sizeof(uint32_t), stream) != cudaSuccess) return NVFP4_ERR_CUDA;
+  auto kern = tiled ? quantize_kernel<true, true> : quantize_kernel<false, true>;
+  const int per_sm = host::blocks_per_sm(reinterpret_cast<const void *>(kern), 256, 0);
+  const int64_t nchunks = (total + 63) / 64;
+  int64_t grid = (int64_t)per_sm * num_sms();
+  if ((nchunks + 7) / 8 < grid) grid = (nchunks + 7) / 8;    // at least one 64-block chunk per warp
+  if (grid < 1) grid = 1;
+  const FastDiv fd = make_fastdiv((uint32_t)nblk);
+  const uint16_t *a_x = x;
+  int64_t a_ld = ld_x, a_k = K, a_rows = rows;
+  const int32_t *a_ri = nullptr, *a_go = nullptr;
+  int a_g = 1;
+  float *a_gs = global_scale;
+  uint8_t *a_q = q, *a_sf = sf;
+  FastDiv a_fd = fd;
+  uint32_t *a_w = words;
+  int32_t *a_st = dev_status;
+  void *args[] = {&a_x, &a_ld, &a_k, &a_rows, &a_ri, &a_go, &a_g, &a_gs, &a_q, &a_sf, &a_fd, &a_w, &a_st};
+  const cudaError_t e = cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(kern), dim3((unsigned)grid),
+                                                    dim3(256), args, 0, stream);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    return NVFP4_OK;
+  }
+  *launched = true;
   return NVFP4_OK;
 }
 
@@ -1068,6 +1185,13 @@ nvfp4_status nvfp4_quantize(const void *x, int64_t rows, int64_t K, int64_t ld_x
   if (rows > 0 && (!x || !q || !sf || !aligned16(x) || !aligned16(q))) return NVFP4_ERR_INVALID_ARG;
   if (rows > ((int64_t)1 << 31)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   const uint16_t *xb = reinterpret_cast<const uint16_t *>(x);
+  if (gs_mode == NVFP4_GS_FROM_AMAX && !group_offsets && !row_index && rows > 0 &&
+      rows * (K / 16) <= (int64_t)0xFFFFFFC0ll) {
+    bool launched = false;
+    const nvfp4_status fs = run_fused_dense(xb, rows, K, ld_x, global_scale, q, sf, sf_layout, workspace,
+                                            dev_status, stream, &launched);
+    if (fs != NVFP4_OK || launched) return fs;
+  }
   nvfp4_status st = run_global_scales(xb, rows, K, ld_x, row_index, group_offsets, G, gs_mode,
                                       global_scale, workspace, dev_status, stream);
   if (st != NVFP4_OK) return st;

@@ -85,6 +85,32 @@ def test_quantize_dense_config1_bitexact(layout):
 
 
 @pytest.mark.parametrize("layout", [0, 1])
+def test_quantize_dense_strided_rows_one_launch(layout):
+    """The ungrouped dynamic quantize runs as one cooperative launch (amax,
+    global scale and encode with a grid-wide wait in between).  Rows with
+    ld_x = K + 64 and a tensor of 524,288 blocks, so every CTA of the resident
+    wave takes part in the wait and warps encode several chunks each: byte-exact
+    to the oracle, the global scale included; the status word stays 0."""
+    L = layer()
+    rows, K, pad = 8192, 1024, 64
+    xw = synthetic.gaussian_bf16(41, synthetic.STREAMS["x"], (rows, K + pad), outlier_frac=0.001)
+    x = np.ascontiguousarray(xw[:, :K])
+    q_ref, sf_ref, gs_ref, st = oracle.quantize(x)
+    assert st == 0
+    xd = bf16_dev(xw)[:, :K]
+    assert xd.stride(0) == K + pad
+    s = status_word()
+    p = L.quantize(xd, layout=layout, dev_status=s)
+    torch.cuda.synchronize()
+    assert int(s.item()) == 0
+    assert to_np(p.gs)[0] == gs_ref[0]
+    assert np.array_equal(to_np(p.q)[:rows], q_ref)
+    sf = to_np(p.sf)
+    sf = untile(sf, rows, K // 16) if layout == 1 else sf.reshape(-1, K // 16)[:rows]
+    assert np.array_equal(sf, sf_ref)
+
+
+@pytest.mark.parametrize("layout", [0, 1])
 def test_quantize_dense_16byte_aligned_input(layout):
     """A dense input that is 16-byte but not 32-byte aligned takes the 16-byte
     load forms of the amax pass and the encode; many chunks per warp and a
