@@ -22,7 +22,8 @@
 namespace nvfp4 {
 
 // ws[2t] = max(u+1), ws[2t+1] = max(256-u) over non-zero blocks of tensor t
-// (0 = no such block), via atomicMax on zero-initialised words.  A CTA takes
+// (0 = no such block), via atomicMax on zero-initialised words; or one such
+// pair per CTA of the tensor (partials), reduced by the scale pass.  A CTA takes
 // kScanChunk consecutive blocks of one tensor, eight per thread (128 bytes of
 // codes in flight per thread); CTAs are short and not persistent.
 constexpr int kScanUnroll = 8;
@@ -30,7 +31,7 @@ constexpr int64_t kScanChunk = 256 * kScanUnroll;
 
 __global__ void __launch_bounds__(256) remap_scan_kernel(
     const uint8_t *__restrict__ q_mx, const uint8_t *__restrict__ e8, int64_t blocks_per_tensor,
-    uint8_t *__restrict__ q_nv, uint32_t *__restrict__ ws, int32_t *dev_status) {
+    uint8_t *__restrict__ q_nv, uint32_t *__restrict__ ws, bool partials, int32_t *dev_status) {
   const int64_t t = blockIdx.y;
   const int64_t b0 = (int64_t)blockIdx.x * kScanChunk;
   const int64_t b1 = min(blocks_per_tensor, b0 + kScanChunk);
@@ -88,7 +89,13 @@ __global__ void __launch_bounds__(256) remap_scan_kernel(
       hi = max(hi, red[0][w]);
       lo = max(lo, red[1][w]);
     }
-    if (hi) {
+    if (partials) {
+      // this CTA's own pair of words: every pair is written, so nothing needs
+      // clearing first, and the scale pass reduces a tensor's pairs
+      const int64_t slot = t * gridDim.x + blockIdx.x;
+      ws[2 * slot] = hi;
+      ws[2 * slot + 1] = lo;
+    } else if (hi) {
       atomicMax(&ws[2 * t], hi);
       atomicMax(&ws[2 * t + 1], lo);
     }
@@ -111,16 +118,27 @@ __device__ __forceinline__ uint32_t e4m3_pow2(int p) {
 // first unit also writes s_g and checks the exponent spread.
 constexpr int64_t kAtomRun = 16;
 
-__device__ __forceinline__ int remap_global_exp(const uint32_t *__restrict__ ws, int64_t t, uint32_t &hi,
+// The tensor's exponent words: one pair (npart == 0), or the max over its
+// npart per-CTA pairs.
+__device__ __forceinline__ int remap_global_exp(const uint32_t *__restrict__ ws, int64_t t, int npart, uint32_t &hi,
                                                 uint32_t &lo) {
-  hi = ws[2 * t];
-  lo = ws[2 * t + 1];
+  if (npart == 0) {
+    hi = ws[2 * t];
+    lo = ws[2 * t + 1];
+  } else {
+    hi = 0;
+    lo = 0;
+    for (int i = 0; i < npart; ++i) {
+      hi = max(hi, ws[2 * (t * npart + i)]);
+      lo = max(lo, ws[2 * (t * npart + i) + 1]);
+    }
+  }
   return hi ? (int)hi - 1 - 127 - 8 : 0;
 }
 
 __global__ void __launch_bounds__(256) remap_scale_atoms_kernel(
     const uint8_t *__restrict__ e8, int64_t rows, int64_t K, int64_t n_tensors,
-    const uint32_t *__restrict__ ws, uint8_t *__restrict__ sf, float *__restrict__ gs, bool vec,
+    const uint32_t *__restrict__ ws, int npart, uint8_t *__restrict__ sf, float *__restrict__ gs, bool vec,
     int32_t *dev_status) {
   const int lane = threadIdx.x & 31;
   const int64_t rb_per_t = rows >> 7, kg_per_row = K >> 6, nb32 = K >> 5;
@@ -133,7 +151,7 @@ __global__ void __launch_bounds__(256) remap_scale_atoms_kernel(
     const int64_t rb = w / runs_per_rb, kg0 = (w - rb * runs_per_rb) * kAtomRun;
     const int64_t kg1 = min(kg_per_row, kg0 + kAtomRun);
     uint32_t hi, lo;
-    const int g = remap_global_exp(ws, t, hi, lo);
+    const int g = remap_global_exp(ws, t, npart, hi, lo);
     if (w == 0 && lane == 0) {
       gs[t] = ldexpf(1.0f, g);   // 2^g exactly, g in [-135, 119] (subnormal below -126)
       if (hi && (256 - (int)lo - 127) - g < -9) report(dev_status, NVFP4_ERR_NOT_REPRESENTABLE);
@@ -185,13 +203,13 @@ __global__ void __launch_bounds__(256) remap_scale_atoms_kernel(
 // 2i+1, written as one 2-byte store.
 __global__ void __launch_bounds__(256) remap_scale_rows_kernel(
     const uint8_t *__restrict__ e8, int64_t per_tensor, int64_t n_tensors, const uint32_t *__restrict__ ws,
-    uint8_t *__restrict__ sf, float *__restrict__ gs, int32_t *dev_status) {
+    int npart, uint8_t *__restrict__ sf, float *__restrict__ gs, int32_t *dev_status) {
   const uint64_t total = (uint64_t)n_tensors * (uint64_t)per_tensor;
   const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
   for (uint64_t i = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += stride) {
     const uint64_t t = i / (uint64_t)per_tensor, within = i - t * (uint64_t)per_tensor;
     uint32_t hi, lo;
-    const int g = remap_global_exp(ws, (int64_t)t, hi, lo);
+    const int g = remap_global_exp(ws, (int64_t)t, npart, hi, lo);
     if (within == 0) {
       gs[t] = ldexpf(1.0f, g);   // 2^g exactly, g in [-135, 119] (subnormal below -126)
       if (hi && (256 - (int)lo - 127) - g < -9) report(dev_status, NVFP4_ERR_NOT_REPRESENTABLE);
@@ -220,13 +238,20 @@ extern "C" nvfp4_status mxfp4_to_nvfp4(const uint8_t *q_mx, const uint8_t *ue8m0
        reinterpret_cast<uintptr_t>(workspace)) & 15u) return NVFP4_ERR_INVALID_ARG;
   if (sf_layout == NVFP4_SF_ROWMAJOR && (reinterpret_cast<uintptr_t>(sf_nv) & 1u)) return NVFP4_ERR_INVALID_ARG;
   uint32_t *ws = reinterpret_cast<uint32_t *>(workspace);
-  if (cudaMemsetAsync(ws, 0, sizeof(uint32_t) * 2 * n_tensors, stream) != cudaSuccess) return NVFP4_ERR_CUDA;
   const int64_t bpt = rows * (K / 32);
   const int64_t xblocks = (bpt + kScanChunk - 1) / kScanChunk;
   if (xblocks > 0x7FFFFFFF) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   dim3 grid1((unsigned)xblocks, (unsigned)n_tensors);
   if (grid1.y > 65535) return NVFP4_ERR_UNSUPPORTED_SHAPE;
-  remap_scan_kernel<<<grid1, 256, 0, stream>>>(q_mx, ue8m0, bpt, q_nv, ws, dev_status);
+  // Up to kMaxPartials scan CTAs per tensor: each writes its own pair of
+  // words (8 bytes per CTA, within nvfp4_workspace_size(n_tensors)) and the
+  // scale pass reduces them, so no clearing launch is needed.  More CTAs per
+  // tensor: atomics on one zero-initialised pair per tensor.
+  constexpr int64_t kMaxPartials = 64;
+  const int npart = xblocks <= kMaxPartials ? (int)xblocks : 0;
+  if (npart == 0 && cudaMemsetAsync(ws, 0, sizeof(uint32_t) * 2 * n_tensors, stream) != cudaSuccess)
+    return NVFP4_ERR_CUDA;
+  remap_scan_kernel<<<grid1, 256, 0, stream>>>(q_mx, ue8m0, bpt, q_nv, ws, npart != 0, dev_status);
   if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_CUDA;
   const int sms = host::sm_count();
   if (sf_layout == NVFP4_SF_MMA_TILED) {
@@ -235,14 +260,14 @@ extern "C" nvfp4_status mxfp4_to_nvfp4(const uint8_t *q_mx, const uint8_t *ue8m0
     if (blocks > (int64_t)sms * 8) blocks = (int64_t)sms * 8;
     // 16-byte exponent loads need 16-byte aligned rows of exponents
     const bool vec = (reinterpret_cast<uintptr_t>(ue8m0) & 15u) == 0 && (K / 32) % 16 == 0;
-    remap_scale_atoms_kernel<<<(unsigned)blocks, 256, 0, stream>>>(ue8m0, rows, K, n_tensors, ws, sf_nv, global_scale,
-                                                                   vec, dev_status);
+    remap_scale_atoms_kernel<<<(unsigned)blocks, 256, 0, stream>>>(ue8m0, rows, K, n_tensors, ws, npart, sf_nv,
+                                                                   global_scale, vec, dev_status);
   } else {
     const int64_t total = n_tensors * bpt;
     int64_t blocks = (total + 255) / 256;
     if (blocks > (int64_t)sms * 8) blocks = (int64_t)sms * 8;
-    remap_scale_rows_kernel<<<(unsigned)blocks, 256, 0, stream>>>(ue8m0, bpt, n_tensors, ws, sf_nv, global_scale,
-                                                                   dev_status);
+    remap_scale_rows_kernel<<<(unsigned)blocks, 256, 0, stream>>>(ue8m0, bpt, n_tensors, ws, npart, sf_nv,
+                                                                   global_scale, dev_status);
   }
   return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
