@@ -728,9 +728,13 @@ def comp_gemm_small(device, iters, warmup, flush):
         L.quantize(x, layout=1, out=a, ws=ws)
         L.grouped_gemm(a, w, N, 0, y=y)
     t_b = timed(both, iters, warmup, flush)
+    # the floor of this measurement: a one-element fill timed the same way
+    z = torch.empty(1, dtype=torch.float32, device=device)
+    t_0 = timed(lambda: z.fill_(1.0), iters, warmup, flush)
     flop = 2.0 * M * N * K
     return {"workload": "gemm_m128_n256_k512_fp32_out", "quantize_us": round(t_q * 1e3, 2),
             "gemm_us": round(t_g * 1e3, 2), "quantize_and_gemm_us": round(t_b * 1e3, 2),
+            "one_element_fill_us": round(t_0 * 1e3, 2),
             "gemm_tflops": round(flop / (t_g * 1e-3) / 1e12, 3), "bound": "launch latency"}
 
 
