@@ -1116,6 +1116,31 @@ def test_gemm_long_k_tolerance(gemm_kernel):
     assert ok.all(), (err.max(), (err / bound).max())
 
 
+def test_gemm_two_blocks_max_experts():
+    """The two-block kernel at the 1024-expert limit of the GEMM tile tables:
+    mostly empty groups, a few of 1-3 rows and one of 200 (two token chunks);
+    bf16 Y bit for bit that of the one-CTA kernel with 256-element stages."""
+    nv = nvmod()
+    rng = np.random.default_rng(29)
+    E, N, K = 1024, 256, 1024
+    counts = np.where(rng.random(E) < 0.8, 0, rng.integers(1, 4, E))
+    counts[700] = 200
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    R = int(offsets[-1])
+    x = synthetic.gaussian_bf16(29, synthetic.STREAMS["x"], (R, K))
+    w = synthetic.gaussian_bf16(29, synthetic.STREAMS["w"], (E * N, K), sigma=0.02)
+    q, sf, gs, qs, ss = _packed_acts(x, None, offsets, E)
+    qw, sw, gw = _packed_weights(w, E, N, K)
+    try:
+        nv.nvfp4_gemm_select_kernel(4)
+        y4 = _run_gemm(qs, ss, gs, qw, sw, gw, offsets, E, R, N, K, 1)
+        nv.nvfp4_gemm_select_kernel(1)
+        y1 = _run_gemm(qs, ss, gs, qw, sw, gw, offsets, E, R, N, K, 1)
+    finally:
+        nv.nvfp4_gemm_select_kernel(0)
+    assert np.array_equal(y4, y1)
+
+
 def test_gemm_two_blocks_long_k_bf16():
     """The two-weight-block kernel on ragged groups with K = 4096 (16 turns of
     its three-slot ring per tile) and 4 weight-block pairs per expert: bf16 Y
