@@ -14,14 +14,16 @@
 // two MMAs, one per block, into two accumulators that read the same token
 // operand.  Per byte of weights a stage carries half the token bytes of the
 // one-block kernels, and three stages fit in shared memory: 96 KB of weights
-// in flight per SM instead of 64 KB.  (A probe of the ring without the math
-// streamed 4.8 TB/s of weights with the one-block layout and 5.5 TB/s with
-// this one.)  The price is tensor memory: two 192-column accumulators and the
-// two scale buffers fill all 512 columns, so the accumulators are not double
-// buffered.  Eight epilogue warps (two per lane quadrant, one per block) drain
-// them, and the MMAs of the next tile wait for that; the ring keeps loading
-// meanwhile.  So the kernel serves long K (K >= 2048), where a tile's main loop
-// is much longer than its drain.  Outputs are bf16 (or SwiGLU h, or NVFP4 h).
+// in flight per SM instead of 64 KB.  (A probe ring of copies without the math
+// streamed 4.8 TB/s of weights with the one-block kernel's two 80 KB slots and
+// 5.5 TB/s with three slots of 32 KB of weights and 24 KB of tokens, the bytes
+// of this kernel's slots.)  The price is tensor memory: two 192-column
+// accumulators and the two scale buffers fill all 512 columns, so the
+// accumulators are not double buffered.  Eight epilogue warps (two per lane
+// quadrant, one per block) drain them, and the MMAs of the next tile wait for
+// that; the ring keeps loading meanwhile.  So the kernel serves K >= 1024 (four
+// or more stages per tile), where a tile's main loop is longer than its drain.
+// Outputs are bf16 (or SwiGLU h, or NVFP4 h).
 #include "gemm_common.cuh"
 #include "host_util.cuh"
 
