@@ -82,11 +82,11 @@ def grouped_gemm_kernel_name(R, E, N, K, bf16_out, swiglu):
     """The kernel nvfp4_grouped_gemm's automatic choice launches for this
     problem (its rule, restated for the bench line's label only)."""
     tag = "<swiglu>" if swiglu else ""
-    if R <= 16 * E:
-        return f"nvfp4::gemm::grouped_gemm_k512_kernel{tag} (deep ring)"
     if N % 256 == 0 and bf16_out and K >= 1024:
         return f"nvfp4::gemm::w2::grouped_gemm_w2_kernel{tag} (two weight blocks per tile)"
-    return f"nvfp4::gemm::grouped_gemm_k512_kernel{tag}" if K % 512 == 0 else f"nvfp4::gemm::grouped_gemm_kernel{tag}"
+    if K % 512 != 0:
+        return f"nvfp4::gemm::grouped_gemm_kernel{tag}"
+    return f"nvfp4::gemm::grouped_gemm_k512_kernel{tag}" + (" (deep ring)" if R <= 16 * E else "")
 FP4_PEAK = PEAKS.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]) * FP4_OVER_BF16
 
 

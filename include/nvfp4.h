@@ -403,13 +403,12 @@ nvfp4_status nvfp4_grouped_gemm_w4a16(const void *x, int64_t ld_x, int64_t x_row
 /*
  * nvfp4_gemm_select_kernel -- which grouped GEMM kernel nvfp4_grouped_gemm runs
  * (process-wide; a tuning and testing switch, not part of the pages' method):
- *   0  automatic (default): when the experts average at most 16 routed rows
- *      (M_total <= 16 * num_experts), one CTA per 128-row weight tile with
- *      512-element K stages and tiles of at most 64 tokens in a ring of three
- *      slots; otherwise, for a bf16 output with N % 256 == 0 and K >= 1024,
- *      the kernel of mode 4; otherwise one CTA per 128-row weight tile with
- *      512-element K stages (tiles of at most 192 tokens, two slots) when
- *      K % 512 == 0 and 256-element stages when not;
+ *   0  automatic (default): for a bf16 output with N % 256 == 0 and
+ *      K >= 1024, the kernel of mode 4; otherwise one CTA per 128-row weight
+ *      tile, with 512-element K stages when K % 512 == 0 (tiles of at most 64
+ *      tokens in a ring of three slots when the experts average at most 16
+ *      routed rows, M_total <= 16 * num_experts; of at most 192 tokens in two
+ *      slots otherwise) and 256-element stages when not;
  *   1  one CTA per tile, 256-element K stages;  2  CTA pairs (tcgen05
  *      cta_group::2, 256 weight rows per tile; N % 256 != 0 is then
  *      NVFP4_ERR_UNSUPPORTED_SHAPE);  3  the three-slot, 64-token ring

@@ -299,12 +299,13 @@ using namespace nvfp4;
 
 namespace {
 
-// 0 automatic (the deep 512-element ring when the groups average at most 16
-// rows; else two weight blocks per tile for bf16 outputs with N % 256 == 0 and
-// K >= 1024; else 512-element stages when K % 512 == 0; else one CTA per tile
-// with 256-element stages), 1 one CTA per tile with 256-element stages, 2 CTA
-// pairs, 3 the deep 512-element ring whenever K % 512 == 0, 4 two weight
-// blocks per tile whenever N % 256 == 0 and the output is bf16 (else as 0)
+// 0 automatic (two weight blocks per tile for bf16 outputs with N % 256 == 0
+// and K >= 1024; else the deep 512-element ring when the groups average at
+// most 16 rows; else 512-element stages when K % 512 == 0; else one CTA per
+// tile with 256-element stages), 1 one CTA per tile with 256-element stages,
+// 2 CTA pairs, 3 the deep 512-element ring whenever K % 512 == 0, 4 two
+// weight blocks per tile whenever N % 256 == 0 and the output is bf16 (else
+// as 0)
 std::atomic<int> g_gemm_kernel{0};
 
 }  // namespace
@@ -318,13 +319,13 @@ bool deep_ring(int64_t M_total, int E) {
 
 // The two-weight-block kernel (gemm_w2.cu) serves NVFP4 operands with a bf16
 // output (plain, SwiGLU h or NVFP4 h) and N % 256 == 0: always in mode 4, and
-// in mode 0 outside the deep ring's regime when K >= 1024 (its single
-// accumulator pair drains between tiles, which a K loop of at least four
-// stages hides behind the ring's loads).
-bool use_w2(int64_t M_total, int E, int64_t N, int64_t K, bool bf16_out) {
+// in mode 0 when K >= 1024 (its single accumulator pair drains between tiles,
+// which a K loop of at least four stages hides behind the ring's loads), for
+// decode-sized groups as well as large ones.
+bool use_w2(int64_t N, int64_t K, bool bf16_out) {
   if (N % 256 != 0 || !bf16_out) return false;
   const int mode = g_gemm_kernel.load();
-  return mode == 4 || (mode == 0 && K >= 1024 && !deep_ring(M_total, E));
+  return mode == 4 || (mode == 0 && K >= 1024);
 }
 
 // One CTA per SM, but no more CTAs than tiles can exist: each expert has at
@@ -358,7 +359,7 @@ extern "C" nvfp4_status nvfp4_grouped_gemm(const uint8_t *a_q, const uint8_t *a_
   if ((reinterpret_cast<uintptr_t>(a_q) | reinterpret_cast<uintptr_t>(b_q) | reinterpret_cast<uintptr_t>(a_sf) |
        reinterpret_cast<uintptr_t>(b_sf) | reinterpret_cast<uintptr_t>(y)) & 15u)
     return NVFP4_ERR_INVALID_ARG;
-  if (use_w2(M_total, E, N, K, out_dtype == NVFP4_OUT_BF16))
+  if (use_w2(N, K, out_dtype == NVFP4_OUT_BF16))
     return gemm::launch_grouped_gemm_w2(a_q, a_sf, a_gs, b_q, b_sf, b_gs, expert_offsets, E, M_total, N, K, y, swiglu,
                                         amax_out, nullptr, dev_status, stream);
   if (g_gemm_kernel == 2)
@@ -418,7 +419,7 @@ extern "C" nvfp4_status nvfp4_grouped_gemm_swiglu_nvfp4(const uint8_t *a_q, cons
   hq.gs = h_gs;
   hq.q = h_q;
   hq.sf = h_sf;
-  if (use_w2(M_total, E, N, K, true))
+  if (use_w2(N, K, true))
     return gemm::launch_grouped_gemm_w2(a_q, a_sf, a_gs, b_q, b_sf, b_gs, expert_offsets, E, M_total, N, K, nullptr,
                                         true, nullptr, &hq, dev_status, stream);
   if ((g_gemm_kernel == 0 || g_gemm_kernel == 3) && K % 512 == 0)

@@ -40,7 +40,8 @@ def status_word():
 def gemm_kernel(request):
     """Run the test on each grouped GEMM kernel: automatic (the two-block
     kernel for bf16 outputs with N % 256 == 0 and K >= 1024, else 512-element K
-    stages when K % 512 == 0), one CTA per tile with 256-element stages, the
+    stages when K % 512 == 0, with the deep ring for decode-sized groups), one
+    CTA per tile with 256-element stages, the
     CTA-pair kernel, the 512-element kernel's deep ring (tiles of at most
     64 tokens, three slots), and two weight blocks per tile (bf16 outputs with
     N % 256 == 0; other calls of that mode run the automatic choice)."""
