@@ -310,11 +310,14 @@ std::atomic<int> g_gemm_kernel{0};
 
 }  // namespace
 
-// The deep ring (64-token tiles, three slots) in mode 3, and in mode 0 for
-// problems of few tokens per expert.
+// Decode-sized groups: the experts average at most 16 routed rows.
+bool small_groups(int64_t M_total, int E) { return M_total <= gemm::kDeepRingMaxRowsPerExpert * (int64_t)E; }
+
+// The deep ring of the one-block kernel (64-token tiles, three slots) in mode
+// 3, and in mode 0 for small groups.
 bool deep_ring(int64_t M_total, int E) {
   const int mode = g_gemm_kernel.load();
-  return mode == 3 || (mode == 0 && M_total <= gemm::kDeepRingMaxRowsPerExpert * (int64_t)E);
+  return mode == 3 || (mode == 0 && small_groups(M_total, E));
 }
 
 // The two-weight-block kernel (gemm_w2.cu) serves NVFP4 operands with a bf16
@@ -361,7 +364,7 @@ extern "C" nvfp4_status nvfp4_grouped_gemm(const uint8_t *a_q, const uint8_t *a_
     return NVFP4_ERR_INVALID_ARG;
   if (use_w2(N, K, out_dtype == NVFP4_OUT_BF16))
     return gemm::launch_grouped_gemm_w2(a_q, a_sf, a_gs, b_q, b_sf, b_gs, expert_offsets, E, M_total, N, K, y, swiglu,
-                                        amax_out, nullptr, dev_status, stream);
+                                        amax_out, nullptr, small_groups(M_total, E), dev_status, stream);
   if (g_gemm_kernel == 2)
     return gemm::launch_grouped_gemm_pair(a_q, a_sf, a_gs, b_q, b_sf, b_gs, expert_offsets, E, M_total, N, K, y,
                                           out_dtype, swiglu, amax_out, dev_status, stream);
@@ -421,7 +424,7 @@ extern "C" nvfp4_status nvfp4_grouped_gemm_swiglu_nvfp4(const uint8_t *a_q, cons
   hq.sf = h_sf;
   if (use_w2(N, K, true))
     return gemm::launch_grouped_gemm_w2(a_q, a_sf, a_gs, b_q, b_sf, b_gs, expert_offsets, E, M_total, N, K, nullptr,
-                                        true, nullptr, &hq, dev_status, stream);
+                                        true, nullptr, &hq, small_groups(M_total, E), dev_status, stream);
   if ((g_gemm_kernel == 0 || g_gemm_kernel == 3) && K % 512 == 0)
     return gemm::launch_grouped_gemm_k512(a_q, a_sf, a_gs, b_q, b_sf, b_gs, expert_offsets, E, M_total, N, K, nullptr,
                                           NVFP4_OUT_BF16, true, nullptr, &hq, false, deep_ring(M_total, E), dev_status, stream);

@@ -31,41 +31,53 @@ namespace nvfp4 {
 namespace gemm {
 namespace w2 {
 
-constexpr int kStages = 3;
 constexpr int W2_STAGE = 2 * W_STAGE;              // 256 rows x 128 B = 32 KB
-constexpr int X2_STAGE = BN * 128;                 // up to 192 token rows x 128 B = 24 KB
 constexpr int SFW2_STAGE = 2 * SFW_STAGE;          // two 128-row blocks x 2 KB
-constexpr int SFX2_STAGE = SFX_STAGE;              // up to two 128-row blocks x 2 KB
 constexpr int EPI2_WARP_BYTES = 2048;              // bf16 staging of 32 tokens x 32 columns
 constexpr int kEpiWarps = 8;
-constexpr int OFF_W = 0;
-constexpr int OFF_X = OFF_W + kStages * W2_STAGE;
-constexpr int OFF_SFW = OFF_X + kStages * X2_STAGE;
-constexpr int OFF_SFX = OFF_SFW + kStages * SFW2_STAGE;
-constexpr int OFF_EPI = OFF_SFX + kStages * SFX2_STAGE;
-constexpr int OFF_BAR = OFF_EPI + kEpiWarps * EPI2_WARP_BYTES;
-// wfull[S], wempty[S], xfull[S], xempty[S], sfw_data[S], sfx_data[S], sf_full[2], sf_free[2], acc_full, acc_empty, drain
-constexpr int NUM_BARS = 6 * kStages + 2 + 2 + 3;
-constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
-constexpr int OFF_GROUPS = OFF_MISC + 16;
 constexpr int kWarps = 15;
 constexpr int kThreads = kWarps * 32;
 constexpr int GROUP_BYTES = 3 * (kMaxExperts + 1) * 4 + 2 * kWarps * 4;   // off / slot / tile + scan scratch
-constexpr int SMEM_BYTES = OFF_GROUPS + GROUP_BYTES + 1024;
-static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-static_assert(OFF_X % 1024 == 0 && X2_STAGE % 1024 == 0 && W2_STAGE % 1024 == 0, "128-byte swizzle atoms");
+constexpr uint32_t kSfStride = 64;                 // per scale buffer: weight blocks 0 and 1 (16 + 16), tokens (32)
+
+// The ring and tensor-memory layout for tiles of at most kCap tokens in
+// kSlots slots.  (192, 3) is the general kernel.  (64, 4), for decode-sized
+// groups, has 8 KB token boxes, so a fourth slot fits (128 KB of weights in
+// flight per SM), and its accumulator pairs take 128 columns each, so two of
+// them fit beside the scale buffers: the epilogue of a tile overlaps the next
+// tile's MMAs.  A 64-token tile starts on a 64-row boundary and stays inside
+// one 128-row block of token scales.
+template <int kCap, int kSlots>
+struct W2Ring {
+  static constexpr int kAccBufs = (4 * kCap + 2 * (int)kSfStride <= (int)TMEM_COLS) ? 2 : 1;
+  static constexpr int X_STAGE = kCap * 128;
+  static constexpr int SFX_BYTES = kCap <= 64 ? SFW_STAGE : SFX_STAGE;
+  static constexpr int OFF_W = 0;
+  static constexpr int OFF_X = OFF_W + kSlots * W2_STAGE;
+  static constexpr int OFF_SFW = OFF_X + kSlots * X_STAGE;
+  static constexpr int OFF_SFX = OFF_SFW + kSlots * SFW2_STAGE;
+  static constexpr int OFF_EPI = OFF_SFX + kSlots * SFX_BYTES;
+  static constexpr int OFF_BAR = OFF_EPI + kEpiWarps * EPI2_WARP_BYTES;
+  // wfull, wempty, xfull, xempty, sfw_data, sfx_data [kSlots]; sf_full[2], sf_free[2],
+  // acc_full[kAccBufs], acc_empty[kAccBufs], drain
+  static constexpr int NUM_BARS = 6 * kSlots + 2 + 2 + 2 * kAccBufs + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  static constexpr int OFF_GROUPS = OFF_MISC + 16;
+  static constexpr int SMEM_BYTES = OFF_GROUPS + GROUP_BYTES + 1024;
+  // tensor memory: accumulator pair b at columns 2 kCap b (block 0) and
+  // 2 kCap b + kCap (block 1), then the two scale buffers
+  static constexpr uint32_t kAccPair = 2 * kCap;
+  static constexpr uint32_t kSf = kAccBufs * 2 * kCap;
+  static_assert(kSf + 2 * kSfStride <= TMEM_COLS, "tensor memory budget");
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(OFF_X % 1024 == 0 && X_STAGE % 1024 == 0 && W2_STAGE % 1024 == 0, "128-byte swizzle atoms");
+};
 
 // warps: 0 weight producer, 1 MMA, 2..5 epilogue of block 0, 6..9 scales,
 // 10 token producer, 11..14 epilogue of block 1
 constexpr int W_EPI_B = 11;
-// tensor memory: accumulators of block 0 and 1 at columns 0 and 192, scale
-// buffers at 384 and 448 (weight block 0: 16 columns, block 1: 16, tokens: 32)
-constexpr uint32_t kAcc1 = BN;
-constexpr uint32_t kSf = 2 * BN;
-constexpr uint32_t kSfStride = 64;
-static_assert(kSf + 2 * kSfStride <= TMEM_COLS, "tensor memory budget");
 
-template <bool kSwiglu, bool kQuantH>
+template <bool kSwiglu, bool kQuantH, int kCap, int kSlots>
 __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_w2_kernel(
     const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x32,
     const __grid_constant__ CUtensorMap tmap_x64, const __grid_constant__ CUtensorMap tmap_x128,
@@ -77,7 +89,10 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_w2_kernel(
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   const uint32_t sbase = smem_u32(smem);
-  const uint32_t bar_wfull = sbase + OFF_BAR;
+  using R = W2Ring<kCap, kSlots>;
+  constexpr int kStages = kSlots;
+  constexpr int kAccBufs = R::kAccBufs;
+  const uint32_t bar_wfull = sbase + R::OFF_BAR;
   const uint32_t bar_wempty = bar_wfull + 8 * kStages;
   const uint32_t bar_xfull = bar_wempty + 8 * kStages;
   const uint32_t bar_xempty = bar_xfull + 8 * kStages;
@@ -85,12 +100,12 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_w2_kernel(
   const uint32_t bar_sfx_data = bar_sfw_data + 8 * kStages;
   const uint32_t bar_sf_full = bar_sfx_data + 8 * kStages;   // [2], count 128 (scale warps)
   const uint32_t bar_sf_free = bar_sf_full + 16;              // [2], count 1 (MMA commit)
-  const uint32_t bar_acc_full = bar_sf_free + 16;             // count 1 (MMA commit)
-  const uint32_t bar_acc_empty = bar_acc_full + 8;            // count 256 (both blocks' epilogue threads)
-  const uint32_t bar_drain = bar_acc_empty + 8;
-  volatile uint32_t *tmem_holder = reinterpret_cast<volatile uint32_t *>(smem + OFF_MISC);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
-  int32_t *s_off = reinterpret_cast<int32_t *>(smem + OFF_GROUPS);
+  const uint32_t bar_acc_full = bar_sf_free + 16;             // [kAccBufs], count 1 (MMA commit)
+  const uint32_t bar_acc_empty = bar_acc_full + 8 * kAccBufs; // [kAccBufs], count 256 (both blocks' epilogues)
+  const uint32_t bar_drain = bar_acc_empty + 8 * kAccBufs;
+  volatile uint32_t *tmem_holder = reinterpret_cast<volatile uint32_t *>(smem + R::OFF_MISC);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + R::OFF_MISC + 4);
+  int32_t *s_off = reinterpret_cast<int32_t *>(smem + R::OFF_GROUPS);
   int32_t *s_slot = s_off + (kMaxExperts + 1);
   int32_t *s_tile = s_slot + (kMaxExperts + 1);
   int32_t *s_scratch = s_tile + (kMaxExperts + 1);
@@ -113,8 +128,10 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_w2_kernel(
       mbar_init(bar_sf_full + 8 * b, 128);
       mbar_init(bar_sf_free + 8 * b, 1);
     }
-    mbar_init(bar_acc_full, 1);
-    mbar_init(bar_acc_empty, 32 * kEpiWarps);
+    for (int b = 0; b < kAccBufs; ++b) {
+      mbar_init(bar_acc_full + 8 * b, 1);
+      mbar_init(bar_acc_empty + 8 * b, 32 * kEpiWarps);
+    }
     mbar_init(bar_drain, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -125,7 +142,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_w2_kernel(
   }
   // tiles of 256 weight rows (wrows = 2 * BM): decode_tile's w_row0 and n_col0
   // are those of the first block; the second block follows 128 rows later
-  build_tile_tables<BN, kThreads>(expert_offsets, E, M_total, n_mtiles, s_off, s_slot, s_tile, s_scratch, dev_status);
+  build_tile_tables<kCap, kThreads>(expert_offsets, E, M_total, n_mtiles, s_off, s_slot, s_tile, s_scratch, dev_status);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -157,7 +174,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_w2_kernel(
       uint32_t armed_parity[kStages] = {};
       bool ok = true;
       for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
-        const Tile T = decode_tile<kSwiglu>(t, s_off, s_slot, s_tile, E, N, 2 * BM, 0);
+        const Tile T = decode_tile<kSwiglu, kCap>(t, s_off, s_slot, s_tile, E, N, 2 * BM, 0);
         const int xr0 = T.x_row0 & ~127;
         const int nrb = ((T.x_row0 & 127) + T.n_valid + 127) >> 7;
         const int xbox = T.n_valid <= 32 ? 32 : T.n_valid <= 64 ? 64 : T.n_valid <= 128 ? 128 : 192;
@@ -175,15 +192,15 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_w2_kernel(
           armed[stage] = true;
           armed_parity[stage] = phase;
           if (is_w) {
-            bulk_load(sbase + OFF_SFW + stage * SFW2_STAGE, sfw_tile + ks * kSfStage, kSfStage, sb);
-            bulk_load(sbase + OFF_SFW + stage * SFW2_STAGE + kSfStage, sfw_tile + sf_row_stride + ks * kSfStage,
+            bulk_load(sbase + R::OFF_SFW + stage * SFW2_STAGE, sfw_tile + ks * kSfStage, kSfStage, sb);
+            bulk_load(sbase + R::OFF_SFW + stage * SFW2_STAGE + kSfStage, sfw_tile + sf_row_stride + ks * kSfStage,
                       kSfStage, sb);
-            tma_load_2d(sbase + OFF_W + stage * W2_STAGE, &tmap_w, ks * 128, T.w_row0, fb, pol);
+            tma_load_2d(sbase + R::OFF_W + stage * W2_STAGE, &tmap_w, ks * 128, T.w_row0, fb, pol);
           } else {
             for (int rb = 0; rb < nrb; ++rb)
-              bulk_load(sbase + OFF_SFX + stage * SFX2_STAGE + rb * kSfStage, sfx_tile + rb * sf_row_stride + ks * kSfStage,
-                        kSfStage, sb);
-            tma_load_2d(sbase + OFF_X + stage * X2_STAGE, xmap, ks * 128, T.x_row0, fb, pol);
+              bulk_load(sbase + R::OFF_SFX + stage * R::SFX_BYTES + rb * kSfStage,
+                        sfx_tile + rb * sf_row_stride + ks * kSfStage, kSfStage, sb);
+            tma_load_2d(sbase + R::OFF_X + stage * R::X_STAGE, xmap, ks * 128, T.x_row0, fb, pol);
           }
           if (++stage == kStages) { stage = 0; phase ^= 1; }
         }
@@ -206,7 +223,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_w2_kernel(
     uint32_t kst = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
-      const Tile T = decode_tile<kSwiglu>(t, s_off, s_slot, s_tile, E, N, 2 * BM, 0);
+      const Tile T = decode_tile<kSwiglu, kCap>(t, s_off, s_slot, s_tile, E, N, 2 * BM, 0);
       const int nrb = ((T.x_row0 & 127) + T.n_valid + 127) >> 7;
       for (int ks = 0; ks < ksteps && ok; ++ks, ++kst) {
         const uint32_t s = kst % kStages, par = (kst / kStages) & 1, sb = kst & 1;
@@ -217,9 +234,9 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_w2_kernel(
           ok = false; break;
         }
         tc_fence_after();
-        const uint32_t tcol = tmem_base + lane_base + kSf + sb * kSfStride;
-        const uint32_t sfw = sbase + OFF_SFW + s * SFW2_STAGE + lane * 16;
-        const uint32_t sfx = sbase + OFF_SFX + s * SFX2_STAGE + lane * 16;
+        const uint32_t tcol = tmem_base + lane_base + R::kSf + sb * kSfStride;
+        const uint32_t sfw = sbase + R::OFF_SFW + s * SFW2_STAGE + lane * 16;
+        const uint32_t sfx = sbase + R::OFF_SFX + s * R::SFX_BYTES + lane * 16;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) tc_st_x4(tcol + kk * 4, lds128(sfw + kk * 512));
 #pragma unroll
@@ -240,12 +257,14 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_w2_kernel(
     uint32_t kst = 0, titer = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++titer) {
-      const Tile T = decode_tile<kSwiglu>(t, s_off, s_slot, s_tile, E, N, 2 * BM, 0);
+      const Tile T = decode_tile<kSwiglu, kCap>(t, s_off, s_slot, s_tile, E, N, 2 * BM, 0);
       const uint32_t n_mma = (T.n_valid + 15) & ~15;
       const uint32_t idesc = idesc_mxf4nvf4(BM, n_mma);
       const uint32_t xoff = (uint32_t)(T.x_row0 & 127) >> 5;
-      // the single accumulator pair: the previous tile's epilogue must have read it
-      if (!mbar_wait_warp(bar_acc_empty, (titer & 1) ^ 1, abort_flag, dev_status)) {
+      // accumulator pair ab: the epilogue of the tile kAccBufs back must have read it
+      const uint32_t ab = titer % kAccBufs;
+      const uint32_t t_acc = tmem_base + ab * R::kAccPair;
+      if (!mbar_wait_warp(bar_acc_empty + 8 * ab, ((titer / kAccBufs) & 1) ^ 1, abort_flag, dev_status)) {
         ok = false; break;
       }
       tc_fence_after();
@@ -258,16 +277,16 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_w2_kernel(
         }
         tc_fence_after();
         if (lane == 0) {
-          const uint32_t t_sf = tmem_base + kSf + sb * kSfStride;
-          const uint64_t dw0 = desc_sw128(sbase + OFF_W + s * W2_STAGE);
-          const uint64_t dw1 = desc_sw128(sbase + OFF_W + s * W2_STAGE + W_STAGE);
-          const uint64_t dx = desc_sw128(sbase + OFF_X + s * X2_STAGE);
+          const uint32_t t_sf = tmem_base + R::kSf + sb * kSfStride;
+          const uint64_t dw0 = desc_sw128(sbase + R::OFF_W + s * W2_STAGE);
+          const uint64_t dw1 = desc_sw128(sbase + R::OFF_W + s * W2_STAGE + W_STAGE);
+          const uint64_t dx = desc_sw128(sbase + R::OFF_X + s * R::X_STAGE);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const uint32_t acc = (ks > 0 || kk > 0) ? 1u : 0u;
             // +32 bytes of K per MMA: +2 in the descriptor's 16-byte address field
-            tc_mma(tmem_base, dw0 + 2 * kk, dx + 2 * kk, idesc, t_sf + kk * 4, t_sf + 32 + kk * 8 + xoff, acc);
-            tc_mma(tmem_base + kAcc1, dw1 + 2 * kk, dx + 2 * kk, idesc, t_sf + 16 + kk * 4, t_sf + 32 + kk * 8 + xoff,
+            tc_mma(t_acc, dw0 + 2 * kk, dx + 2 * kk, idesc, t_sf + kk * 4, t_sf + 32 + kk * 8 + xoff, acc);
+            tc_mma(t_acc + kCap, dw1 + 2 * kk, dx + 2 * kk, idesc, t_sf + 16 + kk * 4, t_sf + 32 + kk * 8 + xoff,
                    acc);
           }
           tc_commit(bar_sf_free + 8 * sb);
@@ -277,7 +296,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_w2_kernel(
         __syncwarp();
       }
       if (!ok) break;
-      if (lane == 0) tc_commit(bar_acc_full);
+      if (lane == 0) tc_commit(bar_acc_full + 8 * ab);
       __syncwarp();
     }
     if (lane == 0) {
@@ -291,19 +310,21 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_w2_kernel(
     const int block = warp >= W_EPI_B ? 1 : 0;
     const int quad = warp & 3;
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
-    const uint32_t epi = sbase + OFF_EPI + (block * 4 + (warp - (block ? W_EPI_B : 2))) * EPI2_WARP_BYTES;
+    const uint32_t epi = sbase + R::OFF_EPI + (block * 4 + (warp - (block ? W_EPI_B : 2))) * EPI2_WARP_BYTES;
     uint32_t titer = 0;
     for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++titer) {
-      Tile T = decode_tile<kSwiglu>(t, s_off, s_slot, s_tile, E, N, 2 * BM, 0);
+      Tile T = decode_tile<kSwiglu, kCap>(t, s_off, s_slot, s_tile, E, N, 2 * BM, 0);
       if (block) {
         T.w_row0 += BM;
         T.n_col0 += kSwiglu ? BM / 2 : BM;
       }
-      if (!mbar_wait_warp(bar_acc_full, titer & 1, abort_flag, dev_status)) break;
+      const uint32_t ab = titer % kAccBufs;
+      if (!mbar_wait_warp(bar_acc_full + 8 * ab, (titer / kAccBufs) & 1, abort_flag, dev_status)) break;
       tc_fence_after();
       const float alpha = __fmul_rn(x_gs[T.e], w_gs[T.e]);
-      epilogue_tile<kSwiglu, true, kQuantH>(T, tmem_base + lane_base + (block ? kAcc1 : 0u), alpha, epi, quad, lane, N,
-                                            y, amax_out, bar_acc_empty, false, hq, dev_status);
+      epilogue_tile<kSwiglu, true, kQuantH>(T, tmem_base + lane_base + ab * R::kAccPair + (block ? kCap : 0), alpha,
+                                            epi, quad, lane, N, y, amax_out, bar_acc_empty + 8 * ab, false, hq,
+                                            dev_status);
     }
   }
 
@@ -321,12 +342,32 @@ nvfp4_status set_wait_budget_w2(long long cycles) {
   return cudaMemcpyToSymbol(c_wait_budget, &cycles, sizeof(cycles)) == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 
+template <int kCap, int kSlots>
+nvfp4_status launch_ring(const CUtensorMap &tw, const CUtensorMap &tx32, const CUtensorMap &tx64,
+                         const CUtensorMap &tx128, const CUtensorMap &tx192, const uint8_t *b_sf, const uint8_t *a_sf,
+                         const float *b_gs, const float *a_gs, const int32_t *expert_offsets, int E, int64_t M_total,
+                         int64_t N, int64_t K, void *y, bool swiglu, float *amax_out, const HQuantOut *hq,
+                         int32_t *dev_status, cudaStream_t stream) {
+  using R = w2::W2Ring<kCap, kSlots>;
+  auto kern = hq ? w2::grouped_gemm_w2_kernel<true, true, kCap, kSlots>
+                 : swiglu ? w2::grouped_gemm_w2_kernel<true, false, kCap, kSlots>
+                          : w2::grouped_gemm_w2_kernel<false, false, kCap, kSlots>;
+  if (!host::set_max_dynamic_smem(reinterpret_cast<const void *>(kern), R::SMEM_BYTES)) return NVFP4_ERR_CUDA;
+  // no more CTAs than tiles: each expert has at most m_e / kCap + 1 token chunks per weight-block pair
+  const int64_t tile_bound = (N / (2 * BM)) * ((M_total + kCap - 1) / kCap + E);
+  const int grid = (int)(tile_bound < host::sm_count() ? tile_bound : host::sm_count());
+  kern<<<grid, w2::kThreads, R::SMEM_BYTES, stream>>>(tw, tx32, tx64, tx128, tx192, b_sf, a_sf, b_gs, a_gs,
+                                                      expert_offsets, E, (int)M_total, (int)N, (int)K, y, amax_out,
+                                                      dev_status, hq ? *hq : HQuantOut{});
+  return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
 // Arguments are validated by the callers; N % 256 == 0, K % 256 == 0, bf16
 // output (or SwiGLU h, or NVFP4 h when hq is given).
 nvfp4_status launch_grouped_gemm_w2(const uint8_t *a_q, const uint8_t *a_sf, const float *a_gs, const uint8_t *b_q,
                                     const uint8_t *b_sf, const float *b_gs, const int32_t *expert_offsets, int E,
                                     int64_t M_total, int64_t N, int64_t K, void *y, bool swiglu, float *amax_out,
-                                    const HQuantOut *hq, int32_t *dev_status, cudaStream_t stream) {
+                                    const HQuantOut *hq, bool deep, int32_t *dev_status, cudaStream_t stream) {
   const int64_t x_rows = nvfp4_padded_rows_bound(M_total, E);
   CUtensorMap tw, tx32, tx64, tx128, tx192;
   if (!make_map(&tw, b_q, (uint64_t)E * N, (uint64_t)K / 2, 2 * BM)) return NVFP4_ERR_CUDA;
@@ -334,15 +375,10 @@ nvfp4_status launch_grouped_gemm_w2(const uint8_t *a_q, const uint8_t *a_sf, con
   if (!make_map(&tx64, a_q, (uint64_t)x_rows, (uint64_t)K / 2, 64)) return NVFP4_ERR_CUDA;
   if (!make_map(&tx128, a_q, (uint64_t)x_rows, (uint64_t)K / 2, 128)) return NVFP4_ERR_CUDA;
   if (!make_map(&tx192, a_q, (uint64_t)x_rows, (uint64_t)K / 2, 192)) return NVFP4_ERR_CUDA;
-  auto kern = hq ? w2::grouped_gemm_w2_kernel<true, true>
-                 : swiglu ? w2::grouped_gemm_w2_kernel<true, false> : w2::grouped_gemm_w2_kernel<false, false>;
-  if (!host::set_max_dynamic_smem(reinterpret_cast<const void *>(kern), w2::SMEM_BYTES)) return NVFP4_ERR_CUDA;
-  const int64_t tile_bound = (N / (2 * BM)) * ((M_total + BN - 1) / BN + E);
-  const int grid = (int)(tile_bound < host::sm_count() ? tile_bound : host::sm_count());
-  kern<<<grid, w2::kThreads, w2::SMEM_BYTES, stream>>>(tw, tx32, tx64, tx128, tx192, b_sf, a_sf, b_gs, a_gs,
-                                                       expert_offsets, E, (int)M_total, (int)N, (int)K, y, amax_out,
-                                                       dev_status, hq ? *hq : HQuantOut{});
-  return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+  if (deep) return launch_ring<64, 4>(tw, tx32, tx64, tx128, tx192, b_sf, a_sf, b_gs, a_gs, expert_offsets, E, M_total,
+                                     N, K, y, swiglu, amax_out, hq, dev_status, stream);
+  return launch_ring<BN, 3>(tw, tx32, tx64, tx128, tx192, b_sf, a_sf, b_gs, a_gs, expert_offsets, E, M_total, N, K, y,
+                            swiglu, amax_out, hq, dev_status, stream);
 }
 
 }  // namespace gemm

@@ -1142,6 +1142,55 @@ def test_gemm_two_blocks_max_experts():
     assert np.array_equal(y4, y1)
 
 
+@pytest.mark.parametrize("swiglu", [False, True])
+def test_gemm_two_blocks_small_groups(swiglu):
+    """Decode-sized groups (at most 16 routed rows per expert on average) take
+    the two-block kernel's 64-token tiles in four slots with two accumulator
+    pairs: expert sizes around the 64-row chunk edges among many empty ones,
+    bf16 Y (or SwiGLU h and its amax) bit for bit those of the one-CTA kernel
+    with 256-element stages."""
+    L = layer()
+    nv = nvmod()
+    counts = [1, 63, 64, 65, 127, 128, 129, 0, 2, 17, 191, 193] + [0] * 60 + [3, 5]
+    E, N, K = len(counts), 512, 1024
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    R = int(offsets[-1])
+    assert R <= 16 * E
+    x = synthetic.gaussian_bf16(37, synthetic.STREAMS["x"], (R, K), outlier_frac=0.001)
+    w = synthetic.gaussian_bf16(37, synthetic.STREAMS["w_gate_up"], (E * N, K), sigma=0.02)
+    q, sf, gs, qs, ss = _packed_acts(x, None, offsets, E)
+    qw, sw, gw = _packed_weights(w, E, N, K)
+    if not swiglu:
+        try:
+            nv.nvfp4_gemm_select_kernel(4)
+            y4 = _run_gemm(qs, ss, gs, qw, sw, gw, offsets, E, R, N, K, 1)
+            nv.nvfp4_gemm_select_kernel(1)
+            y1 = _run_gemm(qs, ss, gs, qw, sw, gw, offsets, E, R, N, K, 1)
+        finally:
+            nv.nvfp4_gemm_select_kernel(0)
+        assert np.array_equal(y4, y1)
+        return
+    bound = nv.nvfp4_padded_rows_bound(R, E)
+    qa = np.zeros((bound, K // 2), np.uint8)
+    qa[:qs.shape[0]] = qs
+    sa = np.zeros((bound, K // 16), np.uint8)
+    sa[:ss.shape[0]] = ss
+    a = L.Packed(to_dev(qa), to_dev(tile(sa)), to_dev(gs), R, K, 1, to_dev(offsets), E)
+    wp = L.Packed(to_dev(qw), to_dev(tile(sw)), to_dev(gw), E * N, K, 1)
+    out = {}
+    try:
+        for mode in (4, 1):
+            nv.nvfp4_gemm_select_kernel(mode)
+            st = status_word()
+            h, amax = L.grouped_gemm_swiglu(a, wp, N, dev_status=st)
+            torch.cuda.synchronize()
+            assert int(st.item()) == 0
+            out[mode] = (to_np(h), to_np(amax))
+    finally:
+        nv.nvfp4_gemm_select_kernel(0)
+    assert np.array_equal(out[4][0], out[1][0]) and np.array_equal(out[4][1], out[1][1])
+
+
 def test_gemm_two_blocks_long_k_bf16():
     """The two-weight-block kernel on ragged groups with K = 4096 (16 turns of
     its three-slot ring per tile) and 4 weight-block pairs per expert: bf16 Y
