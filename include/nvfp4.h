@@ -416,8 +416,9 @@ nvfp4_status nvfp4_grouped_gemm_w4a16(const void *x, int64_t ld_x, int64_t x_row
  *      128-row weight blocks per tile sharing one token tile, three
  *      256-element K stages, whenever N % 256 == 0 and the output is bf16
  *      (plain Y, SwiGLU h, or NVFP4 h from nvfp4_grouped_gemm_swiglu_nvfp4);
- *      other calls run as in mode 0 (mxfp4_grouped_gemm always does).
- *      The modes apply to nvfp4_grouped_gemm_swiglu_nvfp4 too.
+ *      other calls run as in mode 0.
+ *      The modes apply to nvfp4_grouped_gemm_swiglu_nvfp4 too, and modes 0
+ *      and 4 to mxfp4_grouped_gemm (its other modes run as mode 0).
  * All give the same Y up to the fp32 accumulation order inside a tile.
  * Returns NVFP4_ERR_INVALID_ARG for another mode.
  */

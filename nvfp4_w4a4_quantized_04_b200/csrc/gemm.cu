@@ -305,7 +305,7 @@ namespace {
 // tile with 256-element stages), 1 one CTA per tile with 256-element stages,
 // 2 CTA pairs, 3 the deep 512-element ring whenever K % 512 == 0, 4 two
 // weight blocks per tile whenever N % 256 == 0 and the output is bf16 (else
-// as 0)
+// as 0); the MXFP4 GEMM follows the same rule
 std::atomic<int> g_gemm_kernel{0};
 
 }  // namespace
@@ -364,7 +364,7 @@ extern "C" nvfp4_status nvfp4_grouped_gemm(const uint8_t *a_q, const uint8_t *a_
     return NVFP4_ERR_INVALID_ARG;
   if (use_w2(N, K, out_dtype == NVFP4_OUT_BF16))
     return gemm::launch_grouped_gemm_w2(a_q, a_sf, a_gs, b_q, b_sf, b_gs, expert_offsets, E, M_total, N, K, y, swiglu,
-                                        amax_out, nullptr, small_groups(M_total, E), dev_status, stream);
+                                        amax_out, nullptr, false, small_groups(M_total, E), dev_status, stream);
   if (g_gemm_kernel == 2)
     return gemm::launch_grouped_gemm_pair(a_q, a_sf, a_gs, b_q, b_sf, b_gs, expert_offsets, E, M_total, N, K, y,
                                           out_dtype, swiglu, amax_out, dev_status, stream);
@@ -424,7 +424,7 @@ extern "C" nvfp4_status nvfp4_grouped_gemm_swiglu_nvfp4(const uint8_t *a_q, cons
   hq.sf = h_sf;
   if (use_w2(N, K, true))
     return gemm::launch_grouped_gemm_w2(a_q, a_sf, a_gs, b_q, b_sf, b_gs, expert_offsets, E, M_total, N, K, nullptr,
-                                        true, nullptr, &hq, small_groups(M_total, E), dev_status, stream);
+                                        true, nullptr, &hq, false, small_groups(M_total, E), dev_status, stream);
   if ((g_gemm_kernel == 0 || g_gemm_kernel == 3) && K % 512 == 0)
     return gemm::launch_grouped_gemm_k512(a_q, a_sf, a_gs, b_q, b_sf, b_gs, expert_offsets, E, M_total, N, K, nullptr,
                                           NVFP4_OUT_BF16, true, nullptr, &hq, false, deep_ring(M_total, E), dev_status, stream);
@@ -461,6 +461,9 @@ extern "C" nvfp4_status mxfp4_grouped_gemm(const uint8_t *a_q, const uint8_t *a_
   if ((reinterpret_cast<uintptr_t>(a_q) | reinterpret_cast<uintptr_t>(b_q) | reinterpret_cast<uintptr_t>(a_sf) |
        reinterpret_cast<uintptr_t>(b_sf) | reinterpret_cast<uintptr_t>(y)) & 15u)
     return NVFP4_ERR_INVALID_ARG;
+  if (use_w2(N, K, out_dtype == NVFP4_OUT_BF16))
+    return gemm::launch_grouped_gemm_w2(a_q, a_sf, nullptr, b_q, b_sf, nullptr, expert_offsets, E, M_total, N, K, y,
+                                        false, nullptr, nullptr, true, small_groups(M_total, E), dev_status, stream);
   if ((g_gemm_kernel == 0 || g_gemm_kernel == 3) && K % 512 == 0)
     return gemm::launch_grouped_gemm_k512(a_q, a_sf, nullptr, b_q, b_sf, nullptr, expert_offsets, E, M_total, N, K, y,
                                           out_dtype, false, nullptr, nullptr, true, deep_ring(M_total, E), dev_status, stream);

@@ -820,12 +820,14 @@ nvfp4_status set_wait_budget_k512(long long cycles);
 
 // The two-weight-block kernel's launch (gemm_w2.cu): N % 256 == 0, bf16
 // output (SwiGLU h when swiglu, NVFP4 h when hq != nullptr), NVFP4 operands;
-// deep selects tiles of at most 64 tokens in four slots with double-buffered
+// mx selects MXFP4 operands (plain output, a_gs and b_gs not read); deep
+// selects tiles of at most 64 tokens in four slots with double-buffered
 // accumulators (decode-sized groups) instead of 192 tokens in three slots.
 nvfp4_status launch_grouped_gemm_w2(const uint8_t *a_q, const uint8_t *a_sf, const float *a_gs, const uint8_t *b_q,
                                     const uint8_t *b_sf, const float *b_gs, const int32_t *expert_offsets, int E,
                                     int64_t M_total, int64_t N, int64_t K, void *y, bool swiglu, float *amax_out,
-                                    const HQuantOut *hq, bool deep, int32_t *dev_status, cudaStream_t stream);
+                                    const HQuantOut *hq, bool mx, bool deep, int32_t *dev_status,
+                                    cudaStream_t stream);
 nvfp4_status set_wait_budget_w2(long long cycles);
 
 // The pair kernel's launch (gemm_pair.cu).  Requires N % 256 == 0.

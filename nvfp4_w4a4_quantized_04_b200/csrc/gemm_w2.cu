@@ -77,7 +77,10 @@ struct W2Ring {
 // 10 token producer, 11..14 epilogue of block 1
 constexpr int W_EPI_B = 11;
 
-template <bool kSwiglu, bool kQuantH, int kCap, int kSlots>
+// kMx: MXFP4 operands (kind::mxf4, one UE8M0 scale per 32 elements, no global
+// scales; a K stage holds two 512-byte scale atoms per row block instead of
+// four); otherwise NVFP4 (kind::mxf4nvf4, E4M3 per 16 elements).
+template <bool kSwiglu, bool kQuantH, int kCap, int kSlots, bool kMx = false>
 __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_w2_kernel(
     const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x32,
     const __grid_constant__ CUtensorMap tmap_x64, const __grid_constant__ CUtensorMap tmap_x128,
@@ -148,8 +151,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_w2_kernel(
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
   const int total_tiles = s_tile[E];
-  const int64_t sf_row_stride = (int64_t)(K / 64) * 512;     // bytes per 128-row block of scales
-  constexpr uint32_t kSfStage = 2048u;                       // one row block's scales of a K stage
+  const int64_t sf_row_stride = (int64_t)(K / (kMx ? 128 : 64)) * 512;   // bytes per 128-row block of scales
+  constexpr uint32_t kSfStage = kMx ? 1024u : 2048u;                     // one row block's scales of a K stage
 
   if (warp == W_PRODUCER || warp == W_XLOAD) {
     // ================================================================ TMA producers
@@ -237,15 +240,36 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_w2_kernel(
         const uint32_t tcol = tmem_base + lane_base + R::kSf + sb * kSfStride;
         const uint32_t sfw = sbase + R::OFF_SFW + s * SFW2_STAGE + lane * 16;
         const uint32_t sfx = sbase + R::OFF_SFX + s * R::SFX_BYTES + lane * 16;
+        if constexpr (kMx) {
+          // an MX atom covers two MMAs (128 elements): each MMA gets its own 4
+          // columns with its two scales in bytes 0 and 1 of the row's word
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) tc_st_x4(tcol + kk * 4, lds128(sfw + kk * 512));
+          for (int a = 0; a < 2; ++a) {
+            const uint4 w0 = lds128(sfw + a * 512), w1 = lds128(sfw + kSfStage + a * 512);
+            const uint4 x0 = lds128(sfx + a * 512);
+            tc_st_x4(tcol + (2 * a) * 4, lo16x4(w0));
+            tc_st_x4(tcol + (2 * a + 1) * 4, hi16x4(w0));
+            tc_st_x4(tcol + 16 + (2 * a) * 4, lo16x4(w1));
+            tc_st_x4(tcol + 16 + (2 * a + 1) * 4, hi16x4(w1));
+            tc_st_x4(tcol + 32 + (2 * a) * 8, lo16x4(x0));
+            tc_st_x4(tcol + 32 + (2 * a + 1) * 8, hi16x4(x0));
+            if (nrb > 1) {
+              const uint4 x1 = lds128(sfx + kSfStage + a * 512);
+              tc_st_x4(tcol + 32 + (2 * a) * 8 + 4, lo16x4(x1));
+              tc_st_x4(tcol + 32 + (2 * a + 1) * 8 + 4, hi16x4(x1));
+            }
+          }
+        } else {
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) tc_st_x4(tcol + 16 + kk * 4, lds128(sfw + kSfStage + kk * 512));
+          for (int kk = 0; kk < 4; ++kk) tc_st_x4(tcol + kk * 4, lds128(sfw + kk * 512));
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) tc_st_x4(tcol + 32 + kk * 8, lds128(sfx + kk * 512));
-        if (nrb > 1) {
+          for (int kk = 0; kk < 4; ++kk) tc_st_x4(tcol + 16 + kk * 4, lds128(sfw + kSfStage + kk * 512));
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) tc_st_x4(tcol + 32 + kk * 8 + 4, lds128(sfx + kSfStage + kk * 512));
+          for (int kk = 0; kk < 4; ++kk) tc_st_x4(tcol + 32 + kk * 8, lds128(sfx + kk * 512));
+          if (nrb > 1) {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) tc_st_x4(tcol + 32 + kk * 8 + 4, lds128(sfx + kSfStage + kk * 512));
+          }
         }
         tc_wait_st();
         tc_fence_before();
@@ -259,7 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_w2_kernel(
     for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++titer) {
       const Tile T = decode_tile<kSwiglu, kCap>(t, s_off, s_slot, s_tile, E, N, 2 * BM, 0);
       const uint32_t n_mma = (T.n_valid + 15) & ~15;
-      const uint32_t idesc = idesc_mxf4nvf4(BM, n_mma);
+      const uint32_t idesc = kMx ? idesc_mxf4_ue8m0(BM, n_mma) : idesc_mxf4nvf4(BM, n_mma);
       const uint32_t xoff = (uint32_t)(T.x_row0 & 127) >> 5;
       // accumulator pair ab: the epilogue of the tile kAccBufs back must have read it
       const uint32_t ab = titer % kAccBufs;
@@ -285,9 +309,15 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_w2_kernel(
           for (int kk = 0; kk < 4; ++kk) {
             const uint32_t acc = (ks > 0 || kk > 0) ? 1u : 0u;
             // +32 bytes of K per MMA: +2 in the descriptor's 16-byte address field
-            tc_mma(t_acc, dw0 + 2 * kk, dx + 2 * kk, idesc, t_sf + kk * 4, t_sf + 32 + kk * 8 + xoff, acc);
-            tc_mma(t_acc + kCap, dw1 + 2 * kk, dx + 2 * kk, idesc, t_sf + 16 + kk * 4, t_sf + 32 + kk * 8 + xoff,
-                   acc);
+            if constexpr (kMx) {
+              tc_mma_mx(t_acc, dw0 + 2 * kk, dx + 2 * kk, idesc, t_sf + kk * 4, t_sf + 32 + kk * 8 + xoff, acc);
+              tc_mma_mx(t_acc + kCap, dw1 + 2 * kk, dx + 2 * kk, idesc, t_sf + 16 + kk * 4,
+                        t_sf + 32 + kk * 8 + xoff, acc);
+            } else {
+              tc_mma(t_acc, dw0 + 2 * kk, dx + 2 * kk, idesc, t_sf + kk * 4, t_sf + 32 + kk * 8 + xoff, acc);
+              tc_mma(t_acc + kCap, dw1 + 2 * kk, dx + 2 * kk, idesc, t_sf + 16 + kk * 4, t_sf + 32 + kk * 8 + xoff,
+                     acc);
+            }
           }
           tc_commit(bar_sf_free + 8 * sb);
           tc_commit(bar_wempty + 8 * s);
@@ -321,7 +351,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_w2_kernel(
       const uint32_t ab = titer % kAccBufs;
       if (!mbar_wait_warp(bar_acc_full + 8 * ab, (titer / kAccBufs) & 1, abort_flag, dev_status)) break;
       tc_fence_after();
-      const float alpha = __fmul_rn(x_gs[T.e], w_gs[T.e]);
+      const float alpha = kMx ? 1.0f : __fmul_rn(x_gs[T.e], w_gs[T.e]);
       epilogue_tile<kSwiglu, true, kQuantH>(T, tmem_base + lane_base + ab * R::kAccPair + (block ? kCap : 0), alpha,
                                             epi, quad, lane, N, y, amax_out, bar_acc_empty + 8 * ab, false, hq,
                                             dev_status);
@@ -342,16 +372,17 @@ nvfp4_status set_wait_budget_w2(long long cycles) {
   return cudaMemcpyToSymbol(c_wait_budget, &cycles, sizeof(cycles)) == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 
-template <int kCap, int kSlots>
+template <int kCap, int kSlots, bool kMx>
 nvfp4_status launch_ring(const CUtensorMap &tw, const CUtensorMap &tx32, const CUtensorMap &tx64,
                          const CUtensorMap &tx128, const CUtensorMap &tx192, const uint8_t *b_sf, const uint8_t *a_sf,
                          const float *b_gs, const float *a_gs, const int32_t *expert_offsets, int E, int64_t M_total,
                          int64_t N, int64_t K, void *y, bool swiglu, float *amax_out, const HQuantOut *hq,
                          int32_t *dev_status, cudaStream_t stream) {
   using R = w2::W2Ring<kCap, kSlots>;
-  auto kern = hq ? w2::grouped_gemm_w2_kernel<true, true, kCap, kSlots>
-                 : swiglu ? w2::grouped_gemm_w2_kernel<true, false, kCap, kSlots>
-                          : w2::grouped_gemm_w2_kernel<false, false, kCap, kSlots>;
+  auto kern = kMx ? w2::grouped_gemm_w2_kernel<false, false, kCap, kSlots, true>
+             : hq ? w2::grouped_gemm_w2_kernel<true, true, kCap, kSlots>
+                  : swiglu ? w2::grouped_gemm_w2_kernel<true, false, kCap, kSlots>
+                           : w2::grouped_gemm_w2_kernel<false, false, kCap, kSlots>;
   if (!host::set_max_dynamic_smem(reinterpret_cast<const void *>(kern), R::SMEM_BYTES)) return NVFP4_ERR_CUDA;
   // no more CTAs than tiles: each expert has at most m_e / kCap + 1 token chunks per weight-block pair
   const int64_t tile_bound = (N / (2 * BM)) * ((M_total + kCap - 1) / kCap + E);
@@ -363,11 +394,13 @@ nvfp4_status launch_ring(const CUtensorMap &tw, const CUtensorMap &tx32, const C
 }
 
 // Arguments are validated by the callers; N % 256 == 0, K % 256 == 0, bf16
-// output (or SwiGLU h, or NVFP4 h when hq is given).
+// output (or SwiGLU h, or NVFP4 h when hq is given; MXFP4 operands, mx, only
+// with a plain output and without global scales).
 nvfp4_status launch_grouped_gemm_w2(const uint8_t *a_q, const uint8_t *a_sf, const float *a_gs, const uint8_t *b_q,
                                     const uint8_t *b_sf, const float *b_gs, const int32_t *expert_offsets, int E,
                                     int64_t M_total, int64_t N, int64_t K, void *y, bool swiglu, float *amax_out,
-                                    const HQuantOut *hq, bool deep, int32_t *dev_status, cudaStream_t stream) {
+                                    const HQuantOut *hq, bool mx, bool deep, int32_t *dev_status,
+                                    cudaStream_t stream) {
   const int64_t x_rows = nvfp4_padded_rows_bound(M_total, E);
   CUtensorMap tw, tx32, tx64, tx128, tx192;
   if (!make_map(&tw, b_q, (uint64_t)E * N, (uint64_t)K / 2, 2 * BM)) return NVFP4_ERR_CUDA;
@@ -375,10 +408,15 @@ nvfp4_status launch_grouped_gemm_w2(const uint8_t *a_q, const uint8_t *a_sf, con
   if (!make_map(&tx64, a_q, (uint64_t)x_rows, (uint64_t)K / 2, 64)) return NVFP4_ERR_CUDA;
   if (!make_map(&tx128, a_q, (uint64_t)x_rows, (uint64_t)K / 2, 128)) return NVFP4_ERR_CUDA;
   if (!make_map(&tx192, a_q, (uint64_t)x_rows, (uint64_t)K / 2, 192)) return NVFP4_ERR_CUDA;
-  if (deep) return launch_ring<64, 4>(tw, tx32, tx64, tx128, tx192, b_sf, a_sf, b_gs, a_gs, expert_offsets, E, M_total,
-                                     N, K, y, swiglu, amax_out, hq, dev_status, stream);
-  return launch_ring<BN, 3>(tw, tx32, tx64, tx128, tx192, b_sf, a_sf, b_gs, a_gs, expert_offsets, E, M_total, N, K, y,
-                            swiglu, amax_out, hq, dev_status, stream);
+  if (mx && (swiglu || hq)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (deep) {
+    auto launch = mx ? launch_ring<64, 4, true> : launch_ring<64, 4, false>;
+    return launch(tw, tx32, tx64, tx128, tx192, b_sf, a_sf, b_gs, a_gs, expert_offsets, E, M_total, N, K, y, swiglu,
+                  amax_out, hq, dev_status, stream);
+  }
+  auto launch = mx ? launch_ring<BN, 3, true> : launch_ring<BN, 3, false>;
+  return launch(tw, tx32, tx64, tx128, tx192, b_sf, a_sf, b_gs, a_gs, expert_offsets, E, M_total, N, K, y, swiglu,
+                amax_out, hq, dev_status, stream);
 }
 
 }  // namespace gemm

@@ -722,6 +722,57 @@ def test_mx_gemm_grouped_chunk_edges(mx_kernel):
     assert ok.all(), (err.max(), (err / bound).max(), np.argwhere(~ok)[:5])
 
 
+def _mx_gemm_raw(qa, ea, qw, ew, offsets, E, N, K, out_dtype, mode):
+    """MXFP4 GEMM of raw codes and exponent bytes on kernel mode `mode`."""
+    L = layer()
+    nv = nvmod()
+    bound = nv.nvfp4_padded_rows_bound(qa.shape[0], E)
+    qs = np.zeros((bound, K // 2), np.uint8)
+    es = np.zeros((bound, K // 32), np.uint8)
+    rows, _ = slot_rows(offsets)
+    qs[rows] = qa
+    es[rows] = ea
+    s = status_word()
+    nv.nvfp4_gemm_select_kernel(mode)
+    try:
+        y = L.mx_grouped_gemm(to_dev(qs), to_dev(tile(es)), to_dev(qw), to_dev(tile(ew)), N, K, qa.shape[0],
+                              to_dev(offsets), E, out_dtype, dev_status=s)
+        torch.cuda.synchronize()
+    finally:
+        nv.nvfp4_gemm_select_kernel(0)
+    assert int(s.item()) == 0
+    return to_np(y)
+
+
+@pytest.mark.parametrize("counts", [[90, 150, 0, 1, 255, 257, 129, 64],
+                                    [1, 63, 64, 65, 0, 2, 17] + [0] * 30 + [3]],
+                         ids=["groups", "small_groups"])
+def test_mx_gemm_two_blocks_bf16(counts):
+    """bf16 MXFP4 GEMMs with N % 256 == 0 and K >= 1024 run on the two-block
+    kernel (automatic choice; 64-token ring when M_total <= 16 E): its bf16 Y
+    must be the bf16 rounding of the fp32 Y of the one-CTA 256-element kernel,
+    which sits within the fp32 accumulation bound of the fp64 oracle.  UE8M0
+    bytes spread over 2^-57 ... 2^53, a few at 2^-127."""
+    rng = np.random.default_rng(26)
+    E, N, K = len(counts), 512, 1024
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    R = int(offsets[-1])
+    qa = rng.integers(0, 256, (R, K // 2), dtype=np.uint8)
+    ea = rng.integers(70, 181, (R, K // 32), dtype=np.uint8)
+    qw = rng.integers(0, 256, (E * N, K // 2), dtype=np.uint8)
+    ew = rng.integers(70, 181, (E * N, K // 32), dtype=np.uint8)
+    ea[3, :5] = 0
+    ew[N + 7, :5] = 0
+    y32 = _mx_gemm_raw(qa, ea, qw, ew, offsets, E, N, K, 0, 1)
+    y16 = _mx_gemm_raw(qa, ea, qw, ew, offsets, E, N, K, 1, 0)
+    a = oracle.dequantize_mxfp4_f64(qa, ea)
+    b = oracle.dequantize_mxfp4_f64(qw, ew)
+    y_ref, s_ref = oracle.grouped_gemm_f64(a, b.reshape(E, N, K), offsets)
+    ok, err, bnd = gemm_tol(y32, y_ref, s_ref)
+    assert ok.all(), (err.max(), (err / bnd).max())
+    assert np.array_equal(y16, synthetic.f32_to_bf16_bits(y32))
+
+
 def test_mx_gemm_matches_remapped_nvfp4_gemm():
     """The two routes for MXFP4 weights: the direct kind::mxf4 GEMM, and the
     lossless NVFP4 remap followed by the NVFP4 GEMM.  Both multiply the same
