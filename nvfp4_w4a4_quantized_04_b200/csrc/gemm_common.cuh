@@ -565,7 +565,7 @@ __device__ __forceinline__ void epilogue_tile(const Tile &T, uint32_t tacc, floa
                                               int lane, int N, void *__restrict__ y, float *__restrict__ amax_out,
                                               uint32_t acc_empty, bool release_remote,
                                               const HQuantOut &hq = HQuantOut{}, int32_t *dev_status = nullptr) {
-  uint32_t hmax = 0;                           // SwiGLU: max |h| bits of this lane
+  uint32_t hmax2 = 0;                          // SwiGLU: max |h| bits of this lane, two bf16 lanes
   float q_sg = 1.0f, q_tg = 6.0f;
   bool q_bad = false, q_gs_bad = false;
   if constexpr (kQuantH) {
@@ -601,7 +601,6 @@ __device__ __forceinline__ void epilogue_tile(const Tile &T, uint32_t tacc, floa
         const int tok0 = c0 + sub * 32;
         if (tok0 >= T.n_valid) break;
         const int rows_here = min(32, T.n_valid - tok0);
-        const int my0 = gate_lane ? 0 : 16;
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           const uint32_t mine = gate_lane ? r[sub * 32 + 16 + j] : r[sub * 32 + j];
@@ -611,7 +610,6 @@ __device__ __forceinline__ void epilogue_tile(const Tile &T, uint32_t tacc, floa
           const float sv = __fdividef(gv, 1.0f + __expf(-gv));
           const __nv_bfloat16 hv = __float2bfloat16_rn(__fmul_rn(sv, uv));
           const uint16_t hb = *reinterpret_cast<const uint16_t *>(&hv);
-          if (!kQuantH && my0 + j < rows_here) hmax = max(hmax, (uint32_t)(hb & 0x7FFFu));
           asm volatile("st.shared.b16 [%0], %1;" :: "r"(epi + half + j * 32 + (lane & 15) * 2), "h"(hb) : "memory");
         }
         __syncwarp();
@@ -642,6 +640,9 @@ __device__ __forceinline__ void epilogue_tile(const Tile &T, uint32_t tacc, floa
           if (row < rows_here) {
             const uint4 v = lds128(epi + (row >> 4) * 576 + (row & 15) * 32 + chunk * 16);
             *reinterpret_cast<uint4 *>(hbase + (int64_t)row * NH + chunk * 8) = v;
+            // the expert's max |h|, over the real rows only, from the bf16 bits stored
+            hmax2 = __vmaxu2(__vmaxu2(hmax2, v.x & 0x7FFF7FFFu), __vmaxu2(v.y & 0x7FFF7FFFu, v.z & 0x7FFF7FFFu));
+            hmax2 = __vmaxu2(hmax2, v.w & 0x7FFF7FFFu);
           }
         }
         __syncwarp();
@@ -697,6 +698,7 @@ __device__ __forceinline__ void epilogue_tile(const Tile &T, uint32_t tacc, floa
     if (q_gs_bad) report(dev_status, NVFP4_ERR_INVALID_ARG);
     if (q_bad) report(dev_status, NVFP4_ERR_NONFINITE);
   } else if (kSwiglu) {
+    uint32_t hmax = max(hmax2 & 0xFFFFu, hmax2 >> 16);
 #pragma unroll
     for (int d = 16; d > 0; d >>= 1) hmax = max(hmax, __shfl_xor_sync(0xffffffffu, hmax, d));
     if (lane == 0 && hmax) atomicMax(reinterpret_cast<uint32_t *>(amax_out) + T.e, hmax << 16);
