@@ -657,7 +657,10 @@ __device__ __forceinline__ uint2 encode_codes(const uint64_t (&xf)[8], float r) 
 // per lane, so the token's routing is warp-uniform), holds them as fp32 pairs
 // and encodes them once per routed copy, with the scale byte from
 // block_scale_fast and r from the group's table.  The block loads are issued
-// before the routing lookups so the two latencies overlap.
+// before the routing lookups so the two latencies overlap.  Lane c resolves
+// choice c (packed row, expert, s_g, 1/(6 s_g)) into the warp's 16-byte slot
+// c in shared memory, which the copy loop reads back as one broadcast load
+// per copy.
 template <bool kTiled>
 __global__ void __launch_bounds__(256, 3) moe_encode_blocks_kernel(
     const uint16_t *__restrict__ x, int64_t ld_x, int64_t K64, int64_t tokens, const int32_t *__restrict__ slot,
@@ -676,6 +679,8 @@ __global__ void __launch_bounds__(256, 3) moe_encode_blocks_kernel(
   const uint64_t nwork = (uint64_t)tokens * cpr;
   const uint64_t nwarps = ((uint64_t)gridDim.x * blockDim.x) >> 5;
   const bool v8 = ((reinterpret_cast<uintptr_t>(x) & 31u) == 0) && ((ld_x & 15) == 0);
+  __shared__ int4 s_choice[8][32];                           // [warp][choice]: row, expert, s_g, y
+  int4 *my_choices = s_choice[threadIdx.x >> 5];
   bool bad = false;
   for (uint64_t w = ((uint64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; w < nwork; w += nwarps) {
     const uint64_t t = w / cpr;
@@ -696,6 +701,9 @@ __global__ void __launch_bounds__(256, 3) moe_encode_blocks_kernel(
         my_y = ytab[e];
       }
     }
+    __syncwarp();                                            // the previous row's copies have read the slots
+    if (lane < topk) my_choices[lane] = make_int4(my_p, my_e, __float_as_int(my_sg), __float_as_int(my_y));
+    __syncwarp();
     const uint32_t m0 = block_amax_bits(a0, b0), m1 = block_amax_bits(a1, b1);
     if (max(m0, m1) >= 0x7F80u) bad = true;
     const float am0 = __uint_as_float(m0 << 16), am1 = __uint_as_float(m1 << 16);
@@ -707,11 +715,12 @@ __global__ void __launch_bounds__(256, 3) moe_encode_blocks_kernel(
                             bf16x2_to_f32x2(b1.z), bf16x2_to_f32x2(b1.w)};
     const uint32_t jb0 = kTiled ? sf_blk_part(j0) : j0, jb1 = kTiled ? sf_blk_part(j1) : j1;
     for (int c = 0; c < topk; ++c) {
-      const int32_t p = __shfl_sync(0xffffffffu, my_p, c);
+      const int4 ch = my_choices[c];
+      const int32_t p = ch.x;
       if (p < 0) continue;
-      const int32_t e = __shfl_sync(0xffffffffu, my_e, c);
-      const float s_g = __shfl_sync(0xffffffffu, my_sg, c);
-      const float y = __shfl_sync(0xffffffffu, my_y, c);
+      const int32_t e = ch.y;
+      const float s_g = __int_as_float(ch.z);
+      const float y = __int_as_float(ch.w);
       const float t_g = __fmul_rn(6.0f, s_g);
       const bool exact = !(y <= 3.402823466e38f);             // y = inf (or NaN): always divide
       const float *rt = rtab + (int64_t)e * 128;
