@@ -51,11 +51,12 @@ def gemm_kernel(request):
     nv.nvfp4_gemm_select_kernel(0)
 
 
-@pytest.fixture(params=[0, 1, 3], ids=["auto", "k256", "deep_ring"])
+@pytest.fixture(params=[0, 1, 3, 4], ids=["auto", "k256", "deep_ring", "two_blocks"])
 def mx_kernel(request):
     """Run an MXFP4 GEMM test on the kernels that take MXFP4 operands: 512-element
-    K stages (automatic when K % 512 == 0; also with the deep ring) and
-    256-element stages."""
+    K stages (automatic when K % 512 == 0; also with the deep ring), 256-element
+    stages, and two weight blocks per tile (bf16 outputs with N % 256 == 0;
+    other calls of that mode run the automatic choice)."""
     nv = nvmod()
     nv.nvfp4_gemm_select_kernel(request.param)
     yield request.param
@@ -720,6 +721,10 @@ def test_mx_gemm_grouped_chunk_edges(mx_kernel):
     y, y_ref, s_ref = _run_mx_gemm(x, w, offsets, E, N, K, 0)
     ok, err, bound = gemm_tol(y, y_ref, s_ref)
     assert ok.all(), (err.max(), (err / bound).max(), np.argwhere(~ok)[:5])
+    # bf16 Y (the two-block kernel in modes 0 and 4 at K >= 1024 or in mode 4)
+    # is the round-to-nearest-even of the fp32 Y
+    y16, _, _ = _run_mx_gemm(x, w, offsets, E, N, K, 1)
+    assert np.array_equal(y16, synthetic.f32_to_bf16_bits(y))
 
 
 def _mx_gemm_raw(qa, ea, qw, ew, offsets, E, N, K, out_dtype, mode):
