@@ -203,15 +203,20 @@ def nvfp4_grouped_gemm_w4a16(x, ld_x, x_rows, row_index, b_q, b_sf, b_gs, expert
 
 
 def nvfp4_gemm_set_wait_budget(cycles: int) -> int:
-    """Main-loop wait budget of the one-CTA grouped GEMM in SM cycles (0 = default);
-    a switch for testing the timeout path."""
+    """Main-loop wait budget of the grouped GEMM kernels in SM cycles (0 =
+    default): the one-CTA kernels (256- and 512-element stages) and the
+    two-block kernel; a switch for testing the timeout path."""
     st = load_library().nvfp4_gemm_set_wait_budget(cycles)
     _check(st, "nvfp4_gemm_set_wait_budget")
     return st
 
 
 def nvfp4_gemm_select_kernel(mode: int) -> int:
-    """0 automatic (one CTA per tile), 1 one CTA per tile, 2 CTA pairs (N % 256 == 0)."""
+    """Which grouped GEMM kernel runs: 0 automatic (two weight blocks per tile for
+    bf16 outputs with N % 256 == 0 and K >= 1024, else one CTA per tile), 1 one
+    CTA per tile with 256-element K stages, 2 CTA pairs (N % 256 == 0), 3 the
+    64-token ring of the 512-element kernel, 4 two weight blocks per tile
+    whenever N % 256 == 0 and the output is bf16."""
     st = load_library().nvfp4_gemm_select_kernel(mode)
     _check(st, "nvfp4_gemm_select_kernel")
     return st
